@@ -1,0 +1,209 @@
+/*
+ * retroinfer.h -- C ABI of the wave-index decode path for NVIDIA B200 (sm_100a).
+ *
+ * The wave index is the attention-aware vector index of RetroInfer (arXiv
+ * 2505.02922).  Sources, cited by page title and section:
+ *   [P1] "微软新突破：RetroInfer如何让AI模型处理百万级文本不再'卡顿'？"
+ *        (techwalker.com), section 三 (wave index, wave buffer).
+ *   [P2] "KV缓存技术与RetroInfer系统在长上下文推理中的优化实践" (framerc.cn),
+ *        §2.1 Wave索引, §2.2 Wave缓冲, §3.1 cache layout, §3.2 execution
+ *        buffer assembly, §3.3 attention kernels.
+ *   [P3] "RetroInfer: A Vector-Storage Approach for Scalable Long-Context LLM
+ *        Inference" (chatpaper.ai), abstract.
+ *   [P4] "RetroInfer: A Vector Storage Engine for Scalable Long-Context LLM
+ *        Inference" (gist.science), "Technische Samenvatting" §2.
+ *
+ * Conventions for every call below:
+ *  - Tensors are caller-owned DEVICE memory unless a parameter says "host".
+ *    Device pointers must be 16-byte aligned.  bf16 = IEEE bfloat16 stored as
+ *    uint16; fp32 = IEEE binary32.  Layouts are dense, row-major, in the order
+ *    written ([B][H_kv][N][d] means d fastest).
+ *  - Calls that take a stream are asynchronous on it (NULL = legacy default
+ *    stream).  Nothing is allocated by these calls; scratch memory is the
+ *    caller's workspace, sized by the matching *_workspace() query.
+ *  - Invalid arguments are rejected on the host BEFORE any launch: the call
+ *    returns an error status and ri_last_error() describes it.
+ *  - Failures found on the device (a bounded wait that expired, an index that
+ *    was out of range in device-resident input) are written to a status word
+ *    at the start of the workspace; ri_read_device_status() reads it.
+ *  - head_dim must be 128.  GQA: query head h_q uses KV head h_q / G.
+ */
+#ifndef RETROINFER_H_
+#define RETROINFER_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ri_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  RI_OK = 0,
+  RI_ERR_INVALID_ARG = 1, /* bad pointer, size or configuration value        */
+  RI_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels handle   */
+  RI_ERR_WORKSPACE = 3,   /* workspace smaller than the *_workspace() query  */
+  RI_ERR_CAPACITY = 4,    /* a cache or buffer capacity would be exceeded    */
+  RI_ERR_CUDA = 5,        /* a CUDA runtime call failed                      */
+  RI_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired              */
+  RI_ERR_HOST = 7         /* host-side failure (allocation, injected fault)  */
+} ri_status;
+
+/* Index geometry.  Zones [P2 §2.1 items 1-3; P1 三]: the steady zone is the
+ * first `steady_initial` and last `steady_recent` tokens of every sequence;
+ * the other M = max(0, N - steady_initial - steady_recent) "middle" tokens
+ * are indexed.  Segmented clustering [P2 §2.1 pseudocode]: the middle tokens
+ * are cut into contiguous segments of `seg_len` tokens (the last may be
+ * short) and k-means runs on each segment with K_s = min(clusters_per_seg,
+ * L_s) clusters.  Global cluster id = sum of K of earlier segments + local id.
+ * Limits: 1 <= clusters_per_seg <= 512, seg_len >= 1, iters >= 0,
+ * group_size 1..8, head_dim == 128. */
+typedef struct {
+  int32_t batch;            /* B                                    */
+  int32_t num_kv_heads;     /* H_kv                                 */
+  int32_t group_size;       /* G = H_q / H_kv                       */
+  int32_t head_dim;         /* d (must be 128)                      */
+  int32_t seq_len;          /* N, same for every sequence           */
+  int32_t seg_len;          /* tokens per segment (8192)            */
+  int32_t clusters_per_seg; /* K (512)                              */
+  int32_t iters;            /* Lloyd iterations T (10)              */
+  int32_t steady_initial;   /* 4                                    */
+  int32_t steady_recent;    /* 64                                   */
+} ri_index_config;
+
+typedef struct {
+  int32_t middle;       /* M                                         */
+  int32_t num_segments; /* S = ceil(M / seg_len)                     */
+  int32_t clusters;     /* C = sum of K_s over segments              */
+  int32_t steady;       /* min(N, steady_initial + steady_recent)    */
+} ri_geometry;
+
+/* Derived sizes of a configuration.  Host only; validates the config. */
+ri_status ri_index_geometry(const ri_index_config* cfg, ri_geometry* out);
+
+/* The index of every (sequence, KV head).  All device memory, caller-owned,
+ * written by ri_build_index and read by the decode calls.
+ *  Kp, Vp    bf16 [B][H_kv][M][d]  cluster-contiguous copy of the middle
+ *            tokens [P2 §3.1]: clusters in global id order, members of a
+ *            cluster in position order.
+ *  perm      int32 [B][H_kv][M]    absolute token position of each row.
+ *  centroid  bf16 [B][H_kv][C][d]  round-to-nearest-even of the fp32 mean of
+ *            the cluster's keys (an empty cluster keeps its last centroid).
+ *  counts    int32 [B][H_kv][C]    cluster sizes n_c.
+ *  offsets   int32 [B][H_kv][C+1]  row of each cluster's first member in
+ *            Kp/Vp; offsets[C] = M.
+ *  vsum      fp32 [B][H_kv][C][d]  sum of the members' values
+ *            [P2 §2.1 `compute_cluster_sums`].
+ *  Ks, Vs    bf16 [B][H_kv][steady][d]  steady-zone tokens in position order.
+ *  labels    optional (may be NULL) int32 [B][H_kv][M]: cluster id within
+ *            its segment of every middle token, in position order.
+ *  objective optional (may be NULL) fp32 [B][H_kv][S]: per segment, the sum
+ *            of squared distances of keys to their final centroid.          */
+typedef struct {
+  void* Kp;
+  void* Vp;
+  int32_t* perm;
+  void* centroid;
+  int32_t* counts;
+  int32_t* offsets;
+  float* vsum;
+  void* Ks;
+  void* Vs;
+  int32_t* labels;
+  float* objective;
+} ri_index;
+
+/* Bytes of workspace ri_build_index needs (0 on invalid config). */
+size_t ri_build_index_workspace(const ri_index_config* cfg);
+
+/* Segmented k-means index build [P2 §2.1 pseudocode; P3 abstract].
+ * K, V      bf16 [B][H_kv][N][d] device, the keys and values.
+ * init_pos  optional device int32 [B][H_kv][C]: for the clusters of segment
+ *           s, distinct positions in [0, L_s) of the tokens whose keys seed
+ *           the centroids; NULL selects positions floor(j * L_s / K_s).
+ *           Out-of-range entries are clamped and flagged RI_ERR_INVALID_ARG
+ *           in the device status word.
+ * Lloyd's algorithm with squared Euclidean distance, ties to the lower
+ * cluster id, a fixed number of iterations; labels and centroids returned are
+ * those of the last iteration, so every non-empty centroid is the mean of its
+ * final members.  Assignment runs on the tensor cores (tcgen05) with a
+ * rigorous error bound; near ties are re-decided in fp32.
+ * Returns before the work completes; errors in arguments return early. */
+ri_status ri_build_index(const ri_index_config* cfg, const void* K, const void* V,
+                         const int32_t* init_pos, const ri_index* out, void* workspace,
+                         size_t workspace_bytes, ri_stream_t stream);
+
+/* Zone budgets in clusters: k_retrieval = round(0.018 C), k_estimation =
+ * round(0.23 C) by default [P2 §2.1 items 2-3].  The zones are clamped to
+ * C: R = top min(k_r, C), E = next min(k_e, C - |R|). */
+typedef struct {
+  int32_t k_retrieval;
+  int32_t k_estimation;
+} ri_decode_config;
+
+/* Default budgets for C clusters (round half up of 1.8 % and 23 %). */
+ri_status ri_default_budgets(int32_t clusters, ri_decode_config* out);
+
+/* Bytes of workspace the decode calls need (0 on invalid config). */
+size_t ri_decode_workspace(const ri_index_config* cfg, const ri_decode_config* dcfg);
+
+/* One decode step of tripartite attention [P3 abstract; P2 §2.1, §3.3]:
+ *  - scores s[h][c] = q_h . centroid_c / sqrt(d) for every query head of a KV
+ *    head; selection key r_c = sum over the G heads (r_c = -inf if n_c = 0);
+ *  - R = the k_r clusters of largest r (ties to the lower id), E = the next
+ *    k_e;
+ *  - out_h = (sum_{i in steady u R} e^{x_i} v_i + sum_{c in E} e^{s_hc} Vsum_c)
+ *          / (sum_{i in steady u R} e^{x_i} + sum_{c in E} n_c e^{s_hc}),
+ *    x_i = q_h . k_i / sqrt(d); partial results merged by log-sum-exp.
+ * q        bf16 [B][H_kv*G][d].
+ * out      bf16 [B][H_kv*G][d].
+ * lse      optional fp32 [B][H_kv*G]: natural log of the denominator.
+ * sel_ids  optional int32 [B][H_kv][k_r + k_e]: R then E, each in increasing
+ *          id order (entries past the clamped sizes are -1).
+ * Reads Kp/Vp in place through `offsets`. */
+ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                              const void* q, const ri_index* idx, void* out, float* lse,
+                              int32_t* sel_ids, void* workspace, size_t workspace_bytes,
+                              ri_stream_t stream);
+
+/* Steps S1-S2 alone (centroid scoring and cluster selection).  Writes
+ * sel_ids (required here) and keeps scores and the selection in the
+ * workspace for a following ri_attend_selected on the same workspace and
+ * stream.  Also writes, when non-NULL, retr_rows int32 [B][H_kv][k_r + 1]:
+ * the exclusive prefix sum of the sizes of the R clusters in id order (the
+ * execution-buffer row of each retrieval cluster; last entry = total). */
+ri_status ri_select_clusters(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                             const void* q, const ri_index* idx, int32_t* sel_ids,
+                             int32_t* retr_rows, void* workspace, size_t workspace_bytes,
+                             ri_stream_t stream);
+
+/* Steps S4-S6 on the selection left in `workspace` by ri_select_clusters.
+ * exec_K, exec_V: NULL to read the retrieval tokens in place from idx->Kp,
+ * idx->Vp; otherwise bf16 [B][H_kv][exec_rows][d] execution buffers holding,
+ * for every (sequence, head), the R clusters' rows packed in id order from
+ * row 0 [P1 三: the execution buffer feeds attention]. */
+ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                             const void* q, const ri_index* idx, const void* exec_K,
+                             const void* exec_V, int32_t exec_rows, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, ri_stream_t stream);
+
+/* Synchronises `stream` and returns the status word a previous call wrote
+ * into `workspace` (RI_OK if no device-side failure was recorded). */
+ri_status ri_read_device_status(const void* workspace, ri_stream_t stream);
+
+/* Self-test of the bounded device wait: launches one kernel that waits for a
+ * flag in `workspace` that nothing sets, giving up after `limit_ns`
+ * nanoseconds and recording RI_ERR_TIMEOUT in the status word.  workspace
+ * needs 256 bytes. */
+ri_status ri_selftest_wait_timeout(void* workspace, uint64_t limit_ns, ri_stream_t stream);
+
+const char* ri_status_string(ri_status status);
+/* Description of the last error of the calling thread ("" if none). */
+const char* ri_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RETROINFER_H_ */

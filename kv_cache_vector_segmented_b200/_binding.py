@@ -1,0 +1,338 @@
+"""ctypes binding of libretroinfer.so (the C ABI in include/retroinfer.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, and their device pointers plus torch's current CUDA stream are
+passed to the library.  Every step of the path runs in the library's CUDA
+kernels; there is no fallback.  Importing works without a GPU (host-only calls
+such as geometry and budget queries run anywhere); compute calls need CUDA.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libretroinfer.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_segmented_b200.build` "
+        "(nvcc, sm_100a). The wave-index path has no CPU fallback.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+RI_OK = 0
+STATUS_NAMES = {0: "RI_OK", 1: "RI_ERR_INVALID_ARG", 2: "RI_ERR_UNSUPPORTED",
+                3: "RI_ERR_WORKSPACE", 4: "RI_ERR_CAPACITY", 5: "RI_ERR_CUDA",
+                6: "RI_ERR_TIMEOUT", 7: "RI_ERR_HOST"}
+STATUS_CODES = {v: k for k, v in STATUS_NAMES.items()}
+
+
+class RIError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.ri_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+class IndexConfig(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("group_size", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("seq_len", ctypes.c_int32), ("seg_len", ctypes.c_int32),
+                ("clusters_per_seg", ctypes.c_int32), ("iters", ctypes.c_int32),
+                ("steady_initial", ctypes.c_int32), ("steady_recent", ctypes.c_int32)]
+
+    @classmethod
+    def make(cls, batch: int, num_kv_heads: int, group_size: int, seq_len: int,
+             seg_len: int = 8192, clusters_per_seg: int = 512, iters: int = 10,
+             steady_initial: int = 4, steady_recent: int = 64, head_dim: int = 128):
+        return cls(batch, num_kv_heads, group_size, head_dim, seq_len, seg_len,
+                   clusters_per_seg, iters, steady_initial, steady_recent)
+
+
+class Geometry(ctypes.Structure):
+    _fields_ = [("middle", ctypes.c_int32), ("num_segments", ctypes.c_int32),
+                ("clusters", ctypes.c_int32), ("steady", ctypes.c_int32)]
+
+
+class CIndex(ctypes.Structure):
+    _fields_ = [("Kp", ctypes.c_void_p), ("Vp", ctypes.c_void_p), ("perm", ctypes.c_void_p),
+                ("centroid", ctypes.c_void_p), ("counts", ctypes.c_void_p),
+                ("offsets", ctypes.c_void_p), ("vsum", ctypes.c_void_p),
+                ("Ks", ctypes.c_void_p), ("Vs", ctypes.c_void_p),
+                ("labels", ctypes.c_void_p), ("objective", ctypes.c_void_p)]
+
+
+class DecodeConfig(ctypes.Structure):
+    _fields_ = [("k_retrieval", ctypes.c_int32), ("k_estimation", ctypes.c_int32)]
+
+
+_P = ctypes.POINTER
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+lib.ri_status_string.restype = ctypes.c_char_p
+lib.ri_status_string.argtypes = [ctypes.c_int]
+lib.ri_last_error.restype = ctypes.c_char_p
+lib.ri_last_error.argtypes = []
+lib.ri_index_geometry.restype = ctypes.c_int
+lib.ri_index_geometry.argtypes = [_P(IndexConfig), _P(Geometry)]
+lib.ri_default_budgets.restype = ctypes.c_int
+lib.ri_default_budgets.argtypes = [ctypes.c_int32, _P(DecodeConfig)]
+lib.ri_build_index_workspace.restype = _sz
+lib.ri_build_index_workspace.argtypes = [_P(IndexConfig)]
+lib.ri_build_index.restype = ctypes.c_int
+lib.ri_build_index.argtypes = [_P(IndexConfig), _vp, _vp, _vp, _P(CIndex), _vp, _sz, _vp]
+lib.ri_decode_workspace.restype = _sz
+lib.ri_decode_workspace.argtypes = [_P(IndexConfig), _P(DecodeConfig)]
+lib.ri_decode_attention.restype = ctypes.c_int
+lib.ri_decode_attention.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
+                                    _vp, _vp, _vp, _sz, _vp]
+lib.ri_select_clusters.restype = ctypes.c_int
+lib.ri_select_clusters.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
+                                   _vp, _vp, _sz, _vp]
+lib.ri_attend_selected.restype = ctypes.c_int
+lib.ri_attend_selected.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
+                                   _vp, ctypes.c_int32, _vp, _vp, _vp, _sz, _vp]
+lib.ri_read_device_status.restype = ctypes.c_int
+lib.ri_read_device_status.argtypes = [_vp, _vp]
+lib.ri_selftest_wait_timeout.restype = ctypes.c_int
+lib.ri_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
+
+
+def check(status: int, where: str) -> None:
+    if status != RI_OK:
+        raise RIError(status, where)
+
+
+def geometry(cfg: IndexConfig) -> Geometry:
+    g = Geometry()
+    check(lib.ri_index_geometry(ctypes.byref(cfg), ctypes.byref(g)), "ri_index_geometry")
+    return g
+
+
+def default_budgets(clusters: int) -> DecodeConfig:
+    d = DecodeConfig()
+    check(lib.ri_default_budgets(clusters, ctypes.byref(d)), "ri_default_budgets")
+    return d
+
+
+def build_workspace_bytes(cfg: IndexConfig) -> int:
+    n = lib.ri_build_index_workspace(ctypes.byref(cfg))
+    if n == 0:
+        raise RIError(STATUS_CODES["RI_ERR_INVALID_ARG"], "ri_build_index_workspace")
+    return n
+
+
+def decode_workspace_bytes(cfg: IndexConfig, dcfg: DecodeConfig) -> int:
+    n = lib.ri_decode_workspace(ctypes.byref(cfg), ctypes.byref(dcfg))
+    if n == 0:
+        raise RIError(STATUS_CODES["RI_ERR_INVALID_ARG"], "ri_decode_workspace")
+    return n
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned scratch for the library, 1024-byte aligned."""
+    raw = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 1024
+    return raw[off:off + nbytes]
+
+
+@dataclasses.dataclass
+class Index:
+    """Device tensors of a wave index (layouts as in include/retroinfer.h)."""
+
+    cfg: IndexConfig
+    geom: Geometry
+    Kp: torch.Tensor
+    Vp: torch.Tensor
+    perm: torch.Tensor
+    centroid: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    vsum: torch.Tensor
+    Ks: torch.Tensor
+    Vs: torch.Tensor
+    labels: Optional[torch.Tensor] = None
+    objective: Optional[torch.Tensor] = None
+
+    def c_struct(self) -> CIndex:
+        return CIndex(_ptr(self.Kp), _ptr(self.Vp), _ptr(self.perm), _ptr(self.centroid),
+                      _ptr(self.counts), _ptr(self.offsets), _ptr(self.vsum), _ptr(self.Ks),
+                      _ptr(self.Vs), _ptr(self.labels), _ptr(self.objective))
+
+    @property
+    def device(self) -> torch.device:
+        return self.offsets.device
+
+    @classmethod
+    def empty(cls, cfg: IndexConfig, device, labels: bool = True, objective: bool = True):
+        g = geometry(cfg)
+        B, H, d = cfg.batch, cfg.num_kv_heads, cfg.head_dim
+        M, C, S, ns = g.middle, g.clusters, g.num_segments, g.steady
+        bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
+        return cls(cfg=cfg, geom=g,
+                   Kp=torch.empty((B, H, M, d), dtype=bf, device=device),
+                   Vp=torch.empty((B, H, M, d), dtype=bf, device=device),
+                   perm=torch.empty((B, H, M), dtype=i32, device=device),
+                   centroid=torch.empty((B, H, C, d), dtype=bf, device=device),
+                   counts=torch.empty((B, H, C), dtype=i32, device=device),
+                   offsets=torch.empty((B, H, C + 1), dtype=i32, device=device),
+                   vsum=torch.empty((B, H, C, d), dtype=f32, device=device),
+                   Ks=torch.empty((B, H, ns, d), dtype=bf, device=device),
+                   Vs=torch.empty((B, H, ns, d), dtype=bf, device=device),
+                   labels=torch.empty((B, H, M), dtype=i32, device=device) if labels else None,
+                   objective=torch.empty((B, H, S), dtype=f32, device=device) if objective else None)
+
+    def check_shapes(self) -> None:
+        cfg, g = self.cfg, self.geom
+        B, H, d = cfg.batch, cfg.num_kv_heads, cfg.head_dim
+        M, C, ns = g.middle, g.clusters, g.steady
+        dev = self.device
+        _need(self.Kp, "Kp", torch.bfloat16, (B, H, M, d), dev)
+        _need(self.Vp, "Vp", torch.bfloat16, (B, H, M, d), dev)
+        _need(self.perm, "perm", torch.int32, (B, H, M), dev)
+        _need(self.centroid, "centroid", torch.bfloat16, (B, H, C, d), dev)
+        _need(self.counts, "counts", torch.int32, (B, H, C), dev)
+        _need(self.offsets, "offsets", torch.int32, (B, H, C + 1), dev)
+        _need(self.vsum, "vsum", torch.float32, (B, H, C, d), dev)
+        _need(self.Ks, "Ks", torch.bfloat16, (B, H, ns, d), dev)
+        _need(self.Vs, "Vs", torch.bfloat16, (B, H, ns, d), dev)
+
+
+def build_index(K: torch.Tensor, V: torch.Tensor, cfg: IndexConfig,
+                init_pos: Optional[torch.Tensor] = None, out: Optional[Index] = None,
+                workspace: Optional[torch.Tensor] = None) -> Index:
+    """Segmented k-means index build (ri_build_index) on K's device and torch's
+    current stream.  Asynchronous; returns the (possibly given) Index."""
+    dev = K.device
+    if dev.type != "cuda":
+        raise ValueError("build_index needs CUDA tensors")
+    B, H, N, d = cfg.batch, cfg.num_kv_heads, cfg.seq_len, cfg.head_dim
+    _need(K, "K", torch.bfloat16, (B, H, N, d), dev)
+    _need(V, "V", torch.bfloat16, (B, H, N, d), dev)
+    g = geometry(cfg)
+    if init_pos is not None:
+        _need(init_pos, "init_pos", torch.int32, (B, H, g.clusters), dev)
+    idx = out if out is not None else Index.empty(cfg, dev)
+    idx.check_shapes()
+    nbytes = build_workspace_bytes(cfg)
+    ws = workspace if workspace is not None else alloc_workspace(nbytes, dev)
+    cidx = idx.c_struct()
+    check(lib.ri_build_index(ctypes.byref(cfg), K.data_ptr(), V.data_ptr(), _ptr(init_pos),
+                             ctypes.byref(cidx), ws.data_ptr(), ws.numel(), _stream(dev)),
+          "ri_build_index")
+    idx._build_ws = ws  # keep the status word reachable
+    return idx
+
+
+def decode(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = None,
+           workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+           lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+           want_sel: bool = False):
+    """One tripartite decode step (ri_decode_attention).  Returns
+    (out bf16 [B][H_q][d], lse fp32 [B][H_q] or None, sel int32 or None)."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, H * G, d), dev)
+    if dcfg is None:
+        dcfg = default_budgets(index.geom.clusters)
+    nbytes = decode_workspace_bytes(cfg, dcfg)
+    ws = workspace if workspace is not None else alloc_workspace(nbytes, dev)
+    if ws.numel() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    if out is None:
+        out = torch.empty((B, H * G, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, H * G, d), dev)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H * G), dtype=torch.float32, device=dev)
+    sel = (torch.empty((B, H, dcfg.k_retrieval + dcfg.k_estimation), dtype=torch.int32,
+                       device=dev) if want_sel else None)
+    cidx = index.c_struct()
+    check(lib.ri_decode_attention(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                  ctypes.byref(cidx), out.data_ptr(), _ptr(lse), _ptr(sel),
+                                  ws.data_ptr(), ws.numel(), _stream(dev)),
+          "ri_decode_attention")
+    return out, lse, sel
+
+
+def select_clusters(q: torch.Tensor, index: Index, dcfg: DecodeConfig, workspace: torch.Tensor,
+                    sel: Optional[torch.Tensor] = None, retr_rows: Optional[torch.Tensor] = None):
+    """Steps S1-S2 alone (ri_select_clusters); the selection stays in
+    `workspace` for attend_selected.  Returns (sel, retr_rows)."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, H * G, d), dev)
+    k = dcfg.k_retrieval + dcfg.k_estimation
+    if sel is None:
+        sel = torch.empty((B, H, k), dtype=torch.int32, device=dev)
+    if retr_rows is None:
+        retr_rows = torch.empty((B, H, dcfg.k_retrieval + 1), dtype=torch.int32, device=dev)
+    cidx = index.c_struct()
+    check(lib.ri_select_clusters(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                 ctypes.byref(cidx), sel.data_ptr(), retr_rows.data_ptr(),
+                                 workspace.data_ptr(), workspace.numel(), _stream(dev)),
+          "ri_select_clusters")
+    return sel, retr_rows
+
+
+def attend_selected(q: torch.Tensor, index: Index, dcfg: DecodeConfig, workspace: torch.Tensor,
+                    exec_K: Optional[torch.Tensor] = None, exec_V: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Steps S4-S6 on the selection in `workspace` (ri_attend_selected)."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, H * G, d), dev)
+    if out is None:
+        out = torch.empty((B, H * G, d), dtype=torch.bfloat16, device=dev)
+    rows = 0
+    if exec_K is not None:
+        rows = exec_K.shape[2]
+        _need(exec_K, "exec_K", torch.bfloat16, (B, H, rows, d), dev)
+        _need(exec_V, "exec_V", torch.bfloat16, (B, H, rows, d), dev)
+    cidx = index.c_struct()
+    check(lib.ri_attend_selected(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                 ctypes.byref(cidx), _ptr(exec_K), _ptr(exec_V), rows,
+                                 out.data_ptr(), _ptr(lse), workspace.data_ptr(),
+                                 workspace.numel(), _stream(dev)),
+          "ri_attend_selected")
+    return out, lse
+
+
+def read_device_status(workspace: torch.Tensor) -> int:
+    """Synchronises torch's current stream and returns the workspace status."""
+    return lib.ri_read_device_status(workspace.data_ptr(), _stream(workspace.device))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int) -> None:
+    check(lib.ri_selftest_wait_timeout(workspace.data_ptr(), limit_ns,
+                                       _stream(workspace.device)),
+          "ri_selftest_wait_timeout")

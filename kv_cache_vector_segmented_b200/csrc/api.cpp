@@ -1,0 +1,444 @@
+// C ABI of the wave-index path: argument validation, derived geometry,
+// workspace layouts and the launch sequence of each call.  Every check runs
+// on the host before the first launch; nothing here allocates device memory.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <cmath>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "internal.h"
+#include "retroinfer.h"
+
+namespace ri {
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+  }
+  return n;
+}
+
+cudaError_t set_smem_once(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({func, dev});
+  return e;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool make_geometry(const ri_index_config* cfg, Geometry* g) {
+  if (!cfg) {
+    set_error("config is NULL");
+    return false;
+  }
+  const ri_index_config& c = *cfg;
+  if (c.batch < 1 || c.num_kv_heads < 1 || c.seq_len < 1) {
+    set_error("batch, num_kv_heads and seq_len must be >= 1 (got %d, %d, %d)", c.batch,
+              c.num_kv_heads, c.seq_len);
+    return false;
+  }
+  if (c.group_size < 1 || c.group_size > kMaxGroupHost) {
+    set_error("group_size must be in [1, %d] (got %d)", kMaxGroupHost, c.group_size);
+    return false;
+  }
+  if (c.head_dim != 128) {
+    set_error("head_dim must be 128 (got %d)", c.head_dim);
+    return false;
+  }
+  if (c.seg_len < 1 || c.seg_len > 32768) {
+    set_error("seg_len must be in [1, 32768] (got %d)", c.seg_len);
+    return false;
+  }
+  if (c.clusters_per_seg < 1 || c.clusters_per_seg > 512) {
+    set_error("clusters_per_seg must be in [1, 512] (got %d)", c.clusters_per_seg);
+    return false;
+  }
+  if (c.iters < 0 || c.iters > 1000) {
+    set_error("iters must be in [0, 1000] (got %d)", c.iters);
+    return false;
+  }
+  if (c.steady_initial < 0 || c.steady_recent < 0) {
+    set_error("steady_initial and steady_recent must be >= 0");
+    return false;
+  }
+  const long long bhn = (long long)c.batch * c.num_kv_heads * c.seq_len;
+  if (bhn > (1ll << 31) - 1) {
+    set_error("batch * num_kv_heads * seq_len must be < 2^31 (got %lld)", bhn);
+    return false;
+  }
+  g->B = c.batch;
+  g->H = c.num_kv_heads;
+  g->G = c.group_size;
+  g->d = c.head_dim;
+  g->N = c.seq_len;
+  g->seg_len = c.seg_len;
+  g->K = c.clusters_per_seg;
+  g->iters = c.iters;
+  g->s0 = c.steady_initial;
+  g->s1 = c.steady_recent;
+  const long long steady = (long long)c.steady_initial + c.steady_recent;
+  g->M = (int)(c.seq_len > steady ? c.seq_len - steady : 0);
+  g->n_steady = (int)(c.seq_len < steady ? c.seq_len : steady);
+  g->m0 = g->M > 0 ? c.steady_initial : 0;
+  g->S = (g->M + c.seg_len - 1) / c.seg_len;
+  g->K_full = c.clusters_per_seg < c.seg_len ? c.clusters_per_seg : c.seg_len;
+  if (g->S > 0) {
+    g->L_last = g->M - (g->S - 1) * c.seg_len;
+    g->K_last = c.clusters_per_seg < g->L_last ? c.clusters_per_seg : g->L_last;
+    g->C = (g->S - 1) * g->K_full + g->K_last;
+    g->tiles_full = (c.seg_len + 127) / 128;
+    g->tiles_last = (g->L_last + 127) / 128;
+    g->tiles_bh = (g->S - 1) * g->tiles_full + g->tiles_last;
+  } else {
+    g->L_last = g->K_last = g->C = 0;
+    g->tiles_full = g->tiles_last = g->tiles_bh = 0;
+  }
+  return true;
+}
+
+bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L) {
+  if (!dcfg) {
+    set_error("decode config is NULL");
+    return false;
+  }
+  if (dcfg->k_retrieval < 0 || dcfg->k_estimation < 0) {
+    set_error("k_retrieval and k_estimation must be >= 0");
+    return false;
+  }
+  if (dcfg->k_retrieval > 8192) {
+    set_error("k_retrieval must be <= 8192 (got %d)", dcfg->k_retrieval);
+    return false;
+  }
+  if ((long long)dcfg->k_retrieval + dcfg->k_estimation > (1 << 24)) {
+    set_error("k_retrieval + k_estimation too large");
+    return false;
+  }
+  L->k_r = dcfg->k_retrieval;
+  L->k_e = dcfg->k_estimation;
+  L->kr = L->k_r < g.C ? L->k_r : g.C;
+  L->ke = L->k_e < g.C - L->kr ? L->k_e : g.C - L->kr;
+  const long long BH = g.BH();
+  int P = (int)((2 * 148 + BH - 1) / BH);
+  if (P < 1) P = 1;
+  if (P > 64) P = 64;
+  L->P = P;
+  size_t off = kStatusBytesHost;
+  L->off_rkey = off;
+  off = align_up(off + (size_t)BH * g.C * 4, 256);
+  L->off_score = off;
+  off = align_up(off + (size_t)BH * g.G * g.C * 4, 256);
+  L->off_sel = off;
+  off = align_up(off + (size_t)BH * (L->k_r + L->k_e) * 4, 256);
+  L->off_rpre = off;
+  off = align_up(off + (size_t)BH * (L->k_r + 1) * 4, 256);
+  L->off_part = off;
+  off = align_up(off + (size_t)BH * P * g.G * kPartStride * 4, 256);
+  L->total = off;
+  return true;
+}
+
+bool make_build_layout(const Geometry& g, BuildLayout* L) {
+  const size_t BH = (size_t)g.BH();
+  size_t off = kStatusBytesHost;
+  L->off_mu = off;
+  off = align_up(off + BH * g.C * 128 * 4, 1024);
+  L->off_mu_bf16 = off;
+  off = align_up(off + BH * g.C * 128 * 2, 1024);
+  L->off_norm2 = off;
+  off = align_up(off + BH * g.S * 512 * 4, 256);
+  L->off_mumax = off;
+  off = align_up(off + BH * g.S * 4, 256);
+  L->off_counts = off;
+  off = align_up(off + BH * g.C * 4, 256);
+  L->off_labels = off;
+  off = align_up(off + BH * g.M * 4, 256);
+  L->off_knorm = off;
+  off = align_up(off + BH * g.M * 4, 256);
+  L->total = off;
+  return true;
+}
+
+}  // namespace ri
+
+using namespace ri;
+
+#define RI_CHECK(cond, code, ...) \
+  do {                            \
+    if (!(cond)) {                \
+      set_error(__VA_ARGS__);     \
+      return code;                \
+    }                             \
+  } while (0)
+
+static ri_status cuda_fail(cudaError_t e, const char* what) {
+  set_error("%s: %s", what, cudaGetErrorString(e));
+  return RI_ERR_CUDA;
+}
+
+extern "C" {
+
+const char* ri_status_string(ri_status s) {
+  switch (s) {
+    case RI_OK: return "ok";
+    case RI_ERR_INVALID_ARG: return "invalid argument";
+    case RI_ERR_UNSUPPORTED: return "unsupported";
+    case RI_ERR_WORKSPACE: return "workspace too small";
+    case RI_ERR_CAPACITY: return "capacity exceeded";
+    case RI_ERR_CUDA: return "CUDA error";
+    case RI_ERR_TIMEOUT: return "device wait timed out";
+    case RI_ERR_HOST: return "host failure";
+  }
+  return "unknown status";
+}
+
+const char* ri_last_error(void) { return ri::g_last_error; }
+
+ri_status ri_index_geometry(const ri_index_config* cfg, ri_geometry* out) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(out, RI_ERR_INVALID_ARG, "out is NULL");
+  out->middle = g.M;
+  out->num_segments = g.S;
+  out->clusters = g.C;
+  out->steady = g.n_steady;
+  return RI_OK;
+}
+
+ri_status ri_default_budgets(int32_t clusters, ri_decode_config* out) {
+  RI_CHECK(out, RI_ERR_INVALID_ARG, "out is NULL");
+  RI_CHECK(clusters >= 0, RI_ERR_INVALID_ARG, "clusters must be >= 0");
+  // round half up of 1.8 % and 23 % of C, in exact integer arithmetic
+  out->k_retrieval = (int32_t)((18LL * clusters + 500) / 1000);
+  out->k_estimation = (int32_t)((23LL * clusters + 50) / 100);
+  return RI_OK;
+}
+
+size_t ri_build_index_workspace(const ri_index_config* cfg) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return 0;
+  BuildLayout L;
+  make_build_layout(g, &L);
+  return L.total;
+}
+
+size_t ri_decode_workspace(const ri_index_config* cfg, const ri_decode_config* dcfg) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return 0;
+  DecodeLayout L;
+  if (!make_decode_layout(g, dcfg, &L)) return 0;
+  return L.total;
+}
+
+static ri_status check_index_pointers(const Geometry& g, const ri_index* idx, bool for_build) {
+  RI_CHECK(idx, RI_ERR_INVALID_ARG, "index is NULL");
+  if (g.n_steady > 0) {
+    RI_CHECK(idx->Ks && idx->Vs, RI_ERR_INVALID_ARG, "index Ks/Vs is NULL");
+    RI_CHECK(aligned16(idx->Ks) && aligned16(idx->Vs), RI_ERR_INVALID_ARG,
+             "index Ks/Vs must be 16-byte aligned");
+  }
+  RI_CHECK(idx->offsets && aligned16(idx->offsets), RI_ERR_INVALID_ARG,
+           "index offsets must be non-NULL and 16-byte aligned");
+  if (g.M > 0) {
+    const void* ptrs[] = {idx->Kp, idx->Vp, idx->perm, idx->centroid, idx->counts, idx->vsum};
+    const char* names[] = {"Kp", "Vp", "perm", "centroid", "counts", "vsum"};
+    for (int i = 0; i < 6; ++i) {
+      RI_CHECK(ptrs[i], RI_ERR_INVALID_ARG, "index %s is NULL", names[i]);
+      RI_CHECK(aligned16(ptrs[i]), RI_ERR_INVALID_ARG, "index %s must be 16-byte aligned",
+               names[i]);
+    }
+  }
+  if (for_build) {
+    RI_CHECK(!idx->labels || aligned16(idx->labels), RI_ERR_INVALID_ARG,
+             "labels must be 16-byte aligned");
+    RI_CHECK(!idx->objective || aligned16(idx->objective), RI_ERR_INVALID_ARG,
+             "objective must be 16-byte aligned");
+  }
+  return RI_OK;
+}
+
+ri_status ri_build_index(const ri_index_config* cfg, const void* K, const void* V,
+                         const int32_t* init_pos, const ri_index* out, void* workspace,
+                         size_t workspace_bytes, ri_stream_t stream) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(K && V, RI_ERR_INVALID_ARG, "K and V must be non-NULL");
+  RI_CHECK(aligned16(K) && aligned16(V), RI_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
+  RI_CHECK(!init_pos || aligned16(init_pos), RI_ERR_INVALID_ARG,
+           "init_pos must be 16-byte aligned");
+  ri_status st = check_index_pointers(g, out, true);
+  if (st != RI_OK) return st;
+  BuildLayout L;
+  make_build_layout(g, &L);
+  RI_CHECK(workspace, RI_ERR_INVALID_ARG, "workspace is NULL");
+  RI_CHECK((reinterpret_cast<uintptr_t>(workspace) & 1023u) == 0, RI_ERR_INVALID_ARG,
+           "workspace must be 1024-byte aligned");
+  RI_CHECK(workspace_bytes >= L.total, RI_ERR_WORKSPACE,
+           "workspace has %zu bytes, build needs %zu", workspace_bytes, L.total);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  BuildArgs a;
+  a.K = K;
+  a.V = V;
+  a.init_pos = init_pos;
+  a.out = *out;
+  a.ws = static_cast<char*>(workspace);
+  return launch_build(g, L, a, s);
+}
+
+static ri_status prepare_decode(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                const void* q, const ri_index* idx, void* workspace,
+                                size_t workspace_bytes, Geometry* g, DecodeLayout* L) {
+  if (!make_geometry(cfg, g)) return RI_ERR_INVALID_ARG;
+  if (!make_decode_layout(*g, dcfg, L)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(q && aligned16(q), RI_ERR_INVALID_ARG, "q must be non-NULL and 16-byte aligned");
+  ri_status st = check_index_pointers(*g, idx, false);
+  if (st != RI_OK) return st;
+  RI_CHECK(workspace && aligned16(workspace), RI_ERR_INVALID_ARG,
+           "workspace must be non-NULL and 16-byte aligned");
+  RI_CHECK(workspace_bytes >= L->total, RI_ERR_WORKSPACE,
+           "workspace has %zu bytes, decode needs %zu", workspace_bytes, L->total);
+  return RI_OK;
+}
+
+static DecodeArgs decode_args(const void* q, const ri_index* idx, void* out, float* lse,
+                              int32_t* sel, int32_t* rpre, void* ws) {
+  DecodeArgs a;
+  a.q = q;
+  a.centroid = idx->centroid;
+  a.counts = idx->counts;
+  a.offsets = idx->offsets;
+  a.vsum = idx->vsum;
+  a.Kp = idx->Kp;
+  a.Vp = idx->Vp;
+  a.Ks = idx->Ks;
+  a.Vs = idx->Vs;
+  a.exec_K = nullptr;
+  a.exec_V = nullptr;
+  a.exec_rows = 0;
+  a.out = out;
+  a.lse = lse;
+  a.sel_user = sel;
+  a.rpre_user = rpre;
+  a.ws = static_cast<char*>(ws);
+  return a;
+}
+
+ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                              const void* q, const ri_index* idx, void* out, float* lse,
+                              int32_t* sel_ids, void* workspace, size_t workspace_bytes,
+                              ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  ri_status st = prepare_decode(cfg, dcfg, q, idx, workspace, workspace_bytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  RI_CHECK(!sel_ids || aligned16(sel_ids), RI_ERR_INVALID_ARG, "sel_ids must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, workspace);
+  e = launch_select(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  e = launch_attend(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+  return RI_OK;
+}
+
+ri_status ri_select_clusters(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                             const void* q, const ri_index* idx, int32_t* sel_ids,
+                             int32_t* retr_rows, void* workspace, size_t workspace_bytes,
+                             ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  ri_status st = prepare_decode(cfg, dcfg, q, idx, workspace, workspace_bytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(sel_ids && aligned16(sel_ids), RI_ERR_INVALID_ARG,
+           "sel_ids must be non-NULL and 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  DecodeArgs a = decode_args(q, idx, nullptr, nullptr, sel_ids, retr_rows, workspace);
+  e = launch_select(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  return RI_OK;
+}
+
+ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                             const void* q, const ri_index* idx, const void* exec_K,
+                             const void* exec_V, int32_t exec_rows, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  ri_status st = prepare_decode(cfg, dcfg, q, idx, workspace, workspace_bytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  RI_CHECK((exec_K == nullptr) == (exec_V == nullptr), RI_ERR_INVALID_ARG,
+           "exec_K and exec_V must be both NULL or both non-NULL");
+  if (exec_K) {
+    RI_CHECK(aligned16(exec_K) && aligned16(exec_V), RI_ERR_INVALID_ARG,
+             "exec buffers must be 16-byte aligned");
+    RI_CHECK(exec_rows >= 1, RI_ERR_INVALID_ARG, "exec_rows must be >= 1");
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a = decode_args(q, idx, out, lse, nullptr, nullptr, workspace);
+  a.exec_K = exec_K;
+  a.exec_V = exec_V;
+  a.exec_rows = exec_rows;
+  cudaError_t e = launch_attend(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+  return RI_OK;
+}
+
+ri_status ri_read_device_status(const void* workspace, ri_stream_t stream) {
+  RI_CHECK(workspace, RI_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+  if (v != RI_OK) set_error("device reported: %s", ri_status_string((ri_status)v));
+  return (ri_status)v;
+}
+
+ri_status ri_selftest_wait_timeout(void* workspace, uint64_t limit_ns, ri_stream_t stream) {
+  RI_CHECK(workspace && aligned16(workspace), RI_ERR_INVALID_ARG,
+           "workspace must be non-NULL and 16-byte aligned");
+  RI_CHECK(limit_ns > 0 && limit_ns <= 10ull * 1000000000ull, RI_ERR_INVALID_ARG,
+           "limit_ns must be in (0, 10 s]");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  e = launch_wait_timeout_selftest(static_cast<int*>(workspace), limit_ns, s);
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return RI_OK;
+}
+
+}  // extern "C"

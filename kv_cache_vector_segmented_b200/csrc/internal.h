@@ -1,0 +1,104 @@
+// Host-side shapes, workspace layouts and kernel launchers shared by the
+// C ABI (api.cpp) and the CUDA translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "retroinfer.h"
+
+namespace ri {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kMaxGroupHost = 8;          // query heads per KV head
+constexpr size_t kStatusBytesHost = 256;  // status word region at workspace start
+
+// Everything derived from an ri_index_config.
+struct Geometry {
+  int B, H, G, d, N;
+  int seg_len, K;          // tokens per segment, clusters per full segment
+  int iters;
+  int s0, s1;              // steady initial / recent
+  int M;                   // middle tokens
+  int S;                   // segments
+  int C;                   // clusters per (b, h)
+  int n_steady;            // steady tokens per (b, h)
+  int m0;                  // first middle position
+  int K_full;              // clusters of a full segment = min(K, seg_len)
+  int L_last, K_last;      // length / clusters of the last segment
+  int tiles_full, tiles_last, tiles_bh;  // 128-row assignment tiles
+  long long BH() const { return (long long)B * H; }
+};
+
+// Returns false (and sets the thread's last error) for an invalid config.
+bool make_geometry(const ri_index_config* cfg, Geometry* g);
+
+// --------------------------------------------------------------- decode
+struct DecodeLayout {
+  int k_r, k_e;     // requested budgets (sizes of the sel regions)
+  int kr, ke;       // clamped to C
+  int P;            // splits per (b, h) in the attention step
+  size_t off_rkey, off_score, off_sel, off_rpre, off_part, total;
+};
+constexpr int kPartStride = 132;  // m, l, 2 pad, o[128]
+
+bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L);
+
+struct DecodeArgs {
+  const void* q;
+  const void* centroid;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* vsum;
+  const void* Kp;
+  const void* Vp;
+  const void* Ks;
+  const void* Vs;
+  const void* exec_K;  // NULL: read Kp/Vp in place
+  const void* exec_V;
+  int exec_rows;
+  void* out;
+  float* lse;
+  int32_t* sel_user;
+  int32_t* rpre_user;
+  char* ws;
+};
+
+cudaError_t launch_select(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
+                          cudaStream_t s);
+cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
+                          cudaStream_t s);
+
+// --------------------------------------------------------------- build
+struct BuildLayout {
+  // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); norm2 fp32
+  // [BH*S][512] (+inf past K_s); mumax fp32 [BH*S] (max ||mu||); counts int32
+  // [BH][C]; labels int32 [BH][M]; knorm fp32 [BH][M] (||k||).
+  size_t off_mu, off_mu_bf16, off_norm2, off_mumax, off_counts, off_labels, off_knorm, total;
+};
+bool make_build_layout(const Geometry& g, BuildLayout* L);
+
+struct BuildArgs {
+  const void* K;
+  const void* V;
+  const int32_t* init_pos;
+  ri_index out;
+  char* ws;
+};
+
+ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs& a,
+                       cudaStream_t s);
+
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
+                                         cudaStream_t s);
+
+// Thread-local last error.
+void set_error(const char* fmt, ...);
+int num_sms();
+// Raises a kernel's dynamic shared memory limit once per device (outside any
+// stream capture after the first call on that device).
+cudaError_t set_smem_once(const void* func, int bytes);
+
+}  // namespace ri

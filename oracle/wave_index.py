@@ -77,23 +77,22 @@ def bf16_round(x) -> np.ndarray:
 # --------------------------------------------------------------------------
 # zones and segments  [P2 §2.1; P1 三; P4 §2A]
 # --------------------------------------------------------------------------
-def steady_positions(N: int) -> np.ndarray:
+def steady_positions(N: int, s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT) -> np.ndarray:
     """Token positions of the steady zone, in position order.
 
     [P2 §2.1 item 1]: the first 4 and the most recent 64 tokens.  With
     N <= 68 every token is steady."""
-    if N <= STEADY_INITIAL + STEADY_RECENT:
+    if N <= s0 + s1:
         return np.arange(N, dtype=np.int64)
-    return np.concatenate([np.arange(STEADY_INITIAL),
-                           np.arange(N - STEADY_RECENT, N)]).astype(np.int64)
+    return np.concatenate([np.arange(s0), np.arange(N - s1, N)]).astype(np.int64)
 
 
-def middle_range(N: int) -> tuple[int, int]:
+def middle_range(N: int, s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT) -> tuple[int, int]:
     """(first position, count M) of the indexed middle tokens [4, N-64).
 
     Reading: the steady tokens are not indexed, so no token is counted twice."""
-    M = max(0, N - STEADY_INITIAL - STEADY_RECENT)
-    return (STEADY_INITIAL if M > 0 else 0), M
+    M = max(0, N - s0 - s1)
+    return (s0 if M > 0 else 0), M
 
 
 def segments(M: int, seg_len: int = SEGMENT_TOKENS,
@@ -181,7 +180,9 @@ def kmeans(X: np.ndarray, init_pos, iters: int) -> dict:
 
 
 def finalise(Kh: np.ndarray, Vh: np.ndarray, N: int, seg_labels: list[np.ndarray],
-             seg_mu: list[np.ndarray]) -> dict:
+             seg_mu: list[np.ndarray], seg_len: int = SEGMENT_TOKENS,
+             clusters_per_seg: int = CLUSTERS_PER_SEGMENT, s0: int = STEADY_INITIAL,
+             s1: int = STEADY_RECENT) -> dict:
     """Index of one (sequence, KV head) from per-segment labels and centroids.
 
     * cluster-contiguous layout [P2 §3.1: the KV vectors of one cluster are
@@ -196,8 +197,8 @@ def finalise(Kh: np.ndarray, Vh: np.ndarray, N: int, seg_labels: list[np.ndarray
     Kh, Vh: fp64 [N][d] (exact widenings of the bf16 inputs).  Positions in
     `perm` are absolute token positions."""
     d = Kh.shape[1]
-    m0, M = middle_range(N)
-    segs = segments(M)
+    m0, M = middle_range(N, s0, s1)
+    segs = segments(M, seg_len, clusters_per_seg)
     C = sum(s[2] for s in segs)
     perm = np.empty(M, dtype=np.int64)
     counts = np.zeros(C, dtype=np.int64)
@@ -219,13 +220,15 @@ def finalise(Kh: np.ndarray, Vh: np.ndarray, N: int, seg_labels: list[np.ndarray
         mu_all[cbase:cbase + Ks] = mu
         cbase += Ks
     offsets[C] = M
-    sp = steady_positions(N)
+    sp = steady_positions(N, s0, s1)
     return dict(N=N, C=C, perm=perm, counts=counts, offsets=offsets,
                 centroid=centroid, vsum=vsum, mu=mu_all,
                 Kp=Kh[perm], Vp=Vh[perm], Ks=Kh[sp], Vs=Vh[sp])
 
 
-def build_index_head(Kh, Vh, init_pos=None, iters: int = DEFAULT_ITERS) -> dict:
+def build_index_head(Kh, Vh, init_pos=None, iters: int = DEFAULT_ITERS,
+                     seg_len: int = SEGMENT_TOKENS, clusters_per_seg: int = CLUSTERS_PER_SEGMENT,
+                     s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT) -> dict:
     """Segmented clustering of one (sequence, KV head) [P2 §2.1 pseudocode]:
     k-means on every segment independently, then `finalise`.
 
@@ -235,10 +238,10 @@ def build_index_head(Kh, Vh, init_pos=None, iters: int = DEFAULT_ITERS) -> dict:
     Kh = np.asarray(Kh, dtype=np.float64)
     Vh = np.asarray(Vh, dtype=np.float64)
     N = Kh.shape[0]
-    m0, M = middle_range(N)
+    m0, M = middle_range(N, s0, s1)
     labs, mus, objs, hists = [], [], [], []
     cbase = 0
-    for start, L, Ks in segments(M):
+    for start, L, Ks in segments(M, seg_len, clusters_per_seg):
         X = Kh[m0 + start:m0 + start + L]
         ip = strided_init(L, Ks) if init_pos is None else np.asarray(init_pos[cbase:cbase + Ks])
         res = kmeans(X, ip, iters)
@@ -247,14 +250,16 @@ def build_index_head(Kh, Vh, init_pos=None, iters: int = DEFAULT_ITERS) -> dict:
         objs.append(objective(X, res["labels"], res["mu"]))
         hists.append(res["history"])
         cbase += Ks
-    idx = finalise(Kh, Vh, N, labs, mus)
+    idx = finalise(Kh, Vh, N, labs, mus, seg_len, clusters_per_seg, s0, s1)
     idx["labels"] = labs
     idx["objective"] = np.array(objs)
     idx["history"] = hists
     return idx
 
 
-def index_from_labels(Kh, Vh, labels_middle: np.ndarray) -> dict:
+def index_from_labels(Kh, Vh, labels_middle: np.ndarray, seg_len: int = SEGMENT_TOKENS,
+                      clusters_per_seg: int = CLUSTERS_PER_SEGMENT, s0: int = STEADY_INITIAL,
+                      s1: int = STEADY_RECENT) -> dict:
     """Index of one head from given labels of the middle tokens (cluster id
     within the segment), centroids = member means (0 for empty clusters).
 
@@ -263,15 +268,15 @@ def index_from_labels(Kh, Vh, labels_middle: np.ndarray) -> dict:
     Kh = np.asarray(Kh, dtype=np.float64)
     Vh = np.asarray(Vh, dtype=np.float64)
     N = Kh.shape[0]
-    m0, M = middle_range(N)
+    m0, M = middle_range(N, s0, s1)
     labs, mus = [], []
-    for start, L, Ks in segments(M):
+    for start, L, Ks in segments(M, seg_len, clusters_per_seg):
         lab = np.asarray(labels_middle[start:start + L], dtype=np.int64)
         X = Kh[m0 + start:m0 + start + L]
         mu, _ = update(X, lab, np.zeros((Ks, Kh.shape[1])))
         labs.append(lab)
         mus.append(mu)
-    idx = finalise(Kh, Vh, N, labs, mus)
+    idx = finalise(Kh, Vh, N, labs, mus, seg_len, clusters_per_seg, s0, s1)
     idx["labels"] = labs
     return idx
 

@@ -58,7 +58,7 @@ typedef enum {
  * are cut into contiguous segments of `seg_len` tokens (the last may be
  * short) and k-means runs on each segment with K_s = min(clusters_per_seg,
  * L_s) clusters.  Global cluster id = sum of K of earlier segments + local id.
- * Limits: 1 <= clusters_per_seg <= 512, seg_len >= 1, iters >= 0,
+ * Limits: 1 <= clusters_per_seg <= 512, 1 <= seg_len <= 16384, iters >= 0,
  * group_size 1..8, head_dim == 128. */
 typedef struct {
   int32_t batch;            /* B                                    */
@@ -137,7 +137,7 @@ ri_status ri_build_index(const ri_index_config* cfg, const void* K, const void* 
 
 /* Zone budgets in clusters: k_retrieval = round(0.018 C), k_estimation =
  * round(0.23 C) by default [P2 §2.1 items 2-3].  The zones are clamped to
- * C: R = top min(k_r, C), E = next min(k_e, C - |R|). */
+ * C: R = top min(k_r, C), E = next min(k_e, C - |R|).  k_retrieval <= 4096. */
 typedef struct {
   int32_t k_retrieval;
   int32_t k_estimation;

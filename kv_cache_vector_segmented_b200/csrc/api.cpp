@@ -72,8 +72,8 @@ bool make_geometry(const ri_index_config* cfg, Geometry* g) {
     set_error("head_dim must be 128 (got %d)", c.head_dim);
     return false;
   }
-  if (c.seg_len < 1 || c.seg_len > 32768) {
-    set_error("seg_len must be in [1, 32768] (got %d)", c.seg_len);
+  if (c.seg_len < 1 || c.seg_len > kMaxSegLen) {
+    set_error("seg_len must be in [1, %d] (got %d)", kMaxSegLen, c.seg_len);
     return false;
   }
   if (c.clusters_per_seg < 1 || c.clusters_per_seg > 512) {
@@ -132,8 +132,8 @@ bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeL
     set_error("k_retrieval and k_estimation must be >= 0");
     return false;
   }
-  if (dcfg->k_retrieval > 8192) {
-    set_error("k_retrieval must be <= 8192 (got %d)", dcfg->k_retrieval);
+  if (dcfg->k_retrieval > kMaxRetrieval) {
+    set_error("k_retrieval must be <= %d (got %d)", kMaxRetrieval, dcfg->k_retrieval);
     return false;
   }
   if ((long long)dcfg->k_retrieval + dcfg->k_estimation > (1 << 24)) {
@@ -145,21 +145,17 @@ bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeL
   L->kr = L->k_r < g.C ? L->k_r : g.C;
   L->ke = L->k_e < g.C - L->kr ? L->k_e : g.C - L->kr;
   const long long BH = g.BH();
-  int P = (int)((2 * 148 + BH - 1) / BH);
-  if (P < 1) P = 1;
-  if (P > 64) P = 64;
-  L->P = P;
-  size_t off = kStatusBytesHost;
+  if (!decode_plan(g, L)) return false;
+  L->header_bytes = kStatusBytesHost;
+  size_t off = L->header_bytes;
   L->off_rkey = off;
   off = align_up(off + (size_t)BH * g.C * 4, 256);
   L->off_score = off;
-  off = align_up(off + (size_t)BH * g.G * g.C * 4, 256);
+  off = align_up(off + (size_t)BH * 8 * g.C * 4, 256);
   L->off_sel = off;
   off = align_up(off + (size_t)BH * (L->k_r + L->k_e) * 4, 256);
   L->off_rpre = off;
   off = align_up(off + (size_t)BH * (L->k_r + 1) * 4, 256);
-  L->off_part = off;
-  off = align_up(off + (size_t)BH * P * g.G * kPartStride * 4, 256);
   L->total = off;
   return true;
 }
@@ -171,16 +167,18 @@ bool make_build_layout(const Geometry& g, BuildLayout* L) {
   off = align_up(off + BH * g.C * 128 * 4, 1024);
   L->off_mu_bf16 = off;
   off = align_up(off + BH * g.C * 128 * 2, 1024);
-  L->off_norm2 = off;
-  off = align_up(off + BH * g.S * 512 * 4, 256);
-  L->off_mumax = off;
-  off = align_up(off + BH * g.S * 4, 256);
+  L->off_colt = off;
+  off = align_up(off + BH * g.S * 1024 * 4, 256);
+  L->off_ust = off;
+  off = align_up(off + BH * g.S * 2 * 4, 256);
   L->off_counts = off;
   off = align_up(off + BH * g.C * 4, 256);
   L->off_labels = off;
   off = align_up(off + BH * g.M * 4, 256);
   L->off_knorm = off;
   off = align_up(off + BH * g.M * 4, 256);
+  L->off_queue = off;
+  off = align_up(off + build_queue_bytes((long long)BH * g.M), 256);
   L->total = off;
   return true;
 }
@@ -362,13 +360,11 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
   RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
   RI_CHECK(!sel_ids || aligned16(sel_ids), RI_ERR_INVALID_ARG, "sel_ids must be 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, workspace);
-  e = launch_select(g, L, a, s);
-  if (e != cudaSuccess) return cuda_fail(e, "select launch");
-  e = launch_attend(g, L, a, s);
-  if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+  e = launch_decode(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RI_OK;
 }
 
@@ -383,7 +379,7 @@ ri_status ri_select_clusters(const ri_index_config* cfg, const ri_decode_config*
   RI_CHECK(sel_ids && aligned16(sel_ids), RI_ERR_INVALID_ARG,
            "sel_ids must be non-NULL and 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, nullptr, nullptr, sel_ids, retr_rows, workspace);
   e = launch_select(g, L, a, s);
@@ -408,11 +404,14 @@ ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config*
     RI_CHECK(exec_rows >= 1, RI_ERR_INVALID_ARG, "exec_rows must be >= 1");
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // keeps the selection; clears only the status word and the counters
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, out, lse, nullptr, nullptr, workspace);
   a.exec_K = exec_K;
   a.exec_V = exec_V;
   a.exec_rows = exec_rows;
-  cudaError_t e = launch_attend(g, L, a, s);
+  e = launch_attend(g, L, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "attend launch");
   return RI_OK;
 }

@@ -39,10 +39,13 @@ bool make_geometry(const ri_index_config* cfg, Geometry* g);
 struct DecodeLayout {
   int k_r, k_e;     // requested budgets (sizes of the sel regions)
   int kr, ke;       // clamped to C
-  int P;            // splits per (b, h) in the attention step
-  size_t off_rkey, off_score, off_sel, off_rpre, off_part, total;
+  int P;            // blocks per (b, h) unit of the decode kernel
+  // status word [0, 256); rkey fp32 [BH][C], score fp32 [BH][C][8], sel int32
+  // [BH][k_r + k_e], rpre int32 [BH][k_r + 1].
+  size_t header_bytes, off_rkey, off_score, off_sel, off_rpre, total;
 };
-constexpr int kPartStride = 132;  // m, l, 2 pad, o[128]
+constexpr int kPartStride = 132;     // m, l, 2 pad, o[128]
+constexpr int kMaxRetrieval = 4096;  // retrieval clusters per unit held on chip
 
 bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L);
 
@@ -66,18 +69,28 @@ struct DecodeArgs {
   char* ws;
 };
 
+cudaError_t launch_decode(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
+                          cudaStream_t s);
 cudaError_t launch_select(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
+// Chooses the blocks per unit (cluster size) of the decode kernel.
+bool decode_plan(const Geometry& g, DecodeLayout* L);
 cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
 
 // --------------------------------------------------------------- build
+constexpr int kMaxSegLen = 16384;  // segment tokens (member lists live in shared memory)
+
 struct BuildLayout {
-  // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); norm2 fp32
-  // [BH*S][512] (+inf past K_s); mumax fp32 [BH*S] (max ||mu||); counts int32
-  // [BH][C]; labels int32 [BH][M]; knorm fp32 [BH][M] (||k||).
-  size_t off_mu, off_mu_bf16, off_norm2, off_mumax, off_counts, off_labels, off_knorm, total;
+  // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); colt fp32
+  // [BH*S][2][512] (||mu_j||^2, +inf past K_s; error coefficient e_j);
+  // ust fp32 [BH*S][2] (max e_j, max c_j); counts int32 [BH][C]; labels int32
+  // [BH][M]; knorm fp32 [BH][M] (||k||); queue of rows for the exact fix-up
+  // [BH*M] entries.
+  size_t off_mu, off_mu_bf16, off_colt, off_ust, off_counts, off_labels, off_knorm, off_queue,
+      total;
 };
+size_t build_queue_bytes(long long rows);
 bool make_build_layout(const Geometry& g, BuildLayout* L);
 
 struct BuildArgs {

@@ -5,17 +5,25 @@
 // parallel, centroids plus per-cluster value sums) and the cluster-contiguous
 // layout (§3.1: the KV vectors of one cluster stored contiguously).
 //
-// One Lloyd iteration = assignment (tensor cores) + update (segmented sums).
-//   assignment: label_i = argmin_j ||k_i - mu_j||^2
-//             = argmin_j (||mu_j||^2 - 2 k_i . mu_j), ties to the lower j.
-//     tcgen05 MMA: 128 keys x 256 centroids x 128 dims per instruction group,
-//     bf16 operands (keys exact in bf16, centroids rounded to bf16), fp32
-//     accumulators in TMEM.  The bf16 centroid costs at most
-//     2^-7 ||k|| ||mu_j|| in the distance (|mu - bf16(mu)| <= 2^-8 |mu| per
-//     element, Cauchy-Schwarz), plus fp32 accumulation error; every centroid
-//     whose approximate distance lies within twice that bound of the best is
-//     re-evaluated exactly in fp32 (direct difference form).
-//   update: mu_j = mean of members (fp32), an empty cluster keeps mu_j.
+// One Lloyd iteration = assignment (tensor cores) + exact fix-up of near ties
+// + update (segmented sums).
+//
+// Assignment: label = argmin_j ||k - mu_j||^2 = argmin_j (||mu_j||^2 - 2 k.mu_j),
+// ties to the lower j.  tcgen05 MMA computes v_j = k . bf16(mu_j) for 128 keys x
+// 256 centroids per instruction group (keys are exact in bf16; fp32
+// accumulators in TMEM).  a_j = ||mu_j||^2 - 2 v_j then differs from the exact
+// criterion by at most
+//     eps_j(k) = ||k|| e_j + c_j,
+//     e_j = 2 ||mu_j - bf16(mu_j)||  (+ 2^-14 ||mu_j|| for the fp32 accumulation)
+//     c_j = 2^-15 (||mu_j||^2 + 1)   (rounding of ||mu_j||^2 and of a_j)
+// (Cauchy-Schwarz on the rounding residual; n * 2^-23 accumulation bounds with
+// a factor-2 margin).  A centroid can be the exact argmin only if
+// a_j - eps_j <= min_i (a_i + eps_i); when more than one centroid passes, the
+// row is queued and a fix-up kernel decides it exactly in fp32.
+//
+// Update: mu_j = mean of the members (fp32), an empty cluster keeps mu_j; the
+// members of a cluster are gathered in position order, so sums are
+// deterministic.
 #include <float.h>
 #include <math.h>
 
@@ -30,21 +38,30 @@ constexpr int kRows = 128;        // keys per tile = MMA M
 constexpr int kHalfN = 256;       // centroids per MMA = MMA N
 constexpr int kStages = 2;        // key tile ring
 constexpr int kAssignThreads = 192;
+constexpr int kCand = 8;          // candidate slots per row
 constexpr int kUpdateWarps = 8;
 constexpr int kClustersPerWarp = 4;
 constexpr int kClustersPerBlock = kUpdateWarps * kClustersPerWarp;  // 32
-constexpr int kMemberBuf = 256;   // member token queue per warp (update/finalise)
+constexpr uint16_t kCandNone = 0xFFFF;
+constexpr uint16_t kCandFullScan = 0xFFFE;
 
 // Shared memory of the assignment kernel (from a 1024-byte aligned base).
 constexpr uint32_t kSmCent = 0;                                // [2 k-halves][512][128 B]
 constexpr uint32_t kCentHalfK = 512 * 128;                     // 64 KB
 constexpr uint32_t kSmKeys = 2 * kCentHalfK;                   // 128 KB
 constexpr uint32_t kKeyStage = 2 * kRows * 128;                // 32 KB
-constexpr uint32_t kSmNrm = kSmKeys + kStages * kKeyStage;     // [2][512] fp32
-constexpr uint32_t kSmBar = kSmNrm + 2 * 512 * 4;
+constexpr uint32_t kSmCol = kSmKeys + kStages * kKeyStage;     // [2 buf][2][512] fp32
+constexpr uint32_t kColBytes = 2 * 512 * 4;                    // n_j then e_j
+constexpr uint32_t kSmBar = kSmCol + 2 * kColBytes;
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
 constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
 constexpr uint32_t kAssignSmem = kSmMisc + 64 + 1024;          // + alignment slack
+
+// Queue of rows whose label needs an exact decision.
+struct FixEntry {
+  int32_t row;             // bh * M + position in the middle
+  uint16_t cand[kCand];    // candidate cluster ids within the segment
+};
 
 struct UnitInfo {
   int bh, s, unit, seg_start, L, Ks, cbase, tile;
@@ -72,42 +89,85 @@ __device__ __forceinline__ UnitInfo tile_info(const BuildDims& d, long long f) {
   return u;
 }
 
-// Exact squared distance in fp32 between row `row` of a swizzled key tile in
-// shared memory (two 64-column halves of 128-byte rows) and an fp32 centroid.
-__device__ __forceinline__ float exact_dist(const uint8_t* tile, int row, const float* mu) {
-  float acc = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < 16; ++c) {
-    const int kh = c >> 3, ch = c & 7;
-    const uint4 raw = *reinterpret_cast<const uint4*>(tile + kh * (kRows * 128) + row * 128 +
-                                                      ((ch ^ (row & 7)) << 4));
-    float k[8];
-    bf16x8_to_float(raw, k);
-    const float4 m0 = *reinterpret_cast<const float4*>(mu + c * 8);
-    const float4 m1 = *reinterpret_cast<const float4*>(mu + c * 8 + 4);
-    const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+__device__ __forceinline__ float col_c(float n) { return 3.0517578125e-05f * (n + 1.f); }
+
+__device__ __forceinline__ void atomic_max_pos(float* addr, float v) {
+  atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));  // v >= 0
+}
+
+// Column constants of one centroid from its fp32 row (lane holds 4 dims):
+// n = ||mu||^2, e = error coefficient of the bf16 operand (see file header).
+// Writes the packed bf16 row and the table entries; lane 0 raises the unit's
+// maxima (E, Cmax).
+__device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf_row,
+                                               float* col_n, float* col_e, float* ust_unit,
+                                               int lane, bool write_bf16) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
+  if (write_bf16) {
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(bf_row + lane * 4) = packed;
+  }
+  const float2 l2 = __bfloat1622float2(lo), h2 = __bfloat1622float2(hi);
+  const float r0 = m.x - l2.x, r1 = m.y - l2.y, r2 = m.z - h2.x, r3 = m.w - h2.y;
+  float sq = m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
+  float rr = r0 * r0 + r1 * r1 + r2 * r2 + r3 * r3;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float t = k[i] - mm[i];
-      acc = fmaf(t, t, acc);
+  for (int off = 16; off >= 1; off >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    rr += __shfl_xor_sync(0xffffffffu, rr, off);
+  }
+  if (lane == 0) {
+    const float e = 2.f * sqrtf(rr) * 1.0001f + 6.1035156e-05f * sqrtf(sq) + 1e-30f;
+    *col_n = sq;
+    *col_e = e;
+    atomic_max_pos(&ust_unit[0], e);
+    atomic_max_pos(&ust_unit[1], col_c(sq));
+  }
+}
+
+// Ascending 8-slot candidate list; insert returns the value pushed out.
+struct CandList {
+  float a[kCand];
+  int j[kCand];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int i = 0; i < kCand; ++i) {
+      a[i] = FLT_MAX;
+      j[i] = -1;
     }
   }
-  return acc;
-}
+  __device__ __forceinline__ float insert(float na, int nj) {
+#pragma unroll
+    for (int i = 0; i < kCand; ++i) {
+      if (na < a[i]) {
+        const float tf = a[i];
+        const int ti = j[i];
+        a[i] = na;
+        j[i] = nj;
+        na = tf;
+        nj = ti;
+      }
+    }
+    return na;
+  }
+};
 
 // ------------------------------------------------------------- assignment
 __global__ void __launch_bounds__(kAssignThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tm_keys,
                   const __grid_constant__ CUtensorMap tm_cent, BuildDims d,
-                  const float* __restrict__ knorm, const float* __restrict__ norm2,
-                  const float* __restrict__ mumax, const float* __restrict__ mu,
-                  int32_t* __restrict__ labels, int* status) {
+                  const float* __restrict__ knorm, const float* __restrict__ colt,
+                  const float* __restrict__ ust, int32_t* __restrict__ labels,
+                  FixEntry* __restrict__ queue, int* __restrict__ queue_count, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* cent = sm + kSmCent;
   uint8_t* keys = sm + kSmKeys;
-  float* nrm = reinterpret_cast<float*>(sm + kSmNrm);
+  float* colsm = reinterpret_cast<float*>(sm + kSmCol);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
   uint64_t* full = bars;                       // [kStages] TMA -> MMA
   uint64_t* empty = bars + kStages;            // [kStages] epilogue -> TMA
@@ -115,9 +175,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   uint64_t* cent_empty = cent_full + 1;        // MMA -> TMA
   uint64_t* tfull = cent_full + 2;             // [2] MMA -> epilogue
   uint64_t* tempty = tfull + 2;                // [2] epilogue -> MMA
-  uint64_t* nfull = tempty + 2;                // [2] TMA -> epilogue (norms)
-  uint64_t* nempty = nfull + 2;                // [2] epilogue -> TMA  (uses 1 slot each)
-  uint64_t* drain = nfull + 4;                 // MMA drain
+  uint64_t* nfull = tempty + 2;                // [2] TMA -> epilogue (column table)
+  uint64_t* nempty = nfull + 2;                // [2] epilogue -> TMA
+  uint64_t* drain = nempty + 2;                // MMA drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSmMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kSmMisc + 8);
   const int warp = threadIdx.x >> 5;
@@ -162,7 +222,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     uint32_t ce_phase = 0;
     long long it = 0;
     int issued[kStages] = {0, 0};
-    int cent_loads = 0, nrm_loads[2] = {0, 0};
+    int cent_loads = 0, col_loads[2] = {0, 0};
     for (long long f = f_begin; f < f_end; ++f, ++it) {
       if (*abort_flag) break;
       const UnitInfo u = tile_info(d, f);
@@ -182,7 +242,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             tma_load_2d(cent + kh * kCentHalfK + h * kHalfN * 128, &tm_cent, kh * 64,
                         crow + h * kHalfN, cent_full);
         ++cent_loads;
-        // per-unit squared centroid norms for the epilogue (double buffer)
         const int nb = nunits & 1;
         if (nunits >= 2) {
           if (!mbar_wait(&nempty[nb], ((nunits >> 1) - 1) & 1)) {
@@ -191,9 +250,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             break;
           }
         }
-        mbar_arrive_expect_tx(&nfull[nb], 512 * 4);
-        bulk_load(nrm + nb * 512, norm2 + (size_t)u.unit * 512, 512 * 4, &nfull[nb]);
-        ++nrm_loads[nb];
+        mbar_arrive_expect_tx(&nfull[nb], kColBytes);
+        bulk_load(colsm + nb * 1024, colt + (size_t)u.unit * 1024, kColBytes, &nfull[nb]);
+        ++col_loads[nb];
         ++nunits;
         prev_unit = u.unit;
       }
@@ -217,7 +276,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       if (issued[st]) mbar_wait(&full[st], (uint32_t)((issued[st] - 1) & 1));
     if (cent_loads) mbar_wait(cent_full, (uint32_t)((cent_loads - 1) & 1));
     for (int nb = 0; nb < 2; ++nb)
-      if (nrm_loads[nb]) mbar_wait(&nfull[nb], (uint32_t)((nrm_loads[nb] - 1) & 1));
+      if (col_loads[nb]) mbar_wait(&nfull[nb], (uint32_t)((col_loads[nb] - 1) & 1));
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = umma_idesc_bf16_f32(kRows, kHalfN);
@@ -277,7 +336,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     int prev_unit = -1, nunits = 0;
-    float mx = 0.f;
+    float uE = 0.f, uC = 0.f;
     long long it = 0;
     for (long long f = f_begin; f < f_end; ++f, ++it) {
       if (*abort_flag) break;
@@ -289,19 +348,19 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           *abort_flag = 1;
           break;
         }
-        mx = mumax[u.unit];
+        uE = ust[2 * u.unit];
+        uC = ust[2 * u.unit + 1];
         ++nunits;
         prev_unit = u.unit;
       }
-      const float* nr = nrm + ((nunits - 1) & 1) * 512;
+      const float* cn = colsm + ((nunits - 1) & 1) * 1024;  // n_j
+      const float* ce = cn + 512;                             // e_j
       const int t = u.tile * kRows + row;  // token within the segment
       const bool valid = t < u.L;
       const float kn = valid ? knorm[(size_t)u.bh * d.M + u.seg_start + t] : 0.f;
-      // bound on |approx - exact| of one distance, doubled for the window
-      const float eps = 0.0078125f * 1.0157f * kn * mx + 3.0517578e-5f * (kn * kn + mx * mx);
-      const float win = 2.f * eps;
-      float a0 = FLT_MAX, a1 = FLT_MAX, a2 = FLT_MAX, a3 = FLT_MAX;
-      int j0 = -1, j1 = -1, j2 = -1, j3 = -1;
+      const float loose = 2.f * (kn * uE + uC);  // window of the streaming filter
+      CandList cl;
+      cl.init();
       float dropped = FLT_MAX, thr = FLT_MAX;
       bool ok = true;
       for (int h = 0; h < 2; ++h) {
@@ -317,16 +376,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           const int jb = h * kHalfN + ch * 32;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float a = fmaf(-2.f, v[i], nr[jb + i]);
+            const float a = fmaf(-2.f, v[i], cn[jb + i]);
             if (a <= thr) {
-              float na = a;
-              int nj = jb + i;
-              if (na < a0) { float tf = a0; a0 = na; na = tf; int ti = j0; j0 = nj; nj = ti; }
-              if (na < a1) { float tf = a1; a1 = na; na = tf; int ti = j1; j1 = nj; nj = ti; }
-              if (na < a2) { float tf = a2; a2 = na; na = tf; int ti = j2; j2 = nj; nj = ti; }
-              if (na < a3) { float tf = a3; a3 = na; na = tf; int ti = j3; j3 = nj; nj = ti; }
-              dropped = fminf(dropped, na);
-              thr = a0 + win;
+              dropped = fminf(dropped, cl.insert(a, jb + i));
+              thr = cl.a[0] + loose;
             }
           }
         }
@@ -338,41 +391,42 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         *abort_flag = 1;
         break;
       }
-      const int stage = (int)(it % kStages);
-      const uint8_t* tile = keys + stage * kKeyStage;
-      int label = (j0 < 0 || j0 >= u.Ks) ? 0 : j0;
-      if (valid && j0 >= 0 && j0 < u.Ks) {
-        const float lim = a0 + win;
-        const int nc = (a1 <= lim) + (a2 <= lim) + (a3 <= lim);
-        const float* mub = mu + ((size_t)u.bh * d.C + u.cbase) * kHeadDim;
-        if (dropped <= lim) {
-          // more near-ties than the candidate list holds: exact scan
-          float best = FLT_MAX;
-          for (int j = 0; j < u.Ks; ++j) {
-            const float e = exact_dist(tile, row, mub + (size_t)j * kHeadDim);
-            if (e < best) {
-              best = e;
-              label = j;
-            }
-          }
-        } else if (nc > 0) {
-          float best = exact_dist(tile, row, mub + (size_t)j0 * kHeadDim);
-          label = j0;
-          const int cj[3] = {j1, j2, j3};
+      if (valid) {
+        // exact-argmin candidates: lower bound <= least upper bound
+        float U = FLT_MAX;
 #pragma unroll
-          for (int c = 0; c < 3; ++c) {
-            if (c < nc && cj[c] >= 0 && cj[c] < u.Ks) {
-              const float e = exact_dist(tile, row, mub + (size_t)cj[c] * kHeadDim);
-              if (e < best || (e == best && cj[c] < label)) {
-                best = e;
-                label = cj[c];
-              }
-            }
+        for (int i = 0; i < kCand; ++i)
+          if (cl.j[i] >= 0) U = fminf(U, cl.a[i] + kn * ce[cl.j[i]] + col_c(cn[cl.j[i]]));
+        int nsurv = 0;
+        uint16_t cands[kCand];
+#pragma unroll
+        for (int i = 0; i < kCand; ++i) cands[i] = kCandNone;
+#pragma unroll
+        for (int i = 0; i < kCand; ++i) {
+          const bool s = cl.j[i] >= 0 && cl.j[i] < u.Ks &&
+                         cl.a[i] - kn * ce[cl.j[i]] - col_c(cn[cl.j[i]]) <= U;
+          if (s) {
+#pragma unroll
+            for (int k = 0; k < kCand; ++k)
+              if (k == nsurv) cands[k] = (uint16_t)cl.j[i];
+            ++nsurv;
           }
         }
+        // a dropped entry could still be a candidate: decide by a full scan
+        const bool overflow = dropped - 0.5f * loose <= U;
+        const int grow = u.bh * d.M + u.seg_start + t;
+        labels[grow] = (cl.j[0] >= 0 && cl.j[0] < u.Ks) ? cl.j[0] : 0;
+        if (overflow || nsurv != 1) {
+          FixEntry e;
+          e.row = grow;
+#pragma unroll
+          for (int i = 0; i < kCand; ++i) e.cand[i] = cands[i];
+          if (overflow || nsurv == 0) e.cand[0] = kCandFullScan;
+          const int qi = atomicAdd(queue_count, 1);
+          queue[qi] = e;
+        }
       }
-      if (valid) labels[(size_t)u.bh * d.M + u.seg_start + t] = label;
-      mbar_arrive(&empty[stage]);
+      mbar_arrive(&empty[(int)(it % kStages)]);
     }
   }
   __syncwarp();
@@ -382,8 +436,55 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// Exact fp32 decision for the queued rows: one warp per row, lane l holds
+// dims 4l..4l+3; distances in the direct difference form, reduced by a xor
+// butterfly (identical result on every lane), ties to the lower id.
+__global__ void __launch_bounds__(256)
+    fixup_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ mu, BuildDims d,
+                 const FixEntry* __restrict__ queue, const int* __restrict__ queue_count,
+                 int32_t* __restrict__ labels) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nw = (int)((gridDim.x * blockDim.x) >> 5);
+  const int n = *queue_count;
+  for (int e = gw; e < n; e += nw) {
+    const FixEntry en = queue[e];
+    const int bh = en.row / d.M;
+    const int m = en.row - bh * d.M;
+    const int s = m / d.seg_len;
+    const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+    const uint2 raw = *reinterpret_cast<const uint2*>(
+        K + ((size_t)bh * d.N + d.m0 + m) * kHeadDim + lane * 4);
+    const __nv_bfloat162* hk = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    const float2 k01 = __bfloat1622float2(hk[0]), k23 = __bfloat1622float2(hk[1]);
+    const float* mub = mu + ((size_t)bh * d.C + (size_t)s * d.K_full) * kHeadDim + lane * 4;
+    float best = FLT_MAX;
+    int bj = 0;
+    auto consider = [&](int j) {
+      const float4 mm = *reinterpret_cast<const float4*>(mub + (size_t)j * kHeadDim);
+      const float t0 = k01.x - mm.x, t1 = k01.y - mm.y, t2 = k23.x - mm.z, t3 = k23.y - mm.w;
+      float p = t0 * t0 + t1 * t1 + t2 * t2 + t3 * t3;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+      if (p < best || (p == best && j < bj)) {
+        best = p;
+        bj = j;
+      }
+    };
+    if (en.cand[0] == kCandFullScan) {
+      for (int j = 0; j < Ks; ++j) consider(j);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kCand; ++i)
+        if (en.cand[i] != kCandNone && en.cand[i] < Ks) consider(en.cand[i]);
+    }
+    if (lane == 0) labels[en.row] = bj;
+  }
+}
+
 // ------------------------------------------------------------- prep
-// ||k|| of every middle token (one warp per row).
+// ||k|| of every middle token (one warp per row), rounded up so bounds that
+// use it stay upper bounds.
 __global__ void knorm_kernel(const __nv_bfloat16* __restrict__ K, float* __restrict__ knorm,
                              int N, int M, int m0, long long rows) {
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -397,19 +498,15 @@ __global__ void knorm_kernel(const __nv_bfloat16* __restrict__ K, float* __restr
   float s = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) knorm[w] = sqrtf(s);
-}
-
-__device__ __forceinline__ void atomic_max_pos(float* addr, float v) {
-  atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));  // v >= 0
+  if (lane == 0) knorm[w] = sqrtf(s) * 1.0001f;
 }
 
 // Seeds: mu_j = k at the given (or strided) position of the segment.  One
-// warp per (bh, s, j in [0, 512)); j >= K_s only pads the norm table.
+// warp per (bh, s, j in [0, 512)); j >= K_s only pads the column table.
 __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
                             const int32_t* __restrict__ init_pos, BuildDims d,
                             float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                            float* __restrict__ norm2, float* __restrict__ mumax, int* status,
+                            float* __restrict__ colt, float* __restrict__ ust, int* status,
                             long long total) {
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -420,8 +517,12 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
   const bool last = s == d.S - 1;
   const int L = last ? d.L_last : d.seg_len;
   const int Ks = last ? d.K_last : d.K_full;
+  float* cn = colt + (size_t)unit * 1024;
   if (j >= Ks) {
-    if (lane == 0) norm2[(size_t)unit * 512 + j] = INFINITY;
+    if (lane == 0) {
+      cn[j] = INFINITY;
+      cn[512 + j] = 0.f;
+    }
     return;
   }
   const int c = s * d.K_full + j;
@@ -435,61 +536,76 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
   } else {
     p = (int)(((long long)j * L) / Ks);
   }
-  const __nv_bfloat16* src = K + ((size_t)bh * d.N + d.m0 + s * d.seg_len + p) * kHeadDim + lane * 4;
+  const __nv_bfloat16* src =
+      K + ((size_t)bh * d.N + d.m0 + (size_t)s * d.seg_len + p) * kHeadDim + lane * 4;
   const uint2 raw = *reinterpret_cast<const uint2*>(src);
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
   const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  float* dst = mu + ((size_t)bh * d.C + c) * kHeadDim + lane * 4;
-  *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, b.x, b.y);
-  *reinterpret_cast<uint2*>(mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim + lane * 4) = raw;
-  float sq = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-  if (lane == 0) {
-    norm2[(size_t)unit * 512 + j] = sq;
-    atomic_max_pos(&mumax[unit], sqrtf(sq));
-  }
+  const float4 m = make_float4(a.x, a.y, b.x, b.y);
+  *reinterpret_cast<float4*>(mu + ((size_t)bh * d.C + c) * kHeadDim + lane * 4) = m;
+  centroid_stats(m, mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim, &cn[j], &cn[512 + j],
+                 ust + 2 * unit, lane, true);
 }
 
 // ------------------------------------------------------------- update / finalise
-// Member scan shared by update and finalise: the warp walks the segment's
-// labels (shared memory, uint16) in position order and queues the tokens of
-// its clusters [jw, jw + 4); `visit(t, cl)` is called for each member in
-// position order, 8 row loads in flight at a time by the caller's batching.
-struct MemberQueue {
-  int buf[kMemberBuf];  // (t << 2) | cl
-};
-
-template <typename Visit>
-__device__ __forceinline__ void scan_members(const uint16_t* lab, int L, int jw, int nclw,
-                                             MemberQueue& q, Visit&& visit) {
-  const int lane = threadIdx.x & 31;
-  int pos = 0;
-  while (pos < L) {
-    int n = 0;
-    while (pos < L && n <= kMemberBuf - 32) {
-      const int t = pos + lane;
-      const int c = t < L ? (int)lab[t] - jw : -1;
-      const bool mine = c >= 0 && c < nclw;
-      const unsigned m = __ballot_sync(0xffffffffu, mine);
-      if (mine) q.buf[n + __popc(m & ((1u << lane) - 1u))] = (t << 2) | c;
-      n += __popc(m);
-      pos += 32;
+// Members of the block's clusters [j0, j0 + ncl) of one segment, in position
+// order, grouped by cluster: sorted[start[c] .. start[c+1]) are the positions
+// (within the segment) of cluster j0 + c.  Returns the member total.
+// Shared memory: list[L], sorted[L], start[33], wtot[8].
+__device__ int gather_members(const int32_t* __restrict__ lab, int L, int j0, int ncl,
+                              int* list, int* sorted, int* start, int* wtot) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  int run = 0;
+  // 1) compaction of (position, cluster) pairs, position order
+  for (int base = 0; base < L; base += blockDim.x) {
+    const int t = base + threadIdx.x;
+    const int c = t < L ? lab[t] - j0 : -1;
+    const bool mine = c >= 0 && c < ncl;
+    const unsigned m = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0) wtot[warp] = __popc(m);
+    __syncthreads();
+    int before = 0, tot = 0;
+    for (int w = 0; w < kUpdateWarps; ++w) {
+      before += w < warp ? wtot[w] : 0;
+      tot += wtot[w];
     }
-    __syncwarp();
-    visit(n);
-    __syncwarp();
+    if (mine) list[run + before + __popc(m & lt)] = (t << 5) | c;
+    run += tot;
+    __syncthreads();
   }
+  // 2) per-cluster counts and starts
+  if (threadIdx.x < 33) start[threadIdx.x] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < run; i += blockDim.x) atomicAdd(&start[(list[i] & 31) + 1], 1);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int c = 1; c <= 32; ++c) start[c] += start[c - 1];
+  __syncthreads();
+  // 3) stable grouping: warp w moves the members of clusters 4w..4w+3
+  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
+    const int c = warp * kClustersPerWarp + cc;
+    int pos = start[c];
+    for (int base = 0; base < run; base += 32) {
+      const int i = base + lane;
+      const int e = i < run ? list[i] : -1;
+      const bool mine = e >= 0 && (e & 31) == c;
+      const unsigned m = __ballot_sync(0xffffffffu, mine);
+      if (mine) sorted[pos + __popc(m & lt)] = e >> 5;
+      pos += __popc(m);
+    }
+  }
+  __syncthreads();
+  return run;
 }
 
 __global__ void __launch_bounds__(kUpdateWarps * 32)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ labels,
                   BuildDims d, float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                  float* __restrict__ norm2, float* __restrict__ mumax,
+                  float* __restrict__ colt, float* __restrict__ ust,
                   int32_t* __restrict__ counts, int update_mu) {
   extern __shared__ __align__(16) uint8_t smem_u[];
-  uint16_t* lab = reinterpret_cast<uint16_t*>(smem_u);
-  MemberQueue* queues = reinterpret_cast<MemberQueue*>(smem_u + (((size_t)d.seg_len * 2 + 15) & ~(size_t)15));
+  __shared__ int start[33], wtot[kUpdateWarps];
   const int unit = blockIdx.x;
   const int bh = unit / d.S, s = unit % d.S;
   const bool last = s == d.S - 1;
@@ -497,91 +613,62 @@ __global__ void __launch_bounds__(kUpdateWarps * 32)
   const int Ks = last ? d.K_last : d.K_full;
   const int j0 = blockIdx.y * kClustersPerBlock;
   if (j0 >= Ks) return;
+  const int ncl = min(kClustersPerBlock, Ks - j0);
+  int* list = reinterpret_cast<int*>(smem_u);
+  int* sorted = list + d.seg_len;
   const int seg_start = s * d.seg_len;
-  const int32_t* lsrc = labels + (size_t)bh * d.M + seg_start;
-  for (int t = threadIdx.x; t < L; t += blockDim.x) lab[t] = (uint16_t)lsrc[t];
-  __syncthreads();
+  gather_members(labels + (size_t)bh * d.M + seg_start, L, j0, ncl, list, sorted, start, wtot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int jw = j0 + warp * kClustersPerWarp;
-  const int nclw = max(0, min(kClustersPerWarp, Ks - jw));
-  if (nclw == 0) return;
-  MemberQueue& q = queues[warp];
-  float acc[kClustersPerWarp][4];
-  int n[kClustersPerWarp];
-#pragma unroll
-  for (int c = 0; c < kClustersPerWarp; ++c) {
-    n[c] = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[c][i] = 0.f;
-  }
   const __nv_bfloat16* kbase = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
-  scan_members(lab, L, jw, nclw, q, [&](int cnt) {
-    for (int i = 0; i < cnt; i += 8) {
-      uint2 raw[8];
-      int cl[8];
+  float* cn = colt + (size_t)unit * 1024;
+  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
+    const int c = warp * kClustersPerWarp + cc;
+    if (c >= ncl) break;
+    const int b = start[c], e = start[c + 1];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = b; i < e; i += 16) {
+      uint2 raw[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = i + u < cnt ? q.buf[i + u] : -1;
-        cl[u] = e < 0 ? -1 : (e & 3);
-        raw[u] = e < 0 ? make_uint2(0, 0)
-                       : *reinterpret_cast<const uint2*>(kbase + (size_t)(e >> 2) * kHeadDim);
-      }
+      for (int u = 0; u < 16; ++u)
+        raw[u] = i + u < e
+                     ? *reinterpret_cast<const uint2*>(kbase + (size_t)sorted[i + u] * kHeadDim)
+                     : make_uint2(0, 0);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-        const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-#pragma unroll
-        for (int c = 0; c < kClustersPerWarp; ++c) {
-          if (cl[u] == c) {
-            acc[c][0] += a.x;
-            acc[c][1] += a.y;
-            acc[c][2] += b.x;
-            acc[c][3] += b.y;
-            n[c] += 1;
-          }
+      for (int u = 0; u < 16; ++u) {
+        if (i + u < e) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+          const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
+          acc[0] += a.x;
+          acc[1] += a.y;
+          acc[2] += bb.x;
+          acc[3] += bb.y;
         }
       }
     }
-  });
-  float wmax = 0.f;
-#pragma unroll
-  for (int c = 0; c < kClustersPerWarp; ++c) {
-    if (c >= nclw) break;
-    const int j = jw + c;
-    const size_t row = (size_t)bh * d.C + s * d.K_full + j;
-    float* mrow = mu + row * kHeadDim + lane * 4;
-    float4 m;
-    if (update_mu && n[c] > 0) {
-      const float fn = (float)n[c];
-      m = make_float4(acc[c][0] / fn, acc[c][1] / fn, acc[c][2] / fn, acc[c][3] / fn);
-      *reinterpret_cast<float4*>(mrow) = m;
-      __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y), hi = __floats2bfloat162_rn(m.z, m.w);
-      uint2 packed;
-      packed.x = *reinterpret_cast<uint32_t*>(&lo);
-      packed.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(mu_bf16 + row * kHeadDim + lane * 4) = packed;
+    const int j = j0 + c;
+    const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+    const int n = e - b;
+    if (update_mu && n > 0) {
+      const float fn = (float)n;
+      const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
+      *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
+      centroid_stats(m, mu_bf16 + row * kHeadDim, &cn[j], &cn[512 + j], ust + 2 * unit, lane,
+                     true);
     } else {
-      m = *reinterpret_cast<const float4*>(mrow);
+      const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
+      centroid_stats(m, mu_bf16 + row * kHeadDim, &cn[j], &cn[512 + j], ust + 2 * unit, lane,
+                     false);
     }
-    float sq = m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    if (lane == 0) {
-      norm2[(size_t)unit * 512 + j] = sq;
-      counts[row] = n[c];
-    }
-    wmax = fmaxf(wmax, sqrtf(sq));
+    if (lane == 0) counts[row] = n;
   }
-  if (lane == 0) atomic_max_pos(&mumax[unit], wmax);
 }
 
 __global__ void __launch_bounds__(kUpdateWarps * 32)
     finalise_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                     const int32_t* __restrict__ labels, BuildDims d, const float* __restrict__ mu,
-                    const int32_t* __restrict__ counts_ws, ri_index out) {
+                    ri_index out) {
   extern __shared__ __align__(16) uint8_t smem_u[];
-  uint16_t* lab = reinterpret_cast<uint16_t*>(smem_u);
-  MemberQueue* queues = reinterpret_cast<MemberQueue*>(smem_u + (((size_t)d.seg_len * 2 + 15) & ~(size_t)15));
+  __shared__ int start[33], wtot[kUpdateWarps], before_sm;
   const int unit = blockIdx.x;
   const int bh = unit / d.S, s = unit % d.S;
   const bool last = s == d.S - 1;
@@ -589,111 +676,82 @@ __global__ void __launch_bounds__(kUpdateWarps * 32)
   const int Ks = last ? d.K_last : d.K_full;
   const int j0 = blockIdx.y * kClustersPerBlock;
   if (j0 >= Ks) return;
+  const int ncl = min(kClustersPerBlock, Ks - j0);
+  int* list = reinterpret_cast<int*>(smem_u);
+  int* sorted = list + d.seg_len;
   const int seg_start = s * d.seg_len;
   const int cbase = s * d.K_full;
-  const int32_t* lsrc = labels + (size_t)bh * d.M + seg_start;
-  for (int t = threadIdx.x; t < L; t += blockDim.x) {
-    const int v = lsrc[t];
-    lab[t] = (uint16_t)v;
-    if (out.labels && blockIdx.y == 0) out.labels[(size_t)bh * d.M + seg_start + t] = v;
-  }
+  const int32_t* lab = labels + (size_t)bh * d.M + seg_start;
+  if (out.labels && blockIdx.y == 0)
+    for (int t = threadIdx.x; t < L; t += blockDim.x)
+      out.labels[(size_t)bh * d.M + seg_start + t] = lab[t];
   if (blockIdx.y == 0 && s == d.S - 1 && threadIdx.x == 0)
     out.offsets[(size_t)bh * (d.C + 1) + d.C] = d.M;
+  // rows of the segment taken by clusters before j0: tokens with label < j0
+  if (threadIdx.x == 0) before_sm = 0;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int jw = j0 + warp * kClustersPerWarp;
-  const int nclw = max(0, min(kClustersPerWarp, Ks - jw));
-  if (nclw == 0) return;
-  const int32_t* cnt = counts_ws + (size_t)bh * d.C + cbase;
-  // rows before cluster jw within the segment
-  int before = 0;
-  for (int j = lane; j < jw; j += 32) before += cnt[j];
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) before += __shfl_xor_sync(0xffffffffu, before, off);
-  int rowstart[kClustersPerWarp];
   {
-    int r = before;
+    int cnt = 0;
+    for (int t = threadIdx.x; t < L; t += blockDim.x) cnt += lab[t] < j0;
 #pragma unroll
-    for (int c = 0; c < kClustersPerWarp; ++c) {
-      rowstart[c] = r;
-      if (c < nclw) r += cnt[jw + c];
-    }
+    for (int off = 16; off >= 1; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&before_sm, cnt);
   }
-  int rank[kClustersPerWarp] = {0, 0, 0, 0};
-  float vs[kClustersPerWarp][4];
-  float obj = 0.f;
-  float mrow[kClustersPerWarp][4];
-#pragma unroll
-  for (int c = 0; c < kClustersPerWarp; ++c) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) vs[c][i] = 0.f;
-    if (c < nclw) {
-      const float4 m = *reinterpret_cast<const float4*>(
-          mu + ((size_t)bh * d.C + cbase + jw + c) * kHeadDim + lane * 4);
-      mrow[c][0] = m.x; mrow[c][1] = m.y; mrow[c][2] = m.z; mrow[c][3] = m.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mrow[c][i] = 0.f;
-    }
-  }
+  gather_members(lab, L, j0, ncl, list, sorted, start, wtot);
+  const int before = before_sm;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bhN = (size_t)bh * d.N + d.m0 + seg_start;
   const size_t bhM = (size_t)bh * d.M + seg_start;
-  MemberQueue& q = queues[warp];
-  scan_members(lab, L, jw, nclw, q, [&](int cntq) {
-    for (int i = 0; i < cntq; i += 8) {
+  float obj = 0.f;
+  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
+    const int c = warp * kClustersPerWarp + cc;
+    if (c >= ncl) break;
+    const int b = start[c], e = start[c + 1];
+    const size_t crow = (size_t)bh * d.C + cbase + j0 + c;
+    const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
+    float vs[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = b; i < e; i += 8) {
       uint2 kr[8], vr[8];
-      int e[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        e[u] = i + u < cntq ? q.buf[i + u] : -1;
-        const size_t src = (bhN + (e[u] < 0 ? 0 : (e[u] >> 2))) * kHeadDim + lane * 4;
-        kr[u] = e[u] < 0 ? make_uint2(0, 0) : *reinterpret_cast<const uint2*>(K + src);
-        vr[u] = e[u] < 0 ? make_uint2(0, 0) : *reinterpret_cast<const uint2*>(V + src);
+        const bool in = i + u < e;
+        const size_t src = (bhN + (in ? sorted[i + u] : 0)) * kHeadDim + lane * 4;
+        kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
+        vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        if (e[u] < 0) continue;
-        const int t = e[u] >> 2, c = e[u] & 3;
-        int r = 0;
-#pragma unroll
-        for (int cc = 0; cc < kClustersPerWarp; ++cc)
-          if (cc == c) r = rowstart[cc] + rank[cc]++;
-        const size_t dst = (bhM + r) * kHeadDim + lane * 4;
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
-        if (lane == 0) out.perm[bhM + r] = d.m0 + seg_start + t;
-        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
-        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
-        const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
-        const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
-#pragma unroll
-        for (int cc = 0; cc < kClustersPerWarp; ++cc) {
-          if (cc == c) {
-            vs[cc][0] += va.x; vs[cc][1] += va.y; vs[cc][2] += vb.x; vs[cc][3] += vb.y;
-            const float d0 = ka.x - mrow[cc][0], d1 = ka.y - mrow[cc][1];
-            const float d2 = kb.x - mrow[cc][2], d3 = kb.y - mrow[cc][3];
-            obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
-          }
+        if (i + u < e) {
+          const int r = before + i + u;  // rows are in (cluster, position) order
+          const size_t dst = (bhM + r) * kHeadDim + lane * 4;
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
+          if (lane == 0) out.perm[bhM + r] = d.m0 + seg_start + sorted[i + u];
+          const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
+          const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+          const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
+          const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
+          vs[0] += va.x;
+          vs[1] += va.y;
+          vs[2] += vb.x;
+          vs[3] += vb.y;
+          const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
+          obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
         }
       }
     }
-  });
-#pragma unroll
-  for (int c = 0; c < kClustersPerWarp; ++c) {
-    if (c >= nclw) break;
-    const size_t row = (size_t)bh * d.C + cbase + jw + c;
-    *reinterpret_cast<float4*>(out.vsum + row * kHeadDim + lane * 4) =
-        make_float4(vs[c][0], vs[c][1], vs[c][2], vs[c][3]);
-    __nv_bfloat162 lo = __floats2bfloat162_rn(mrow[c][0], mrow[c][1]);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(mrow[c][2], mrow[c][3]);
+    *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
+        make_float4(vs[0], vs[1], vs[2], vs[3]);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
     uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + row * kHeadDim +
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + crow * kHeadDim +
                               lane * 4) = packed;
     if (lane == 0) {
-      out.counts[row] = cnt[jw + c];
-      out.offsets[(size_t)bh * (d.C + 1) + cbase + jw + c] = seg_start + rowstart[c];
+      out.counts[crow] = e - b;
+      out.offsets[(size_t)bh * (d.C + 1) + cbase + j0 + c] = seg_start + before + b;
     }
   }
   if (out.objective) {
@@ -763,14 +821,16 @@ bool make_map_bf16(CUtensorMap* map, const void* base, unsigned long long rows, 
     }                                                          \
   } while (0)
 
+size_t build_queue_bytes(long long rows) { return (size_t)rows * sizeof(FixEntry); }
+
 ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs& a,
                        cudaStream_t st) {
   char* ws = a.ws;
   int* status = reinterpret_cast<int*>(ws);
+  int* queue_count = reinterpret_cast<int*>(ws + 64);
   const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.K);
   const __nv_bfloat16* V = static_cast<const __nv_bfloat16*>(a.V);
   const long long BH = g.BH();
-  // steady buffers
   if (g.n_steady > 0)
     steady_kernel<<<(unsigned)BH, 256, 0, st>>>(K, V, static_cast<__nv_bfloat16*>(a.out.Ks),
                                                 static_cast<__nv_bfloat16*>(a.out.Vs), g.N, g.s0,
@@ -787,11 +847,12 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   d.total_tiles = BH * g.tiles_bh;
   float* mu = reinterpret_cast<float*>(ws + L.off_mu);
   __nv_bfloat16* mu_bf16 = reinterpret_cast<__nv_bfloat16*>(ws + L.off_mu_bf16);
-  float* norm2 = reinterpret_cast<float*>(ws + L.off_norm2);
-  float* mumax = reinterpret_cast<float*>(ws + L.off_mumax);
+  float* colt = reinterpret_cast<float*>(ws + L.off_colt);
+  float* ust = reinterpret_cast<float*>(ws + L.off_ust);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
   int32_t* labels = reinterpret_cast<int32_t*>(ws + L.off_labels);
   float* knorm = reinterpret_cast<float*>(ws + L.off_knorm);
+  FixEntry* queue = reinterpret_cast<FixEntry*>(ws + L.off_queue);
   const long long units = BH * g.S;
 
   CUtensorMap tm_keys, tm_cent;
@@ -803,35 +864,37 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   const long long rows = BH * g.M;
   knorm_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(K, knorm, g.N, g.M, g.m0, rows);
   RI_CUDA_TRY(cudaGetLastError());
-  RI_CUDA_TRY(cudaMemsetAsync(mumax, 0, units * sizeof(float), st));
+  RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
   const long long init_total = units * kMaxClustersPerSeg;
   init_kernel<<<(unsigned)((init_total + 7) / 8), 256, 0, st>>>(K, a.init_pos, d, mu, mu_bf16,
-                                                                 norm2, mumax, status, init_total);
+                                                                 colt, ust, status, init_total);
   RI_CUDA_TRY(cudaGetLastError());
 
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
-  const size_t upd_smem = align_up(g.seg_len * 2, 16) + kUpdateWarps * sizeof(MemberQueue);
-  const int upd_smem_max = (int)(32768 * 2 + kUpdateWarps * sizeof(MemberQueue));
+  const size_t upd_smem = (size_t)g.seg_len * 2 * sizeof(int);
+  const int upd_smem_max = (int)(kMaxSegLen * 2 * sizeof(int));
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(update_kernel), upd_smem_max));
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(finalise_kernel), upd_smem_max));
-  const unsigned grid_assign =
-      (unsigned)(d.total_tiles < (long long)num_sms() ? d.total_tiles : num_sms());
+  const int sms = num_sms();
+  const unsigned grid_assign = (unsigned)(d.total_tiles < (long long)sms ? d.total_tiles : sms);
   const dim3 grid_upd((unsigned)units, (unsigned)((g.K_full + kClustersPerBlock - 1) /
                                                   kClustersPerBlock));
   const int rounds = g.iters > 0 ? g.iters : 1;
   for (int t = 0; t < rounds; ++t) {
+    RI_CUDA_TRY(cudaMemsetAsync(queue_count, 0, sizeof(int), st));
     assign_kernel<<<grid_assign, kAssignThreads, kAssignSmem, st>>>(
-        tm_keys, tm_cent, d, knorm, norm2, mumax, mu, labels, status);
+        tm_keys, tm_cent, d, knorm, colt, ust, labels, queue, queue_count, status);
     RI_CUDA_TRY(cudaGetLastError());
-    RI_CUDA_TRY(cudaMemsetAsync(mumax, 0, units * sizeof(float), st));
+    fixup_kernel<<<(unsigned)(4 * sms), 256, 0, st>>>(K, mu, d, queue, queue_count, labels);
+    RI_CUDA_TRY(cudaGetLastError());
+    RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
     update_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(
-        K, labels, d, mu, mu_bf16, norm2, mumax, counts, g.iters > 0 ? 1 : 0);
+        K, labels, d, mu, mu_bf16, colt, ust, counts, g.iters > 0 ? 1 : 0);
     RI_CUDA_TRY(cudaGetLastError());
   }
   if (a.out.objective)
     RI_CUDA_TRY(cudaMemsetAsync(a.out.objective, 0, units * sizeof(float), st));
-  finalise_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(K, V, labels, d, mu,
-                                                                  counts, a.out);
+  finalise_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(K, V, labels, d, mu, a.out);
   RI_CUDA_TRY(cudaGetLastError());
   return RI_OK;
 }

@@ -168,6 +168,33 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
                               int32_t* sel_ids, void* workspace, size_t workspace_bytes,
                               ri_stream_t stream);
 
+/* ri_decode_attention without a caller workspace.  The pages describe no
+ * such call; it exists for callers that must not allocate (or own) scratch:
+ * the scratch is a fixed device array of RI_STATIC_SCRATCH_BYTES inside this
+ * library, one per device.  Same arguments, results and checks as
+ * ri_decode_attention, minus workspace/workspace_bytes, plus:
+ *  - device_status: optional device int32.  When non-NULL the call's device
+ *    status word (RI_OK, or the first device-side failure) is copied there,
+ *    ordered on `stream` after the kernel.
+ * Limits and rules:
+ *  - Returns RI_ERR_CAPACITY when ri_decode_workspace() for (cfg, dcfg)
+ *    exceeds RI_STATIC_SCRATCH_BYTES (4 MiB: e.g. one 128K-token sequence
+ *    with 8 KV heads fits; batch 16 of 128K does not).
+ *  - The first call on a device looks up the array's address (and loads the
+ *    module if it is loaded lazily); make one call, or any call that can
+ *    fail fast, before capturing a stream into a CUDA graph.
+ *  - Every call on a device shares the one array: calls whose executions
+ *    overlap (on different streams or from different threads) race and
+ *    give wrong results.  Order them on one stream.
+ *  - Nothing needs to start at zero: each call clears the status word and
+ *    counters it uses (stream-ordered) before its kernel runs.
+ * Allocates nothing: no cudaMalloc, no host allocation. */
+#define RI_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+ri_status ri_decode_attention_static(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                     const void* q, const ri_index* idx, void* out, float* lse,
+                                     int32_t* sel_ids, int32_t* device_status,
+                                     ri_stream_t stream);
+
 /* Steps S1-S2 alone (centroid scoring and cluster selection).  Writes
  * sel_ids (required here) and keeps scores and the selection in the
  * workspace for a following ri_attend_selected on the same workspace and

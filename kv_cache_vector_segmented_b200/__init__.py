@@ -14,7 +14,8 @@ _EXPORTS = (
     "LIB_PATH", "CIndex", "DecodeConfig", "Geometry", "Index", "IndexConfig", "RIError",
     "STATUS_CODES", "STATUS_NAMES", "alloc_workspace", "attend_selected", "build_index",
     "build_workspace_bytes", "decode", "decode_workspace_bytes", "default_budgets", "geometry",
-    "lib", "read_device_status", "select_clusters", "selftest_wait_timeout")
+    "lib", "read_device_status", "select_clusters", "selftest_wait_timeout", "decode_static",
+    "STATIC_SCRATCH_BYTES")
 
 __all__ = list(_EXPORTS)
 

@@ -92,6 +92,9 @@ lib.ri_decode_workspace.argtypes = [_P(IndexConfig), _P(DecodeConfig)]
 lib.ri_decode_attention.restype = ctypes.c_int
 lib.ri_decode_attention.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
                                     _vp, _vp, _vp, _sz, _vp]
+lib.ri_decode_attention_static.restype = ctypes.c_int
+lib.ri_decode_attention_static.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex),
+                                           _vp, _vp, _vp, _vp, _vp]
 lib.ri_select_clusters.restype = ctypes.c_int
 lib.ri_select_clusters.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
                                    _vp, _vp, _sz, _vp]
@@ -279,6 +282,39 @@ def decode(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = None,
                                   ctypes.byref(cidx), out.data_ptr(), _ptr(lse), _ptr(sel),
                                   ws.data_ptr(), ws.numel(), _stream(dev)),
           "ri_decode_attention")
+    return out, lse, sel
+
+
+STATIC_SCRATCH_BYTES = 4 << 20  # RI_STATIC_SCRATCH_BYTES
+
+
+def decode_static(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = None,
+                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  want_lse: bool = True, want_sel: bool = False,
+                  device_status: Optional[torch.Tensor] = None):
+    """ri_decode_attention_static: one decode step whose scratch is the
+    library's fixed device array (no workspace argument).  Returns
+    (out, lse or None, sel or None)."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, H * G, d), dev)
+    if dcfg is None:
+        dcfg = default_budgets(index.geom.clusters)
+    if out is None:
+        out = torch.empty((B, H * G, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, H * G, d), dev)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H * G), dtype=torch.float32, device=dev)
+    sel = (torch.empty((B, H, dcfg.k_retrieval + dcfg.k_estimation), dtype=torch.int32,
+                       device=dev) if want_sel else None)
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32, (1,), dev)
+    cidx = index.c_struct()
+    check(lib.ri_decode_attention_static(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                         ctypes.byref(cidx), out.data_ptr(), _ptr(lse),
+                                         _ptr(sel), _ptr(device_status), _stream(dev)),
+          "ri_decode_attention_static")
     return out, lse, sel
 
 

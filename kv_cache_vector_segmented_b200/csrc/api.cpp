@@ -52,6 +52,7 @@ cudaError_t set_smem_once(const void* func, int bytes) {
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool make_geometry(const ri_index_config* cfg, Geometry* g) {
   if (!cfg) {
@@ -365,6 +366,39 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
   DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, workspace);
   e = launch_decode(g, L, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return RI_OK;
+}
+
+ri_status ri_decode_attention_static(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                     const void* q, const ri_index* idx, void* out, float* lse,
+                                     int32_t* sel_ids, int32_t* device_status,
+                                     ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  if (!make_decode_layout(g, dcfg, &L)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(L.total <= kStaticScratchBytes, RI_ERR_CAPACITY,
+           "decode needs %zu bytes of scratch, the static array holds %zu", L.total,
+           kStaticScratchBytes);
+  RI_CHECK(!device_status || aligned4(device_status), RI_ERR_INVALID_ARG,
+           "device_status must be 4-byte aligned");
+  void* ws = nullptr;
+  cudaError_t e = static_decode_scratch(&ws);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+  ri_status st = prepare_decode(cfg, dcfg, q, idx, ws, kStaticScratchBytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  RI_CHECK(!sel_ids || aligned16(sel_ids), RI_ERR_INVALID_ARG, "sel_ids must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = cudaMemsetAsync(ws, 0, L.header_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, ws);
+  e = launch_decode(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if (device_status) {
+    e = cudaMemcpyAsync(device_status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying the device status");
+  }
   return RI_OK;
 }
 

@@ -78,6 +78,11 @@ bool decode_plan(const Geometry& g, DecodeLayout* L);
 cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
 
+// Fixed scratch of ri_decode_attention_static (static_scratch.cu): the
+// current device's copy, looked up once per device.
+constexpr size_t kStaticScratchBytes = RI_STATIC_SCRATCH_BYTES;
+cudaError_t static_decode_scratch(void** addr);
+
 // --------------------------------------------------------------- build
 constexpr int kMaxSegLen = 16384;  // segment tokens (member lists live in shared memory)
 

@@ -147,7 +147,8 @@ bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeL
   L->ke = L->k_e < g.C - L->kr ? L->k_e : g.C - L->kr;
   const long long BH = g.BH();
   if (!decode_plan(g, L)) return false;
-  L->header_bytes = kStatusBytesHost;
+  L->off_ctrl = kStatusBytesHost;
+  L->header_bytes = align_up(L->off_ctrl + (size_t)6 * BH * 4, 256);
   size_t off = L->header_bytes;
   L->off_rkey = off;
   off = align_up(off + (size_t)BH * g.C * 4, 256);
@@ -157,6 +158,10 @@ bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeL
   off = align_up(off + (size_t)BH * (L->k_r + L->k_e) * 4, 256);
   L->off_rpre = off;
   off = align_up(off + (size_t)BH * (L->k_r + 1) * 4, 256);
+  L->off_rrow = off;
+  off = align_up(off + (size_t)BH * (L->k_r > 0 ? L->k_r : 1) * 4, 256);
+  L->off_part = off;
+  off = align_up(off + (size_t)BH * L->S * g.G * kPartStride * 4, 256);
   L->total = off;
   return true;
 }

@@ -1,5 +1,5 @@
-// Tripartite decode attention over the wave index (sm_100a): one kernel
-// launch per decode step, one thread-block cluster per (sequence, KV head).
+// Tripartite decode attention over the wave index (sm_100a): one persistent,
+// cooperative kernel launch per decode step, one block per SM.
 //
 // Steps (RetroInfer; "KV缓存技术与RetroInfer系统在长上下文推理中的优化实践",
 // framerc.cn, §2.1 zones, §2.2 step 1 index query, §3.3 attention over the
@@ -10,76 +10,90 @@
 //   S5 estimation term    each c in E adds n_c e^{s} / e^{s} Vsum_c
 //   S6 merge              log-sum-exp over the split partials
 //
-// The P blocks of a unit form one cluster (P <= 16).  Block j
-//   A) scores 128-centroid tiles [T j / P, T (j+1) / P) on the tensor cores:
-//      TMA brings a tile (128-byte swizzle), one thread issues tcgen05.mma
-//      with the unit's G query rows (padded to N = 16) as the B operand, four
-//      warps read the fp32 scores from TMEM; the block keeps its keys r_c;
-//   B) selects R and E together with the other blocks of the cluster through
-//      distributed shared memory: the key range, a 2048-bucket value
-//      histogram and the boundary buckets' members are gathered in block 0,
-//      every block ranks the few boundary keys exactly, then scatters its R
-//      and E members to their positions (R ids to block 0, each E id to the
-//      block that attends it).  If a boundary bucket is crowded (heavy ties),
-//      every block instead runs the exact selection over all C keys;
-//   C) attends its share of the steady + retrieval tokens and of the
-//      estimation clusters (16-byte cp.async copies into shared memory, three
-//      buffers in flight; 16-lane groups with shuffle reductions);
-//   D) leaves its partial (m, l, o) in shared memory; block 0 merges the P
-//      partials through distributed shared memory.
-// Cluster barriers are hardware barriers; every block executes the same
-// sequence of them (no block leaves early), and the mbarrier waits of step A
-// are bounded.
-#include <cooperative_groups.h>
-#include <map>
-#include <mutex>
-#include <tuple>
+// A unit is one (sequence, KV head).  Work flows between blocks through
+// per-unit counters in the workspace; no block ever waits for a block that
+// could be waiting for it, and the cooperative launch keeps every block
+// resident, so the waits below always end (they are bounded in any case).
+//   A) Every block scores 128-centroid tiles t = blockIdx + k gridDim of the
+//      flattened (unit, tile) list on the tensor cores: TMA brings the tile
+//      and the unit's query rows (128-byte swizzle), one thread issues
+//      tcgen05.mma (M = 128 centroids, N = 16 query rows, K = 128), four
+//      warps read the fp32 scores from TMEM, store s and r and fold r into
+//      the unit's key range; a fifth warp counts finished tiles per unit.
+//   B) Block NB - 1 - u ranks unit u's C keys exactly once its tiles are all
+//      scored (value histogram over the key range, exact order inside the
+//      two boundary buckets), writes R and E in id order and the R clusters'
+//      token prefix and first rows, then raises the unit's ready flag.
+//   C) Every block takes (unit, slice) pairs: the unit's steady tokens, R
+//      tokens and E clusters form one item list cut into S equal slices, and
+//      each warp of the block a contiguous run of the slice.  A warp streams
+//      its items through a private ring of shared-memory slots with 16-byte
+//      cp.async copies (the ring's depth in flight) and folds each into one
+//      online-softmax state: a token adds e^{x} v after its logit x, an E
+//      cluster adds n_c e^{s} and e^{s} Vsum_c.  The block combines its warps
+//      into the slice's partial (m, l, o) in the workspace.
+//   D) The block that finishes a unit's last slice (atomic ticket) merges the
+//      S partials by log-sum-exp and writes out and lse.
 #include <float.h>
 #include <math.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "common.cuh"
 #include "internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace ri {
 
 namespace {
 
 constexpr float kScale = 0.08838834764831845f;  // 1/sqrt(128)
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kTileC = 128;          // centroids per MMA tile (M)
-constexpr int kQRows = 16;           // MMA N: query rows padded to 16
-constexpr int kStagesA = 2;
+constexpr int kQRows = 16;           // MMA N: query rows (the unit's G, then others)
+constexpr int kStagesA = 4;
+constexpr uint32_t kTileBytes = kTileC * kHeadDim * 2;  // 32 KB
+constexpr uint32_t kQBytes = kQRows * kHeadDim * 2;     // 4 KB
+constexpr uint32_t kStageBytes = kTileBytes + kQBytes;  // 1024-byte multiple
 constexpr int kNB = 2048;            // value buckets of the selection
 constexpr int kBoundaryCap = 256;    // keys ranked exactly in a boundary bucket
-constexpr int kPer = 32;             // fallback: keys per thread and round
-constexpr int kRound = kThreads * kPer;
-constexpr int kTokChunk = 64;        // tokens per copy chunk (K and V rows: 32 KB)
-constexpr int kEChunk = 56;          // estimation clusters per chunk (value sum + scores)
-constexpr uint32_t kChunkBytes = 32768;
-constexpr int kChunkBufs = 2;        // copy buffers of the attention step
-static_assert(kTokChunk * 512 <= (int)kChunkBytes && kEChunk * 544 <= (int)kChunkBytes, "chunk");
-constexpr int kMaxClusterBlocks = 16;  // blocks per unit (cluster size)
-constexpr uint32_t kTileBytes = kTileC * kHeadDim * 2;  // 32 KB
-constexpr uint32_t kStageBytes = 65536;  // A: 2 TMA stages; C: 2 copy buffers; D: partials
-static_assert(kStagesA * kTileBytes <= kStageBytes && kChunkBufs * kChunkBytes <= kStageBytes, "stage");
-constexpr uint32_t kPartOff = 40960;  // own partial [G][132] inside the stage region
-constexpr uint32_t kMiscBytes = 512;
+constexpr int kRound = 8192;         // keys per selection round (all threads)
+constexpr int kMaxWarps = 32;
+constexpr int kRoundItems = 134;      // work items (token or E cluster) per copy round
+constexpr uint32_t kBufBytes = 81920;  // one round: tokens (padded to 16) x 512 B + E x 548 B
+constexpr uint32_t kRegionBytes = 2 * kBufBytes;
+constexpr float kRescale = 8.f;      // online softmax: new reference only when the max
+                                     // grows by more than this (terms stay <= e^8)
+static_assert(kStagesA * kStageBytes <= kRegionBytes, "stages");
+static_assert(16 * 512 + (kRoundItems - 1) * 548 <= (int)kBufBytes &&
+                  (kRoundItems + 15) * 512 <= (int)kBufBytes, "round");
+static_assert(kNB * 4 + 2 * kBoundaryCap * 8 <= (int)kRegionBytes, "select");
 
-// Shared memory map of one launch (byte offsets from a 1024-byte aligned base),
-// sized from the configuration so that small problems fit two blocks per SM.
-struct SmemLayout {
-  uint32_t q, lkeys, hist, gslice, cand, rpre, rbase, rtrip, ecnt, eslice, misc, total;
-  int lkeys_cap;   // keys (floats) the lkeys region holds
-  int eslice_cap;  // estimation clusters one block handles
+// Threads per block (registers: up to 128 each).
+template <int G>
+struct Shape {
+  static constexpr int kThreads = 512;
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kPer = kRound / kThreads;  // keys per thread and round
 };
+
+// Shared memory map (byte offsets from a 1024-byte aligned base).
+constexpr uint32_t kOffRpre = kRegionBytes;                        // int [kMaxRetrieval + 4]
+constexpr uint32_t kOffRrow = kOffRpre + (kMaxRetrieval + 4) * 4;  // int [kMaxRetrieval]
+constexpr uint32_t kOffMisc = kOffRrow + kMaxRetrieval * 4;
+constexpr uint32_t kMiscBytes = 3072;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + base alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(kOffMisc % 16 == 0, "misc alignment");
+
+// Selection scratch inside the region (free outside steps A and C).
+constexpr uint32_t kOffHist = 0;
+constexpr uint32_t kOffCand = kOffHist + kNB * 4;
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
 
-struct FusedParams {
+struct Params {
   const __nv_bfloat16* q;
   const int32_t* counts;
   const int32_t* offsets;
@@ -96,24 +110,31 @@ struct FusedParams {
   float* rkey;     // ws [BH][C]
   int32_t* sel;    // ws [BH][k_r + k_e]
   int32_t* rpre;   // ws [BH][k_r + 1]
-  int* status;
-  int G, C, M, n_steady, k_r, k_e, kr, ke, P, exec_rows, mode;
-  SmemLayout L;
+  int32_t* rrow;   // ws [BH][k_r]
+  float* part;     // ws [BH][S][G][kPartStride]
+  int* status;     // ws status word
+  int* done;       // ws [BH] scored tiles
+  int* ready;      // ws [BH] selection published
+  int* ticket;     // ws [BH] finished slices
+  uint32_t* kmax;  // ws [BH] max order key of the finite selection keys
+  uint32_t* kmin;  // ws [BH] max of the complemented order keys (= min key)
+  int* ninf;       // ws [BH] empty clusters (key -inf)
+  int BH, C, M, n_steady, k_r, k_e, kr, ke, S, exec_rows, mode;
 };
 
 struct Misc {
   uint64_t full[kStagesA], empty[kStagesA], tfull[2], tempty[2], drain;
   uint32_t tmem;
   int abort_flag;
+  int epi_done;  // epilogue's finished tiles (step A)
+  int flag;
   int bucket[2], above[2], ncand[2];
   uint32_t Tu[2];
   int Tid[2];
-  int wtot[2][kWarps];
-  float red[2][kWarps];
-  int scan[kWarps + 4];
-  float rlo, rhi;      // this block's key range (finite keys)
-  int rninf;           // this block's -inf keys
-  int cntR, cntE;      // this block's R / E members
+  int wtot[2][kMaxWarps];
+  int scan[kMaxWarps + 4];
+  float wm[kMaxWarps][8];  // per-warp partial maxima (block combine)
+  float wl[kMaxWarps][8];  // per-warp partial denominators
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area");
 
@@ -131,6 +152,30 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_volatile(const int* p) {
+  return *reinterpret_cast<const volatile int*>(p);
+}
+
+__device__ __forceinline__ float float_from_order_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // 64-bit selection order: larger key first, lower id first among equal keys.
 __device__ __forceinline__ unsigned long long ord64(uint32_t u, int id) {
   return ((unsigned long long)u << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)id);
@@ -143,41 +188,52 @@ __device__ __forceinline__ int bucket_of(float r, float lo, float scale) {
   return b < 0 ? 0 : (b >= kNB ? kNB - 1 : b);
 }
 
-// Block-wide inclusive prefix of one int per thread (thread order); returns
-// the exclusive prefix and writes the block total to *total.
-__device__ __forceinline__ int block_excl_scan(int v, int* scratch /* [kWarps] */, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += t;
-  }
-  if (lane == 31) scratch[warp] = incl;
-  __syncthreads();
-  int excl = incl - v, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    if (w < warp) excl += scratch[w];
-    tot += scratch[w];
-  }
-  __syncthreads();
-  *total = tot;
-  return excl;
+// ---- warp-level tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 acc)
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// d += A . B with A 16x16 row-major (regs a0..a3), B 16x8 column-major (b0, b1)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// 2^x by the hardware approximation (ex2.approx; -inf gives +0)
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ void kth_in_bucket_slow(const float* keys, bool cached, int C, int b, float lo,
-                                   float scale, int k, Misc* ms, int* hist, uint32_t* Tu,
-                                   int* Tid) {
-  auto key = [&](int c) { return cached ? keys[c] : __ldcg(keys + c); };
+// The k-th (1-based, from the top) key of value bucket b with its id, by an
+// MSD radix walk over the bucket's keys (for crowded buckets: heavy ties).
+template <int NT>
+__device__ void kth_in_bucket_slow(const float* keys, int C, int b, float lo, float scale, int k,
+                                   Misc* ms, int* hist, uint32_t* Tu, int* Tid) {
+  constexpr int NW = NT / 32;
   uint32_t prefix = 0, mask = 0;
   int remaining = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += kThreads) {
-      const float r = key(c);
+    for (int c = threadIdx.x; c < C; c += NT) {
+      const float r = __ldcg(keys + c);
       if (bucket_of(r, lo, scale) != b) continue;
       const uint32_t u = float_order_key(r);
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
@@ -203,16 +259,16 @@ __device__ void kth_in_bucket_slow(const float* keys, bool cached, int C, int b,
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int run = 0;
-  for (int base = 0; base < C; base += kThreads) {
+  for (int base = 0; base < C; base += NT) {
     const int c = base + threadIdx.x;
-    const float r = c < C ? key(c) : 0.f;
+    const float r = c < C ? __ldcg(keys + c) : 0.f;
     const bool eq = c < C && bucket_of(r, lo, scale) == b && float_order_key(r) == prefix;
     const unsigned mk = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) ms->wtot[0][warp] = __popc(mk);
     __syncthreads();
     int before = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       before += w < warp ? ms->wtot[0][w] : 0;
       tot += ms->wtot[0][w];
     }
@@ -226,196 +282,273 @@ __device__ void kth_in_bucket_slow(const float* keys, bool cached, int C, int b,
   __syncthreads();
 }
 
+// Block-wide exclusive prefix of one int per thread (thread order); the
+// block total goes to *total.  One warp scans the per-warp totals.
+template <int NT>
+__device__ __forceinline__ int block_scan(int v, int* scratch /* [NT / 32 + 1] */, int* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int wt = lane < NW ? scratch[lane] : 0;
+    int wi = wt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += t;
+    }
+    if (lane < NW) scratch[lane] = wi - wt;
+    if (lane == 31) scratch[NW] = wi;
+  }
+  __syncthreads();
+  const int excl = scratch[warp] + incl - v;
+  *total = scratch[NW];
+  __syncthreads();  // scratch is reused by the next scan
+  return excl;
+}
+
+// OR of a predicate over the 128 threads of warps 4-7 (named barrier 1).
+__device__ __forceinline__ bool epilogue_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// Bounded wait of one thread until a counter other blocks raise reaches
+// `target`; gives up early when any block has recorded a failure.
+__device__ bool wait_count(const int* counter, int target, const int* status) {
+  if (ld_acquire(counter) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (ld_acquire(counter) >= target) return true;
+    if (ld_volatile(status) != 0) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(32);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int G>
-__global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
-    fused_decode_kernel(const __grid_constant__ CUtensorMap tm_cent, const FusedParams p) {
+__global__ void __launch_bounds__(Shape<G>::kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_cent,
+                  const __grid_constant__ CUtensorMap tm_q, const Params p) {
+  constexpr int NT = Shape<G>::kThreads;
+  constexpr int NW = Shape<G>::kWarps;
+  constexpr int kPer = Shape<G>::kPer;
+
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  cg::cluster_group cluster = cg::this_cluster();
-  Misc* ms = reinterpret_cast<Misc*>(sm + p.L.misc);
-  float* keys = reinterpret_cast<float*>(sm + p.L.lkeys);   // fallback key cache
-  float* lkeys = keys;                                        // own chunk's keys (fast path)
-  int* hist = reinterpret_cast<int*>(sm + p.L.hist);
-  int* gslice = reinterpret_cast<int*>(sm + p.L.gslice);
-  unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + p.L.cand);
-  int32_t* rpre_sm = reinterpret_cast<int32_t*>(sm + p.L.rpre);
-  int32_t* rbase_sm = reinterpret_cast<int32_t*>(sm + p.L.rbase);
-  int32_t* rtrip = reinterpret_cast<int32_t*>(sm + p.L.rtrip);  // [3][kr]: id, size, row
-  int32_t* eslice = reinterpret_cast<int32_t*>(sm + p.L.eslice);
+  Misc* ms = reinterpret_cast<Misc*>(sm + kOffMisc);
+  int32_t* rpre_sm = reinterpret_cast<int32_t*>(sm + kOffRpre);
+  int32_t* rrow_sm = reinterpret_cast<int32_t*>(sm + kOffRrow);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / p.P;
-  const int j = blockIdx.x - bh * p.P;  // rank in the cluster
   const int C = p.C;
-  const int tiles = C > 0 ? (C + kTileC - 1) / kTileC : 0;
-  const int t_begin = (int)((long long)tiles * j / p.P);
-  const int t_end = (int)((long long)tiles * (j + 1) / p.P);
-  const int c_begin = t_begin * kTileC;
-  const int c_end = min(t_end * kTileC, C);
-  const int n_loc = max(0, c_end - c_begin);
   const int kr = p.kr, ke = p.ke;
-  auto e_first = [&](int r) { return (int)((long long)ke * r / p.P); };
-  const int e0 = e_first(j), e1 = e_first(j + 1);
+  const int tiles_h = C > 0 ? (C + kTileC - 1) / kTileC : 0;
 
-  if (threadIdx.x == 0) ms->abort_flag = 0;
+  if (threadIdx.x == 0) {
+    ms->abort_flag = 0;
+    ms->epi_done = 0;
+    for (int i = 0; i < kStagesA; ++i) {
+      mbar_init(&ms->full[i], 1);
+      mbar_init(&ms->empty[i], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&ms->tfull[h], 1);
+      mbar_init(&ms->tempty[h], 128);
+    }
+    mbar_init(&ms->drain, 1);
+    fence_barrier_init();
+  }
   __syncthreads();
 
-  // ============================================================ phase A
-  if (p.mode != kModeAttend && C > 0) {
-    const int nt = t_end - t_begin;
-    uint8_t* qsm = sm + p.L.q;
-    if (threadIdx.x == 0) {
-      for (int i = 0; i < kStagesA; ++i) {
-        mbar_init(&ms->full[i], 1);
-        mbar_init(&ms->empty[i], 1);
+  // ============================================================ step A
+  if (p.mode != kModeAttend && tiles_h > 0) {
+    const int total_tiles = p.BH * tiles_h;
+    const int nt = total_tiles > (int)blockIdx.x
+                       ? (total_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
+                       : 0;
+    if (nt > 0) {
+      if (warp == 1) {
+        tmem_alloc(&ms->tmem, 32);
+        tmem_relinquish();
       }
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(&ms->tfull[h], 1);
-        mbar_init(&ms->tempty[h], 128);
-      }
-      mbar_init(&ms->drain, 1);
-      fence_barrier_init();
-    }
-    // B operand: the unit's G query rows, zero rows up to 16, in the 128-byte
-    // swizzle layout (row n, 16-byte chunk c stored at chunk c ^ (n & 7)).
-    for (int i = threadIdx.x; i < 2 * kQRows * 8; i += kThreads) {
-      const int kh = i / (kQRows * 8), n = (i / 8) % kQRows, c = i % 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n < G) v = ldg_nc_v4(p.q + ((size_t)bh * G + n) * kHeadDim + kh * 64 + c * 8);
-      *reinterpret_cast<uint4*>(qsm + kh * (kQRows * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();
-    if (warp == 1) {
-      tmem_alloc(&ms->tmem, 32);
-      tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = ms->tmem;
-    if (warp == 0 && lane == 0) {
-      // TMA producer
-      tma_prefetch_desc(&tm_cent);
-      int issued[kStagesA] = {0, 0};
-      for (int it = 0; it < nt; ++it) {
-        if (ms->abort_flag) break;
-        const int st = it % kStagesA;
-        if (it >= kStagesA && !mbar_wait(&ms->empty[st], ((it / kStagesA) - 1) & 1)) {
-          record_status(p.status, RI_ERR_TIMEOUT);
-          ms->abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&ms->full[st], kTileBytes);
-        const int row = bh * C + (t_begin + it) * kTileC;
-        for (int kh = 0; kh < 2; ++kh)
-          tma_load_2d(sm + st * kTileBytes + kh * (kTileC * 128), &tm_cent, kh * 64,
-                      row, &ms->full[st]);
-        ++issued[st];
-      }
-      for (int st = 0; st < kStagesA; ++st)
-        if (issued[st]) mbar_wait(&ms->full[st], (uint32_t)((issued[st] - 1) & 1));
-    } else if (warp == 1 && lane == 0) {
-      // MMA issuer: D[128 x 16] = tile[128 x 128] . Q[16 x 128]^T
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileC, kQRows);
-      const uint32_t st_addr = smem_u32(sm);
-      const uint32_t q_addr = smem_u32(qsm);
-      for (int it = 0; it < nt; ++it) {
-        if (ms->abort_flag) break;
-        const int st = it % kStagesA, buf = it & 1;
-        if (!mbar_wait(&ms->full[st], (uint32_t)((it / kStagesA) & 1)) ||
-            (it >= 2 && !mbar_wait(&ms->tempty[buf], (uint32_t)(((it >> 1) - 1) & 1)))) {
-          record_status(p.status, RI_ERR_TIMEOUT);
-          ms->abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = st * kTileBytes + (kk >> 2) * (kTileC * 128) + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * (kQRows * 128) + (kk & 3) * 32;
-          umma_bf16(tmem + buf * kQRows, umma_desc_sw128(st_addr + aoff),
-                    umma_desc_sw128(q_addr + boff), idesc, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&ms->empty[st]);
-        umma_commit(&ms->tfull[buf]);
-      }
-      umma_commit(&ms->drain);
-      mbar_wait(&ms->drain, 0);
-    } else if (warp >= 4) {
-      // epilogue: one centroid per thread
-      const int quad = warp & 3;
-      const int r = quad * 32 + lane;
-      for (int it = 0; it < nt; ++it) {
-        if (ms->abort_flag) break;
-        const int buf = it & 1;
-        const int c = (t_begin + it) * kTileC + r;
-        // issued before the wait so the load overlaps the MMA
-        const int cnt = c < C ? __ldg(p.counts + (size_t)bh * C + c) : 0;
-        if (!mbar_wait(&ms->tfull[buf], (uint32_t)((it >> 1) & 1))) {
-          record_status(p.status, RI_ERR_TIMEOUT);
-          ms->abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + buf * kQRows, v);
-        tc_fence_before();
-        mbar_arrive(&ms->tempty[buf]);
-        if (c < C) {
-          float s[8];
-          float rs = 0.f;
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            s[g] = g < G ? v[g] * kScale : 0.f;
-            if (g < G) rs += s[g];
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      const uint32_t tmem = ms->tmem;
+      if (warp == 0 && lane == 0) {
+        // TMA producer: centroid tile and the unit's query rows per stage
+        tma_prefetch_desc(&tm_cent);
+        tma_prefetch_desc(&tm_q);
+        int issued[kStagesA] = {0, 0, 0, 0};
+        for (int it = 0; it < nt; ++it) {
+          if (ld_volatile(&ms->abort_flag)) break;
+          const int st = it % kStagesA;
+          if (it >= kStagesA && !mbar_wait(&ms->empty[st], ((it / kStagesA) - 1) & 1)) {
+            record_status(p.status, RI_ERR_TIMEOUT);
+            ms->abort_flag = 1;
+            break;
           }
-          float4* dst = reinterpret_cast<float4*>(p.score + ((size_t)bh * C + c) * 8);
-          dst[0] = make_float4(s[0], s[1], s[2], s[3]);
-          dst[1] = make_float4(s[4], s[5], s[6], s[7]);
-          const float key = cnt > 0 ? rs : -INFINITY;
-          p.rkey[(size_t)bh * C + c] = key;
-          lkeys[c - c_begin] = key;
+          const int t = (int)blockIdx.x + it * (int)gridDim.x;
+          const int u = t / tiles_h, ti = t - u * tiles_h;
+          uint8_t* stage = sm + st * kStageBytes;
+          mbar_arrive_expect_tx(&ms->full[st], kStageBytes);
+          const int row = u * C + ti * kTileC;
+          for (int kh = 0; kh < 2; ++kh) {
+            tma_load_2d(stage + kh * (kTileC * 128), &tm_cent, kh * 64, row, &ms->full[st]);
+            tma_load_2d(stage + kTileBytes + kh * (kQRows * 128), &tm_q, kh * 64, u * G,
+                        &ms->full[st]);
+          }
+          ++issued[st];
+        }
+        for (int st = 0; st < kStagesA; ++st)
+          if (issued[st]) mbar_wait(&ms->full[st], (uint32_t)((issued[st] - 1) & 1));
+      } else if (warp == 1 && lane == 0) {
+        // MMA issuer: D[128 x 16] = tile[128 x 128] . Q[16 x 128]^T
+        constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileC, kQRows);
+        const uint32_t base = smem_u32(sm);
+        for (int it = 0; it < nt; ++it) {
+          if (ld_volatile(&ms->abort_flag)) break;
+          const int st = it % kStagesA, buf = it & 1;
+          if (!mbar_wait(&ms->full[st], (uint32_t)((it / kStagesA) & 1)) ||
+              (it >= 2 && !mbar_wait(&ms->tempty[buf], (uint32_t)(((it >> 1) - 1) & 1)))) {
+            record_status(p.status, RI_ERR_TIMEOUT);
+            ms->abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = base + st * kStageBytes;
+          const uint32_t b_addr = a_addr + kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * (kTileC * 128) + (kk & 3) * 32;
+            const uint32_t boff = (kk >> 2) * (kQRows * 128) + (kk & 3) * 32;
+            umma_bf16(tmem + buf * kQRows, umma_desc_sw128(a_addr + aoff),
+                      umma_desc_sw128(b_addr + boff), idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&ms->empty[st]);
+          umma_commit(&ms->tfull[buf]);
+        }
+        umma_commit(&ms->drain);
+        mbar_wait(&ms->drain, 0);
+      } else if (warp == 2 && lane == 0) {
+        // publisher: counts the epilogue's finished tiles into the units'
+        // tile counters (one gpu-scope fence per batch of tiles)
+        int published = 0;
+        const unsigned long long t0 = globaltimer_ns();
+        while (published < nt) {
+          const int e = ld_acquire_cta(&ms->epi_done);
+          if (e > published) {
+            __threadfence();
+            for (int i = published; i < e; ++i) {
+              const int t = (int)blockIdx.x + i * (int)gridDim.x;
+              atomicAdd(p.done + t / tiles_h, 1);
+            }
+            published = e;
+          } else if (ld_volatile(&ms->abort_flag)) {
+            break;
+          } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_status(p.status, RI_ERR_TIMEOUT);
+            ms->abort_flag = 1;
+            break;
+          }
+        }
+      } else if (warp >= 4 && warp < 8) {
+        // epilogue: one centroid per thread; the unit's key range on the side
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        for (int it = 0; it < nt; ++it) {
+          const int buf = it & 1;
+          const int t = (int)blockIdx.x + it * (int)gridDim.x;
+          const int u = t / tiles_h, ti = t - u * tiles_h;
+          const int c = ti * kTileC + r;
+          // issued before the wait so the load overlaps the MMA
+          const int cnt = c < C ? __ldg(p.counts + (size_t)u * C + c) : 0;
+          const bool ok = mbar_wait(&ms->tfull[buf], (uint32_t)((it >> 1) & 1));
+          // the 128 epilogue threads leave together (they share named barrier 1)
+          if (epilogue_any(!ok)) {
+            if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
+            ms->abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + buf * kQRows, v);
+          tc_fence_before();
+          mbar_arrive(&ms->tempty[buf]);
+          uint32_t kmx = 0, kmn = 0;
+          bool empty = false;
+          if (c < C) {
+            float s[8];
+            float rs = 0.f;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              s[g] = g < G ? v[g] * kScale : 0.f;
+              if (g < G) rs += s[g];
+            }
+            float4* dst = reinterpret_cast<float4*>(p.score + ((size_t)u * C + c) * 8);
+            dst[0] = make_float4(s[0], s[1], s[2], s[3]);
+            dst[1] = make_float4(s[4], s[5], s[6], s[7]);
+            p.rkey[(size_t)u * C + c] = cnt > 0 ? rs : -INFINITY;
+            if (cnt > 0) {
+              kmx = float_order_key(rs);
+              kmn = ~kmx;
+            } else {
+              empty = true;
+            }
+          }
+          kmx = __reduce_max_sync(0xffffffffu, kmx);
+          kmn = __reduce_max_sync(0xffffffffu, kmn);
+          const int ne = __popc(__ballot_sync(0xffffffffu, empty));
+          if (lane == 0) {
+            if (kmx) atomicMax(p.kmax + u, kmx);
+            if (kmn) atomicMax(p.kmin + u, kmn);
+            if (ne) atomicAdd(p.ninf + u, ne);
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (threadIdx.x == 128) st_release_cta(&ms->epi_done, it + 1);
         }
       }
+      __syncwarp();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (warp == 1) tmem_dealloc(tmem, 32);
     }
-    __syncwarp();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 32);
-
   }
 
-  // ============================================================ phase B
-  // Exact selection over all C keys of the unit by every block (the
-  // fallback for crowded boundary buckets): keys from the rkey workspace.
-  auto select_all_keys = [&]() {
-    // Thread t of round rd owns the keys of ids [rd kRound + 32 t, +32): every
-    // pass below works on 32 keys held in registers (independent, unrolled).
-    const float* rk = p.rkey + (size_t)bh * C;
-    const bool cached = C <= p.L.lkeys_cap;
-    const bool vec = (C & 3) == 0;
-    if (cached) {
-      if (vec) {
-        for (int i = threadIdx.x; i < C / 4; i += kThreads) cp_async16(keys + 4 * i, rk + 4 * i);
-      } else {
-        for (int i = threadIdx.x; i < C; i += kThreads) cp_async4(keys + i, rk + i);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-    }
-    const float* K = cached ? keys : rk;
+  // ============================================================ step B
+  // Exact selection over the C keys of unit u by this block alone.  Keys are
+  // taken in rounds of kRound ids; thread t holds ids round_base + kPer t + j
+  // in registers (16-byte loads).  The key range comes from step A.
+  auto select_unit = [&](int u) {
+    int* hist = reinterpret_cast<int*>(sm + kOffHist);
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kOffCand);
+    const float* rk = p.rkey + (size_t)u * C;
     const int rounds = (C + kRound - 1) / kRound;
-    auto load32 = [&](int rd, float (&kk)[kPer]) {
+    const bool vec = (C & 3) == 0;
+    float kk[kPer];
+    auto load_round = [&](int rd) {
       const int c0 = rd * kRound + threadIdx.x * kPer;
       if (vec && c0 + kPer <= C) {
 #pragma unroll
         for (int i = 0; i < kPer; i += 4) {
-          const float4 v = cached ? *reinterpret_cast<const float4*>(K + c0 + i)
-                                  : __ldcg(reinterpret_cast<const float4*>(K + c0 + i));
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(rk + c0 + i));
           kk[i] = v.x;
           kk[i + 1] = v.y;
           kk[i + 2] = v.z;
@@ -423,101 +556,57 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          const int c = c0 + i;
-          kk[i] = c < C ? (cached ? K[c] : __ldcg(K + c)) : 0.f;
-        }
+        for (int i = 0; i < kPer; ++i) kk[i] = c0 + i < C ? __ldcg(rk + c0 + i) : 0.f;
       }
     };
-    // 1) range of the finite keys, number of -inf keys (empty clusters)
-    float lo = FLT_MAX, hi = -FLT_MAX;
-    int ninf = 0;
-    for (int rd = 0; rd < rounds; ++rd) {
-      float kk[kPer];
-      load32(rd, kk);
-      const int c0 = rd * kRound + threadIdx.x * kPer;
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        if (c0 + i < C) {
-          if (kk[i] == -INFINITY) {
-            ++ninf;
-          } else {
-            lo = fminf(lo, kk[i]);
-            hi = fmaxf(hi, kk[i]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-      ninf += __shfl_xor_sync(0xffffffffu, ninf, off);
-    }
-    if (lane == 0) {
-      ms->red[0][warp] = lo;
-      ms->red[1][warp] = hi;
-      ms->wtot[0][warp] = ninf;
-    }
-    for (int i = threadIdx.x; i < kNB; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    lo = FLT_MAX;
-    hi = -FLT_MAX;
-    ninf = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      lo = fminf(lo, ms->red[0][w]);
-      hi = fmaxf(hi, ms->red[1][w]);
-      ninf += ms->wtot[0][w];
-    }
+    load_round(0);
+    for (int i = threadIdx.x; i < kNB; i += NT) hist[i] = 0;
+    if (threadIdx.x < 2) ms->ncand[threadIdx.x] = 0;
+    const uint32_t kmx = __ldcg(p.kmax + u), kmn = __ldcg(p.kmin + u);
+    const int ninf = __ldcg(p.ninf + u);
     const int nfin = C - ninf;
+    const float lo = nfin > 0 ? float_from_order_key(~kmn) : 0.f;
+    const float hi = nfin > 0 ? float_from_order_key(kmx) : 0.f;
     const float scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
-    // 2) histogram over value buckets (monotone in the key)
+    __syncthreads();
+    // 1) histogram over value buckets (monotone in the key)
     for (int rd = 0; rd < rounds; ++rd) {
-      float kk[kPer];
-      load32(rd, kk);
+      if (rd > 0) load_round(rd);
       const int c0 = rd * kRound + threadIdx.x * kPer;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int b = bucket_of(kk[i], lo, scale);
-        if (c0 + i < C && b >= 0) atomicAdd(&hist[b], 1);
+      for (int j = 0; j < kPer; ++j) {
+        const int b = bucket_of(kk[j], lo, scale);
+        if (c0 + j < C && b >= 0) atomicAdd(&hist[b], 1);
       }
     }
     __syncthreads();
-    // 3) boundary buckets of ranks kA = kr and kB = kr + ke from the top:
-    //    thread t owns buckets kNB-1-8t .. kNB-8-8t (descending)
+    // 2) boundary buckets of ranks kr and kr + ke from the top: thread t
+    //    owns kNB / NT consecutive buckets, the highest for t = 0
     {
-      int hc[kNB / kThreads];
+      constexpr int BPT = kNB / NT;
+      int hc[BPT];
       int sum = 0;
 #pragma unroll
-      for (int i = 0; i < kNB / kThreads; ++i) {
-        hc[i] = hist[kNB - 1 - (kNB / kThreads) * threadIdx.x - i];
+      for (int i = 0; i < BPT; ++i) {
+        hc[i] = hist[kNB - 1 - BPT * threadIdx.x - i];
         sum += hc[i];
       }
-      int incl = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      if (lane == 31) ms->scan[warp] = incl;
       if (threadIdx.x < 2) {
         const int k = threadIdx.x == 0 ? kr : kr + ke;
         ms->bucket[threadIdx.x] = k <= 0 ? -2 : (k > nfin ? -1 : -3);
         ms->above[threadIdx.x] = k > nfin ? nfin : 0;
       }
-      __syncthreads();
-      int excl = incl - sum;
-      for (int w = 0; w < warp; ++w) excl += ms->scan[w];
+      int total_fin;
+      const int excl = block_scan<NT>(sum, ms->scan, &total_fin);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
         const int k = w == 0 ? kr : kr + ke;
         if (k > 0 && k <= nfin && excl < k && excl + sum >= k) {
           int cum = excl;
 #pragma unroll
-          for (int i = 0; i < kNB / kThreads; ++i) {
+          for (int i = 0; i < BPT; ++i) {
             if (cum + hc[i] >= k) {
-              ms->bucket[w] = kNB - 1 - (kNB / kThreads) * threadIdx.x - i;
+              ms->bucket[w] = kNB - 1 - BPT * threadIdx.x - i;
               ms->above[w] = cum;
               break;
             }
@@ -527,30 +616,39 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
       }
       __syncthreads();
     }
-    // 4) exact order inside each boundary bucket
-    for (int w = 0; w < 2; ++w) {
-      const int b = ms->bucket[w];
-      if (b == -2) continue;
-      const int k = (w == 0 ? kr : kr + ke) - ms->above[w];  // 1-based rank in the bucket
-      const int nb = b >= 0 ? hist[b] : ninf;
-      if (nb <= kBoundaryCap) {
-        if (threadIdx.x == 0) ms->ncand[w] = 0;
-        __syncthreads();
-        for (int rd = 0; rd < rounds; ++rd) {
-          float kk[kPer];
-          load32(rd, kk);
-          const int c0 = rd * kRound + threadIdx.x * kPer;
+    // 3) exact order inside each boundary bucket: members of both buckets
+    //    gathered in one pass, ranked by (key desc, id asc)
+    int bk[2];
+    bool small[2];
 #pragma unroll
-          for (int i = 0; i < kPer; ++i) {
-            if (c0 + i < C && bucket_of(kk[i], lo, scale) == b) {
+    for (int w = 0; w < 2; ++w) {
+      bk[w] = ms->bucket[w];
+      const int nb = bk[w] >= 0 ? hist[bk[w]] : (bk[w] == -1 ? ninf : 0);
+      small[w] = bk[w] != -2 && nb <= kBoundaryCap;
+    }
+    if (small[0] || small[1]) {
+      for (int rd = 0; rd < rounds; ++rd) {
+        if (rounds > 1) load_round(rd);
+        const int c0 = rd * kRound + threadIdx.x * kPer;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          const int b = bucket_of(kk[j], lo, scale);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            if (small[w] && b == bk[w] && c0 + j < C) {
               const int slot = atomicAdd(&ms->ncand[w], 1);
-              cand[w * kBoundaryCap + slot] = ord64(float_order_key(kk[i]), c0 + i);
+              cand[w * kBoundaryCap + slot] = ord64(float_order_key(kk[j]), c0 + j);
             }
           }
         }
-        __syncthreads();
+      }
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        if (!small[w]) continue;
+        const int k = (w == 0 ? kr : kr + ke) - ms->above[w];  // 1-based rank in the bucket
         const int n = ms->ncand[w];
-        for (int i = threadIdx.x; i < n; i += kThreads) {
+        for (int i = threadIdx.x; i < n; i += NT) {
           const unsigned long long me = cand[w * kBoundaryCap + i];
           int rank = 0;
           for (int t = 0; t < n; ++t) rank += cand[w * kBoundaryCap + t] > me;
@@ -559,754 +657,548 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1)
             ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(me & 0xFFFFFFFFull));
           }
         }
-        __syncthreads();
-      } else {
-        uint32_t Tu;
-        int Tid;
-        kth_in_bucket_slow(K, cached, C, b, lo, scale, k, ms, hist, &Tu, &Tid);
-        if (threadIdx.x == 0) {
-          ms->Tu[w] = Tu;
-          ms->Tid[w] = Tid;
-        }
-        __syncthreads();
       }
     }
-    const bool selA = ms->bucket[0] != -2, selB = ms->bucket[1] != -2;
+    for (int w = 0; w < 2; ++w) {
+      if (bk[w] == -2 || small[w]) continue;
+      uint32_t Tu;
+      int Tid;
+      const int k = (w == 0 ? kr : kr + ke) - ms->above[w];
+      kth_in_bucket_slow<NT>(rk, C, bk[w], lo, scale, k, ms, hist, &Tu, &Tid);
+      if (threadIdx.x == 0) {
+        ms->Tu[w] = Tu;
+        ms->Tid[w] = Tid;
+      }
+    }
+    __syncthreads();
+    const bool selA = bk[0] != -2, selB = bk[1] != -2;
     const unsigned long long TA = selA ? ord64(ms->Tu[0], ms->Tid[0]) : ~0ull;
     const unsigned long long TB = selB ? ord64(ms->Tu[1], ms->Tid[1]) : ~0ull;
-    // 5) membership and compaction in id order
-    const bool write_global = p.mode == kModeSelect && j == 0;
-    const bool report = p.mode == kModeFull && p.sel_user != nullptr;
-    int32_t* selg = p.sel + (size_t)bh * (p.k_r + p.k_e);
-    int32_t* selu = p.sel_user ? p.sel_user + (size_t)bh * (p.k_r + p.k_e) : nullptr;
+    // 4) membership and compaction in id order; R ids go to rrow_sm for now
+    int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
+    int32_t* selu = p.sel_user ? p.sel_user + (size_t)u * (p.k_r + p.k_e) : nullptr;
     int baseR = 0, baseE = 0;
     for (int rd = 0; rd < rounds; ++rd) {
-      float kk[kPer];
-      load32(rd, kk);
+      if (rounds > 1) load_round(rd);
       const int c0 = rd * kRound + threadIdx.x * kPer;
       uint32_t mR = 0, mE = 0;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        if (c0 + i < C) {
-          const unsigned long long o = ord64(float_order_key(kk[i]), c0 + i);
+      for (int j = 0; j < kPer; ++j) {
+        if (c0 + j < C) {
+          const unsigned long long o = ord64(float_order_key(kk[j]), c0 + j);
           const bool inR = selA && o >= TA;
           const bool inE = !inR && selB && o >= TB;
-          mR |= (uint32_t)inR << i;
-          mE |= (uint32_t)inE << i;
+          mR |= (uint32_t)inR << j;
+          mE |= (uint32_t)inE << j;
         }
       }
       // block exclusive scan of (count R, count E) packed in one int
-      const int v = (__popc(mR) << 16) | __popc(mE);
-      int incl = v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      if (lane == 31) ms->scan[warp] = incl;
-      __syncthreads();
-      int excl = incl - v, tot = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) excl += ms->scan[w];
-        tot += ms->scan[w];
-      }
-      __syncthreads();
+      int tot;
+      const int excl = block_scan<NT>((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
       int pr = baseR + (excl >> 16), pe = baseE + (excl & 0xFFFF);
       while (mR) {
         const int c = c0 + __ffs(mR) - 1;
         mR &= mR - 1;
-        rbase_sm[pr] = c;  // cluster ids for now; row offsets below
-        if (write_global) selg[pr] = c;
-        if (report && j == 0) selu[pr] = c;
+        rrow_sm[pr] = c;
+        selg[pr] = c;
+        if (selu) selu[pr] = c;
         ++pr;
       }
       while (mE) {
         const int c = c0 + __ffs(mE) - 1;
         mE &= mE - 1;
-        if (pe >= e0 && pe < e1) {
-          eslice[pe - e0] = c;
-          if (report) selu[p.k_r + pe] = c;
-        }
-        if (write_global) selg[p.k_r + pe] = c;
+        selg[p.k_r + pe] = c;
+        if (selu) selu[p.k_r + pe] = c;
         ++pe;
       }
       baseR += tot >> 16;
       baseE += tot & 0xFFFF;
     }
+    for (int i = kr + threadIdx.x; i < p.k_r; i += NT) {
+      selg[i] = -1;
+      if (selu) selu[i] = -1;
+    }
+    for (int i = ke + threadIdx.x; i < p.k_e; i += NT) {
+      selg[p.k_r + i] = -1;
+      if (selu) selu[p.k_r + i] = -1;
+    }
     __syncthreads();
-    // 6) sizes of the R clusters (prefix = execution-buffer rows) and their
+    // 5) sizes of the R clusters (prefix = execution-buffer rows) and their
     //    first rows in Kp/Vp; loads issued together, then one block scan
     {
-      constexpr int kPerR = kMaxRetrieval / kThreads;  // 16
-      const int per = (kr + kThreads - 1) / kThreads;
+      constexpr int kPerR = kMaxRetrieval / NT;
+      const int per = (kr + NT - 1) / NT;
       const int i0 = min(kr, (int)threadIdx.x * per), i1 = min(kr, i0 + per);
       int cn[kPerR], of[kPerR];
 #pragma unroll
-      for (int u = 0; u < kPerR; ++u) {
-        const int i = i0 + u;
+      for (int w = 0; w < kPerR; ++w) {
+        const int i = i0 + w;
         const bool in = i < i1;
-        const int c = in ? rbase_sm[i] : 0;
-        cn[u] = in ? __ldg(p.counts + (size_t)bh * C + c) : 0;
-        of[u] = (in && !p.exec_rows) ? __ldg(p.offsets + (size_t)bh * (C + 1) + c) : 0;
+        const int c = in ? rrow_sm[i] : 0;
+        cn[w] = in ? __ldg(p.counts + (size_t)u * C + c) : 0;
+        of[w] = in ? __ldg(p.offsets + (size_t)u * (C + 1) + c) : 0;
       }
       int loc = 0;
 #pragma unroll
-      for (int u = 0; u < kPerR; ++u) loc += cn[u];
-      int incl = loc;
+      for (int w = 0; w < kPerR; ++w) loc += cn[w];
+      int total;
+      int run = block_scan<NT>(loc, ms->scan, &total);
+      int32_t* rp = p.rpre + (size_t)u * (p.k_r + 1);
+      int32_t* rr = p.rrow + (size_t)u * (p.k_r > 0 ? p.k_r : 1);
+      int32_t* ru = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      if (lane == 31) ms->scan[warp] = incl;
-      __syncthreads();
-      int run = incl - loc, total = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) run += ms->scan[w];
-        total += ms->scan[w];
-      }
-#pragma unroll
-      for (int u = 0; u < kPerR; ++u) {
-        const int i = i0 + u;
+      for (int w = 0; w < kPerR; ++w) {
+        const int i = i0 + w;
         if (i < i1) {
-          rpre_sm[i] = run;
-          rbase_sm[i] = of[u];
-          run += cn[u];
+          rp[i] = run;
+          rr[i] = of[w];
+          if (ru) ru[i] = run;
+          run += cn[w];
         }
       }
-      if (threadIdx.x == 0) rpre_sm[kr] = total;
-      __syncthreads();
+      for (int i = kr + threadIdx.x; i <= p.k_r; i += NT) {
+        rp[i] = total;
+        if (ru) ru[i] = total;
+      }
     }
-    if (write_global) {
-      for (int i = kr + threadIdx.x; i < p.k_r; i += kThreads) selg[i] = -1;
-      for (int i = ke + threadIdx.x; i < p.k_e; i += kThreads) selg[p.k_r + i] = -1;
-      for (int i = threadIdx.x; i <= p.k_r; i += kThreads)
-        p.rpre[(size_t)bh * (p.k_r + 1) + i] = rpre_sm[i < kr ? i : kr];
-      if (p.rpre_user)
-        for (int i = threadIdx.x; i <= p.k_r; i += kThreads)
-          p.rpre_user[(size_t)bh * (p.k_r + 1) + i] = rpre_sm[i < kr ? i : kr];
-      __syncthreads();
-      if (p.sel_user)
-        for (int i = threadIdx.x; i < p.k_r + p.k_e; i += kThreads) selu[i] = __ldcg(selg + i);
-    }
-    if (report) {
-      if (j == 0)
-        for (int i = kr + threadIdx.x; i < p.k_r; i += kThreads) selu[i] = -1;
-      if (j == p.P - 1)
-        for (int i = ke + threadIdx.x; i < p.k_e; i += kThreads) selu[p.k_r + i] = -1;
-    }
+    // 6) publish
+    __threadfence();
     __syncthreads();
+    if (threadIdx.x == 0) st_release(p.ready + u, 1);
   };
 
-  if (p.mode == kModeAttend) {
-    // selection left in the workspace by a select call
-    const int32_t* selb = p.sel + (size_t)bh * (p.k_r + p.k_e);
-    for (int i = threadIdx.x; i <= kr; i += kThreads)
-      rpre_sm[i] = p.rpre[(size_t)bh * (p.k_r + 1) + i];
-    for (int i = threadIdx.x; i < kr; i += kThreads)
-      rbase_sm[i] = p.exec_rows ? 0 : p.offsets[(size_t)bh * (C + 1) + selb[i]];
-    for (int i = e0 + threadIdx.x; i < e1; i += kThreads) eslice[i - e0] = selb[p.k_r + i];
-    __syncthreads();
-  } else if (C > 0) {
-    // ---- B1: key range of the unit (finite keys), -inf count
-    {
-      float lo = FLT_MAX, hi = -FLT_MAX;
-      int ninf = 0;
-      for (int i = threadIdx.x; i < n_loc; i += kThreads) {
-        const float r = lkeys[i];
-        if (r == -INFINITY) {
-          ++ninf;
-        } else {
-          lo = fminf(lo, r);
-          hi = fmaxf(hi, r);
-        }
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-        ninf += __shfl_xor_sync(0xffffffffu, ninf, off);
-      }
-      if (lane == 0) {
-        ms->red[0][warp] = lo;
-        ms->red[1][warp] = hi;
-        ms->wtot[0][warp] = ninf;
-      }
-      for (int i = threadIdx.x; i < kNB; i += kThreads) hist[i] = 0;
-      if (threadIdx.x < 2) ms->ncand[threadIdx.x] = 0;
-      __syncthreads();
+  // Unit u is selected by block NB - 1 - (u mod NB): the blocks at the end
+  // of the grid score the fewest tiles.
+  if (p.mode != kModeAttend && tiles_h > 0) {
+    for (int u = (int)gridDim.x - 1 - (int)blockIdx.x; u < p.BH; u += (int)gridDim.x) {
       if (threadIdx.x == 0) {
-        float l2 = FLT_MAX, h2 = -FLT_MAX;
-        int n2 = 0;
-        for (int w = 0; w < kWarps; ++w) {
-          l2 = fminf(l2, ms->red[0][w]);
-          h2 = fmaxf(h2, ms->red[1][w]);
-          n2 += ms->wtot[0][w];
-        }
-        ms->rlo = l2;
-        ms->rhi = h2;
-        ms->rninf = n2;
-      }
-    }
-    cluster.sync();  // S1: every block's range; histograms and counters zeroed
-    float lo = FLT_MAX, hi = -FLT_MAX;
-    int ninf = 0;
-    for (int r = 0; r < p.P; ++r) {
-      const Misc* mr = cluster.map_shared_rank(ms, r);
-      lo = fminf(lo, mr->rlo);
-      hi = fmaxf(hi, mr->rhi);
-      ninf += mr->rninf;
-    }
-    const int nfin = C - ninf;
-    const float scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
-    // ---- B2: value histogram of the unit: local histograms, then a
-    //      reduce-scatter (block r sums bucket slice r over the cluster) and an
-    //      all-gather of the slices, both through distributed shared memory
-    for (int i = threadIdx.x; i < n_loc; i += kThreads) {
-      const int b = bucket_of(lkeys[i], lo, scale);
-      if (b >= 0) atomicAdd(hist + b, 1);
-    }
-    cluster.sync();  // S2: local histograms complete
-    {
-      const int b0 = kNB * j / p.P, b1 = kNB * (j + 1) / p.P;
-      for (int b = b0 + threadIdx.x; b < b1; b += kThreads) {
-        int sum = 0;
-        for (int r = 0; r < p.P; ++r) sum += cluster.map_shared_rank(hist, r)[b];
-        gslice[b - b0] = sum;
-      }
-    }
-    cluster.sync();  // S2b: reduced slices complete; local histograms no longer read
-    for (int b = threadIdx.x; b < kNB; b += kThreads) {
-      int r = (int)(((long long)(b + 1) * p.P + kNB - 1) / kNB) - 1;  // slice owning b
-      hist[b] = cluster.map_shared_rank(gslice, r)[b - kNB * r / p.P];
-    }
-    __syncthreads();
-    // ---- B3: boundary buckets of ranks kA = kr and kB = kr + ke from the
-    //      top; thread t owns buckets kNB-1-8t .. kNB-8-8t (descending)
-    {
-      int hc[kNB / kThreads];
-      int sum = 0;
-#pragma unroll
-      for (int i = 0; i < kNB / kThreads; ++i) {
-        hc[i] = hist[kNB - 1 - (kNB / kThreads) * threadIdx.x - i];
-        sum += hc[i];
-      }
-      if (threadIdx.x < 2) {
-        const int k = threadIdx.x == 0 ? kr : kr + ke;
-        ms->bucket[threadIdx.x] = k <= 0 ? -2 : (k > nfin ? -1 : -3);
-        ms->above[threadIdx.x] = k > nfin ? nfin : 0;
-      }
-      int tot;
-      const int excl = block_excl_scan(sum, ms->scan, &tot);
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int k = w == 0 ? kr : kr + ke;
-        if (k > 0 && k <= nfin && excl < k && excl + sum >= k) {
-          int cum = excl;
-#pragma unroll
-          for (int i = 0; i < kNB / kThreads; ++i) {
-            if (cum + hc[i] >= k) {
-              ms->bucket[w] = kNB - 1 - (kNB / kThreads) * threadIdx.x - i;
-              ms->above[w] = cum;
-              break;
-            }
-            cum += hc[i];
-          }
-        }
+        const bool ok = wait_count(p.done + u, tiles_h, p.status);
+        if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
+        ms->flag = ok;
       }
       __syncthreads();
+      if (!ms->flag) break;
+      __threadfence();
+      select_unit(u);
     }
-    bool crowded = false;
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      const int b = ms->bucket[w];
-      const int nb = b >= 0 ? hist[b] : (b == -1 ? ninf : 0);
-      crowded |= nb > kBoundaryCap;
-    }
-    if (crowded) {
-      cluster.sync();  // every block has gathered the slices
-      select_all_keys();
-    } else {
-      // ---- B4: members of the boundary buckets, gathered in block 0
-      unsigned long long* cand0 = cluster.map_shared_rank(cand, 0);
-      int* ncand0 = cluster.map_shared_rank(&ms->ncand[0], 0);
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int b = ms->bucket[w];
-        if (b == -2) continue;
-        for (int i = threadIdx.x; i < n_loc; i += kThreads) {
-          const float r = lkeys[i];
-          if (bucket_of(r, lo, scale) == b) {
-            const int slot = atomicAdd(ncand0 + w, 1);
-            cand0[w * kBoundaryCap + slot] = ord64(float_order_key(r), c_begin + i);
-          }
-        }
-      }
-      cluster.sync();  // S3
-      // thresholds: the k-th member of each boundary bucket in exact order
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int b = ms->bucket[w];
-        if (b == -2) continue;
-        const int n = ncand0[w];
-        const int k = (w == 0 ? kr : kr + ke) - ms->above[w];
-        if (j != 0)
-          for (int i = threadIdx.x; i < n; i += kThreads)
-            cand[w * kBoundaryCap + i] = cand0[w * kBoundaryCap + i];
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kThreads) {
-          const unsigned long long me = cand[w * kBoundaryCap + i];
-          int rank = 0;
-          for (int t = 0; t < n; ++t) rank += cand[w * kBoundaryCap + t] > me;
-          if (rank == k - 1) {
-            ms->Tu[w] = (uint32_t)(me >> 32);
-            ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(me & 0xFFFFFFFFull));
-          }
-        }
-        __syncthreads();
-      }
-      const bool selA = ms->bucket[0] != -2, selB = ms->bucket[1] != -2;
-      const unsigned long long TA = selA ? ord64(ms->Tu[0], ms->Tid[0]) : ~0ull;
-      const unsigned long long TB = selB ? ord64(ms->Tu[1], ms->Tid[1]) : ~0ull;
-      // ---- B5: this block's members, in id order: thread t owns the local
-      //      keys [t kk, t kk + kk); positions from a block scan and the
-      //      cluster prefix of the blocks' member counts
-      const int kk = (n_loc + kThreads - 1) / kThreads;  // <= 32 (n_loc <= 8192)
-      const int l0 = min(n_loc, (int)threadIdx.x * kk), l1 = min(n_loc, l0 + kk);
-      uint32_t mR = 0, mE = 0;
-      for (int i = l0; i < l1; ++i) {
-        const unsigned long long o = ord64(float_order_key(lkeys[i]), c_begin + i);
-        const bool inR = selA && o >= TA;
-        const bool inE = !inR && selB && o >= TB;
-        mR |= (uint32_t)inR << (i - l0);
-        mE |= (uint32_t)inE << (i - l0);
-      }
-      int tot;
-      const int x = block_excl_scan((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
+  }
+  if (p.mode == kModeSelect) return;
+
+  // ============================================================ step C
+  const int npairs = p.BH * p.S;
+  const bool exec = p.exec_rows > 0;
+  const long long lim_rows = exec ? p.exec_rows : p.M;
+  const long long row_base_stride = exec ? p.exec_rows : p.M;
+  const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
+  for (int pi = blockIdx.x; pi < npairs; pi += gridDim.x) {
+    const int u = pi % p.BH, s = pi / p.BH;
+    if (p.mode == kModeFull && tiles_h > 0) {
       if (threadIdx.x == 0) {
-        ms->cntR = tot >> 16;
-        ms->cntE = tot & 0xFFFF;
+        const bool ok = wait_count(p.ready + u, 1, p.status);
+        if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
+        ms->flag = ok;
       }
-      cluster.sync();  // S4
-      int baseR = 0, baseE = 0;
-      for (int r = 0; r < j; ++r) {
-        const Misc* mr = cluster.map_shared_rank(ms, r);
-        baseR += mr->cntR;
-        baseE += mr->cntE;
-      }
-      const bool write_global = p.mode == kModeSelect;
-      const bool report = p.mode == kModeFull && p.sel_user != nullptr;
-      int32_t* selg = p.sel + (size_t)bh * (p.k_r + p.k_e);
-      int32_t* selu = p.sel_user ? p.sel_user + (size_t)bh * (p.k_r + p.k_e) : nullptr;
-      // R members: (id, size, first row) to block 0
-      int32_t* rtrip0 = cluster.map_shared_rank(rtrip, 0);
-      int pr = baseR + (x >> 16), pe = baseE + (x & 0xFFFF);
-      while (mR) {
-        const int c = c_begin + l0 + __ffs(mR) - 1;
-        mR &= mR - 1;
-        rtrip0[pr] = c;
-        rtrip0[kr + pr] = __ldg(p.counts + (size_t)bh * C + c);
-        rtrip0[2 * kr + pr] = p.exec_rows ? 0 : __ldg(p.offsets + (size_t)bh * (C + 1) + c);
-        if (write_global) selg[pr] = c;
-        if (report) selu[pr] = c;
-        ++pr;
-      }
-      // E members: each id to the block that attends it
-      while (mE) {
-        const int c = c_begin + l0 + __ffs(mE) - 1;
-        mE &= mE - 1;
-        const int owner = (int)(((long long)(pe + 1) * p.P + ke - 1) / ke) - 1;
-        cluster.map_shared_rank(eslice, owner)[pe - e_first(owner)] = c;
-        if (write_global) selg[p.k_r + pe] = c;
-        if (report) selu[p.k_r + pe] = c;
-        ++pe;
-      }
-      cluster.sync();  // S5: R triples complete in block 0, E slices in their blocks
-      // ---- B6: prefix of the R clusters' sizes (execution-buffer rows)
-      constexpr int kPerR = kMaxRetrieval / kThreads;  // 16
-      const int per = (kr + kThreads - 1) / kThreads;
-      const int i0 = min(kr, (int)threadIdx.x * per), i1 = min(kr, i0 + per);
-      int cn[kPerR], of[kPerR];
-#pragma unroll
-      for (int u = 0; u < kPerR; ++u) {
-        const bool in = i0 + u < i1;
-        cn[u] = in ? rtrip0[kr + i0 + u] : 0;
-        of[u] = in ? rtrip0[2 * kr + i0 + u] : 0;
-      }
-      int loc = 0;
-#pragma unroll
-      for (int u = 0; u < kPerR; ++u) loc += cn[u];
-      int total;
-      int run = block_excl_scan(loc, ms->scan, &total);
-#pragma unroll
-      for (int u = 0; u < kPerR; ++u) {
-        const int i = i0 + u;
-        if (i < i1) {
-          rpre_sm[i] = run;
-          rbase_sm[i] = of[u];
-          run += cn[u];
-        }
-      }
-      if (threadIdx.x == 0) rpre_sm[kr] = total;
       __syncthreads();
-      if (j == 0 && (write_global || report)) {
-        // tails of the id lists and the execution-buffer prefix
-        int32_t* dst = write_global ? selg : selu;
-        for (int i = kr + threadIdx.x; i < p.k_r; i += kThreads) {
-          if (write_global) selg[i] = -1;
-          if (p.sel_user) p.sel_user[(size_t)bh * (p.k_r + p.k_e) + i] = -1;
+      if (!ms->flag) break;
+    }
+    // the unit's R prefix and first rows, coalesced into shared memory
+    if (C > 0) {
+      const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
+      const int32_t* rrg = p.rrow + (size_t)u * (p.k_r > 0 ? p.k_r : 1);
+      for (int i0 = 0; i0 <= kr; i0 += 4 * NT) {
+        int a[4], b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = i0 + j * NT + threadIdx.x;
+          a[j] = i <= kr ? __ldcg(rpg + i) : 0;
+          b[j] = (!exec && i < kr) ? __ldcg(rrg + i) : 0;
         }
-        for (int i = ke + threadIdx.x; i < p.k_e; i += kThreads) {
-          if (write_global) selg[p.k_r + i] = -1;
-          if (p.sel_user) p.sel_user[(size_t)bh * (p.k_r + p.k_e) + p.k_r + i] = -1;
-        }
-        (void)dst;
-        if (write_global) {
-          for (int i = threadIdx.x; i <= p.k_r; i += kThreads)
-            p.rpre[(size_t)bh * (p.k_r + 1) + i] = rpre_sm[i < kr ? i : kr];
-          if (p.rpre_user)
-            for (int i = threadIdx.x; i <= p.k_r; i += kThreads)
-              p.rpre_user[(size_t)bh * (p.k_r + 1) + i] = rpre_sm[i < kr ? i : kr];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = i0 + j * NT + threadIdx.x;
+          if (i <= kr) rpre_sm[i] = a[j];
+          if (i < kr) rrow_sm[i] = b[j];
         }
       }
-      if (write_global && p.sel_user)
-        for (int i = threadIdx.x; i < kr; i += kThreads)
-          p.sel_user[(size_t)bh * (p.k_r + p.k_e) + i] = rtrip0[i];
-      if (write_global && p.sel_user)
-        for (int i = e0 + threadIdx.x; i < e1; i += kThreads)
-          p.sel_user[(size_t)bh * (p.k_r + p.k_e) + p.k_r + i] = eslice[i - e0];
+    } else if (threadIdx.x == 0) {
+      rpre_sm[0] = 0;
     }
-  } else {
-    if (threadIdx.x == 0) rpre_sm[0] = 0;
-    if (p.mode != kModeAttend && p.sel_user && j == 0)
-      for (int i = threadIdx.x; i < p.k_r + p.k_e; i += kThreads)
-        p.sel_user[(size_t)bh * (p.k_r + p.k_e) + i] = -1;
-    if (p.mode == kModeSelect && j == 0) {
-      int32_t* selg = p.sel + (size_t)bh * (p.k_r + p.k_e);
-      for (int i = threadIdx.x; i < p.k_r + p.k_e; i += kThreads) selg[i] = -1;
-      for (int i = threadIdx.x; i <= p.k_r; i += kThreads) {
-        p.rpre[(size_t)bh * (p.k_r + 1) + i] = 0;
-        if (p.rpre_user) p.rpre_user[(size_t)bh * (p.k_r + 1) + i] = 0;
-      }
-    }
-    __syncthreads();
-  }
-
-  if (p.mode == kModeSelect) {
-    cluster.sync();  // block 0's R triples were read by every block
-    return;
-  }
-
-  // ============================================================ phase C
-  // Work items of this block: tokens [t0, t1) of steady + retrieval, then
-  // estimation clusters [e0, e1).  They are brought into shared memory in
-  // chunks by 16-byte cp.async copies (double buffered: the next chunk is in
-  // flight while the current one is consumed); a 16-lane group handles one
-  // token or cluster at a time, lane l16 owning dims 8 l16 .. 8 l16 + 7.
-  const int l16 = threadIdx.x & 15;
-  const int hw = threadIdx.x >> 4;  // 16 half-warps
-  float qv[G][8];
+    // A fragments of Q (rows = query heads, padded to 16 with zeros):
+    // qa[kk][0] = Q[gid][16 kk + 2 tig ..], qa[kk][1] = Q[gid][16 kk + 8 + 2 tig ..]
+    uint32_t qa[8][2];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const uint4 raw = ldg_nc_v4(p.q + ((size_t)bh * G + g) * kHeadDim + l16 * 8);
-    bf16x8_to_float(raw, qv[g]);
-  }
-  float m[G], l[G], o[G][8];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[g][i] = 0.f;
-  }
-  const long long T_R = C > 0 ? rpre_sm[kr] : 0;
-  const long long T = p.n_steady + T_R;
-  const long long t0 = T * j / p.P, t1 = T * (j + 1) / p.P;
-  const size_t steady_base = (size_t)bh * p.n_steady * kHeadDim;
-  const size_t rbase_rows = p.exec_rows ? (size_t)bh * p.exec_rows : (size_t)bh * p.M;
-  const long long lim_rows = p.exec_rows ? p.exec_rows : p.M;
-  // Everything this block reads below is first requested into L2 in bulk,
-  // so the chunked copies wait on L2 rather than on a round trip to HBM each.
-  {
-    const long long s_end = min(t1, (long long)p.n_steady);
-    if (threadIdx.x == 0 && t0 < s_end) {
-      const uint32_t bytes = (uint32_t)((s_end - t0) * kHeadDim * 2);
-      prefetch_l2_bulk(p.Ks + steady_base + (size_t)t0 * kHeadDim, bytes);
-      prefetch_l2_bulk(p.Vs + steady_base + (size_t)t0 * kHeadDim, bytes);
-    }
-    const long long r0 = max(t0, (long long)p.n_steady) - p.n_steady;
-    const long long r1 = t1 - p.n_steady;
-    if (r1 > r0) {
-      if (p.exec_rows) {
-        if (threadIdx.x == 0 && r1 <= p.exec_rows) {
-          const uint32_t bytes = (uint32_t)((r1 - r0) * kHeadDim * 2);
-          prefetch_l2_bulk(p.Kr + (rbase_rows + (size_t)r0) * kHeadDim, bytes);
-          prefetch_l2_bulk(p.Vr + (rbase_rows + (size_t)r0) * kHeadDim, bytes);
-        }
+    for (int kk = 0; kk < 8; ++kk) {
+      if (gid < G) {
+        const __nv_bfloat16* qr = p.q + ((size_t)u * G + gid) * kHeadDim + kk * 16 + tig * 2;
+        qa[kk][0] = *reinterpret_cast<const uint32_t*>(qr);
+        qa[kk][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
       } else {
-        int first = 0, hi = kr - 1;  // last cluster with rpre <= r0
-        while (first < hi) {
-          const int mid = (first + hi + 1) >> 1;
-          if (rpre_sm[mid] <= r0) first = mid; else hi = mid - 1;
+        qa[kk][0] = qa[kk][1] = 0u;
+      }
+    }
+    __syncthreads();
+    const int n_st = p.n_steady;
+    const int T_R = C > 0 ? rpre_sm[kr] : 0;
+    const long long W = (long long)n_st + T_R + ke;
+    const long long w0 = W * s / p.S, w1 = W * (s + 1) / p.S;
+    const int tok_end = n_st + T_R;  // items below are tokens, above E clusters
+    const int nrounds = (int)((w1 - w0 + kRoundItems - 1) / kRoundItems);
+    struct Round {
+      int ta, ntok, npad, ea, ne;
+      uint32_t off_v, off_ev, off_es, off_en;
+    };
+    auto round_of = [&](int r) {
+      const long long a = w0 + (long long)r * kRoundItems;
+      const long long b = min(w1, a + kRoundItems);
+      Round rd;
+      rd.ta = (int)min(a, (long long)tok_end);
+      rd.ntok = (int)min(b, (long long)tok_end) - rd.ta;
+      rd.npad = (rd.ntok + 15) & ~15;
+      rd.ea = (int)(max(a, (long long)tok_end) - tok_end);
+      rd.ne = (int)(max(b, (long long)tok_end) - tok_end) - rd.ea;
+      rd.off_v = rd.npad * 256;
+      rd.off_ev = 2 * rd.npad * 256;
+      rd.off_es = rd.off_ev + rd.ne * 512;
+      rd.off_en = rd.off_es + rd.ne * 32;
+      return rd;
+    };
+    // 16-byte chunk c of token row t, XOR-swizzled for conflict-free ldmatrix
+    auto row_chunk = [](int t, int c) { return (uint32_t)(t * 256 + ((c ^ (t & 7)) << 4)); };
+
+    // ---- copies of round r into buffer r & 1, issued by every warp: warp w
+    // takes items [n w / NW, n (w + 1) / NW) of the round; one cp.async group
+    // per thread and round.  Token rows: lanes 0-15 copy K, 16-31 copy V.
+    auto issue = [&](int r) {
+      const Round rd = round_of(r);
+      uint8_t* buf = sm + (r & 1) * kBufBytes;
+      const int n = rd.ntok + rd.ne;
+      const int j0 = n * warp / NW, j1 = n * (warp + 1) / NW;
+      // tokens of this warp
+      const int t0 = min(j0, rd.ntok), t1 = min(j1, rd.ntok);
+      if (t1 > t0) {
+        int ci = 0;
+        const int first_r = rd.ta + t0 - n_st;  // R index of the first token (if any)
+        if (!exec && rd.ta + t1 > n_st && kr > 0) {
+          const int r0 = max(first_r, 0);
+          int lo = 0, hi = kr - 1;  // last cluster with rpre <= r0
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (rpre_sm[mid] <= r0) lo = mid; else hi = mid - 1;
+          }
+          ci = lo;
         }
-        for (int i = first + threadIdx.x; i < kr && rpre_sm[i] < r1; i += kThreads) {
-          const long long a = max((long long)rpre_sm[i], r0);
-          const long long b = min((long long)rpre_sm[i + 1], r1);
-          const long long row = (long long)rbase_sm[i] + (a - rpre_sm[i]);
-          if (b > a && row >= 0 && row + (b - a) <= lim_rows) {
-            const uint32_t bytes = (uint32_t)((b - a) * kHeadDim * 2);
-            prefetch_l2_bulk(p.Kr + (rbase_rows + (size_t)row) * kHeadDim, bytes);
-            prefetch_l2_bulk(p.Vr + (rbase_rows + (size_t)row) * kHeadDim, bytes);
+        for (int t = t0; t < t1; ++t) {
+          const int it = rd.ta + t;
+          const __nv_bfloat16* src = nullptr;
+          if (it < n_st) {
+            src = (lane < 16 ? p.Ks : p.Vs) + ((size_t)u * n_st + it) * kHeadDim;
+          } else {
+            const int rpos = it - n_st;
+            long long row;
+            if (exec) {
+              row = rpos;
+            } else {
+              while (ci + 1 < kr && rpre_sm[ci + 1] <= rpos) ++ci;
+              row = (long long)rrow_sm[ci] + (rpos - rpre_sm[ci]);
+            }
+            if (row >= 0 && row < lim_rows)
+              src = (lane < 16 ? p.Kr : p.Vr) + ((size_t)u * row_base_stride + row) * kHeadDim;
+          }
+          const int c = lane & 15;
+          uint8_t* dst = buf + (lane < 16 ? 0u : rd.off_v) + row_chunk(t, c);
+          if (src) {
+            cp_async16(dst, src + c * 8);
+          } else {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            if (lane == 0) record_status(p.status, RI_ERR_INVALID_ARG);
           }
         }
       }
-    }
-    for (int e = e0 + threadIdx.x; e < e1; e += kThreads) {
-      const int c = eslice[e - e0];
-      prefetch_l2_bulk(p.vsum + ((size_t)bh * C + c) * kHeadDim, kHeadDim * 4);
-      prefetch_l2_bulk(p.score + ((size_t)bh * C + c) * 8, 32);
-      prefetch_l2(p.counts + (size_t)bh * C + c);
-    }
-  }
-  const int n_tok_chunks = (int)((t1 - t0 + kTokChunk - 1) / kTokChunk);
-  const int n_e_chunks = (e1 - e0 + kEChunk - 1) / kEChunk;
-  const int n_chunks = n_tok_chunks + n_e_chunks;
-  uint8_t* cbuf = sm;                                      // [kChunkBufs][kChunkBytes]
-  int* ecnt = reinterpret_cast<int*>(sm + p.L.ecnt);       // [kChunkBufs][kEChunk]
-
-  // issue the copies of chunk k into buffer k % 3 (4 threads per item)
-  auto issue = [&](int k) {
-    uint8_t* buf = cbuf + (k % kChunkBufs) * kChunkBytes;
-    const int slot = threadIdx.x >> 2, part = threadIdx.x & 3;
-    if (k < n_tok_chunks) {
-      const long long tok = t0 + (long long)k * kTokChunk + slot;
-      if (slot < kTokChunk && tok < t1) {
-        const __nv_bfloat16* kp = nullptr;
-        const __nv_bfloat16* vp = nullptr;
-        if (tok < p.n_steady) {
-          kp = p.Ks + steady_base + (size_t)tok * kHeadDim;
-          vp = p.Vs + steady_base + (size_t)tok * kHeadDim;
-        } else {
-          const int tt = (int)(tok - p.n_steady);
-          long long row;
-          if (p.exec_rows) {
-            row = tt;
-          } else {
-            int lo = 0, hi = kr - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (rpre_sm[mid] <= tt) lo = mid; else hi = mid - 1;
-            }
-            row = (long long)rbase_sm[lo] + (tt - rpre_sm[lo]);
-          }
-          // rows outside the source buffer (an inconsistent index, or an
-          // execution buffer smaller than the selection) are zero, flagged
-          if (row >= 0 && row < lim_rows) {
-            kp = p.Kr + (rbase_rows + (size_t)row) * kHeadDim;
-            vp = p.Vr + (rbase_rows + (size_t)row) * kHeadDim;
-          } else if (part == 0) {
+      // padding rows of the last token tile (zeros: no NaN into the MMA)
+      if (warp == NW - 1)
+        for (int i = lane; i < (rd.npad - rd.ntok) * 32; i += 32) {
+          const int t = rd.ntok + (i >> 5), c = i & 15;
+          *reinterpret_cast<uint4*>(buf + ((i & 16) ? rd.off_v : 0u) + row_chunk(t, c)) =
+              make_uint4(0, 0, 0, 0);
+        }
+      // E clusters of this warp
+      const int e0 = max(j0, rd.ntok) - rd.ntok, e1 = max(j1, rd.ntok) - rd.ntok;
+      for (int eb = e0; eb < e1; eb += 32) {
+        const int ne = min(32, e1 - eb);
+        int idv = -1;
+        if (lane < ne) idv = __ldcg(p.sel + (size_t)u * (p.k_r + p.k_e) + p.k_r + rd.ea + eb + lane);
+        for (int i = 0; i < ne; ++i) {
+          const int c = __shfl_sync(0xffffffffu, idv, i);
+          const int e = eb + i;
+          if (c >= 0 && c < C) {
+            const size_t uc = (size_t)u * C + c;
+            cp_async16(buf + rd.off_ev + e * 512 + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
+            if (lane < 2) cp_async16(buf + rd.off_es + e * 32 + lane * 16, p.score + uc * 8 + lane * 4);
+            if (lane == 2) cp_async4(buf + rd.off_en + e * 4, p.counts + uc);
+          } else if (lane == 0) {
+            *reinterpret_cast<int*>(buf + rd.off_en + e * 4) = 0;
             record_status(p.status, RI_ERR_INVALID_ARG);
           }
         }
-        uint8_t* dst = buf + slot * 512;
-        if (kp) {
-          // parts 0-1: K row halves, parts 2-3: V row halves (128 bytes each)
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(part < 2 ? kp : vp) + (part & 1) * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) cp_async16(dst + part * 128 + c * 16, src + c * 16);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(dst + part * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-        }
       }
-    } else {
-      const int e = e0 + (k - n_tok_chunks) * kEChunk + slot;
-      if (slot < kEChunk && e < e1) {
-        const int c = eslice[e - e0];
-        uint8_t* dst = buf + slot * 544;
-        const uint8_t* vs = reinterpret_cast<const uint8_t*>(p.vsum + ((size_t)bh * C + c) * kHeadDim);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) cp_async16(dst + part * 128 + q * 16, vs + part * 128 + q * 16);
-        if (part == 0) {
-          const uint8_t* sc = reinterpret_cast<const uint8_t*>(p.score + ((size_t)bh * C + c) * 8);
-          cp_async16(dst + 512, sc);
-          cp_async16(dst + 528, sc + 16);
-        } else if (part == 1) {
-          cp_async4(&ecnt[(k % kChunkBufs) * kEChunk + slot], p.counts + (size_t)bh * C + c);
-        }
-      }
-    }
-  };
+      cp_async_commit();
+    };
 
-  for (int k = 0; k < kChunkBufs - 1; ++k) {
-    if (k < n_chunks) issue(k);
-    cp_async_commit();
-  }
-  for (int k = 0; k < n_chunks; ++k) {
-    if (k + kChunkBufs - 1 < n_chunks) issue(k + kChunkBufs - 1);
-    cp_async_commit();
-    cp_async_wait<kChunkBufs - 1>();
-    __syncthreads();
-    const uint8_t* buf = cbuf + (k % kChunkBufs) * kChunkBytes;
-    if (k < n_tok_chunks) {
-      const long long base = t0 + (long long)k * kTokChunk;
-      const int nitems = (int)min((long long)kTokChunk, t1 - base);
-      // every 16-lane group runs the same trip count (the shuffles are warp-wide)
+    // ---- state.  Tokens (tensor cores): O^T[d][g] fragments, lane holds
+    // d = 16 j + gid (+8), g = 2 tig (+1); running max / sum of row g = gid
+    // in log2 units.  E clusters (CUDA cores): lane owns dims 4 lane .. +3.
+    float ot[8][4];
+    float tm = -INFINITY, tl = 0.f;
+    float ea[G][4], em[G], el[G];
 #pragma unroll
-      for (int u = 0; u < kTokChunk / 16; ++u) {
-        const int slot = u * 16 + hw;
-        const bool live = slot < nitems;
-        const uint8_t* row = buf + (live ? slot : 0) * 512;
-        float kf[8], vf[8];
-        bf16x8_to_float(*reinterpret_cast<const uint4*>(row + l16 * 16), kf);
-        bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 256 + l16 * 16), vf);
-        float x[G];
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float a = 0.f;
+      for (int i = 0; i < 4; ++i) ot[j][i] = 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a = fmaf(qv[g][i], kf[i], a);
-          x[g] = a;
-        }
+    for (int g = 0; g < G; ++g) {
+      em[g] = -INFINITY;
+      el[g] = 0.f;
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
+      for (int i = 0; i < 4; ++i) ea[g][i] = 0.f;
+    }
+    constexpr float kScale2 = kScale * 1.4426950408889634f;  // to log2 units
+    constexpr float kLog2e = 1.4426950408889634f;
+    for (int r = 0; r < 2 && r < nrounds; ++r) issue(r);
+    for (int r = 0; r < nrounds; ++r) {
+      const Round rd = round_of(r);
+      const uint8_t* buf = sm + (r & 1) * kBufBytes;
+      if (r + 1 < nrounds) cp_async_wait<1>(); else cp_async_wait<0>();
+      __syncthreads();
+      // token tiles of 16: tile j on warp j % NW
+      const int ntiles = rd.npad >> 4;
+      for (int tj = warp; tj < ntiles; tj += NW) {
+        const uint32_t kbase = smem_u32(buf) + tj * 16 * 256;
+        const uint32_t vbase = smem_u32(buf + rd.off_v) + tj * 16 * 256;
+        // S = Q K^T for tokens 16 tj .. +15: two n-tiles of 8 tokens
+        float sacc[2][4];
 #pragma unroll
-          for (int g = 0; g < G; ++g) x[g] += __shfl_xor_sync(0xffffffffu, x[g], off);
-        if (live) {
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float s = x[g] * kScale;
-            const float mn = fmaxf(m[g], s);
-            const float corr = __expf(m[g] - mn);
-            const float pw = __expf(s - mn);
-            l[g] = l[g] * corr + pw;
+          for (int i = 0; i < 4; ++i) sacc[h][i] = 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[g][i] = fmaf(o[g][i], corr, pw * vf[i]);
-            m[g] = mn;
+        for (int kp = 0; kp < 4; ++kp) {  // dims 32 kp .. 32 kp + 31
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // matrices: (tokens 8h.., dim chunk 4kp + m) for m = 0..3
+            const int tr = h * 8 + (lane & 7), ch = kp * 4 + (lane >> 3);
+            uint32_t b[4];
+            ldmatrix_x4(b, kbase + row_chunk(tr, ch));
+            mma_bf16_16816(sacc[h], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b[0], b[1]);
+            mma_bf16_16816(sacc[h], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b[2], b[3]);
           }
         }
+        // row g = gid: logits of tokens 8h + 2 tig (+1); mask the padding
+        float x[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int t = tj * 16 + h * 8 + tig * 2 + i;
+            x[h * 2 + i] = t < rd.ntok ? sacc[h][i] * kScale2 : -INFINITY;
+          }
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        float corr = 1.f;
+        if (mx > tm + kRescale * kLog2e) {  // new reference (also the first tile)
+          corr = tm == -INFINITY ? 0.f : ex2f(tm - mx);
+          tm = mx;
+          tl *= corr;
+        }
+        // O^T columns g = 2 tig, 2 tig + 1 rescale by the factors of rows g
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+          const float c0 = __shfl_sync(0xffffffffu, corr, (tig * 2) * 4);
+          const float c1 = __shfl_sync(0xffffffffu, corr, (tig * 2 + 1) * 4);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            ot[j][0] *= c0;
+            ot[j][1] *= c1;
+            ot[j][2] *= c0;
+            ot[j][3] *= c1;
+          }
+        }
+        float pv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          pv[i] = ex2f(x[i] - tm);
+          tl += pv[i];
+        }
+        const uint32_t pb0 = pack_bf16x2(pv[0], pv[1]);  // tokens 2 tig, +1
+        const uint32_t pb1 = pack_bf16x2(pv[2], pv[3]);  // tokens 8 + 2 tig, +1
+        // O^T += V^T P^T: 8 dim groups of 16
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          // matrices: (tokens 8 (m >> 1).., dim chunk 2 j + (m & 1)) for m = 0..3
+          const int m4 = lane >> 3;
+          const int tr = (m4 >> 1) * 8 + (lane & 7), ch = j * 2 + (m4 & 1);
+          uint32_t a[4];
+          ldmatrix_x4_trans(a, vbase + row_chunk(tr, ch));
+          mma_bf16_16816(ot[j], a[0], a[1], a[2], a[3], pb0, pb1);
+        }
       }
-    } else {
-      const int base = e0 + (k - n_tok_chunks) * kEChunk;
-      const int nitems = min(kEChunk, e1 - base);
-      for (int slot = hw; slot < nitems; slot += 16) {
-        const int n = ecnt[(k % kChunkBufs) * kEChunk + slot];
+      // E clusters: cluster e on warp e % NW, lane owns dims 4 lane .. 4 lane + 3
+      for (int e = warp; e < rd.ne; e += NW) {
+        const int n = *reinterpret_cast<const int*>(buf + rd.off_en + e * 4);
         if (n <= 0) continue;
-        const uint8_t* row = buf + slot * 544;
-        const float4 v0 = *reinterpret_cast<const float4*>(row + l16 * 32);
-        const float4 v1 = *reinterpret_cast<const float4*>(row + l16 * 32 + 16);
-        const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        const float* sc = reinterpret_cast<const float*>(row + 512);
+        const float4 v = *reinterpret_cast<const float4*>(buf + rd.off_ev + e * 512 + lane * 16);
+        const float* sc = reinterpret_cast<const float*>(buf + rd.off_es + e * 32);
         const float nf = (float)n;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float s = sc[g];
-          const float mn = fmaxf(m[g], s);
-          const float corr = __expf(m[g] - mn);
-          const float pw = __expf(s - mn);
-          l[g] = l[g] * corr + nf * pw;
+          const float sg = sc[g] * kLog2e;
+          if (sg > em[g] + kRescale * kLog2e) {
+            const float c = em[g] == -INFINITY ? 0.f : ex2f(em[g] - sg);
+            el[g] *= c;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[g][i] = fmaf(o[g][i], corr, pw * vv[i]);
-          m[g] = mn;
+            for (int i = 0; i < 4; ++i) ea[g][i] *= c;
+            em[g] = sg;
+          }
+          const float w = ex2f(sg - em[g]);
+          el[g] = fmaf(nf, w, el[g]);
+          ea[g][0] = fmaf(w, v.x, ea[g][0]);
+          ea[g][1] = fmaf(w, v.y, ea[g][1]);
+          ea[g][2] = fmaf(w, v.z, ea[g][2]);
+          ea[g][3] = fmaf(w, v.w, ea[g][3]);
         }
+      }
+      __syncthreads();  // buffer r & 1 is free again
+      if (r + 2 < nrounds) issue(r + 2);
+    }
+    // ---- warp state -> shared memory: per head g the warp's reference
+    // maximum (natural log), denominator and numerator [128]
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(sm);  // [NW][G][128]
+    {
+      tl += __shfl_xor_sync(0xffffffffu, tl, 1);
+      tl += __shfl_xor_sync(0xffffffffu, tl, 2);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mtg = __shfl_sync(0xffffffffu, tm, g * 4);
+        const float ltg = __shfl_sync(0xffffffffu, tl, g * 4);
+        const float mw = fmaxf(mtg, em[g]);
+        const float ft = mtg == -INFINITY ? 0.f : ex2f(mtg - mw);
+        const float fe = em[g] == -INFINITY ? 0.f : ex2f(em[g] - mw);
+        if (lane == 0) {
+          ms->wm[warp][g] = mw == -INFINITY ? -INFINITY : mw * 0.6931471805599453f;
+          ms->wl[warp][g] = ltg * ft + el[g] * fe;
+        }
+        float4* rw = reinterpret_cast<float4*>(red + ((size_t)warp * G + g) * kHeadDim + lane * 4);
+        *rw = make_float4(ea[g][0] * fe, ea[g][1] * fe, ea[g][2] * fe, ea[g][3] * fe);
+      }
+      __syncwarp();
+      // token numerators: lane holds O^T[16 j + gid (+8)][2 tig (+1)]
+      float ftv[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int g = tig * 2 + k;
+        const float mtg = __shfl_sync(0xffffffffu, tm, (g < 8 ? g : 0) * 4);
+        float emg = -INFINITY;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg)
+          if (gg == g) emg = em[gg];
+        const float mw = fmaxf(mtg, emg);
+        ftv[k] = (g < G && mtg != -INFINITY) ? ex2f(mtg - mw) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int g = tig * 2 + k;
+          if (g < G) {
+            float* rg = red + ((size_t)warp * G + g) * kHeadDim + j * 16 + gid;
+            rg[0] += ot[j][k] * ftv[k];
+            rg[8] += ot[j][2 + k] * ftv[k];
+          }
+        }
+    }
+    __syncthreads();
+    float* part = p.part + ((size_t)u * p.S + s) * G * kPartStride;
+    // warp g: the block maximum of head g and the warps' factors (in wm)
+    if (warp < G) {
+      const int g = warp;
+      const float wmv = lane < NW ? ms->wm[lane][g] : -INFINITY;
+      float mb = wmv;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+      const float f = (wmv == -INFINITY) ? 0.f : __expf(wmv - mb);
+      float lw = lane < NW ? f * ms->wl[lane][g] : 0.f;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+      __syncwarp();
+      if (lane < NW) ms->wm[lane][g] = f;
+      if (lane == 0) {
+        part[(size_t)g * kPartStride + 0] = mb;
+        part[(size_t)g * kPartStride + 1] = lw;
       }
     }
     __syncthreads();
-  }
-  cp_async_wait<0>();
-  // merge the two half-warps of each warp (lanes l and l + 16 hold the same dims)
+    for (int idx = threadIdx.x; idx < G * kHeadDim; idx += NT) {
+      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+      float a = 0.f;
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m[g], 16);
-    const float lo2 = __shfl_xor_sync(0xffffffffu, l[g], 16);
-    const float mn = fmaxf(m[g], mo);
-    const float fa = mn == -INFINITY ? 0.f : __expf(m[g] - mn);
-    const float fb = mn == -INFINITY ? 0.f : __expf(mo - mn);
-    l[g] = l[g] * fa + lo2 * fb;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float oo = __shfl_xor_sync(0xffffffffu, o[g][i], 16);
-      o[g][i] = o[g][i] * fa + oo * fb;
+      for (int w = 0; w < NW; ++w) a = fmaf(ms->wm[w][g], red[((size_t)w * G + g) * kHeadDim + d], a);
+      part[(size_t)g * kPartStride + 4 + d] = a;
     }
-    m[g] = mn;
-  }
-  // block merge over the 8 warps, then this block's partial into shared memory
-  float* wst = reinterpret_cast<float*>(sm);  // [8 warps][G][132]
-  float* mypart = reinterpret_cast<float*>(sm + kPartOff);  // [G][132]
-  __syncthreads();
-  if (lane < 16) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float* row = wst + ((size_t)warp * G + g) * kPartStride;
-      if (lane == 0) {
-        row[0] = m[g];
-        row[1] = l[g];
+    // ============================================================ step D
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) ms->flag = atomicAdd(p.ticket + u, 1) == p.S - 1;
+    __syncthreads();
+    if (ms->flag) {
+      // the last slice of unit u merges the S partials (log-sum-exp)
+      __threadfence();
+      const float* pu = p.part + (size_t)u * p.S * G * kPartStride;
+      float* fq = reinterpret_cast<float*>(sm);  // [S][G] maxima, then weights
+      float* lq = fq + p.S * G;                  // [S][G] denominators
+      float* tot = lq + p.S * G;                 // [G] max, [G] denominator
+      for (int i = threadIdx.x; i < p.S * G; i += NT) {
+        fq[i] = __ldcg(pu + (size_t)i * kPartStride);
+        lq[i] = __ldcg(pu + (size_t)i * kPartStride + 1);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) row[4 + l16 * 8 + i] = o[g][i];
-    }
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kThreads) {
-    const int g = idx / kHeadDim, dd = idx % kHeadDim;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, wst[((size_t)w * G + g) * kPartStride]);
-    float ls = 0.f, os = 0.f;
-    if (mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float* row = wst + ((size_t)w * G + g) * kPartStride;
-        const float f = __expf(row[0] - mx);
-        ls += row[1] * f;
-        os += row[4 + dd] * f;
-      }
-    }
-    mypart[(size_t)g * kPartStride + 4 + dd] = os;
-    if (dd == 0) {
-      mypart[(size_t)g * kPartStride + 0] = mx;
-      mypart[(size_t)g * kPartStride + 1] = ls;
-    }
-  }
-  // ============================================================ phase D
-  cluster.sync();  // S6: every block's partial is in its shared memory
-  if (j == 0) {
-    for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kThreads) {
-      const int g = idx / kHeadDim, dd = idx % kHeadDim;
-      float mr[kMaxClusterBlocks], lr[kMaxClusterBlocks], orr[kMaxClusterBlocks];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < kMaxClusterBlocks; ++r) {
-        if (r < p.P) {
-          const float* rp = cluster.map_shared_rank(mypart, r) + (size_t)g * kPartStride;
-          mr[r] = rp[0];
-          lr[r] = rp[1];
-          orr[r] = rp[4 + dd];
-          mx = fmaxf(mx, mr[r]);
+      __syncthreads();
+      if (threadIdx.x < G) {
+        const int g = threadIdx.x;
+        float mx = -INFINITY;
+        for (int q = 0; q < p.S; ++q) mx = fmaxf(mx, fq[q * G + g]);
+        float ls = 0.f;
+        for (int q = 0; q < p.S; ++q) {
+          const float f = (mx == -INFINITY || fq[q * G + g] == -INFINITY)
+                              ? 0.f : __expf(fq[q * G + g] - mx);
+          fq[q * G + g] = f;
+          ls = fmaf(lq[q * G + g], f, ls);
         }
+        tot[g] = mx;
+        tot[G + g] = ls;
       }
-      float ls = 0.f, os = 0.f;
-      if (mx != -INFINITY) {
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < G * kHeadDim; idx += NT) {
+        const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+        float os = 0.f;
+        int q = 0;
+        for (; q + 8 <= p.S; q += 8) {
+          float v[8];
 #pragma unroll
-        for (int r = 0; r < kMaxClusterBlocks; ++r) {
-          if (r < p.P) {
-            const float f = __expf(mr[r] - mx);
-            ls += lr[r] * f;
-            os += orr[r] * f;
-          }
+          for (int k = 0; k < 8; ++k) v[k] = __ldcg(pu + ((size_t)(q + k) * G + g) * kPartStride + 4 + d);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) os = fmaf(fq[(q + k) * G + g], v[k], os);
         }
+        for (; q < p.S; ++q)
+          os = fmaf(fq[q * G + g], __ldcg(pu + ((size_t)q * G + g) * kPartStride + 4 + d), os);
+        const float ls = tot[G + g];
+        // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
+        const bool any = ls > 0.f;
+        const size_t hq = (size_t)u * G + g;
+        p.out[hq * kHeadDim + d] = __float2bfloat16_rn(any ? os / ls : 0.f);
+        if (p.lse && d == 0) p.lse[hq] = any ? tot[g] + logf(ls) : -INFINITY;
       }
-      // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
-      const bool any = ls > 0.f;
-      const size_t hq = (size_t)bh * G + g;
-      p.out[hq * kHeadDim + dd] = __float2bfloat16_rn(any ? os / ls : 0.f);
-      if (p.lse && dd == 0) p.lse[hq] = any ? mx + logf(ls) : -INFINITY;
     }
+    __syncthreads();  // the region is reused by the next pair's copies
   }
-  cluster.sync();  // S7: block 0 is done reading the other blocks' partials
 }
 
 // ------------------------------------------------------------------ host
@@ -1328,79 +1220,55 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// bf16 [rows][128] row-major, boxes of 64 columns x box_rows, 128-byte swizzle
+cudaError_t encode_rows(CUtensorMap* map, const void* base, unsigned long long rows,
+                        unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 template <int G>
 cudaError_t prepare_kernel() {
-  auto kern = fused_decode_kernel<G>;
-  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), 232448);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-}
-
-SmemLayout make_smem_layout(const Geometry& g, int kr, int ke, int P) {
-  SmemLayout s;
-  uint32_t off = kStageBytes;
-  auto take = [&](uint32_t bytes) {
-    const uint32_t o = off;
-    off = (off + bytes + 15u) & ~15u;
-    return o;
-  };
-  s.q = take(2 * kQRows * 128);  // 1024-aligned: right after the 64 KB stage region
-  const int tiles = g.C > 0 ? (g.C + kTileC - 1) / kTileC : 1;
-  const int per = (tiles + P - 1) / P;
-  s.lkeys_cap = per * kTileC;
-  s.lkeys = take((uint32_t)s.lkeys_cap * 4);
-  s.hist = take(kNB * 4);
-  s.gslice = take((kNB / P + 8) * 4);
-  s.cand = take(2 * kBoundaryCap * 8);
-  s.rpre = take((uint32_t)(kr + 4) * 4);
-  s.rbase = take((uint32_t)(kr + 4) * 4);
-  s.rtrip = take((uint32_t)(3 * kr + 4) * 4);
-  s.ecnt = take(kChunkBufs * kEChunk * 4);
-  s.eslice_cap = (ke + P - 1) / P + 1;
-  s.eslice = take((uint32_t)s.eslice_cap * 4);
-  s.misc = take(kMiscBytes);
-  s.total = off + 1024;  // alignment slack of the dynamic shared memory base
-  return s;
+  return set_smem_once(reinterpret_cast<const void*>(decode_kernel<G>), (int)kSmemBytes);
 }
 
 template <int G>
-int active_clusters(int P, uint32_t smem) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)P);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)P;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+int blocks_per_sm() {
   int n = 0;
   if (prepare_kernel<G>() != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, fused_decode_kernel<G>, &cfg) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, Shape<G>::kThreads,
+                                                    kSmemBytes) != cudaSuccess)
     n = 0;
   cudaGetLastError();
   return n;
 }
 
-int active_clusters_g(int G, int P, uint32_t smem) {
+int blocks_per_sm_g(int G) {
   switch (G) {
-    case 1: return active_clusters<1>(P, smem);
-    case 2: return active_clusters<2>(P, smem);
-    case 3: return active_clusters<3>(P, smem);
-    case 4: return active_clusters<4>(P, smem);
-    case 5: return active_clusters<5>(P, smem);
-    case 6: return active_clusters<6>(P, smem);
-    case 7: return active_clusters<7>(P, smem);
-    default: return active_clusters<8>(P, smem);
+    case 1: return blocks_per_sm<1>();
+    case 2: return blocks_per_sm<2>();
+    case 3: return blocks_per_sm<3>();
+    case 4: return blocks_per_sm<4>();
+    case 5: return blocks_per_sm<5>();
+    case 6: return blocks_per_sm<6>();
+    case 7: return blocks_per_sm<7>();
+    default: return blocks_per_sm<8>();
   }
 }
 
 template <int G>
-cudaError_t launch_fused_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
-                           int mode, cudaStream_t s) {
-  FusedParams p;
+cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a, int mode,
+                     cudaStream_t s) {
+  Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.counts = a.counts;
   p.offsets = a.offsets;
@@ -1418,8 +1286,17 @@ cudaError_t launch_fused_g(const Geometry& g, const DecodeLayout& L, const Decod
   p.rkey = reinterpret_cast<float*>(a.ws + L.off_rkey);
   p.sel = reinterpret_cast<int32_t*>(a.ws + L.off_sel);
   p.rpre = reinterpret_cast<int32_t*>(a.ws + L.off_rpre);
+  p.rrow = reinterpret_cast<int32_t*>(a.ws + L.off_rrow);
+  p.part = reinterpret_cast<float*>(a.ws + L.off_part);
   p.status = reinterpret_cast<int*>(a.ws);
-  p.G = G;
+  const long long BH = g.BH();
+  p.done = reinterpret_cast<int*>(a.ws + L.off_ctrl);
+  p.ready = p.done + BH;
+  p.ticket = p.ready + BH;
+  p.kmax = reinterpret_cast<uint32_t*>(p.ticket + BH);
+  p.kmin = p.kmax + BH;
+  p.ninf = reinterpret_cast<int*>(p.kmin + BH);
+  p.BH = (int)BH;
   p.C = g.C;
   p.M = g.M;
   p.n_steady = g.n_steady;
@@ -1427,127 +1304,111 @@ cudaError_t launch_fused_g(const Geometry& g, const DecodeLayout& L, const Decod
   p.k_e = L.k_e;
   p.kr = L.kr;
   p.ke = L.ke;
-  p.P = L.P;
+  p.S = L.S;
   p.exec_rows = exec ? a.exec_rows : 0;
   p.mode = mode;
-  p.L = make_smem_layout(g, L.kr, L.ke, L.P);
 
-  CUtensorMap map;
-  memset(&map, 0, sizeof(map));
-  if (g.C > 0) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)g.BH() * g.C};
-    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kTileC};
-    cuuint32_t estr[2] = {1, 1};
-    if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.centroid), dims,
-           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+  CUtensorMap map_c, map_q;
+  memset(&map_c, 0, sizeof(map_c));
+  memset(&map_q, 0, sizeof(map_q));
+  if (g.C > 0 && mode != kModeAttend) {
+    cudaError_t e = encode_rows(&map_c, a.centroid, (unsigned long long)BH * g.C, kTileC);
+    if (e == cudaSuccess) e = encode_rows(&map_q, a.q, (unsigned long long)BH * G, kQRows);
+    if (e != cudaSuccess) return e;
   }
   cudaError_t e = prepare_kernel<G>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(g.BH() * L.P));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = p.L.total;
+  cfg.gridDim = dim3((unsigned)L.NB);
+  cfg.blockDim = dim3(Shape<G>::kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)L.P;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fused_decode_kernel<G>, map, p);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<G>, map_c, map_q, p);
 }
 
-cudaError_t launch_fused(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a, int mode,
-                         cudaStream_t s) {
+cudaError_t launch_mode(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a, int mode,
+                        cudaStream_t s) {
   switch (g.G) {
-    case 1: return launch_fused_g<1>(g, L, a, mode, s);
-    case 2: return launch_fused_g<2>(g, L, a, mode, s);
-    case 3: return launch_fused_g<3>(g, L, a, mode, s);
-    case 4: return launch_fused_g<4>(g, L, a, mode, s);
-    case 5: return launch_fused_g<5>(g, L, a, mode, s);
-    case 6: return launch_fused_g<6>(g, L, a, mode, s);
-    case 7: return launch_fused_g<7>(g, L, a, mode, s);
-    default: return launch_fused_g<8>(g, L, a, mode, s);
+    case 1: return launch_g<1>(g, L, a, mode, s);
+    case 2: return launch_g<2>(g, L, a, mode, s);
+    case 3: return launch_g<3>(g, L, a, mode, s);
+    case 4: return launch_g<4>(g, L, a, mode, s);
+    case 5: return launch_g<5>(g, L, a, mode, s);
+    case 6: return launch_g<6>(g, L, a, mode, s);
+    case 7: return launch_g<7>(g, L, a, mode, s);
+    default: return launch_g<8>(g, L, a, mode, s);
   }
 }
 
 }  // namespace
 
-// Blocks per unit of the decode kernel (one thread-block cluster, <= 16):
-// the largest P whose clusters all fit on the device at once (one wave),
-// with at least ceil(C / 8192) blocks so a block's keys fit its local mask.
-// Without a device the plan is P = 16 capped by the tiles.
+// Launch shape of the decode kernel: one block per SM (NB), and S slices of
+// the attention work per unit.  S is the smallest count whose makespan
+// (ceil(units x S / NB') slices of 1/S of a unit per block) is within 5 % of
+// the best over S <= 64, with at least ~32 items per slice; NB' leaves the
+// selector blocks free when units <= NB / 2.
 bool decode_plan(const Geometry& g, DecodeLayout* L) {
-  const int tiles = g.C > 0 ? (g.C + kTileC - 1) / kTileC : 1;
-  const int pmin = g.C > 0 ? (g.C + 8191) / 8192 : 1;
-  const int pmax = tiles < kMaxClusterBlocks ? tiles : kMaxClusterBlocks;
-  if (pmin > kMaxClusterBlocks) {
-    set_error("%d clusters per head: more than %d blocks per head needed", g.C,
-              kMaxClusterBlocks);
-    return false;
-  }
+  int nb = 148;
   int dev = -1;
-  const bool have_dev = cudaGetDevice(&dev) == cudaSuccess;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        sms > 0) {
+      static std::mutex mu;
+      static std::map<std::pair<int, int>, int> cache;
+      int per;
+      {
+        std::lock_guard<std::mutex> lk(mu);
+        auto key = std::make_pair(dev, g.G);
+        auto it = cache.find(key);
+        if (it == cache.end()) it = cache.emplace(key, blocks_per_sm_g(g.G)).first;
+        per = it->second;
+      }
+      if (per < 1) {
+        set_error("decode kernel cannot be resident on this device");
+        return false;
+      }
+      nb = sms;  // one block per SM
+    }
+  }
   cudaGetLastError();
   const long long units = g.BH();
-  int chosen = -1, fallback = -1;
-  for (int P = pmax; P >= pmin && P >= 1; --P) {
-    // balance: the same critical path with fewer blocks
-    const int per = (tiles + P - 1) / P;
-    const int Pb = (tiles + per - 1) / per;
-    if (Pb != P) continue;
-    const SmemLayout s = make_smem_layout(g, L->kr, L->ke, P);
-    if (s.total > 232448) continue;
-    if (!have_dev) {
-      chosen = P;
-      break;
-    }
-    static std::mutex mu;
-    static std::map<std::tuple<int, int, int, uint32_t>, int> cache;
-    int n;
-    {
-      std::lock_guard<std::mutex> lk(mu);
-      auto key = std::make_tuple(dev, g.G, P, s.total);
-      auto it = cache.find(key);
-      if (it == cache.end()) it = cache.emplace(key, active_clusters_g(g.G, P, s.total)).first;
-      n = it->second;
-    }
-    if (n <= 0) continue;
-    if (fallback < 0) fallback = P;
-    if (n >= units) {
-      chosen = P;
-      break;
-    }
-  }
-  if (chosen < 0) chosen = fallback;
-  if (chosen < 0) {
-    set_error("no launchable decode configuration (C = %d, k_r = %d, k_e = %d)", g.C, L->kr,
-              L->ke);
-    return false;
-  }
-  L->P = chosen;
+  const double avg_r = g.C > 0 ? (double)L->kr * g.M / g.C : 0.0;
+  const double w_est = g.n_steady + avg_r + L->ke;
+  int s_max = (int)(w_est / 32.0);
+  s_max = s_max < 1 ? 1 : (s_max > 64 ? 64 : s_max);
+  // with few units the selector blocks (the last `units` blocks) take no slices
+  const long long nbp = units <= nb / 2 ? nb - units : nb;
+  auto makespan = [&](int S) {
+    return (double)((units * S + nbp - 1) / nbp) / (double)S;
+  };
+  double best = 1e30;
+  for (int S = 1; S <= s_max; ++S) best = best < makespan(S) ? best : makespan(S);
+  int S = 1;
+  while (S < s_max && makespan(S) > 1.05 * best) ++S;
+  L->NB = nb;
+  L->S = S;
   return true;
 }
 
 cudaError_t launch_select(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s) {
-  return launch_fused(g, L, a, kModeSelect, s);
+  return launch_mode(g, L, a, kModeSelect, s);
 }
 
 cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s) {
-  return launch_fused(g, L, a, kModeAttend, s);
+  return launch_mode(g, L, a, kModeAttend, s);
 }
 
 cudaError_t launch_decode(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s) {
-  return launch_fused(g, L, a, kModeFull, s);
+  return launch_mode(g, L, a, kModeFull, s);
 }
 
 // ------------------------------------------------------------------- self-test
@@ -1560,13 +1421,12 @@ __global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
       record_status(status, RI_ERR_TIMEOUT);
       return;
     }
-    __nanosleep(1000);
   }
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
                                          cudaStream_t s) {
-  wait_timeout_kernel<<<1, 1, 0, s>>>(status, limit_ns);
+  wait_timeout_kernel<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();
 }
 

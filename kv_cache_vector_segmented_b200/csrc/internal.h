@@ -39,10 +39,14 @@ bool make_geometry(const ri_index_config* cfg, Geometry* g);
 struct DecodeLayout {
   int k_r, k_e;     // requested budgets (sizes of the sel regions)
   int kr, ke;       // clamped to C
-  int P;            // blocks per (b, h) unit of the decode kernel
-  // status word [0, 256); rkey fp32 [BH][C], score fp32 [BH][C][8], sel int32
-  // [BH][k_r + k_e], rpre int32 [BH][k_r + 1].
-  size_t header_bytes, off_rkey, off_score, off_sel, off_rpre, total;
+  int NB;           // blocks of the decode kernel (one per SM)
+  int S;            // slices of the attention work per (b, h) unit
+  // status word [0, 256); counters done/ready/ticket/kmax/kmin/ninf [6][BH] (both
+  // cleared by every call: header_bytes); rkey fp32 [BH][C], score fp32
+  // [BH][C][8], sel int32 [BH][k_r + k_e], rpre int32 [BH][k_r + 1], rrow
+  // int32 [BH][max(k_r, 1)], part fp32 [BH][S][G][kPartStride].
+  size_t header_bytes, off_ctrl, off_rkey, off_score, off_sel, off_rpre, off_rrow, off_part,
+      total;
 };
 constexpr int kPartStride = 132;     // m, l, 2 pad, o[128]
 constexpr int kMaxRetrieval = 4096;  // retrieval clusters per unit held on chip
@@ -73,7 +77,7 @@ cudaError_t launch_decode(const Geometry& g, const DecodeLayout& L, const Decode
                           cudaStream_t s);
 cudaError_t launch_select(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
-// Chooses the blocks per unit (cluster size) of the decode kernel.
+// Chooses the launch shape of the decode kernel (blocks, slices per unit).
 bool decode_plan(const Geometry& g, DecodeLayout* L);
 cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);

@@ -301,9 +301,10 @@ def run_ours(args, ws_n, rank, local):
     mean_bytes = float(np.mean(step_bytes))
     gbs_sel = float(np.mean(bytes_sel)) / (ms_sel * 1e-3) / 1e9
     gbs_att = float(np.mean(bytes_att)) / (ms_att * 1e-3) / 1e9
-    # one fused_decode_kernel launch (plus a 256-byte status memset node) per
-    # decode step: the step time is an upper bound on the kernel's duration
-    dominant = ("fused_decode_kernel (S1-S6, one launch per step)",
+    # one decode_kernel launch (cooperative, S1-S6) plus a small memset node
+    # (status word and counters) per decode step: the step time is an upper
+    # bound on the kernel's duration
+    dominant = ("decode_kernel (S1-S6, one cooperative launch per step)",
                 mean_bytes / (ms_per_step * 1e-3) / 1e9, ms_per_step, mean_bytes)
     traffic, sha = _traffic_from_profiles(os.path.join(ROOT, "kv_cache_vector_segmented_b200",
                                                        "csrc", "decode.cu"))

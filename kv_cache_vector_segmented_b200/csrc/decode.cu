@@ -68,7 +68,6 @@ constexpr float kRescale = 8.f;      // online softmax: new reference only when 
 static_assert(kStagesA * kStageBytes <= kRegionBytes, "stages");
 static_assert(16 * 512 + (kRoundItems - 1) * 548 <= (int)kBufBytes &&
                   (kRoundItems + 15) * 512 <= (int)kBufBytes, "round");
-static_assert(kNB * 4 + 2 * kBoundaryCap * 8 <= (int)kRegionBytes, "select");
 
 // Threads per block (registers: up to 128 each).
 template <int G>
@@ -89,7 +88,13 @@ static_assert(kOffMisc % 16 == 0, "misc alignment");
 
 // Selection scratch inside the region (free outside steps A and C).
 constexpr uint32_t kOffHist = 0;
-constexpr uint32_t kOffCand = kOffHist + kNB * 4;
+constexpr uint32_t kOffCand = kOffHist + kNB * 4;                // [2][kBoundaryCap] u64
+constexpr uint32_t kOffSelCnt = kOffCand + 2 * kBoundaryCap * 8;  // int [kRound]
+constexpr uint32_t kOffSelOff = kOffSelCnt + kRound * 4;          // int [kRound]
+constexpr uint32_t kOffSelE = kOffSelOff + kRound * 4;            // int [kRound]
+constexpr uint32_t kOffSelRid = kOffSelE + kRound * 4;            // int [kMaxRetrieval]
+constexpr uint32_t kOffSelRcnt = kOffSelRid + kMaxRetrieval * 4;  // int [kMaxRetrieval]
+static_assert(kOffSelRcnt + kMaxRetrieval * 4 <= kRegionBytes, "selection scratch");
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
 
@@ -120,6 +125,7 @@ struct Params {
   uint32_t* kmin;  // ws [BH] max of the complemented order keys (= min key)
   int* ninf;       // ws [BH] empty clusters (key -inf)
   int BH, C, M, n_steady, k_r, k_e, kr, ke, S, exec_rows, mode;
+  int nbp;         // blocks that take attention slices (the rest are selectors)
 };
 
 struct Misc {
@@ -537,13 +543,21 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
   // taken in rounds of kRound ids; thread t holds ids round_base + kPer t + j
   // in registers (16-byte loads).  The key range comes from step A.
   auto select_unit = [&](int u) {
-    int* hist = reinterpret_cast<int*>(sm + kOffHist);
+    int* hist = reinterpret_cast<int*>(sm + kOffHist);        // [kNB]
     unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kOffCand);
+    int* cnt_sm = reinterpret_cast<int*>(sm + kOffSelCnt);    // [kRound] sizes of the round
+    int* off_sm = reinterpret_cast<int*>(sm + kOffSelOff);    // [kRound] first rows of the round
+    int* ecomp = reinterpret_cast<int*>(sm + kOffSelE);       // [kRound] E ids of the round
+    int* rid_sm = reinterpret_cast<int*>(sm + kOffSelRid);    // [kMaxRetrieval] R ids
+    int* rcnt_sm = reinterpret_cast<int*>(sm + kOffSelRcnt);  // [kMaxRetrieval] R sizes
     const float* rk = p.rkey + (size_t)u * C;
+    const int32_t* cg = p.counts + (size_t)u * C;
+    const int32_t* og = p.offsets + (size_t)u * (C + 1);
     const int rounds = (C + kRound - 1) / kRound;
     const bool vec = (C & 3) == 0;
     float kk[kPer];
-    auto load_round = [&](int rd) {
+    // keys of round rd into registers; sizes and first rows into shared memory
+    auto load_round = [&](int rd, bool with_meta) {
       const int c0 = rd * kRound + threadIdx.x * kPer;
       if (vec && c0 + kPer <= C) {
 #pragma unroll
@@ -554,12 +568,39 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
           kk[i + 2] = v.z;
           kk[i + 3] = v.w;
         }
-      } else {
+        if (with_meta) {
+          // every load issued before the first store (no load waits on a store)
+          int4 cv[kPer / 4];
+          int ov[kPer];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) kk[i] = c0 + i < C ? __ldcg(rk + c0 + i) : 0.f;
+          for (int i = 0; i < kPer / 4; ++i) cv[i] = __ldg(reinterpret_cast<const int4*>(cg + c0) + i);
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) ov[i] = __ldg(og + c0 + i);
+#pragma unroll
+          for (int i = 0; i < kPer / 4; ++i)
+            *reinterpret_cast<int4*>(cnt_sm + threadIdx.x * kPer + 4 * i) = cv[i];
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) off_sm[threadIdx.x * kPer + i] = ov[i];
+        }
+      } else {
+        int cv[kPer], ov[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const bool in = c0 + i < C;
+          kk[i] = in ? __ldcg(rk + c0 + i) : 0.f;
+          cv[i] = (with_meta && in) ? __ldg(cg + c0 + i) : 0;
+          ov[i] = (with_meta && in) ? __ldg(og + c0 + i) : 0;
+        }
+        if (with_meta) {
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) {
+            cnt_sm[threadIdx.x * kPer + i] = cv[i];
+            off_sm[threadIdx.x * kPer + i] = ov[i];
+          }
+        }
       }
     };
-    load_round(0);
+    load_round(0, false);
     for (int i = threadIdx.x; i < kNB; i += NT) hist[i] = 0;
     if (threadIdx.x < 2) ms->ncand[threadIdx.x] = 0;
     const uint32_t kmx = __ldcg(p.kmax + u), kmn = __ldcg(p.kmin + u);
@@ -571,7 +612,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
     __syncthreads();
     // 1) histogram over value buckets (monotone in the key)
     for (int rd = 0; rd < rounds; ++rd) {
-      if (rd > 0) load_round(rd);
+      if (rd > 0) load_round(rd, false);
       const int c0 = rd * kRound + threadIdx.x * kPer;
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
@@ -616,8 +657,9 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
       }
       __syncthreads();
     }
-    // 3) exact order inside each boundary bucket: members of both buckets
-    //    gathered in one pass, ranked by (key desc, id asc)
+    // 3) exact order inside each boundary bucket: the members of both
+    //    buckets are gathered (warp-aggregated slots) and sorted by
+    //    (key desc, id asc): a warp-wide bitonic sort when <= 32, else ranking
     int bk[2];
     bool small[2];
 #pragma unroll
@@ -628,33 +670,66 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
     }
     if (small[0] || small[1]) {
       for (int rd = 0; rd < rounds; ++rd) {
-        if (rounds > 1) load_round(rd);
+        if (rounds > 1) load_round(rd, false);
         const int c0 = rd * kRound + threadIdx.x * kPer;
+        uint32_t cm[2] = {0u, 0u};
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
           const int b = bucket_of(kk[j], lo, scale);
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            if (small[w] && b == bk[w] && c0 + j < C) {
-              const int slot = atomicAdd(&ms->ncand[w], 1);
-              cand[w * kBoundaryCap + slot] = ord64(float_order_key(kk[j]), c0 + j);
-            }
+          for (int w = 0; w < 2; ++w)
+            if (small[w] && b == bk[w] && c0 + j < C) cm[w] |= 1u << j;
+        }
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (!small[w]) continue;
+          const int cnt = __popc(cm[w]);
+          int incl = cnt;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += t;
+          }
+          const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+          int base = 0;
+          if (lane == 0 && wtot > 0) base = atomicAdd(&ms->ncand[w], wtot);
+          base = __shfl_sync(0xffffffffu, base, 0) + incl - cnt;
+          uint32_t m = cm[w];
+          while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            cand[w * kBoundaryCap + base++] = ord64(float_order_key(kk[j]), c0 + j);
           }
         }
       }
       __syncthreads();
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        if (!small[w]) continue;
+      if (warp < 2 && small[warp]) {
+        const int w = warp;
         const int k = (w == 0 ? kr : kr + ke) - ms->above[w];  // 1-based rank in the bucket
         const int n = ms->ncand[w];
-        for (int i = threadIdx.x; i < n; i += NT) {
-          const unsigned long long me = cand[w * kBoundaryCap + i];
-          int rank = 0;
-          for (int t = 0; t < n; ++t) rank += cand[w * kBoundaryCap + t] > me;
-          if (rank == k - 1) {
-            ms->Tu[w] = (uint32_t)(me >> 32);
-            ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(me & 0xFFFFFFFFull));
+        if (n <= 32) {
+          unsigned long long v = lane < n ? cand[w * kBoundaryCap + lane] : 0ull;
+#pragma unroll
+          for (int kb = 2; kb <= 32; kb <<= 1)
+#pragma unroll
+            for (int jb = kb >> 1; jb > 0; jb >>= 1) {
+              const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, jb);
+              const bool keep_max = ((lane & jb) == 0) == ((lane & kb) == 0);
+              v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+            }
+          if (lane == k - 1) {
+            ms->Tu[w] = (uint32_t)(v >> 32);
+            ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+          }
+        } else {
+          for (int i = lane; i < n; i += 32) {
+            const unsigned long long me = cand[w * kBoundaryCap + i];
+            int rank = 0;
+            for (int t = 0; t < n; ++t) rank += cand[w * kBoundaryCap + t] > me;
+            if (rank == k - 1) {
+              ms->Tu[w] = (uint32_t)(me >> 32);
+              ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(me & 0xFFFFFFFFull));
+            }
           }
         }
       }
@@ -672,59 +747,65 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
     }
     __syncthreads();
     const bool selA = bk[0] != -2, selB = bk[1] != -2;
-    const unsigned long long TA = selA ? ord64(ms->Tu[0], ms->Tid[0]) : ~0ull;
-    const unsigned long long TB = selB ? ord64(ms->Tu[1], ms->Tid[1]) : ~0ull;
-    // 4) membership and compaction in id order; R ids go to rrow_sm for now
+    const uint32_t TuA = ms->Tu[0], TuB = ms->Tu[1];
+    const int TidA = ms->Tid[0], TidB = ms->Tid[1];
+    // 4) membership (order key, then id) and compaction in id order: R ids,
+    //    sizes and first rows to shared memory, E ids per round to shared
+    //    memory and then out in coalesced stores
     int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
     int32_t* selu = p.sel_user ? p.sel_user + (size_t)u * (p.k_r + p.k_e) : nullptr;
     int baseR = 0, baseE = 0;
     for (int rd = 0; rd < rounds; ++rd) {
-      if (rounds > 1) load_round(rd);
+      if (rounds > 1) {
+        __syncthreads();  // previous round's E ids are written out
+        load_round(rd, false);
+      }
       const int c0 = rd * kRound + threadIdx.x * kPer;
       uint32_t mR = 0, mE = 0;
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
-        if (c0 + j < C) {
-          const unsigned long long o = ord64(float_order_key(kk[j]), c0 + j);
-          const bool inR = selA && o >= TA;
-          const bool inE = !inR && selB && o >= TB;
-          mR |= (uint32_t)inR << j;
-          mE |= (uint32_t)inE << j;
-        }
+        const uint32_t o = float_order_key(kk[j]);
+        const int c = c0 + j;
+        const bool inR = c < C && selA && (o > TuA || (o == TuA && c <= TidA));
+        const bool inE = c < C && !inR && selB && (o > TuB || (o == TuB && c <= TidB));
+        mR |= (uint32_t)inR << j;
+        mE |= (uint32_t)inE << j;
       }
-      // block exclusive scan of (count R, count E) packed in one int
       int tot;
       const int excl = block_scan<NT>((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
-      int pr = baseR + (excl >> 16), pe = baseE + (excl & 0xFFFF);
+      int pr = baseR + (excl >> 16), pe = excl & 0xFFFF;
       while (mR) {
-        const int c = c0 + __ffs(mR) - 1;
+        const int j = __ffs(mR) - 1;
         mR &= mR - 1;
-        rrow_sm[pr] = c;
-        selg[pr] = c;
-        if (selu) selu[pr] = c;
+        rid_sm[pr] = c0 + j;
         ++pr;
       }
       while (mE) {
-        const int c = c0 + __ffs(mE) - 1;
+        const int j = __ffs(mE) - 1;
         mE &= mE - 1;
-        selg[p.k_r + pe] = c;
-        if (selu) selu[p.k_r + pe] = c;
-        ++pe;
+        ecomp[pe++] = c0 + j;
+      }
+      __syncthreads();
+      const int nE = tot & 0xFFFF;
+      for (int i = threadIdx.x; i < nE; i += NT) {
+        selg[p.k_r + baseE + i] = ecomp[i];
+        if (selu) selu[p.k_r + baseE + i] = ecomp[i];
       }
       baseR += tot >> 16;
-      baseE += tot & 0xFFFF;
+      baseE += nE;
     }
-    for (int i = kr + threadIdx.x; i < p.k_r; i += NT) {
-      selg[i] = -1;
-      if (selu) selu[i] = -1;
+    for (int i = threadIdx.x; i < p.k_r; i += NT) {
+      const int v = i < kr ? rid_sm[i] : -1;
+      selg[i] = v;
+      if (selu) selu[i] = v;
     }
     for (int i = ke + threadIdx.x; i < p.k_e; i += NT) {
       selg[p.k_r + i] = -1;
       if (selu) selu[p.k_r + i] = -1;
     }
-    __syncthreads();
-    // 5) sizes of the R clusters (prefix = execution-buffer rows) and their
-    //    first rows in Kp/Vp; loads issued together, then one block scan
+    // 5) R token prefix (execution-buffer rows) and first rows, id order:
+    //    sizes and first rows of the R clusters gathered (loads issued
+    //    together), then one block scan
     {
       constexpr int kPerR = kMaxRetrieval / NT;
       const int per = (kr + NT - 1) / NT;
@@ -733,42 +814,46 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
 #pragma unroll
       for (int w = 0; w < kPerR; ++w) {
         const int i = i0 + w;
-        const bool in = i < i1;
-        const int c = in ? rrow_sm[i] : 0;
-        cn[w] = in ? __ldg(p.counts + (size_t)u * C + c) : 0;
-        of[w] = in ? __ldg(p.offsets + (size_t)u * (C + 1) + c) : 0;
+        const int c = i < i1 ? rid_sm[i] : 0;
+        cn[w] = i < i1 ? __ldg(cg + c) : 0;
+        of[w] = i < i1 ? __ldg(og + c) : 0;
       }
       int loc = 0;
 #pragma unroll
-      for (int w = 0; w < kPerR; ++w) loc += cn[w];
+      for (int w = 0; w < kPerR; ++w) {
+        const int i = i0 + w;
+        if (i < i1) {
+          rcnt_sm[i] = cn[w];
+          rrow_sm[i] = of[w];
+        }
+        loc += cn[w];
+      }
       int total;
       int run = block_scan<NT>(loc, ms->scan, &total);
       int32_t* rp = p.rpre + (size_t)u * (p.k_r + 1);
       int32_t* rr = p.rrow + (size_t)u * (p.k_r > 0 ? p.k_r : 1);
       int32_t* ru = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
-#pragma unroll
-      for (int w = 0; w < kPerR; ++w) {
-        const int i = i0 + w;
-        if (i < i1) {
-          rp[i] = run;
-          rr[i] = of[w];
-          if (ru) ru[i] = run;
-          run += cn[w];
-        }
+      for (int i = i0; i < i1; ++i) {
+        rp[i] = run;
+        if (ru) ru[i] = run;
+        run += rcnt_sm[i];
       }
+      for (int i = threadIdx.x; i < kr; i += NT) rr[i] = rrow_sm[i];
       for (int i = kr + threadIdx.x; i <= p.k_r; i += NT) {
         rp[i] = total;
         if (ru) ru[i] = total;
       }
     }
-    // 6) publish
-    __threadfence();
+    // 6) publish: one fence after the block barrier covers the block's stores
     __syncthreads();
-    if (threadIdx.x == 0) st_release(p.ready + u, 1);
+    if (threadIdx.x == 0) {
+      __threadfence();
+      st_release(p.ready + u, 1);
+    }
   };
 
-  // Unit u is selected by block NB - 1 - (u mod NB): the blocks at the end
-  // of the grid score the fewest tiles.
+  // Unit u is selected by block NB - 1 - (u mod NB) once its tiles are all
+  // scored (the blocks at the end of the grid score the fewest tiles).
   if (p.mode != kModeAttend && tiles_h > 0) {
     for (int u = (int)gridDim.x - 1 - (int)blockIdx.x; u < p.BH; u += (int)gridDim.x) {
       if (threadIdx.x == 0) {
@@ -790,7 +875,7 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
   const long long lim_rows = exec ? p.exec_rows : p.M;
   const long long row_base_stride = exec ? p.exec_rows : p.M;
   const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
-  for (int pi = blockIdx.x; pi < npairs; pi += gridDim.x) {
+  for (int pi = blockIdx.x; pi < npairs && (int)blockIdx.x < p.nbp; pi += p.nbp) {
     const int u = pi % p.BH, s = pi / p.BH;
     if (p.mode == kModeFull && tiles_h > 0) {
       if (threadIdx.x == 0) {
@@ -1296,6 +1381,7 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   p.kmax = reinterpret_cast<uint32_t*>(p.ticket + BH);
   p.kmin = p.kmax + BH;
   p.ninf = reinterpret_cast<int*>(p.kmin + BH);
+  p.nbp = L.NBP;
   p.BH = (int)BH;
   p.C = g.C;
   p.M = g.M;
@@ -1392,6 +1478,7 @@ bool decode_plan(const Geometry& g, DecodeLayout* L) {
   int S = 1;
   while (S < s_max && makespan(S) > 1.05 * best) ++S;
   L->NB = nb;
+  L->NBP = (int)nbp;
   L->S = S;
   return true;
 }

@@ -40,9 +40,10 @@ struct DecodeLayout {
   int k_r, k_e;     // requested budgets (sizes of the sel regions)
   int kr, ke;       // clamped to C
   int NB;           // blocks of the decode kernel (one per SM)
+  int NBP;          // of which take attention slices (the rest select)
   int S;            // slices of the attention work per (b, h) unit
-  // status word [0, 256); counters done/ready/ticket/kmax/kmin/ninf [6][BH] (both
-  // cleared by every call: header_bytes); rkey fp32 [BH][C], score fp32
+  // status word [0, 256); counters done/ready/ticket/kmax/kmin/ninf [6][BH]
+  // (both cleared by every call: header_bytes); rkey fp32 [BH][C], score fp32
   // [BH][C][8], sel int32 [BH][k_r + k_e], rpre int32 [BH][k_r + 1], rrow
   // int32 [BH][max(k_r, 1)], part fp32 [BH][S][G][kPartStride].
   size_t header_bytes, off_ctrl, off_rkey, off_score, off_sel, off_rpre, off_rrow, off_part,

@@ -432,6 +432,29 @@ def run_reference(args, ws_n, rank):
             "setup_s": time.perf_counter() - t0 - sum(times)}
 
 
+def run_profile_case():
+    """Small case for an ncu capture of the two kernels of the path: one
+    128K-token layer of the benchmark geometry (about 1.1 GB on the device),
+    one index build (10 k-means iterations) and 6 decode calls."""
+    import kv_cache_vector_segmented_b200 as R
+    import oracle as O
+    dev = torch.device("cuda", 0)
+    cfg = R.IndexConfig.make(B, H, G, N, iters=10)
+    kv = S.make_kv(B, H, N, seed=0)
+    m0, M = O.middle_range(N)
+    segs = O.segments(M)
+    ip = S.init_positions([s[1] for s in segs], [s[2] for s in segs], B, H, seed=3)
+    idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
+    q = S.make_queries(kv, G, seed=10).to(dev)
+    dcfg = R.default_budgets(idx.geom.clusters)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, dcfg), dev)
+    for _ in range(6):
+        R.decode(q, idx, dcfg, workspace=ws)
+    torch.cuda.synchronize()
+    assert R.read_device_status(ws) == 0
+    print("profile case done", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,7 +462,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="run only the small case used for ncu captures")
     args = ap.parse_args()
+    if args.ncu_case:
+        run_profile_case()
+        return
     if args.warmup < 3:
         args.warmup = 3
     ws_n, rank, local = _dist()

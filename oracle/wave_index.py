@@ -376,32 +376,43 @@ def decode(q: np.ndarray, index: list[list[dict]], k_r: int, k_e: int) -> dict:
 # --------------------------------------------------------------------------
 class LRUClusterCache:
     """Reference model of the GPU block cache's bookkeeping: a mapping table
-    cluster -> slot and an LRU order [P2 §2.2 "同步访问路径" / "异步更新路径"].
+    cluster -> blocks and an LRU order over clusters [P2 §2.2 "同步访问路径" /
+    "异步更新路径"; P2 §3.1: the cache is made of fixed 2 KB physical blocks,
+    8 rows of 128 bf16 values].
 
-    `access(ids)` looks every requested cluster up (hit or miss), then admits
-    the misses, evicting least recently used clusters that are not requested in
-    this same step; all requested clusters become most recent, in request
-    order.  Capacity is counted in clusters.  Returns (hits, misses) lists."""
+    Capacity is counted in blocks; a cluster occupies `blocks(c)` of them
+    (ceil(rows / 8) in the library; 1 when no sizes are given, so capacity is
+    then counted in clusters).  `access(ids)` looks every requested cluster up
+    (hit or miss), then admits the misses in request order, evicting least
+    recently used clusters that are not requested in this same step until the
+    miss fits; a miss that cannot fit is served without being cached.  All
+    requested resident clusters become most recent, in request order.  A
+    cluster of zero blocks holds no rows: it counts as a hit and is not
+    tracked.  Returns (hits, misses) lists."""
 
-    def __init__(self, capacity: int):
+    def __init__(self, capacity: int, blocks=None):
         self.capacity = capacity
-        self.slot_of: dict[int, int] = {}
+        self.blocks = blocks if blocks is not None else (lambda c: 1)
+        self.slot_of: dict[int, list[int]] = {}
         self.order: list[int] = []          # least recent first
         self.free = list(range(capacity))[::-1]
 
     def access(self, ids) -> tuple[list[int], list[int]]:
         ids = [int(i) for i in ids]
-        hits = [i for i in ids if i in self.slot_of]
-        misses = [i for i in ids if i not in self.slot_of]
+        hits = [i for i in ids if i in self.slot_of or self.blocks(i) == 0]
+        misses = [i for i in ids if i not in self.slot_of and self.blocks(i) > 0]
         req = set(ids)
         for i in misses:
-            if not self.free:
+            need = self.blocks(i)
+            while len(self.free) < need:
                 victim = next((v for v in self.order if v not in req), None)
                 if victim is None:
-                    continue                # cache smaller than one step's set
+                    break                   # every resident cluster is requested
                 self.order.remove(victim)
-                self.free.append(self.slot_of.pop(victim))
-            self.slot_of[i] = self.free.pop()
+                self.free.extend(self.slot_of.pop(victim))
+            if len(self.free) < need:
+                continue                    # served without being cached
+            self.slot_of[i] = [self.free.pop() for _ in range(need)]
             self.order.append(i)
         for i in ids:
             if i in self.slot_of:

@@ -329,6 +329,22 @@ def test_empty_clusters_rank_last():
 
 
 # ---------------------------------------------------------------- LRU model
+def test_lru_model_golden_blocks_sequence():
+    rows = _golden_rows("lru_blocks_sequence.txt")
+    cap = int(rows[0].split()[1])
+    sizes = {int(k): int(v) for k, v in (t.split(":") for t in rows[1].split()[1:])}
+    cache = O.LRUClusterCache(cap, blocks=lambda c: sizes[c])
+    for r in rows[2:]:
+        req, hits, misses, resident = [p.split() for p in r.split("|")]
+        h, m = cache.access([int(x) for x in req])
+        assert h == [int(x) for x in hits if x != "-"]
+        assert m == [int(x) for x in misses if x != "-"]
+        assert sorted(cache.slot_of) == sorted(int(x) for x in resident)
+        used = [b for bl in cache.slot_of.values() for b in bl]
+        assert len(used) == len(set(used)) and len(used) + len(cache.free) == cap
+        assert all(len(cache.slot_of[c]) == sizes[c] for c in cache.slot_of)
+
+
 def test_lru_model_golden_sequence():
     rows = _golden_rows("lru_sequence.txt")
     cap = int(rows[0].split()[1])
@@ -339,4 +355,5 @@ def test_lru_model_golden_sequence():
         assert h == [int(x) for x in hits if x != "-"]
         assert m == [int(x) for x in misses if x != "-"]
         assert sorted(cache.slot_of) == sorted(int(x) for x in resident)
-        assert len(set(cache.slot_of.values())) == len(cache.slot_of)
+        used = [b for bl in cache.slot_of.values() for b in bl]
+        assert len(used) == len(set(used)) == len(cache.slot_of)

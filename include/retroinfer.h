@@ -216,6 +216,104 @@ ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config*
                              const void* exec_V, int32_t exec_rows, void* out, float* lse,
                              void* workspace, size_t workspace_bytes, ri_stream_t stream);
 
+/* ---- Wave buffer: GPU block cache and execution-buffer gather ----------
+ * [P2 §2.2 wave buffer (mapping table, LRU replacement, synchronous access
+ * path); §3.1 cache layout (fixed 2 KB physical blocks: 8 rows x 128 bf16);
+ * §3.2 execution buffer assembly; P4 §2B].  With the full K/V of a layer in
+ * pinned host memory, each decode step (1) selects clusters on the device
+ * (ri_select_clusters), (2) plans on the host which retrieval clusters are
+ * served by the GPU block cache and which come over the host link
+ * (ri_cache_plan), (3) gathers them into the execution buffer and admits the
+ * misses into the cache (ri_gather_blocks, twice: fetch list, then admit
+ * list), and (4) attends over the execution buffer (ri_attend_selected). */
+
+/* One copy of n_rows consecutive K rows and the same V rows of one unit
+ * (unit = b * H_kv + h).  Rows are relative to the unit's block of the
+ * source / destination buffer (see ri_gather_buffers). */
+typedef struct {
+  int32_t unit;
+  int32_t src_kind; /* RI_SRC_HOST, RI_SRC_CACHE or RI_SRC_EXEC */
+  int32_t src_row;
+  int32_t dst_kind; /* RI_DST_EXEC or RI_DST_CACHE */
+  int32_t dst_row;
+  int32_t n_rows;
+} ri_copy_desc;
+enum { RI_SRC_HOST = 0, RI_SRC_CACHE = 1, RI_SRC_EXEC = 2 };
+enum { RI_DST_EXEC = 0, RI_DST_CACHE = 1 };
+
+/* Cache geometry.  Each unit owns a pool of blocks_per_unit blocks of
+ * block_rows rows; a cluster of n rows occupies ceil(n / block_rows) blocks.
+ * Limits: units >= 1, blocks_per_unit >= 1, 1 <= block_rows <= 1024. */
+typedef struct {
+  int32_t units;
+  int32_t blocks_per_unit;
+  int32_t block_rows; /* 8 in the pages' layout */
+} ri_cache_config;
+
+/* Opaque host-side state: per unit the mapping table cluster -> blocks, the
+ * LRU order of clusters and the free blocks.  Created empty; host memory
+ * only (the device pool is caller-owned, see ri_gather_buffers). */
+typedef struct ri_cache ri_cache;
+
+/* Per-call counts from ri_cache_plan (summed over units). */
+typedef struct {
+  int64_t hit_clusters, miss_clusters, uncached_clusters; /* uncached: served, not admitted */
+  int64_t hit_rows, miss_rows;                            /* rows from the cache / the host */
+} ri_cache_stats;
+
+ri_status ri_cache_create(const ri_cache_config* cfg, ri_cache** out);
+void ri_cache_destroy(ri_cache* cache);
+
+/* One step of the synchronous access path, on the host.  For every unit u:
+ * the retrieval clusters are sel_ids[u * sel_stride + i], i < k_retrieval,
+ * up to the first negative entry (id order, as ri_select_clusters writes
+ * them); counts / offsets are the index's [units][C] / [units][C + 1] arrays
+ * copied to the host.  The execution-buffer rows follow the clusters in this
+ * order from row 0 (ri_select_clusters' retr_rows).  Lookup first (hit:
+ * resident; a cluster of 0 rows is a hit and is not cached), then the misses
+ * are admitted in order, evicting least recently used clusters not requested
+ * in this step until the miss fits (else it is served uncached), and every
+ * requested resident cluster becomes most recent in request order.  Writes
+ * the copy plan: `fetch` (cache->exec for hits, host->exec for misses) and
+ * `admit` (exec->cache for admitted misses), each split into copies of at
+ * most 16 rows; *n_fetch / *n_admit get their lengths.  Fails with
+ * RI_ERR_CAPACITY (state unchanged) when a list would exceed its capacity,
+ * RI_ERR_INVALID_ARG for bad pointers, ids or sizes.  Not thread-safe for one
+ * cache. */
+ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_stride,
+                        int32_t k_retrieval, const int32_t* counts, const int32_t* offsets,
+                        int32_t clusters, ri_copy_desc* fetch, int32_t fetch_cap,
+                        int32_t* n_fetch, ri_copy_desc* admit, int32_t admit_cap,
+                        int32_t* n_admit, ri_cache_stats* stats);
+
+/* Buffers of the gather: bf16 [units][rows][128] each, dense.
+ *  host_K, host_V   the index's Kp, Vp in pinned (page-locked) host memory,
+ *                   rows = M; read by the device through unified addressing.
+ *  cache_K, cache_V device pool, rows = pool_rows (= blocks_per_unit *
+ *                   block_rows); may be NULL when no descriptor uses them.
+ *  exec_K, exec_V   device execution buffers, rows = exec_rows. */
+typedef struct {
+  const void* host_K;
+  const void* host_V;
+  void* cache_K;
+  void* cache_V;
+  void* exec_K;
+  void* exec_V;
+  int32_t units;
+  int32_t M;
+  int32_t pool_rows;
+  int32_t exec_rows;
+} ri_gather_buffers;
+
+/* Executes n_desc copies (desc: device array) with 16-byte vector loads and
+ * stores, one warp per copy.  Copies of one call must not overlap in their
+ * destinations or write what another reads (ri_cache_plan's fetch and admit
+ * lists satisfy this when run as two calls, fetch first).  A copy whose rows
+ * fall outside its buffers is skipped and RI_ERR_INVALID_ARG recorded in
+ * the status word of `workspace` (>= 256 device bytes; cleared by the call). */
+ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
+                           int32_t n_desc, void* workspace, ri_stream_t stream);
+
 /* Synchronises `stream` and returns the status word a previous call wrote
  * into `workspace` (RI_OK if no device-side failure was recorded). */
 ri_status ri_read_device_status(const void* workspace, ri_stream_t stream);

@@ -15,7 +15,8 @@ _EXPORTS = (
     "STATUS_CODES", "STATUS_NAMES", "alloc_workspace", "attend_selected", "build_index",
     "build_workspace_bytes", "decode", "decode_workspace_bytes", "default_budgets", "geometry",
     "lib", "read_device_status", "select_clusters", "selftest_wait_timeout", "decode_static",
-    "STATIC_SCRATCH_BYTES")
+    "STATIC_SCRATCH_BYTES", "BlockCache", "CopyDesc", "gather_blocks", "SRC_HOST", "SRC_CACHE",
+    "SRC_EXEC", "DST_EXEC", "DST_CACHE")
 
 __all__ = list(_EXPORTS)
 

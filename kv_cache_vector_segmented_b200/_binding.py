@@ -13,6 +13,8 @@ import dataclasses
 import os
 from typing import Optional
 
+import numpy as np
+
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -105,6 +107,45 @@ lib.ri_read_device_status.restype = ctypes.c_int
 lib.ri_read_device_status.argtypes = [_vp, _vp]
 lib.ri_selftest_wait_timeout.restype = ctypes.c_int
 lib.ri_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
+
+
+class CopyDesc(ctypes.Structure):
+    _fields_ = [("unit", ctypes.c_int32), ("src_kind", ctypes.c_int32),
+                ("src_row", ctypes.c_int32), ("dst_kind", ctypes.c_int32),
+                ("dst_row", ctypes.c_int32), ("n_rows", ctypes.c_int32)]
+
+
+class CacheConfig(ctypes.Structure):
+    _fields_ = [("units", ctypes.c_int32), ("blocks_per_unit", ctypes.c_int32),
+                ("block_rows", ctypes.c_int32)]
+
+
+class CacheStats(ctypes.Structure):
+    _fields_ = [("hit_clusters", ctypes.c_int64), ("miss_clusters", ctypes.c_int64),
+                ("uncached_clusters", ctypes.c_int64), ("hit_rows", ctypes.c_int64),
+                ("miss_rows", ctypes.c_int64)]
+
+
+class GatherBuffers(ctypes.Structure):
+    _fields_ = [("host_K", _vp), ("host_V", _vp), ("cache_K", _vp), ("cache_V", _vp),
+                ("exec_K", _vp), ("exec_V", _vp), ("units", ctypes.c_int32),
+                ("M", ctypes.c_int32), ("pool_rows", ctypes.c_int32),
+                ("exec_rows", ctypes.c_int32)]
+
+
+SRC_HOST, SRC_CACHE, SRC_EXEC = 0, 1, 2
+DST_EXEC, DST_CACHE = 0, 1
+
+lib.ri_cache_create.restype = ctypes.c_int
+lib.ri_cache_create.argtypes = [_P(CacheConfig), _P(_vp)]
+lib.ri_cache_destroy.restype = None
+lib.ri_cache_destroy.argtypes = [_vp]
+lib.ri_cache_plan.restype = ctypes.c_int
+lib.ri_cache_plan.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp,
+                              ctypes.c_int32, _vp, ctypes.c_int32, _P(ctypes.c_int32), _vp,
+                              ctypes.c_int32, _P(ctypes.c_int32), _P(CacheStats)]
+lib.ri_gather_blocks.restype = ctypes.c_int
+lib.ri_gather_blocks.argtypes = [_P(GatherBuffers), _vp, ctypes.c_int32, _vp, _vp]
 
 
 def check(status: int, where: str) -> None:
@@ -372,3 +413,82 @@ def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int) -> None:
     check(lib.ri_selftest_wait_timeout(workspace.data_ptr(), limit_ns,
                                        _stream(workspace.device)),
           "ri_selftest_wait_timeout")
+
+
+class BlockCache:
+    """Host state of the GPU block cache (ri_cache_*): per unit a mapping
+    table cluster -> blocks and an LRU order; the device pool itself is a
+    pair of caller-owned tensors [units][blocks_per_unit * block_rows][128]."""
+
+    def __init__(self, units: int, blocks_per_unit: int, block_rows: int = 8):
+        self.cfg = CacheConfig(units, blocks_per_unit, block_rows)
+        h = _vp()
+        check(lib.ri_cache_create(ctypes.byref(self.cfg), ctypes.byref(h)), "ri_cache_create")
+        self._h = h
+        self._destroy = lib.ri_cache_destroy  # still reachable at interpreter exit
+
+    @property
+    def pool_rows(self) -> int:
+        return self.cfg.blocks_per_unit * self.cfg.block_rows
+
+    def plan(self, sel_ids: np.ndarray, k_retrieval: int, counts: np.ndarray,
+             offsets: np.ndarray):
+        """One step (ri_cache_plan) on host arrays: sel_ids int32 [units][stride]
+        (R first, id order, -1 padded), counts int32 [units][C], offsets int32
+        [units][C + 1].  Returns (fetch int32 [n][6], admit int32 [m][6], stats)."""
+        sel = np.ascontiguousarray(sel_ids, dtype=np.int32).reshape(self.cfg.units, -1)
+        cnt = np.ascontiguousarray(counts, dtype=np.int32).reshape(self.cfg.units, -1)
+        off = np.ascontiguousarray(offsets, dtype=np.int32).reshape(self.cfg.units, -1)
+        C = cnt.shape[1]
+        # copies per requested cluster <= blocks of it, each <= 16 rows
+        req = sel[:, :k_retrieval]
+        n = np.where(req >= 0, np.take_along_axis(cnt, np.clip(req, 0, C - 1), axis=1), 0)
+        n = np.maximum(n, 0)
+        br = self.cfg.block_rows
+        per = (n.astype(np.int64) + br - 1) // br * ((br + 15) // 16) + (n + 15) // 16
+        cap = int(per.sum()) + 1
+        fetch = np.zeros((cap, 6), dtype=np.int32)
+        admit = np.zeros((cap, 6), dtype=np.int32)
+        nf, na = ctypes.c_int32(0), ctypes.c_int32(0)
+        st = CacheStats()
+        check(lib.ri_cache_plan(self._h, sel.ctypes.data, sel.shape[1], k_retrieval,
+                                cnt.ctypes.data, off.ctypes.data, C, fetch.ctypes.data, cap,
+                                ctypes.byref(nf), admit.ctypes.data, cap, ctypes.byref(na),
+                                ctypes.byref(st)),
+              "ri_cache_plan")
+        stats = {f: getattr(st, f) for f, _ in CacheStats._fields_}
+        return fetch[:nf.value].copy(), admit[:na.value].copy(), stats
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+
+def gather_blocks(desc: torch.Tensor, host_K: torch.Tensor, host_V: torch.Tensor,
+                  exec_K: torch.Tensor, exec_V: torch.Tensor, workspace: torch.Tensor,
+                  cache_K: Optional[torch.Tensor] = None,
+                  cache_V: Optional[torch.Tensor] = None) -> None:
+    """ri_gather_blocks: desc int32 [n][6] on the device; host_K/V pinned CPU
+    bf16 [B][H][M][d]; exec_K/V device bf16 [B][H][rows][d]; cache_K/V device
+    bf16 [B][H][pool_rows][d] or None."""
+    dev = exec_K.device
+    B, H, rows, d = exec_K.shape
+    if not (host_K.is_pinned() and host_V.is_pinned()):
+        raise ValueError("host_K and host_V must be pinned")
+    _need(desc, "desc", torch.int32, (desc.shape[0], 6), dev)
+    _need(exec_V, "exec_V", torch.bfloat16, tuple(exec_K.shape), dev)
+    M = host_K.shape[2]
+    pool = 0
+    if cache_K is not None:
+        pool = cache_K.shape[2]
+        _need(cache_K, "cache_K", torch.bfloat16, (B, H, pool, d), dev)
+        _need(cache_V, "cache_V", torch.bfloat16, (B, H, pool, d), dev)
+    bufs = GatherBuffers(host_K.data_ptr(), host_V.data_ptr(), _ptr(cache_K), _ptr(cache_V),
+                         exec_K.data_ptr(), exec_V.data_ptr(), B * H, M, pool, rows)
+    check(lib.ri_gather_blocks(ctypes.byref(bufs), desc.data_ptr(), desc.shape[0],
+                               workspace.data_ptr(), _stream(dev)),
+          "ri_gather_blocks")

@@ -88,6 +88,19 @@ cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const Decode
 constexpr size_t kStaticScratchBytes = RI_STATIC_SCRATCH_BYTES;
 cudaError_t static_decode_scratch(void** addr);
 
+// --------------------------------------------------------------- gather
+struct GatherArgs {
+  const void* host_K;
+  const void* host_V;
+  void* cache_K;
+  void* cache_V;
+  void* exec_K;
+  void* exec_V;
+  int units, M, pool_rows, exec_rows;
+};
+cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_desc, int* status,
+                          cudaStream_t s);
+
 // --------------------------------------------------------------- build
 constexpr int kMaxSegLen = 16384;  // segment tokens (member lists live in shared memory)
 

@@ -1,0 +1,103 @@
+"""The wave buffer's synchronous access path on the GPU: select clusters,
+plan the copies on the host (block cache with LRU), gather the retrieval
+clusters from pinned host memory / the cache pool into the execution buffer,
+admit the misses into the cache, then attend over the execution buffer.
+
+Bars (bit-exact: byte copies): the execution buffer holds exactly the index's
+Kp/Vp rows of the R clusters in id order; attention over it equals the decode
+call that reads Kp/Vp in place, bit for bit (same rows, same kernel path)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def R():
+    if not torch.cuda.is_available():
+        pytest.skip("needs CUDA")
+    import kv_cache_vector_segmented_b200 as R
+    return R
+
+
+@pytest.mark.parametrize("cache_frac", [0.05, 0.5])
+def test_gather_access_path(R, cache_frac):
+    dev = torch.device("cuda:0")
+    B, H, G, N = 1, 2, 4, 40000
+    kv = S.make_kv(B, H, N, seed=31)
+    m0, M = O.middle_range(N)
+    segs = O.segments(M, 8192, 512)
+    ip = S.init_positions([s[1] for s in segs], [s[2] for s in segs], B, H, seed=32)
+    cfg = R.IndexConfig.make(B, H, G, N, iters=4)
+    idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
+    C = idx.geom.clusters
+    dcfg = R.default_budgets(C)
+    k_r = dcfg.k_retrieval
+    hK = idx.Kp.cpu().pin_memory()
+    hV = idx.Vp.cpu().pin_memory()
+    counts = idx.counts.cpu().numpy().reshape(B * H, C)
+    offsets = idx.offsets.cpu().numpy().reshape(B * H, C + 1)
+    br = 8
+    blocks = (counts.astype(np.int64) + br - 1) // br
+    bpu = max(4, int(cache_frac * blocks.sum(axis=1).max()))
+    cache = R.BlockCache(B * H, bpu, br)
+    cK = torch.zeros((B, H, cache.pool_rows, 128), dtype=torch.bfloat16, device=dev)
+    cV = torch.zeros_like(cK)
+    exec_rows = int(np.sort(counts, axis=1)[:, ::-1][:, :k_r].sum(axis=1).max())
+    eK = torch.zeros((B, H, exec_rows, 128), dtype=torch.bfloat16, device=dev)
+    eV = torch.zeros_like(eK)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, dcfg), dev)
+    gws = R.alloc_workspace(256, dev)
+    qs = S.drift_queries(S.make_queries(kv, G, seed=33), 6, seed=34)
+    Kp = idx.Kp.reshape(B * H, M, 128)
+    Vp = idx.Vp.reshape(B * H, M, 128)
+    hits_seen = 0
+    for step, q in enumerate(qs):
+        q = q.contiguous().to(dev)
+        sel, rr = R.select_clusters(q, idx, dcfg, ws)
+        sel_h = sel.cpu().numpy().reshape(B * H, -1)
+        fetch, admit, st = cache.plan(sel_h, k_r, counts, offsets)
+        if step == 0:
+            assert st["hit_clusters"] == int((counts[np.arange(B * H)[:, None],
+                                                     np.maximum(sel_h[:, :k_r], 0)] == 0).sum())
+        hits_seen += st["hit_rows"]
+        for plan in (fetch, admit):  # fetch first, then admission into the pool
+            R.gather_blocks(torch.from_numpy(plan).to(dev), hK, hV, eK, eV, gws, cK, cV)
+        torch.cuda.synchronize()
+        assert R.read_device_status(gws) == 0
+        rr_h = rr.cpu().numpy().reshape(B * H, -1)
+        for u in range(B * H):
+            ids = [int(c) for c in sel_h[u, :k_r] if c >= 0]
+            rows = np.concatenate([np.arange(offsets[u, c], offsets[u, c] + counts[u, c])
+                                   for c in ids]) if ids else np.zeros(0, np.int64)
+            assert len(rows) == rr_h[u, -1]
+            ridx = torch.from_numpy(rows.astype(np.int64)).to(dev)
+            b, h = divmod(u, H)
+            assert torch.equal(eK[b, h, :len(rows)], Kp[u].index_select(0, ridx))
+            assert torch.equal(eV[b, h, :len(rows)], Vp[u].index_select(0, ridx))
+        lse_e = torch.empty((B, H * G), dtype=torch.float32, device=dev)
+        out_e, lse_e = R.attend_selected(q, idx, dcfg, ws, exec_K=eK, exec_V=eV, lse=lse_e)
+        out_d, lse_d, _ = R.decode(q, idx, dcfg)
+        torch.cuda.synchronize()
+        assert torch.equal(out_e, out_d)
+        assert torch.equal(lse_e, lse_d)
+    assert hits_seen > 0  # drifting queries revisit clusters: the cache serves some rows
+    cache.close()
+
+
+def test_gather_rejects_out_of_range_copies(R):
+    dev = torch.device("cuda:0")
+    hK = torch.zeros((1, 1, 32, 128), dtype=torch.bfloat16).pin_memory()
+    hV = torch.zeros_like(hK).pin_memory()
+    eK = torch.zeros((1, 1, 16, 128), dtype=torch.bfloat16, device=dev)
+    eV = torch.zeros_like(eK)
+    gws = R.alloc_workspace(256, dev)
+    # source rows [30, 40) fall outside the 32 host rows: skipped and flagged
+    desc = torch.tensor([[0, R.SRC_HOST, 30, R.DST_EXEC, 0, 10]], dtype=torch.int32, device=dev)
+    R.gather_blocks(desc, hK, hV, eK, eV, gws)
+    torch.cuda.synchronize()
+    assert R.read_device_status(gws) == R.STATUS_CODES["RI_ERR_INVALID_ARG"]

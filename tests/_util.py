@@ -43,6 +43,42 @@ def oracle_index_heads(kv: S.KVHeads, cfg_iters=None, init_pos=None, use_labels=
     return heads
 
 
+def oracle_index_unit(kv: S.KVHeads, b: int, h: int, seg_len=8192, clusters=512):
+    """Oracle index of one (sequence, KV head) from the generator's planted
+    labels (folded into each segment's cluster range)."""
+    N = kv.K.shape[2]
+    Kh = kv.K[b, h].double().numpy()
+    Vh = kv.V[b, h].double().numpy()
+    m0, M = O.middle_range(N)
+    comp = kv.component[b, h, m0:m0 + M].astype(np.int64)
+    lab = np.empty(M, dtype=np.int64)
+    for start, L, Ks in O.segments(M, seg_len, clusters):
+        lab[start:start + L] = comp[start:start + L] % Ks
+    return O.index_from_labels(Kh, Vh, lab, seg_len, clusters)
+
+
+def put_unit(idx, b: int, h: int, o) -> None:
+    """Writes one unit of an oracle index into a device Index."""
+    g = idx.geom
+    if g.middle:
+        idx.Kp[b, h] = torch.from_numpy(o["Kp"]).to(torch.bfloat16)
+        idx.Vp[b, h] = torch.from_numpy(o["Vp"]).to(torch.bfloat16)
+        idx.perm[b, h] = torch.from_numpy(o["perm"].astype(np.int32))
+        idx.centroid[b, h] = torch.from_numpy(o["centroid"]).to(torch.bfloat16)
+        idx.counts[b, h] = torch.from_numpy(o["counts"].astype(np.int32))
+        idx.vsum[b, h] = torch.from_numpy(o["vsum"]).float()
+    idx.offsets[b, h] = torch.from_numpy(o["offsets"].astype(np.int32))
+    idx.Ks[b, h] = torch.from_numpy(o["Ks"]).to(torch.bfloat16)
+    idx.Vs[b, h] = torch.from_numpy(o["Vs"]).to(torch.bfloat16)
+
+
+def consumed_unit(o):
+    """One unit of the oracle index as the device holds it (vsum in fp32)."""
+    o2 = dict(o)
+    o2["vsum"] = o["vsum"].astype(np.float32).astype(np.float64)
+    return o2
+
+
 def to_device_index(R, cfg, heads, device):
     """Device Index holding the oracle's index (bf16 / fp32 / int32 exactly as
     the library stores them)."""

@@ -128,33 +128,6 @@ __device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf
   }
 }
 
-// Ascending 8-slot candidate list; insert returns the value pushed out.
-struct CandList {
-  float a[kCand];
-  int j[kCand];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int i = 0; i < kCand; ++i) {
-      a[i] = FLT_MAX;
-      j[i] = -1;
-    }
-  }
-  __device__ __forceinline__ float insert(float na, int nj) {
-#pragma unroll
-    for (int i = 0; i < kCand; ++i) {
-      if (na < a[i]) {
-        const float tf = a[i];
-        const int ti = j[i];
-        a[i] = na;
-        j[i] = nj;
-        na = tf;
-        nj = ti;
-      }
-    }
-    return na;
-  }
-};
-
 // ------------------------------------------------------------- assignment
 __global__ void __launch_bounds__(kAssignThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tm_keys,
@@ -358,33 +331,81 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       const int t = u.tile * kRows + row;  // token within the segment
       const bool valid = t < u.L;
       const float kn = valid ? knorm[(size_t)u.bh * d.M + u.seg_start + t] : 0.f;
-      const float loose = 2.f * (kn * uE + uC);  // window of the streaming filter
-      CandList cl;
-      cl.init();
-      float dropped = FLT_MAX, thr = FLT_MAX;
+      const float loose = 2.f * (kn * uE + uC);  // window around the row minimum
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
+      // pass 1: a_j = ||mu_j||^2 - 2 k.mu_j; per 32-column chunk its minimum,
+      // over the row the minimum m (four independent min chains)
+      float cm[16];
+      float m = FLT_MAX;
       bool ok = true;
-      for (int h = 0; h < 2; ++h) {
-        if (!mbar_wait(&tfull[h], (uint32_t)(it & 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll 1
-        for (int ch = 0; ch < 8; ++ch) {
+      for (int cp = 0; cp < 8; ++cp) {  // columns 64 cp .. 64 cp + 63 (half cp / 4)
+        if ((cp & 3) == 0) {
+          if (!mbar_wait(&tfull[cp >> 2], (uint32_t)(it & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(taddr + cp * 64, r0);
+        tmem_ld32_nowait(taddr + cp * 64 + 32, r1);
+        tmem_wait_ld();
+        const int jb = cp * 64;
+        float m4[4] = {FLT_MAX, FLT_MAX, FLT_MAX, FLT_MAX};
+        float n4[4] = {FLT_MAX, FLT_MAX, FLT_MAX, FLT_MAX};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          m4[i & 3] = fminf(m4[i & 3], fmaf(-2.f, __uint_as_float(r0[i]), cn[jb + i]));
+          n4[i & 3] = fminf(n4[i & 3], fmaf(-2.f, __uint_as_float(r1[i]), cn[jb + 32 + i]));
+        }
+        cm[2 * cp] = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3]));
+        cm[2 * cp + 1] = fminf(fminf(n4[0], n4[1]), fminf(n4[2], n4[3]));
+        m = fminf(m, fminf(cm[2 * cp], cm[2 * cp + 1]));
+      }
+      // pass 2: the candidates a_j <= m + loose, from the chunks that can hold
+      // one (warp-uniform: the TMEM loads are warp-collective); in id order,
+      // at most kCand kept, the rest counted
+      const float thr = m + loose;
+      int cj[kCand];
+      float ca[kCand];
+      int nc = 0, best = -1;
+      float besta = FLT_MAX;
+#pragma unroll
+      for (int i = 0; i < kCand; ++i) {
+        cj[i] = -1;
+        ca[i] = FLT_MAX;
+      }
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          const bool need = cm[c] <= thr;
+          if (!__any_sync(0xffffffffu, need)) continue;
           float v[32];
-          tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + h * kHalfN + ch * 32, v);
-          const int jb = h * kHalfN + ch * 32;
+          tmem_ld32(taddr + c * 32, v);
+          if (!need) continue;
+          const int jb = c * 32;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float a = fmaf(-2.f, v[i], cn[jb + i]);
             if (a <= thr) {
-              dropped = fminf(dropped, cl.insert(a, jb + i));
-              thr = cl.a[0] + loose;
+              if (a < besta) {
+                besta = a;
+                best = jb + i;
+              }
+#pragma unroll
+              for (int k = 0; k < kCand; ++k)
+                if (k == nc) {
+                  cj[k] = jb + i;
+                  ca[k] = a;
+                }
+              ++nc;
             }
           }
         }
         tc_fence_before();
-        mbar_arrive(&tempty[h]);
+        mbar_arrive(&tempty[0]);
+        mbar_arrive(&tempty[1]);
       }
       if (!ok) {
         record_status(status, RI_ERR_TIMEOUT);
@@ -396,26 +417,26 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         float U = FLT_MAX;
 #pragma unroll
         for (int i = 0; i < kCand; ++i)
-          if (cl.j[i] >= 0) U = fminf(U, cl.a[i] + kn * ce[cl.j[i]] + col_c(cn[cl.j[i]]));
+          if (cj[i] >= 0) U = fminf(U, ca[i] + kn * ce[cj[i]] + col_c(cn[cj[i]]));
         int nsurv = 0;
         uint16_t cands[kCand];
 #pragma unroll
         for (int i = 0; i < kCand; ++i) cands[i] = kCandNone;
 #pragma unroll
         for (int i = 0; i < kCand; ++i) {
-          const bool s = cl.j[i] >= 0 && cl.j[i] < u.Ks &&
-                         cl.a[i] - kn * ce[cl.j[i]] - col_c(cn[cl.j[i]]) <= U;
-          if (s) {
+          const bool sv = cj[i] >= 0 && cj[i] < u.Ks &&
+                          ca[i] - kn * ce[cj[i]] - col_c(cn[cj[i]]) <= U;
+          if (sv) {
 #pragma unroll
             for (int k = 0; k < kCand; ++k)
-              if (k == nsurv) cands[k] = (uint16_t)cl.j[i];
+              if (k == nsurv) cands[k] = (uint16_t)cj[i];
             ++nsurv;
           }
         }
-        // a dropped entry could still be a candidate: decide by a full scan
-        const bool overflow = dropped - 0.5f * loose <= U;
+        // more candidates than slots: decide by a full scan
+        const bool overflow = nc > kCand;
         const int grow = u.bh * d.M + u.seg_start + t;
-        labels[grow] = (cl.j[0] >= 0 && cl.j[0] < u.Ks) ? cl.j[0] : 0;
+        labels[grow] = (best >= 0 && best < u.Ks) ? best : 0;
         if (overflow || nsurv != 1) {
           FixEntry e;
           e.row = grow;

@@ -173,8 +173,8 @@ bool make_build_layout(const Geometry& g, BuildLayout* L) {
   off = align_up(off + BH * g.C * 128 * 4, 1024);
   L->off_mu_bf16 = off;
   off = align_up(off + BH * g.C * 128 * 2, 1024);
-  L->off_colt = off;
-  off = align_up(off + BH * g.S * 1024 * 4, 256);
+  L->off_nsplit = off;
+  off = align_up(off + BH * g.S * 512 * 16 * 2, 1024);
   L->off_ust = off;
   off = align_up(off + BH * g.S * 2 * 4, 256);
   L->off_counts = off;

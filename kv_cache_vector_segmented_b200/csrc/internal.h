@@ -105,12 +105,12 @@ cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_d
 constexpr int kMaxSegLen = 16384;  // segment tokens (member lists live in shared memory)
 
 struct BuildLayout {
-  // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); colt fp32
-  // [BH*S][2][512] (||mu_j||^2, +inf past K_s; error coefficient e_j);
-  // ust fp32 [BH*S][2] (max e_j, max c_j); counts int32 [BH][C]; labels int32
-  // [BH][M]; knorm fp32 [BH][M] (||k||); queue of rows for the exact fix-up
-  // [BH*M] entries.
-  size_t off_mu, off_mu_bf16, off_colt, off_ust, off_counts, off_labels, off_knorm, off_queue,
+  // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); nsplit
+  // [BH*S][512][16] bf16 (-||mu_j||^2 / 2 in three bf16 parts, -inf past K_s;
+  // plain K-major MMA operand layout); ust fp32 [BH*S][2] (max e_j, max c_j);
+  // counts int32 [BH][C]; labels int32 [BH][M]; knorm fp32 [BH][M] (||k||);
+  // queue of rows for the exact fix-up [BH*M] entries.
+  size_t off_mu, off_mu_bf16, off_nsplit, off_ust, off_counts, off_labels, off_knorm, off_queue,
       total;
 };
 size_t build_queue_bytes(long long rows);

@@ -9,17 +9,20 @@
 // + update (segmented sums).
 //
 // Assignment: label = argmin_j ||k - mu_j||^2 = argmin_j (||mu_j||^2 - 2 k.mu_j),
-// ties to the lower j.  tcgen05 MMA computes v_j = k . bf16(mu_j) for 128 keys x
-// 256 centroids per instruction group (keys are exact in bf16; fp32
-// accumulators in TMEM).  a_j = ||mu_j||^2 - 2 v_j then differs from the exact
-// criterion by at most
+// ties to the lower j.  The TMEM accumulator of each (key, centroid) pair
+// starts at h_j = -||mu_j||^2 / 2 (fp32, stored by the epilogue) and tcgen05
+// MMA adds k . bf16(mu_j) for 128 keys x 256 centroids per instruction group
+// (keys are exact in bf16), so w_j = -a_j / 2 and the argmin is the argmax of
+// w.  a_j = -2 w_j (exact scaling) differs from the exact criterion by at most
 //     eps_j(k) = ||k|| e_j + c_j,
 //     e_j = 2 ||mu_j - bf16(mu_j)||  (+ 2^-14 ||mu_j|| for the fp32 accumulation)
 //     c_j = 2^-15 (||mu_j||^2 + 1)   (rounding of ||mu_j||^2 and of a_j)
-// (Cauchy-Schwarz on the rounding residual; n * 2^-23 accumulation bounds with
-// a factor-2 margin).  A centroid can be the exact argmin only if
-// a_j - eps_j <= min_i (a_i + eps_i); when more than one centroid passes, the
-// row is queued and a fix-up kernel decides it exactly in fp32.
+// (Cauchy-Schwarz on the rounding residual; the fp32 accumulation over the
+// eight K=16 steps, start value included, stays below 2^-19 (||mu_j||^2 +
+// ||k|| ||mu_j||), far inside these terms).  A centroid can be the exact
+// argmin only if a_j - eps_j <= min_i (a_i + eps_i); when more than one
+// centroid passes, the row is queued and a fix-up kernel decides it exactly
+// in fp32.
 //
 // Update: mu_j = mean of the members (fp32), an empty cluster keeps mu_j; the
 // members of a cluster are gathered in position order, so sums are
@@ -36,8 +39,10 @@ namespace {
 
 constexpr int kRows = 128;        // keys per tile = MMA M
 constexpr int kHalfN = 256;       // centroids per MMA = MMA N
+constexpr int kQuarterN = 128;    // centroid columns per epilogue warp
 constexpr int kStages = 2;        // key tile ring
-constexpr int kAssignThreads = 192;
+constexpr int kEpiWarps = 16;       // assignment epilogue: 4 lane quadrants x 4 column quarters
+constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
 constexpr int kCand = 8;          // candidate slots per row
 constexpr int kUpdateWarps = 8;
 constexpr int kClustersPerWarp = 4;
@@ -50,12 +55,17 @@ constexpr uint32_t kSmCent = 0;                                // [2 k-halves][5
 constexpr uint32_t kCentHalfK = 512 * 128;                     // 64 KB
 constexpr uint32_t kSmKeys = 2 * kCentHalfK;                   // 128 KB
 constexpr uint32_t kKeyStage = 2 * kRows * 128;                // 32 KB
-constexpr uint32_t kSmCol = kSmKeys + kStages * kKeyStage;     // [2 buf][2][512] fp32
-constexpr uint32_t kColBytes = 2 * 512 * 4;                    // n_j then e_j
-constexpr uint32_t kSmBar = kSmCol + 2 * kColBytes;
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
+constexpr uint32_t kNsTileBytes = 512 * 32;                    // [512][16] bf16, plain K-major
+constexpr uint32_t kSmNs = kSmKeys + kStages * kKeyStage;      // -||mu_j||^2 / 2 in 3 bf16 parts
+constexpr uint32_t kSmOnes = kSmNs + kNsTileBytes;             // [128][16] bf16 (1, 1, 1, 0...)
+constexpr uint32_t kSmBar = kSmOnes + kRows * 32;
+constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1 + 8;
 constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
-constexpr uint32_t kAssignSmem = kSmMisc + 64 + 1024;          // + alignment slack
+// hand-over from column quarters 0-2 to quarter 3 of a TMEM lane quadrant
+constexpr uint32_t kSmXR = (kSmMisc + 64 + 15) / 16 * 16;            // [3][128] f32
+constexpr uint32_t kSmXMask = kSmXR + 3 * kRows * 4;                  // [3][4 chunks][128] u32
+constexpr uint32_t kAssignSmem = kSmXMask + 3 * 4 * kRows * 4 + 1024;  // + alignment
+static_assert(kAssignSmem <= 227 * 1024, "assignment kernel shared memory");
 
 // Queue of rows whose label needs an exact decision.
 struct FixEntry {
@@ -69,13 +79,13 @@ struct UnitInfo {
 
 struct BuildDims {
   int N, M, C, S, seg_len, K_full, L_last, K_last, tiles_full, tiles_last, tiles_bh, m0;
-  long long total_tiles;
+  int total_tiles;
 };
 
-__device__ __forceinline__ UnitInfo tile_info(const BuildDims& d, long long f) {
+__device__ __forceinline__ UnitInfo tile_info(const BuildDims& d, int f) {
   UnitInfo u;
-  u.bh = (int)(f / d.tiles_bh);
-  int rem = (int)(f - (long long)u.bh * d.tiles_bh);
+  u.bh = f / d.tiles_bh;
+  int rem = f - u.bh * d.tiles_bh;
   int s = rem / d.tiles_full;
   if (s >= d.S - 1) s = d.S - 1;
   u.s = s;
@@ -95,12 +105,32 @@ __device__ __forceinline__ void atomic_max_pos(float* addr, float v) {
   atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));  // v >= 0
 }
 
+// Entry of centroid j (K half kc) in a unit's [512][16] bf16 tile of
+// ||mu||^2 terms, stored in the plain K-major layout of the MMA operand:
+// 8-row x 16-byte core matrices, K halves 128 bytes apart, row groups 256.
+__device__ __forceinline__ uint4* ns_entry(uint8_t* tile, int j, int kc) {
+  return reinterpret_cast<uint4*>(tile + (j >> 3) * 256 + kc * 128 + (j & 7) * 16);
+}
+
+// h = -||mu||^2 / 2 as b1 + b2 + b3 (bf16, each the rounded remainder of the
+// previous: the subtractions are exact, |h - b1 - b2 - b3| <= 2^-27 |h|),
+// packed as the first three K entries.
+__device__ __forceinline__ uint4 split3_bf16(float h) {
+  const __nv_bfloat16 b1 = __float2bfloat16_rn(h);
+  const float r1 = h - __bfloat162float(b1);
+  const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(b2);
+  const __nv_bfloat16 b3 = __float2bfloat16_rn(r2);
+  return make_uint4((uint32_t)__bfloat16_as_ushort(b1) | ((uint32_t)__bfloat16_as_ushort(b2) << 16),
+                    (uint32_t)__bfloat16_as_ushort(b3), 0u, 0u);
+}
+
 // Column constants of one centroid from its fp32 row (lane holds 4 dims):
-// n = ||mu||^2, e = error coefficient of the bf16 operand (see file header).
-// Writes the packed bf16 row and the table entries; lane 0 raises the unit's
-// maxima (E, Cmax).
+// the bf16 row (MMA operand), the entry of -||mu||^2 / 2 in the unit's tile,
+// and the unit's maxima of e = error coefficient of the bf16 operand and of
+// c (see file header).
 __device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf_row,
-                                               float* col_n, float* col_e, float* ust_unit,
+                                               uint8_t* ns_tile, int j, float* ust_unit,
                                                int lane, bool write_bf16) {
   const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
   const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
@@ -121,10 +151,11 @@ __device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf
   }
   if (lane == 0) {
     const float e = 2.f * sqrtf(rr) * 1.0001f + 6.1035156e-05f * sqrtf(sq) + 1e-30f;
-    *col_n = sq;
-    *col_e = e;
+    *ns_entry(ns_tile, j, 0) = split3_bf16(-0.5f * sq);
     atomic_max_pos(&ust_unit[0], e);
     atomic_max_pos(&ust_unit[1], col_c(sq));
+  } else if (lane == 1) {
+    *ns_entry(ns_tile, j, 1) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -132,7 +163,7 @@ __device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf
 __global__ void __launch_bounds__(kAssignThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap tm_keys,
                   const __grid_constant__ CUtensorMap tm_cent, BuildDims d,
-                  const float* __restrict__ knorm, const float* __restrict__ colt,
+                  const float* __restrict__ knorm, const uint8_t* __restrict__ nsplit,
                   const float* __restrict__ ust, int32_t* __restrict__ labels,
                   FixEntry* __restrict__ queue, int* __restrict__ queue_count, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -140,42 +171,51 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* cent = sm + kSmCent;
   uint8_t* keys = sm + kSmKeys;
-  float* colsm = reinterpret_cast<float*>(sm + kSmCol);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSmBar);
   uint64_t* full = bars;                       // [kStages] TMA -> MMA
-  uint64_t* empty = bars + kStages;            // [kStages] epilogue -> TMA
-  uint64_t* cent_full = bars + 2 * kStages;    // TMA -> MMA
+  uint64_t* empty = bars + kStages;            // [kStages] MMA -> TMA
+  uint64_t* cent_full = bars + 2 * kStages;    // TMA -> MMA (centroids + ||mu||^2 terms)
   uint64_t* cent_empty = cent_full + 1;        // MMA -> TMA
-  uint64_t* tfull = cent_full + 2;             // [2] MMA -> epilogue
-  uint64_t* tempty = tfull + 2;                // [2] epilogue -> MMA
-  uint64_t* nfull = tempty + 2;                // [2] TMA -> epilogue (column table)
-  uint64_t* nempty = nfull + 2;                // [2] epilogue -> TMA
-  uint64_t* drain = nempty + 2;                // MMA drain
+  uint64_t* tfull = cent_full + 2;             // [2 column halves] MMA -> epilogue
+  uint64_t* tempty = tfull + 2;                // [2 column halves] epilogue -> MMA
+  uint64_t* drain = tempty + 2;                // MMA drain
+  uint64_t* xfull = drain + 1;                 // [4 lane quadrants] quarters 0-2 -> quarter 3
+  uint64_t* xempty = xfull + 4;                // [4 lane quadrants] quarter 3 -> quarters 0-2
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSmMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kSmMisc + 8);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const long long F = d.total_tiles;
-  const long long f_begin = F * blockIdx.x / gridDim.x;
-  const long long f_end = F * (blockIdx.x + 1) / gridDim.x;
+  const int F = d.total_tiles;
+  const int f_begin = (int)((long long)F * blockIdx.x / gridDim.x);
+  const int f_end = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 128);
+      mbar_init(&empty[i], 1);
     }
     mbar_init(cent_full, 1);
     mbar_init(cent_empty, 1);
     for (int h = 0; h < 2; ++h) {
       mbar_init(&tfull[h], 1);
-      mbar_init(&tempty[h], 128);
-      mbar_init(&nfull[h], 1);
-      mbar_init(&nempty[h], 128);
+      mbar_init(&tempty[h], 8 * 32);  // the 8 epilogue warps reading that half
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&xfull[i], 3 * 32);
+      mbar_init(&xempty[i], 32);
+    }
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  if (warp >= 2 && warp < 10) {
+    // the constant A operand of the extra K step: k' = (1, 1, 1, 0, ..., 0)
+    const int e = threadIdx.x - 64;  // 256 threads: (row, K half) pairs
+    const int r = e >> 1, kc = e & 1;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (kc == 0) v = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    *reinterpret_cast<uint4*>(sm + kSmOnes + (r >> 3) * 256 + kc * 128 + (r & 7) * 16) = v;
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -191,47 +231,36 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     // ----------------------------------------------------------- producer
     tma_prefetch_desc(&tm_keys);
     tma_prefetch_desc(&tm_cent);
-    int prev_unit = -1, nunits = 0;
+    int prev_unit = -1;
     uint32_t ce_phase = 0;
-    long long it = 0;
+    int it = 0;
     int issued[kStages] = {0, 0};
-    int cent_loads = 0, col_loads[2] = {0, 0};
-    for (long long f = f_begin; f < f_end; ++f, ++it) {
+    int cent_loads = 0;
+    for (int f = f_begin; f < f_end; ++f, ++it) {
       if (*abort_flag) break;
       const UnitInfo u = tile_info(d, f);
       if (u.unit != prev_unit) {
         if (prev_unit >= 0) {
-          if (!mbar_wait(cent_empty, ce_phase)) {
+          if (!mbar_wait_suspend(cent_empty, ce_phase)) {
             record_status(status, RI_ERR_TIMEOUT);
             *abort_flag = 1;
             break;
           }
           ce_phase ^= 1;
         }
-        mbar_arrive_expect_tx(cent_full, 4 * kHalfN * 128);
+        mbar_arrive_expect_tx(cent_full, 4 * kHalfN * 128 + kNsTileBytes);
         const int crow = u.bh * d.C + u.cbase;
         for (int kh = 0; kh < 2; ++kh)
           for (int h = 0; h < 2; ++h)
             tma_load_2d(cent + kh * kCentHalfK + h * kHalfN * 128, &tm_cent, kh * 64,
                         crow + h * kHalfN, cent_full);
+        bulk_load(sm + kSmNs, nsplit + (size_t)u.unit * kNsTileBytes, kNsTileBytes, cent_full);
         ++cent_loads;
-        const int nb = nunits & 1;
-        if (nunits >= 2) {
-          if (!mbar_wait(&nempty[nb], ((nunits >> 1) - 1) & 1)) {
-            record_status(status, RI_ERR_TIMEOUT);
-            *abort_flag = 1;
-            break;
-          }
-        }
-        mbar_arrive_expect_tx(&nfull[nb], kColBytes);
-        bulk_load(colsm + nb * 1024, colt + (size_t)u.unit * 1024, kColBytes, &nfull[nb]);
-        ++col_loads[nb];
-        ++nunits;
         prev_unit = u.unit;
       }
-      const int stage = (int)(it % kStages);
+      const int stage = it % kStages;
       if (it >= kStages) {
-        if (!mbar_wait(&empty[stage], (uint32_t)(((it / kStages) - 1) & 1))) {
+        if (!mbar_wait_suspend(&empty[stage], (uint32_t)(((it / kStages) - 1) & 1))) {
           record_status(status, RI_ERR_TIMEOUT);
           *abort_flag = 1;
           break;
@@ -246,24 +275,23 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     }
     // wait for every copy this thread started before the block may exit
     for (int st = 0; st < kStages; ++st)
-      if (issued[st]) mbar_wait(&full[st], (uint32_t)((issued[st] - 1) & 1));
-    if (cent_loads) mbar_wait(cent_full, (uint32_t)((cent_loads - 1) & 1));
-    for (int nb = 0; nb < 2; ++nb)
-      if (col_loads[nb]) mbar_wait(&nfull[nb], (uint32_t)((col_loads[nb] - 1) & 1));
+      if (issued[st]) mbar_wait_suspend(&full[st], (uint32_t)((issued[st] - 1) & 1));
+    if (cent_loads) mbar_wait_suspend(cent_full, (uint32_t)((cent_loads - 1) & 1));
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = umma_idesc_bf16_f32(kRows, kHalfN);
     const uint32_t cent_addr = smem_u32(cent);
     const uint32_t keys_addr = smem_u32(keys);
+    const uint64_t ones_desc = umma_desc_kmajor_plain(smem_u32(sm + kSmOnes), 128, 256);
     int prev_unit = -1;
     uint32_t cf_phase = 0;
-    long long it = 0;
-    for (long long f = f_begin; f < f_end; ++f, ++it) {
+    int it = 0;
+    for (int f = f_begin; f < f_end; ++f, ++it) {
       if (*abort_flag) break;
       const UnitInfo u = tile_info(d, f);
       if (u.unit != prev_unit) {
         if (prev_unit >= 0) umma_commit(cent_empty);
-        if (!mbar_wait(cent_full, cf_phase)) {
+        if (!mbar_wait_suspend(cent_full, cf_phase)) {
           record_status(status, RI_ERR_TIMEOUT);
           *abort_flag = 1;
           break;
@@ -271,8 +299,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         cf_phase ^= 1;
         prev_unit = u.unit;
       }
-      const int stage = (int)(it % kStages);
-      if (!mbar_wait(&full[stage], (uint32_t)((it / kStages) & 1))) {
+      const int stage = it % kStages;
+      if (!mbar_wait_suspend(&full[stage], (uint32_t)((it / kStages) & 1))) {
         record_status(status, RI_ERR_TIMEOUT);
         *abort_flag = 1;
         break;
@@ -280,7 +308,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       tc_fence_after();
       bool ok = true;
       for (int h = 0; h < 2; ++h) {
-        if (it > 0 && !mbar_wait(&tempty[h], (uint32_t)((it - 1) & 1))) {
+        // the epilogue has read this half of the previous tile
+        if (it > 0 && !mbar_wait_suspend(&tempty[h], (uint32_t)((it - 1) & 1))) {
           ok = false;
           break;
         }
@@ -293,6 +322,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           const uint64_t bdesc = umma_desc_sw128(cent_addr + coff);
           umma_bf16(tmem + h * kHalfN, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
         }
+        // + 1 * (-||mu_j||^2 / 2) as three bf16 parts
+        const uint64_t ndesc =
+            umma_desc_kmajor_plain(smem_u32(sm + kSmNs) + h * (kHalfN / 8) * 256, 128, 256);
+        umma_bf16(tmem + h * kHalfN, ones_desc, ndesc, idesc, 1u);
         umma_commit(&tfull[h]);
       }
       if (!ok) {
@@ -300,154 +333,154 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         *abort_flag = 1;
         break;
       }
+      umma_commit(&empty[stage]);  // the key stage is free once these MMAs complete
     }
     // every MMA issued by this thread has completed once `drain` flips
     umma_commit(drain);
-    mbar_wait(drain, 0);
+    mbar_wait_suspend(drain, 0);
   } else if (warp >= 2) {
     // ----------------------------------------------------------- epilogue
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;
-    int prev_unit = -1, nunits = 0;
+    // Warp (lane quadrant q, column quarter Qc) reads columns
+    // [128 Qc, 128 Qc + 128) of the 32 TMEM lanes of quadrant q once per
+    // tile.  Per 32-column chunk: its maximum, and the mask of entries within
+    // the window of the running maximum R (w_j >= R - delta; a threshold at
+    // or below the row's final one keeps every candidate).  Masks of chunks
+    // whose maximum ends below R_quarter - delta are dropped: what remains
+    // holds every entry with w_j >= R_quarter - delta, and an entry outside
+    // that window only in a chunk whose own maximum is a second candidate.
+    // Quarters 0-2 hand (R, masks) to quarter 3, which decides the row: a
+    // quarter takes part iff its maximum is within delta of the row maximum
+    // W (then its entries are candidates, or the row has two or more
+    // candidates anyway).
+    const int ew = warp - 2;
+    const int Qc = ew >> 2;  // column quarter; half Qc / 2
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(Qc * kQuarterN);
+    float* xR = reinterpret_cast<float*>(sm + kSmXR);             // [3][128]
+    uint32_t* xm = reinterpret_cast<uint32_t*>(sm + kSmXMask);    // [3][4][128]
+    int prev_unit = -1;
     float uE = 0.f, uC = 0.f;
-    long long it = 0;
-    for (long long f = f_begin; f < f_end; ++f, ++it) {
-      if (*abort_flag) break;
+    int it = 0;
+    for (int f = f_begin; f < f_end; ++f, ++it) {
       const UnitInfo u = tile_info(d, f);
       if (u.unit != prev_unit) {
-        if (prev_unit >= 0) mbar_arrive(&nempty[(nunits - 1) & 1]);
-        if (!mbar_wait(&nfull[nunits & 1], (uint32_t)((nunits >> 1) & 1))) {
-          record_status(status, RI_ERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
+        prev_unit = u.unit;
         uE = ust[2 * u.unit];
         uC = ust[2 * u.unit + 1];
-        ++nunits;
-        prev_unit = u.unit;
       }
-      const float* cn = colsm + ((nunits - 1) & 1) * 1024;  // n_j
-      const float* ce = cn + 512;                             // e_j
       const int t = u.tile * kRows + row;  // token within the segment
       const bool valid = t < u.L;
       const float kn = valid ? knorm[(size_t)u.bh * d.M + u.seg_start + t] : 0.f;
-      const float loose = 2.f * (kn * uE + uC);  // window around the row minimum
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
-      // pass 1: a_j = ||mu_j||^2 - 2 k.mu_j; per 32-column chunk its minimum,
-      // over the row the minimum m (four independent min chains)
-      float cm[16];
-      float m = FLT_MAX;
-      bool ok = true;
-#pragma unroll 1
-      for (int cp = 0; cp < 8; ++cp) {  // columns 64 cp .. 64 cp + 63 (half cp / 4)
-        if ((cp & 3) == 0) {
-          if (!mbar_wait(&tfull[cp >> 2], (uint32_t)(it & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-        uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(taddr + cp * 64, r0);
-        tmem_ld32_nowait(taddr + cp * 64 + 32, r1);
-        tmem_wait_ld();
-        const int jb = cp * 64;
-        float m4[4] = {FLT_MAX, FLT_MAX, FLT_MAX, FLT_MAX};
-        float n4[4] = {FLT_MAX, FLT_MAX, FLT_MAX, FLT_MAX};
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          m4[i & 3] = fminf(m4[i & 3], fmaf(-2.f, __uint_as_float(r0[i]), cn[jb + i]));
-          n4[i & 3] = fminf(n4[i & 3], fmaf(-2.f, __uint_as_float(r1[i]), cn[jb + 32 + i]));
-        }
-        cm[2 * cp] = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3]));
-        cm[2 * cp + 1] = fminf(fminf(n4[0], n4[1]), fminf(n4[2], n4[3]));
-        m = fminf(m, fminf(cm[2 * cp], cm[2 * cp + 1]));
-      }
-      // pass 2: the candidates a_j <= m + loose, from the chunks that can hold
-      // one (warp-uniform: the TMEM loads are warp-collective); in id order,
-      // at most kCand kept, the rest counted
-      const float thr = m + loose;
-      int cj[kCand];
-      float ca[kCand];
-      int nc = 0, best = -1;
-      float besta = FLT_MAX;
-#pragma unroll
-      for (int i = 0; i < kCand; ++i) {
-        cj[i] = -1;
-        ca[i] = FLT_MAX;
-      }
-      if (ok) {
-#pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
-          const bool need = cm[c] <= thr;
-          if (!__any_sync(0xffffffffu, need)) continue;
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-          if (!need) continue;
-          const int jb = c * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = fmaf(-2.f, v[i], cn[jb + i]);
-            if (a <= thr) {
-              if (a < besta) {
-                besta = a;
-                best = jb + i;
-              }
-#pragma unroll
-              for (int k = 0; k < kCand; ++k)
-                if (k == nc) {
-                  cj[k] = jb + i;
-                  ca[k] = a;
-                }
-              ++nc;
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&tempty[0]);
-        mbar_arrive(&tempty[1]);
-      }
-      if (!ok) {
+      if (*abort_flag) break;
+      if (!mbar_wait_suspend(&tfull[Qc >> 1], (uint32_t)(it & 1))) {
         record_status(status, RI_ERR_TIMEOUT);
         *abort_flag = 1;
         break;
       }
-      if (valid) {
-        // exact-argmin candidates: lower bound <= least upper bound
-        float U = FLT_MAX;
+      // half the window a_j <= min a + 2 (||k|| E + C), in units of w = -a / 2
+      const float delta = kn * uE + uC;
+      float cm[4];
+      uint32_t hit[4];
+      float R = -FLT_MAX;
+      tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < kCand; ++i)
-          if (cj[i] >= 0) U = fminf(U, ca[i] + kn * ce[cj[i]] + col_c(cn[cj[i]]));
-        int nsurv = 0;
-        uint16_t cands[kCand];
+      for (int cp = 0; cp < 2; ++cp) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(taddr + cp * 64, r0);
+        tmem_ld32_nowait(taddr + cp * 64 + 32, r1);
+        tmem_wait_ld();
+        // both chunk maxima first (independent chains), one threshold
+        float m4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+        float n4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
-        for (int i = 0; i < kCand; ++i) cands[i] = kCandNone;
+        for (int i = 0; i < 32; i += 2) {
+          const int k = (i >> 1) & 3;
+          m4[k] = fmax3f(m4[k], __uint_as_float(r0[i]), __uint_as_float(r0[i + 1]));
+          n4[k] = fmax3f(n4[k], __uint_as_float(r1[i]), __uint_as_float(r1[i + 1]));
+        }
+        cm[2 * cp] = fmax3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        cm[2 * cp + 1] = fmax3f(n4[0], n4[1], fmaxf(n4[2], n4[3]));
+        R = fmax3f(R, cm[2 * cp], cm[2 * cp + 1]);
+        const float tr = R - delta;
+        uint32_t a4[4] = {0u, 0u, 0u, 0u}, b4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < kCand; ++i) {
-          const bool sv = cj[i] >= 0 && cj[i] < u.Ks &&
-                          ca[i] - kn * ce[cj[i]] - col_c(cn[cj[i]]) <= U;
-          if (sv) {
+        for (int i = 0; i < 32; ++i) {
+          a4[i & 3] |= (__uint_as_float(r0[i]) >= tr ? 1u : 0u) << i;
+          b4[i & 3] |= (__uint_as_float(r1[i]) >= tr ? 1u : 0u) << i;
+        }
+        hit[2 * cp] = (a4[0] | a4[1]) | (a4[2] | a4[3]);
+        hit[2 * cp + 1] = (b4[0] | b4[1]) | (b4[2] | b4[3]);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[Qc >> 1]);  // these columns are free for the next tile
+      const float thr = R - delta;
 #pragma unroll
-            for (int k = 0; k < kCand; ++k)
-              if (k == nsurv) cands[k] = (uint16_t)cj[i];
-            ++nsurv;
+      for (int c = 0; c < 4; ++c)
+        if (cm[c] < thr) hit[c] = 0u;
+      if (Qc < 3) {
+        if (it >= 1 && !mbar_wait_suspend(&xempty[q], (uint32_t)((it - 1) & 1))) {
+          record_status(status, RI_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        xR[Qc * kRows + row] = R;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xm[(Qc * 4 + c) * kRows + row] = hit[c];
+        mbar_arrive(&xfull[q]);
+        continue;
+      }
+      if (!mbar_wait_suspend(&xfull[q], (uint32_t)(it & 1))) {
+        record_status(status, RI_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      float Rq[4];
+      uint32_t mq[16];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        Rq[k] = xR[k * kRows + row];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mq[k * 4 + c] = xm[(k * 4 + c) * kRows + row];
+      }
+      mbar_arrive(&xempty[q]);
+      Rq[3] = R;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) mq[12 + c] = hit[c];
+      if (!valid) continue;
+      const float W = fmaxf(fmaxf(Rq[0], Rq[1]), fmaxf(Rq[2], Rq[3]));
+      int ntot = 0, lab = -1;
+#pragma unroll
+      for (int c = 15; c >= 0; --c) {
+        if (Rq[c >> 2] < W - delta) mq[c] = 0u;  // quarter without candidates
+        ntot += __popc(mq[c]);
+        if (mq[c]) lab = c * 32 + __ffs(mq[c]) - 1;
+      }
+      const int grow = u.bh * d.M + u.seg_start + t;
+      labels[grow] = lab >= 0 ? lab : 0;
+      if (ntot != 1) {
+        // two or more candidates (ids in increasing order): exact fix-up
+        FixEntry e;
+        e.row = grow;
+#pragma unroll
+        for (int i = 0; i < kCand; ++i) e.cand[i] = kCandNone;
+        if (ntot > kCand || ntot == 0) {
+          e.cand[0] = kCandFullScan;
+        } else {
+          int k = 0;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            uint32_t m = mq[c];
+            while (m) {
+              const int b = __ffs(m) - 1;
+              m &= m - 1u;
+              e.cand[k++] = (uint16_t)(c * 32 + b);
+            }
           }
         }
-        // more candidates than slots: decide by a full scan
-        const bool overflow = nc > kCand;
-        const int grow = u.bh * d.M + u.seg_start + t;
-        labels[grow] = (best >= 0 && best < u.Ks) ? best : 0;
-        if (overflow || nsurv != 1) {
-          FixEntry e;
-          e.row = grow;
-#pragma unroll
-          for (int i = 0; i < kCand; ++i) e.cand[i] = cands[i];
-          if (overflow || nsurv == 0) e.cand[0] = kCandFullScan;
-          const int qi = atomicAdd(queue_count, 1);
-          queue[qi] = e;
-        }
+        const int qi = atomicAdd(queue_count, 1);
+        queue[qi] = e;
       }
-      mbar_arrive(&empty[(int)(it % kStages)]);
     }
   }
   __syncwarp();
@@ -527,7 +560,7 @@ __global__ void knorm_kernel(const __nv_bfloat16* __restrict__ K, float* __restr
 __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
                             const int32_t* __restrict__ init_pos, BuildDims d,
                             float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                            float* __restrict__ colt, float* __restrict__ ust, int* status,
+                            uint8_t* __restrict__ nsplit, float* __restrict__ ust, int* status,
                             long long total) {
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -538,12 +571,11 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
   const bool last = s == d.S - 1;
   const int L = last ? d.L_last : d.seg_len;
   const int Ks = last ? d.K_last : d.K_full;
-  float* cn = colt + (size_t)unit * 1024;
+  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
   if (j >= Ks) {
-    if (lane == 0) {
-      cn[j] = INFINITY;
-      cn[512 + j] = 0.f;
-    }
+    // padding column: w_j = -inf, never a candidate
+    if (lane < 2)
+      *ns_entry(ns, j, lane) = lane == 0 ? make_uint4(0xFF80u, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   const int c = s * d.K_full + j;
@@ -564,8 +596,8 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
   const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
   const float4 m = make_float4(a.x, a.y, b.x, b.y);
   *reinterpret_cast<float4*>(mu + ((size_t)bh * d.C + c) * kHeadDim + lane * 4) = m;
-  centroid_stats(m, mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim, &cn[j], &cn[512 + j],
-                 ust + 2 * unit, lane, true);
+  centroid_stats(m, mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim, ns, j, ust + 2 * unit, lane,
+                 true);
 }
 
 // ------------------------------------------------------------- update / finalise
@@ -623,7 +655,7 @@ __device__ int gather_members(const int32_t* __restrict__ lab, int L, int j0, in
 __global__ void __launch_bounds__(kUpdateWarps * 32)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ labels,
                   BuildDims d, float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                  float* __restrict__ colt, float* __restrict__ ust,
+                  uint8_t* __restrict__ nsplit, float* __restrict__ ust,
                   int32_t* __restrict__ counts, int update_mu) {
   extern __shared__ __align__(16) uint8_t smem_u[];
   __shared__ int start[33], wtot[kUpdateWarps];
@@ -641,7 +673,7 @@ __global__ void __launch_bounds__(kUpdateWarps * 32)
   gather_members(labels + (size_t)bh * d.M + seg_start, L, j0, ncl, list, sorted, start, wtot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const __nv_bfloat16* kbase = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
-  float* cn = colt + (size_t)unit * 1024;
+  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
   for (int cc = 0; cc < kClustersPerWarp; ++cc) {
     const int c = warp * kClustersPerWarp + cc;
     if (c >= ncl) break;
@@ -673,12 +705,10 @@ __global__ void __launch_bounds__(kUpdateWarps * 32)
       const float fn = (float)n;
       const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
       *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
-      centroid_stats(m, mu_bf16 + row * kHeadDim, &cn[j], &cn[512 + j], ust + 2 * unit, lane,
-                     true);
+      centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, true);
     } else {
       const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
-      centroid_stats(m, mu_bf16 + row * kHeadDim, &cn[j], &cn[512 + j], ust + 2 * unit, lane,
-                     false);
+      centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, false);
     }
     if (lane == 0) counts[row] = n;
   }
@@ -865,10 +895,14 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   d.N = g.N; d.M = g.M; d.C = g.C; d.S = g.S; d.seg_len = g.seg_len; d.K_full = g.K_full;
   d.L_last = g.L_last; d.K_last = g.K_last; d.tiles_full = g.tiles_full;
   d.tiles_last = g.tiles_last; d.tiles_bh = g.tiles_bh; d.m0 = g.m0;
-  d.total_tiles = BH * g.tiles_bh;
+  if (BH * g.tiles_bh > 0x7fffffffLL) {
+    set_error("too many key tiles (%lld)", BH * g.tiles_bh);
+    return RI_ERR_UNSUPPORTED;
+  }
+  d.total_tiles = (int)(BH * g.tiles_bh);
   float* mu = reinterpret_cast<float*>(ws + L.off_mu);
   __nv_bfloat16* mu_bf16 = reinterpret_cast<__nv_bfloat16*>(ws + L.off_mu_bf16);
-  float* colt = reinterpret_cast<float*>(ws + L.off_colt);
+  uint8_t* nsplit = reinterpret_cast<uint8_t*>(ws + L.off_nsplit);
   float* ust = reinterpret_cast<float*>(ws + L.off_ust);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
   int32_t* labels = reinterpret_cast<int32_t*>(ws + L.off_labels);
@@ -888,7 +922,7 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
   const long long init_total = units * kMaxClustersPerSeg;
   init_kernel<<<(unsigned)((init_total + 7) / 8), 256, 0, st>>>(K, a.init_pos, d, mu, mu_bf16,
-                                                                 colt, ust, status, init_total);
+                                                                 nsplit, ust, status, init_total);
   RI_CUDA_TRY(cudaGetLastError());
 
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
@@ -897,20 +931,20 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(update_kernel), upd_smem_max));
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(finalise_kernel), upd_smem_max));
   const int sms = num_sms();
-  const unsigned grid_assign = (unsigned)(d.total_tiles < (long long)sms ? d.total_tiles : sms);
+  const unsigned grid_assign = (unsigned)(d.total_tiles < sms ? d.total_tiles : sms);
   const dim3 grid_upd((unsigned)units, (unsigned)((g.K_full + kClustersPerBlock - 1) /
                                                   kClustersPerBlock));
   const int rounds = g.iters > 0 ? g.iters : 1;
   for (int t = 0; t < rounds; ++t) {
     RI_CUDA_TRY(cudaMemsetAsync(queue_count, 0, sizeof(int), st));
     assign_kernel<<<grid_assign, kAssignThreads, kAssignSmem, st>>>(
-        tm_keys, tm_cent, d, knorm, colt, ust, labels, queue, queue_count, status);
+        tm_keys, tm_cent, d, knorm, nsplit, ust, labels, queue, queue_count, status);
     RI_CUDA_TRY(cudaGetLastError());
     fixup_kernel<<<(unsigned)(4 * sms), 256, 0, st>>>(K, mu, d, queue, queue_count, labels);
     RI_CUDA_TRY(cudaGetLastError());
     RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
     update_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(
-        K, labels, d, mu, mu_bf16, colt, ust, counts, g.iters > 0 ? 1 : 0);
+        K, labels, d, mu, mu_bf16, nsplit, ust, counts, g.iters > 0 ? 1 : 0);
     RI_CUDA_TRY(cudaGetLastError());
   }
   if (a.out.objective)

@@ -185,6 +185,10 @@ bool make_build_layout(const Geometry& g, BuildLayout* L) {
   off = align_up(off + BH * g.M * 4, 256);
   L->off_queue = off;
   off = align_up(off + build_queue_bytes((long long)BH * g.M), 256);
+  L->off_members = off;
+  off = align_up(off + BH * g.M * 4, 256);
+  L->off_mstart = off;
+  off = align_up(off + BH * g.S * 513 * 4, 256);
   L->total = off;
   return true;
 }

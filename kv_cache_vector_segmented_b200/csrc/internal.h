@@ -102,16 +102,18 @@ cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_d
                           cudaStream_t s);
 
 // --------------------------------------------------------------- build
-constexpr int kMaxSegLen = 16384;  // segment tokens (member lists live in shared memory)
+constexpr int kMaxSegLen = 16384;  // segment tokens (the sort stages labels in shared memory)
 
 struct BuildLayout {
   // mu fp32 [BH][C][d]; mu_bf16 [BH][C][d] (MMA operand); nsplit
   // [BH*S][512][16] bf16 (-||mu_j||^2 / 2 in three bf16 parts, -inf past K_s;
   // plain K-major MMA operand layout); ust fp32 [BH*S][2] (max e_j, max c_j);
   // counts int32 [BH][C]; labels int32 [BH][M]; knorm fp32 [BH][M] (||k||);
-  // queue of rows for the exact fix-up [BH*M] entries.
+  // queue of rows for the exact fix-up [BH*M] entries; members int32 [BH][M]
+  // (positions within the segment, grouped by cluster in position order);
+  // mstart int32 [BH*S][513] (first member of each cluster).
   size_t off_mu, off_mu_bf16, off_nsplit, off_ust, off_counts, off_labels, off_knorm, off_queue,
-      total;
+      off_members, off_mstart, total;
 };
 size_t build_queue_bytes(long long rows);
 bool make_build_layout(const Geometry& g, BuildLayout* L);

@@ -44,9 +44,8 @@ constexpr int kStages = 2;        // key tile ring
 constexpr int kEpiWarps = 16;       // assignment epilogue: 4 lane quadrants x 4 column quarters
 constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
 constexpr int kCand = 8;          // candidate slots per row
-constexpr int kUpdateWarps = 8;
-constexpr int kClustersPerWarp = 4;
-constexpr int kClustersPerBlock = kUpdateWarps * kClustersPerWarp;  // 32
+constexpr int kUpdateWarps = 8;   // update / finalise: one warp per cluster
+constexpr int kSortThreads = 1024;
 constexpr uint16_t kCandNone = 0xFFFF;
 constexpr uint16_t kCandFullScan = 0xFFFE;
 
@@ -601,209 +600,214 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
 }
 
 // ------------------------------------------------------------- update / finalise
-// Members of the block's clusters [j0, j0 + ncl) of one segment, in position
-// order, grouped by cluster: sorted[start[c] .. start[c+1]) are the positions
-// (within the segment) of cluster j0 + c.  Returns the member total.
-// Shared memory: list[L], sorted[L], start[33], wtot[8].
-__device__ int gather_members(const int32_t* __restrict__ lab, int L, int j0, int ncl,
-                              int* list, int* sorted, int* start, int* wtot) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  int run = 0;
-  // 1) compaction of (position, cluster) pairs, position order
-  for (int base = 0; base < L; base += blockDim.x) {
-    const int t = base + threadIdx.x;
-    const int c = t < L ? lab[t] - j0 : -1;
-    const bool mine = c >= 0 && c < ncl;
-    const unsigned m = __ballot_sync(0xffffffffu, mine);
-    if (lane == 0) wtot[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, tot = 0;
-    for (int w = 0; w < kUpdateWarps; ++w) {
-      before += w < warp ? wtot[w] : 0;
-      tot += wtot[w];
-    }
-    if (mine) list[run + before + __popc(m & lt)] = (t << 5) | c;
-    run += tot;
-    __syncthreads();
-  }
-  // 2) per-cluster counts and starts
-  if (threadIdx.x < 33) start[threadIdx.x] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < run; i += blockDim.x) atomicAdd(&start[(list[i] & 31) + 1], 1);
-  __syncthreads();
-  if (threadIdx.x == 0)
-    for (int c = 1; c <= 32; ++c) start[c] += start[c - 1];
-  __syncthreads();
-  // 3) stable grouping: warp w moves the members of clusters 4w..4w+3
-  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
-    const int c = warp * kClustersPerWarp + cc;
-    int pos = start[c];
-    for (int base = 0; base < run; base += 32) {
-      const int i = base + lane;
-      const int e = i < run ? list[i] : -1;
-      const bool mine = e >= 0 && (e & 31) == c;
-      const unsigned m = __ballot_sync(0xffffffffu, mine);
-      if (mine) sorted[pos + __popc(m & lt)] = e >> 5;
-      pos += __popc(m);
-    }
-  }
-  __syncthreads();
-  return run;
-}
-
-__global__ void __launch_bounds__(kUpdateWarps * 32)
-    update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ labels,
-                  BuildDims d, float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                  uint8_t* __restrict__ nsplit, float* __restrict__ ust,
-                  int32_t* __restrict__ counts, int update_mu) {
-  extern __shared__ __align__(16) uint8_t smem_u[];
-  __shared__ int start[33], wtot[kUpdateWarps];
+// Stable counting sort of one segment's positions by label (one block of
+// kSortThreads per unit): members[unit rows] lists the positions of cluster 0,
+// then cluster 1, ..., each cluster's in increasing position; mstart[unit][j]
+// is the first entry of cluster j (mstart[unit][512] = L).  Warp w owns
+// positions [w P, w P + P): per-warp histograms, a column scan over warps,
+// then each warp places its positions in order (ranks among equal labels of
+// one 32-position step by match_any).
+// Shared memory: lab[L] u16, cnt[32][512] i32, tot scan scratch.
+__global__ void __launch_bounds__(kSortThreads)
+    sort_kernel(const int32_t* __restrict__ labels, BuildDims d, int32_t* __restrict__ members,
+                int32_t* __restrict__ mstart) {
+  extern __shared__ __align__(16) uint8_t smem_s[];
+  constexpr int NW = kSortThreads / 32;
+  int* cnt = reinterpret_cast<int*>(smem_s);                                  // [NW][512]
+  int* cstart = cnt + NW * kMaxClustersPerSeg;                                // [513]
+  int* wsum = cstart + kMaxClustersPerSeg + 1;                                // [NW]
+  uint16_t* lab = reinterpret_cast<uint16_t*>(wsum + NW);                     // [L]
   const int unit = blockIdx.x;
   const int bh = unit / d.S, s = unit % d.S;
   const bool last = s == d.S - 1;
   const int L = last ? d.L_last : d.seg_len;
-  const int Ks = last ? d.K_last : d.K_full;
-  const int j0 = blockIdx.y * kClustersPerBlock;
-  if (j0 >= Ks) return;
-  const int ncl = min(kClustersPerBlock, Ks - j0);
-  int* list = reinterpret_cast<int*>(smem_u);
-  int* sorted = list + d.seg_len;
   const int seg_start = s * d.seg_len;
-  gather_members(labels + (size_t)bh * d.M + seg_start, L, j0, ncl, list, sorted, start, wtot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const __nv_bfloat16* kbase = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
-  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
-  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
-    const int c = warp * kClustersPerWarp + cc;
-    if (c >= ncl) break;
-    const int b = start[c], e = start[c + 1];
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = b; i < e; i += 16) {
-      uint2 raw[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u)
-        raw[u] = i + u < e
-                     ? *reinterpret_cast<const uint2*>(kbase + (size_t)sorted[i + u] * kHeadDim)
-                     : make_uint2(0, 0);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (i + u < e) {
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-          const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
-          acc[0] += a.x;
-          acc[1] += a.y;
-          acc[2] += bb.x;
-          acc[3] += bb.y;
-        }
-      }
+  const int32_t* src = labels + (size_t)bh * d.M + seg_start;
+  for (int i = threadIdx.x; i < NW * kMaxClustersPerSeg; i += kSortThreads) cnt[i] = 0;
+  for (int i = threadIdx.x; i < L; i += kSortThreads) lab[i] = (uint16_t)src[i];
+  __syncthreads();
+  const int P = ((L + NW - 1) / NW + 31) & ~31;  // positions per warp, whole steps
+  const int p0 = warp * P, p1 = min(L, p0 + P);
+  int* mycnt = cnt + warp * kMaxClustersPerSeg;
+  for (int p = p0 + lane; p < p1; p += 32) atomicAdd(&mycnt[lab[p]], 1);
+  __syncthreads();
+  // column scan: cnt[w][c] <- first slot of warp w's members of cluster c
+  int run = 0;
+  const int c = threadIdx.x;
+  if (c < kMaxClustersPerSeg) {
+    for (int w = 0; w < NW; ++w) {
+      const int v = cnt[w * kMaxClustersPerSeg + c];
+      cnt[w * kMaxClustersPerSeg + c] = run;
+      run += v;
     }
-    const int j = j0 + c;
-    const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
-    const int n = e - b;
-    if (update_mu && n > 0) {
-      const float fn = (float)n;
-      const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
-      *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
-      centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, true);
-    } else {
-      const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
-      centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, false);
-    }
-    if (lane == 0) counts[row] = n;
   }
+  // exclusive scan of the cluster totals (run) over c: warp sums, then offsets
+  int incl = run;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (c < kMaxClustersPerSeg) {
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const int first = before + incl - run;
+    cstart[c] = first;
+    for (int w = 0; w < NW; ++w) cnt[w * kMaxClustersPerSeg + c] += first;
+  }
+  if (c == 0) cstart[kMaxClustersPerSeg] = L;
+  __syncthreads();
+  // placement in position order
+  int32_t* out = members + (size_t)bh * d.M + seg_start;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    const bool in = p < p1;
+    const int cl = in ? (int)lab[p] : -1 - lane;  // out-of-range lanes match nobody
+    const unsigned grp = __match_any_sync(0xffffffffu, cl);
+    if (in) {
+      const int slot = mycnt[cl] + __popc(grp & lt);
+      out[slot] = p;
+    }
+    __syncwarp();
+    if (in && (grp & lt) == 0) mycnt[cl] += __popc(grp);
+    __syncwarp();
+  }
+  int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+  for (int i = threadIdx.x; i <= kMaxClustersPerSeg; i += kSortThreads) ms[i] = cstart[i];
 }
 
+// One warp per cluster: mu_j = mean of the members (fp32, summed in position
+// order; an empty cluster keeps mu_j), the column constants of the new
+// centroid and the cluster size.
+__global__ void __launch_bounds__(kUpdateWarps * 32)
+    update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ members,
+                  const int32_t* __restrict__ mstart, BuildDims d, float* __restrict__ mu,
+                  __nv_bfloat16* __restrict__ mu_bf16, uint8_t* __restrict__ nsplit,
+                  float* __restrict__ ust, int32_t* __restrict__ counts, int update_mu) {
+  const int unit = blockIdx.x;
+  const int bh = unit / d.S, s = unit % d.S;
+  const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.y * kUpdateWarps + warp;
+  if (j >= Ks) return;
+  const int seg_start = s * d.seg_len;
+  const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+  const int b = ms[j], e = ms[j + 1];
+  const int32_t* mem = members + (size_t)bh * d.M + seg_start;
+  const __nv_bfloat16* kbase = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i = b; i < e; i += 16) {
+    uint2 raw[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      raw[u] = i + u < e ? *reinterpret_cast<const uint2*>(kbase + (size_t)mem[i + u] * kHeadDim)
+                         : make_uint2(0, 0);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (i + u < e) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+        const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
+        acc[0] += a.x;
+        acc[1] += a.y;
+        acc[2] += bb.x;
+        acc[3] += bb.y;
+      }
+    }
+  }
+  const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
+  const int n = e - b;
+  if (update_mu && n > 0) {
+    const float fn = (float)n;
+    const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
+    *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
+    centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, true);
+  } else {
+    const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
+    centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, false);
+  }
+  if (lane == 0) counts[row] = n;
+}
+
+// Cluster-contiguous layout of the final labels (members / mstart from the
+// last sort): one warp per cluster copies its members' K and V rows in
+// (cluster, position) order, with the permutation, offsets, sizes, value
+// sums, the bf16 centroid and the members' squared distances.
 __global__ void __launch_bounds__(kUpdateWarps * 32)
     finalise_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
-                    const int32_t* __restrict__ labels, BuildDims d, const float* __restrict__ mu,
-                    ri_index out) {
-  extern __shared__ __align__(16) uint8_t smem_u[];
-  __shared__ int start[33], wtot[kUpdateWarps], before_sm;
+                    const int32_t* __restrict__ labels, const int32_t* __restrict__ members,
+                    const int32_t* __restrict__ mstart, BuildDims d,
+                    const float* __restrict__ mu, ri_index out) {
   const int unit = blockIdx.x;
   const int bh = unit / d.S, s = unit % d.S;
   const bool last = s == d.S - 1;
   const int L = last ? d.L_last : d.seg_len;
   const int Ks = last ? d.K_last : d.K_full;
-  const int j0 = blockIdx.y * kClustersPerBlock;
-  if (j0 >= Ks) return;
-  const int ncl = min(kClustersPerBlock, Ks - j0);
-  int* list = reinterpret_cast<int*>(smem_u);
-  int* sorted = list + d.seg_len;
   const int seg_start = s * d.seg_len;
-  const int cbase = s * d.K_full;
-  const int32_t* lab = labels + (size_t)bh * d.M + seg_start;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (out.labels && blockIdx.y == 0)
     for (int t = threadIdx.x; t < L; t += blockDim.x)
-      out.labels[(size_t)bh * d.M + seg_start + t] = lab[t];
-  if (blockIdx.y == 0 && s == d.S - 1 && threadIdx.x == 0)
+      out.labels[(size_t)bh * d.M + seg_start + t] = labels[(size_t)bh * d.M + seg_start + t];
+  if (blockIdx.y == 0 && last && threadIdx.x == 0)
     out.offsets[(size_t)bh * (d.C + 1) + d.C] = d.M;
-  // rows of the segment taken by clusters before j0: tokens with label < j0
-  if (threadIdx.x == 0) before_sm = 0;
-  __syncthreads();
-  {
-    int cnt = 0;
-    for (int t = threadIdx.x; t < L; t += blockDim.x) cnt += lab[t] < j0;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if ((threadIdx.x & 31) == 0) atomicAdd(&before_sm, cnt);
-  }
-  gather_members(lab, L, j0, ncl, list, sorted, start, wtot);
-  const int before = before_sm;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.y * kUpdateWarps + warp;
+  if (j >= Ks) return;
+  const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+  const int b = ms[j], e = ms[j + 1];
+  const int32_t* mem = members + (size_t)bh * d.M + seg_start;
   const size_t bhN = (size_t)bh * d.N + d.m0 + seg_start;
   const size_t bhM = (size_t)bh * d.M + seg_start;
+  const size_t crow = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+  const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
+  float vs[4] = {0.f, 0.f, 0.f, 0.f};
   float obj = 0.f;
-  for (int cc = 0; cc < kClustersPerWarp; ++cc) {
-    const int c = warp * kClustersPerWarp + cc;
-    if (c >= ncl) break;
-    const int b = start[c], e = start[c + 1];
-    const size_t crow = (size_t)bh * d.C + cbase + j0 + c;
-    const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
-    float vs[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = b; i < e; i += 8) {
-      uint2 kr[8], vr[8];
+  for (int i = b; i < e; i += 8) {
+    uint2 kr[8], vr[8];
+    int pos[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool in = i + u < e;
-        const size_t src = (bhN + (in ? sorted[i + u] : 0)) * kHeadDim + lane * 4;
-        kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
-        vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const bool in = i + u < e;
+      pos[u] = in ? mem[i + u] : 0;
+      const size_t src = (bhN + pos[u]) * kHeadDim + lane * 4;
+      kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
+      vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (i + u < e) {
-          const int r = before + i + u;  // rows are in (cluster, position) order
-          const size_t dst = (bhM + r) * kHeadDim + lane * 4;
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
-          if (lane == 0) out.perm[bhM + r] = d.m0 + seg_start + sorted[i + u];
-          const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
-          const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
-          const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
-          const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
-          vs[0] += va.x;
-          vs[1] += va.y;
-          vs[2] += vb.x;
-          vs[3] += vb.y;
-          const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
-          obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
-        }
+    for (int u = 0; u < 8; ++u) {
+      if (i + u < e) {
+        const size_t dst = (bhM + i + u) * kHeadDim + lane * 4;  // rows in (cluster, position) order
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
+        if (lane == 0) out.perm[bhM + i + u] = d.m0 + seg_start + pos[u];
+        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
+        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+        const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
+        const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
+        vs[0] += va.x;
+        vs[1] += va.y;
+        vs[2] += vb.x;
+        vs[3] += vb.y;
+        const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
+        obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
       }
     }
-    *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
-        make_float4(vs[0], vs[1], vs[2], vs[3]);
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
-    uint2 packed;
-    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + crow * kHeadDim +
-                              lane * 4) = packed;
-    if (lane == 0) {
-      out.counts[crow] = e - b;
-      out.offsets[(size_t)bh * (d.C + 1) + cbase + j0 + c] = seg_start + before + b;
-    }
+  }
+  *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
+      make_float4(vs[0], vs[1], vs[2], vs[3]);
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+  packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + crow * kHeadDim +
+                            lane * 4) = packed;
+  if (lane == 0) {
+    out.counts[crow] = e - b;
+    out.offsets[(size_t)bh * (d.C + 1) + (size_t)s * d.K_full + j] = seg_start + b;
   }
   if (out.objective) {
 #pragma unroll
@@ -908,6 +912,8 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   int32_t* labels = reinterpret_cast<int32_t*>(ws + L.off_labels);
   float* knorm = reinterpret_cast<float*>(ws + L.off_knorm);
   FixEntry* queue = reinterpret_cast<FixEntry*>(ws + L.off_queue);
+  int32_t* members = reinterpret_cast<int32_t*>(ws + L.off_members);
+  int32_t* mstart = reinterpret_cast<int32_t*>(ws + L.off_mstart);
   const long long units = BH * g.S;
 
   CUtensorMap tm_keys, tm_cent;
@@ -926,14 +932,16 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   RI_CUDA_TRY(cudaGetLastError());
 
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
-  const size_t upd_smem = (size_t)g.seg_len * 2 * sizeof(int);
-  const int upd_smem_max = (int)(kMaxSegLen * 2 * sizeof(int));
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(update_kernel), upd_smem_max));
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(finalise_kernel), upd_smem_max));
+  auto sort_smem = [](int L) {
+    constexpr int NW = kSortThreads / 32;
+    return (size_t)(NW * kMaxClustersPerSeg + kMaxClustersPerSeg + 1 + NW) * sizeof(int) +
+           (size_t)L * sizeof(uint16_t);
+  };
+  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(sort_kernel),
+                            (int)sort_smem(kMaxSegLen)));
   const int sms = num_sms();
   const unsigned grid_assign = (unsigned)(d.total_tiles < sms ? d.total_tiles : sms);
-  const dim3 grid_upd((unsigned)units, (unsigned)((g.K_full + kClustersPerBlock - 1) /
-                                                  kClustersPerBlock));
+  const dim3 grid_upd((unsigned)units, (unsigned)(kMaxClustersPerSeg / kUpdateWarps));
   const int rounds = g.iters > 0 ? g.iters : 1;
   for (int t = 0; t < rounds; ++t) {
     RI_CUDA_TRY(cudaMemsetAsync(queue_count, 0, sizeof(int), st));
@@ -942,14 +950,18 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
     RI_CUDA_TRY(cudaGetLastError());
     fixup_kernel<<<(unsigned)(4 * sms), 256, 0, st>>>(K, mu, d, queue, queue_count, labels);
     RI_CUDA_TRY(cudaGetLastError());
+    sort_kernel<<<(unsigned)units, kSortThreads, sort_smem(g.seg_len), st>>>(labels, d, members,
+                                                                             mstart);
+    RI_CUDA_TRY(cudaGetLastError());
     RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
-    update_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(
-        K, labels, d, mu, mu_bf16, nsplit, ust, counts, g.iters > 0 ? 1 : 0);
+    update_kernel<<<grid_upd, kUpdateWarps * 32, 0, st>>>(
+        K, members, mstart, d, mu, mu_bf16, nsplit, ust, counts, g.iters > 0 ? 1 : 0);
     RI_CUDA_TRY(cudaGetLastError());
   }
   if (a.out.objective)
     RI_CUDA_TRY(cudaMemsetAsync(a.out.objective, 0, units * sizeof(float), st));
-  finalise_kernel<<<grid_upd, kUpdateWarps * 32, upd_smem, st>>>(K, V, labels, d, mu, a.out);
+  finalise_kernel<<<grid_upd, kUpdateWarps * 32, 0, st>>>(K, V, labels, members, mstart, d, mu,
+                                                          a.out);
   RI_CUDA_TRY(cudaGetLastError());
   return RI_OK;
 }

@@ -189,6 +189,8 @@ bool make_build_layout(const Geometry& g, BuildLayout* L) {
   off = align_up(off + BH * g.M * 4, 256);
   L->off_mstart = off;
   off = align_up(off + BH * g.S * 513 * 4, 256);
+  L->off_ecs = off;
+  off = align_up(off + BH * g.S * 512 * 8, 256);
   L->total = off;
   return true;
 }

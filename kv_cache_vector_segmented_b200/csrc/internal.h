@@ -111,9 +111,10 @@ struct BuildLayout {
   // counts int32 [BH][C]; labels int32 [BH][M]; knorm fp32 [BH][M] (||k||);
   // queue of rows for the exact fix-up [BH*M] entries; members int32 [BH][M]
   // (positions within the segment, grouped by cluster in position order);
-  // mstart int32 [BH*S][513] (first member of each cluster).
+  // mstart int32 [BH*S][513] (first member of each cluster); ecs fp32
+  // [BH*S][512][2] (e_j, c_j of each centroid, reduced into ust).
   size_t off_mu, off_mu_bf16, off_nsplit, off_ust, off_counts, off_labels, off_knorm, off_queue,
-      off_members, off_mstart, total;
+      off_members, off_mstart, off_ecs, total;
 };
 size_t build_queue_bytes(long long rows);
 bool make_build_layout(const Geometry& g, BuildLayout* L);

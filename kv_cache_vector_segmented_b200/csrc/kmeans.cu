@@ -100,10 +100,6 @@ __device__ __forceinline__ UnitInfo tile_info(const BuildDims& d, int f) {
 
 __device__ __forceinline__ float col_c(float n) { return 3.0517578125e-05f * (n + 1.f); }
 
-__device__ __forceinline__ void atomic_max_pos(float* addr, float v) {
-  atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));  // v >= 0
-}
-
 // Entry of centroid j (K half kc) in a unit's [512][16] bf16 tile of
 // ||mu||^2 terms, stored in the plain K-major layout of the MMA operand:
 // 8-row x 16-byte core matrices, K halves 128 bytes apart, row groups 256.
@@ -125,12 +121,12 @@ __device__ __forceinline__ uint4 split3_bf16(float h) {
 }
 
 // Column constants of one centroid from its fp32 row (lane holds 4 dims):
-// the bf16 row (MMA operand), the entry of -||mu||^2 / 2 in the unit's tile,
-// and the unit's maxima of e = error coefficient of the bf16 operand and of
-// c (see file header).
-__device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf_row,
-                                               uint8_t* ns_tile, int j, float* ust_unit,
-                                               int lane, bool write_bf16) {
+// the bf16 row (MMA operand) and the entry of -||mu||^2 / 2 in the unit's
+// tile.  Returns (e, c) on every lane: e = error coefficient of the bf16
+// operand, c = rounding term (see file header).
+__device__ __forceinline__ float2 centroid_stats(const float4 m, __nv_bfloat16* bf_row,
+                                                 uint8_t* ns_tile, int j, int lane,
+                                                 bool write_bf16) {
   const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
   const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
   if (write_bf16) {
@@ -148,14 +144,12 @@ __device__ __forceinline__ void centroid_stats(const float4 m, __nv_bfloat16* bf
     sq += __shfl_xor_sync(0xffffffffu, sq, off);
     rr += __shfl_xor_sync(0xffffffffu, rr, off);
   }
-  if (lane == 0) {
-    const float e = 2.f * sqrtf(rr) * 1.0001f + 6.1035156e-05f * sqrtf(sq) + 1e-30f;
+  if (lane == 0)
     *ns_entry(ns_tile, j, 0) = split3_bf16(-0.5f * sq);
-    atomic_max_pos(&ust_unit[0], e);
-    atomic_max_pos(&ust_unit[1], col_c(sq));
-  } else if (lane == 1) {
+  else if (lane == 1)
     *ns_entry(ns_tile, j, 1) = make_uint4(0u, 0u, 0u, 0u);
-  }
+  const float e = 2.f * sqrtf(rr) * 1.0001f + 6.1035156e-05f * sqrtf(sq) + 1e-30f;
+  return make_float2(e, col_c(sq));
 }
 
 // ------------------------------------------------------------- assignment
@@ -536,22 +530,27 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------- prep
-// ||k|| of every middle token (one warp per row), rounded up so bounds that
-// use it stay upper bounds.
+// ||k|| of every middle token (four lanes per row, 16-byte loads), rounded
+// up so bounds that use it stay upper bounds.
 __global__ void knorm_kernel(const __nv_bfloat16* __restrict__ K, float* __restrict__ knorm,
                              int N, int M, int m0, long long rows) {
-  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (w >= rows) return;
-  const long long bh = w / M, m = w % M;
-  const __nv_bfloat16* src = K + ((size_t)bh * N + m0 + m) * kHeadDim + lane * 4;
-  const uint2 raw = *reinterpret_cast<const uint2*>(src);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  float s = a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y;
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 2;
+  const int part = threadIdx.x & 3;
+  float s = 0.f;
+  if (r < rows) {
+    const long long bh = r / M, m = r % M;
+    const uint4* src = reinterpret_cast<const uint4*>(K + ((size_t)bh * N + m0 + m) * kHeadDim);
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) knorm[w] = sqrtf(s) * 1.0001f;
+    for (int i = 0; i < 4; ++i) {
+      float f[8];
+      bf16x8_to_float(ldg_nc_v4(src + i * 4 + part), f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s += f[k] * f[k];
+    }
+  }
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  if (r < rows && part == 0) knorm[r] = sqrtf(s) * 1.0001f;
 }
 
 // Seeds: mu_j = k at the given (or strided) position of the segment.  One
@@ -559,11 +558,12 @@ __global__ void knorm_kernel(const __nv_bfloat16* __restrict__ K, float* __restr
 __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
                             const int32_t* __restrict__ init_pos, BuildDims d,
                             float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_bf16,
-                            uint8_t* __restrict__ nsplit, float* __restrict__ ust, int* status,
+                            uint8_t* __restrict__ nsplit, float2* __restrict__ ecs, int* status,
                             long long total) {
+  // blocks of 8 warps: kMaxClustersPerSeg is a multiple of 8, so a block's
+  // warps share one unit and `total` fills whole blocks
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (w >= total) return;
   const int unit = (int)(w / kMaxClustersPerSeg);
   const int j = (int)(w % kMaxClustersPerSeg);
   const int bh = unit / d.S, s = unit % d.S;
@@ -571,32 +571,59 @@ __global__ void init_kernel(const __nv_bfloat16* __restrict__ K,
   const int L = last ? d.L_last : d.seg_len;
   const int Ks = last ? d.K_last : d.K_full;
   uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
-  if (j >= Ks) {
+  if (w < total && j >= Ks) {
     // padding column: w_j = -inf, never a candidate
     if (lane < 2)
-      *ns_entry(ns, j, lane) = lane == 0 ? make_uint4(0xFF80u, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
-    return;
-  }
-  const int c = s * d.K_full + j;
-  int p;
-  if (init_pos) {
-    p = init_pos[(size_t)bh * d.C + c];
-    if (p < 0 || p >= L) {
-      if (lane == 0) record_status(status, RI_ERR_INVALID_ARG);
-      p = p < 0 ? 0 : L - 1;
+      *ns_entry(ns, j, lane) =
+          lane == 0 ? make_uint4(0xFF80u, 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+  } else if (w < total) {
+    const int c = s * d.K_full + j;
+    int p;
+    if (init_pos) {
+      p = init_pos[(size_t)bh * d.C + c];
+      if (p < 0 || p >= L) {
+        if (lane == 0) record_status(status, RI_ERR_INVALID_ARG);
+        p = p < 0 ? 0 : L - 1;
+      }
+    } else {
+      p = (int)(((long long)j * L) / Ks);
     }
-  } else {
-    p = (int)(((long long)j * L) / Ks);
+    const __nv_bfloat16* src =
+        K + ((size_t)bh * d.N + d.m0 + (size_t)s * d.seg_len + p) * kHeadDim + lane * 4;
+    const uint2 raw = *reinterpret_cast<const uint2*>(src);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+    const float4 m = make_float4(a.x, a.y, b.x, b.y);
+    *reinterpret_cast<float4*>(mu + ((size_t)bh * d.C + c) * kHeadDim + lane * 4) = m;
+    const float2 ec =
+        centroid_stats(m, mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim, ns, j, lane, true);
+    if (lane == 0) ecs[w] = ec;
   }
-  const __nv_bfloat16* src =
-      K + ((size_t)bh * d.N + d.m0 + (size_t)s * d.seg_len + p) * kHeadDim + lane * 4;
-  const uint2 raw = *reinterpret_cast<const uint2*>(src);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  const float4 m = make_float4(a.x, a.y, b.x, b.y);
-  *reinterpret_cast<float4*>(mu + ((size_t)bh * d.C + c) * kHeadDim + lane * 4) = m;
-  centroid_stats(m, mu_bf16 + ((size_t)bh * d.C + c) * kHeadDim, ns, j, ust + 2 * unit, lane,
-                 true);
+}
+
+// Per unit: E = max e_j, Cmax = max c_j over its K_s centroids (one warp per
+// unit, from the per-centroid values the update wrote).
+__global__ void unit_max_kernel(const float2* __restrict__ ecs, BuildDims d,
+                                float* __restrict__ ust, int units) {
+  const int unit = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
+  const int lane = threadIdx.x & 31;
+  if (unit >= units) return;
+  const int Ks = unit % d.S == d.S - 1 ? d.K_last : d.K_full;
+  float2 r = make_float2(0.f, 0.f);
+  for (int j = lane; j < Ks; j += 32) {
+    const float2 v = ecs[(size_t)unit * kMaxClustersPerSeg + j];
+    r.x = fmaxf(r.x, v.x);
+    r.y = fmaxf(r.y, v.y);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    r.x = fmaxf(r.x, __shfl_xor_sync(0xffffffffu, r.x, off));
+    r.y = fmaxf(r.y, __shfl_xor_sync(0xffffffffu, r.y, off));
+  }
+  if (lane == 0) {
+    ust[2 * unit] = r.x;
+    ust[2 * unit + 1] = r.y;
+  }
 }
 
 // ------------------------------------------------------------- update / finalise
@@ -683,136 +710,149 @@ __global__ void __launch_bounds__(kSortThreads)
 // One warp per cluster: mu_j = mean of the members (fp32, summed in position
 // order; an empty cluster keeps mu_j), the column constants of the new
 // centroid and the cluster size.
-__global__ void __launch_bounds__(kUpdateWarps * 32)
+__global__ void __launch_bounds__(kUpdateWarps * 32, 4)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ members,
                   const int32_t* __restrict__ mstart, BuildDims d, float* __restrict__ mu,
                   __nv_bfloat16* __restrict__ mu_bf16, uint8_t* __restrict__ nsplit,
-                  float* __restrict__ ust, int32_t* __restrict__ counts, int update_mu) {
-  const int unit = blockIdx.x;
-  const int bh = unit / d.S, s = unit % d.S;
-  const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+                  float2* __restrict__ ecs, int32_t* __restrict__ counts, int update_mu) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.y * kUpdateWarps + warp;
-  if (j >= Ks) return;
-  const int seg_start = s * d.seg_len;
-  const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
-  const int b = ms[j], e = ms[j + 1];
-  const int32_t* mem = members + (size_t)bh * d.M + seg_start;
-  const __nv_bfloat16* kbase = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int i = b; i < e; i += 16) {
-    uint2 raw[16];
+  {
+    const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
+    const int bh = unit / d.S, s = unit % d.S;
+    const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+    if (j >= Ks) return;
+    const int seg_start = s * d.seg_len;
+    const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+    const int b = ms[j], e = ms[j + 1];
+    const int32_t* mem = members + (size_t)bh * d.M + seg_start;
+    const __nv_bfloat16* kbase =
+        K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = b; i < e; i += 32) {
+      const int nb = min(32, e - i);
+      const int pos = lane < nb ? mem[i + lane] : 0;  // 32 member positions, one load
+      for (int u0 = 0; u0 < nb; u0 += 16) {
+        uint2 raw[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
-      raw[u] = i + u < e ? *reinterpret_cast<const uint2*>(kbase + (size_t)mem[i + u] * kHeadDim)
-                         : make_uint2(0, 0);
+        for (int u = 0; u < 16; ++u) {
+          const int p = __shfl_sync(0xffffffffu, pos, (u0 + u) & 31);
+          raw[u] = u0 + u < nb ? *reinterpret_cast<const uint2*>(kbase + (size_t)p * kHeadDim)
+                               : make_uint2(0, 0);
+        }
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      if (i + u < e) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-        const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
-        acc[0] += a.x;
-        acc[1] += a.y;
-        acc[2] += bb.x;
-        acc[3] += bb.y;
+        for (int u = 0; u < 16; ++u) {
+          if (u0 + u < nb) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+            const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
+            acc[0] += a.x;
+            acc[1] += a.y;
+            acc[2] += bb.x;
+            acc[3] += bb.y;
+          }
+        }
       }
     }
+    const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+    uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
+    const int n = e - b;
+    float2 ec;
+    if (update_mu && n > 0) {
+      const float fn = (float)n;
+      const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
+      *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
+      ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, true);
+    } else {
+      const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
+      ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, false);
+    }
+    if (lane == 0) {
+      counts[row] = n;
+      ecs[(size_t)unit * kMaxClustersPerSeg + j] = ec;
+    }
   }
-  const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
-  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
-  const int n = e - b;
-  if (update_mu && n > 0) {
-    const float fn = (float)n;
-    const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
-    *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
-    centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, true);
-  } else {
-    const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
-    centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, ust + 2 * unit, lane, false);
-  }
-  if (lane == 0) counts[row] = n;
 }
 
 // Cluster-contiguous layout of the final labels (members / mstart from the
 // last sort): one warp per cluster copies its members' K and V rows in
 // (cluster, position) order, with the permutation, offsets, sizes, value
 // sums, the bf16 centroid and the members' squared distances.
-__global__ void __launch_bounds__(kUpdateWarps * 32)
+__global__ void __launch_bounds__(kUpdateWarps * 32, 4)
     finalise_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                     const int32_t* __restrict__ labels, const int32_t* __restrict__ members,
                     const int32_t* __restrict__ mstart, BuildDims d,
                     const float* __restrict__ mu, ri_index out) {
-  const int unit = blockIdx.x;
-  const int bh = unit / d.S, s = unit % d.S;
-  const bool last = s == d.S - 1;
-  const int L = last ? d.L_last : d.seg_len;
-  const int Ks = last ? d.K_last : d.K_full;
-  const int seg_start = s * d.seg_len;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (out.labels && blockIdx.y == 0)
-    for (int t = threadIdx.x; t < L; t += blockDim.x)
-      out.labels[(size_t)bh * d.M + seg_start + t] = labels[(size_t)bh * d.M + seg_start + t];
-  if (blockIdx.y == 0 && last && threadIdx.x == 0)
-    out.offsets[(size_t)bh * (d.C + 1) + d.C] = d.M;
-  const int j = blockIdx.y * kUpdateWarps + warp;
-  if (j >= Ks) return;
-  const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
-  const int b = ms[j], e = ms[j + 1];
-  const int32_t* mem = members + (size_t)bh * d.M + seg_start;
-  const size_t bhN = (size_t)bh * d.N + d.m0 + seg_start;
-  const size_t bhM = (size_t)bh * d.M + seg_start;
-  const size_t crow = (size_t)bh * d.C + (size_t)s * d.K_full + j;
-  const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
-  float vs[4] = {0.f, 0.f, 0.f, 0.f};
-  float obj = 0.f;
-  for (int i = b; i < e; i += 8) {
-    uint2 kr[8], vr[8];
-    int pos[8];
+  {
+    const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
+    const int bh = unit / d.S, s = unit % d.S;
+    const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+    const int L = s == d.S - 1 ? d.L_last : d.seg_len;
+    if (out.labels && blockIdx.y == 0)
+      for (int t = threadIdx.x; t < L; t += blockDim.x)
+        out.labels[(size_t)bh * d.M + s * d.seg_len + t] =
+            labels[(size_t)bh * d.M + s * d.seg_len + t];
+    if (blockIdx.y == 0 && s == d.S - 1 && threadIdx.x == 0)
+      out.offsets[(size_t)bh * (d.C + 1) + d.C] = d.M;
+    if (j >= Ks) return;
+    const int seg_start = s * d.seg_len;
+    const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+    const int b = ms[j], e = ms[j + 1];
+    const int32_t* mem = members + (size_t)bh * d.M + seg_start;
+    const size_t bhN = (size_t)bh * d.N + d.m0 + seg_start;
+    const size_t bhM = (size_t)bh * d.M + seg_start;
+    const size_t crow = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+    const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
+    float vs[4] = {0.f, 0.f, 0.f, 0.f};
+    float obj = 0.f;
+    for (int i = b; i < e; i += 8) {
+      uint2 kr[8], vr[8];
+      int pos[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const bool in = i + u < e;
-      pos[u] = in ? mem[i + u] : 0;
-      const size_t src = (bhN + pos[u]) * kHeadDim + lane * 4;
-      kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
-      vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
-    }
+      for (int u = 0; u < 8; ++u) {
+        const bool in = i + u < e;
+        pos[u] = in ? mem[i + u] : 0;
+        const size_t src = (bhN + pos[u]) * kHeadDim + lane * 4;
+        kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
+        vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
+      }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (i + u < e) {
-        const size_t dst = (bhM + i + u) * kHeadDim + lane * 4;  // rows in (cluster, position) order
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
-        if (lane == 0) out.perm[bhM + i + u] = d.m0 + seg_start + pos[u];
-        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
-        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
-        const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
-        const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
-        vs[0] += va.x;
-        vs[1] += va.y;
-        vs[2] += vb.x;
-        vs[3] += vb.y;
-        const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
-        obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+      for (int u = 0; u < 8; ++u) {
+        if (i + u < e) {
+          const size_t dst = (bhM + i + u) * kHeadDim + lane * 4;  // (cluster, position) order
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
+          if (lane == 0) out.perm[bhM + i + u] = d.m0 + seg_start + pos[u];
+          const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
+          const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+          const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
+          const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
+          vs[0] += va.x;
+          vs[1] += va.y;
+          vs[2] += vb.x;
+          vs[3] += vb.y;
+          const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
+          obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+        }
       }
     }
-  }
-  *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
-      make_float4(vs[0], vs[1], vs[2], vs[3]);
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
-  uint2 packed;
-  packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-  packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + crow * kHeadDim +
-                            lane * 4) = packed;
-  if (lane == 0) {
-    out.counts[crow] = e - b;
-    out.offsets[(size_t)bh * (d.C + 1) + (size_t)s * d.K_full + j] = seg_start + b;
-  }
-  if (out.objective) {
+    *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
+        make_float4(vs[0], vs[1], vs[2], vs[3]);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.centroid) + crow * kHeadDim +
+                              lane * 4) = packed;
+    if (lane == 0) {
+      out.counts[crow] = e - b;
+      out.offsets[(size_t)bh * (d.C + 1) + (size_t)s * d.K_full + j] = seg_start + b;
+    }
+    if (out.objective) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, off);
-    if (lane == 0) atomicAdd(&out.objective[unit], obj);
+      for (int off = 16; off >= 1; off >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, off);
+      if (lane == 0) atomicAdd(&out.objective[unit], obj);
+    }
   }
 }
 
@@ -914,6 +954,7 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   FixEntry* queue = reinterpret_cast<FixEntry*>(ws + L.off_queue);
   int32_t* members = reinterpret_cast<int32_t*>(ws + L.off_members);
   int32_t* mstart = reinterpret_cast<int32_t*>(ws + L.off_mstart);
+  float2* ecs = reinterpret_cast<float2*>(ws + L.off_ecs);
   const long long units = BH * g.S;
 
   CUtensorMap tm_keys, tm_cent;
@@ -923,12 +964,13 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
     return RI_ERR_CUDA;
   }
   const long long rows = BH * g.M;
-  knorm_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(K, knorm, g.N, g.M, g.m0, rows);
+  knorm_kernel<<<(unsigned)((rows + 63) / 64), 256, 0, st>>>(K, knorm, g.N, g.M, g.m0, rows);
   RI_CUDA_TRY(cudaGetLastError());
-  RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
   const long long init_total = units * kMaxClustersPerSeg;
   init_kernel<<<(unsigned)((init_total + 7) / 8), 256, 0, st>>>(K, a.init_pos, d, mu, mu_bf16,
-                                                                 nsplit, ust, status, init_total);
+                                                                 nsplit, ecs, status, init_total);
+  RI_CUDA_TRY(cudaGetLastError());
+  unit_max_kernel<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(ecs, d, ust, (int)units);
   RI_CUDA_TRY(cudaGetLastError());
 
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
@@ -953,9 +995,10 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
     sort_kernel<<<(unsigned)units, kSortThreads, sort_smem(g.seg_len), st>>>(labels, d, members,
                                                                              mstart);
     RI_CUDA_TRY(cudaGetLastError());
-    RI_CUDA_TRY(cudaMemsetAsync(ust, 0, units * 2 * sizeof(float), st));
     update_kernel<<<grid_upd, kUpdateWarps * 32, 0, st>>>(
-        K, members, mstart, d, mu, mu_bf16, nsplit, ust, counts, g.iters > 0 ? 1 : 0);
+        K, members, mstart, d, mu, mu_bf16, nsplit, ecs, counts, g.iters > 0 ? 1 : 0);
+    RI_CUDA_TRY(cudaGetLastError());
+    unit_max_kernel<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(ecs, d, ust, (int)units);
     RI_CUDA_TRY(cudaGetLastError());
   }
   if (a.out.objective)

@@ -1239,41 +1239,46 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
       __threadfence();
       const float* pu = p.part + (size_t)u * p.S * G * kPartStride;
       float* fq = reinterpret_cast<float*>(sm);  // [S][G] maxima, then weights
-      float* lq = fq + p.S * G;                  // [S][G] denominators
-      float* tot = lq + p.S * G;                 // [G] max, [G] denominator
-      for (int i = threadIdx.x; i < p.S * G; i += NT) {
-        fq[i] = __ldcg(pu + (size_t)i * kPartStride);
-        lq[i] = __ldcg(pu + (size_t)i * kPartStride + 1);
-      }
-      __syncthreads();
-      if (threadIdx.x < G) {
-        const int g = threadIdx.x;
+      float* tot = fq + p.S * G;                 // [G] max, [G] denominator
+      if (warp < G) {
+        // warp g: the slices' maxima and denominators of query head g
+        const int g = warp;
         float mx = -INFINITY;
-        for (int q = 0; q < p.S; ++q) mx = fmaxf(mx, fq[q * G + g]);
-        float ls = 0.f;
-        for (int q = 0; q < p.S; ++q) {
-          const float f = (mx == -INFINITY || fq[q * G + g] == -INFINITY)
-                              ? 0.f : __expf(fq[q * G + g] - mx);
-          fq[q * G + g] = f;
-          ls = fmaf(lq[q * G + g], f, ls);
+        for (int q = lane; q < p.S; q += 32) {
+          const float m = __ldcg(pu + ((size_t)q * G + g) * kPartStride);
+          fq[q * G + g] = m;
+          mx = fmaxf(mx, m);
         }
-        tot[g] = mx;
-        tot[G + g] = ls;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        float ls = 0.f;
+        for (int q = lane; q < p.S; q += 32) {
+          const float m = fq[q * G + g];
+          const float f = (mx == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - mx);
+          fq[q * G + g] = f;
+          ls = fmaf(__ldcg(pu + ((size_t)q * G + g) * kPartStride + 1), f, ls);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+        if (lane == 0) {
+          tot[g] = mx;
+          tot[G + g] = ls;
+        }
       }
       __syncthreads();
       for (int idx = threadIdx.x; idx < G * kHeadDim; idx += NT) {
         const int g = idx / kHeadDim, d = idx - g * kHeadDim;
         float os = 0.f;
-        int q = 0;
-        for (; q + 8 <= p.S; q += 8) {
-          float v[8];
+        for (int q0 = 0; q0 < p.S; q0 += 16) {
+          float v[16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = __ldcg(pu + ((size_t)(q + k) * G + g) * kPartStride + 4 + d);
+          for (int k = 0; k < 16; ++k)
+            v[k] = q0 + k < p.S ? __ldcg(pu + ((size_t)(q0 + k) * G + g) * kPartStride + 4 + d)
+                                : 0.f;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) os = fmaf(fq[(q + k) * G + g], v[k], os);
+          for (int k = 0; k < 16; ++k)
+            if (q0 + k < p.S) os = fmaf(fq[(q0 + k) * G + g], v[k], os);
         }
-        for (; q < p.S; ++q)
-          os = fmaf(fq[q * G + g], __ldcg(pu + ((size_t)q * G + g) * kPartStride + 4 + d), os);
         const float ls = tot[G + g];
         // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
         const bool any = ls > 0.f;

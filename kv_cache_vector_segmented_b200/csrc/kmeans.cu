@@ -46,6 +46,10 @@ constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
 constexpr int kCand = 8;          // candidate slots per row
 constexpr int kUpdateWarps = 8;   // update / finalise: one warp per cluster
 constexpr int kSortThreads = 1024;
+constexpr int kGatherRows = 32;   // member rows per cp.async chunk of the update
+constexpr int kUpdateSmem = kUpdateWarps * kGatherRows * 128 * 2;  // 64 KB
+constexpr int kFinRows = 16;      // member rows (K and V) per cp.async chunk of the finalise
+constexpr int kFinSmem = kUpdateWarps * kFinRows * 512;             // 64 KB
 constexpr uint16_t kCandNone = 0xFFFF;
 constexpr uint16_t kCandFullScan = 0xFFFE;
 
@@ -709,66 +713,69 @@ __global__ void __launch_bounds__(kSortThreads)
 
 // One warp per cluster: mu_j = mean of the members (fp32, summed in position
 // order; an empty cluster keeps mu_j), the column constants of the new
-// centroid and the cluster size.
-__global__ void __launch_bounds__(kUpdateWarps * 32, 4)
+// centroid and the cluster size.  Members are fetched 32 rows at a time with
+// 16-byte cp.async copies into the warp's 8 KB of shared memory (the
+// transfers need no registers, so a warp keeps a whole chunk in flight).
+__global__ void __launch_bounds__(kUpdateWarps * 32, 3)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ members,
                   const int32_t* __restrict__ mstart, BuildDims d, float* __restrict__ mu,
                   __nv_bfloat16* __restrict__ mu_bf16, uint8_t* __restrict__ nsplit,
                   float2* __restrict__ ecs, int32_t* __restrict__ counts, int update_mu) {
+  extern __shared__ __align__(16) uint8_t smem_g[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  {
-    const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
-    const int bh = unit / d.S, s = unit % d.S;
-    const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
-    if (j >= Ks) return;
-    const int seg_start = s * d.seg_len;
-    const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
-    const int b = ms[j], e = ms[j + 1];
-    const int32_t* mem = members + (size_t)bh * d.M + seg_start;
-    const __nv_bfloat16* kbase =
-        K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim + lane * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = b; i < e; i += 32) {
-      const int nb = min(32, e - i);
-      const int pos = lane < nb ? mem[i + lane] : 0;  // 32 member positions, one load
-      for (int u0 = 0; u0 < nb; u0 += 16) {
-        uint2 raw[16];
+  const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
+  const int bh = unit / d.S, s = unit % d.S;
+  const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
+  if (j >= Ks) return;
+  uint8_t* wb = smem_g + (size_t)warp * kGatherRows * kHeadDim * 2;  // [32 rows][256 B]
+  const int seg_start = s * d.seg_len;
+  const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
+  const int b = ms[j], e = ms[j + 1];
+  const int32_t* mem = members + (size_t)bh * d.M + seg_start;
+  const __nv_bfloat16* kseg = K + ((size_t)bh * d.N + d.m0 + seg_start) * kHeadDim;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i = b; i < e; i += kGatherRows) {
+    const int nb = min(kGatherRows, e - i);
+    const int pos = lane < nb ? mem[i + lane] : 0;  // 32 member positions, one load
+    // row r = 2 k + (lane >> 4), 16-byte chunk lane & 15
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int p = __shfl_sync(0xffffffffu, pos, (u0 + u) & 31);
-          raw[u] = u0 + u < nb ? *reinterpret_cast<const uint2*>(kbase + (size_t)p * kHeadDim)
-                               : make_uint2(0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (u0 + u < nb) {
-            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-            const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
-            acc[0] += a.x;
-            acc[1] += a.y;
-            acc[2] += bb.x;
-            acc[3] += bb.y;
-          }
-        }
-      }
+    for (int k = 0; k < kGatherRows / 2; ++k) {
+      const int r = 2 * k + (lane >> 4);
+      const int p = __shfl_sync(0xffffffffu, pos, r);
+      if (r < nb)
+        cp_async16(wb + r * (kHeadDim * 2) + (lane & 15) * 16,
+                   kseg + (size_t)p * kHeadDim + (lane & 15) * 8);
     }
-    const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
-    uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
-    const int n = e - b;
-    float2 ec;
-    if (update_mu && n > 0) {
-      const float fn = (float)n;
-      const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
-      *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
-      ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, true);
-    } else {
-      const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
-      ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, false);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+    for (int r = 0; r < nb; ++r) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(wb + r * (kHeadDim * 2) + lane * 8);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      const float2 a = __bfloat1622float2(h[0]), bb = __bfloat1622float2(h[1]);
+      acc[0] += a.x;
+      acc[1] += a.y;
+      acc[2] += bb.x;
+      acc[3] += bb.y;
     }
-    if (lane == 0) {
-      counts[row] = n;
-      ecs[(size_t)unit * kMaxClustersPerSeg + j] = ec;
-    }
+    __syncwarp();  // the buffer is refilled by the next chunk
+  }
+  const size_t row = (size_t)bh * d.C + (size_t)s * d.K_full + j;
+  uint8_t* ns = nsplit + (size_t)unit * kNsTileBytes;
+  const int n = e - b;
+  float2 ec;
+  if (update_mu && n > 0) {
+    const float fn = (float)n;
+    const float4 m = make_float4(acc[0] / fn, acc[1] / fn, acc[2] / fn, acc[3] / fn);
+    *reinterpret_cast<float4*>(mu + row * kHeadDim + lane * 4) = m;
+    ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, true);
+  } else {
+    const float4 m = *reinterpret_cast<const float4*>(mu + row * kHeadDim + lane * 4);
+    ec = centroid_stats(m, mu_bf16 + row * kHeadDim, ns, j, lane, false);
+  }
+  if (lane == 0) {
+    counts[row] = n;
+    ecs[(size_t)unit * kMaxClustersPerSeg + j] = ec;
   }
 }
 
@@ -776,11 +783,12 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 4)
 // last sort): one warp per cluster copies its members' K and V rows in
 // (cluster, position) order, with the permutation, offsets, sizes, value
 // sums, the bf16 centroid and the members' squared distances.
-__global__ void __launch_bounds__(kUpdateWarps * 32, 4)
+__global__ void __launch_bounds__(kUpdateWarps * 32, 3)
     finalise_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                     const int32_t* __restrict__ labels, const int32_t* __restrict__ members,
                     const int32_t* __restrict__ mstart, BuildDims d,
                     const float* __restrict__ mu, ri_index out) {
+  extern __shared__ __align__(16) uint8_t smem_f[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   {
     const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
@@ -801,42 +809,58 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 4)
     const size_t bhN = (size_t)bh * d.N + d.m0 + seg_start;
     const size_t bhM = (size_t)bh * d.M + seg_start;
     const size_t crow = (size_t)bh * d.C + (size_t)s * d.K_full + j;
-    const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
-    float vs[4] = {0.f, 0.f, 0.f, 0.f};
-    float obj = 0.f;
-    for (int i = b; i < e; i += 8) {
-      uint2 kr[8], vr[8];
-      int pos[8];
+    // lane l < 16 moves 16-byte chunk l of each member's K row, lane 16 + l
+    // chunk l of its V row: 16 rows per cp.async chunk through the warp's 8 KB
+    uint8_t* wb = smem_f + (size_t)warp * kFinRows * 512;  // [16 rows][K 256 B | V 256 B]
+    const int ch = lane & 15;
+    const bool is_v = lane >= 16;
+    float mk[8];  // this lane's 8 centroid dims (K lanes)
+    {
+      const float4 m0v = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + ch * 8);
+      const float4 m1v = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + ch * 8 + 4);
+      mk[0] = m0v.x; mk[1] = m0v.y; mk[2] = m0v.z; mk[3] = m0v.w;
+      mk[4] = m1v.x; mk[5] = m1v.y; mk[6] = m1v.z; mk[7] = m1v.w;
+    }
+    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // V sums (V lanes)
+    float obj = 0.f;                                           // squared distances (K lanes)
+    const __nv_bfloat16* src_base = (is_v ? V : K) + bhN * kHeadDim + ch * 8;
+    __nv_bfloat16* dst_base = static_cast<__nv_bfloat16*>(is_v ? out.Vp : out.Kp) + ch * 8;
+    for (int i = b; i < e; i += kFinRows) {
+      const int nb = min(kFinRows, e - i);
+      const int pos = lane < nb ? mem[i + lane] : 0;
+      if (lane < nb) out.perm[bhM + i + lane] = d.m0 + seg_start + pos;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool in = i + u < e;
-        pos[u] = in ? mem[i + u] : 0;
-        const size_t src = (bhN + pos[u]) * kHeadDim + lane * 4;
-        kr[u] = in ? *reinterpret_cast<const uint2*>(K + src) : make_uint2(0, 0);
-        vr[u] = in ? *reinterpret_cast<const uint2*>(V + src) : make_uint2(0, 0);
+      for (int r = 0; r < kFinRows; ++r) {
+        const int pr = __shfl_sync(0xffffffffu, pos, r);
+        if (r < nb) cp_async16(wb + r * 512 + lane * 16, src_base + (size_t)pr * kHeadDim);
       }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncwarp();
+      for (int r = 0; r < nb; ++r) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(wb + r * 512 + lane * 16);
+        *reinterpret_cast<uint4*>(dst_base + (bhM + i + r) * kHeadDim) = raw;  // (cluster, position) order
+        float f[8];
+        bf16x8_to_float(raw, f);
+        if (is_v) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (i + u < e) {
-          const size_t dst = (bhM + i + u) * kHeadDim + lane * 4;  // (cluster, position) order
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Kp) + dst) = kr[u];
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out.Vp) + dst) = vr[u];
-          if (lane == 0) out.perm[bhM + i + u] = d.m0 + seg_start + pos[u];
-          const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kr[u]);
-          const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
-          const float2 ka = __bfloat1622float2(kh[0]), kb = __bfloat1622float2(kh[1]);
-          const float2 va = __bfloat1622float2(vh[0]), vb = __bfloat1622float2(vh[1]);
-          vs[0] += va.x;
-          vs[1] += va.y;
-          vs[2] += vb.x;
-          vs[3] += vb.y;
-          const float d0 = ka.x - m.x, d1 = ka.y - m.y, d2 = kb.x - m.z, d3 = kb.y - m.w;
-          obj += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+          for (int k = 0; k < 8; ++k) acc8[k] += f[k];
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float dd = f[k] - mk[k];
+            obj = fmaf(dd, dd, obj);
+          }
         }
       }
+      __syncwarp();  // the buffer is refilled by the next chunk
     }
-    *reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + lane * 4) =
-        make_float4(vs[0], vs[1], vs[2], vs[3]);
+    if (is_v) {
+      float4* vdst = reinterpret_cast<float4*>(out.vsum + crow * kHeadDim + ch * 8);
+      vdst[0] = make_float4(acc8[0], acc8[1], acc8[2], acc8[3]);
+      vdst[1] = make_float4(acc8[4], acc8[5], acc8[6], acc8[7]);
+    }
+    const float4 m = *reinterpret_cast<const float4*>(mu + crow * kHeadDim + lane * 4);
     const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y);
     const __nv_bfloat162 hi = __floats2bfloat162_rn(m.z, m.w);
     uint2 packed;
@@ -981,6 +1005,8 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   };
   RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(sort_kernel),
                             (int)sort_smem(kMaxSegLen)));
+  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(update_kernel), kUpdateSmem));
+  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(finalise_kernel), kFinSmem));
   const int sms = num_sms();
   const unsigned grid_assign = (unsigned)(d.total_tiles < sms ? d.total_tiles : sms);
   const dim3 grid_upd((unsigned)units, (unsigned)(kMaxClustersPerSeg / kUpdateWarps));
@@ -995,7 +1021,7 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
     sort_kernel<<<(unsigned)units, kSortThreads, sort_smem(g.seg_len), st>>>(labels, d, members,
                                                                              mstart);
     RI_CUDA_TRY(cudaGetLastError());
-    update_kernel<<<grid_upd, kUpdateWarps * 32, 0, st>>>(
+    update_kernel<<<grid_upd, kUpdateWarps * 32, kUpdateSmem, st>>>(
         K, members, mstart, d, mu, mu_bf16, nsplit, ecs, counts, g.iters > 0 ? 1 : 0);
     RI_CUDA_TRY(cudaGetLastError());
     unit_max_kernel<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(ecs, d, ust, (int)units);
@@ -1003,8 +1029,8 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   }
   if (a.out.objective)
     RI_CUDA_TRY(cudaMemsetAsync(a.out.objective, 0, units * sizeof(float), st));
-  finalise_kernel<<<grid_upd, kUpdateWarps * 32, 0, st>>>(K, V, labels, members, mstart, d, mu,
-                                                          a.out);
+  finalise_kernel<<<grid_upd, kUpdateWarps * 32, kFinSmem, st>>>(K, V, labels, members, mstart,
+                                                                 d, mu, a.out);
   RI_CUDA_TRY(cudaGetLastError());
   return RI_OK;
 }

@@ -131,6 +131,14 @@ def test_kmeans_small_segments_and_strided_seeds(R):
     _check_layout(R, kv, idx, 300, 64)
 
 
+def test_kmeans_max_segment_length(R):
+    """Segments of the largest supported length (16384 tokens, 512
+    clusters) plus a ragged 500-token last segment: the counting sort's
+    largest shared-memory footprint and 512 positions per warp."""
+    kv, idx, frac = _compare_kmeans(R, 1, 1, 68 + 16384 + 500, 3, seg_len=16384, seed=12)
+    _check_layout(R, kv, idx, 16384, 512)
+
+
 def test_kmeans_one_token_per_cluster(R):
     """K_s = L_s: every token is its own centroid, objective zero."""
     kv, idx, frac = _compare_kmeans(R, 1, 1, 68 + 200, 3, seed=4)

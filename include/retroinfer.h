@@ -272,7 +272,8 @@ void ri_cache_destroy(ri_cache* cache);
  * order from row 0 (ri_select_clusters' retr_rows).  Lookup first (hit:
  * resident; a cluster of 0 rows is a hit and is not cached), then the misses
  * are admitted in order, evicting least recently used clusters not requested
- * in this step until the miss fits (else it is served uncached), and every
+ * in this step until the miss fits (a miss that cannot fit even after every
+ * such eviction is served uncached and evicts nothing), and every
  * requested resident cluster becomes most recent in request order.  Writes
  * the copy plan: `fetch` (cache->exec for hits, host->exec for misses) and
  * `admit` (exec->cache for admitted misses), each split into copies of at

@@ -25,6 +25,7 @@ struct Entry {
 struct Unit {
   std::unordered_map<int, Entry> table;
   std::list<int> lru;            // least recently used first
+  long long lru_blocks = 0;      // blocks held by the clusters in `lru`
   std::vector<int> free;         // stack: the next block is free.back()
 };
 
@@ -178,7 +179,10 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         run += rows_of(ids[i]);
         auto it = U.table.find(ids[i]);
         hit[i] = rows_of(ids[i]) == 0 || it != U.table.end();
-        if (it != U.table.end()) U.lru.erase(it->second.pos);
+        if (it != U.table.end()) {
+          U.lru.erase(it->second.pos);
+          U.lru_blocks -= (long long)it->second.blocks.size();
+        }
       }
       for (size_t i = 0; i < ids.size(); ++i) {
         const int c = ids[i], n = rows_of(c);
@@ -200,16 +204,18 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         st.miss_rows += n;
         emit(f, u, RI_SRC_HOST, first_row(c), RI_DST_EXEC, erow[i], n);
         const int need = (n + br - 1) / br;
-        while ((int)U.free.size() < need && !U.lru.empty()) {
+        if ((long long)U.free.size() + U.lru_blocks < need) {
+          // cannot fit even after every eviction: served uncached, nothing evicted
+          ++st.uncached_clusters;
+          continue;
+        }
+        while ((int)U.free.size() < need) {
           const int v = U.lru.front();
           U.lru.pop_front();
           std::vector<int>& vb = U.table[v].blocks;
+          U.lru_blocks -= (long long)vb.size();
           U.free.insert(U.free.end(), vb.begin(), vb.end());
           U.table.erase(v);
-        }
-        if ((int)U.free.size() < need) {
-          ++st.uncached_clusters;
-          continue;
         }
         Entry e;
         for (int k = 0; k < need; ++k) {
@@ -227,6 +233,7 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         auto it = U.table.find(c);
         if (it == U.table.end()) continue;
         U.lru.push_back(c);
+        U.lru_blocks += (long long)it->second.blocks.size();
         it->second.pos = std::prev(U.lru.end());
       }
     }

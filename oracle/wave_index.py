@@ -385,8 +385,10 @@ class LRUClusterCache:
     then counted in clusters).  `access(ids)` looks every requested cluster up
     (hit or miss), then admits the misses in request order, evicting least
     recently used clusters that are not requested in this same step until the
-    miss fits; a miss that cannot fit is served without being cached.  All
-    requested resident clusters become most recent, in request order.  A
+    miss fits; a miss that cannot fit even after every such eviction (larger
+    than the free blocks plus those of the evictable residents) is served
+    without being cached and evicts nothing.  All requested resident clusters
+    become most recent, in request order.  A
     cluster of zero blocks holds no rows: it counts as a hit and is not
     tracked.  Returns (hits, misses) lists."""
 
@@ -404,14 +406,13 @@ class LRUClusterCache:
         req = set(ids)
         for i in misses:
             need = self.blocks(i)
+            evictable = sum(len(self.slot_of[v]) for v in self.order if v not in req)
+            if len(self.free) + evictable < need:
+                continue                    # cannot fit: served uncached, nothing evicted
             while len(self.free) < need:
-                victim = next((v for v in self.order if v not in req), None)
-                if victim is None:
-                    break                   # every resident cluster is requested
+                victim = next(v for v in self.order if v not in req)
                 self.order.remove(victim)
                 self.free.extend(self.slot_of.pop(victim))
-            if len(self.free) < need:
-                continue                    # served without being cached
             self.slot_of[i] = [self.free.pop() for _ in range(need)]
             self.order.append(i)
         for i in ids:

@@ -123,6 +123,23 @@ def test_plan_matches_model_random(seed):
     _run(units, cap, br, counts, offsets, steps, k_r)
 
 
+def test_cluster_larger_than_the_cache_is_served_uncached():
+    """A cluster needing more blocks than the whole cache is copied from host
+    memory every time and never admitted; the residents stay in place."""
+    br = 8
+    counts, offsets = _index_arrays([[8, 40, 16, 3]])  # cluster 1: 5 blocks
+    steps = [_sel([[0, 2]], 3), _sel([[1]], 3), _sel([[0, 1, 2]], 3), _sel([[1, 3]], 3)]
+    _run(1, 4, br, counts, offsets, steps, 3)
+    c = R.BlockCache(1, 4, br)
+    c.plan(steps[0], 3, counts, offsets)
+    f, a, st = c.plan(steps[1], 3, counts, offsets)
+    assert st["uncached_clusters"] == 1 and len(a) == 0
+    assert all(int(r[1]) == R.SRC_HOST for r in f)
+    f, a, st = c.plan(steps[2], 3, counts, offsets)
+    assert st["hit_clusters"] == 2 and st["uncached_clusters"] == 1
+    c.close()
+
+
 def test_plan_rejects_bad_input_and_keeps_state():
     counts, offsets = _index_arrays([[9, 3, 16, 1]])
     c = R.BlockCache(1, 2, 8)

@@ -136,3 +136,19 @@ def test_workspace_sizes_scale(R):
     cfg = R.IndexConfig.make(1, 8, 4, 131072)
     d = R.default_budgets(R.geometry(cfg).clusters)
     assert R.decode_workspace_bytes(cfg, d) < 8 << 20
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 1, 8192 + 68), (2, 3, 20000), (1, 8, 131072)])
+def test_build_workspace_holds_every_array(R, B, H, N):
+    """The build workspace is at least the sum of the arrays the build uses
+    (sizes written out from their shapes): fp32 and bf16 centroids, the
+    ||mu||^2 operand tiles, the per-unit maxima, sizes, labels, key norms,
+    the fix-up queue (one 20-byte entry per key), the sorted member lists,
+    their cluster starts and the per-centroid error terms."""
+    g = R.geometry(R.IndexConfig.make(B, H, 4, N))
+    BH, C, M = B * H, g.clusters, N - 68
+    S = -(-M // 8192)
+    need = (BH * C * 128 * 4 + BH * C * 128 * 2 + BH * S * 512 * 16 * 2 + BH * S * 2 * 4
+            + BH * C * 4 + BH * M * 4 + BH * M * 4 + BH * M * 20 + BH * M * 4
+            + BH * S * 513 * 4 + BH * S * 512 * 8)
+    assert R.build_workspace_bytes(R.IndexConfig.make(B, H, 4, N)) >= need

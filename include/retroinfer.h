@@ -287,6 +287,20 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
                         int32_t* n_fetch, ri_copy_desc* admit, int32_t admit_cap,
                         int32_t* n_admit, ri_cache_stats* stats);
 
+/* Rows of the execution buffer one step can need, per unit: the sum of the
+ * k_retrieval largest cluster sizes (the retrieval zone is the k_retrieval
+ * top-scoring clusters, "KV缓存技术与RetroInfer系统在长上下文推理中的优化实践"
+ * (framerc.cn) §2.2 execution buffer / §2.1 retrieval zone).  Host planning
+ * for the buffer's allocation, made once per index and budget:
+ *   counts  int32 [units][clusters], host memory (the index's sizes copied
+ *           back); every entry >= 0
+ *   out     int32 [units], host memory, written on success
+ * k_retrieval >= clusters sums every size; 0 gives 0.  RI_ERR_INVALID_ARG for
+ * NULL pointers, units < 1, clusters < 1, k_retrieval < 0 or a negative size
+ * (out untouched); RI_ERR_CAPACITY when a sum exceeds INT32_MAX. */
+ri_status ri_max_retrieval_rows(const int32_t* counts, int32_t units, int32_t clusters,
+                                int32_t k_retrieval, int32_t* out);
+
 /* Buffers of the gather: bf16 [units][rows][128] each, dense.
  *  host_K, host_V   the index's Kp, Vp in pinned (page-locked) host memory,
  *                   rows = M; read by the device through unified addressing.

@@ -16,7 +16,7 @@ _EXPORTS = (
     "build_workspace_bytes", "decode", "decode_workspace_bytes", "default_budgets", "geometry",
     "lib", "read_device_status", "select_clusters", "selftest_wait_timeout", "decode_static",
     "STATIC_SCRATCH_BYTES", "BlockCache", "CopyDesc", "gather_blocks", "SRC_HOST", "SRC_CACHE",
-    "SRC_EXEC", "DST_EXEC", "DST_CACHE")
+    "SRC_EXEC", "DST_EXEC", "DST_CACHE", "max_retrieval_rows")
 
 __all__ = list(_EXPORTS)
 

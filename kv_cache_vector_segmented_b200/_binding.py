@@ -144,6 +144,8 @@ lib.ri_cache_plan.restype = ctypes.c_int
 lib.ri_cache_plan.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp,
                               ctypes.c_int32, _vp, ctypes.c_int32, _P(ctypes.c_int32), _vp,
                               ctypes.c_int32, _P(ctypes.c_int32), _P(CacheStats)]
+lib.ri_max_retrieval_rows.restype = ctypes.c_int
+lib.ri_max_retrieval_rows.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
 lib.ri_gather_blocks.restype = ctypes.c_int
 lib.ri_gather_blocks.argtypes = [_P(GatherBuffers), _vp, ctypes.c_int32, _vp, _vp]
 
@@ -466,6 +468,18 @@ class BlockCache:
 
     def __del__(self):
         self.close()
+
+
+def max_retrieval_rows(counts: np.ndarray, k_retrieval: int) -> np.ndarray:
+    """ri_max_retrieval_rows on host sizes int32 [units][C]: per unit the sum
+    of the k_retrieval largest sizes (rows of the execution buffer)."""
+    cnt = np.ascontiguousarray(counts, dtype=np.int32)
+    cnt = cnt.reshape(-1, cnt.shape[-1])
+    out = np.zeros(cnt.shape[0], dtype=np.int32)
+    check(lib.ri_max_retrieval_rows(cnt.ctypes.data, cnt.shape[0], cnt.shape[1], k_retrieval,
+                                    out.ctypes.data),
+          "ri_max_retrieval_rows")
+    return out
 
 
 def gather_blocks(desc: torch.Tensor, host_K: torch.Tensor, host_V: torch.Tensor,

@@ -5,6 +5,8 @@
 // cluster -> blocks, the LRU order of resident clusters and a stack of free
 // blocks.  ri_cache_plan turns one step's retrieval clusters into copy
 // descriptors for ri_gather_blocks.
+#include <algorithm>
+#include <functional>
 #include <iterator>
 #include <list>
 #include <new>
@@ -246,6 +248,44 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
   *n_fetch = (int32_t)f.size();
   *n_admit = (int32_t)a.size();
   if (stats) *stats = st;
+  return RI_OK;
+}
+
+ri_status ri_max_retrieval_rows(const int32_t* counts, int32_t units, int32_t clusters,
+                                int32_t k_retrieval, int32_t* out) {
+  if (!counts || !out || units < 1 || clusters < 1 || k_retrieval < 0) {
+    ri::set_error("max_retrieval_rows: NULL pointer or bad sizes (units %d, clusters %d, k %d)",
+                  units, clusters, k_retrieval);
+    return RI_ERR_INVALID_ARG;
+  }
+  const size_t total = (size_t)units * clusters;
+  for (size_t i = 0; i < total; ++i) {
+    if (counts[i] < 0) {
+      ri::set_error("max_retrieval_rows: negative cluster size at entry %zu", i);
+      return RI_ERR_INVALID_ARG;
+    }
+  }
+  const int k = k_retrieval < clusters ? k_retrieval : clusters;
+  std::vector<int32_t> row, res((size_t)units);
+  try {
+    row.resize((size_t)clusters);
+  } catch (...) {
+    ri::set_error("max_retrieval_rows: out of host memory");
+    return RI_ERR_HOST;
+  }
+  for (int32_t u = 0; u < units; ++u) {
+    std::copy(counts + (size_t)u * clusters, counts + (size_t)(u + 1) * clusters, row.begin());
+    if (k > 0 && k < clusters)
+      std::nth_element(row.begin(), row.begin() + (k - 1), row.end(), std::greater<int32_t>());
+    long long sum = 0;
+    for (int i = 0; i < k; ++i) sum += row[(size_t)i];
+    if (sum > 0x7fffffffLL) {
+      ri::set_error("max_retrieval_rows: unit %d needs %lld rows", u, sum);
+      return RI_ERR_CAPACITY;
+    }
+    res[(size_t)u] = (int32_t)sum;
+  }
+  std::copy(res.begin(), res.end(), out);
   return RI_OK;
 }
 

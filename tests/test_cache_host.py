@@ -169,3 +169,25 @@ def test_cache_create_rejects_bad_config():
         R.BlockCache(1, 0, 8)
     with pytest.raises(R.RIError):
         R.BlockCache(1, 4, 0)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_max_retrieval_rows_matches_sorted_sums(seed):
+    """Sum of the k largest sizes per unit, against a full sort."""
+    rng = np.random.default_rng(seed)
+    counts = rng.integers(0, 60, size=(5, 300)).astype(np.int32)
+    counts[2] = 0                      # a unit with only empty clusters
+    counts[3, ::7] = 200               # ties among the largest
+    for k in (0, 1, 5, 147, 299, 300, 1000):
+        want = np.sort(counts, axis=1)[:, ::-1][:, :k].sum(axis=1)
+        np.testing.assert_array_equal(R.max_retrieval_rows(counts, k), want)
+
+
+def test_max_retrieval_rows_rejects_bad_input():
+    with pytest.raises(R.RIError):
+        R.max_retrieval_rows(np.array([[3, -1, 2]], dtype=np.int32), 2)
+    with pytest.raises(R.RIError):
+        R.max_retrieval_rows(np.array([[3, 1, 2]], dtype=np.int32), -1)
+    big = np.full((1, 3), 2 ** 30, dtype=np.int32)
+    with pytest.raises(R.RIError):
+        R.max_retrieval_rows(big, 3)   # 3 * 2^30 rows do not fit an int32

@@ -124,10 +124,17 @@ def _traffic_from_profiles(kernel_src: str):
     return None, sha
 
 
+def _segment_sizes(geom, seg_len=8192, clusters=512):
+    """(tokens, clusters) of each 8K segment of the middle tokens, from the
+    library's own geometry (the seeded initial positions need them)."""
+    M = geom.middle
+    return [(min(seg_len, M - s * seg_len), min(clusters, M - s * seg_len))
+            for s in range(geom.num_segments)]
+
+
 # --------------------------------------------------------------------- ours
 def run_ours(args, ws_n, rank, local):
     import kv_cache_vector_segmented_b200 as R
-    import oracle as O
     from kv_cache_vector_segmented_b200.shard import max_over_ranks
 
     dev = torch.device("cuda", local)
@@ -139,9 +146,9 @@ def run_ours(args, ws_n, rank, local):
 
     # ---- inputs: one 128K-token layer, seeded per rank
     kv = S.make_kv(B, H, N, seed=1000 * rank)
-    m0, M = O.middle_range(N)
-    segs = O.segments(M)
-    ip = S.init_positions([s[1] for s in segs], [s[2] for s in segs], B, H, seed=1000 * rank + 3)
+    M = geom.middle
+    segs = _segment_sizes(geom)
+    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B, H, seed=1000 * rank + 3)
     Kd, Vd = kv.K.to(dev), kv.V.to(dev)
     ipd = torch.from_numpy(ip).to(dev)
 
@@ -437,13 +444,11 @@ def run_profile_case():
     128K-token layer of the benchmark geometry (about 1.1 GB on the device),
     one index build (10 k-means iterations) and 6 decode calls."""
     import kv_cache_vector_segmented_b200 as R
-    import oracle as O
     dev = torch.device("cuda", 0)
     cfg = R.IndexConfig.make(B, H, G, N, iters=10)
     kv = S.make_kv(B, H, N, seed=0)
-    m0, M = O.middle_range(N)
-    segs = O.segments(M)
-    ip = S.init_positions([s[1] for s in segs], [s[2] for s in segs], B, H, seed=3)
+    segs = _segment_sizes(R.geometry(cfg))
+    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B, H, seed=3)
     idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
     q = S.make_queries(kv, G, seed=10).to(dev)
     dcfg = R.default_budgets(idx.geom.clusters)

@@ -460,6 +460,94 @@ def run_profile_case():
     print("profile case done", flush=True)
 
 
+def run_cfg5():
+    """Llama3-8B-1048K geometry, batch 1, 1M-token context: K/V rows in pinned
+    host memory, a GPU block cache of 5 % of each head's 2 KB blocks (LRU),
+    64 decode steps with drifting queries.  Each step: selection on the
+    device, the cache plan on the host, the gather of hits (cache) and misses
+    (host) into the execution buffer, admission of the misses, attention.
+    Wall-clock per step (the host plan and the step's sync are part of the
+    synchronous access path); the gather of the fetch list is also timed
+    with CUDA events for the host-link rate."""
+    import kv_cache_vector_segmented_b200 as R
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B5, H5, G5, N5 = 1, 8, 4, 1 << 20
+    steps, warm = 64, 3
+    cfg = R.IndexConfig.make(B5, H5, G5, N5, iters=10)
+    geom = R.geometry(cfg)
+    kv = S.make_kv(B5, H5, N5, seed=0)
+    segs = _segment_sizes(geom)
+    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B5, H5, seed=3)
+    idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
+    torch.cuda.synchronize()
+    del kv.K, kv.V  # the host copy that matters from here on is the permuted one
+    C = geom.clusters
+    d = R.default_budgets(C)
+    k_r = d.k_retrieval
+    hK = idx.Kp.cpu().pin_memory()
+    hV = idx.Vp.cpu().pin_memory()
+    counts = idx.counts.cpu().numpy().reshape(B5 * H5, C)
+    offsets = idx.offsets.cpu().numpy().reshape(B5 * H5, C + 1)
+    br = 8
+    blocks = (counts.astype(np.int64) + br - 1) // br
+    cache = R.BlockCache(B5 * H5, max(1, int(0.05 * blocks.sum(axis=1).max())), br)
+    cK = torch.zeros((B5, H5, cache.pool_rows, 128), dtype=torch.bfloat16, device=dev)
+    cV = torch.zeros_like(cK)
+    exec_rows = int(R.max_retrieval_rows(counts, k_r).max())
+    eK = torch.empty((B5, H5, exec_rows, 128), dtype=torch.bfloat16, device=dev)
+    eV = torch.empty_like(eK)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, d), dev)
+    gws = R.alloc_workspace(256, dev)
+    out = torch.empty((B5, H5 * G5, 128), dtype=torch.bfloat16, device=dev)
+    qs = [q.contiguous().to(dev) for q in
+          S.drift_queries(S.make_queries(kv, G5, seed=52), warm + steps, seed=53)]
+    hit_rows = miss_rows = 0
+    gather_ms = 0.0
+    t0 = time.perf_counter()
+    for i, qd in enumerate(qs):
+        if i == warm:
+            torch.cuda.synchronize()
+            hit_rows = miss_rows = 0
+            gather_ms = 0.0
+            t0 = time.perf_counter()
+        sel, _ = R.select_clusters(qd, idx, d, ws)
+        fetch, admit, st = cache.plan(sel.cpu().numpy().reshape(B5 * H5, -1), k_r, counts,
+                                      offsets)
+        hit_rows += st["hit_rows"]
+        miss_rows += st["miss_rows"]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fd = torch.from_numpy(fetch).to(dev)
+        e0.record()
+        R.gather_blocks(fd, hK, hV, eK, eV, gws, cK, cV)
+        e1.record()
+        R.gather_blocks(torch.from_numpy(admit).to(dev), hK, hV, eK, eV, gws, cK, cV)
+        R.attend_selected(qd, idx, d, ws, exec_K=eK, exec_V=eV, out=out)
+        e1.synchronize()
+        gather_ms += e0.elapsed_time(e1)
+    torch.cuda.synchronize()
+    wall_s = time.perf_counter() - t0
+    status = max(R.read_device_status(ws), R.read_device_status(gws))
+    cache.close()
+    host_bytes = miss_rows * 2 * 128 * 2  # K and V rows of the misses, bf16
+    return {
+        "leg": "config 5", "metric": "decode steps/s with K/V in host memory", "unit": "steps/s",
+        "value": steps / wall_s, "ms_per_step": 1e3 * wall_s / steps, "steps": steps,
+        "warmup": warm, "n_gpus": 1, "data": "synthetic",
+        "config": {"workload": "llama3-8b-1048k decode, 1M context, batch 1, 32 q / 8 kv heads, "
+                               "K/V rows in pinned host memory, 5 % LRU block cache per head",
+                   "clusters_per_head": C, "k_retrieval": k_r, "k_estimation": d.k_estimation,
+                   "cache_blocks_per_head": cache.cfg.blocks_per_unit, "exec_rows": exec_rows,
+                   "timing": "wall clock per step, host plan and the step's device sync "
+                             "included; fetch gather by CUDA events"},
+        "hit_rate_rows": hit_rows / max(1, hit_rows + miss_rows),
+        "host_bytes_per_step": host_bytes / steps,
+        "fetch_gather_ms_per_step": gather_ms / steps,
+        "host_link_gbs": host_bytes / max(1e-9, gather_ms * 1e-3) / 1e9,
+        "device_status": int(status),
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -469,9 +557,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
                     help="run only the small case used for ncu captures")
+    ap.add_argument("--cfg5", action="store_true",
+                    help="run only the 1M-token host-memory leg (block cache, gather, "
+                         "attention) and print its own JSON line")
     args = ap.parse_args()
     if args.ncu_case:
         run_profile_case()
+        return
+    if args.cfg5:
+        print(json.dumps(run_cfg5()), flush=True)
         return
     if args.warmup < 3:
         args.warmup = 3

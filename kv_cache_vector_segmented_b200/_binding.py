@@ -429,6 +429,11 @@ class BlockCache:
         self._h = h
         self._destroy = lib.ri_cache_destroy  # still reachable at interpreter exit
 
+    def _grow(self, cap: int) -> None:
+        self._out_cap = cap
+        self._fetch = np.empty((cap, 6), dtype=np.int32)
+        self._admit = np.empty((cap, 6), dtype=np.int32)
+
     @property
     def pool_rows(self) -> int:
         return self.cfg.blocks_per_unit * self.cfg.block_rows
@@ -442,22 +447,24 @@ class BlockCache:
         cnt = np.ascontiguousarray(counts, dtype=np.int32).reshape(self.cfg.units, -1)
         off = np.ascontiguousarray(offsets, dtype=np.int32).reshape(self.cfg.units, -1)
         C = cnt.shape[1]
-        # copies per requested cluster <= blocks of it, each <= 16 rows
-        req = sel[:, :k_retrieval]
-        n = np.where(req >= 0, np.take_along_axis(cnt, np.clip(req, 0, C - 1), axis=1), 0)
-        n = np.maximum(n, 0)
-        br = self.cfg.block_rows
-        per = (n.astype(np.int64) + br - 1) // br * ((br + 15) // 16) + (n + 15) // 16
-        cap = int(per.sum()) + 1
-        fetch = np.zeros((cap, 6), dtype=np.int32)
-        admit = np.zeros((cap, 6), dtype=np.int32)
+        # output lists reused across steps (the library writes every entry it
+        # reports; the used prefixes are copied out below).  A list that would
+        # overflow makes the library refuse with RI_ERR_CAPACITY and leave its
+        # state unchanged: grow and plan again.
+        if getattr(self, "_out_cap", 0) < 1:
+            self._grow(max(1024, 4 * self.cfg.units * max(1, k_retrieval)))
         nf, na = ctypes.c_int32(0), ctypes.c_int32(0)
         st = CacheStats()
-        check(lib.ri_cache_plan(self._h, sel.ctypes.data, sel.shape[1], k_retrieval,
-                                cnt.ctypes.data, off.ctypes.data, C, fetch.ctypes.data, cap,
-                                ctypes.byref(nf), admit.ctypes.data, cap, ctypes.byref(na),
-                                ctypes.byref(st)),
-              "ri_cache_plan")
+        while True:
+            rc = lib.ri_cache_plan(self._h, sel.ctypes.data, sel.shape[1], k_retrieval,
+                                   cnt.ctypes.data, off.ctypes.data, C, self._fetch.ctypes.data,
+                                   self._out_cap, ctypes.byref(nf), self._admit.ctypes.data,
+                                   self._out_cap, ctypes.byref(na), ctypes.byref(st))
+            if rc != STATUS_CODES["RI_ERR_CAPACITY"]:
+                break
+            self._grow(2 * self._out_cap)
+        check(rc, "ri_cache_plan")
+        fetch, admit = self._fetch, self._admit
         stats = {f: getattr(st, f) for f, _ in CacheStats._fields_}
         return fetch[:nf.value].copy(), admit[:na.value].copy(), stats
 

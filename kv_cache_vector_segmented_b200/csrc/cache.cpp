@@ -2,15 +2,14 @@
 // "KV缓存技术与RetroInfer系统在长上下文推理中的优化实践" (framerc.cn) §2.2 wave
 // buffer: mapping table + LRU replacement, synchronous access path; §3.1:
 // fixed physical blocks of 8 rows x 128 bf16).  Per unit: a mapping table
-// cluster -> blocks, the LRU order of resident clusters and a stack of free
-// blocks.  ri_cache_plan turns one step's retrieval clusters into copy
-// descriptors for ri_gather_blocks.
+// cluster -> chain of blocks, the LRU order of resident clusters and a stack
+// of free blocks, all as flat arrays indexed by cluster id or block id (one
+// step touches each requested cluster in O(1) plus its blocks).
+// ri_cache_plan turns one step's retrieval clusters into copy descriptors
+// for ri_gather_blocks.
 #include <algorithm>
 #include <functional>
-#include <iterator>
-#include <list>
 #include <new>
-#include <unordered_map>
 #include <vector>
 
 #include "internal.h"
@@ -19,16 +18,41 @@ namespace {
 
 constexpr int kChunkRows = 16;  // rows per copy descriptor
 
-struct Entry {
-  std::vector<int> blocks;
-  std::list<int>::iterator pos;  // in the LRU list
+struct Cluster {            // per cluster id
+  int32_t head = -1;       // first block of the cluster's chain, -1 if not resident
+  int32_t nblk = 0;        // blocks in the chain
+  int32_t prev = -1;       // LRU links (-1 at the ends)
+  int32_t next = -1;
+  int32_t in_lru = 0;
 };
 
 struct Unit {
-  std::unordered_map<int, Entry> table;
-  std::list<int> lru;            // least recently used first
-  long long lru_blocks = 0;      // blocks held by the clusters in `lru`
-  std::vector<int> free;         // stack: the next block is free.back()
+  std::vector<Cluster> cl;        // grown to the largest cluster count seen
+  std::vector<int32_t> link;      // per block: next block of the same cluster, -1 at the end
+  std::vector<int32_t> free;      // stack: the next block is free.back()
+  int32_t lru_head = -1, lru_tail = -1;  // least / most recently used
+  long long lru_blocks = 0;       // blocks held by the clusters in the LRU list
+
+  void grow(int32_t clusters) {
+    if ((int32_t)cl.size() < clusters) cl.resize(clusters);
+  }
+  void unlink(int32_t c) {
+    Cluster& x = cl[c];
+    if (x.prev >= 0) cl[x.prev].next = x.next; else lru_head = x.next;
+    if (x.next >= 0) cl[x.next].prev = x.prev; else lru_tail = x.prev;
+    x.prev = x.next = -1;
+    x.in_lru = 0;
+    lru_blocks -= x.nblk;
+  }
+  void push_back(int32_t c) {
+    Cluster& x = cl[c];
+    x.prev = lru_tail;
+    x.next = -1;
+    if (lru_tail >= 0) cl[lru_tail].next = c; else lru_head = c;
+    lru_tail = c;
+    x.in_lru = 1;
+    lru_blocks += x.nblk;
+  }
 };
 
 }  // namespace
@@ -40,20 +64,18 @@ struct ri_cache {
 
 namespace {
 
-// Appends the copies of `rows` rows (src..., dst...) split into chunks.
-bool emit(std::vector<ri_copy_desc>& out, int unit, int src_kind, int src_row, int dst_kind,
-          int dst_row, int rows) {
+// Writes the copies of `rows` rows (src..., dst...) split into chunks.
+inline void emit(ri_copy_desc* out, int32_t* n, int unit, int src_kind, int src_row,
+                 int dst_kind, int dst_row, int rows) {
   for (int r = 0; r < rows; r += kChunkRows) {
-    ri_copy_desc d;
+    ri_copy_desc& d = out[(*n)++];
     d.unit = unit;
     d.src_kind = src_kind;
     d.src_row = src_row + r;
     d.dst_kind = dst_kind;
     d.dst_row = dst_row + r;
     d.n_rows = rows - r < kChunkRows ? rows - r : kChunkRows;
-    out.push_back(d);
   }
-  return true;
 }
 
 }  // namespace
@@ -80,6 +102,7 @@ ri_status ri_cache_create(const ri_cache_config* cfg, ri_cache** out) {
   try {
     c->units.resize(cfg->units);
     for (Unit& u : c->units) {
+      u.link.assign(cfg->blocks_per_unit, -1);
       u.free.reserve(cfg->blocks_per_unit);
       for (int b = cfg->blocks_per_unit - 1; b >= 0; --b) u.free.push_back(b);
     }
@@ -111,8 +134,19 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
   }
   const int br = cache->cfg.block_rows;
   const int nu = cache->cfg.units;
-  // validate every requested id and size first: the state changes only on success
+  try {
+    for (Unit& U : cache->units) U.grow(clusters);
+  } catch (...) {
+    ri::set_error("cache plan: out of host memory");
+    return RI_ERR_HOST;
+  }
+  // one read-only pass: every requested id and size checked, and the exact
+  // fetch copies / admit copies if every miss were admitted counted; the
+  // state changes only when all is valid and both lists fit
+  auto chunks = [](long long rows) { return (rows + kChunkRows - 1) / kChunkRows; };
+  long long nf = 0, na = 0;
   for (int u = 0; u < nu; ++u) {
+    const Unit& U = cache->units[u];
     int prev = -1;
     for (int i = 0; i < k_retrieval; ++i) {
       const int c = sel_ids[(size_t)u * sel_stride + i];
@@ -129,20 +163,8 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         ri::set_error("cache plan: unit %d cluster %d: negative size or row", u, c);
         return RI_ERR_INVALID_ARG;
       }
-    }
-  }
-  // sizing pass (read only): exact fetch copies, admit copies if every miss
-  // were admitted; the state changes only when both lists fit
-  auto chunks = [](long long rows) { return (rows + kChunkRows - 1) / kChunkRows; };
-  long long nf = 0, na = 0;
-  for (int u = 0; u < nu; ++u) {
-    const Unit& U = cache->units[u];
-    for (int i = 0; i < k_retrieval; ++i) {
-      const int c = sel_ids[(size_t)u * sel_stride + i];
-      if (c < 0) break;
-      const int n = counts[(size_t)u * clusters + c];
       if (n == 0) continue;
-      if (U.table.count(c)) {
+      if (U.cl[c].head >= 0) {
         for (long long k = 0; k * br < n; ++k) nf += chunks(n - k * br < br ? n - k * br : br);
       } else {
         nf += chunks(n);
@@ -155,98 +177,80 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
                   nf, na, fetch_cap, admit_cap);
     return RI_ERR_CAPACITY;
   }
-  std::vector<ri_copy_desc> f, a;
+  int32_t nfo = 0, nao = 0;
   ri_cache_stats st = {0, 0, 0, 0, 0};
-  try {
-    f.reserve((size_t)nf);
-    a.reserve((size_t)na);
-    for (int u = 0; u < nu; ++u) {
-      Unit& U = cache->units[u];
-      std::vector<int> ids;
-      for (int i = 0; i < k_retrieval; ++i) {
-        const int c = sel_ids[(size_t)u * sel_stride + i];
-        if (c < 0) break;
-        ids.push_back(c);
+  for (int u = 0; u < nu; ++u) {
+    Unit& U = cache->units[u];
+    const int32_t* sel = sel_ids + (size_t)u * sel_stride;
+    const int32_t* cnt = counts + (size_t)u * clusters;
+    const int32_t* off = offsets + (size_t)u * (clusters + 1);
+    int nid = 0;
+    while (nid < k_retrieval && sel[nid] >= 0) ++nid;
+    // lookup before any admission; requested resident clusters leave the
+    // LRU list for the step (they cannot be evicted by it), so the next
+    // victim is always the list's head
+    for (int i = 0; i < nid; ++i)
+      if (U.cl[sel[i]].in_lru) U.unlink(sel[i]);
+    int run = 0;  // execution-buffer row of the next cluster
+    for (int i = 0; i < nid; ++i) {
+      const int c = sel[i], n = cnt[c];
+      const int erow = run;
+      run += n;
+      if (n == 0) {
+        ++st.hit_clusters;
+        continue;
       }
-      auto rows_of = [&](int c) { return counts[(size_t)u * clusters + c]; };
-      auto first_row = [&](int c) { return offsets[(size_t)u * (clusters + 1) + c]; };
-      // lookup before any admission; requested resident clusters leave the
-      // LRU list for the step (they cannot be evicted by it), so the next
-      // victim is always the list's front
-      std::vector<char> hit(ids.size());
-      std::vector<int> erow(ids.size());
-      int run = 0;
-      for (size_t i = 0; i < ids.size(); ++i) {
-        erow[i] = run;
-        run += rows_of(ids[i]);
-        auto it = U.table.find(ids[i]);
-        hit[i] = rows_of(ids[i]) == 0 || it != U.table.end();
-        if (it != U.table.end()) {
-          U.lru.erase(it->second.pos);
-          U.lru_blocks -= (long long)it->second.blocks.size();
-        }
-      }
-      for (size_t i = 0; i < ids.size(); ++i) {
-        const int c = ids[i], n = rows_of(c);
-        if (n == 0) {
-          ++st.hit_clusters;
-          continue;
-        }
-        if (hit[i]) {
-          ++st.hit_clusters;
-          st.hit_rows += n;
-          const std::vector<int>& bl = U.table[c].blocks;
-          for (size_t k = 0; k < bl.size(); ++k) {
-            const int rows = n - (int)k * br < br ? n - (int)k * br : br;
-            emit(f, u, RI_SRC_CACHE, bl[k] * br, RI_DST_EXEC, erow[i] + (int)k * br, rows);
-          }
-          continue;
-        }
-        ++st.miss_clusters;
-        st.miss_rows += n;
-        emit(f, u, RI_SRC_HOST, first_row(c), RI_DST_EXEC, erow[i], n);
-        const int need = (n + br - 1) / br;
-        if ((long long)U.free.size() + U.lru_blocks < need) {
-          // cannot fit even after every eviction: served uncached, nothing evicted
-          ++st.uncached_clusters;
-          continue;
-        }
-        while ((int)U.free.size() < need) {
-          const int v = U.lru.front();
-          U.lru.pop_front();
-          std::vector<int>& vb = U.table[v].blocks;
-          U.lru_blocks -= (long long)vb.size();
-          U.free.insert(U.free.end(), vb.begin(), vb.end());
-          U.table.erase(v);
-        }
-        Entry e;
-        for (int k = 0; k < need; ++k) {
-          e.blocks.push_back(U.free.back());
-          U.free.pop_back();
-        }
-        for (int k = 0; k < need; ++k) {
+      Cluster& x = U.cl[c];
+      if (x.head >= 0) {
+        ++st.hit_clusters;
+        st.hit_rows += n;
+        int k = 0;
+        for (int b = x.head; b >= 0; b = U.link[b], ++k) {
           const int rows = n - k * br < br ? n - k * br : br;
-          emit(a, u, RI_SRC_EXEC, erow[i] + k * br, RI_DST_CACHE, e.blocks[k] * br, rows);
+          emit(fetch, &nfo, u, RI_SRC_CACHE, b * br, RI_DST_EXEC, erow + k * br, rows);
         }
-        U.table.emplace(c, std::move(e));
+        continue;
       }
-      // requested resident clusters become most recent, in request order
-      for (int c : ids) {
-        auto it = U.table.find(c);
-        if (it == U.table.end()) continue;
-        U.lru.push_back(c);
-        U.lru_blocks += (long long)it->second.blocks.size();
-        it->second.pos = std::prev(U.lru.end());
+      ++st.miss_clusters;
+      st.miss_rows += n;
+      emit(fetch, &nfo, u, RI_SRC_HOST, off[c], RI_DST_EXEC, erow, n);
+      const int need = (n + br - 1) / br;
+      if ((long long)U.free.size() + U.lru_blocks < need) {
+        // cannot fit even after every eviction: served uncached, nothing evicted
+        ++st.uncached_clusters;
+        continue;
       }
+      while ((int)U.free.size() < need) {
+        const int v = U.lru_head;
+        U.unlink(v);
+        Cluster& y = U.cl[v];
+        for (int b = y.head; b >= 0;) {
+          const int nb = U.link[b];
+          U.link[b] = -1;
+          U.free.push_back(b);
+          b = nb;
+        }
+        y.head = -1;
+        y.nblk = 0;
+      }
+      int last = -1;
+      for (int k = 0; k < need; ++k) {
+        const int b = U.free.back();
+        U.free.pop_back();
+        if (last < 0) x.head = b; else U.link[last] = b;
+        U.link[b] = -1;
+        last = b;
+        const int rows = n - k * br < br ? n - k * br : br;
+        emit(admit, &nao, u, RI_SRC_EXEC, erow + k * br, RI_DST_CACHE, b * br, rows);
+      }
+      x.nblk = need;
     }
-  } catch (...) {
-    ri::set_error("cache plan: out of host memory");
-    return RI_ERR_HOST;
+    // requested resident clusters become most recent, in request order
+    for (int i = 0; i < nid; ++i)
+      if (U.cl[sel[i]].head >= 0) U.push_back(sel[i]);
   }
-  for (size_t i = 0; i < f.size(); ++i) fetch[i] = f[i];
-  for (size_t i = 0; i < a.size(); ++i) admit[i] = a[i];
-  *n_fetch = (int32_t)f.size();
-  *n_admit = (int32_t)a.size();
+  *n_fetch = nfo;
+  *n_admit = nao;
   if (stats) *stats = st;
   return RI_OK;
 }

@@ -512,8 +512,9 @@ def run_cfg5():
             gather_ms = 0.0
             t0 = time.perf_counter()
         sel, _ = R.select_clusters(qd, idx, d, ws)
-        fetch, admit, st = cache.plan(sel.cpu().numpy().reshape(B5 * H5, -1), k_r, counts,
-                                      offsets)
+        # only the retrieval ids (the first k_r of each unit) go back to the host
+        sel_r = sel.reshape(B5 * H5, -1)[:, :k_r].cpu().numpy()
+        fetch, admit, st = cache.plan(sel_r, k_r, counts, offsets)
         hit_rows += st["hit_rows"]
         miss_rows += st["miss_rows"]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

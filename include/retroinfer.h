@@ -277,7 +277,8 @@ void ri_cache_destroy(ri_cache* cache);
  * requested resident cluster becomes most recent in request order.  Writes
  * the copy plan: `fetch` (cache->exec for hits, host->exec for misses) and
  * `admit` (exec->cache for admitted misses), each split into copies of at
- * most 16 rows; *n_fetch / *n_admit get their lengths.  Fails with
+ * most 16 rows (a cluster's blocks that are adjacent in the pool share one
+ * copy); *n_fetch / *n_admit get their lengths.  Fails with
  * RI_ERR_CAPACITY (state unchanged) when a list would exceed its capacity,
  * RI_ERR_INVALID_ARG for bad pointers, ids or sizes.  Not thread-safe for one
  * cache. */

@@ -78,6 +78,29 @@ inline void emit(ri_copy_desc* out, int32_t* n, int unit, int src_kind, int src_
   }
 }
 
+// Copies of block-sized pieces, merged while both sides stay contiguous and
+// the copy stays within kChunkRows rows.
+struct Runs {
+  ri_copy_desc* out;
+  int32_t* n;
+  int unit, src_kind, dst_kind;
+  int src = 0, dst = 0, rows = 0;
+  void add(int s, int d, int r) {
+    if (rows > 0 && s == src + rows && d == dst + rows && rows + r <= kChunkRows) {
+      rows += r;
+      return;
+    }
+    flush();
+    src = s;
+    dst = d;
+    rows = r;
+  }
+  void flush() {
+    if (rows > 0) emit(out, n, unit, src_kind, src, dst_kind, dst, rows);
+    rows = 0;
+  }
+};
+
 }  // namespace
 
 extern "C" {
@@ -204,11 +227,13 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
       if (x.head >= 0) {
         ++st.hit_clusters;
         st.hit_rows += n;
+        Runs runs{fetch, &nfo, u, RI_SRC_CACHE, RI_DST_EXEC};
         int k = 0;
         for (int b = x.head; b >= 0; b = U.link[b], ++k) {
           const int rows = n - k * br < br ? n - k * br : br;
-          emit(fetch, &nfo, u, RI_SRC_CACHE, b * br, RI_DST_EXEC, erow + k * br, rows);
+          runs.add(b * br, erow + k * br, rows);
         }
+        runs.flush();
         continue;
       }
       ++st.miss_clusters;
@@ -233,6 +258,7 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         y.head = -1;
         y.nblk = 0;
       }
+      Runs runs{admit, &nao, u, RI_SRC_EXEC, RI_DST_CACHE};
       int last = -1;
       for (int k = 0; k < need; ++k) {
         const int b = U.free.back();
@@ -241,8 +267,9 @@ ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_str
         U.link[b] = -1;
         last = b;
         const int rows = n - k * br < br ? n - k * br : br;
-        emit(admit, &nao, u, RI_SRC_EXEC, erow + k * br, RI_DST_CACHE, b * br, rows);
+        runs.add(erow + k * br, b * br, rows);
       }
+      runs.flush();
       x.nblk = need;
     }
     // requested resident clusters become most recent, in request order

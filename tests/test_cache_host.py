@@ -20,6 +20,22 @@ def _chunks(unit, sk, sr, dk, dr, n):
     return [(unit, sk, sr + r, dk, dr + r, min(CHUNK, n - r)) for r in range(0, n, CHUNK)]
 
 
+def _block_copies(unit, sk, dk, pieces):
+    """Copies of a cluster's block-sized pieces (src row, dst row, rows) in
+    order, adjacent pieces merged while the copy stays within CHUNK rows."""
+    out, cur = [], None
+    for s, d, r in pieces:
+        if cur and s == cur[0] + cur[2] and d == cur[1] + cur[2] and cur[2] + r <= CHUNK:
+            cur = (cur[0], cur[1], cur[2] + r)
+            continue
+        if cur:
+            out += _chunks(unit, sk, cur[0], dk, cur[1], cur[2])
+        cur = (s, d, r)
+    if cur:
+        out += _chunks(unit, sk, cur[0], dk, cur[1], cur[2])
+    return out
+
+
 def expected_plan(models, sel, k_r, counts, offsets, br):
     fetch, admit = [], []
     stats = dict(hit_clusters=0, miss_clusters=0, uncached_clusters=0, hit_rows=0, miss_rows=0)
@@ -39,17 +55,17 @@ def expected_plan(models, sel, k_r, counts, offsets, br):
             if c in before:
                 stats["hit_clusters"] += 1
                 stats["hit_rows"] += n
-                for k, b in enumerate(before[c]):
-                    rows = min(br, n - k * br)
-                    fetch += _chunks(u, R.SRC_CACHE, b * br, R.DST_EXEC, erow[c] + k * br, rows)
+                fetch += _block_copies(u, R.SRC_CACHE, R.DST_EXEC,
+                                       [(b * br, erow[c] + k * br, min(br, n - k * br))
+                                        for k, b in enumerate(before[c])])
                 continue
             stats["miss_clusters"] += 1
             stats["miss_rows"] += n
             fetch += _chunks(u, R.SRC_HOST, int(offsets[u, c]), R.DST_EXEC, erow[c], n)
             if c in model.slot_of:
-                for k, b in enumerate(model.slot_of[c]):
-                    rows = min(br, n - k * br)
-                    admit += _chunks(u, R.SRC_EXEC, erow[c] + k * br, R.DST_CACHE, b * br, rows)
+                admit += _block_copies(u, R.SRC_EXEC, R.DST_CACHE,
+                                       [(erow[c] + k * br, b * br, min(br, n - k * br))
+                                        for k, b in enumerate(model.slot_of[c])])
             else:
                 stats["uncached_clusters"] += 1
     return fetch, admit, stats

@@ -328,6 +328,40 @@ def test_empty_clusters_rank_last():
     assert len(set(res["E"]) - set(live)) == max(0, 350 - len(live))
 
 
+# ---------------------------------------------------------------- seeding
+def test_strided_init_golden():
+    """Default seeding floor(j * L / K) against hand-derived positions."""
+    n = 0
+    for r in _golden_rows("strided_init.txt"):
+        kind, rest = r.split(None, 1)
+        if kind == "full":
+            head, vals = rest.split(":")
+            L, K = (int(x) for x in head.split())
+            want = [int(x) for x in vals.split()]
+            assert len(want) == K
+            assert O.strided_init(L, K).tolist() == want
+        else:
+            head, vals = rest.split("@")
+            L, K = (int(x) for x in head.split())
+            got = O.strided_init(L, K)
+            assert len(got) == K
+            for t in vals.split():
+                j, v = (int(x) for x in t.split("="))
+                assert int(got[j]) == v, (L, K, j)
+        n += 1
+    assert n == 6
+
+
+@pytest.mark.parametrize("L,K", [(8124, 512), (300, 64), (513, 512), (16384, 512), (5, 5)])
+def test_strided_init_spacing(L, K):
+    """Seeds are distinct, start at 0, stay inside the segment and are evenly
+    spaced: consecutive gaps are floor(L/K) or ceil(L/K)."""
+    p = O.strided_init(L, K)
+    assert p[0] == 0 and p[-1] < L and len(np.unique(p)) == K
+    gaps = np.diff(p)
+    assert set(gaps.tolist()) <= {L // K, -(-L // K)}
+
+
 # ---------------------------------------------------------------- LRU model
 def test_lru_model_golden_blocks_sequence():
     rows = _golden_rows("lru_blocks_sequence.txt")

@@ -19,13 +19,19 @@
  *    uint16; fp32 = IEEE binary32.  Layouts are dense, row-major, in the order
  *    written ([B][H_kv][N][d] means d fastest).
  *  - Calls that take a stream are asynchronous on it (NULL = legacy default
- *    stream).  Nothing is allocated by these calls; scratch memory is the
- *    caller's workspace, sized by the matching *_workspace() query.
+ *    stream).  The current CUDA device must be the one that holds the
+ *    stream and the tensors of the call.  Nothing is allocated by these
+ *    calls; scratch memory is the caller's workspace, sized by the matching
+ *    *_workspace() query, whose first 256 bytes (the status region) must be
+ *    zero before its first use.
  *  - Invalid arguments are rejected on the host BEFORE any launch: the call
  *    returns an error status and ri_last_error() describes it.
  *  - Failures found on the device (a bounded wait that expired, an index that
  *    was out of range in device-resident input) are written to a status word
- *    at the start of the workspace; ri_read_device_status() reads it.
+ *    at the start of the workspace; ri_read_device_status() reads and clears
+ *    it.  The decode calls never clear it themselves (no extra launch per
+ *    step): the first failure stays recorded until it is read.  The build
+ *    and gather calls clear it when they start.
  *  - head_dim must be 128.  GQA: query head h_q uses KV head h_q / G.
  */
 #ifndef RETROINFER_H_
@@ -146,7 +152,11 @@ typedef struct {
 /* Default budgets for C clusters (round half up of 1.8 % and 23 %). */
 ri_status ri_default_budgets(int32_t clusters, ri_decode_config* out);
 
-/* Bytes of workspace the decode calls need (0 on invalid config). */
+/* Bytes of workspace the decode calls need (0 on invalid or unsupported
+ * config).  The same workspace serves every decode call of the
+ * configuration; it holds the status region, the per-head centroid scores of
+ * the last scoring pass and the selection handed from ri_select_clusters to
+ * ri_attend_selected. */
 size_t ri_decode_workspace(const ri_index_config* cfg, const ri_decode_config* dcfg);
 
 /* One decode step of tripartite attention [P3 abstract; P2 §2.1, §3.3]:
@@ -162,7 +172,11 @@ size_t ri_decode_workspace(const ri_index_config* cfg, const ri_decode_config* d
  * lse      optional fp32 [B][H_kv*G]: natural log of the denominator.
  * sel_ids  optional int32 [B][H_kv][k_r + k_e]: R then E, each in increasing
  *          id order (entries past the clamped sizes are -1).
- * Reads Kp/Vp in place through `offsets`. */
+ * Reads Kp/Vp in place through `offsets`.  One thread-block cluster works on
+ * each (sequence, KV head); C (clusters per sequence and KV head) must be at
+ * most 65536, else RI_ERR_UNSUPPORTED.  A retrieval cluster whose rows fall
+ * outside Kp, or a negative size, is not attended and RI_ERR_INVALID_ARG is
+ * recorded in the status word. */
 ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config* dcfg,
                               const void* q, const ri_index* idx, void* out, float* lse,
                               int32_t* sel_ids, void* workspace, size_t workspace_bytes,
@@ -180,15 +194,19 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
  *  - Returns RI_ERR_CAPACITY when ri_decode_workspace() for (cfg, dcfg)
  *    exceeds RI_STATIC_SCRATCH_BYTES (4 MiB: e.g. one 128K-token sequence
  *    with 8 KV heads fits; batch 16 of 128K does not).
- *  - The first call on a device looks up the array's address (and loads the
- *    module if it is loaded lazily); make one call, or any call that can
- *    fail fast, before capturing a stream into a CUDA graph.
+ *  - The array used is the current device's; the current device must hold
+ *    `stream`, q, out and the index.
+ *  - The first call on a device (and group size) looks up the array's
+ *    address, sets the kernel's attributes and queries how many thread-block
+ *    clusters the device holds (and loads the module if it is loaded
+ *    lazily); make one call, or any call that can fail fast, before
+ *    capturing a stream into a CUDA graph.  Those results are kept in fixed
+ *    tables inside the library: no call allocates device or host memory.
  *  - Every call on a device shares the one array: calls whose executions
  *    overlap (on different streams or from different threads) race and
  *    give wrong results.  Order them on one stream.
- *  - Nothing needs to start at zero: each call clears the status word and
- *    counters it uses (stream-ordered) before its kernel runs.
- * Allocates nothing: no cudaMalloc, no host allocation. */
+ *  - Each call clears the status word (stream-ordered) before its kernel
+ *    runs; nothing else in the array has to start at zero. */
 #define RI_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
 ri_status ri_decode_attention_static(const ri_index_config* cfg, const ri_decode_config* dcfg,
                                      const void* q, const ri_index* idx, void* out, float* lse,
@@ -330,15 +348,34 @@ typedef struct {
 ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
                            int32_t n_desc, void* workspace, ri_stream_t stream);
 
-/* Synchronises `stream` and returns the status word a previous call wrote
- * into `workspace` (RI_OK if no device-side failure was recorded). */
-ri_status ri_read_device_status(const void* workspace, ri_stream_t stream);
+/* Synchronises `stream` and returns the status word previous calls wrote
+ * into `workspace` (RI_OK if no device-side failure was recorded); a failure
+ * read is cleared, so the next read reports only later failures. */
+ri_status ri_read_device_status(void* workspace, ri_stream_t stream);
 
 /* Self-test of the bounded device wait: launches one kernel that waits for a
  * flag in `workspace` that nothing sets, giving up after `limit_ns`
  * nanoseconds and recording RI_ERR_TIMEOUT in the status word.  workspace
  * needs 256 bytes. */
 ri_status ri_selftest_wait_timeout(void* workspace, uint64_t limit_ns, ri_stream_t stream);
+
+/* Self-test of the decode kernel's own bounded waits: one ri_decode_attention
+ * step (same arguments, lse and sel_ids not written) with one hand-off inside
+ * the kernel left unreleased and every wait limited to limit_ns nanoseconds
+ * (at most 10 s):
+ *   hand_off 1: the first centroid tile's copy is never issued (the MMA
+ *               issuer's wait expires);
+ *   hand_off 2: the first tile's MMA completion is never signalled (the
+ *               scoring epilogue's wait expires);
+ *   hand_off 3: the first attention chunk's copies are never issued (the
+ *               attention warps' wait expires).
+ * The kernel records RI_ERR_TIMEOUT in the status word, every block returns
+ * after the copies it issued have landed, and the device stays usable; `out`
+ * holds no meaningful result. */
+ri_status ri_selftest_decode_timeout(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                     const void* q, const ri_index* idx, void* out,
+                                     void* workspace, size_t workspace_bytes, int32_t hand_off,
+                                     uint64_t limit_ns, ri_stream_t stream);
 
 const char* ri_status_string(ri_status status);
 /* Description of the last error of the calling thread ("" if none). */

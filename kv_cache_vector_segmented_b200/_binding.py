@@ -107,6 +107,9 @@ lib.ri_read_device_status.restype = ctypes.c_int
 lib.ri_read_device_status.argtypes = [_vp, _vp]
 lib.ri_selftest_wait_timeout.restype = ctypes.c_int
 lib.ri_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
+lib.ri_selftest_decode_timeout.restype = ctypes.c_int
+lib.ri_selftest_decode_timeout.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex),
+                                           _vp, _vp, _sz, ctypes.c_int32, ctypes.c_uint64, _vp]
 
 
 class CopyDesc(ctypes.Structure):
@@ -203,10 +206,13 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device=N
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
-    """Caller-owned scratch for the library, 1024-byte aligned."""
+    """Caller-owned scratch for the library, 1024-byte aligned, with its
+    status region (the first 256 bytes) zeroed."""
     raw = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
     off = (-raw.data_ptr()) % 1024
-    return raw[off:off + nbytes]
+    ws = raw[off:off + nbytes]
+    ws[:min(256, nbytes)].zero_()
+    return ws
 
 
 @dataclasses.dataclass
@@ -354,10 +360,12 @@ def decode_static(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = 
     if device_status is not None:
         _need(device_status, "device_status", torch.int32, (1,), dev)
     cidx = index.c_struct()
-    check(lib.ri_decode_attention_static(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
-                                         ctypes.byref(cidx), out.data_ptr(), _ptr(lse),
-                                         _ptr(sel), _ptr(device_status), _stream(dev)),
-          "ri_decode_attention_static")
+    # the library uses the current device's array: make the index's device current
+    with torch.cuda.device(dev):
+        check(lib.ri_decode_attention_static(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                             ctypes.byref(cidx), out.data_ptr(), _ptr(lse),
+                                             _ptr(sel), _ptr(device_status), _stream(dev)),
+              "ri_decode_attention_static")
     return out, lse, sel
 
 
@@ -407,8 +415,31 @@ def attend_selected(q: torch.Tensor, index: Index, dcfg: DecodeConfig, workspace
 
 
 def read_device_status(workspace: torch.Tensor) -> int:
-    """Synchronises torch's current stream and returns the workspace status."""
+    """Synchronises torch's current stream and returns the workspace status
+    (a failure read is cleared)."""
     return lib.ri_read_device_status(workspace.data_ptr(), _stream(workspace.device))
+
+
+FAULT_SCORE_COPY, FAULT_SCORE_COMMIT, FAULT_ATTEND_COPY = 1, 2, 3
+
+
+def selftest_decode_timeout(q: torch.Tensor, index: Index, dcfg: DecodeConfig,
+                            workspace: torch.Tensor, hand_off: int, limit_ns: int,
+                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """ri_selftest_decode_timeout: one decode step with one hand-off inside
+    the kernel left unreleased and every wait limited to limit_ns."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, H * G, d), dev)
+    if out is None:
+        out = torch.empty((B, H * G, d), dtype=torch.bfloat16, device=dev)
+    cidx = index.c_struct()
+    check(lib.ri_selftest_decode_timeout(ctypes.byref(cfg), ctypes.byref(dcfg), q.data_ptr(),
+                                         ctypes.byref(cidx), out.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel(), hand_off, limit_ns, _stream(dev)),
+          "ri_selftest_decode_timeout")
+    return out
 
 
 def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int) -> None:

@@ -9,8 +9,6 @@
 
 #include <cmath>
 #include <mutex>
-#include <set>
-#include <utility>
 
 #include "internal.h"
 #include "retroinfer.h"
@@ -38,16 +36,22 @@ int num_sms() {
   return n;
 }
 
-cudaError_t set_smem_once(const void* func, int bytes) {
-  static std::mutex mu;
-  static std::set<std::pair<const void*, int>> done;
+namespace {
+constexpr int kMaxDevicesHost = 64;
+std::mutex g_smem_mu;
+bool g_smem_done[kMaxDevicesHost][kSmemSlots];
+}  // namespace
+
+cudaError_t set_smem_once(int slot, const void* func, int bytes) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lk(mu);
-  if (done.count({func, dev})) return cudaSuccess;
+  if (dev < 0 || dev >= kMaxDevicesHost || slot < 0 || slot >= kSmemSlots)
+    return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  if (g_smem_done[dev][slot]) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert({func, dev});
+  if (e == cudaSuccess) g_smem_done[dev][slot] = true;
   return e;
 }
 
@@ -124,46 +128,44 @@ bool make_geometry(const ri_index_config* cfg, Geometry* g) {
   return true;
 }
 
-bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L) {
+ri_status make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L) {
   if (!dcfg) {
     set_error("decode config is NULL");
-    return false;
+    return RI_ERR_INVALID_ARG;
   }
   if (dcfg->k_retrieval < 0 || dcfg->k_estimation < 0) {
     set_error("k_retrieval and k_estimation must be >= 0");
-    return false;
+    return RI_ERR_INVALID_ARG;
   }
   if (dcfg->k_retrieval > kMaxRetrieval) {
     set_error("k_retrieval must be <= %d (got %d)", kMaxRetrieval, dcfg->k_retrieval);
-    return false;
+    return RI_ERR_INVALID_ARG;
   }
   if ((long long)dcfg->k_retrieval + dcfg->k_estimation > (1 << 24)) {
     set_error("k_retrieval + k_estimation too large");
-    return false;
+    return RI_ERR_INVALID_ARG;
   }
   L->k_r = dcfg->k_retrieval;
   L->k_e = dcfg->k_estimation;
   L->kr = L->k_r < g.C ? L->k_r : g.C;
   L->ke = L->k_e < g.C - L->kr ? L->k_e : g.C - L->kr;
+  L->Gp = g.G <= 4 ? 4 : 8;
+  L->CS = 0;  // chosen per device by decode_plan
+  if ((long long)g.C > (long long)kMaxClusterBlocks * kMaxIdsPerBlock) {
+    set_error("%d clusters per (sequence, KV head): the decode kernel handles at most %d", g.C,
+              kMaxClusterBlocks * kMaxIdsPerBlock);
+    return RI_ERR_UNSUPPORTED;
+  }
   const long long BH = g.BH();
-  if (!decode_plan(g, L)) return false;
-  L->off_ctrl = kStatusBytesHost;
-  L->header_bytes = align_up(L->off_ctrl + (size_t)6 * BH * 4, 256);
-  size_t off = L->header_bytes;
-  L->off_rkey = off;
-  off = align_up(off + (size_t)BH * g.C * 4, 256);
+  size_t off = kStatusBytesHost;
   L->off_score = off;
-  off = align_up(off + (size_t)BH * 8 * g.C * 4, 256);
+  off = align_up(off + (size_t)BH * g.C * L->Gp * 4, 256);
   L->off_sel = off;
   off = align_up(off + (size_t)BH * (L->k_r + L->k_e) * 4, 256);
   L->off_rpre = off;
   off = align_up(off + (size_t)BH * (L->k_r + 1) * 4, 256);
-  L->off_rrow = off;
-  off = align_up(off + (size_t)BH * (L->k_r > 0 ? L->k_r : 1) * 4, 256);
-  L->off_part = off;
-  off = align_up(off + (size_t)BH * L->S * g.G * kPartStride * 4, 256);
   L->total = off;
-  return true;
+  return RI_OK;
 }
 
 bool make_build_layout(const Geometry& g, BuildLayout* L) {
@@ -262,7 +264,7 @@ size_t ri_decode_workspace(const ri_index_config* cfg, const ri_decode_config* d
   Geometry g;
   if (!make_geometry(cfg, &g)) return 0;
   DecodeLayout L;
-  if (!make_decode_layout(g, dcfg, &L)) return 0;
+  if (make_decode_layout(g, dcfg, &L) != RI_OK) return 0;
   return L.total;
 }
 
@@ -327,7 +329,8 @@ static ri_status prepare_decode(const ri_index_config* cfg, const ri_decode_conf
                                 const void* q, const ri_index* idx, void* workspace,
                                 size_t workspace_bytes, Geometry* g, DecodeLayout* L) {
   if (!make_geometry(cfg, g)) return RI_ERR_INVALID_ARG;
-  if (!make_decode_layout(*g, dcfg, L)) return RI_ERR_INVALID_ARG;
+  const ri_status ls = make_decode_layout(*g, dcfg, L);
+  if (ls != RI_OK) return ls;
   RI_CHECK(q && aligned16(q), RI_ERR_INVALID_ARG, "q must be non-NULL and 16-byte aligned");
   ri_status st = check_index_pointers(*g, idx, false);
   if (st != RI_OK) return st;
@@ -340,6 +343,9 @@ static ri_status prepare_decode(const ri_index_config* cfg, const ri_decode_conf
 
 static DecodeArgs decode_args(const void* q, const ri_index* idx, void* out, float* lse,
                               int32_t* sel, int32_t* rpre, void* ws) {
+  DecodeArgs a0;
+  a0.wait_ns = kWaitLimitNsHost;
+  a0.fault = RI_FAULT_NONE;
   DecodeArgs a;
   a.q = q;
   a.centroid = idx->centroid;
@@ -358,6 +364,8 @@ static DecodeArgs decode_args(const void* q, const ri_index* idx, void* out, flo
   a.sel_user = sel;
   a.rpre_user = rpre;
   a.ws = static_cast<char*>(ws);
+  a.wait_ns = a0.wait_ns;
+  a.fault = a0.fault;
   return a;
 }
 
@@ -371,11 +379,33 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
   if (st != RI_OK) return st;
   RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
   RI_CHECK(!sel_ids || aligned16(sel_ids), RI_ERR_INVALID_ARG, "sel_ids must be 16-byte aligned");
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, workspace);
-  e = launch_decode(g, L, a, s);
+  cudaError_t e = launch_decode(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return RI_OK;
+}
+
+ri_status ri_selftest_decode_timeout(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                     const void* q, const ri_index* idx, void* out,
+                                     void* workspace, size_t workspace_bytes, int32_t hand_off,
+                                     uint64_t limit_ns, ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  ri_status st = prepare_decode(cfg, dcfg, q, idx, workspace, workspace_bytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  RI_CHECK(hand_off >= RI_FAULT_SCORE_COPY && hand_off <= RI_FAULT_ATTEND_COPY,
+           RI_ERR_INVALID_ARG, "hand_off must be 1, 2 or 3 (got %d)", hand_off);
+  RI_CHECK(limit_ns > 0 && limit_ns <= 10ull * 1000000000ull, RI_ERR_INVALID_ARG,
+           "limit_ns must be in (0, 10 s]");
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a = decode_args(q, idx, out, nullptr, nullptr, nullptr, workspace);
+  a.wait_ns = limit_ns;
+  a.fault = hand_off;
+  cudaError_t e = launch_decode(g, L, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RI_OK;
 }
@@ -387,7 +417,8 @@ ri_status ri_decode_attention_static(const ri_index_config* cfg, const ri_decode
   Geometry g;
   DecodeLayout L;
   if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
-  if (!make_decode_layout(g, dcfg, &L)) return RI_ERR_INVALID_ARG;
+  const ri_status ls = make_decode_layout(g, dcfg, &L);
+  if (ls != RI_OK) return ls;
   RI_CHECK(L.total <= kStaticScratchBytes, RI_ERR_CAPACITY,
            "decode needs %zu bytes of scratch, the static array holds %zu", L.total,
            kStaticScratchBytes);
@@ -400,8 +431,9 @@ ri_status ri_decode_attention_static(const ri_index_config* cfg, const ri_decode
   if (st != RI_OK) return st;
   RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
   RI_CHECK(!sel_ids || aligned16(sel_ids), RI_ERR_INVALID_ARG, "sel_ids must be 16-byte aligned");
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  e = cudaMemsetAsync(ws, 0, L.header_bytes, s);
+  e = cudaMemsetAsync(ws, 0, kStatusBytesHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, out, lse, sel_ids, nullptr, ws);
   e = launch_decode(g, L, a, s);
@@ -423,11 +455,10 @@ ri_status ri_select_clusters(const ri_index_config* cfg, const ri_decode_config*
   if (st != RI_OK) return st;
   RI_CHECK(sel_ids && aligned16(sel_ids), RI_ERR_INVALID_ARG,
            "sel_ids must be non-NULL and 16-byte aligned");
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, nullptr, nullptr, sel_ids, retr_rows, workspace);
-  e = launch_select(g, L, a, s);
+  cudaError_t e = launch_select(g, L, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return RI_OK;
 }
@@ -448,15 +479,13 @@ ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config*
              "exec buffers must be 16-byte aligned");
     RI_CHECK(exec_rows >= 1, RI_ERR_INVALID_ARG, "exec_rows must be >= 1");
   }
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // keeps the selection; clears only the status word and the counters
-  cudaError_t e = cudaMemsetAsync(workspace, 0, L.header_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   DecodeArgs a = decode_args(q, idx, out, lse, nullptr, nullptr, workspace);
   a.exec_K = exec_K;
   a.exec_V = exec_V;
   a.exec_rows = exec_rows;
-  e = launch_attend(g, L, a, s);
+  cudaError_t e = launch_attend(g, L, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "attend launch");
   return RI_OK;
 }
@@ -497,14 +526,19 @@ ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* de
   return RI_OK;
 }
 
-ri_status ri_read_device_status(const void* workspace, ri_stream_t stream) {
+ri_status ri_read_device_status(void* workspace, ri_stream_t stream) {
   RI_CHECK(workspace, RI_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
-  if (v != RI_OK) set_error("device reported: %s", ri_status_string((ri_status)v));
+  if (v != RI_OK) {
+    set_error("device reported: %s", ri_status_string((ri_status)v));
+    e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status");
+  }
   return (ri_status)v;
 }
 

@@ -1,5 +1,5 @@
-// Tripartite decode attention over the wave index (sm_100a): one persistent,
-// cooperative kernel launch per decode step, one block per SM.
+// Tripartite decode attention over the wave index (sm_100a): one thread-block
+// cluster per unit (one sequence and KV head), one block per SM.
 //
 // Steps (RetroInfer; "KV缓存技术与RetroInfer系统在长上下文推理中的优化实践",
 // framerc.cn, §2.1 zones, §2.2 step 1 index query, §3.3 attention over the
@@ -10,37 +10,50 @@
 //   S5 estimation term    each c in E adds n_c e^{s} / e^{s} Vsum_c
 //   S6 merge              log-sum-exp over the split partials
 //
-// A unit is one (sequence, KV head).  Work flows between blocks through
-// per-unit counters in the workspace; no block ever waits for a block that
-// could be waiting for it, and the cooperative launch keeps every block
-// resident, so the waits below always end (they are bounded in any case).
-//   A) Every block scores 128-centroid tiles t = blockIdx + k gridDim of the
-//      flattened (unit, tile) list on the tensor cores: TMA brings the tile
-//      and the unit's query rows (128-byte swizzle), one thread issues
-//      tcgen05.mma (M = 128 centroids, N = 16 query rows, K = 128), four
-//      warps read the fp32 scores from TMEM, store s and r and fold r into
-//      the unit's key range; a fifth warp counts finished tiles per unit.
-//   B) Block NB - 1 - u ranks unit u's C keys exactly once its tiles are all
-//      scored (value histogram over the key range, exact order inside the
-//      two boundary buckets), writes R and E in id order and the R clusters'
-//      token prefix and first rows, then raises the unit's ready flag.
-//   C) Every block takes (unit, slice) pairs: the unit's steady tokens, R
-//      tokens and E clusters form one item list cut into S equal slices, and
-//      each warp of the block a contiguous run of the slice.  A warp streams
-//      its items through a private ring of shared-memory slots with 16-byte
-//      cp.async copies (the ring's depth in flight) and folds each into one
-//      online-softmax state: a token adds e^{x} v after its logit x, an E
-//      cluster adds n_c e^{s} and e^{s} Vsum_c.  The block combines its warps
-//      into the slice's partial (m, l, o) in the workspace.
-//   D) The block that finishes a unit's last slice (atomic ticket) merges the
-//      S partials by log-sum-exp and writes out and lse.
+// The CS blocks of a cluster share one unit.  Block b owns a contiguous,
+// balanced range of the unit's 128-centroid tiles; the blocks exchange data
+// only through distributed shared memory and the cluster barrier, never
+// through global counters, so no block waits on another cluster.
+//   A) Scoring: TMA brings the block's centroid tiles (128-byte swizzle, a
+//      ring of 4 stages) and the unit's query rows once; one thread issues
+//      tcgen05.mma (M = 128 centroids, N = 16 query rows, K = 128), each tile
+//      into its own TMEM columns; four epilogue warps read the fp32 scores,
+//      keep the keys r_c, sizes and first rows in shared memory and write
+//      the per-head scores s to the workspace (the estimation term reads
+//      them back).
+//   B) Selection, exact, cluster-wide: the key range (barrier 1), a 4096-
+//      bucket value histogram kept in slices across the blocks and filled
+//      by remote reductions (barrier 2), then every block reads the merged
+//      histogram and finds the two boundary buckets (ranks k_r and
+//      k_r + k_e).  The members of a boundary bucket are ranked exactly by
+//      (key desc, id asc): gathered from all blocks when there are few of
+//      them (barrier 3), else by a radix walk over the 32-bit order key and
+//      a final id count (crowded buckets, heavy ties).  Each block lists its
+//      own R clusters (first row, token prefix) and E clusters (id, size) in
+//      id order (barrier 4).
+//   C) Attention: the unit's items (steady tokens, R tokens, E clusters) are
+//      split evenly over the blocks: block b takes an equal share of the
+//      tokens and an equal share of the E clusters, wherever their owners
+//      are.  One producer warp walks the owners' lists and issues bulk
+//      copies (cp.async.bulk) of whole row runs, value-sum rows and scores
+//      into a ring of 8 stages of 30 items; fifteen consumer warps fold
+//      each item into an online-softmax state on CUDA cores, half a warp
+//      per item (16 lanes x 8 dims, warp-shuffle reductions for q.k).  A
+//      token adds e^{x} v after its logit x; an E cluster adds n_c e^{s} to
+//      the denominator and e^{s} Vsum_c to the numerator.
+//   D) Merge: the block's warps are combined in shared memory, every block
+//      writes its partial (max, denominator, numerator) into block 0's
+//      shared memory (barriers 5 and 6) and block 0 merges them by
+//      log-sum-exp into out and lse.
+// Every wait on an mbarrier is bounded; on expiry the block records
+// RI_ERR_TIMEOUT in the status word, stops issuing work, lets the copies it
+// issued land and still takes part in every cluster barrier.
 #include <float.h>
+#include <limits.h>
 #include <math.h>
 #include <string.h>
 
-#include <map>
 #include <mutex>
-#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -50,51 +63,53 @@ namespace ri {
 namespace {
 
 constexpr float kScale = 0.08838834764831845f;  // 1/sqrt(128)
-constexpr int kTileC = 128;          // centroids per MMA tile (M)
-constexpr int kQRows = 16;           // MMA N: query rows (the unit's G, then others)
-constexpr int kStagesA = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale2 = 8.f * kLog2e;  // online softmax: new reference only when the
+                                           // maximum grows by more than e^8
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kConsumers = 15;  // warps 0..14 fold items in step C
+constexpr int kProducer = 15;   // warp 15 issues the copies of step C
+
+constexpr int kTileC = 128;  // centroids per MMA tile (M)
+constexpr int kQRows = 16;   // MMA N: the unit's query rows, then padding
 constexpr uint32_t kTileBytes = kTileC * kHeadDim * 2;  // 32 KB
 constexpr uint32_t kQBytes = kQRows * kHeadDim * 2;     // 4 KB
-constexpr uint32_t kStageBytes = kTileBytes + kQBytes;  // 1024-byte multiple
-constexpr int kNB = 2048;            // value buckets of the selection
-constexpr int kBoundaryCap = 256;    // keys ranked exactly in a boundary bucket
-constexpr int kRound = 8192;         // keys per selection round (all threads)
-constexpr int kMaxWarps = 32;
-constexpr int kRoundItems = 134;      // work items (token or E cluster) per copy round
-constexpr uint32_t kBufBytes = 81920;  // one round: tokens (padded to 16) x 512 B + E x 548 B
-constexpr uint32_t kRegionBytes = 2 * kBufBytes;
-constexpr float kRescale = 8.f;      // online softmax: new reference only when the max
-                                     // grows by more than this (terms stay <= e^8)
-static_assert(kStagesA * kStageBytes <= kRegionBytes, "stages");
-static_assert(16 * 512 + (kRoundItems - 1) * 548 <= (int)kBufBytes &&
-                  (kRoundItems + 15) * 512 <= (int)kBufBytes, "round");
+constexpr int kStagesA = 4;
+constexpr int kMaxTilesPerBlock = kMaxIdsPerBlock / kTileC;  // 32
 
-// Threads per block (registers: up to 128 each).
-template <int G>
-struct Shape {
-  static constexpr int kThreads = 512;
-  static constexpr int kWarps = kThreads / 32;
-  static constexpr int kPer = kRound / kThreads;  // keys per thread and round
-};
+constexpr int kNB = 4096;  // value buckets of the selection histogram
+constexpr int kBPT = kNB / kThreads;
+constexpr int kCand = 256;  // boundary-bucket members ranked directly
+constexpr int kKPT = kMaxIdsPerBlock / kThreads;  // own ids per thread (contiguous)
+
+constexpr int kItems = 30;  // items per chunk of step C
+constexpr uint32_t kStageC = 16384;
+constexpr int kStagesC = 8;
+constexpr uint32_t kOffVRow = kItems * 256;  // V rows of a token chunk
+constexpr uint32_t kOffESc = kItems * 512;   // scores of an estimation chunk
+static_assert(kOffESc + kItems * 32 <= kStageC, "stage");
 
 // Shared memory map (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t kOffRpre = kRegionBytes;                        // int [kMaxRetrieval + 4]
-constexpr uint32_t kOffRrow = kOffRpre + (kMaxRetrieval + 4) * 4;  // int [kMaxRetrieval]
-constexpr uint32_t kOffMisc = kOffRrow + kMaxRetrieval * 4;
-constexpr uint32_t kMiscBytes = 3072;
+constexpr uint32_t kRingBytes = kStagesC * kStageC;
+static_assert(kStagesA * kTileBytes == kRingBytes, "ring");
+constexpr uint32_t kOffQ = kRingBytes;                          // q tile (4 KB)
+constexpr uint32_t kOffKeys = kOffQ + kQBytes;                  // float keys[P], then lists
+constexpr uint32_t kOffMeta = kOffKeys + kMaxIdsPerBlock * 8;   // int2 (first row, size)[P]
+constexpr uint32_t kOffMisc = kOffMeta + kMaxIdsPerBlock * 8;
+constexpr uint32_t kMiscBytes = 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kOffMisc % 16 == 0, "misc alignment");
 
-// Selection scratch inside the region (free outside steps A and C).
-constexpr uint32_t kOffHist = 0;
-constexpr uint32_t kOffCand = kOffHist + kNB * 4;                // [2][kBoundaryCap] u64
-constexpr uint32_t kOffSelCnt = kOffCand + 2 * kBoundaryCap * 8;  // int [kRound]
-constexpr uint32_t kOffSelOff = kOffSelCnt + kRound * 4;          // int [kRound]
-constexpr uint32_t kOffSelE = kOffSelOff + kRound * 4;            // int [kRound]
-constexpr uint32_t kOffSelRid = kOffSelE + kRound * 4;            // int [kMaxRetrieval]
-constexpr uint32_t kOffSelRcnt = kOffSelRid + kMaxRetrieval * 4;  // int [kMaxRetrieval]
-static_assert(kOffSelRcnt + kMaxRetrieval * 4 <= kRegionBytes, "selection scratch");
+// Inside the ring while it is free (between steps A and C, and after C).
+constexpr uint32_t kRHist = 0;                      // int [slice] merged histogram slice
+constexpr uint32_t kRDig = kRHist + kNB * 4;        // int [4 passes][2][256] digit slices
+constexpr uint32_t kRCand = kRDig + 4 * 2 * 256 * 4;  // u64 [2][kCand] own boundary members
+constexpr uint32_t kRAll = kRCand + 2 * kCand * 8;  // u64 [2][kCand] gathered members
+constexpr uint32_t kRRid = kRAll + 2 * kCand * 8;   // u16 [P] own R clusters (local index)
+static_assert(kRRid + kMaxIdsPerBlock * 2 <= kRingBytes, "selection scratch");
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
 
@@ -111,69 +126,111 @@ struct Params {
   float* lse;
   int32_t* sel_user;
   int32_t* rpre_user;
-  float* score;    // ws [BH][C][8]
-  float* rkey;     // ws [BH][C]
-  int32_t* sel;    // ws [BH][k_r + k_e]
-  int32_t* rpre;   // ws [BH][k_r + 1]
-  int32_t* rrow;   // ws [BH][k_r]
-  float* part;     // ws [BH][S][G][kPartStride]
-  int* status;     // ws status word
-  int* done;       // ws [BH] scored tiles
-  int* ready;      // ws [BH] selection published
-  int* ticket;     // ws [BH] finished slices
-  uint32_t* kmax;  // ws [BH] max order key of the finite selection keys
-  uint32_t* kmin;  // ws [BH] max of the complemented order keys (= min key)
-  int* ninf;       // ws [BH] empty clusters (key -inf)
-  int BH, C, M, n_steady, k_r, k_e, kr, ke, S, exec_rows, mode;
-  int nbp;         // blocks that take attention slices (the rest are selectors)
+  float* score;   // ws [BH][C][Gp]
+  int32_t* sel;   // ws [BH][k_r + k_e]
+  int32_t* rpre;  // ws [BH][k_r + 1]
+  int* status;
+  unsigned long long wait_ns;
+  int fault;
+  int BH, C, M, n_steady, k_r, k_e, kr, ke, tiles, exec_rows, mode;
 };
 
 struct Misc {
-  uint64_t full[kStagesA], empty[kStagesA], tfull[2], tempty[2], drain;
+  uint64_t fullA[kStagesA], emptyA[kStagesA], tdone[kMaxTilesPerBlock], qbar, drain;
+  uint64_t fullC[kStagesC], emptyC[kStagesC];
   uint32_t tmem;
   int abort_flag;
-  int epi_done;  // epilogue's finished tiles (step A)
-  int flag;
-  int bucket[2], above[2], ncand[2];
-  uint32_t Tu[2];
-  int Tid[2];
-  int wtot[2][kMaxWarps];
-  int scan[kMaxWarps + 4];
-  float wm[kMaxWarps][8];  // per-warp partial maxima (block combine)
-  float wl[kMaxWarps][8];  // per-warp partial denominators
+  // published to the other blocks of the cluster
+  uint32_t pub_kmax, pub_kmin;
+  int pub_ninf;
+  int pub_ncand[2];
+  int pub_nR, pub_nE, pub_tokR;
+  int pub_idcnt[2];
+  int pub_tid[2];
+  // cluster-wide values every block gathers
+  int nRp[kMaxClusterBlocks + 1], nEp[kMaxClusterBlocks + 1], tokRp[kMaxClusterBlocks + 1];
+  int candp[2][kMaxClusterBlocks + 1];
+  float lo, scale;
+  int nfin, ninf;
+  int bucket[2], above[2], nmem[2], kp[2], slow[2], digit[2], owner[2];
+  unsigned long long thr[2];
+  int ecount[kStagesC][32];
+  int scan[kWarps + 4];
+  int T_R;
+  float wm[kWarps][8], wl[kWarps][8];
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area");
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nrank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Cluster barrier in its non-.aligned form: several call sites follow
+// per-thread loops after which a warp need not have reconverged.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+  cluster_arrive();
+  cluster_wait();
+}
+// Address of the same shared-memory location in block `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_cl_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int2 ld_cl_v2(uint32_t addr) {
+  int2 v;
+  asm volatile("ld.shared::cluster.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_cl_u64(uint32_t addr) {
+  unsigned long long v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cl_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_cl_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Completes `bytes` of an mbarrier's expected transaction count without a copy
+// (a copy that was skipped because its rows were out of range).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        "=r"(r[7])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_cta(const int* p) {
-  int v;
-  asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_cta(int* p, int v) {
-  asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
 __device__ __forceinline__ int ld_volatile(const int* p) {
   return *reinterpret_cast<const volatile int*>(p);
 }
@@ -194,31 +251,6 @@ __device__ __forceinline__ int bucket_of(float r, float lo, float scale) {
   return b < 0 ? 0 : (b >= kNB ? kNB - 1 : b);
 }
 
-// ---- warp-level tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 acc)
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-// d += A . B with A 16x16 row-major (regs a0..a3), B 16x8 column-major (b0, b1)
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
-                                               uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 // 2^x by the hardware approximation (ex2.approx; -inf gives +0)
 __device__ __forceinline__ float ex2f(float x) {
   float y;
@@ -226,73 +258,9 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// The k-th (1-based, from the top) key of value bucket b with its id, by an
-// MSD radix walk over the bucket's keys (for crowded buckets: heavy ties).
-template <int NT>
-__device__ void kth_in_bucket_slow(const float* keys, int C, int b, float lo, float scale, int k,
-                                   Misc* ms, int* hist, uint32_t* Tu, int* Tid) {
-  constexpr int NW = NT / 32;
-  uint32_t prefix = 0, mask = 0;
-  int remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
-    __syncthreads();
-    for (int c = threadIdx.x; c < C; c += NT) {
-      const float r = __ldcg(keys + c);
-      if (bucket_of(r, lo, scale) != b) continue;
-      const uint32_t u = float_order_key(r);
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int cum = 0, dg = 255;
-      for (; dg > 0; --dg) {
-        if (cum + hist[dg] >= remaining) break;
-        cum += hist[dg];
-      }
-      ms->scan[0] = dg;
-      ms->scan[1] = remaining - cum;
-    }
-    __syncthreads();
-    prefix |= (uint32_t)ms->scan[0] << shift;
-    mask |= 255u << shift;
-    remaining = ms->scan[1];
-    __syncthreads();
-  }
-  // the remaining-th smallest id among the bucket's keys equal to prefix
-  if (threadIdx.x == 0) ms->scan[2] = -1;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int run = 0;
-  for (int base = 0; base < C; base += NT) {
-    const int c = base + threadIdx.x;
-    const float r = c < C ? __ldcg(keys + c) : 0.f;
-    const bool eq = c < C && bucket_of(r, lo, scale) == b && float_order_key(r) == prefix;
-    const unsigned mk = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) ms->wtot[0][warp] = __popc(mk);
-    __syncthreads();
-    int before = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      before += w < warp ? ms->wtot[0][w] : 0;
-      tot += ms->wtot[0][w];
-    }
-    const int rank = run + before + __popc(mk & ((1u << lane) - 1u));
-    if (eq && rank == remaining - 1) ms->scan[2] = c;
-    run += tot;
-    __syncthreads();
-  }
-  *Tu = prefix;
-  *Tid = ms->scan[2];
-  __syncthreads();
-}
-
 // Block-wide exclusive prefix of one int per thread (thread order); the
 // block total goes to *total.  One warp scans the per-warp totals.
-template <int NT>
-__device__ __forceinline__ int block_scan(int v, int* scratch /* [NT / 32 + 1] */, int* total) {
-  constexpr int NW = NT / 32;
+__device__ __forceinline__ int block_scan(int v, int* scratch /* [kWarps + 1] */, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -303,19 +271,19 @@ __device__ __forceinline__ int block_scan(int v, int* scratch /* [NT / 32 + 1] *
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int wt = lane < NW ? scratch[lane] : 0;
+    const int wt = lane < kWarps ? scratch[lane] : 0;
     int wi = wt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, wi, off);
       if (lane >= off) wi += t;
     }
-    if (lane < NW) scratch[lane] = wi - wt;
-    if (lane == 31) scratch[NW] = wi;
+    if (lane < kWarps) scratch[lane] = wi - wt;
+    if (lane == 31) scratch[kWarps] = wi;
   }
   __syncthreads();
   const int excl = scratch[warp] + incl - v;
-  *total = scratch[NW];
+  *total = scratch[kWarps];
   __syncthreads();  // scratch is reused by the next scan
   return excl;
 }
@@ -332,323 +300,316 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
   return r != 0;
 }
 
-// Bounded wait of one thread until a counter other blocks raise reaches
-// `target`; gives up early when any block has recorded a failure.
-__device__ bool wait_count(const int* counter, int target, const int* status) {
-  if (ld_acquire(counter) >= target) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (ld_acquire(counter) >= target) return true;
-    if (ld_volatile(status) != 0) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(32);
+// Bounded wait of every lane of a warp (each lane acquires the phase); true
+// only when every lane saw it complete.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long lim) {
+  const bool ok = mbar_wait(bar, parity, lim);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Online-softmax state of one lane: up to four query heads, eight dims each.
+struct Acc {
+  float m[4], l[4], o[4][8];
+};
+
+__device__ __forceinline__ void acc_add(Acc& a, int j, float x, float w_n, const float (&v)[8]) {
+  if (x > a.m[j] + kRescale2) {  // new reference (also the first item)
+    const float c = a.m[j] == -INFINITY ? 0.f : ex2f(a.m[j] - x);
+    a.l[j] *= c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a.o[j][i] *= c;
+    a.m[j] = x;
   }
+  const float pj = ex2f(x - a.m[j]);
+  a.l[j] = fmaf(w_n, pj, a.l[j]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a.o[j][i] = fmaf(pj, v[i], a.o[j][i]);
 }
 
 // ------------------------------------------------------------------ kernel
 template <int G>
-__global__ void __launch_bounds__(Shape<G>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_cent,
                   const __grid_constant__ CUtensorMap tm_q, const Params p) {
-  constexpr int NT = Shape<G>::kThreads;
-  constexpr int NW = Shape<G>::kWarps;
-  constexpr int kPer = Shape<G>::kPer;
+  constexpr int Gp = G <= 4 ? 4 : 8;        // scores stored per cluster
+  constexpr int HPL = G < 4 ? G : 4;        // query heads per lane in step C
+  constexpr int kPasses = G <= 4 ? 1 : 2;   // item passes per chunk and warp in step C
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   Misc* ms = reinterpret_cast<Misc*>(sm + kOffMisc);
-  int32_t* rpre_sm = reinterpret_cast<int32_t*>(sm + kOffRpre);
-  int32_t* rrow_sm = reinterpret_cast<int32_t*>(sm + kOffRrow);
+  float* keys = reinterpret_cast<float*>(sm + kOffKeys);
+  int2* lists = reinterpret_cast<int2*>(sm + kOffKeys);
+  int2* meta = reinterpret_cast<int2*>(sm + kOffMeta);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int CS = (int)cluster_nrank();
+  const int b = (int)cluster_rank();
+  const int u = (int)blockIdx.x / CS;
   const int C = p.C;
-  const int kr = p.kr, ke = p.ke;
-  const int tiles_h = C > 0 ? (C + kTileC - 1) / kTileC : 0;
+  const unsigned long long lim = p.wait_ns;
+  const bool selecting = p.mode != kModeAttend && C > 0;
+  // this block's tiles [t0, t1) of the unit's ceil(C / 128) tiles
+  const int t0 = (int)((long long)p.tiles * b / CS), t1 = (int)((long long)p.tiles * (b + 1) / CS);
+  const int id0 = t0 * kTileC;
+  const int nid = selecting ? max(0, min(C, t1 * kTileC) - id0) : 0;
+  const int ntiles = (nid + kTileC - 1) / kTileC;
+  const uint32_t sm_base = smem_u32(sm);
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     ms->abort_flag = 0;
-    ms->epi_done = 0;
+    ms->pub_kmax = ms->pub_kmin = 0u;
+    ms->pub_ninf = 0;
+    ms->pub_ncand[0] = ms->pub_ncand[1] = 0;
+    ms->pub_idcnt[0] = ms->pub_idcnt[1] = 0;
+    ms->pub_tid[0] = ms->pub_tid[1] = -1;
+    ms->pub_nR = ms->pub_nE = ms->pub_tokR = 0;
+    ms->thr[0] = ms->thr[1] = 0ull;
     for (int i = 0; i < kStagesA; ++i) {
-      mbar_init(&ms->full[i], 1);
-      mbar_init(&ms->empty[i], 1);
+      mbar_init(&ms->fullA[i], 1);
+      mbar_init(&ms->emptyA[i], 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&ms->tfull[h], 1);
-      mbar_init(&ms->tempty[h], 128);
-    }
+    for (int i = 0; i < kMaxTilesPerBlock; ++i) mbar_init(&ms->tdone[i], 1);
+    mbar_init(&ms->qbar, 1);
     mbar_init(&ms->drain, 1);
+    for (int i = 0; i < kStagesC; ++i) {
+      mbar_init(&ms->fullC[i], 1);
+      mbar_init(&ms->emptyC[i], kConsumers);
+    }
     fence_barrier_init();
   }
   __syncthreads();
 
   // ============================================================ step A
-  if (p.mode != kModeAttend && tiles_h > 0) {
-    const int total_tiles = p.BH * tiles_h;
-    const int nt = total_tiles > (int)blockIdx.x
-                       ? (total_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
-                       : 0;
-    if (nt > 0) {
-      if (warp == 1) {
-        tmem_alloc(&ms->tmem, 32);
-        tmem_relinquish();
-      }
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      const uint32_t tmem = ms->tmem;
-      if (warp == 0 && lane == 0) {
-        // TMA producer: centroid tile and the unit's query rows per stage
-        tma_prefetch_desc(&tm_cent);
-        tma_prefetch_desc(&tm_q);
-        int issued[kStagesA] = {0, 0, 0, 0};
-        for (int it = 0; it < nt; ++it) {
-          if (ld_volatile(&ms->abort_flag)) break;
-          const int st = it % kStagesA;
-          if (it >= kStagesA && !mbar_wait(&ms->empty[st], ((it / kStagesA) - 1) & 1)) {
-            record_status(p.status, RI_ERR_TIMEOUT);
-            ms->abort_flag = 1;
-            break;
-          }
-          const int t = (int)blockIdx.x + it * (int)gridDim.x;
-          const int u = t / tiles_h, ti = t - u * tiles_h;
-          uint8_t* stage = sm + st * kStageBytes;
-          mbar_arrive_expect_tx(&ms->full[st], kStageBytes);
-          const int row = u * C + ti * kTileC;
-          for (int kh = 0; kh < 2; ++kh) {
-            tma_load_2d(stage + kh * (kTileC * 128), &tm_cent, kh * 64, row, &ms->full[st]);
-            tma_load_2d(stage + kTileBytes + kh * (kQRows * 128), &tm_q, kh * 64, u * G,
-                        &ms->full[st]);
-          }
-          ++issued[st];
-        }
-        for (int st = 0; st < kStagesA; ++st)
-          if (issued[st]) mbar_wait(&ms->full[st], (uint32_t)((issued[st] - 1) & 1));
-      } else if (warp == 1 && lane == 0) {
-        // MMA issuer: D[128 x 16] = tile[128 x 128] . Q[16 x 128]^T
-        constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileC, kQRows);
-        const uint32_t base = smem_u32(sm);
-        for (int it = 0; it < nt; ++it) {
-          if (ld_volatile(&ms->abort_flag)) break;
-          const int st = it % kStagesA, buf = it & 1;
-          if (!mbar_wait(&ms->full[st], (uint32_t)((it / kStagesA) & 1)) ||
-              (it >= 2 && !mbar_wait(&ms->tempty[buf], (uint32_t)(((it >> 1) - 1) & 1)))) {
-            record_status(p.status, RI_ERR_TIMEOUT);
-            ms->abort_flag = 1;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = base + st * kStageBytes;
-          const uint32_t b_addr = a_addr + kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * (kTileC * 128) + (kk & 3) * 32;
-            const uint32_t boff = (kk >> 2) * (kQRows * 128) + (kk & 3) * 32;
-            umma_bf16(tmem + buf * kQRows, umma_desc_sw128(a_addr + aoff),
-                      umma_desc_sw128(b_addr + boff), idesc, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&ms->empty[st]);
-          umma_commit(&ms->tfull[buf]);
-        }
-        umma_commit(&ms->drain);
-        mbar_wait(&ms->drain, 0);
-      } else if (warp == 2 && lane == 0) {
-        // publisher: counts the epilogue's finished tiles into the units'
-        // tile counters (one gpu-scope fence per batch of tiles)
-        int published = 0;
-        const unsigned long long t0 = globaltimer_ns();
-        while (published < nt) {
-          const int e = ld_acquire_cta(&ms->epi_done);
-          if (e > published) {
-            __threadfence();
-            for (int i = published; i < e; ++i) {
-              const int t = (int)blockIdx.x + i * (int)gridDim.x;
-              atomicAdd(p.done + t / tiles_h, 1);
-            }
-            published = e;
-          } else if (ld_volatile(&ms->abort_flag)) {
-            break;
-          } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            record_status(p.status, RI_ERR_TIMEOUT);
-            ms->abort_flag = 1;
-            break;
-          }
-        }
-      } else if (warp >= 4 && warp < 8) {
-        // epilogue: one centroid per thread; the unit's key range on the side
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;
-        for (int it = 0; it < nt; ++it) {
-          const int buf = it & 1;
-          const int t = (int)blockIdx.x + it * (int)gridDim.x;
-          const int u = t / tiles_h, ti = t - u * tiles_h;
-          const int c = ti * kTileC + r;
-          // issued before the wait so the load overlaps the MMA
-          const int cnt = c < C ? __ldg(p.counts + (size_t)u * C + c) : 0;
-          const bool ok = mbar_wait(&ms->tfull[buf], (uint32_t)((it >> 1) & 1));
-          // the 128 epilogue threads leave together (they share named barrier 1)
-          if (epilogue_any(!ok)) {
-            if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
-            ms->abort_flag = 1;
-            break;
-          }
-          tc_fence_after();
-          float v[16];
-          tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + buf * kQRows, v);
-          tc_fence_before();
-          mbar_arrive(&ms->tempty[buf]);
-          uint32_t kmx = 0, kmn = 0;
-          bool empty = false;
-          if (c < C) {
-            float s[8];
-            float rs = 0.f;
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              s[g] = g < G ? v[g] * kScale : 0.f;
-              if (g < G) rs += s[g];
-            }
-            float4* dst = reinterpret_cast<float4*>(p.score + ((size_t)u * C + c) * 8);
-            dst[0] = make_float4(s[0], s[1], s[2], s[3]);
-            dst[1] = make_float4(s[4], s[5], s[6], s[7]);
-            p.rkey[(size_t)u * C + c] = cnt > 0 ? rs : -INFINITY;
-            if (cnt > 0) {
-              kmx = float_order_key(rs);
-              kmn = ~kmx;
-            } else {
-              empty = true;
-            }
-          }
-          kmx = __reduce_max_sync(0xffffffffu, kmx);
-          kmn = __reduce_max_sync(0xffffffffu, kmn);
-          const int ne = __popc(__ballot_sync(0xffffffffu, empty));
-          if (lane == 0) {
-            if (kmx) atomicMax(p.kmax + u, kmx);
-            if (kmn) atomicMax(p.kmin + u, kmn);
-            if (ne) atomicAdd(p.ninf + u, ne);
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (threadIdx.x == 128) st_release_cta(&ms->epi_done, it + 1);
-        }
-      }
-      __syncwarp();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      if (warp == 1) tmem_dealloc(tmem, 32);
+  if (ntiles > 0) {
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)ntiles * kQRows) ncols <<= 1;
+    if (warp == 1) {
+      tmem_alloc(&ms->tmem, ncols);
+      tmem_relinquish();
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms->tmem;
+    if (warp == 0 && lane == 0) {
+      // TMA producer: the unit's query rows once, then the block's tiles
+      tma_prefetch_desc(&tm_cent);
+      tma_prefetch_desc(&tm_q);
+      mbar_arrive_expect_tx(&ms->qbar, kQBytes);
+      tma_load_2d(sm + kOffQ, &tm_q, 0, u * G, &ms->qbar);
+      tma_load_2d(sm + kOffQ + kQRows * 128, &tm_q, 64, u * G, &ms->qbar);
+      int issued[kStagesA] = {0, 0, 0, 0};
+      for (int it = 0; it < ntiles; ++it) {
+        if (ld_volatile(&ms->abort_flag)) break;
+        const int st = it % kStagesA;
+        if (it >= kStagesA && !mbar_wait(&ms->emptyA[st], ((it / kStagesA) - 1) & 1, lim)) {
+          record_status(p.status, RI_ERR_TIMEOUT);
+          ms->abort_flag = 1;
+          break;
+        }
+        uint8_t* stage = sm + st * kTileBytes;
+        mbar_arrive_expect_tx(&ms->fullA[st], kTileBytes);
+        const int row = u * C + id0 + it * kTileC;
+        if (!(p.fault == RI_FAULT_SCORE_COPY && it == 0)) {
+          tma_load_2d(stage, &tm_cent, 0, row, &ms->fullA[st]);
+          tma_load_2d(stage + kTileC * 128, &tm_cent, 64, row, &ms->fullA[st]);
+        }
+        ++issued[st];
+      }
+      // every copy issued lands before its stage is reused or the block exits
+      for (int st = 0; st < kStagesA; ++st)
+        if (issued[st]) mbar_wait(&ms->fullA[st], (uint32_t)((issued[st] - 1) & 1), lim);
+      mbar_wait(&ms->qbar, 0, lim);
+    } else if (warp == 1 && lane == 0) {
+      // MMA issuer: D[128 x 16] = tile[128 x 128] . Q[16 x 128]^T per tile
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileC, kQRows);
+      const uint32_t qaddr = sm_base + kOffQ;
+      bool ok = mbar_wait(&ms->qbar, 0, lim);
+      if (!ok) {
+        record_status(p.status, RI_ERR_TIMEOUT);
+        ms->abort_flag = 1;
+      }
+      for (int it = 0; ok && it < ntiles; ++it) {
+        if (ld_volatile(&ms->abort_flag)) break;
+        const int st = it % kStagesA;
+        if (!mbar_wait(&ms->fullA[st], (uint32_t)((it / kStagesA) & 1), lim)) {
+          record_status(p.status, RI_ERR_TIMEOUT);
+          ms->abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = sm_base + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (kTileC * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (kQRows * 128) + (kk & 3) * 32;
+          umma_bf16(tmem + it * kQRows, umma_desc_sw128(a_addr + aoff),
+                    umma_desc_sw128(qaddr + boff), idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ms->emptyA[st]);
+        if (!(p.fault == RI_FAULT_SCORE_COMMIT && it == 0)) umma_commit(&ms->tdone[it]);
+      }
+      // the MMAs issued have completed before TMEM is released
+      umma_commit(&ms->drain);
+      if (!mbar_wait(&ms->drain, 0, lim)) {
+        record_status(p.status, RI_ERR_TIMEOUT);
+        ms->abort_flag = 1;
+      }
+    } else if (warp >= 4 && warp < 8) {
+      // epilogue: one centroid per thread
+      const int quad = warp & 3;
+      const int rr = quad * 32 + lane;
+      uint32_t kmx = 0, kmn = 0;
+      int ninf = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int cl = it * kTileC + rr;
+        const bool valid = cl < nid;
+        const size_t gc = (size_t)u * C + id0 + cl;
+        int cnt = 0, off = 0;
+        if (valid) {  // issued before the wait so the loads overlap the MMA
+          cnt = __ldg(p.counts + gc);
+          off = __ldg(p.offsets + (size_t)u * (C + 1) + id0 + cl);
+        }
+        const bool ok = mbar_wait(&ms->tdone[it], 0, lim);
+        if (epilogue_any(!ok)) {  // the 128 threads leave together
+          if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
+          ms->abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        float v[8];
+        tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + it * kQRows, v);
+        if (valid) {
+          float s[Gp];
+          float rs = 0.f;
+#pragma unroll
+          for (int g = 0; g < Gp; ++g) {
+            s[g] = g < G ? v[g] * kScale : 0.f;
+            if (g < G) rs += s[g];
+          }
+          float4* dst = reinterpret_cast<float4*>(p.score + gc * Gp);
+          dst[0] = make_float4(s[0], s[1], s[2], s[3]);
+          if constexpr (Gp == 8) dst[1] = make_float4(s[4], s[5], s[6], s[7]);
+          keys[cl] = cnt > 0 ? rs : -INFINITY;
+          meta[cl] = make_int2(off, cnt);
+          if (cnt > 0) {
+            const uint32_t o = float_order_key(rs);
+            kmx = max(kmx, o);
+            kmn = max(kmn, ~o);
+          } else {
+            ++ninf;
+          }
+        }
+      }
+      kmx = __reduce_max_sync(0xffffffffu, kmx);
+      kmn = __reduce_max_sync(0xffffffffu, kmn);
+      ninf = __reduce_add_sync(0xffffffffu, ninf);
+      if (lane == 0) {
+        atomicMax(&ms->pub_kmax, kmx);
+        atomicMax(&ms->pub_kmin, kmn);
+        atomicAdd(&ms->pub_ninf, ninf);
+      }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, ncols);
+  }
+  __syncthreads();
+  if (ms->abort_flag && nid > 0) {
+    // a failed scoring pass leaves no usable key: the block's clusters are
+    // treated as empty (selected only past every finite key, never attended)
+    for (int i = tid; i < nid; i += kThreads) {
+      keys[i] = -INFINITY;
+      meta[i] = make_int2(0, 0);
+    }
+    if (tid == 0) {
+      ms->pub_kmax = ms->pub_kmin = 0u;
+      ms->pub_ninf = nid;
+    }
+    __syncthreads();
   }
 
   // ============================================================ step B
-  // Exact selection over the C keys of unit u by this block alone.  Keys are
-  // taken in rounds of kRound ids; thread t holds ids round_base + kPer t + j
-  // in registers (16-byte loads).  The key range comes from step A.
-  auto select_unit = [&](int u) {
-    int* hist = reinterpret_cast<int*>(sm + kOffHist);        // [kNB]
-    unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kOffCand);
-    int* cnt_sm = reinterpret_cast<int*>(sm + kOffSelCnt);    // [kRound] sizes of the round
-    int* off_sm = reinterpret_cast<int*>(sm + kOffSelOff);    // [kRound] first rows of the round
-    int* ecomp = reinterpret_cast<int*>(sm + kOffSelE);       // [kRound] E ids of the round
-    int* rid_sm = reinterpret_cast<int*>(sm + kOffSelRid);    // [kMaxRetrieval] R ids
-    int* rcnt_sm = reinterpret_cast<int*>(sm + kOffSelRcnt);  // [kMaxRetrieval] R sizes
-    const float* rk = p.rkey + (size_t)u * C;
-    const int32_t* cg = p.counts + (size_t)u * C;
-    const int32_t* og = p.offsets + (size_t)u * (C + 1);
-    const int rounds = (C + kRound - 1) / kRound;
-    const bool vec = (C & 3) == 0;
-    float kk[kPer];
-    // keys of round rd into registers; sizes and first rows into shared memory
-    auto load_round = [&](int rd, bool with_meta) {
-      const int c0 = rd * kRound + threadIdx.x * kPer;
-      if (vec && c0 + kPer <= C) {
-#pragma unroll
-        for (int i = 0; i < kPer; i += 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(rk + c0 + i));
-          kk[i] = v.x;
-          kk[i + 1] = v.y;
-          kk[i + 2] = v.z;
-          kk[i + 3] = v.w;
-        }
-        if (with_meta) {
-          // every load issued before the first store (no load waits on a store)
-          int4 cv[kPer / 4];
-          int ov[kPer];
-#pragma unroll
-          for (int i = 0; i < kPer / 4; ++i) cv[i] = __ldg(reinterpret_cast<const int4*>(cg + c0) + i);
-#pragma unroll
-          for (int i = 0; i < kPer; ++i) ov[i] = __ldg(og + c0 + i);
-#pragma unroll
-          for (int i = 0; i < kPer / 4; ++i)
-            *reinterpret_cast<int4*>(cnt_sm + threadIdx.x * kPer + 4 * i) = cv[i];
-#pragma unroll
-          for (int i = 0; i < kPer; ++i) off_sm[threadIdx.x * kPer + i] = ov[i];
-        }
-      } else {
-        int cv[kPer], ov[kPer];
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          const bool in = c0 + i < C;
-          kk[i] = in ? __ldcg(rk + c0 + i) : 0.f;
-          cv[i] = (with_meta && in) ? __ldg(cg + c0 + i) : 0;
-          ov[i] = (with_meta && in) ? __ldg(og + c0 + i) : 0;
-        }
-        if (with_meta) {
-#pragma unroll
-          for (int i = 0; i < kPer; ++i) {
-            cnt_sm[threadIdx.x * kPer + i] = cv[i];
-            off_sm[threadIdx.x * kPer + i] = ov[i];
-          }
-        }
+  const int kA = p.kr, kB = p.kr + p.ke;
+  const bool onA = kA > 0, onB = p.ke > 0;
+  if (selecting) {
+    const int HS = (kNB + CS - 1) / CS;   // histogram buckets per block
+    const int DS = (256 + CS - 1) / CS;   // radix digits per block
+    int* hist = reinterpret_cast<int*>(sm + kRHist);
+    int* dig = reinterpret_cast<int*>(sm + kRDig);
+    const uint32_t hist_a = sm_base + kRHist, dig_a = sm_base + kRDig;
+    for (int i = tid; i < HS; i += kThreads) hist[i] = 0;
+    for (int i = tid; i < 4 * 2 * 256; i += kThreads) dig[i] = 0;
+    cluster_sync();  // 1: every block's key range published, slices zeroed
+
+    if (warp == 0) {
+      uint32_t kx = 0, kn = 0;
+      int ni = 0;
+      if (lane < CS) {
+        kx = ld_cl_u32(mapa(smem_u32(&ms->pub_kmax), lane));
+        kn = ld_cl_u32(mapa(smem_u32(&ms->pub_kmin), lane));
+        ni = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_ninf), lane));
       }
-    };
-    load_round(0, false);
-    for (int i = threadIdx.x; i < kNB; i += NT) hist[i] = 0;
-    if (threadIdx.x < 2) ms->ncand[threadIdx.x] = 0;
-    const uint32_t kmx = __ldcg(p.kmax + u), kmn = __ldcg(p.kmin + u);
-    const int ninf = __ldcg(p.ninf + u);
-    const int nfin = C - ninf;
-    const float lo = nfin > 0 ? float_from_order_key(~kmn) : 0.f;
-    const float hi = nfin > 0 ? float_from_order_key(kmx) : 0.f;
-    const float scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
-    __syncthreads();
-    // 1) histogram over value buckets (monotone in the key)
-    for (int rd = 0; rd < rounds; ++rd) {
-      if (rd > 0) load_round(rd, false);
-      const int c0 = rd * kRound + threadIdx.x * kPer;
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int b = bucket_of(kk[j], lo, scale);
-        if (c0 + j < C && b >= 0) atomicAdd(&hist[b], 1);
+      kx = __reduce_max_sync(0xffffffffu, kx);
+      kn = __reduce_max_sync(0xffffffffu, kn);
+      ni = __reduce_add_sync(0xffffffffu, ni);
+      if (lane == 0) {
+        const int nfin = C - ni;
+        const float lo = nfin > 0 ? float_from_order_key(~kn) : 0.f;
+        const float hi = nfin > 0 ? float_from_order_key(kx) : 0.f;
+        ms->lo = lo;
+        ms->scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
+        ms->nfin = nfin;
+        ms->ninf = ni;
       }
     }
     __syncthreads();
-    // 2) boundary buckets of ranks kr and kr + ke from the top: thread t
-    //    owns kNB / NT consecutive buckets, the highest for t = 0
+    const float lo = ms->lo, scale = ms->scale;
+    const int nfin = ms->nfin, ninf = ms->ninf;
+    for (int i = tid; i < nid; i += kThreads) {
+      const int bk = bucket_of(keys[i], lo, scale);
+      if (bk >= 0) red_cl_add(mapa(hist_a + 4u * (uint32_t)(bk % HS), (uint32_t)(bk / HS)), 1u);
+    }
+    cluster_sync();  // 2: merged histogram complete
+
+    // boundary buckets of ranks kA and kB from the top: thread t owns the
+    // kBPT consecutive buckets below kNB - kBPT t
     {
-      constexpr int BPT = kNB / NT;
-      int hc[BPT];
+      int hc[kBPT];
       int sum = 0;
 #pragma unroll
-      for (int i = 0; i < BPT; ++i) {
-        hc[i] = hist[kNB - 1 - BPT * threadIdx.x - i];
-        sum += hc[i];
+      for (int i = 0; i < kBPT; ++i) {
+        const int j = kNB - 1 - kBPT * tid - i;
+        hc[i] = (int)ld_cl_u32(mapa(hist_a + 4u * (uint32_t)(j % HS), (uint32_t)(j / HS)));
       }
-      if (threadIdx.x < 2) {
-        const int k = threadIdx.x == 0 ? kr : kr + ke;
-        ms->bucket[threadIdx.x] = k <= 0 ? -2 : (k > nfin ? -1 : -3);
-        ms->above[threadIdx.x] = k > nfin ? nfin : 0;
+#pragma unroll
+      for (int i = 0; i < kBPT; ++i) sum += hc[i];
+      if (tid < 2) {
+        const int k = tid == 0 ? kA : kB;
+        const bool on = tid == 0 ? onA : onB;
+        ms->bucket[tid] = !on ? -2 : (k > nfin ? -1 : -3);
+        ms->above[tid] = k > nfin ? nfin : 0;
+        ms->nmem[tid] = k > nfin ? ninf : 0;
       }
       int total_fin;
-      const int excl = block_scan<NT>(sum, ms->scan, &total_fin);
+      const int excl = block_scan(sum, ms->scan, &total_fin);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        const int k = w == 0 ? kr : kr + ke;
-        if (k > 0 && k <= nfin && excl < k && excl + sum >= k) {
+        const int k = w == 0 ? kA : kB;
+        const bool on = w == 0 ? onA : onB;
+        if (on && k <= nfin && excl < k && excl + sum >= k) {
           int cum = excl;
 #pragma unroll
-          for (int i = 0; i < BPT; ++i) {
+          for (int i = 0; i < kBPT; ++i) {
             if (cum + hc[i] >= k) {
-              ms->bucket[w] = kNB - 1 - BPT * threadIdx.x - i;
+              ms->bucket[w] = kNB - 1 - kBPT * tid - i;
               ms->above[w] = cum;
+              ms->nmem[w] = hc[i];
               break;
             }
             cum += hc[i];
@@ -656,638 +617,715 @@ __global__ void __launch_bounds__(Shape<G>::kThreads, 1)
         }
       }
       __syncthreads();
+      if (tid < 2) {
+        const int k = tid == 0 ? kA : kB;
+        ms->kp[tid] = k - ms->above[tid];
+        ms->slow[tid] = ms->bucket[tid] != -2 && ms->nmem[tid] > kCand;
+      }
+      __syncthreads();
     }
-    // 3) exact order inside each boundary bucket: the members of both
-    //    buckets are gathered (warp-aggregated slots) and sorted by
-    //    (key desc, id asc): a warp-wide bitonic sort when <= 32, else ranking
-    int bk[2];
-    bool small[2];
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      bk[w] = ms->bucket[w];
-      const int nb = bk[w] >= 0 ? hist[bk[w]] : (bk[w] == -1 ? ninf : 0);
-      small[w] = bk[w] != -2 && nb <= kBoundaryCap;
-    }
-    if (small[0] || small[1]) {
-      for (int rd = 0; rd < rounds; ++rd) {
-        if (rounds > 1) load_round(rd, false);
-        const int c0 = rd * kRound + threadIdx.x * kPer;
-        uint32_t cm[2] = {0u, 0u};
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-          const int b = bucket_of(kk[j], lo, scale);
-#pragma unroll
-          for (int w = 0; w < 2; ++w)
-            if (small[w] && b == bk[w] && c0 + j < C) cm[w] |= 1u << j;
-        }
+    const int bk0 = ms->bucket[0], bk1 = ms->bucket[1];
+    const bool fast0 = bk0 != -2 && !ms->slow[0], fast1 = bk1 != -2 && !ms->slow[1];
+    const bool slow0 = ms->slow[0], slow1 = ms->slow[1];
+
+    // ---- few members: gather them from every block and rank them directly
+    if (fast0 || fast1) {
+      unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kRCand);
+      unsigned long long* all = reinterpret_cast<unsigned long long*>(sm + kRAll);
+      for (int i = tid; i < nid; i += kThreads) {
+        const float key = keys[i];
+        const int bk = bucket_of(key, lo, scale);
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-          if (!small[w]) continue;
-          const int cnt = __popc(cm[w]);
-          int incl = cnt;
+          if ((w == 0 ? fast0 : fast1) && bk == (w == 0 ? bk0 : bk1)) {
+            const int slot = atomicAdd(&ms->pub_ncand[w], 1);
+            if (slot < kCand) cand[w * kCand + slot] = ord64(float_order_key(key), id0 + i);
+          }
+        }
+      }
+      cluster_sync();  // 3: every block's boundary members listed
+      if (warp < 2) {
+        const int w = warp;
+        int n = 0;
+        if (lane < CS)
+          n = min(kCand, (int)ld_cl_u32(mapa(smem_u32(&ms->pub_ncand[w]), lane)));
+        int incl = n;
 #pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += t;
-          }
-          const int wtot = __shfl_sync(0xffffffffu, incl, 31);
-          int base = 0;
-          if (lane == 0 && wtot > 0) base = atomicAdd(&ms->ncand[w], wtot);
-          base = __shfl_sync(0xffffffffu, base, 0) + incl - cnt;
-          uint32_t m = cm[w];
-          while (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1;
-            cand[w * kBoundaryCap + base++] = ord64(float_order_key(kk[j]), c0 + j);
-          }
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += t;
+        }
+        if (lane < CS) ms->candp[w][lane + 1] = incl;
+        if (lane == 0) ms->candp[w][0] = 0;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        if (!(w == 0 ? fast0 : fast1)) continue;
+        const int n = min(kCand, ms->candp[w][CS]);
+        for (int j = tid; j < n; j += kThreads) {
+          int ob = 0;
+          while (ob + 1 < CS && ms->candp[w][ob + 1] <= j) ++ob;
+          all[w * kCand + j] = ld_cl_u64(
+              mapa(sm_base + kRCand + 8u * (uint32_t)(w * kCand + j - ms->candp[w][ob]), ob));
         }
       }
       __syncthreads();
-      if (warp < 2 && small[warp]) {
-        const int w = warp;
-        const int k = (w == 0 ? kr : kr + ke) - ms->above[w];  // 1-based rank in the bucket
-        const int n = ms->ncand[w];
-        if (n <= 32) {
-          unsigned long long v = lane < n ? cand[w * kBoundaryCap + lane] : 0ull;
 #pragma unroll
-          for (int kb = 2; kb <= 32; kb <<= 1)
+      for (int w = 0; w < 2; ++w) {
+        if (!(w == 0 ? fast0 : fast1)) continue;
+        const int n = min(kCand, ms->candp[w][CS]);
+        const int kp = ms->kp[w];  // 1-based rank inside the bucket
+        for (int j = tid; j < n; j += kThreads) {
+          const unsigned long long me = all[w * kCand + j];
+          int greater = 0;
+          for (int t = 0; t < n; ++t) greater += all[w * kCand + t] > me;
+          if (greater == kp - 1) ms->thr[w] = me;
+        }
+      }
+      __syncthreads();
+    }
+
+    // ---- crowded bucket: radix walk over the order key, then the id count
+    if (slow0 || slow1) {
+      uint32_t prefix[2] = {0u, 0u}, mask[2] = {0u, 0u};
+      int kp[2] = {ms->kp[0], ms->kp[1]};
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < nid; i += kThreads) {
+          const float key = keys[i];
+          const int bk = bucket_of(key, lo, scale);
+          const uint32_t o = float_order_key(key);
 #pragma unroll
-            for (int jb = kb >> 1; jb > 0; jb >>= 1) {
-              const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, jb);
-              const bool keep_max = ((lane & jb) == 0) == ((lane & kb) == 0);
-              v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+          for (int w = 0; w < 2; ++w) {
+            if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) &&
+                (o & mask[w]) == prefix[w]) {
+              const int d = (int)((o >> shift) & 255u);
+              red_cl_add(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
+                              (uint32_t)(d / DS)),
+                         1u);
             }
-          if (lane == k - 1) {
-            ms->Tu[w] = (uint32_t)(v >> 32);
-            ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
           }
-        } else {
-          for (int i = lane; i < n; i += 32) {
-            const unsigned long long me = cand[w * kBoundaryCap + i];
-            int rank = 0;
-            for (int t = 0; t < n; ++t) rank += cand[w * kBoundaryCap + t] > me;
-            if (rank == k - 1) {
-              ms->Tu[w] = (uint32_t)(me >> 32);
-              ms->Tid[w] = (int)(0xFFFFFFFFu - (uint32_t)(me & 0xFFFFFFFFull));
+        }
+        cluster_sync();  // digit counts of this pass complete
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (!(w == 0 ? slow0 : slow1)) continue;
+          const int d = 255 - tid;  // thread order = digits from the top
+          int v = 0;
+          if (tid < 256)
+            v = (int)ld_cl_u32(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
+                                    (uint32_t)(d / DS)));
+          int tot;
+          const int excl = block_scan(v, ms->scan, &tot);
+          if (tid < 256 && excl < kp[w] && excl + v >= kp[w]) {
+            ms->digit[w] = d;
+            ms->above[w] = excl;
+          }
+          __syncthreads();
+          prefix[w] |= (uint32_t)ms->digit[w] << shift;
+          mask[w] |= 255u << shift;
+          kp[w] -= ms->above[w];
+          __syncthreads();
+        }
+      }
+      // members equal to the found key, in id order: per-block counts, then
+      // the block holding the kp-th one names its id
+      const int kper = (max(nid, 1) + kThreads - 1) / kThreads;
+      const int i0 = tid * kper, i1 = min(i0 + kper, nid);
+      int eqc[2] = {0, 0};
+      for (int i = i0; i < i1; ++i) {
+        const float key = keys[i];
+        const int bk = bucket_of(key, lo, scale);
+        const uint32_t o = float_order_key(key);
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) && o == prefix[w]) ++eqc[w];
+      }
+      int ex[2], tot[2];
+#pragma unroll
+      for (int w = 0; w < 2; ++w) ex[w] = block_scan(eqc[w], ms->scan, &tot[w]);
+      if (tid == 0) {
+        ms->pub_idcnt[0] = tot[0];
+        ms->pub_idcnt[1] = tot[1];
+      }
+      cluster_sync();  // per-block counts of equal keys published
+      if (warp < 2) {
+        const int w = warp;
+        int n = 0;
+        if (lane < CS) n = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_idcnt[w]), lane));
+        int incl = n;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += t;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < CS && incl - n < kp[w] && incl >= kp[w]);
+        if (lane == 0) ms->owner[w] = hit ? __ffs(hit) - 1 : -1;
+        if (hit && lane == __ffs(hit) - 1) ms->candp[w][0] = incl - n;  // equal keys before it
+      }
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        if (!(w == 0 ? slow0 : slow1) || ms->owner[w] != b) continue;
+        const int r = kp[w] - ms->candp[w][0];  // 1-based among this block's equal keys
+        if (eqc[w] > 0 && ex[w] < r && ex[w] + eqc[w] >= r) {
+          int seen = ex[w];
+          for (int i = i0; i < i1; ++i) {
+            const float key = keys[i];
+            if (bucket_of(key, lo, scale) == (w == 0 ? bk0 : bk1) &&
+                float_order_key(key) == prefix[w] && ++seen == r) {
+              ms->pub_tid[w] = id0 + i;
+              break;
             }
           }
         }
       }
-    }
-    for (int w = 0; w < 2; ++w) {
-      if (bk[w] == -2 || small[w]) continue;
-      uint32_t Tu;
-      int Tid;
-      const int k = (w == 0 ? kr : kr + ke) - ms->above[w];
-      kth_in_bucket_slow<NT>(rk, C, bk[w], lo, scale, k, ms, hist, &Tu, &Tid);
-      if (threadIdx.x == 0) {
-        ms->Tu[w] = Tu;
-        ms->Tid[w] = Tid;
+      cluster_sync();  // the boundary ids named
+      if (tid < 2 && (tid == 0 ? slow0 : slow1)) {
+        const int w = tid;
+        const int ob = ms->owner[w];
+        const int id = ob >= 0 ? (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tid[w]), (uint32_t)ob)) : -1;
+        ms->thr[w] = ord64(prefix[w], id);
+        if (ob < 0 || id < 0) record_status(p.status, RI_ERR_INVALID_ARG);
       }
+      __syncthreads();
     }
-    __syncthreads();
-    const bool selA = bk[0] != -2, selB = bk[1] != -2;
-    const uint32_t TuA = ms->Tu[0], TuB = ms->Tu[1];
-    const int TidA = ms->Tid[0], TidB = ms->Tid[1];
-    // 4) membership (order key, then id) and compaction in id order: R ids,
-    //    sizes and first rows to shared memory, E ids per round to shared
-    //    memory and then out in coalesced stores
-    int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
-    int32_t* selu = p.sel_user ? p.sel_user + (size_t)u * (p.k_r + p.k_e) : nullptr;
-    int baseR = 0, baseE = 0;
-    for (int rd = 0; rd < rounds; ++rd) {
-      if (rounds > 1) {
-        __syncthreads();  // previous round's E ids are written out
-        load_round(rd, false);
-      }
-      const int c0 = rd * kRound + threadIdx.x * kPer;
-      uint32_t mR = 0, mE = 0;
+    const unsigned long long thrA = onA ? ms->thr[0] : ~0ull, thrB = onB ? ms->thr[1] : ~0ull;
+
+    // ---- classification of the block's ids and the id-ordered lists
+    {
+      const int kper = (max(nid, 1) + kThreads - 1) / kThreads;
+      const int i0 = tid * kper, i1 = min(i0 + kper, nid);
+      float kk[kKPT];
+      int2 mm[kKPT];
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const uint32_t o = float_order_key(kk[j]);
-        const int c = c0 + j;
-        const bool inR = c < C && selA && (o > TuA || (o == TuA && c <= TidA));
-        const bool inE = c < C && !inR && selB && (o > TuB || (o == TuB && c <= TidB));
+      for (int j = 0; j < kKPT; ++j) {
+        const int i = i0 + j;
+        if (j < kper && i < i1) {
+          kk[j] = keys[i];
+          mm[j] = meta[i];
+        }
+      }
+      uint32_t mR = 0, mE = 0;
+      int tokr = 0;
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < kKPT; ++j) {
+        const int i = i0 + j;
+        if (!(j < kper && i < i1)) continue;
+        const unsigned long long o = ord64(float_order_key(kk[j]), id0 + i);
+        const bool inR = onA && o >= thrA;
+        const bool inE = !inR && onB && o >= thrB;
+        if (inR || inE) {
+          const int off = mm[j].x, cnt = mm[j].y;
+          const bool ok = inR ? (cnt >= 0 && off >= 0 && (long long)off + cnt <= p.M)
+                              : cnt >= 0;
+          if (!ok) {
+            bad = true;
+            mm[j] = make_int2(0, 0);
+          }
+        }
+        if (inR) tokr += mm[j].y;
         mR |= (uint32_t)inR << j;
         mE |= (uint32_t)inE << j;
       }
-      int tot;
-      const int excl = block_scan<NT>((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
-      int pr = baseR + (excl >> 16), pe = excl & 0xFFFF;
-      while (mR) {
-        const int j = __ffs(mR) - 1;
-        mR &= mR - 1;
-        rid_sm[pr] = c0 + j;
-        ++pr;
-      }
-      while (mE) {
-        const int j = __ffs(mE) - 1;
-        mE &= mE - 1;
-        ecomp[pe++] = c0 + j;
-      }
-      __syncthreads();
-      const int nE = tot & 0xFFFF;
-      for (int i = threadIdx.x; i < nE; i += NT) {
-        selg[p.k_r + baseE + i] = ecomp[i];
-        if (selu) selu[p.k_r + baseE + i] = ecomp[i];
-      }
-      baseR += tot >> 16;
-      baseE += nE;
-    }
-    for (int i = threadIdx.x; i < p.k_r; i += NT) {
-      const int v = i < kr ? rid_sm[i] : -1;
-      selg[i] = v;
-      if (selu) selu[i] = v;
-    }
-    for (int i = ke + threadIdx.x; i < p.k_e; i += NT) {
-      selg[p.k_r + i] = -1;
-      if (selu) selu[p.k_r + i] = -1;
-    }
-    // 5) R token prefix (execution-buffer rows) and first rows, id order:
-    //    sizes and first rows of the R clusters gathered (loads issued
-    //    together), then one block scan
-    {
-      constexpr int kPerR = kMaxRetrieval / NT;
-      const int per = (kr + NT - 1) / NT;
-      const int i0 = min(kr, (int)threadIdx.x * per), i1 = min(kr, i0 + per);
-      int cn[kPerR], of[kPerR];
+      if (bad) record_status(p.status, RI_ERR_INVALID_ARG);
+      int tot, ttot;
+      const int excl = block_scan((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
+      int texcl = block_scan(tokr, ms->scan, &ttot);
+      const int nR = tot >> 16, nE = tot & 0xFFFF;
+      // keys are all in registers now: the lists take their place
+      uint16_t* rid = reinterpret_cast<uint16_t*>(sm + kRRid);
+      int pr = excl >> 16, pe = nR + (excl & 0xFFFF);
 #pragma unroll
-      for (int w = 0; w < kPerR; ++w) {
-        const int i = i0 + w;
-        const int c = i < i1 ? rid_sm[i] : 0;
-        cn[w] = i < i1 ? __ldg(cg + c) : 0;
-        of[w] = i < i1 ? __ldg(og + c) : 0;
-      }
-      int loc = 0;
-#pragma unroll
-      for (int w = 0; w < kPerR; ++w) {
-        const int i = i0 + w;
-        if (i < i1) {
-          rcnt_sm[i] = cn[w];
-          rrow_sm[i] = of[w];
+      for (int j = 0; j < kKPT; ++j) {
+        if ((mR >> j) & 1u) {
+          lists[pr] = make_int2(mm[j].x, texcl);
+          rid[pr] = (uint16_t)(i0 + j);
+          texcl += mm[j].y;
+          ++pr;
+        } else if ((mE >> j) & 1u) {
+          lists[pe++] = make_int2(id0 + i0 + j, mm[j].y);
         }
-        loc += cn[w];
       }
-      int total;
-      int run = block_scan<NT>(loc, ms->scan, &total);
-      int32_t* rp = p.rpre + (size_t)u * (p.k_r + 1);
-      int32_t* rr = p.rrow + (size_t)u * (p.k_r > 0 ? p.k_r : 1);
-      int32_t* ru = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
-      for (int i = i0; i < i1; ++i) {
-        rp[i] = run;
-        if (ru) ru[i] = run;
-        run += rcnt_sm[i];
-      }
-      for (int i = threadIdx.x; i < kr; i += NT) rr[i] = rrow_sm[i];
-      for (int i = kr + threadIdx.x; i <= p.k_r; i += NT) {
-        rp[i] = total;
-        if (ru) ru[i] = total;
+      if (tid == 0) {
+        ms->pub_nR = nR;
+        ms->pub_nE = nE;
+        ms->pub_tokR = ttot;
       }
     }
-    // 6) publish: one fence after the block barrier covers the block's stores
+    cluster_sync();  // 4: every block's lists and totals published
+    if (warp == 0) {
+      int a = 0, e = 0, t = 0;
+      if (lane < CS) {
+        a = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_nR), lane));
+        e = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_nE), lane));
+        t = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tokR), lane));
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, a, off);
+        const int y = __shfl_up_sync(0xffffffffu, e, off);
+        const int z = __shfl_up_sync(0xffffffffu, t, off);
+        if (lane >= off) {
+          a += x;
+          e += y;
+          t += z;
+        }
+      }
+      if (lane < CS) {
+        ms->nRp[lane + 1] = a;
+        ms->nEp[lane + 1] = e;
+        ms->tokRp[lane + 1] = t;
+      }
+      if (lane == 0) ms->nRp[0] = ms->nEp[0] = ms->tokRp[0] = 0;
+    }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      st_release(p.ready + u, 1);
-    }
-  };
-
-  // Unit u is selected by block NB - 1 - (u mod NB) once its tiles are all
-  // scored (the blocks at the end of the grid score the fewest tiles).
-  if (p.mode != kModeAttend && tiles_h > 0) {
-    for (int u = (int)gridDim.x - 1 - (int)blockIdx.x; u < p.BH; u += (int)gridDim.x) {
-      if (threadIdx.x == 0) {
-        const bool ok = wait_count(p.done + u, tiles_h, p.status);
-        if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
-        ms->flag = ok;
+    // selected ids (R then E, each in id order) and the R token prefix
+    {
+      const bool to_ws = p.mode == kModeSelect;
+      const int ksel = p.k_r + p.k_e;
+      int32_t* selw = to_ws ? p.sel + (size_t)u * ksel : nullptr;
+      int32_t* selu = p.sel_user ? p.sel_user + (size_t)u * ksel : nullptr;
+      int32_t* rpw = to_ws ? p.rpre + (size_t)u * (p.k_r + 1) : nullptr;
+      int32_t* rpu = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
+      if (selw || selu || rpw || rpu) {
+        const uint16_t* rid = reinterpret_cast<const uint16_t*>(sm + kRRid);
+        const int nR = ms->pub_nR, nE = ms->pub_nE;
+        const int rb = ms->nRp[b], eb = ms->nEp[b], tb = ms->tokRp[b];
+        for (int i = tid; i < nR; i += kThreads) {
+          const int g = rb + i;
+          if (g >= p.k_r) break;
+          if (selw) selw[g] = id0 + rid[i];
+          if (selu) selu[g] = id0 + rid[i];
+          if (rpw) rpw[g] = tb + lists[i].y;
+          if (rpu) rpu[g] = tb + lists[i].y;
+        }
+        for (int i = tid; i < nE; i += kThreads) {
+          const int e = eb + i;
+          if (e >= p.k_e) break;
+          if (selw) selw[p.k_r + e] = lists[nR + i].x;
+          if (selu) selu[p.k_r + e] = lists[nR + i].x;
+        }
+        if (b == CS - 1) {
+          for (int g = ms->nRp[CS] + tid; g < p.k_r; g += kThreads) {
+            if (selw) selw[g] = -1;
+            if (selu) selu[g] = -1;
+          }
+          for (int e = ms->nEp[CS] + tid; e < p.k_e; e += kThreads) {
+            if (selw) selw[p.k_r + e] = -1;
+            if (selu) selu[p.k_r + e] = -1;
+          }
+          for (int g = min(ms->nRp[CS], p.k_r) + tid; g <= p.k_r; g += kThreads) {
+            if (rpw) rpw[g] = ms->tokRp[CS];
+            if (rpu) rpu[g] = ms->tokRp[CS];
+          }
+        }
       }
-      __syncthreads();
-      if (!ms->flag) break;
-      __threadfence();
-      select_unit(u);
     }
   }
-  if (p.mode == kModeSelect) return;
+  if (C == 0 && p.mode != kModeAttend && b == 0) {
+    // no indexed token: empty zones
+    const int ksel = p.k_r + p.k_e;
+    for (int i = tid; i < ksel; i += kThreads) {
+      if (p.sel_user) p.sel_user[(size_t)u * ksel + i] = -1;
+      if (p.mode == kModeSelect) p.sel[(size_t)u * ksel + i] = -1;
+    }
+    for (int i = tid; i <= p.k_r; i += kThreads) {
+      if (p.rpre_user) p.rpre_user[(size_t)u * (p.k_r + 1) + i] = 0;
+      if (p.mode == kModeSelect) p.rpre[(size_t)u * (p.k_r + 1) + i] = 0;
+    }
+  }
+  if (p.mode == kModeSelect) {
+    cluster_sync();  // no block leaves while others read its lists
+    return;
+  }
 
   // ============================================================ step C
-  const int npairs = p.BH * p.S;
+  // the unit's totals: R clusters, R tokens, E clusters
+  int KR, KE, T_R;
   const bool exec = p.exec_rows > 0;
-  const long long lim_rows = exec ? p.exec_rows : p.M;
-  const long long row_base_stride = exec ? p.exec_rows : p.M;
-  const int gid = lane >> 2, tig = lane & 3;  // mma fragment coordinates
-  for (int pi = blockIdx.x; pi < npairs && (int)blockIdx.x < p.nbp; pi += p.nbp) {
-    const int u = pi % p.BH, s = pi / p.BH;
-    if (p.mode == kModeFull && tiles_h > 0) {
-      if (threadIdx.x == 0) {
-        const bool ok = wait_count(p.ready + u, 1, p.status);
-        if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
-        ms->flag = ok;
-      }
-      __syncthreads();
-      if (!ms->flag) break;
+  const int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
+  const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
+  if (selecting) {
+    KR = ms->nRp[CS];
+    KE = ms->nEp[CS];
+    T_R = ms->tokRp[CS];
+  } else if (C > 0) {  // attend: the selection left in the workspace
+    KR = p.kr;
+    KE = p.ke;
+    if (tid == 0) ms->T_R = __ldcg(rpg + KR);
+    __syncthreads();
+    T_R = ms->T_R;
+    const long long lim_rows = exec ? p.exec_rows : p.M;
+    if (T_R < 0 || T_R > lim_rows) {
+      if (tid == 0) record_status(p.status, RI_ERR_INVALID_ARG);
+      T_R = 0;
+      KR = 0;
     }
-    // the unit's R prefix and first rows, coalesced into shared memory
-    if (C > 0) {
-      const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
-      const int32_t* rrg = p.rrow + (size_t)u * (p.k_r > 0 ? p.k_r : 1);
-      for (int i0 = 0; i0 <= kr; i0 += 4 * NT) {
-        int a[4], b[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = i0 + j * NT + threadIdx.x;
-          a[j] = i <= kr ? __ldcg(rpg + i) : 0;
-          b[j] = (!exec && i < kr) ? __ldcg(rrg + i) : 0;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = i0 + j * NT + threadIdx.x;
-          if (i <= kr) rpre_sm[i] = a[j];
-          if (i < kr) rrow_sm[i] = b[j];
-        }
+  } else {
+    KR = KE = T_R = 0;
+  }
+  const int n_st = p.n_steady;
+  const long long T = (long long)n_st + T_R;
+  const long long ta = T * b / CS, tb = T * (b + 1) / CS;
+  const int ea = (int)((long long)KE * b / CS), eb = (int)((long long)KE * (b + 1) / CS);
+  const int ntok = (int)(tb - ta), ne = eb - ea;
+  const int nct = (ntok + kItems - 1) / kItems, nce = (ne + kItems - 1) / kItems;
+  const int nch = nct + nce;
+  // the ring was written by the generic proxy in step B: order that before
+  // the bulk copies that write it again
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  if (warp == kProducer) {
+    // ---- R list access: entry g -> (first row, first token), in the unit's
+    // token order (owners' lists in a cluster, the workspace after a select)
+    const uint32_t lists_a = sm_base + kOffKeys;
+    auto r_entry = [&](int g, int& row, int& gs) {
+      if (g >= KR) {
+        row = 0;
+        gs = T_R;
+        return;
       }
-    } else if (threadIdx.x == 0) {
-      rpre_sm[0] = 0;
-    }
-    // A fragments of Q (rows = query heads, padded to 16 with zeros):
-    // qa[kk][0] = Q[gid][16 kk + 2 tig ..], qa[kk][1] = Q[gid][16 kk + 8 + 2 tig ..]
-    uint32_t qa[8][2];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      if (gid < G) {
-        const __nv_bfloat16* qr = p.q + ((size_t)u * G + gid) * kHeadDim + kk * 16 + tig * 2;
-        qa[kk][0] = *reinterpret_cast<const uint32_t*>(qr);
-        qa[kk][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+      if (selecting) {
+        int ob = 0;
+        while (ob + 1 < CS && ms->nRp[ob + 1] <= g) ++ob;
+        const int2 e = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(g - ms->nRp[ob]), (uint32_t)ob));
+        row = e.x;
+        gs = ms->tokRp[ob] + e.y;
       } else {
-        qa[kk][0] = qa[kk][1] = 0u;
+        gs = __ldcg(rpg + g);
+        if (exec) {
+          row = gs;
+        } else {
+          const int id = __ldcg(selg + g);
+          row = (id >= 0 && id < C) ? __ldcg(p.offsets + (size_t)u * (C + 1) + id) : -1;
+        }
       }
-    }
-    __syncthreads();
-    const int n_st = p.n_steady;
-    const int T_R = C > 0 ? rpre_sm[kr] : 0;
-    const long long W = (long long)n_st + T_R + ke;
-    const long long w0 = W * s / p.S, w1 = W * (s + 1) / p.S;
-    const int tok_end = n_st + T_R;  // items below are tokens, above E clusters
-    const int nrounds = (int)((w1 - w0 + kRoundItems - 1) / kRoundItems);
-    struct Round {
-      int ta, ntok, npad, ea, ne;
-      uint32_t off_v, off_ev, off_es, off_en;
     };
-    auto round_of = [&](int r) {
-      const long long a = w0 + (long long)r * kRoundItems;
-      const long long b = min(w1, a + kRoundItems);
-      Round rd;
-      rd.ta = (int)min(a, (long long)tok_end);
-      rd.ntok = (int)min(b, (long long)tok_end) - rd.ta;
-      rd.npad = (rd.ntok + 15) & ~15;
-      rd.ea = (int)(max(a, (long long)tok_end) - tok_end);
-      rd.ne = (int)(max(b, (long long)tok_end) - tok_end) - rd.ea;
-      rd.off_v = rd.npad * 256;
-      rd.off_ev = 2 * rd.npad * 256;
-      rd.off_es = rd.off_ev + rd.ne * 512;
-      rd.off_en = rd.off_es + rd.ne * 32;
-      return rd;
-    };
-    // 16-byte chunk c of token row t, XOR-swizzled for conflict-free ldmatrix
-    auto row_chunk = [](int t, int c) { return (uint32_t)(t * 256 + ((c ^ (t & 7)) << 4)); };
-
-    // ---- copies of round r into buffer r & 1, issued by every warp: warp w
-    // takes items [n w / NW, n (w + 1) / NW) of the round; one cp.async group
-    // per thread and round.  Token rows: lanes 0-15 copy K, 16-31 copy V.
-    auto issue = [&](int r) {
-      const Round rd = round_of(r);
-      uint8_t* buf = sm + (r & 1) * kBufBytes;
-      const int n = rd.ntok + rd.ne;
-      const int j0 = n * warp / NW, j1 = n * (warp + 1) / NW;
-      // tokens of this warp
-      const int t0 = min(j0, rd.ntok), t1 = min(j1, rd.ntok);
-      if (t1 > t0) {
-        int ci = 0;
-        const int first_r = rd.ta + t0 - n_st;  // R index of the first token (if any)
-        if (!exec && rd.ta + t1 > n_st && kr > 0) {
-          const int r0 = max(first_r, 0);
-          int lo = 0, hi = kr - 1;  // last cluster with rpre <= r0
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (rpre_sm[mid] <= r0) lo = mid; else hi = mid - 1;
-          }
-          ci = lo;
-        }
-        for (int t = t0; t < t1; ++t) {
-          const int it = rd.ta + t;
-          const __nv_bfloat16* src = nullptr;
-          if (it < n_st) {
-            src = (lane < 16 ? p.Ks : p.Vs) + ((size_t)u * n_st + it) * kHeadDim;
-          } else {
-            const int rpos = it - n_st;
-            long long row;
-            if (exec) {
-              row = rpos;
-            } else {
-              while (ci + 1 < kr && rpre_sm[ci + 1] <= rpos) ++ci;
-              row = (long long)rrow_sm[ci] + (rpos - rpre_sm[ci]);
-            }
-            if (row >= 0 && row < lim_rows)
-              src = (lane < 16 ? p.Kr : p.Vr) + ((size_t)u * row_base_stride + row) * kHeadDim;
-          }
-          const int c = lane & 15;
-          uint8_t* dst = buf + (lane < 16 ? 0u : rd.off_v) + row_chunk(t, c);
-          if (src) {
-            cp_async16(dst, src + c * 8);
-          } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-            if (lane == 0) record_status(p.status, RI_ERR_INVALID_ARG);
-          }
-        }
-      }
-      // padding rows of the last token tile (zeros: no NaN into the MMA)
-      if (warp == NW - 1)
-        for (int i = lane; i < (rd.npad - rd.ntok) * 32; i += 32) {
-          const int t = rd.ntok + (i >> 5), c = i & 15;
-          *reinterpret_cast<uint4*>(buf + ((i & 16) ? rd.off_v : 0u) + row_chunk(t, c)) =
-              make_uint4(0, 0, 0, 0);
-        }
-      // E clusters of this warp
-      const int e0 = max(j0, rd.ntok) - rd.ntok, e1 = max(j1, rd.ntok) - rd.ntok;
-      for (int eb = e0; eb < e1; eb += 32) {
-        const int ne = min(32, e1 - eb);
-        int idv = -1;
-        if (lane < ne) idv = __ldcg(p.sel + (size_t)u * (p.k_r + p.k_e) + p.k_r + rd.ea + eb + lane);
-        for (int i = 0; i < ne; ++i) {
-          const int c = __shfl_sync(0xffffffffu, idv, i);
-          const int e = eb + i;
-          if (c >= 0 && c < C) {
-            const size_t uc = (size_t)u * C + c;
-            cp_async16(buf + rd.off_ev + e * 512 + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
-            if (lane < 2) cp_async16(buf + rd.off_es + e * 32 + lane * 16, p.score + uc * 8 + lane * 4);
-            if (lane == 2) cp_async4(buf + rd.off_en + e * 4, p.counts + uc);
-          } else if (lane == 0) {
-            *reinterpret_cast<int*>(buf + rd.off_en + e * 4) = 0;
-            record_status(p.status, RI_ERR_INVALID_ARG);
-          }
-        }
-      }
-      cp_async_commit();
-    };
-
-    // ---- state.  Tokens (tensor cores): O^T[d][g] fragments, lane holds
-    // d = 16 j + gid (+8), g = 2 tig (+1); running max / sum of row g = gid
-    // in log2 units.  E clusters (CUDA cores): lane owns dims 4 lane .. +3.
-    float ot[8][4];
-    float tm = -INFINITY, tl = 0.f;
-    float ea[G][4], em[G], el[G];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ot[j][i] = 0.f;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      em[g] = -INFINITY;
-      el[g] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ea[g][i] = 0.f;
-    }
-    constexpr float kScale2 = kScale * 1.4426950408889634f;  // to log2 units
-    constexpr float kLog2e = 1.4426950408889634f;
-    for (int r = 0; r < 2 && r < nrounds; ++r) issue(r);
-    for (int r = 0; r < nrounds; ++r) {
-      const Round rd = round_of(r);
-      const uint8_t* buf = sm + (r & 1) * kBufBytes;
-      if (r + 1 < nrounds) cp_async_wait<1>(); else cp_async_wait<0>();
-      __syncthreads();
-      // token tiles of 16: tile j on warp j % NW
-      const int ntiles = rd.npad >> 4;
-      for (int tj = warp; tj < ntiles; tj += NW) {
-        const uint32_t kbase = smem_u32(buf) + tj * 16 * 256;
-        const uint32_t vbase = smem_u32(buf + rd.off_v) + tj * 16 * 256;
-        // S = Q K^T for tokens 16 tj .. +15: two n-tiles of 8 tokens
-        float sacc[2][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sacc[h][i] = 0.f;
-#pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {  // dims 32 kp .. 32 kp + 31
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // matrices: (tokens 8h.., dim chunk 4kp + m) for m = 0..3
-            const int tr = h * 8 + (lane & 7), ch = kp * 4 + (lane >> 3);
-            uint32_t b[4];
-            ldmatrix_x4(b, kbase + row_chunk(tr, ch));
-            mma_bf16_16816(sacc[h], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b[0], b[1]);
-            mma_bf16_16816(sacc[h], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b[2], b[3]);
-          }
-        }
-        // row g = gid: logits of tokens 8h + 2 tig (+1); mask the padding
-        float x[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int t = tj * 16 + h * 8 + tig * 2 + i;
-            x[h * 2 + i] = t < rd.ntok ? sacc[h][i] * kScale2 : -INFINITY;
-          }
-        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        float corr = 1.f;
-        if (mx > tm + kRescale * kLog2e) {  // new reference (also the first tile)
-          corr = tm == -INFINITY ? 0.f : ex2f(tm - mx);
-          tm = mx;
-          tl *= corr;
-        }
-        // O^T columns g = 2 tig, 2 tig + 1 rescale by the factors of rows g
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
-          const float c0 = __shfl_sync(0xffffffffu, corr, (tig * 2) * 4);
-          const float c1 = __shfl_sync(0xffffffffu, corr, (tig * 2 + 1) * 4);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            ot[j][0] *= c0;
-            ot[j][1] *= c1;
-            ot[j][2] *= c0;
-            ot[j][3] *= c1;
-          }
-        }
-        float pv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          pv[i] = ex2f(x[i] - tm);
-          tl += pv[i];
-        }
-        const uint32_t pb0 = pack_bf16x2(pv[0], pv[1]);  // tokens 2 tig, +1
-        const uint32_t pb1 = pack_bf16x2(pv[2], pv[3]);  // tokens 8 + 2 tig, +1
-        // O^T += V^T P^T: 8 dim groups of 16
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // matrices: (tokens 8 (m >> 1).., dim chunk 2 j + (m & 1)) for m = 0..3
-          const int m4 = lane >> 3;
-          const int tr = (m4 >> 1) * 8 + (lane & 7), ch = j * 2 + (m4 & 1);
-          uint32_t a[4];
-          ldmatrix_x4_trans(a, vbase + row_chunk(tr, ch));
-          mma_bf16_16816(ot[j], a[0], a[1], a[2], a[3], pb0, pb1);
-        }
-      }
-      // E clusters: cluster e on warp e % NW, lane owns dims 4 lane .. 4 lane + 3
-      for (int e = warp; e < rd.ne; e += NW) {
-        const int n = *reinterpret_cast<const int*>(buf + rd.off_en + e * 4);
-        if (n <= 0) continue;
-        const float4 v = *reinterpret_cast<const float4*>(buf + rd.off_ev + e * 512 + lane * 16);
-        const float* sc = reinterpret_cast<const float*>(buf + rd.off_es + e * 32);
-        const float nf = (float)n;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float sg = sc[g] * kLog2e;
-          if (sg > em[g] + kRescale * kLog2e) {
-            const float c = em[g] == -INFINITY ? 0.f : ex2f(em[g] - sg);
-            el[g] *= c;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) ea[g][i] *= c;
-            em[g] = sg;
-          }
-          const float w = ex2f(sg - em[g]);
-          el[g] = fmaf(nf, w, el[g]);
-          ea[g][0] = fmaf(w, v.x, ea[g][0]);
-          ea[g][1] = fmaf(w, v.y, ea[g][1]);
-          ea[g][2] = fmaf(w, v.z, ea[g][2]);
-          ea[g][3] = fmaf(w, v.w, ea[g][3]);
-        }
-      }
-      __syncthreads();  // buffer r & 1 is free again
-      if (r + 2 < nrounds) issue(r + 2);
-    }
-    // ---- warp state -> shared memory: per head g the warp's reference
-    // maximum (natural log), denominator and numerator [128]
-    __syncthreads();
-    float* red = reinterpret_cast<float*>(sm);  // [NW][G][128]
+    // first R entry whose tokens reach R token j (32-ary search)
+    int gb = 0;
     {
-      tl += __shfl_xor_sync(0xffffffffu, tl, 1);
-      tl += __shfl_xor_sync(0xffffffffu, tl, 2);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mtg = __shfl_sync(0xffffffffu, tm, g * 4);
-        const float ltg = __shfl_sync(0xffffffffu, tl, g * 4);
-        const float mw = fmaxf(mtg, em[g]);
-        const float ft = mtg == -INFINITY ? 0.f : ex2f(mtg - mw);
-        const float fe = em[g] == -INFINITY ? 0.f : ex2f(em[g] - mw);
-        if (lane == 0) {
-          ms->wm[warp][g] = mw == -INFINITY ? -INFINITY : mw * 0.6931471805599453f;
-          ms->wl[warp][g] = ltg * ft + el[g] * fe;
+      const long long j0 = max(ta - n_st, 0ll);
+      if (KR > 0 && tb > n_st && j0 < T_R) {
+        int lo_g = 0, hi_g = KR;  // answer in [lo_g, hi_g)
+        while (hi_g - lo_g > 1) {
+          const int span = hi_g - lo_g;
+          const int step = (span + 31) / 32;
+          const int g = lo_g + lane * step;
+          int row, gs = INT_MAX;
+          if (g < hi_g) r_entry(g, row, gs);
+          const unsigned le = __ballot_sync(0xffffffffu, g < hi_g && gs <= j0);
+          const int L = le ? 31 - __clz(le) : 0;
+          lo_g = lo_g + L * step;
+          hi_g = min(hi_g, lo_g + step);
+          if (step == 1) break;
         }
-        float4* rw = reinterpret_cast<float4*>(red + ((size_t)warp * G + g) * kHeadDim + lane * 4);
-        *rw = make_float4(ea[g][0] * fe, ea[g][1] * fe, ea[g][2] * fe, ea[g][3] * fe);
+        gb = lo_g;
       }
-      __syncwarp();
-      // token numerators: lane holds O^T[16 j + gid (+8)][2 tig (+1)]
-      float ftv[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int g = tig * 2 + k;
-        const float mtg = __shfl_sync(0xffffffffu, tm, (g < 8 ? g : 0) * 4);
-        float emg = -INFINITY;
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg)
-          if (gg == g) emg = em[gg];
-        const float mw = fmaxf(mtg, emg);
-        ftv[k] = (g < G && mtg != -INFINITY) ? ex2f(mtg - mw) : 0.f;
+    }
+    // batch of 32 consecutive R entries, one per lane
+    int brow = 0, bgs = 0, bcnt = 0, bend = 0;  // bend: first token after the batch
+    auto load_batch = [&]() {
+      int row, gs;
+      r_entry(gb + lane, row, gs);
+      int nrow, ngs;
+      r_entry(gb + 32, nrow, ngs);
+      const int next = __shfl_down_sync(0xffffffffu, gs, 1);
+      brow = row;
+      bgs = gs;
+      bcnt = (lane == 31 ? ngs : next) - gs;
+      bend = __shfl_sync(0xffffffffu, gs + bcnt, 31);
+    };
+    if (KR > 0) load_batch();
+    const long long lim_rows = exec ? p.exec_rows : p.M;
+    const __nv_bfloat16* Kr = p.Kr + (size_t)u * (exec ? p.exec_rows : p.M) * kHeadDim;
+    const __nv_bfloat16* Vr = p.Vr + (size_t)u * (exec ? p.exec_rows : p.M) * kHeadDim;
+    int issued = 0;
+    for (int k = 0; k < nch; ++k) {
+      if (ld_volatile(&ms->abort_flag)) break;
+      const int st = k % kStagesC;
+      if (k >= kStagesC && !warp_wait(&ms->emptyC[st], ((k / kStagesC) - 1) & 1, lim)) {
+        if (lane == 0) {
+          record_status(p.status, RI_ERR_TIMEOUT);
+          ms->abort_flag = 1;
+        }
+        break;
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int g = tig * 2 + k;
-          if (g < G) {
-            float* rg = red + ((size_t)warp * G + g) * kHeadDim + j * 16 + gid;
-            rg[0] += ot[j][k] * ftv[k];
-            rg[8] += ot[j][2 + k] * ftv[k];
+      uint8_t* stage = sm + st * kStageC;
+      uint64_t* bar = &ms->fullC[st];
+      const bool skip = p.fault == RI_FAULT_ATTEND_COPY && k == 0;
+      if (k < nct) {
+        const long long i0 = ta + (long long)k * kItems;
+        const long long i1 = min(tb, i0 + kItems);
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(i1 - i0) * 512u);
+        __syncwarp();
+        // steady tokens
+        const long long s1 = min(i1, (long long)n_st);
+        if (lane == 0 && i0 < s1 && !skip) {
+          const uint32_t n = (uint32_t)(s1 - i0);
+          const size_t r0 = (size_t)u * n_st + (size_t)i0;
+          bulk_load(stage, p.Ks + r0 * kHeadDim, n * 256u, bar);
+          bulk_load(stage + kOffVRow, p.Vs + r0 * kHeadDim, n * 256u, bar);
+        }
+        // R tokens [j0, j1) of this chunk
+        const long long a0 = max(i0, (long long)n_st);
+        if (a0 < i1) {
+          const int j0 = (int)(a0 - n_st), j1 = (int)(i1 - n_st);
+          const uint32_t slot0 = (uint32_t)(a0 - i0);
+          while (true) {
+            const int lo_t = max(j0, bgs), hi_t = min(j1, bgs + bcnt);
+            if (lo_t < hi_t) {
+              const uint32_t n = (uint32_t)(hi_t - lo_t);
+              const long long row = (long long)brow + (lo_t - bgs);
+              const uint32_t slot = slot0 + (uint32_t)(lo_t - j0);
+              if (skip) {
+              } else if (row >= 0 && row + n <= lim_rows) {
+                bulk_load(stage + slot * 256u, Kr + (size_t)row * kHeadDim, n * 256u, bar);
+                bulk_load(stage + kOffVRow + slot * 256u, Vr + (size_t)row * kHeadDim, n * 256u,
+                          bar);
+              } else {
+                record_status(p.status, RI_ERR_INVALID_ARG);
+                mbar_complete_tx(bar, 2u * n * 256u);
+              }
+            }
+            if (bend >= j1 || gb + 32 >= KR) break;
+            gb += 32;
+            load_batch();
           }
         }
+      } else {
+        const int e0 = ea + (k - nct) * kItems;
+        const int n = min(kItems, eb - e0);
+        int id = -1, cnt = 0;
+        if (lane < n) {
+          const int e = e0 + lane;
+          if (selecting) {
+            int ob = 0;
+            while (ob + 1 < CS && ms->nEp[ob + 1] <= e) ++ob;
+            const int nR_ob = ms->nRp[ob + 1] - ms->nRp[ob];
+            const int2 v = ld_cl_v2(
+                mapa(lists_a + 8u * (uint32_t)(nR_ob + e - ms->nEp[ob]), (uint32_t)ob));
+            id = v.x;
+            cnt = v.y;
+          } else {
+            id = __ldcg(selg + p.k_r + e);
+            cnt = (id >= 0 && id < C) ? __ldg(p.counts + (size_t)u * C + id) : 0;
+          }
+          const bool ok = id >= 0 && id < C && cnt >= 0;
+          ms->ecount[st][lane] = ok ? cnt : 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)n * (512u + Gp * 4u));
+        __syncwarp();
+        if (lane < n && !skip) {
+          if (id >= 0 && id < C) {
+            const size_t uc = (size_t)u * C + id;
+            bulk_load(stage + lane * 512u, p.vsum + uc * kHeadDim, 512u, bar);
+            bulk_load(stage + kOffESc + lane * 32u, p.score + uc * Gp, Gp * 4u, bar);
+          } else {
+            record_status(p.status, RI_ERR_INVALID_ARG);
+            mbar_complete_tx(bar, 512u + Gp * 4u);
+          }
+        }
+      }
+      ++issued;
     }
-    __syncthreads();
-    float* part = p.part + ((size_t)u * p.S + s) * G * kPartStride;
-    // warp g: the block maximum of head g and the warps' factors (in wm)
-    if (warp < G) {
-      const int g = warp;
-      const float wmv = lane < NW ? ms->wm[lane][g] : -INFINITY;
-      float mb = wmv;
+    // after a failure the copies already issued still land before the block
+    // leaves (their stages may never be consumed)
+    if (ld_volatile(&ms->abort_flag) && lane == 0)
+      for (int k = max(0, issued - kStagesC); k < issued; ++k)
+        mbar_wait(&ms->fullC[k % kStagesC], (uint32_t)((k / kStagesC) & 1), lim);
+  }
+
+  // ---- consumers: online softmax over the chunks
+  Acc acc;
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
-      const float f = (wmv == -INFINITY) ? 0.f : __expf(wmv - mb);
-      float lw = lane < NW ? f * ms->wl[lane][g] : 0.f;
+  for (int j = 0; j < 4; ++j) {
+    acc.m[j] = -INFINITY;
+    acc.l[j] = 0.f;
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-      __syncwarp();
-      if (lane < NW) ms->wm[lane][g] = f;
-      if (lane == 0) {
-        part[(size_t)g * kPartStride + 0] = mb;
-        part[(size_t)g * kPartStride + 1] = lw;
+    for (int i = 0; i < 8; ++i) acc.o[j][i] = 0.f;
+  }
+  const int half = lane >> 4, l16 = lane & 15;
+  // query head of lane head j (G > 4: the half-warps split the heads)
+  auto head_of = [&](int j) { return G <= 4 ? j : 4 * half + j; };
+  if (warp < kConsumers) {
+    float qf[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = head_of(j);
+      if (j < HPL && g < G) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+            p.q + ((size_t)u * G + g) * kHeadDim + l16 * 8));
+        bf16x8_to_float(raw, qf[j]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qf[j][i] = 0.f;
       }
     }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < G * kHeadDim; idx += NT) {
-      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-      float a = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) a = fmaf(ms->wm[w][g], red[((size_t)w * G + g) * kHeadDim + d], a);
-      part[(size_t)g * kPartStride + 4 + d] = a;
-    }
-    // ============================================================ step D
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) ms->flag = atomicAdd(p.ticket + u, 1) == p.S - 1;
-    __syncthreads();
-    if (ms->flag) {
-      // the last slice of unit u merges the S partials (log-sum-exp)
-      __threadfence();
-      const float* pu = p.part + (size_t)u * p.S * G * kPartStride;
-      float* fq = reinterpret_cast<float*>(sm);  // [S][G] maxima, then weights
-      float* tot = fq + p.S * G;                 // [G] max, [G] denominator
-      if (warp < G) {
-        // warp g: the slices' maxima and denominators of query head g
-        const int g = warp;
-        float mx = -INFINITY;
-        for (int q = lane; q < p.S; q += 32) {
-          const float m = __ldcg(pu + ((size_t)q * G + g) * kPartStride);
-          fq[q * G + g] = m;
-          mx = fmaxf(mx, m);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        float ls = 0.f;
-        for (int q = lane; q < p.S; q += 32) {
-          const float m = fq[q * G + g];
-          const float f = (mx == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - mx);
-          fq[q * G + g] = f;
-          ls = fmaf(__ldcg(pu + ((size_t)q * G + g) * kPartStride + 1), f, ls);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+    constexpr float kQK = kScale * kLog2e;
+    for (int k = 0; k < nch; ++k) {
+      const int st = k % kStagesC;
+      if (!warp_wait(&ms->fullC[st], (uint32_t)((k / kStagesC) & 1), lim)) {
         if (lane == 0) {
-          tot[g] = mx;
-          tot[G + g] = ls;
+          record_status(p.status, RI_ERR_TIMEOUT);
+          ms->abort_flag = 1;
+        }
+        break;
+      }
+      const uint8_t* stage = sm + st * kStageC;
+      const bool tok = k < nct;
+      const int n_items = tok ? min(kItems, ntok - k * kItems) : min(kItems, ne - (k - nct) * kItems);
+#pragma unroll
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int it = G <= 4 ? warp + kConsumers * half : warp + kConsumers * ps;
+        const bool valid = it < n_items;
+        const int itc = valid ? it : 0;
+        if (tok) {
+          const uint4 kraw = *reinterpret_cast<const uint4*>(stage + itc * 256 + l16 * 16);
+          const uint4 vraw = *reinterpret_cast<const uint4*>(stage + kOffVRow + itc * 256 + l16 * 16);
+          float kf[8], vf[8];
+          bf16x8_to_float(kraw, kf);
+          bf16x8_to_float(vraw, vf);
+          float d[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            d[j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d[j] = fmaf(qf[j][i], kf[i], d[j]);
+          }
+#pragma unroll
+          for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (j < HPL) d[j] += __shfl_xor_sync(0xffffffffu, d[j], off);
+          if (valid) {
+#pragma unroll
+            for (int j = 0; j < HPL; ++j)
+              if (head_of(j) < G) acc_add(acc, j, d[j] * kQK, 1.f, vf);
+          }
+        } else if (valid) {
+          const int n = ms->ecount[st][itc];
+          if (n > 0) {
+            const float4* vr = reinterpret_cast<const float4*>(stage + itc * 512 + l16 * 32);
+            const float4 v0 = vr[0], v1 = vr[1];
+            const float vf[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const float* sc = reinterpret_cast<const float*>(stage + kOffESc + itc * 32);
+            const float nf = (float)n;
+#pragma unroll
+            for (int j = 0; j < HPL; ++j)
+              if (head_of(j) < G) acc_add(acc, j, sc[head_of(j)] * kLog2e, nf, vf);
+          }
         }
       }
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < G * kHeadDim; idx += NT) {
-        const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-        float os = 0.f;
-        for (int q0 = 0; q0 < p.S; q0 += 16) {
-          float v[16];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->emptyC[st]);
+    }
+    if (G <= 4) {
+      // the two half-warps hold the same heads: combine them
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            v[k] = q0 + k < p.S ? __ldcg(pu + ((size_t)(q0 + k) * G + g) * kPartStride + 4 + d)
-                                : 0.f;
+      for (int j = 0; j < HPL; ++j) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, acc.m[j], 16);
+        const float l2 = __shfl_xor_sync(0xffffffffu, acc.l[j], 16);
+        const float mm = fmaxf(acc.m[j], m2);
+        const float f1 = acc.m[j] == -INFINITY ? 0.f : ex2f(acc.m[j] - mm);
+        const float f2 = m2 == -INFINITY ? 0.f : ex2f(m2 - mm);
+        acc.l[j] = acc.l[j] * f1 + l2 * f2;
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (q0 + k < p.S) os = fmaf(fq[(q0 + k) * G + g], v[k], os);
+        for (int i = 0; i < 8; ++i) {
+          const float o2 = __shfl_xor_sync(0xffffffffu, acc.o[j][i], 16);
+          acc.o[j][i] = acc.o[j][i] * f1 + o2 * f2;
         }
-        const float ls = tot[G + g];
-        // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
-        const bool any = ls > 0.f;
-        const size_t hq = (size_t)u * G + g;
-        p.out[hq * kHeadDim + d] = __float2bfloat16_rn(any ? os / ls : 0.f);
-        if (p.lse && d == 0) p.lse[hq] = any ? tot[g] + logf(ls) : -INFINITY;
+        acc.m[j] = mm;
       }
     }
-    __syncthreads();  // the region is reused by the next pair's copies
+  }
+  __syncthreads();  // every chunk consumed: the ring is free
+
+  // ============================================================ step D
+  // warps -> block partial (max in log2 units, denominator, numerator)
+  float* wo = reinterpret_cast<float*>(sm);  // [kConsumers][G][128]
+  if (warp < kConsumers && (G > 4 || half == 0)) {
+#pragma unroll
+    for (int j = 0; j < HPL; ++j) {
+      const int g = head_of(j);
+      if (g < G) {
+        float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + l16 * 8);
+        dst[0] = make_float4(acc.o[j][0], acc.o[j][1], acc.o[j][2], acc.o[j][3]);
+        dst[1] = make_float4(acc.o[j][4], acc.o[j][5], acc.o[j][6], acc.o[j][7]);
+        if (l16 == 0) {
+          ms->wm[warp][g] = acc.m[j];
+          ms->wl[warp][g] = acc.l[j];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  constexpr int kOutPer = (G * kHeadDim + kThreads - 1) / kThreads;
+  float bo[kOutPer], bmv[kOutPer], blv[kOutPer];
+#pragma unroll
+  for (int r = 0; r < kOutPer; ++r) {
+    const int idx = tid + r * kThreads;
+    bo[r] = 0.f;
+    bmv[r] = -INFINITY;
+    blv[r] = 0.f;
+    if (idx < G * kHeadDim) {
+      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) mx = fmaxf(mx, ms->wm[w][g]);
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) {
+        const float mw = ms->wm[w][g];
+        const float f = mw == -INFINITY ? 0.f : ex2f(mw - mx);
+        L = fmaf(f, ms->wl[w][g], L);
+        O = fmaf(f, wo[((size_t)w * G + g) * kHeadDim + d], O);
+      }
+      bo[r] = O;
+      bmv[r] = mx;
+      blv[r] = L;
+    }
+  }
+  cluster_sync();  // 5: every block done with step C (block 0's ring is free)
+  // every block's partial into block 0: [CS][G][2 + 128] floats
+  const uint32_t area = sm_base;
+#pragma unroll
+  for (int r = 0; r < kOutPer; ++r) {
+    const int idx = tid + r * kThreads;
+    if (idx < G * kHeadDim) {
+      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+      const uint32_t base = area + 4u * (uint32_t)((b * G + g) * (kHeadDim + 2));
+      st_cl_f32(mapa(base + 4u * (2 + d), 0), bo[r]);
+      if (d == 0) {
+        st_cl_f32(mapa(base, 0), bmv[r]);
+        st_cl_f32(mapa(base + 4u, 0), blv[r]);
+      }
+    }
+  }
+  cluster_arrive();  // 6: partials stored (release)
+  if (b != 0) return;
+  cluster_wait();
+  const float* pa = reinterpret_cast<const float*>(sm);
+  for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
+    const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+    float mx = -INFINITY;
+    for (int q = 0; q < CS; ++q) mx = fmaxf(mx, pa[(q * G + g) * (kHeadDim + 2)]);
+    float L = 0.f, O = 0.f;
+    for (int q = 0; q < CS; ++q) {
+      const float* pq = pa + (q * G + g) * (kHeadDim + 2);
+      const float f = pq[0] == -INFINITY ? 0.f : ex2f(pq[0] - mx);
+      L = fmaf(f, pq[1], L);
+      O = fmaf(f, pq[2 + d], O);
+    }
+    // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
+    const bool any = L > 0.f;
+    const size_t hq = (size_t)u * G + g;
+    p.out[hq * kHeadDim + d] = __float2bfloat16_rn(any ? O / L : 0.f);
+    if (p.lse && d == 0) p.lse[hq] = any ? mx * kLn2 + logf(L) : -INFINITY;
   }
 }
 
@@ -1310,9 +1348,30 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [rows][128] row-major, boxes of 64 columns x box_rows, 128-byte swizzle
+// bf16 [rows][128] row-major, boxes of 64 columns x box_rows, 128-byte
+// swizzle.  Maps are kept in a small fixed table keyed by (base, rows, box):
+// a decode step reuses the maps of its centroid and query buffers.
+struct MapSlot {
+  const void* base;
+  unsigned long long rows;
+  unsigned box;
+  CUtensorMap map;
+};
+constexpr int kMapSlots = 64;
+std::mutex g_map_mu;
+MapSlot g_maps[kMapSlots];
+int g_map_next = 0;
+
 cudaError_t encode_rows(CUtensorMap* map, const void* base, unsigned long long rows,
                         unsigned box_rows) {
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (int i = 0; i < kMapSlots; ++i)
+      if (g_maps[i].base == base && g_maps[i].rows == rows && g_maps[i].box == box_rows) {
+        *map = g_maps[i].map;
+        return cudaSuccess;
+      }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
@@ -1323,36 +1382,73 @@ cudaError_t encode_rows(CUtensorMap* map, const void* base, unsigned long long r
          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapSlot& s = g_maps[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapSlots;
+  s.base = base;
+  s.rows = rows;
+  s.box = box_rows;
+  s.map = *map;
   return cudaSuccess;
 }
 
-template <int G>
-cudaError_t prepare_kernel() {
-  return set_smem_once(reinterpret_cast<const void*>(decode_kernel<G>), (int)kSmemBytes);
-}
-
-template <int G>
-int blocks_per_sm() {
-  int n = 0;
-  if (prepare_kernel<G>() != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, Shape<G>::kThreads,
-                                                    kSmemBytes) != cudaSuccess)
-    n = 0;
-  cudaGetLastError();
-  return n;
-}
-
-int blocks_per_sm_g(int G) {
+const void* kernel_of(int G) {
   switch (G) {
-    case 1: return blocks_per_sm<1>();
-    case 2: return blocks_per_sm<2>();
-    case 3: return blocks_per_sm<3>();
-    case 4: return blocks_per_sm<4>();
-    case 5: return blocks_per_sm<5>();
-    case 6: return blocks_per_sm<6>();
-    case 7: return blocks_per_sm<7>();
-    default: return blocks_per_sm<8>();
+    case 1: return reinterpret_cast<const void*>(decode_kernel<1>);
+    case 2: return reinterpret_cast<const void*>(decode_kernel<2>);
+    case 3: return reinterpret_cast<const void*>(decode_kernel<3>);
+    case 4: return reinterpret_cast<const void*>(decode_kernel<4>);
+    case 5: return reinterpret_cast<const void*>(decode_kernel<5>);
+    case 6: return reinterpret_cast<const void*>(decode_kernel<6>);
+    case 7: return reinterpret_cast<const void*>(decode_kernel<7>);
+    default: return reinterpret_cast<const void*>(decode_kernel<8>);
   }
+}
+
+// Per device and group size: kernel attributes set, and how many clusters of
+// each size can be resident at once (fixed tables, filled on first use).
+constexpr int kMaxDevices = 64;
+struct DevState {
+  int ready[kMaxGroupHost + 1];
+  int n_active[kMaxGroupHost + 1][kMaxClusterBlocks + 1];
+};
+std::mutex g_dev_mu;
+DevState g_dev[kMaxDevices];
+
+cudaError_t device_state(int G, const int** n_active) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevState& s = g_dev[dev];
+  if (!s.ready[G]) {
+    const void* fn = kernel_of(G);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    for (int cs = 1; cs <= kMaxClusterBlocks; ++cs) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)cs);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+      s.n_active[G][cs] = n;
+    }
+    cudaGetLastError();
+    s.ready[G] = 1;
+  }
+  *n_active = s.n_active[G];
+  return cudaSuccess;
 }
 
 template <int G>
@@ -1373,21 +1469,12 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   p.sel_user = a.sel_user;
   p.rpre_user = a.rpre_user;
   p.score = reinterpret_cast<float*>(a.ws + L.off_score);
-  p.rkey = reinterpret_cast<float*>(a.ws + L.off_rkey);
   p.sel = reinterpret_cast<int32_t*>(a.ws + L.off_sel);
   p.rpre = reinterpret_cast<int32_t*>(a.ws + L.off_rpre);
-  p.rrow = reinterpret_cast<int32_t*>(a.ws + L.off_rrow);
-  p.part = reinterpret_cast<float*>(a.ws + L.off_part);
   p.status = reinterpret_cast<int*>(a.ws);
-  const long long BH = g.BH();
-  p.done = reinterpret_cast<int*>(a.ws + L.off_ctrl);
-  p.ready = p.done + BH;
-  p.ticket = p.ready + BH;
-  p.kmax = reinterpret_cast<uint32_t*>(p.ticket + BH);
-  p.kmin = p.kmax + BH;
-  p.ninf = reinterpret_cast<int*>(p.kmin + BH);
-  p.nbp = L.NBP;
-  p.BH = (int)BH;
+  p.wait_ns = a.wait_ns;
+  p.fault = a.fault;
+  p.BH = (int)g.BH();
   p.C = g.C;
   p.M = g.M;
   p.n_steady = g.n_steady;
@@ -1395,7 +1482,7 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   p.k_e = L.k_e;
   p.kr = L.kr;
   p.ke = L.ke;
-  p.S = L.S;
+  p.tiles = (g.C + kTileC - 1) / kTileC;
   p.exec_rows = exec ? a.exec_rows : 0;
   p.mode = mode;
 
@@ -1403,20 +1490,20 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   memset(&map_c, 0, sizeof(map_c));
   memset(&map_q, 0, sizeof(map_q));
   if (g.C > 0 && mode != kModeAttend) {
-    cudaError_t e = encode_rows(&map_c, a.centroid, (unsigned long long)BH * g.C, kTileC);
-    if (e == cudaSuccess) e = encode_rows(&map_q, a.q, (unsigned long long)BH * G, kQRows);
+    cudaError_t e = encode_rows(&map_c, a.centroid, (unsigned long long)g.BH() * g.C, kTileC);
+    if (e == cudaSuccess) e = encode_rows(&map_q, a.q, (unsigned long long)g.BH() * G, kQRows);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = prepare_kernel<G>();
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)L.NB);
-  cfg.blockDim = dim3(Shape<G>::kThreads);
+  cfg.gridDim = dim3((unsigned)(g.BH() * L.CS));
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)L.CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, decode_kernel<G>, map_c, map_q, p);
@@ -1438,53 +1525,44 @@ cudaError_t launch_mode(const Geometry& g, const DecodeLayout& L, const DecodeAr
 
 }  // namespace
 
-// Launch shape of the decode kernel: one block per SM (NB), and S slices of
-// the attention work per unit.  S is the smallest count whose makespan
-// (ceil(units x S / NB') slices of 1/S of a unit per block) is within 5 % of
-// the best over S <= 64, with at least ~32 items per slice; NB' leaves the
-// selector blocks free when units <= NB / 2.
+// Launch shape: one cluster of CS blocks per unit, CS between the smallest
+// size whose blocks hold the unit's clusters (at most kMaxIdsPerBlock ids per
+// block) and kMaxClusterBlocks.  Each size is scored by the waves it needs
+// (units over the clusters of that size the device holds at once) times the
+// share of a unit one block carries, plus a small per-block term for the
+// cluster barriers; the cheapest size wins.
 bool decode_plan(const Geometry& g, DecodeLayout* L) {
-  int nb = 148;
-  int dev = -1;
-  if (cudaGetDevice(&dev) == cudaSuccess) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-        sms > 0) {
-      static std::mutex mu;
-      static std::map<std::pair<int, int>, int> cache;
-      int per;
-      {
-        std::lock_guard<std::mutex> lk(mu);
-        auto key = std::make_pair(dev, g.G);
-        auto it = cache.find(key);
-        if (it == cache.end()) it = cache.emplace(key, blocks_per_sm_g(g.G)).first;
-        per = it->second;
-      }
-      if (per < 1) {
-        set_error("decode kernel cannot be resident on this device");
-        return false;
-      }
-      nb = sms;  // one block per SM
+  const int* n_active = nullptr;
+  if (device_state(g.G, &n_active) != cudaSuccess) {
+    cudaGetLastError();
+    set_error("decode kernel cannot be configured on this device");
+    return false;
+  }
+  const long long units = g.BH();
+  const int tiles = (g.C + kTileC - 1) / kTileC;
+  const int cs_min = tiles > 0 ? (tiles + kMaxTilesPerBlock - 1) / kMaxTilesPerBlock : 1;
+  if (cs_min > kMaxClusterBlocks) {
+    set_error("%d clusters per (sequence, KV head) exceed the decode kernel's limit of %d", g.C,
+              kMaxClusterBlocks * kMaxIdsPerBlock);
+    return false;
+  }
+  int best = -1;
+  double best_cost = 1e30;
+  for (int cs = cs_min; cs <= kMaxClusterBlocks; ++cs) {
+    const int n = n_active[cs];
+    if (n < 1) continue;
+    const long long waves = (units + n - 1) / n;
+    const double cost = (double)waves * (1.0 / cs + 0.02);
+    if (cost < best_cost - 1e-12) {
+      best_cost = cost;
+      best = cs;
     }
   }
-  cudaGetLastError();
-  const long long units = g.BH();
-  const double avg_r = g.C > 0 ? (double)L->kr * g.M / g.C : 0.0;
-  const double w_est = g.n_steady + avg_r + L->ke;
-  int s_max = (int)(w_est / 32.0);
-  s_max = s_max < 1 ? 1 : (s_max > 64 ? 64 : s_max);
-  // with few units the selector blocks (the last `units` blocks) take no slices
-  const long long nbp = units <= nb / 2 ? nb - units : nb;
-  auto makespan = [&](int S) {
-    return (double)((units * S + nbp - 1) / nbp) / (double)S;
-  };
-  double best = 1e30;
-  for (int S = 1; S <= s_max; ++S) best = best < makespan(S) ? best : makespan(S);
-  int S = 1;
-  while (S < s_max && makespan(S) > 1.05 * best) ++S;
-  L->NB = nb;
-  L->NBP = (int)nbp;
-  L->S = S;
+  if (best < 0) {
+    set_error("decode kernel cannot be resident on this device (cluster of %d blocks)", cs_min);
+    return false;
+  }
+  L->CS = best;
   return true;
 }
 

@@ -14,6 +14,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kMaxGroupHost = 8;          // query heads per KV head
 constexpr size_t kStatusBytesHost = 256;  // status word region at workspace start
+constexpr unsigned long long kWaitLimitNsHost = 2000000000ull;  // bounded device waits: 2 s
 
 // Everything derived from an ri_index_config.
 struct Geometry {
@@ -36,23 +37,33 @@ struct Geometry {
 bool make_geometry(const ri_index_config* cfg, Geometry* g);
 
 // --------------------------------------------------------------- decode
-struct DecodeLayout {
-  int k_r, k_e;     // requested budgets (sizes of the sel regions)
-  int kr, ke;       // clamped to C
-  int NB;           // blocks of the decode kernel (one per SM)
-  int NBP;          // of which take attention slices (the rest select)
-  int S;            // slices of the attention work per (b, h) unit
-  // status word [0, 256); counters done/ready/ticket/kmax/kmin/ninf [6][BH]
-  // (both cleared by every call: header_bytes); rkey fp32 [BH][C], score fp32
-  // [BH][C][8], sel int32 [BH][k_r + k_e], rpre int32 [BH][k_r + 1], rrow
-  // int32 [BH][max(k_r, 1)], part fp32 [BH][S][G][kPartStride].
-  size_t header_bytes, off_ctrl, off_rkey, off_score, off_sel, off_rpre, off_rrow, off_part,
-      total;
-};
-constexpr int kPartStride = 132;     // m, l, 2 pad, o[128]
-constexpr int kMaxRetrieval = 4096;  // retrieval clusters per unit held on chip
+constexpr int kMaxIdsPerBlock = 4096;  // clusters of a unit one decode block scores
+constexpr int kMaxClusterBlocks = 16;  // blocks of the thread-block cluster of one unit
+constexpr int kMaxRetrieval = 4096;    // k_retrieval limit (retrieval-row prefix)
 
-bool make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L);
+struct DecodeLayout {
+  int k_r, k_e;  // requested budgets (sizes of the sel regions)
+  int kr, ke;    // clamped to C
+  int CS;        // blocks per unit (thread-block cluster size)
+  int Gp;        // scores stored per cluster: 4 (G <= 4) or 8
+  // status region [0, 256); score fp32 [BH][C][Gp]; sel int32 [BH][k_r + k_e];
+  // rpre int32 [BH][k_r + 1] (the last two hold a selection between
+  // ri_select_clusters and ri_attend_selected)
+  size_t off_score, off_sel, off_rpre, total;
+};
+
+// RI_OK, or the status of the first failed check (the thread's last error
+// says which).
+ri_status make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, DecodeLayout* L);
+
+// Test hook of the decode kernel's bounded waits: which hand-off is left
+// unreleased (0 in every public call).
+enum {
+  RI_FAULT_NONE = 0,
+  RI_FAULT_SCORE_COPY = 1,    // the first centroid tile's copy is never issued
+  RI_FAULT_SCORE_COMMIT = 2,  // the first tile's MMA completion is never signalled
+  RI_FAULT_ATTEND_COPY = 3    // the first attention chunk's copies are never issued
+};
 
 struct DecodeArgs {
   const void* q;
@@ -72,13 +83,15 @@ struct DecodeArgs {
   int32_t* sel_user;
   int32_t* rpre_user;
   char* ws;
+  unsigned long long wait_ns;  // limit of every bounded wait
+  int fault;                   // RI_FAULT_* (test hook)
 };
 
 cudaError_t launch_decode(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
 cudaError_t launch_select(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
-// Chooses the launch shape of the decode kernel (blocks, slices per unit).
+// Chooses the launch shape of the decode kernel (blocks per unit).
 bool decode_plan(const Geometry& g, DecodeLayout* L);
 cudaError_t launch_attend(const Geometry& g, const DecodeLayout& L, const DecodeArgs& a,
                           cudaStream_t s);
@@ -137,7 +150,9 @@ cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_n
 void set_error(const char* fmt, ...);
 int num_sms();
 // Raises a kernel's dynamic shared memory limit once per device (outside any
-// stream capture after the first call on that device).
-cudaError_t set_smem_once(const void* func, int bytes);
+// stream capture after the first call on that device).  `slot` names the
+// kernel in a fixed table (kSmemSlots entries).
+constexpr int kSmemSlots = 16;
+cudaError_t set_smem_once(int slot, const void* func, int bytes);
 
 }  // namespace ri

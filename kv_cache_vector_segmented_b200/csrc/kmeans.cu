@@ -997,16 +997,16 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   unit_max_kernel<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(ecs, d, ust, (int)units);
   RI_CUDA_TRY(cudaGetLastError());
 
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
+  RI_CUDA_TRY(set_smem_once(0, reinterpret_cast<const void*>(assign_kernel), (int)kAssignSmem));
   auto sort_smem = [](int L) {
     constexpr int NW = kSortThreads / 32;
     return (size_t)(NW * kMaxClustersPerSeg + kMaxClustersPerSeg + 1 + NW) * sizeof(int) +
            (size_t)L * sizeof(uint16_t);
   };
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(sort_kernel),
+  RI_CUDA_TRY(set_smem_once(1, reinterpret_cast<const void*>(sort_kernel),
                             (int)sort_smem(kMaxSegLen)));
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(update_kernel), kUpdateSmem));
-  RI_CUDA_TRY(set_smem_once(reinterpret_cast<const void*>(finalise_kernel), kFinSmem));
+  RI_CUDA_TRY(set_smem_once(2, reinterpret_cast<const void*>(update_kernel), kUpdateSmem));
+  RI_CUDA_TRY(set_smem_once(3, reinterpret_cast<const void*>(finalise_kernel), kFinSmem));
   const int sms = num_sms();
   const unsigned grid_assign = (unsigned)(d.total_tiles < sms ? d.total_tiles : sms);
   const dim3 grid_upd((unsigned)units, (unsigned)(kMaxClustersPerSeg / kUpdateWarps));

@@ -180,3 +180,87 @@ def test_wait_timeout_selftest_reports_status(R):
     # the context is still healthy
     x = torch.ones(4, device=dev)
     assert float(x.sum()) == 4.0
+
+
+# ---------------------------------------------------------------- selection
+def _decode_index(R, heads, B, H, G, N, seg_len=8192, clusters=512):
+    dev = torch.device("cuda:0")
+    cfg = R.IndexConfig.make(B, H, G, N, seg_len=seg_len, clusters_per_seg=clusters)
+    return U.to_device_index(R, cfg, heads, dev)
+
+
+def test_decode_heavy_ties_are_broken_by_id(R):
+    """Every centroid equal: all selection keys tie exactly on both sides,
+    so R must be the k_r lowest ids and E the next k_e, bit for bit.  More
+    than 256 keys share the boundary bucket, which takes the radix walk over
+    the order key and the per-block id count."""
+    dev = torch.device("cuda:0")
+    kv = S.make_kv(1, 2, 3 * 8192 + 68, seed=41)
+    q = S.make_queries(kv, 4, seed=42)
+    heads = U.oracle_index_heads(kv, use_labels=True)
+    for o in heads[0]:
+        o["centroid"][:] = o["centroid"][0]
+    idx = _decode_index(R, heads, 1, 2, 4, kv.K.shape[2])
+    for k in [(147, 300), (0, 700), (1000, 200), (5, 1531)]:
+        d = R.DecodeConfig(*k)
+        out, lse, sel = R.decode(q.to(dev), idx, d, want_sel=True)
+        ora = O.decode(q.double().numpy(), U.as_consumed(heads), *k)
+        for h in range(2):
+            C = heads[0][h]["C"]
+            kr = min(k[0], C)
+            ke = min(k[1], C - kr)
+            live = np.flatnonzero(heads[0][h]["counts"] > 0)
+            order = np.concatenate([live, np.flatnonzero(heads[0][h]["counts"] == 0)])
+            assert sel[0, h, :kr].tolist() == sorted(order[:kr].tolist())
+            assert sel[0, h, k[0]:k[0] + ke].tolist() == sorted(order[kr:kr + ke].tolist())
+        U.compare_output(out, ora["out"])
+        np.testing.assert_allclose(lse.cpu().numpy(), ora["lse"], rtol=1e-4, atol=1e-4)
+
+
+def test_decode_zero_query_selects_lowest_ids(R):
+    """q = 0: every score is exactly 0, the selection is the lowest ids and
+    the output is the plain average of the attended values."""
+    dev = torch.device("cuda:0")
+    kv = S.make_kv(1, 1, 2 * 8192 + 500, seed=43)
+    q = torch.zeros((1, 4, 128), dtype=torch.bfloat16)
+    heads = U.oracle_index_heads(kv, use_labels=True)
+    idx = _decode_index(R, heads, 1, 1, 4, kv.K.shape[2])
+    d = R.default_budgets(idx.geom.clusters)
+    out, lse, sel = R.decode(q.to(dev), idx, d, want_sel=True)
+    ora = O.decode(q.double().numpy(), U.as_consumed(heads), d.k_retrieval, d.k_estimation)
+    assert U.compare_selection(sel, ora, d.k_retrieval, d.k_estimation, q, U.as_consumed(heads),
+                               4) == 0
+    U.compare_output(out, ora["out"])
+
+
+@pytest.mark.parametrize("B,H,G,N", [(5, 4, 4, 9000),     # 20 units
+                                     (8, 8, 4, 5000),     # 64 units: small clusters of blocks
+                                     (10, 16, 2, 3000),   # 160 units: more than one wave
+                                     (1, 1, 8, 40000)])   # one unit, every block of a cluster
+def test_decode_cluster_shapes(R, B, H, G, N):
+    """Unit counts that give different thread-block cluster sizes (and more
+    units than clusters resident at once)."""
+    r = _run_case(R, B, H, G, N, use_labels=True, seed=B * 7 + H, clusters=256 if N < 9000 else 512)
+    assert r["tolerated"] <= B * H
+
+
+# ---------------------------------------------------------------- bounded waits
+@pytest.mark.parametrize("hand_off", [1, 2, 3])
+def test_decode_kernel_wait_expires_and_reports_timeout(R, hand_off):
+    """One hand-off inside the decode kernel never released (a tile copy, an
+    MMA completion, an attention chunk copy) with a 2 ms limit: the kernel
+    records RI_ERR_TIMEOUT and returns, and the next normal call on the same
+    workspace and context gives the oracle's answer."""
+    dev = torch.device("cuda:0")
+    kv = S.make_kv(1, 2, 8192 + 68 + 3000, seed=44)
+    q = S.make_queries(kv, 4, seed=45)
+    heads = U.oracle_index_heads(kv, use_labels=True)
+    idx = _decode_index(R, heads, 1, 2, 4, kv.K.shape[2])
+    d = R.default_budgets(idx.geom.clusters)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(idx.cfg, d), dev)
+    R.selftest_decode_timeout(q.to(dev), idx, d, ws, hand_off, 2_000_000)
+    assert R.read_device_status(ws) == R.STATUS_CODES["RI_ERR_TIMEOUT"]
+    out, lse, sel = R.decode(q.to(dev), idx, d, workspace=ws, want_sel=True)
+    assert R.read_device_status(ws) == 0
+    ora = O.decode(q.double().numpy(), U.as_consumed(heads), d.k_retrieval, d.k_estimation)
+    U.compare_output(out, ora["out"])

@@ -367,8 +367,8 @@ ri_status ri_selftest_wait_timeout(void* workspace, uint64_t limit_ns, ri_stream
  *               issuer's wait expires);
  *   hand_off 2: the first tile's MMA completion is never signalled (the
  *               scoring epilogue's wait expires);
- *   hand_off 3: the first attention chunk's copies are never issued (the
- *               attention warps' wait expires).
+ *   hand_off 3: the cluster sizes loaded beside the scoring are never
+ *               signalled ready (the scoring epilogue's wait expires).
  * The kernel records RI_ERR_TIMEOUT in the status word, every block returns
  * after the copies it issued have landed, and the device stays usable; `out`
  * holds no meaningful result. */

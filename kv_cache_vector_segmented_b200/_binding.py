@@ -420,7 +420,7 @@ def read_device_status(workspace: torch.Tensor) -> int:
     return lib.ri_read_device_status(workspace.data_ptr(), _stream(workspace.device))
 
 
-FAULT_SCORE_COPY, FAULT_SCORE_COMMIT, FAULT_ATTEND_COPY = 1, 2, 3
+FAULT_SCORE_COPY, FAULT_SCORE_COMMIT, FAULT_SCORE_SIZES = 1, 2, 3
 
 
 def selftest_decode_timeout(q: torch.Tensor, index: Index, dcfg: DecodeConfig,

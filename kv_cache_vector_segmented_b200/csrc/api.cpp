@@ -396,7 +396,7 @@ ri_status ri_selftest_decode_timeout(const ri_index_config* cfg, const ri_decode
   ri_status st = prepare_decode(cfg, dcfg, q, idx, workspace, workspace_bytes, &g, &L);
   if (st != RI_OK) return st;
   RI_CHECK(out && aligned16(out), RI_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
-  RI_CHECK(hand_off >= RI_FAULT_SCORE_COPY && hand_off <= RI_FAULT_ATTEND_COPY,
+  RI_CHECK(hand_off >= RI_FAULT_SCORE_COPY && hand_off <= RI_FAULT_SCORE_SIZES,
            RI_ERR_INVALID_ARG, "hand_off must be 1, 2 or 3 (got %d)", hand_off);
   RI_CHECK(limit_ns > 0 && limit_ns <= 10ull * 1000000000ull, RI_ERR_INVALID_ARG,
            "limit_ns must be in (0, 10 s]");

@@ -13,34 +13,40 @@
 // The CS blocks of a cluster share one unit.  Block b owns a contiguous,
 // balanced range of the unit's 128-centroid tiles; the blocks exchange data
 // only through distributed shared memory and the cluster barrier, never
-// through global counters, so no block waits on another cluster.
+// through global counters, so no block waits on another cluster.  Data a
+// block needs from the others is pushed into its shared memory before the
+// barrier that publishes it wherever possible (a remote load costs a round
+// trip after the barrier; a remote store does not).
 //   A) Scoring: TMA brings the block's centroid tiles (128-byte swizzle, a
 //      ring of 4 stages) and the unit's query rows once; one thread issues
 //      tcgen05.mma (M = 128 centroids, N = 16 query rows, K = 128), each tile
 //      into its own TMEM columns; four epilogue warps read the fp32 scores,
-//      keep the keys r_c, sizes and first rows in shared memory and write
-//      the per-head scores s to the workspace (the estimation term reads
-//      them back).
-//   B) Selection, exact, cluster-wide: the key range (barrier 1), a 4096-
-//      bucket value histogram kept in slices across the blocks and filled
-//      by remote reductions (barrier 2), then every block reads the merged
-//      histogram and finds the two boundary buckets (ranks k_r and
-//      k_r + k_e).  The members of a boundary bucket are ranked exactly by
-//      (key desc, id asc): gathered from all blocks when there are few of
-//      them (barrier 3), else by a radix walk over the 32-bit order key and
-//      a final id count (crowded buckets, heavy ties).  Each block lists its
-//      own R clusters (first row, token prefix) and E clusters (id, size) in
-//      id order (barrier 4).
+//      keep the keys r_c in shared memory and write the per-head scores s
+//      to the workspace (the estimation term reads them back).  Eight other
+//      warps load the clusters' sizes and first rows meanwhile.
+//   B) Selection, exact, cluster-wide: the key range (barrier 1), each
+//      block's histogram of its own keys over 4096 value buckets and its
+//      sums over groups of 32 buckets, the group sums pushed to every block
+//      (barrier 2); every block finds the two boundary groups (ranks k_r and
+//      k_r + k_e from the top), reads those groups' 32 bucket counts from
+//      every block and finds the boundary buckets.  The members of a
+//      boundary bucket are ranked exactly by (key desc, id asc): pushed to
+//      every block when there are few of them (barrier 3), else found by a
+//      radix walk over the 32-bit order key and a final id count (crowded
+//      buckets, heavy ties).  Each block lists its own R clusters (first
+//      row, token prefix) and E clusters (id, size) in id order and pushes
+//      its totals (barrier 4).  Rows of clusters certain to be selected are
+//      prefetched into L2 as soon as the boundary groups are known.
 //   C) Attention: the unit's items (steady tokens, R tokens, E clusters) are
-//      split evenly over the blocks: block b takes an equal share of the
-//      tokens and an equal share of the E clusters, wherever their owners
-//      are.  One producer warp walks the owners' lists and issues bulk
-//      copies (cp.async.bulk) of whole row runs, value-sum rows and scores
-//      into a ring of 8 stages of 30 items; fifteen consumer warps fold
-//      each item into an online-softmax state on CUDA cores, half a warp
-//      per item (16 lanes x 8 dims, warp-shuffle reductions for q.k).  A
-//      token adds e^{x} v after its logit x; an E cluster adds n_c e^{s} to
-//      the denominator and e^{s} Vsum_c to the numerator.
+//      split evenly over the blocks and, inside a block, over its sixteen
+//      warps.  A planner warp turns the block's token range into row runs
+//      (from the owners' lists); every warp then streams its items through
+//      its own ring of shared-memory slots with 16-byte cp.async copies, six
+//      steps ahead, and folds them into an online-softmax state on CUDA
+//      cores, half a warp per item (16 lanes x 8 dims, warp-shuffle
+//      reductions for q.k).  A token adds e^{x} v after its logit x; an E
+//      cluster adds n_c e^{s} to the denominator and e^{s} Vsum_c to the
+//      numerator.
 //   D) Merge: the block's warps are combined in shared memory, every block
 //      writes its partial (max, denominator, numerator) into block 0's
 //      shared memory (barriers 5 and 6) and block 0 merges them by
@@ -70,8 +76,6 @@ constexpr float kRescale2 = 8.f * kLog2e;  // online softmax: new reference only
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kConsumers = 15;  // warps 0..14 fold items in step C
-constexpr int kProducer = 15;   // warp 15 issues the copies of step C
 
 constexpr int kTileC = 128;  // centroids per MMA tile (M)
 constexpr int kQRows = 16;   // MMA N: the unit's query rows, then padding
@@ -79,39 +83,67 @@ constexpr uint32_t kTileBytes = kTileC * kHeadDim * 2;  // 32 KB
 constexpr uint32_t kQBytes = kQRows * kHeadDim * 2;     // 4 KB
 constexpr int kStagesA = 4;
 constexpr int kMaxTilesPerBlock = kMaxIdsPerBlock / kTileC;  // 32
+constexpr int kMaxCS = kMaxClusterBlocks;
 
 constexpr int kNB = 4096;  // value buckets of the selection histogram
-constexpr int kBPT = kNB / kThreads;
+constexpr int kGroups = kNB / 32;
 constexpr int kCand = 256;  // boundary-bucket members ranked directly
 constexpr int kKPT = kMaxIdsPerBlock / kThreads;  // own ids per thread (contiguous)
 
-constexpr int kItems = 30;  // items per chunk of step C
-constexpr uint32_t kStageC = 16384;
-constexpr int kStagesC = 8;
-constexpr uint32_t kOffVRow = kItems * 256;  // V rows of a token chunk
-constexpr uint32_t kOffESc = kItems * 512;   // scores of an estimation chunk
-static_assert(kOffESc + kItems * 32 <= kStageC, "stage");
+// Step C: per warp a ring of slots; a slot holds one item (K and V rows of a
+// token, or the value sum of an E cluster) plus its scores or a token flag.
+constexpr uint32_t kSlot = 544;                      // 512 data + 32 scores / flag
+constexpr uint32_t kWarpRing = 8192;
+constexpr int kMaxRuns = 1024;                       // row runs planned per window
 
 // Shared memory map (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t kRingBytes = kStagesC * kStageC;
+constexpr uint32_t kRingBytes = kWarps * kWarpRing;  // 128 KB
 static_assert(kStagesA * kTileBytes == kRingBytes, "ring");
 constexpr uint32_t kOffQ = kRingBytes;                          // q tile (4 KB)
 constexpr uint32_t kOffKeys = kOffQ + kQBytes;                  // float keys[P], then lists
 constexpr uint32_t kOffMeta = kOffKeys + kMaxIdsPerBlock * 8;   // int2 (first row, size)[P]
-constexpr uint32_t kOffMisc = kOffMeta + kMaxIdsPerBlock * 8;
+constexpr uint32_t kOffRuns = kOffMeta + kMaxIdsPerBlock * 8;   // int4 runs[kMaxRuns]
+constexpr uint32_t kOffMisc = kOffRuns + kMaxRuns * 16;
 constexpr uint32_t kMiscBytes = 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory");
 
-// Inside the ring while it is free (between steps A and C, and after C).
-constexpr uint32_t kRHist = 0;                      // int [slice] merged histogram slice
-constexpr uint32_t kRDig = kRHist + kNB * 4;        // int [4 passes][2][256] digit slices
-constexpr uint32_t kRCand = kRDig + 4 * 2 * 256 * 4;  // u64 [2][kCand] own boundary members
-constexpr uint32_t kRAll = kRCand + 2 * kCand * 8;  // u64 [2][kCand] gathered members
-constexpr uint32_t kRRid = kRAll + 2 * kCand * 8;   // u16 [P] own R clusters (local index)
-static_assert(kRRid + kMaxIdsPerBlock * 2 <= kRingBytes, "selection scratch");
+// Inside the ring between steps A and C.
+constexpr uint32_t kRHist = 0;                          // int [kNB] own histogram
+constexpr uint32_t kRDig = kRHist + kNB * 4;            // int [4 passes][2][256] digit slices
+constexpr uint32_t kRGin = kRDig + 4 * 2 * 256 * 4;     // int [kMaxCS][kGroups] pushed group sums
+constexpr uint32_t kRCin = kRGin + kMaxCS * kGroups * 4;  // u64 [2][kMaxCS][kCand] pushed members
+constexpr uint32_t kRAll = kRCin + 2 * kMaxCS * kCand * 8;  // u64 [2][kCand] gathered members
+constexpr uint32_t kRRid = kRAll + 2 * kCand * 8;       // u16 [P] own R clusters (local index)
+constexpr uint32_t kRLgs = kRRid + kMaxIdsPerBlock * 2;  // int [kGroups] own group sums
+static_assert(kRLgs + kGroups * 4 <= kRingBytes, "selection scratch");
+static_assert(kCand == 256 && kThreads == 2 * kCand, "ranking maps two boundaries to 2 x 256 threads");
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
+
+// Phase timestamps for profiling builds (-DRI_DEBUG_PHASES): %globaltimer of
+// phase boundaries per block; nothing is recorded in normal builds.
+#ifdef RI_DEBUG_PHASES
+constexpr int kStampBlocks = 4096, kStamps = 64;
+__device__ unsigned long long g_phase_ns[kStampBlocks][kStamps];
+#define RI_STAMP(i, t)                                          \
+  do {                                                          \
+    if (threadIdx.x == (t) && blockIdx.x < kStampBlocks)        \
+      g_phase_ns[blockIdx.x][(i)] = globaltimer_ns();           \
+  } while (0)
+#define RI_STAMP_VAL(i, t, v)                                   \
+  do {                                                          \
+    if (threadIdx.x == (t) && blockIdx.x < kStampBlocks)        \
+      g_phase_ns[blockIdx.x][(i)] = (unsigned long long)(v);    \
+  } while (0)
+#else
+#define RI_STAMP(i, t) \
+  do {                 \
+  } while (0)
+#define RI_STAMP_VAL(i, t, v) \
+  do {                        \
+  } while (0)
+#endif
 
 struct Params {
   const __nv_bfloat16* q;
@@ -136,27 +168,30 @@ struct Params {
 };
 
 struct Misc {
-  uint64_t fullA[kStagesA], emptyA[kStagesA], tdone[kMaxTilesPerBlock], qbar, drain;
-  uint64_t fullC[kStagesC], emptyC[kStagesC];
+  uint64_t fullA[kStagesA], emptyA[kStagesA], tdone[kMaxTilesPerBlock], qbar, drain, metabar;
   uint32_t tmem;
   int abort_flag;
-  // published to the other blocks of the cluster
-  uint32_t pub_kmax, pub_kmin;
-  int pub_ninf;
-  int pub_ncand[2];
-  int pub_nR, pub_nE, pub_tokR;
-  int pub_idcnt[2];
+  uint32_t own_kmax, own_kmin;  // this block's key range (order keys) and empty clusters
+  int own_ninf;
+  int own_ncand[2];
+  int own_nR, own_nE, own_tokR;
+  int pub_idcnt[2];  // crowded path: read by the other blocks
   int pub_tid[2];
-  // cluster-wide values every block gathers
-  int nRp[kMaxClusterBlocks + 1], nEp[kMaxClusterBlocks + 1], tokRp[kMaxClusterBlocks + 1];
-  int candp[2][kMaxClusterBlocks + 1];
+  // pushed by every block of the cluster (slot = the sender's rank)
+  uint4 rng_in[kMaxCS];   // (max key, max complemented key, empty clusters, 0)
+  int candn_in[2][kMaxCS];
+  uint4 tot_in[kMaxCS];   // (R clusters, E clusters, R tokens, 0)
+  // cluster-wide values
+  int nRp[kMaxCS + 1], nEp[kMaxCS + 1], tokRp[kMaxCS + 1];
+  int candp[2][kMaxCS + 1];
   float lo, scale;
   int nfin, ninf;
   int bucket[2], above[2], nmem[2], kp[2], slow[2], digit[2], owner[2];
   unsigned long long thr[2];
-  int ecount[kStagesC][32];
+  int gsum[kGroups];  // cluster-wide group counts
+  int fine[2][32];    // cluster-wide bucket counts of the two boundary groups
   int scan[kWarps + 4];
-  int T_R;
+  int T_R, nruns, wend_lo, wend_hi;
   float wm[kWarps][8], wl[kWarps][8];
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area");
@@ -172,13 +207,15 @@ __device__ __forceinline__ uint32_t cluster_nrank() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
-// Cluster barrier in its non-.aligned form: several call sites follow
-// per-thread loops after which a warp need not have reconverged.
+// Cluster barrier in its .aligned form (whole warps); several call sites
+// follow per-thread loops, so each call first reconverges the warp.
 __device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_sync() {
   cluster_arrive();
@@ -201,10 +238,24 @@ __device__ __forceinline__ int2 ld_cl_v2(uint32_t addr) {
                : "memory");
   return v;
 }
-__device__ __forceinline__ unsigned long long ld_cl_u64(uint32_t addr) {
-  unsigned long long v;
-  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ int4 ld_cl_v4(uint32_t addr) {
+  int4 v;
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
   return v;
+}
+__device__ __forceinline__ void st_cl_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_cl_u64(uint32_t addr, unsigned long long v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_cl_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void st_cl_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
@@ -212,13 +263,6 @@ __device__ __forceinline__ void st_cl_f32(uint32_t addr, float v) {
 __device__ __forceinline__ void red_cl_add(uint32_t addr, uint32_t v) {
   asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
-// Completes `bytes` of an mbarrier's expected transaction count without a copy
-// (a copy that was skipped because its rows were out of range).
-__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   uint32_t r[8];
   asm volatile(
@@ -300,12 +344,12 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
   return r != 0;
 }
 
-// Bounded wait of every lane of a warp (each lane acquires the phase); true
-// only when every lane saw it complete.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
-                                          unsigned long long lim) {
-  const bool ok = mbar_wait(bar, parity, lim);
-  return __all_sync(0xffffffffu, ok);
+// Bounded wait on an mbarrier phase; the waiting thread is suspended in
+// hardware between probes (it resumes as soon as the phase completes), so
+// waiting warps leave the issue slots to the warps doing the work.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
+                                         unsigned long long lim) {
+  return mbar_wait_suspend(bar, parity, 20000u, lim);
 }
 
 // Online-softmax state of one lane: up to four query heads, eight dims each.
@@ -334,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_q, const Params p) {
   constexpr int Gp = G <= 4 ? 4 : 8;        // scores stored per cluster
   constexpr int HPL = G < 4 ? G : 4;        // query heads per lane in step C
-  constexpr int kPasses = G <= 4 ? 1 : 2;   // item passes per chunk and warp in step C
+  constexpr int kIPS = G <= 4 ? 2 : 1;      // items per warp step (one per half-warp)
+  constexpr int kNSW = kWarpRing / (kIPS * kSlot);  // slots ring depth per warp
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -343,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* keys = reinterpret_cast<float*>(sm + kOffKeys);
   int2* lists = reinterpret_cast<int2*>(sm + kOffKeys);
   int2* meta = reinterpret_cast<int2*>(sm + kOffMeta);
+  int4* runs = reinterpret_cast<int4*>(sm + kOffRuns);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int CS = (int)cluster_nrank();
@@ -360,12 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     ms->abort_flag = 0;
-    ms->pub_kmax = ms->pub_kmin = 0u;
-    ms->pub_ninf = 0;
-    ms->pub_ncand[0] = ms->pub_ncand[1] = 0;
+    ms->own_kmax = ms->own_kmin = 0u;
+    ms->own_ninf = 0;
+    ms->own_ncand[0] = ms->own_ncand[1] = 0;
     ms->pub_idcnt[0] = ms->pub_idcnt[1] = 0;
     ms->pub_tid[0] = ms->pub_tid[1] = -1;
-    ms->pub_nR = ms->pub_nE = ms->pub_tokR = 0;
+    ms->own_nR = ms->own_nE = ms->own_tokR = 0;
     ms->thr[0] = ms->thr[1] = 0ull;
     for (int i = 0; i < kStagesA; ++i) {
       mbar_init(&ms->fullA[i], 1);
@@ -374,13 +420,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kMaxTilesPerBlock; ++i) mbar_init(&ms->tdone[i], 1);
     mbar_init(&ms->qbar, 1);
     mbar_init(&ms->drain, 1);
-    for (int i = 0; i < kStagesC; ++i) {
-      mbar_init(&ms->fullC[i], 1);
-      mbar_init(&ms->emptyC[i], kConsumers);
-    }
+    mbar_init(&ms->metabar, 8);
     fence_barrier_init();
   }
   __syncthreads();
+  // 0: the block has started (waited on before the first remote access)
+  cluster_arrive();
+  RI_STAMP(0, 0);
+  if (p.mode != kModeSelect && tid == 32 * 3 && p.n_steady > 0) {
+    // this block's share of the steady rows into L2 (read in step C)
+    const int s0 = p.n_steady * b / CS, s1 = p.n_steady * (b + 1) / CS;
+    if (s1 > s0) {
+      const size_t r0 = (size_t)u * p.n_steady + s0;
+      prefetch_l2_bulk(p.Ks + r0 * kHeadDim, (uint32_t)(s1 - s0) * 256u);
+      prefetch_l2_bulk(p.Vs + r0 * kHeadDim, (uint32_t)(s1 - s0) * 256u);
+    }
+  }
 
   // ============================================================ step A
   if (ntiles > 0) {
@@ -405,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < ntiles; ++it) {
         if (ld_volatile(&ms->abort_flag)) break;
         const int st = it % kStagesA;
-        if (it >= kStagesA && !mbar_wait(&ms->emptyA[st], ((it / kStagesA) - 1) & 1, lim)) {
+        if (it >= kStagesA && !wait_bar(&ms->emptyA[st], ((it / kStagesA) - 1) & 1, lim)) {
           record_status(p.status, RI_ERR_TIMEOUT);
           ms->abort_flag = 1;
           break;
@@ -421,13 +476,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every copy issued lands before its stage is reused or the block exits
       for (int st = 0; st < kStagesA; ++st)
-        if (issued[st]) mbar_wait(&ms->fullA[st], (uint32_t)((issued[st] - 1) & 1), lim);
-      mbar_wait(&ms->qbar, 0, lim);
+        if (issued[st]) wait_bar(&ms->fullA[st], (uint32_t)((issued[st] - 1) & 1), lim);
+      wait_bar(&ms->qbar, 0, lim);
     } else if (warp == 1 && lane == 0) {
       // MMA issuer: D[128 x 16] = tile[128 x 128] . Q[16 x 128]^T per tile
       constexpr uint32_t idesc = umma_idesc_bf16_f32(kTileC, kQRows);
       const uint32_t qaddr = sm_base + kOffQ;
-      bool ok = mbar_wait(&ms->qbar, 0, lim);
+      bool ok = wait_bar(&ms->qbar, 0, lim);
       if (!ok) {
         record_status(p.status, RI_ERR_TIMEOUT);
         ms->abort_flag = 1;
@@ -435,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; ok && it < ntiles; ++it) {
         if (ld_volatile(&ms->abort_flag)) break;
         const int st = it % kStagesA;
-        if (!mbar_wait(&ms->fullA[st], (uint32_t)((it / kStagesA) & 1), lim)) {
+        if (!wait_bar(&ms->fullA[st], (uint32_t)((it / kStagesA) & 1), lim)) {
           record_status(p.status, RI_ERR_TIMEOUT);
           ms->abort_flag = 1;
           break;
@@ -454,26 +509,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the MMAs issued have completed before TMEM is released
       umma_commit(&ms->drain);
-      if (!mbar_wait(&ms->drain, 0, lim)) {
+      if (!wait_bar(&ms->drain, 0, lim)) {
         record_status(p.status, RI_ERR_TIMEOUT);
         ms->abort_flag = 1;
       }
+    } else if (warp >= 8) {
+      // sizes and first rows of the block's clusters, all loads in flight at
+      // once while the tiles arrive
+      const int32_t* cg = p.counts + (size_t)u * C + id0;
+      const int32_t* og = p.offsets + (size_t)u * (C + 1) + id0;
+      for (int i0 = tid - 256; i0 < nid; i0 += 4 * 256) {
+        int cv[4], ov[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + r * 256;
+          cv[r] = i < nid ? __ldg(cg + i) : 0;
+          ov[r] = i < nid ? __ldg(og + i) : 0;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (i0 + r * 256 < nid) meta[i0 + r * 256] = make_int2(ov[r], cv[r]);
+      }
+      __syncwarp();
+      if (lane == 0 && p.fault != RI_FAULT_SCORE_SIZES) mbar_arrive(&ms->metabar);
     } else if (warp >= 4 && warp < 8) {
       // epilogue: one centroid per thread
       const int quad = warp & 3;
       const int rr = quad * 32 + lane;
       uint32_t kmx = 0, kmn = 0;
       int ninf = 0;
+      bool ok = wait_bar(&ms->metabar, 0, lim);
       for (int it = 0; it < ntiles; ++it) {
         const int cl = it * kTileC + rr;
         const bool valid = cl < nid;
         const size_t gc = (size_t)u * C + id0 + cl;
-        int cnt = 0, off = 0;
-        if (valid) {  // issued before the wait so the loads overlap the MMA
-          cnt = __ldg(p.counts + gc);
-          off = __ldg(p.offsets + (size_t)u * (C + 1) + id0 + cl);
-        }
-        const bool ok = mbar_wait(&ms->tdone[it], 0, lim);
+        ok = ok && wait_bar(&ms->tdone[it], 0, lim);
         if (epilogue_any(!ok)) {  // the 128 threads leave together
           if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
           ms->abort_flag = 1;
@@ -483,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[8];
         tmem_ld8(tmem + ((uint32_t)(quad * 32) << 16) + it * kQRows, v);
         if (valid) {
+          const int cnt = meta[cl].y;
           float s[Gp];
           float rs = 0.f;
 #pragma unroll
@@ -494,7 +565,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[0] = make_float4(s[0], s[1], s[2], s[3]);
           if constexpr (Gp == 8) dst[1] = make_float4(s[4], s[5], s[6], s[7]);
           keys[cl] = cnt > 0 ? rs : -INFINITY;
-          meta[cl] = make_int2(off, cnt);
           if (cnt > 0) {
             const uint32_t o = float_order_key(rs);
             kmx = max(kmx, o);
@@ -508,9 +578,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       kmn = __reduce_max_sync(0xffffffffu, kmn);
       ninf = __reduce_add_sync(0xffffffffu, ninf);
       if (lane == 0) {
-        atomicMax(&ms->pub_kmax, kmx);
-        atomicMax(&ms->pub_kmin, kmn);
-        atomicAdd(&ms->pub_ninf, ninf);
+        atomicMax(&ms->own_kmax, kmx);
+        atomicMax(&ms->own_kmin, kmn);
+        atomicAdd(&ms->own_ninf, ninf);
       }
     }
     __syncwarp();
@@ -520,6 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, ncols);
   }
   __syncthreads();
+  RI_STAMP(1, 0);
   if (ms->abort_flag && nid > 0) {
     // a failed scoring pass leaves no usable key: the block's clusters are
     // treated as empty (selected only past every finite key, never attended)
@@ -528,32 +599,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       meta[i] = make_int2(0, 0);
     }
     if (tid == 0) {
-      ms->pub_kmax = ms->pub_kmin = 0u;
-      ms->pub_ninf = nid;
+      ms->own_kmax = ms->own_kmin = 0u;
+      ms->own_ninf = nid;
     }
     __syncthreads();
   }
+  cluster_wait();  // 0: every block of the cluster has started
 
   // ============================================================ step B
   const int kA = p.kr, kB = p.kr + p.ke;
   const bool onA = kA > 0, onB = p.ke > 0;
   if (selecting) {
-    const int HS = (kNB + CS - 1) / CS;   // histogram buckets per block
-    const int DS = (256 + CS - 1) / CS;   // radix digits per block
+    const int DS = (256 + CS - 1) / CS;  // radix digits per block (crowded buckets)
     int* hist = reinterpret_cast<int*>(sm + kRHist);
     int* dig = reinterpret_cast<int*>(sm + kRDig);
+    int* lgs = reinterpret_cast<int*>(sm + kRLgs);
+    const int* gin = reinterpret_cast<const int*>(sm + kRGin);
+    unsigned long long* cin = reinterpret_cast<unsigned long long*>(sm + kRCin);
+    unsigned long long* all = reinterpret_cast<unsigned long long*>(sm + kRAll);
     const uint32_t hist_a = sm_base + kRHist, dig_a = sm_base + kRDig;
-    for (int i = tid; i < HS; i += kThreads) hist[i] = 0;
+    // this block's key range and empty count, pushed to every block
+    if (tid < CS)
+      st_cl_v4(mapa(smem_u32(&ms->rng_in[b]), (uint32_t)tid),
+               make_uint4(ms->own_kmax, ms->own_kmin, (uint32_t)ms->own_ninf, 0u));
+    for (int i = tid; i < kNB; i += kThreads) hist[i] = 0;
     for (int i = tid; i < 4 * 2 * 256; i += kThreads) dig[i] = 0;
-    cluster_sync();  // 1: every block's key range published, slices zeroed
+    if (tid < 64) ms->fine[tid >> 5][tid & 31] = 0;
+    cluster_sync();  // 1: key ranges pushed
+    RI_STAMP(2, 0);
 
     if (warp == 0) {
       uint32_t kx = 0, kn = 0;
       int ni = 0;
       if (lane < CS) {
-        kx = ld_cl_u32(mapa(smem_u32(&ms->pub_kmax), lane));
-        kn = ld_cl_u32(mapa(smem_u32(&ms->pub_kmin), lane));
-        ni = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_ninf), lane));
+        const uint4 v = ms->rng_in[lane];
+        kx = v.x;
+        kn = v.y;
+        ni = (int)v.z;
       }
       kx = __reduce_max_sync(0xffffffffu, kx);
       kn = __reduce_max_sync(0xffffffffu, kn);
@@ -571,49 +653,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     const float lo = ms->lo, scale = ms->scale;
     const int nfin = ms->nfin, ninf = ms->ninf;
+    // the block's own histogram and group sums; the group sums are pushed
     for (int i = tid; i < nid; i += kThreads) {
       const int bk = bucket_of(keys[i], lo, scale);
-      if (bk >= 0) red_cl_add(mapa(hist_a + 4u * (uint32_t)(bk % HS), (uint32_t)(bk / HS)), 1u);
+      if (bk >= 0) atomicAdd(&hist[bk], 1);
     }
-    cluster_sync();  // 2: merged histogram complete
+    __syncthreads();
+    for (int g = warp; g < kGroups; g += kWarps) {
+      const int v = __reduce_add_sync(0xffffffffu, hist[g * 32 + lane]);
+      if (lane == 0) lgs[g] = v;
+    }
+    __syncthreads();
+    if (tid < 32 * CS) {
+      const int q = tid >> 5, j = tid & 31;  // target block, 16-byte piece
+      const int4 v = reinterpret_cast<const int4*>(lgs)[j];
+      st_cl_v4(mapa(sm_base + kRGin + 4u * (uint32_t)(b * kGroups + 4 * j), (uint32_t)q),
+               make_uint4((uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w));
+    }
+    cluster_sync();  // 2: group sums pushed; histograms final
+    RI_STAMP(3, 0);
 
-    // boundary buckets of ranks kA and kB from the top: thread t owns the
-    // kBPT consecutive buckets below kNB - kBPT t
+    // boundary buckets of ranks kA and kB from the top: first the group,
+    // then the bucket inside it
     {
-      int hc[kBPT];
-      int sum = 0;
-#pragma unroll
-      for (int i = 0; i < kBPT; ++i) {
-        const int j = kNB - 1 - kBPT * tid - i;
-        hc[i] = (int)ld_cl_u32(mapa(hist_a + 4u * (uint32_t)(j % HS), (uint32_t)(j / HS)));
+      if (tid < kGroups) {
+        int v = 0;
+        for (int q = 0; q < CS; ++q) v += gin[q * kGroups + tid];
+        ms->gsum[tid] = v;
       }
-#pragma unroll
-      for (int i = 0; i < kBPT; ++i) sum += hc[i];
       if (tid < 2) {
         const int k = tid == 0 ? kA : kB;
         const bool on = tid == 0 ? onA : onB;
         ms->bucket[tid] = !on ? -2 : (k > nfin ? -1 : -3);
         ms->above[tid] = k > nfin ? nfin : 0;
         ms->nmem[tid] = k > nfin ? ninf : 0;
+        ms->digit[tid] = -1;  // boundary group (finite case)
       }
+      __syncthreads();
+      const int gi = kGroups - 1 - tid;  // thread order = groups from the top
+      const int gs = tid < kGroups ? ms->gsum[gi] : 0;
       int total_fin;
-      const int excl = block_scan(sum, ms->scan, &total_fin);
+      const int excl = block_scan(gs, ms->scan, &total_fin);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
         const int k = w == 0 ? kA : kB;
         const bool on = w == 0 ? onA : onB;
-        if (on && k <= nfin && excl < k && excl + sum >= k) {
-          int cum = excl;
-#pragma unroll
-          for (int i = 0; i < kBPT; ++i) {
-            if (cum + hc[i] >= k) {
-              ms->bucket[w] = kNB - 1 - kBPT * tid - i;
-              ms->above[w] = cum;
-              ms->nmem[w] = hc[i];
-              break;
+        if (tid < kGroups && on && k <= nfin && excl < k && excl + gs >= k) {
+          ms->digit[w] = gi;
+          ms->above[w] = excl;
+        }
+      }
+      __syncthreads();
+      // the two boundary groups' bucket counts, summed over the blocks
+      if (tid < 2 * 8 * CS) {
+        const int w = tid / (8 * CS), r = tid - w * 8 * CS;
+        const int q = r >> 3, j = r & 7;
+        const int g = ms->digit[w];
+        if (g >= 0) {
+          const int4 v = ld_cl_v4(mapa(hist_a + 4u * (uint32_t)(g * 32 + 4 * j), (uint32_t)q));
+          if (v.x) atomicAdd(&ms->fine[w][4 * j], v.x);
+          if (v.y) atomicAdd(&ms->fine[w][4 * j + 1], v.y);
+          if (v.z) atomicAdd(&ms->fine[w][4 * j + 2], v.z);
+          if (v.w) atomicAdd(&ms->fine[w][4 * j + 3], v.w);
+        }
+      }
+      if (p.mode == kModeFull) {
+        // clusters certain to be selected whatever the exact order inside the
+        // boundary groups: their rows (R) and value sums (E) start moving
+        // into L2 while the selection finishes
+        const int gA = ms->digit[0], gB = ms->digit[1];
+        const bool finA = onA && kA <= nfin, infA = onA && kA > nfin;
+        const bool finB = onB && kB <= nfin, infB = onB && kB > nfin;
+        for (int i = tid; i < nid; i += kThreads) {
+          const float key = keys[i];
+          if (key == -INFINITY) continue;
+          const int g = bucket_of(key, lo, scale) >> 5;
+          const bool sureR = infA || (finA && g > gA);
+          const bool sureE = !sureR && ((finB && g > gB) || infB) && (!onA || (finA && g < gA));
+          if (sureR) {
+            const int2 mt = meta[i];
+            if (mt.y > 0 && mt.x >= 0 && (long long)mt.x + mt.y <= p.M) {
+              const size_t r0 = (size_t)u * p.M + mt.x;
+              prefetch_l2_bulk(p.Kr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
+              prefetch_l2_bulk(p.Vr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
             }
-            cum += hc[i];
+          } else if (sureE) {
+            prefetch_l2_bulk(p.vsum + ((size_t)u * C + id0 + i) * kHeadDim, 512u);
           }
+        }
+      }
+      __syncthreads();
+      if (warp < 2 && ms->digit[warp] >= 0) {
+        const int w = warp, g = ms->digit[w];
+        const int k = w == 0 ? kA : kB;
+        const int bkt = g * 32 + 31 - lane;  // lane order = buckets from the top
+        const int v = ms->fine[w][31 - lane];
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += t;
+        }
+        const int base = ms->above[w];
+        const unsigned hit = __ballot_sync(0xffffffffu, base + incl - v < k && base + incl >= k);
+        const int L = __ffs(hit) - 1;
+        if (lane == L) {
+          ms->bucket[w] = bkt;
+          ms->above[w] = base + incl - v;
+          ms->nmem[w] = v;
         }
       }
       __syncthreads();
@@ -623,32 +770,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         ms->slow[tid] = ms->bucket[tid] != -2 && ms->nmem[tid] > kCand;
       }
       __syncthreads();
+      RI_STAMP(12, 0);
+      RI_STAMP_VAL(20, 0, ms->nmem[0]);
+      RI_STAMP_VAL(21, 0, ms->nmem[1]);
+      RI_STAMP_VAL(22, 0, ms->slow[0] * 2 + ms->slow[1]);
     }
     const int bk0 = ms->bucket[0], bk1 = ms->bucket[1];
     const bool fast0 = bk0 != -2 && !ms->slow[0], fast1 = bk1 != -2 && !ms->slow[1];
     const bool slow0 = ms->slow[0], slow1 = ms->slow[1];
 
-    // ---- few members: gather them from every block and rank them directly
+    // ---- few members: every block pushes its members of the boundary
+    // buckets to every block, which ranks them all directly
     if (fast0 || fast1) {
-      unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kRCand);
-      unsigned long long* all = reinterpret_cast<unsigned long long*>(sm + kRAll);
       for (int i = tid; i < nid; i += kThreads) {
         const float key = keys[i];
         const int bk = bucket_of(key, lo, scale);
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           if ((w == 0 ? fast0 : fast1) && bk == (w == 0 ? bk0 : bk1)) {
-            const int slot = atomicAdd(&ms->pub_ncand[w], 1);
-            if (slot < kCand) cand[w * kCand + slot] = ord64(float_order_key(key), id0 + i);
+            const int slot = atomicAdd(&ms->own_ncand[w], 1);
+            if (slot < kCand)
+              cin[(w * kMaxCS + b) * kCand + slot] = ord64(float_order_key(key), id0 + i);
           }
         }
       }
-      cluster_sync();  // 3: every block's boundary members listed
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int n = min(kCand, ms->own_ncand[w]);
+        // (target, member) pairs, the count first
+        for (int t = tid; t < CS * (n + 1); t += kThreads) {
+          const int q = t / (n + 1), j = t - q * (n + 1);
+          if (j == n)
+            st_cl_u32(mapa(smem_u32(&ms->candn_in[w][b]), (uint32_t)q), (uint32_t)n);
+          else if (q != b)
+            st_cl_u64(mapa(sm_base + kRCin + 8u * (uint32_t)((w * kMaxCS + b) * kCand + j),
+                           (uint32_t)q),
+                      cin[(w * kMaxCS + b) * kCand + j]);
+        }
+      }
+      RI_STAMP(13, 0);
+      cluster_sync();  // 3: every block's boundary members pushed
+      RI_STAMP(14, 0);
       if (warp < 2) {
         const int w = warp;
-        int n = 0;
-        if (lane < CS)
-          n = min(kCand, (int)ld_cl_u32(mapa(smem_u32(&ms->pub_ncand[w]), lane)));
+        const int n = lane < CS ? min(kCand, ms->candn_in[w][lane]) : 0;
         int incl = n;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -666,28 +832,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = tid; j < n; j += kThreads) {
           int ob = 0;
           while (ob + 1 < CS && ms->candp[w][ob + 1] <= j) ++ob;
-          all[w * kCand + j] = ld_cl_u64(
-              mapa(sm_base + kRCand + 8u * (uint32_t)(w * kCand + j - ms->candp[w][ob]), ob));
+          all[w * kCand + j] = cin[(w * kMaxCS + ob) * kCand + j - ms->candp[w][ob]];
         }
       }
       __syncthreads();
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        if (!(w == 0 ? fast0 : fast1)) continue;
+      {
+        // threads [256 w, 256 w + n) rank boundary w's members (kCand = 256)
+        const int w = tid >> 8, j = tid & 255;
         const int n = min(kCand, ms->candp[w][CS]);
-        const int kp = ms->kp[w];  // 1-based rank inside the bucket
-        for (int j = tid; j < n; j += kThreads) {
-          const unsigned long long me = all[w * kCand + j];
+        if ((w == 0 ? fast0 : fast1) && j < n) {
+          const unsigned long long* aw = all + w * kCand;
+          const unsigned long long me = aw[j];
           int greater = 0;
-          for (int t = 0; t < n; ++t) greater += all[w * kCand + t] > me;
-          if (greater == kp - 1) ms->thr[w] = me;
+#pragma unroll 8
+          for (int t = 0; t < n; ++t) greater += aw[t] > me;
+          if (greater == ms->kp[w] - 1) ms->thr[w] = me;  // kp: 1-based rank in the bucket
         }
       }
       __syncthreads();
+      RI_STAMP(15, 0);
     }
 
     // ---- crowded bucket: radix walk over the order key, then the id count
     if (slow0 || slow1) {
+      RI_STAMP(16, 0);
       uint32_t prefix[2] = {0u, 0u}, mask[2] = {0u, 0u};
       int kp[2] = {ms->kp[0], ms->kp[1]};
       for (int pass = 0; pass < 4; ++pass) {
@@ -760,7 +928,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = __shfl_up_sync(0xffffffffu, incl, off);
           if (lane >= off) incl += t;
         }
-        const unsigned hit = __ballot_sync(0xffffffffu, lane < CS && incl - n < kp[w] && incl >= kp[w]);
+        const unsigned hit =
+            __ballot_sync(0xffffffffu, lane < CS && incl - n < kp[w] && incl >= kp[w]);
         if (lane == 0) ms->owner[w] = hit ? __ffs(hit) - 1 : -1;
         if (hit && lane == __ffs(hit) - 1) ms->candp[w][0] = incl - n;  // equal keys before it
       }
@@ -785,13 +954,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid < 2 && (tid == 0 ? slow0 : slow1)) {
         const int w = tid;
         const int ob = ms->owner[w];
-        const int id = ob >= 0 ? (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tid[w]), (uint32_t)ob)) : -1;
+        const int id =
+            ob >= 0 ? (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tid[w]), (uint32_t)ob)) : -1;
         ms->thr[w] = ord64(prefix[w], id);
         if (ob < 0 || id < 0) record_status(p.status, RI_ERR_INVALID_ARG);
       }
       __syncthreads();
     }
     const unsigned long long thrA = onA ? ms->thr[0] : ~0ull, thrB = onB ? ms->thr[1] : ~0ull;
+    RI_STAMP(4, 0);
 
     // ---- classification of the block's ids and the id-ordered lists
     {
@@ -850,18 +1021,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (tid == 0) {
-        ms->pub_nR = nR;
-        ms->pub_nE = nE;
-        ms->pub_tokR = ttot;
+        ms->own_nR = nR;
+        ms->own_nE = nE;
+        ms->own_tokR = ttot;
       }
+      if (tid < CS)
+        st_cl_v4(mapa(smem_u32(&ms->tot_in[b]), (uint32_t)tid),
+                 make_uint4((uint32_t)nR, (uint32_t)nE, (uint32_t)ttot, 0u));
     }
-    cluster_sync();  // 4: every block's lists and totals published
+    RI_STAMP(17, 0);
+    cluster_sync();  // 4: every block's lists published and totals pushed
+    RI_STAMP(5, 0);
     if (warp == 0) {
       int a = 0, e = 0, t = 0;
       if (lane < CS) {
-        a = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_nR), lane));
-        e = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_nE), lane));
-        t = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tokR), lane));
+        const uint4 v = ms->tot_in[lane];
+        a = (int)v.x;
+        e = (int)v.y;
+        t = (int)v.z;
       }
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -882,6 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ms->nRp[0] = ms->nEp[0] = ms->tokRp[0] = 0;
     }
     __syncthreads();
+    RI_STAMP(18, 0);
     // selected ids (R then E, each in id order) and the R token prefix
     {
       const bool to_ws = p.mode == kModeSelect;
@@ -892,7 +1070,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t* rpu = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
       if (selw || selu || rpw || rpu) {
         const uint16_t* rid = reinterpret_cast<const uint16_t*>(sm + kRRid);
-        const int nR = ms->pub_nR, nE = ms->pub_nE;
+        const int nR = ms->own_nR, nE = ms->own_nE;
         const int rb = ms->nRp[b], eb = ms->nEp[b], tb = ms->tokRp[b];
         for (int i = tid; i < nR; i += kThreads) {
           const int g = rb + i;
@@ -937,10 +1115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.mode == kModeSelect) p.rpre[(size_t)u * (p.k_r + 1) + i] = 0;
     }
   }
-  if (p.mode == kModeSelect) {
-    cluster_sync();  // no block leaves while others read its lists
-    return;
-  }
+  // after barrier 4 nothing reads another block's shared memory in a select
+  if (p.mode == kModeSelect) return;
 
   // ============================================================ step C
   // the unit's totals: R clusters, R tokens, E clusters
@@ -948,6 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool exec = p.exec_rows > 0;
   const int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
   const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
+  const long long lim_rows = exec ? p.exec_rows : p.M;
   if (selecting) {
     KR = ms->nRp[CS];
     KE = ms->nEp[CS];
@@ -958,7 +1135,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) ms->T_R = __ldcg(rpg + KR);
     __syncthreads();
     T_R = ms->T_R;
-    const long long lim_rows = exec ? p.exec_rows : p.M;
     if (T_R < 0 || T_R > lim_rows) {
       if (tid == 0) record_status(p.status, RI_ERR_INVALID_ARG);
       T_R = 0;
@@ -971,176 +1147,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long T = (long long)n_st + T_R;
   const long long ta = T * b / CS, tb = T * (b + 1) / CS;
   const int ea = (int)((long long)KE * b / CS), eb = (int)((long long)KE * (b + 1) / CS);
-  const int ntok = (int)(tb - ta), ne = eb - ea;
-  const int nct = (ntok + kItems - 1) / kItems, nce = (ne + kItems - 1) / kItems;
-  const int nch = nct + nce;
-  // the ring was written by the generic proxy in step B: order that before
-  // the bulk copies that write it again
-  fence_proxy_async_smem();
-  __syncthreads();
-
-  if (warp == kProducer) {
-    // ---- R list access: entry g -> (first row, first token), in the unit's
-    // token order (owners' lists in a cluster, the workspace after a select)
+  const int ne = min(eb - ea, kMaxIdsPerBlock);
+  // the block's E entries (id, size) into shared memory (the sizes and first
+  // rows of step A are no longer needed there), all loads in flight together:
+  // from the owners' lists in the cluster, or from the workspace after a select
+  int2* eplan = meta;
+  if (selecting) {
     const uint32_t lists_a = sm_base + kOffKeys;
-    auto r_entry = [&](int g, int& row, int& gs) {
-      if (g >= KR) {
-        row = 0;
-        gs = T_R;
-        return;
-      }
-      if (selecting) {
-        int ob = 0;
-        while (ob + 1 < CS && ms->nRp[ob + 1] <= g) ++ob;
-        const int2 e = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(g - ms->nRp[ob]), (uint32_t)ob));
-        row = e.x;
-        gs = ms->tokRp[ob] + e.y;
-      } else {
-        gs = __ldcg(rpg + g);
-        if (exec) {
-          row = gs;
-        } else {
-          const int id = __ldcg(selg + g);
-          row = (id >= 0 && id < C) ? __ldcg(p.offsets + (size_t)u * (C + 1) + id) : -1;
-        }
-      }
-    };
-    // first R entry whose tokens reach R token j (32-ary search)
-    int gb = 0;
-    {
-      const long long j0 = max(ta - n_st, 0ll);
-      if (KR > 0 && tb > n_st && j0 < T_R) {
-        int lo_g = 0, hi_g = KR;  // answer in [lo_g, hi_g)
-        while (hi_g - lo_g > 1) {
-          const int span = hi_g - lo_g;
-          const int step = (span + 31) / 32;
-          const int g = lo_g + lane * step;
-          int row, gs = INT_MAX;
-          if (g < hi_g) r_entry(g, row, gs);
-          const unsigned le = __ballot_sync(0xffffffffu, g < hi_g && gs <= j0);
-          const int L = le ? 31 - __clz(le) : 0;
-          lo_g = lo_g + L * step;
-          hi_g = min(hi_g, lo_g + step);
-          if (step == 1) break;
-        }
-        gb = lo_g;
-      }
+    for (int e = tid; e < ne; e += kThreads) {
+      const int ge = ea + e;
+      int ob = 0;
+      while (ob + 1 < CS && ms->nEp[ob + 1] <= ge) ++ob;
+      const int nR_ob = ms->nRp[ob + 1] - ms->nRp[ob];
+      eplan[e] = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(nR_ob + ge - ms->nEp[ob]), (uint32_t)ob));
     }
-    // batch of 32 consecutive R entries, one per lane
-    int brow = 0, bgs = 0, bcnt = 0, bend = 0;  // bend: first token after the batch
-    auto load_batch = [&]() {
-      int row, gs;
-      r_entry(gb + lane, row, gs);
-      int nrow, ngs;
-      r_entry(gb + 32, nrow, ngs);
-      const int next = __shfl_down_sync(0xffffffffu, gs, 1);
-      brow = row;
-      bgs = gs;
-      bcnt = (lane == 31 ? ngs : next) - gs;
-      bend = __shfl_sync(0xffffffffu, gs + bcnt, 31);
-    };
-    if (KR > 0) load_batch();
-    const long long lim_rows = exec ? p.exec_rows : p.M;
-    const __nv_bfloat16* Kr = p.Kr + (size_t)u * (exec ? p.exec_rows : p.M) * kHeadDim;
-    const __nv_bfloat16* Vr = p.Vr + (size_t)u * (exec ? p.exec_rows : p.M) * kHeadDim;
-    int issued = 0;
-    for (int k = 0; k < nch; ++k) {
-      if (ld_volatile(&ms->abort_flag)) break;
-      const int st = k % kStagesC;
-      if (k >= kStagesC && !warp_wait(&ms->emptyC[st], ((k / kStagesC) - 1) & 1, lim)) {
-        if (lane == 0) {
-          record_status(p.status, RI_ERR_TIMEOUT);
-          ms->abort_flag = 1;
-        }
-        break;
-      }
-      uint8_t* stage = sm + st * kStageC;
-      uint64_t* bar = &ms->fullC[st];
-      const bool skip = p.fault == RI_FAULT_ATTEND_COPY && k == 0;
-      if (k < nct) {
-        const long long i0 = ta + (long long)k * kItems;
-        const long long i1 = min(tb, i0 + kItems);
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(i1 - i0) * 512u);
-        __syncwarp();
-        // steady tokens
-        const long long s1 = min(i1, (long long)n_st);
-        if (lane == 0 && i0 < s1 && !skip) {
-          const uint32_t n = (uint32_t)(s1 - i0);
-          const size_t r0 = (size_t)u * n_st + (size_t)i0;
-          bulk_load(stage, p.Ks + r0 * kHeadDim, n * 256u, bar);
-          bulk_load(stage + kOffVRow, p.Vs + r0 * kHeadDim, n * 256u, bar);
-        }
-        // R tokens [j0, j1) of this chunk
-        const long long a0 = max(i0, (long long)n_st);
-        if (a0 < i1) {
-          const int j0 = (int)(a0 - n_st), j1 = (int)(i1 - n_st);
-          const uint32_t slot0 = (uint32_t)(a0 - i0);
-          while (true) {
-            const int lo_t = max(j0, bgs), hi_t = min(j1, bgs + bcnt);
-            if (lo_t < hi_t) {
-              const uint32_t n = (uint32_t)(hi_t - lo_t);
-              const long long row = (long long)brow + (lo_t - bgs);
-              const uint32_t slot = slot0 + (uint32_t)(lo_t - j0);
-              if (skip) {
-              } else if (row >= 0 && row + n <= lim_rows) {
-                bulk_load(stage + slot * 256u, Kr + (size_t)row * kHeadDim, n * 256u, bar);
-                bulk_load(stage + kOffVRow + slot * 256u, Vr + (size_t)row * kHeadDim, n * 256u,
-                          bar);
-              } else {
-                record_status(p.status, RI_ERR_INVALID_ARG);
-                mbar_complete_tx(bar, 2u * n * 256u);
-              }
-            }
-            if (bend >= j1 || gb + 32 >= KR) break;
-            gb += 32;
-            load_batch();
-          }
-        }
-      } else {
-        const int e0 = ea + (k - nct) * kItems;
-        const int n = min(kItems, eb - e0);
-        int id = -1, cnt = 0;
-        if (lane < n) {
-          const int e = e0 + lane;
-          if (selecting) {
-            int ob = 0;
-            while (ob + 1 < CS && ms->nEp[ob + 1] <= e) ++ob;
-            const int nR_ob = ms->nRp[ob + 1] - ms->nRp[ob];
-            const int2 v = ld_cl_v2(
-                mapa(lists_a + 8u * (uint32_t)(nR_ob + e - ms->nEp[ob]), (uint32_t)ob));
-            id = v.x;
-            cnt = v.y;
-          } else {
-            id = __ldcg(selg + p.k_r + e);
-            cnt = (id >= 0 && id < C) ? __ldg(p.counts + (size_t)u * C + id) : 0;
-          }
-          const bool ok = id >= 0 && id < C && cnt >= 0;
-          ms->ecount[st][lane] = ok ? cnt : 0;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)n * (512u + Gp * 4u));
-        __syncwarp();
-        if (lane < n && !skip) {
-          if (id >= 0 && id < C) {
-            const size_t uc = (size_t)u * C + id;
-            bulk_load(stage + lane * 512u, p.vsum + uc * kHeadDim, 512u, bar);
-            bulk_load(stage + kOffESc + lane * 32u, p.score + uc * Gp, Gp * 4u, bar);
-          } else {
-            record_status(p.status, RI_ERR_INVALID_ARG);
-            mbar_complete_tx(bar, 512u + Gp * 4u);
-          }
-        }
-      }
-      ++issued;
+  } else {
+    for (int e = tid; e < ne; e += kThreads) {
+      const int id = __ldcg(selg + p.k_r + ea + e);
+      const int cnt = (id >= 0 && id < C) ? __ldg(p.counts + (size_t)u * C + id) : 0;
+      eplan[e] = make_int2(id, cnt);
     }
-    // after a failure the copies already issued still land before the block
-    // leaves (their stages may never be consumed)
-    if (ld_volatile(&ms->abort_flag) && lane == 0)
-      for (int k = max(0, issued - kStagesC); k < issued; ++k)
-        mbar_wait(&ms->fullC[k % kStagesC], (uint32_t)((k / kStagesC) & 1), lim);
   }
 
-  // ---- consumers: online softmax over the chunks
+  // R list access for the planner: entry g -> (first row, first token) in the
+  // unit's token order (owners' lists in a cluster, the workspace after a
+  // select); g = KR gives (0, T_R)
+  const uint32_t lists_a = sm_base + kOffKeys;
+  auto r_entry = [&](int g, int& row, int& gs) {
+    if (g >= KR) {
+      row = 0;
+      gs = T_R;
+      return;
+    }
+    if (selecting) {
+      int ob = 0;
+      while (ob + 1 < CS && ms->nRp[ob + 1] <= g) ++ob;
+      const int2 e = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(g - ms->nRp[ob]), (uint32_t)ob));
+      row = e.x;
+      gs = ms->tokRp[ob] + e.y;
+    } else {
+      gs = __ldcg(rpg + g);
+      const int id = __ldcg(selg + g);
+      row = (id >= 0 && id < C) ? __ldcg(p.offsets + (size_t)u * (C + 1) + id) : -1;
+    }
+  };
+
+  // online-softmax state of this lane
   Acc acc;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -1152,103 +1204,292 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int half = lane >> 4, l16 = lane & 15;
   // query head of lane head j (G > 4: the half-warps split the heads)
   auto head_of = [&](int j) { return G <= 4 ? j : 4 * half + j; };
-  if (warp < kConsumers) {
-    float qf[4][8];
+  float qf[4][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = head_of(j);
-      if (j < HPL && g < G) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
-            p.q + ((size_t)u * G + g) * kHeadDim + l16 * 8));
-        bf16x8_to_float(raw, qf[j]);
-      } else {
+  for (int j = 0; j < 4; ++j) {
+    const int g = head_of(j);
+    if (j < HPL && g < G) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+          p.q + ((size_t)u * G + g) * kHeadDim + l16 * 8));
+      bf16x8_to_float(raw, qf[j]);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) qf[j][i] = 0.f;
+      for (int i = 0; i < 8; ++i) qf[j][i] = 0.f;
+    }
+  }
+  constexpr float kQK = kScale * kLog2e;
+  const __nv_bfloat16* Kr = p.Kr + (size_t)u * lim_rows * kHeadDim;
+  const __nv_bfloat16* Vr = p.Vr + (size_t)u * lim_rows * kHeadDim;
+  const __nv_bfloat16* Ksu = p.Ks + (size_t)u * n_st * kHeadDim;
+  const __nv_bfloat16* Vsu = p.Vs + (size_t)u * n_st * kHeadDim;
+  uint8_t* wring = sm + warp * kWarpRing;
+  RI_STAMP(19, 0);
+
+  // windows of at most kMaxRuns row runs (one window unless the block's token
+  // range crosses more than kMaxRuns clusters)
+  long long wt = ta;
+  int gnext = 0;  // first R entry not yet planned
+  bool first_window = true;
+  while (true) {
+    // ---- planner (warp 0): row runs {row, first token in the window, source}
+    if (warp == 0) {
+      int nr = 0;
+      long long cur = wt;
+      if (cur < n_st && cur < tb) {
+        if (lane == 0) runs[0] = make_int4((int)cur, 0, 0, 0);
+        nr = 1;
+        cur = min(tb, (long long)n_st);
+      }
+      if (cur < tb && exec) {
+        if (lane == 0) {
+          const int j0 = (int)(cur - n_st), cnt = (int)(tb - cur);
+          const bool ok = j0 >= 0 && (long long)j0 + cnt <= lim_rows;
+          if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
+          runs[nr] = make_int4(j0, (int)(cur - wt), ok ? 1 : 2, 0);
+        }
+        nr += 1;
+        cur = tb;
+      } else if (cur < tb) {
+        const int j1 = (int)(tb - n_st);
+        int g = gnext;
+        if (first_window) {
+          // first entry whose tokens reach R token j0 (32-ary search)
+          const int j0 = (int)(cur - n_st);
+          int lo_g = 0, hi_g = KR;
+          while (hi_g - lo_g > 1) {
+            const int step = (hi_g - lo_g + 31) / 32;
+            const int gg = lo_g + lane * step;
+            int row, gs = INT_MAX;
+            if (gg < hi_g) r_entry(gg, row, gs);
+            const unsigned le = __ballot_sync(0xffffffffu, gg < hi_g && gs <= j0);
+            const int L = le ? 31 - __clz(le) : 0;
+            lo_g = lo_g + L * step;
+            hi_g = min(hi_g, lo_g + step);
+            if (step == 1) break;
+          }
+          g = lo_g;
+        }
+        while (cur < tb && nr < kMaxRuns) {
+          int row, gs, nrow, ngs;
+          r_entry(g + lane, row, gs);
+          r_entry(g + 32, nrow, ngs);
+          const int next = __shfl_down_sync(0xffffffffu, gs, 1);
+          const int cnt = (lane == 31 ? ngs : next) - gs;
+          const int jc = (int)(cur - n_st);
+          const int lo_t = max(jc, gs), hi_t = min(j1, gs + cnt);
+          const bool emit = g + lane < KR && lo_t < hi_t;
+          const unsigned em = __ballot_sync(0xffffffffu, emit);
+          const int pos = nr + __popc(em & ((1u << lane) - 1u));
+          bool ok = true;
+          if (emit) {
+            const long long r0 = (long long)row + (lo_t - gs);
+            ok = row >= 0 && r0 + (hi_t - lo_t) <= lim_rows;
+            if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
+            if (pos < kMaxRuns) runs[pos] = make_int4((int)r0, (int)(lo_t + n_st - wt), ok ? 1 : 2, 0);
+          }
+          // how far the runs written cover (the window may stop at kMaxRuns)
+          const int taken = min(__popc(em), kMaxRuns - nr);
+          if (taken < __popc(em)) {
+            // last run kept ends where the first dropped one starts
+            int kpos = -1;
+            if (emit && pos == kMaxRuns) kpos = lo_t;
+            const unsigned kb = __ballot_sync(0xffffffffu, kpos >= 0);
+            const int stop = __shfl_sync(0xffffffffu, kpos, kb ? __ffs(kb) - 1 : 0);
+            nr = kMaxRuns;
+            cur = (long long)stop + n_st;
+            gnext = g + (kb ? __ffs(kb) - 1 : 0);
+            break;
+          }
+          nr += taken;
+          const int bend = __shfl_sync(0xffffffffu, gs + cnt, 31);
+          cur = min((long long)tb, (long long)bend + n_st);
+          g += 32;
+          gnext = g;
+          if (g >= KR) {
+            cur = tb;
+            break;
+          }
+        }
+      }
+      if (lane == 0) {
+        ms->nruns = nr;
+        ms->wend_lo = (int)(cur - wt);  // tokens in this window
       }
     }
-    constexpr float kQK = kScale * kLog2e;
-    for (int k = 0; k < nch; ++k) {
-      const int st = k % kStagesC;
-      if (!warp_wait(&ms->fullC[st], (uint32_t)((k / kStagesC) & 1), lim)) {
-        if (lane == 0) {
-          record_status(p.status, RI_ERR_TIMEOUT);
-          ms->abort_flag = 1;
-        }
-        break;
+    __syncthreads();
+    const int nr = ms->nruns;
+    const int nwt = ms->wend_lo;
+    const long long wend = wt + nwt;
+    const bool last = wend >= tb;
+    const int I = nwt + (last ? ne : 0);
+    const int ia = (int)((long long)I * warp / kWarps), ib = (int)((long long)I * (warp + 1) / kWarps);
+    const int nsteps = (ib - ia + kIPS - 1) / kIPS;
+    // load cursor: run and offset of item ia (tokens only)
+    int cr = 0, co = 0;
+    if (ia < nwt && nr > 0) {
+      int lo_r = 0, hi_r = nr - 1;  // last run with first token <= ia
+      while (lo_r < hi_r) {
+        const int mid = (lo_r + hi_r + 1) >> 1;
+        if (runs[mid].y <= ia) lo_r = mid; else hi_r = mid - 1;
       }
-      const uint8_t* stage = sm + st * kStageC;
-      const bool tok = k < nct;
-      const int n_items = tok ? min(kItems, ntok - k * kItems) : min(kItems, ne - (k - nct) * kItems);
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const int it = G <= 4 ? warp + kConsumers * half : warp + kConsumers * ps;
-        const bool valid = it < n_items;
-        const int itc = valid ? it : 0;
-        if (tok) {
-          const uint4 kraw = *reinterpret_cast<const uint4*>(stage + itc * 256 + l16 * 16);
-          const uint4 vraw = *reinterpret_cast<const uint4*>(stage + kOffVRow + itc * 256 + l16 * 16);
-          float kf[8], vf[8];
+      cr = lo_r;
+      co = ia - runs[lo_r].y;
+    }
+    auto run_len = [&](int r) { return (r + 1 < nr ? runs[r + 1].y : nwt) - runs[r].y; };
+    // issue the copies of step s (this lane's 16 bytes of each of its rows)
+    auto issue = [&](int s) {
+      uint8_t* slot = wring + (uint32_t)(s % kNSW) * (kIPS * kSlot) + (G <= 4 ? half : 0) * kSlot;
+      const int i = ia + s * kIPS + (G <= 4 ? half : 0);
+      // G > 4: both half-warps fold the same item (different heads); half 0 copies it
+      if (s < nsteps && i < ib && (G <= 4 || half == 0)) {
+        if (i < nwt) {
+          int r = cr, o = co + (G <= 4 ? half : 0);
+          while (r < nr - 1 && o >= run_len(r)) {
+            o -= run_len(r);
+            ++r;
+          }
+          const int4 rn = runs[r];
+          const bool ok = rn.z != 2;
+          if (ok) {
+            const size_t row = (size_t)rn.x + o;
+            const __nv_bfloat16* ks = (rn.z == 0 ? Ksu : Kr) + row * kHeadDim + l16 * 8;
+            const __nv_bfloat16* vs = (rn.z == 0 ? Vsu : Vr) + row * kHeadDim + l16 * 8;
+            cp_async16(slot + l16 * 16, ks);
+            cp_async16(slot + 256 + l16 * 16, vs);
+          }
+          if (l16 == 0) *reinterpret_cast<int*>(slot + 512) = ok ? 1 : 0;
+        } else {
+          const int2 ev = eplan[i - nwt];
+          if (ev.x >= 0 && ev.x < C) {
+            const size_t uc = (size_t)u * C + ev.x;
+            const float* vrow = p.vsum + uc * kHeadDim + l16 * 8;
+            cp_async16(slot + l16 * 32, vrow);
+            cp_async16(slot + l16 * 32 + 16, vrow + 4);
+            if (l16 < Gp / 4) cp_async16(slot + 512 + l16 * 16, p.score + uc * Gp + l16 * 4);
+          }
+        }
+      }
+      cp_async_commit();
+      // the cursor moves kIPS items (warp-uniform)
+      if (s < nsteps) {
+        co += kIPS;
+        while (cr < nr - 1 && co >= run_len(cr)) {
+          co -= run_len(cr);
+          ++cr;
+        }
+      }
+    };
+#ifdef RI_DEBUG_PHASES
+    long long cyc_issue = 0, cyc_wait = 0, cyc_comp = 0, cyc_t = clock64();
+#define RI_CYC(acc_)                  \
+  do {                                \
+    const long long n_ = clock64();   \
+    acc_ += n_ - cyc_t;               \
+    cyc_t = n_;                       \
+  } while (0)
+#else
+#define RI_CYC(acc_) \
+  do {               \
+  } while (0)
+#endif
+    for (int s = 0; s < kNSW - 1; ++s) issue(s);
+    RI_CYC(cyc_issue);
+    for (int s = 0; s < nsteps; ++s) {
+      issue(s + kNSW - 1);
+      RI_CYC(cyc_issue);
+      cp_async_wait<kNSW - 1>();
+      __syncwarp();
+      RI_CYC(cyc_wait);
+      const uint8_t* slot =
+          wring + (uint32_t)(s % kNSW) * (kIPS * kSlot) + (G <= 4 ? half : 0) * kSlot;
+      {
+        const int i = ia + s * kIPS + (G <= 4 ? half : 0);
+        const bool valid = i < ib;
+        const bool tok = valid && i < nwt;
+        // tokens: logits need all 16 lanes of the half (shuffles run unconditionally)
+        float kf[8], vf[8];
+        {
+          uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
+          if (tok) {
+            kraw = *reinterpret_cast<const uint4*>(slot + l16 * 16);
+            vraw = *reinterpret_cast<const uint4*>(slot + 256 + l16 * 16);
+          }
           bf16x8_to_float(kraw, kf);
           bf16x8_to_float(vraw, vf);
-          float d[4];
+        }
+        float d[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            d[j] = 0.f;
+        for (int j = 0; j < 4; ++j) {
+          d[j] = 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d[j] = fmaf(qf[j][i], kf[i], d[j]);
-          }
+          for (int t = 0; t < 8; ++t) d[j] = fmaf(qf[j][t], kf[t], d[j]);
+        }
 #pragma unroll
-          for (int off = 8; off >= 1; off >>= 1)
+        for (int off = 8; off >= 1; off >>= 1)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (j < HPL) d[j] += __shfl_xor_sync(0xffffffffu, d[j], off);
-          if (valid) {
+          for (int j = 0; j < 4; ++j)
+            if (j < HPL) d[j] += __shfl_xor_sync(0xffffffffu, d[j], off);
+        if (tok) {
+          if (*reinterpret_cast<const int*>(slot + 512)) {
 #pragma unroll
             for (int j = 0; j < HPL; ++j)
               if (head_of(j) < G) acc_add(acc, j, d[j] * kQK, 1.f, vf);
           }
         } else if (valid) {
-          const int n = ms->ecount[st][itc];
-          if (n > 0) {
-            const float4* vr = reinterpret_cast<const float4*>(stage + itc * 512 + l16 * 32);
-            const float4 v0 = vr[0], v1 = vr[1];
-            const float vf[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const float* sc = reinterpret_cast<const float*>(stage + kOffESc + itc * 32);
-            const float nf = (float)n;
+          const int2 ev = eplan[i - nwt];
+          if (ev.y > 0 && ev.x >= 0 && ev.x < C) {
+            const float4 v0 = *reinterpret_cast<const float4*>(slot + l16 * 32);
+            const float4 v1 = *reinterpret_cast<const float4*>(slot + l16 * 32 + 16);
+            const float ve[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const float* sc = reinterpret_cast<const float*>(slot + 512);
+            const float nf = (float)ev.y;
 #pragma unroll
             for (int j = 0; j < HPL; ++j)
-              if (head_of(j) < G) acc_add(acc, j, sc[head_of(j)] * kLog2e, nf, vf);
+              if (head_of(j) < G) acc_add(acc, j, sc[head_of(j)] * kLog2e, nf, ve);
           }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->emptyC[st]);
+      RI_CYC(cyc_comp);
     }
-    if (G <= 4) {
-      // the two half-warps hold the same heads: combine them
-#pragma unroll
-      for (int j = 0; j < HPL; ++j) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, acc.m[j], 16);
-        const float l2 = __shfl_xor_sync(0xffffffffu, acc.l[j], 16);
-        const float mm = fmaxf(acc.m[j], m2);
-        const float f1 = acc.m[j] == -INFINITY ? 0.f : ex2f(acc.m[j] - mm);
-        const float f2 = m2 == -INFINITY ? 0.f : ex2f(m2 - mm);
-        acc.l[j] = acc.l[j] * f1 + l2 * f2;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float o2 = __shfl_xor_sync(0xffffffffu, acc.o[j][i], 16);
-          acc.o[j][i] = acc.o[j][i] * f1 + o2 * f2;
-        }
-        acc.m[j] = mm;
-      }
+#ifdef RI_DEBUG_PHASES
+    if (lane == 0 && blockIdx.x < kStampBlocks && warp < 8) {
+      g_phase_ns[blockIdx.x][24 + warp * 4 + 0] = cyc_issue;
+      g_phase_ns[blockIdx.x][24 + warp * 4 + 1] = cyc_wait;
+      g_phase_ns[blockIdx.x][24 + warp * 4 + 2] = cyc_comp;
+      g_phase_ns[blockIdx.x][24 + warp * 4 + 3] = (unsigned long long)nsteps;
     }
+#endif
+    cp_async_wait<0>();
+    __syncthreads();  // the runs table and the slots are free again
+    if (last) break;
+    wt = wend;
+    first_window = false;
   }
-  __syncthreads();  // every chunk consumed: the ring is free
+  RI_STAMP(6, 0);
 
   // ============================================================ step D
+  if (G <= 4) {
+    // the two half-warps hold the same heads: combine them
+#pragma unroll
+    for (int j = 0; j < HPL; ++j) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, acc.m[j], 16);
+      const float l2 = __shfl_xor_sync(0xffffffffu, acc.l[j], 16);
+      const float mm = fmaxf(acc.m[j], m2);
+      const float f1 = acc.m[j] == -INFINITY ? 0.f : ex2f(acc.m[j] - mm);
+      const float f2 = m2 == -INFINITY ? 0.f : ex2f(m2 - mm);
+      acc.l[j] = acc.l[j] * f1 + l2 * f2;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float o2 = __shfl_xor_sync(0xffffffffu, acc.o[j][i], 16);
+        acc.o[j][i] = acc.o[j][i] * f1 + o2 * f2;
+      }
+      acc.m[j] = mm;
+    }
+  }
   // warps -> block partial (max in log2 units, denominator, numerator)
-  float* wo = reinterpret_cast<float*>(sm);  // [kConsumers][G][128]
-  if (warp < kConsumers && (G > 4 || half == 0)) {
+  float* wo = reinterpret_cast<float*>(sm);  // [kWarps][G][128]
+  if (G > 4 || half == 0) {
 #pragma unroll
     for (int j = 0; j < HPL; ++j) {
       const int g = head_of(j);
@@ -1276,10 +1517,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = idx / kHeadDim, d = idx - g * kHeadDim;
       float mx = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumers; ++w) mx = fmaxf(mx, ms->wm[w][g]);
+      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, ms->wm[w][g]);
       float L = 0.f, O = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumers; ++w) {
+      for (int w = 0; w < kWarps; ++w) {
         const float mw = ms->wm[w][g];
         const float f = mw == -INFINITY ? 0.f : ex2f(mw - mx);
         L = fmaf(f, ms->wl[w][g], L);
@@ -1291,6 +1532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   cluster_sync();  // 5: every block done with step C (block 0's ring is free)
+  RI_STAMP(7, 0);
   // every block's partial into block 0: [CS][G][2 + 128] floats
   const uint32_t area = sm_base;
 #pragma unroll
@@ -1327,6 +1569,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     p.out[hq * kHeadDim + d] = __float2bfloat16_rn(any ? O / L : 0.f);
     if (p.lse && d == 0) p.lse[hq] = any ? mx * kLn2 + logf(L) : -INFINITY;
   }
+#ifdef RI_DEBUG_PHASES
+  __syncthreads();
+#endif
+  RI_STAMP(8, 0);
 }
 
 // ------------------------------------------------------------------ host
@@ -1601,3 +1847,12 @@ cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_n
 }
 
 }  // namespace ri
+
+#ifdef RI_DEBUG_PHASES
+// Profiling builds only: copies the phase timestamps of the last launch.
+extern "C" int ri_debug_phase_times(unsigned long long* host, int blocks) {
+  if (blocks > ri::kStampBlocks) blocks = ri::kStampBlocks;
+  return (int)cudaMemcpyFromSymbol(host, ri::g_phase_ns,
+                                   sizeof(unsigned long long) * ri::kStamps * blocks);
+}
+#endif

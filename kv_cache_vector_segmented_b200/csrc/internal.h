@@ -62,7 +62,7 @@ enum {
   RI_FAULT_NONE = 0,
   RI_FAULT_SCORE_COPY = 1,    // the first centroid tile's copy is never issued
   RI_FAULT_SCORE_COMMIT = 2,  // the first tile's MMA completion is never signalled
-  RI_FAULT_ATTEND_COPY = 3    // the first attention chunk's copies are never issued
+  RI_FAULT_SCORE_SIZES = 3    // the cluster sizes loaded for scoring are never signalled
 };
 
 struct DecodeArgs {

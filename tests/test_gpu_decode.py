@@ -248,7 +248,7 @@ def test_decode_cluster_shapes(R, B, H, G, N):
 @pytest.mark.parametrize("hand_off", [1, 2, 3])
 def test_decode_kernel_wait_expires_and_reports_timeout(R, hand_off):
     """One hand-off inside the decode kernel never released (a tile copy, an
-    MMA completion, an attention chunk copy) with a 2 ms limit: the kernel
+    MMA completion, the cluster sizes beside the scoring) with a 2 ms limit: the kernel
     records RI_ERR_TIMEOUT and returns, and the next normal call on the same
     workspace and context gives the oracle's answer."""
     dev = torch.device("cuda:0")

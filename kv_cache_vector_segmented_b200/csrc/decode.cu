@@ -90,20 +90,22 @@ constexpr int kGroups = kNB / 32;
 constexpr int kCand = 256;  // boundary-bucket members ranked directly
 constexpr int kKPT = kMaxIdsPerBlock / kThreads;  // own ids per thread (contiguous)
 
-// Step C: per warp a ring of slots; a slot holds one item (K and V rows of a
-// token, or the value sum of an E cluster) plus its scores or a token flag.
-constexpr uint32_t kSlot = 544;                      // 512 data + 32 scores / flag
-constexpr uint32_t kWarpRing = 8192;
-constexpr int kMaxRuns = 1024;                       // row runs planned per window
+// Step C: warps 0..7 fold the tokens in tiles of 16 on the tensor cores
+// (double-buffered, 16 KB each), warps 8..15 the estimation clusters on CUDA
+// cores; the token rows of up to kWindowTokens tokens are planned at a time.
+constexpr int kTokenWarps = 8;
+constexpr int kEWarps = kWarps - kTokenWarps;
+constexpr uint32_t kTokenWarpBytes = 16384;
+constexpr int kWindowTokens = 4096;
 
 // Shared memory map (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t kRingBytes = kWarps * kWarpRing;  // 128 KB
+constexpr uint32_t kRingBytes = kTokenWarps * kTokenWarpBytes;  // 128 KB
 static_assert(kStagesA * kTileBytes == kRingBytes, "ring");
 constexpr uint32_t kOffQ = kRingBytes;                          // q tile (4 KB)
 constexpr uint32_t kOffKeys = kOffQ + kQBytes;                  // float keys[P], then lists
 constexpr uint32_t kOffMeta = kOffKeys + kMaxIdsPerBlock * 8;   // int2 (first row, size)[P]
-constexpr uint32_t kOffRuns = kOffMeta + kMaxIdsPerBlock * 8;   // int4 runs[kMaxRuns]
-constexpr uint32_t kOffMisc = kOffRuns + kMaxRuns * 16;
+constexpr uint32_t kOffRuns = kOffMeta + kMaxIdsPerBlock * 8;   // int token rows[kWindowTokens]
+constexpr uint32_t kOffMisc = kOffRuns + kWindowTokens * 4;
 constexpr uint32_t kMiscBytes = 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + base alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory");
@@ -352,23 +354,41 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
   return mbar_wait_suspend(bar, parity, 20000u, lim);
 }
 
-// Online-softmax state of one lane: up to four query heads, eight dims each.
-struct Acc {
-  float m[4], l[4], o[4][8];
-};
-
-__device__ __forceinline__ void acc_add(Acc& a, int j, float x, float w_n, const float (&v)[8]) {
-  if (x > a.m[j] + kRescale2) {  // new reference (also the first item)
-    const float c = a.m[j] == -INFINITY ? 0.f : ex2f(a.m[j] - x);
-    a.l[j] *= c;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a.o[j][i] *= c;
-    a.m[j] = x;
-  }
-  const float pj = ex2f(x - a.m[j]);
-  a.l[j] = fmaf(w_n, pj, a.l[j]);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a.o[j][i] = fmaf(pj, v[i], a.o[j][i]);
+// ---- warp-level tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 acc)
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// d += A . B with A 16x16 row-major (regs a0..a3), B 16x8 column-major (b0, b1)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// 16-byte global -> shared copy; with fill == false the 16 bytes are zeroed
+// and nothing is read.
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool fill) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(fill ? 16 : 0)
+               : "memory");
+}
+// Barrier of the token warps only (named barrier 2, 256 threads).
+__device__ __forceinline__ void token_bar() {
+  asm volatile("bar.sync 2, 256;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ kernel
@@ -377,9 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_cent,
                   const __grid_constant__ CUtensorMap tm_q, const Params p) {
   constexpr int Gp = G <= 4 ? 4 : 8;        // scores stored per cluster
-  constexpr int HPL = G < 4 ? G : 4;        // query heads per lane in step C
-  constexpr int kIPS = G <= 4 ? 2 : 1;      // items per warp step (one per half-warp)
-  constexpr int kNSW = kWarpRing / (kIPS * kSlot);  // slots ring depth per warp
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -388,7 +405,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* keys = reinterpret_cast<float*>(sm + kOffKeys);
   int2* lists = reinterpret_cast<int2*>(sm + kOffKeys);
   int2* meta = reinterpret_cast<int2*>(sm + kOffMeta);
-  int4* runs = reinterpret_cast<int4*>(sm + kOffRuns);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int CS = (int)cluster_nrank();
@@ -1192,69 +1208,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  // online-softmax state of this lane
-  Acc acc;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    acc.m[j] = -INFINITY;
-    acc.l[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc.o[j][i] = 0.f;
-  }
-  const int half = lane >> 4, l16 = lane & 15;
-  // query head of lane head j (G > 4: the half-warps split the heads)
-  auto head_of = [&](int j) { return G <= 4 ? j : 4 * half + j; };
-  float qf[4][8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int g = head_of(j);
-    if (j < HPL && g < G) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
-          p.q + ((size_t)u * G + g) * kHeadDim + l16 * 8));
-      bf16x8_to_float(raw, qf[j]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qf[j][i] = 0.f;
-    }
-  }
-  constexpr float kQK = kScale * kLog2e;
-  const __nv_bfloat16* Kr = p.Kr + (size_t)u * lim_rows * kHeadDim;
-  const __nv_bfloat16* Vr = p.Vr + (size_t)u * lim_rows * kHeadDim;
-  const __nv_bfloat16* Ksu = p.Ks + (size_t)u * n_st * kHeadDim;
-  const __nv_bfloat16* Vsu = p.Vs + (size_t)u * n_st * kHeadDim;
-  uint8_t* wring = sm + warp * kWarpRing;
+  // ---- tensor-core helpers of the token tiles are below the kernel's
+  // selection code; the state of the two kinds of warps:
+  //  token warps (0..7): O^T fragments ot[j][i] (lane holds dims 16 j + gid
+  //   (+8), heads 2 tig (+1)), the running maximum tm of head gid (log2
+  //   units) and the lane's share tl of head gid's denominator;
+  //  estimation warps (8..15): per head the maximum em, denominator el and
+  //   numerators eo[g][4] of dims 4 lane .. 4 lane + 3.
+  // Each kind of warp writes its partial into wo [kWarps][G][128] (the ring,
+  // once every warp is done with it) and wm / wl.
+  float* wo = reinterpret_cast<float*>(sm);
+  // the E entries are staged; the ring was last written by the TMA (async
+  // proxy) and by step B: order both before the copies of step C
+  fence_proxy_async_smem();
+  __syncthreads();
   RI_STAMP(19, 0);
-
-  // windows of at most kMaxRuns row runs (one window unless the block's token
-  // range crosses more than kMaxRuns clusters)
-  long long wt = ta;
-  int gnext = 0;  // first R entry not yet planned
-  bool first_window = true;
-  while (true) {
-    // ---- planner (warp 0): row runs {row, first token in the window, source}
-    if (warp == 0) {
-      int nr = 0;
-      long long cur = wt;
-      if (cur < n_st && cur < tb) {
-        if (lane == 0) runs[0] = make_int4((int)cur, 0, 0, 0);
-        nr = 1;
-        cur = min(tb, (long long)n_st);
+  if (warp < kTokenWarps) {
+    const int gid = lane >> 2, tig = lane & 3;
+    float ot[8][4];
+    float tm = -INFINITY, tl = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ot[j][i] = 0.f;
+    // A fragments of Q (rows = query heads, padded to 16 with zeros):
+    // qa[kk][0] = Q[gid][16 kk + 2 tig ..], qa[kk][1] = Q[gid][16 kk + 8 + 2 tig ..]
+    uint32_t qa[8][2];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      if (gid < G) {
+        const __nv_bfloat16* qr = p.q + ((size_t)u * G + gid) * kHeadDim + kk * 16 + tig * 2;
+        qa[kk][0] = __ldg(reinterpret_cast<const unsigned int*>(qr));
+        qa[kk][1] = __ldg(reinterpret_cast<const unsigned int*>(qr + 8));
+      } else {
+        qa[kk][0] = qa[kk][1] = 0u;
       }
-      if (cur < tb && exec) {
-        if (lane == 0) {
-          const int j0 = (int)(cur - n_st), cnt = (int)(tb - cur);
-          const bool ok = j0 >= 0 && (long long)j0 + cnt <= lim_rows;
-          if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
-          runs[nr] = make_int4(j0, (int)(cur - wt), ok ? 1 : 2, 0);
+    }
+    const __nv_bfloat16* Kr = p.Kr + (size_t)u * lim_rows * kHeadDim;
+    const __nv_bfloat16* Vr = p.Vr + (size_t)u * lim_rows * kHeadDim;
+    const __nv_bfloat16* Ksu = p.Ks + (size_t)u * n_st * kHeadDim;
+    const __nv_bfloat16* Vsu = p.Vs + (size_t)u * n_st * kHeadDim;
+    const __nv_bfloat16* safe = n_st > 0 ? Ksu : Kr;  // a readable address for zero fills
+    uint8_t* wbuf = sm + warp * kTokenWarpBytes;       // two tiles of 16 rows (K then V)
+    int* rowtab = reinterpret_cast<int*>(sm + kOffRuns);
+    // 16-byte chunk c of token row t of a tile, XOR-swizzled for ldmatrix
+    auto row_chunk = [](int t, int c) { return (uint32_t)(t * 256 + ((c ^ (t & 7)) << 4)); };
+    long long wt = ta;
+    while (true) {
+      // ---- planner (warp 0): the window's token rows (R rows >= 0, steady
+      // rows as -1 - row, INT_MIN for rows out of range)
+      if (warp == 0) {
+        const long long wend = min(tb, wt + kWindowTokens);
+        long long cur = wt;
+        if (cur < n_st && cur < wend) {
+          const int s1 = (int)min(wend, (long long)n_st);
+          for (int t = (int)cur + lane; t < s1; t += 32) rowtab[t - wt] = -1 - t;
+          cur = s1;
         }
-        nr += 1;
-        cur = tb;
-      } else if (cur < tb) {
-        const int j1 = (int)(tb - n_st);
-        int g = gnext;
-        if (first_window) {
-          // first entry whose tokens reach R token j0 (32-ary search)
-          const int j0 = (int)(cur - n_st);
+        if (cur < wend && exec) {
+          for (long long t = cur + lane; t < wend; t += 32) {
+            const long long j = t - n_st;
+            rowtab[t - wt] = j < lim_rows ? (int)j : INT_MIN;
+          }
+          if (lane == 0 && (long long)(wend - n_st) > lim_rows)
+            record_status(p.status, RI_ERR_INVALID_ARG);
+          cur = wend;
+        } else if (cur < wend) {
+          // first R entry whose tokens reach R token j0 (32-ary search)
+          const int j0 = (int)(cur - n_st), j1 = (int)(wend - n_st);
           int lo_g = 0, hi_g = KR;
           while (hi_g - lo_g > 1) {
             const int step = (hi_g - lo_g + 31) / 32;
@@ -1267,244 +1288,235 @@ __global__ void __launch_bounds__(kThreads, 1)
             hi_g = min(hi_g, lo_g + step);
             if (step == 1) break;
           }
-          g = lo_g;
+          // batches of 32 entries, one per lane: each lane writes its rows
+          for (int g = lo_g; g < KR; g += 32) {
+            int row, gs, nrow, ngs;
+            r_entry(g + lane, row, gs);
+            r_entry(g + 32, nrow, ngs);
+            const int next = __shfl_down_sync(0xffffffffu, gs, 1);
+            const int cnt = (lane == 31 ? ngs : next) - gs;
+            const int lo_t = max(j0, gs), hi_t = min(j1, gs + cnt);
+            if (g + lane < KR && lo_t < hi_t) {
+              const long long r0 = (long long)row + (lo_t - gs);
+              const bool ok = row >= 0 && r0 + (hi_t - lo_t) <= lim_rows;
+              if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
+              for (int t = lo_t; t < hi_t; ++t)
+                rowtab[t + n_st - wt] = ok ? (int)(r0 + (t - lo_t)) : INT_MIN;
+            }
+            const int bend = __shfl_sync(0xffffffffu, gs + cnt, 31);
+            if (bend >= j1) break;
+          }
+          cur = wend;
         }
-        while (cur < tb && nr < kMaxRuns) {
-          int row, gs, nrow, ngs;
-          r_entry(g + lane, row, gs);
-          r_entry(g + 32, nrow, ngs);
-          const int next = __shfl_down_sync(0xffffffffu, gs, 1);
-          const int cnt = (lane == 31 ? ngs : next) - gs;
-          const int jc = (int)(cur - n_st);
-          const int lo_t = max(jc, gs), hi_t = min(j1, gs + cnt);
-          const bool emit = g + lane < KR && lo_t < hi_t;
-          const unsigned em = __ballot_sync(0xffffffffu, emit);
-          const int pos = nr + __popc(em & ((1u << lane) - 1u));
-          bool ok = true;
-          if (emit) {
-            const long long r0 = (long long)row + (lo_t - gs);
-            ok = row >= 0 && r0 + (hi_t - lo_t) <= lim_rows;
-            if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
-            if (pos < kMaxRuns) runs[pos] = make_int4((int)r0, (int)(lo_t + n_st - wt), ok ? 1 : 2, 0);
+        if (lane == 0) ms->wend_lo = (int)(cur - wt);
+      }
+      token_bar();
+      const int nwt = ms->wend_lo;
+      const int ntile = (nwt + 15) >> 4;
+      // ---- tiles warp, warp + kTokenWarps, ...: copies one tile ahead
+      auto issue = [&](int tj, int slot) {
+        if (tj < ntile) {
+          uint8_t* kb = wbuf + slot * 8192;
+          const int t = lane >> 1, c0 = (lane & 1) * 8;
+          const int tok = tj * 16 + t;
+          const int code = tok < nwt ? rowtab[tok] : INT_MIN;
+          const __nv_bfloat16 *ks = safe, *vs = safe;
+          bool fill = code != INT_MIN;
+          if (code >= 0) {
+            ks = Kr + (size_t)code * kHeadDim;
+            vs = Vr + (size_t)code * kHeadDim;
+          } else if (fill) {
+            ks = Ksu + (size_t)(-1 - code) * kHeadDim;
+            vs = Vsu + (size_t)(-1 - code) * kHeadDim;
           }
-          // how far the runs written cover (the window may stop at kMaxRuns)
-          const int taken = min(__popc(em), kMaxRuns - nr);
-          if (taken < __popc(em)) {
-            // last run kept ends where the first dropped one starts
-            int kpos = -1;
-            if (emit && pos == kMaxRuns) kpos = lo_t;
-            const unsigned kb = __ballot_sync(0xffffffffu, kpos >= 0);
-            const int stop = __shfl_sync(0xffffffffu, kpos, kb ? __ffs(kb) - 1 : 0);
-            nr = kMaxRuns;
-            cur = (long long)stop + n_st;
-            gnext = g + (kb ? __ffs(kb) - 1 : 0);
-            break;
+#pragma unroll
+          for (int c = c0; c < c0 + 8; ++c) {
+            cp_async16_zfill(kb + row_chunk(t, c), fill ? ks + c * 8 : safe, fill);
+            cp_async16_zfill(kb + 4096 + row_chunk(t, c), fill ? vs + c * 8 : safe, fill);
           }
-          nr += taken;
-          const int bend = __shfl_sync(0xffffffffu, gs + cnt, 31);
-          cur = min((long long)tb, (long long)bend + n_st);
-          g += 32;
-          gnext = g;
-          if (g >= KR) {
-            cur = tb;
-            break;
+        }
+        cp_async_commit();
+      };
+      constexpr float kQK = kScale * kLog2e;
+      int slot = 0;
+      issue(warp, 0);
+      for (int tj = warp; tj < ntile; tj += kTokenWarps) {
+        issue(tj + kTokenWarps, slot ^ 1);
+        cp_async_wait<1>();
+        __syncwarp();
+        const uint32_t kbase = smem_u32(wbuf + slot * 8192);
+        const uint32_t vbase = kbase + 4096;
+        // S = Q K^T for tokens 16 tj .. +15: two n-tiles of 8 tokens
+        float sacc[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sacc[h][i] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {  // dims 32 kp .. 32 kp + 31
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // matrices: (tokens 8h.., dim chunk 4kp + m) for m = 0..3
+            const int tr = h * 8 + (lane & 7), ch = kp * 4 + (lane >> 3);
+            uint32_t bq[4];
+            ldmatrix_x4(bq, kbase + row_chunk(tr, ch));
+            mma_bf16_16816(sacc[h], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, bq[0], bq[1]);
+            mma_bf16_16816(sacc[h], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, bq[2], bq[3]);
           }
+        }
+        // row gid: logits of tokens 8h + 2 tig (+1); padding and rows out of range masked
+        float x[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int t = tj * 16 + h * 8 + tig * 2 + i;
+            const bool ok = t < nwt && rowtab[t] != INT_MIN;
+            x[h * 2 + i] = ok ? sacc[h][i] * kQK : -INFINITY;
+          }
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        float corr = 1.f;
+        if (mx > tm + kRescale2) {  // new reference (also the first tile)
+          corr = tm == -INFINITY ? 0.f : ex2f(tm - mx);
+          tm = mx;
+          tl *= corr;
+        }
+        // O^T columns 2 tig, 2 tig + 1 rescale by the factors of those rows
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+          const float c0 = __shfl_sync(0xffffffffu, corr, (tig * 2) * 4);
+          const float c1 = __shfl_sync(0xffffffffu, corr, (tig * 2 + 1) * 4);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            ot[j][0] *= c0;
+            ot[j][1] *= c1;
+            ot[j][2] *= c0;
+            ot[j][3] *= c1;
+          }
+        }
+        float pv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          pv[i] = ex2f(x[i] - tm);
+          tl += pv[i];
+        }
+        const uint32_t pb0 = pack_bf16x2(pv[0], pv[1]);  // tokens 2 tig, +1
+        const uint32_t pb1 = pack_bf16x2(pv[2], pv[3]);  // tokens 8 + 2 tig, +1
+        // O^T += V^T P^T: 8 dim groups of 16
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          // matrices: (tokens 8 (m >> 1).., dim chunk 2 j + (m & 1)) for m = 0..3
+          const int m4 = lane >> 3;
+          const int tr = (m4 >> 1) * 8 + (lane & 7), ch = j * 2 + (m4 & 1);
+          uint32_t av[4];
+          ldmatrix_x4_trans(av, vbase + row_chunk(tr, ch));
+          mma_bf16_16816(ot[j], av[0], av[1], av[2], av[3], pb0, pb1);
+        }
+        __syncwarp();
+        slot ^= 1;
+      }
+      cp_async_wait<0>();
+      token_bar();  // the row table is rebuilt for the next window
+      const long long wend = wt + nwt;
+      if (wend >= tb) break;
+      wt = wend;
+    }
+    __syncthreads();  // every warp done with step C: the ring is free
+    tl += __shfl_xor_sync(0xffffffffu, tl, 1);
+    tl += __shfl_xor_sync(0xffffffffu, tl, 2);
+    if (tig == 0 && gid < G) {
+      ms->wm[warp][gid] = tm;
+      ms->wl[warp][gid] = tl;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int g = tig * 2 + k;
+        if (g < G) {
+          float* rg = wo + ((size_t)warp * G + g) * kHeadDim + j * 16 + gid;
+          rg[0] = ot[j][k];
+          rg[8] = ot[j][2 + k];
         }
       }
+  } else {
+    float em[G], el[G], eo[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      em[g] = -INFINITY;
+      el[g] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) eo[g][i] = 0.f;
+    }
+    // ---- estimation clusters [ea', eb') of this warp, in batches: value-sum
+    // rows (lane: dims 4 lane .. 4 lane + 3) and scores straight from L2
+    constexpr int kEB = G <= 4 ? 8 : 4;  // clusters per batch
+    const int ew = warp - kTokenWarps;
+    const int e0 = ne * ew / kEWarps, e1 = ne * (ew + 1) / kEWarps;
+    for (int eb0 = e0; eb0 < e1; eb0 += kEB) {
+      float4 vv[kEB];
+      float sc[kEB][Gp];
+      float nf[kEB];
+#pragma unroll
+      for (int k = 0; k < kEB; ++k) {
+        const int e = eb0 + k;
+        const int2 ev = e < e1 ? eplan[e] : make_int2(-1, 0);
+        const bool ok = ev.x >= 0 && ev.x < C && ev.y > 0;
+        nf[k] = ok ? (float)ev.y : 0.f;
+        const size_t uc = (size_t)u * C + (ok ? ev.x : 0);
+        vv[k] = ok ? __ldg(reinterpret_cast<const float4*>(p.vsum + uc * kHeadDim) + lane)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g4 = 0; g4 < Gp / 4; ++g4) {
+          const float4 s4 = ok ? __ldcg(reinterpret_cast<const float4*>(p.score + uc * Gp) + g4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          sc[k][4 * g4] = s4.x;
+          sc[k][4 * g4 + 1] = s4.y;
+          sc[k][4 * g4 + 2] = s4.z;
+          sc[k][4 * g4 + 3] = s4.w;
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float bm = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kEB; ++k)
+          if (nf[k] > 0.f) bm = fmaxf(bm, sc[k][g] * kLog2e);
+        if (bm > em[g] + kRescale2) {  // new reference
+          const float c = em[g] == -INFINITY ? 0.f : ex2f(em[g] - bm);
+          el[g] *= c;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) eo[g][i] *= c;
+          em[g] = bm;
+        }
+#pragma unroll
+        for (int k = 0; k < kEB; ++k) {
+          const float w = nf[k] > 0.f ? ex2f(sc[k][g] * kLog2e - em[g]) : 0.f;
+          el[g] = fmaf(nf[k], w, el[g]);
+          eo[g][0] = fmaf(w, vv[k].x, eo[g][0]);
+          eo[g][1] = fmaf(w, vv[k].y, eo[g][1]);
+          eo[g][2] = fmaf(w, vv[k].z, eo[g][2]);
+          eo[g][3] = fmaf(w, vv[k].w, eo[g][3]);
+        }
+      }
+    }
+    __syncthreads();  // every warp done with step C: the ring is free
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      *reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + lane * 4) =
+          make_float4(eo[g][0], eo[g][1], eo[g][2], eo[g][3]);
       if (lane == 0) {
-        ms->nruns = nr;
-        ms->wend_lo = (int)(cur - wt);  // tokens in this window
-      }
-    }
-    __syncthreads();
-    const int nr = ms->nruns;
-    const int nwt = ms->wend_lo;
-    const long long wend = wt + nwt;
-    const bool last = wend >= tb;
-    const int I = nwt + (last ? ne : 0);
-    const int ia = (int)((long long)I * warp / kWarps), ib = (int)((long long)I * (warp + 1) / kWarps);
-    const int nsteps = (ib - ia + kIPS - 1) / kIPS;
-    // load cursor: run and offset of item ia (tokens only)
-    int cr = 0, co = 0;
-    if (ia < nwt && nr > 0) {
-      int lo_r = 0, hi_r = nr - 1;  // last run with first token <= ia
-      while (lo_r < hi_r) {
-        const int mid = (lo_r + hi_r + 1) >> 1;
-        if (runs[mid].y <= ia) lo_r = mid; else hi_r = mid - 1;
-      }
-      cr = lo_r;
-      co = ia - runs[lo_r].y;
-    }
-    auto run_len = [&](int r) { return (r + 1 < nr ? runs[r + 1].y : nwt) - runs[r].y; };
-    // issue the copies of step s (this lane's 16 bytes of each of its rows)
-    auto issue = [&](int s) {
-      uint8_t* slot = wring + (uint32_t)(s % kNSW) * (kIPS * kSlot) + (G <= 4 ? half : 0) * kSlot;
-      const int i = ia + s * kIPS + (G <= 4 ? half : 0);
-      // G > 4: both half-warps fold the same item (different heads); half 0 copies it
-      if (s < nsteps && i < ib && (G <= 4 || half == 0)) {
-        if (i < nwt) {
-          int r = cr, o = co + (G <= 4 ? half : 0);
-          while (r < nr - 1 && o >= run_len(r)) {
-            o -= run_len(r);
-            ++r;
-          }
-          const int4 rn = runs[r];
-          const bool ok = rn.z != 2;
-          if (ok) {
-            const size_t row = (size_t)rn.x + o;
-            const __nv_bfloat16* ks = (rn.z == 0 ? Ksu : Kr) + row * kHeadDim + l16 * 8;
-            const __nv_bfloat16* vs = (rn.z == 0 ? Vsu : Vr) + row * kHeadDim + l16 * 8;
-            cp_async16(slot + l16 * 16, ks);
-            cp_async16(slot + 256 + l16 * 16, vs);
-          }
-          if (l16 == 0) *reinterpret_cast<int*>(slot + 512) = ok ? 1 : 0;
-        } else {
-          const int2 ev = eplan[i - nwt];
-          if (ev.x >= 0 && ev.x < C) {
-            const size_t uc = (size_t)u * C + ev.x;
-            const float* vrow = p.vsum + uc * kHeadDim + l16 * 8;
-            cp_async16(slot + l16 * 32, vrow);
-            cp_async16(slot + l16 * 32 + 16, vrow + 4);
-            if (l16 < Gp / 4) cp_async16(slot + 512 + l16 * 16, p.score + uc * Gp + l16 * 4);
-          }
-        }
-      }
-      cp_async_commit();
-      // the cursor moves kIPS items (warp-uniform)
-      if (s < nsteps) {
-        co += kIPS;
-        while (cr < nr - 1 && co >= run_len(cr)) {
-          co -= run_len(cr);
-          ++cr;
-        }
-      }
-    };
-#ifdef RI_DEBUG_PHASES
-    long long cyc_issue = 0, cyc_wait = 0, cyc_comp = 0, cyc_t = clock64();
-#define RI_CYC(acc_)                  \
-  do {                                \
-    const long long n_ = clock64();   \
-    acc_ += n_ - cyc_t;               \
-    cyc_t = n_;                       \
-  } while (0)
-#else
-#define RI_CYC(acc_) \
-  do {               \
-  } while (0)
-#endif
-    for (int s = 0; s < kNSW - 1; ++s) issue(s);
-    RI_CYC(cyc_issue);
-    for (int s = 0; s < nsteps; ++s) {
-      issue(s + kNSW - 1);
-      RI_CYC(cyc_issue);
-      cp_async_wait<kNSW - 1>();
-      __syncwarp();
-      RI_CYC(cyc_wait);
-      const uint8_t* slot =
-          wring + (uint32_t)(s % kNSW) * (kIPS * kSlot) + (G <= 4 ? half : 0) * kSlot;
-      {
-        const int i = ia + s * kIPS + (G <= 4 ? half : 0);
-        const bool valid = i < ib;
-        const bool tok = valid && i < nwt;
-        // tokens: logits need all 16 lanes of the half (shuffles run unconditionally)
-        float kf[8], vf[8];
-        {
-          uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
-          if (tok) {
-            kraw = *reinterpret_cast<const uint4*>(slot + l16 * 16);
-            vraw = *reinterpret_cast<const uint4*>(slot + 256 + l16 * 16);
-          }
-          bf16x8_to_float(kraw, kf);
-          bf16x8_to_float(vraw, vf);
-        }
-        float d[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          d[j] = 0.f;
-#pragma unroll
-          for (int t = 0; t < 8; ++t) d[j] = fmaf(qf[j][t], kf[t], d[j]);
-        }
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (j < HPL) d[j] += __shfl_xor_sync(0xffffffffu, d[j], off);
-        if (tok) {
-          if (*reinterpret_cast<const int*>(slot + 512)) {
-#pragma unroll
-            for (int j = 0; j < HPL; ++j)
-              if (head_of(j) < G) acc_add(acc, j, d[j] * kQK, 1.f, vf);
-          }
-        } else if (valid) {
-          const int2 ev = eplan[i - nwt];
-          if (ev.y > 0 && ev.x >= 0 && ev.x < C) {
-            const float4 v0 = *reinterpret_cast<const float4*>(slot + l16 * 32);
-            const float4 v1 = *reinterpret_cast<const float4*>(slot + l16 * 32 + 16);
-            const float ve[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const float* sc = reinterpret_cast<const float*>(slot + 512);
-            const float nf = (float)ev.y;
-#pragma unroll
-            for (int j = 0; j < HPL; ++j)
-              if (head_of(j) < G) acc_add(acc, j, sc[head_of(j)] * kLog2e, nf, ve);
-          }
-        }
-      }
-      __syncwarp();
-      RI_CYC(cyc_comp);
-    }
-#ifdef RI_DEBUG_PHASES
-    if (lane == 0 && blockIdx.x < kStampBlocks && warp < 8) {
-      g_phase_ns[blockIdx.x][24 + warp * 4 + 0] = cyc_issue;
-      g_phase_ns[blockIdx.x][24 + warp * 4 + 1] = cyc_wait;
-      g_phase_ns[blockIdx.x][24 + warp * 4 + 2] = cyc_comp;
-      g_phase_ns[blockIdx.x][24 + warp * 4 + 3] = (unsigned long long)nsteps;
-    }
-#endif
-    cp_async_wait<0>();
-    __syncthreads();  // the runs table and the slots are free again
-    if (last) break;
-    wt = wend;
-    first_window = false;
-  }
-  RI_STAMP(6, 0);
-
-  // ============================================================ step D
-  if (G <= 4) {
-    // the two half-warps hold the same heads: combine them
-#pragma unroll
-    for (int j = 0; j < HPL; ++j) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, acc.m[j], 16);
-      const float l2 = __shfl_xor_sync(0xffffffffu, acc.l[j], 16);
-      const float mm = fmaxf(acc.m[j], m2);
-      const float f1 = acc.m[j] == -INFINITY ? 0.f : ex2f(acc.m[j] - mm);
-      const float f2 = m2 == -INFINITY ? 0.f : ex2f(m2 - mm);
-      acc.l[j] = acc.l[j] * f1 + l2 * f2;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float o2 = __shfl_xor_sync(0xffffffffu, acc.o[j][i], 16);
-        acc.o[j][i] = acc.o[j][i] * f1 + o2 * f2;
-      }
-      acc.m[j] = mm;
-    }
-  }
-  // warps -> block partial (max in log2 units, denominator, numerator)
-  float* wo = reinterpret_cast<float*>(sm);  // [kWarps][G][128]
-  if (G > 4 || half == 0) {
-#pragma unroll
-    for (int j = 0; j < HPL; ++j) {
-      const int g = head_of(j);
-      if (g < G) {
-        float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + l16 * 8);
-        dst[0] = make_float4(acc.o[j][0], acc.o[j][1], acc.o[j][2], acc.o[j][3]);
-        dst[1] = make_float4(acc.o[j][4], acc.o[j][5], acc.o[j][6], acc.o[j][7]);
-        if (l16 == 0) {
-          ms->wm[warp][g] = acc.m[j];
-          ms->wl[warp][g] = acc.l[j];
-        }
+        ms->wm[warp][g] = em[g];
+        ms->wl[warp][g] = el[g];
       }
     }
   }
   __syncthreads();
+  RI_STAMP(6, 0);
+
+  // ============================================================ step D
+  // warps -> block partial (max in log2 units, denominator, numerator)
   constexpr int kOutPer = (G * kHeadDim + kThreads - 1) / kThreads;
   float bo[kOutPer], bmv[kOutPer], blv[kOutPer];
 #pragma unroll

@@ -97,6 +97,11 @@ constexpr int kTokenWarps = 8;
 constexpr int kEWarps = kWarps - kTokenWarps;
 constexpr uint32_t kTokenWarpBytes = 16384;
 constexpr int kWindowTokens = 4096;
+// estimation warps: rings of kESlots slots (value sum 512 B + scores 32 B)
+// in the size-and-row area of step A, free by then
+constexpr uint32_t kSlotE = 544;
+constexpr uint32_t kEWarpBytes = 4096;
+constexpr int kESlots = (int)(kEWarpBytes / kSlotE);
 
 // Shared memory map (byte offsets from a 1024-byte aligned base).
 constexpr uint32_t kRingBytes = kTokenWarps * kTokenWarpBytes;  // 128 KB
@@ -118,7 +123,9 @@ constexpr uint32_t kRCin = kRGin + kMaxCS * kGroups * 4;  // u64 [2][kMaxCS][kCa
 constexpr uint32_t kRAll = kRCin + 2 * kMaxCS * kCand * 8;  // u64 [2][kCand] gathered members
 constexpr uint32_t kRRid = kRAll + 2 * kCand * 8;       // u16 [P] own R clusters (local index)
 constexpr uint32_t kRLgs = kRRid + kMaxIdsPerBlock * 2;  // int [kGroups] own group sums
-static_assert(kRLgs + kGroups * 4 <= kRingBytes, "selection scratch");
+constexpr uint32_t kRTin = kRLgs + kGroups * 4;  // int [2][512] pushed per-tile equal-key counts
+constexpr uint32_t kRTcnt = kRTin + 2 * 512 * 4;  // int4 [512] pushed per-tile list counts
+static_assert(kRTcnt + 512 * 16 <= kRingBytes, "selection scratch");
 static_assert(kCand == 256 && kThreads == 2 * kCand, "ranking maps two boundaries to 2 x 256 threads");
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
@@ -234,12 +241,6 @@ __device__ __forceinline__ uint32_t ld_cl_u32(uint32_t addr) {
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
-__device__ __forceinline__ int2 ld_cl_v2(uint32_t addr) {
-  int2 v;
-  asm volatile("ld.shared::cluster.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr)
-               : "memory");
-  return v;
-}
 __device__ __forceinline__ int4 ld_cl_v4(uint32_t addr) {
   int4 v;
   asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
@@ -306,7 +307,7 @@ __device__ __forceinline__ float ex2f(float x) {
 
 // Block-wide exclusive prefix of one int per thread (thread order); the
 // block total goes to *total.  One warp scans the per-warp totals.
-__device__ __forceinline__ int block_scan(int v, int* scratch /* [kWarps + 1] */, int* total) {
+__device__ __noinline__ int block_scan(int v, int* scratch /* [kWarps + 1] */, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -391,6 +392,125 @@ __device__ __forceinline__ void token_bar() {
   asm volatile("bar.sync 2, 256;" ::: "memory");
 }
 
+// Thresholds of the boundary buckets holding more than kCand keys (heavy
+// ties): an MSD radix walk over the 32-bit order key, one byte per pass with
+// the digit counts reduced into their owner blocks, then the boundary id
+// among the keys equal to the key found (per-block counts in id order).
+// Called by every thread of every block of the cluster (cluster barriers).
+__device__ __noinline__ void crowded_thresholds(const float* keys, int nid, float lo, float scale,
+                                                int bk0, int bk1, bool slow0, bool slow1,
+                                                Misc* ms, uint32_t dig_a, const int* tin,
+                                                uint32_t tin_a, int CS, int b, int ntl,
+                                                int tiles, int* status) {
+  const int tid = threadIdx.x;
+  const int DS = (256 + CS - 1) / CS;
+      RI_STAMP(16, 0);
+      uint32_t prefix[2] = {0u, 0u}, mask[2] = {0u, 0u};
+      int kp[2] = {ms->kp[0], ms->kp[1]};
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < nid; i += kThreads) {
+          const float key = keys[i];
+          const int bk = bucket_of(key, lo, scale);
+          const uint32_t o = float_order_key(key);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) &&
+                (o & mask[w]) == prefix[w]) {
+              const int d = (int)((o >> shift) & 255u);
+              red_cl_add(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
+                              (uint32_t)(d / DS)),
+                         1u);
+            }
+          }
+        }
+        cluster_sync();  // digit counts of this pass complete
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (!(w == 0 ? slow0 : slow1)) continue;
+          const int d = 255 - tid;  // thread order = digits from the top
+          int v = 0;
+          if (tid < 256)
+            v = (int)ld_cl_u32(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
+                                    (uint32_t)(d / DS)));
+          int tot;
+          const int excl = block_scan(v, ms->scan, &tot);
+          if (tid < 256 && excl < kp[w] && excl + v >= kp[w]) {
+            ms->digit[w] = d;
+            ms->above[w] = excl;
+          }
+          __syncthreads();
+          prefix[w] |= (uint32_t)ms->digit[w] << shift;
+          mask[w] |= 255u << shift;
+          kp[w] -= ms->above[w];
+          __syncthreads();
+        }
+      }
+      // members equal to the found key, counted per tile (tiles are in id
+      // order and dealt round-robin to the blocks): every block pushes its
+      // tiles' counts to every block, a scan over the tiles finds the tile
+      // holding the kp-th one, and the block owning that tile names its id
+      if (tid < 64) ms->fine[tid >> 5][tid & 31] = 0;
+      if (tid < 2) ms->owner[tid] = -1;
+      __syncthreads();
+      for (int i = tid; i < nid; i += kThreads) {
+        const float key = keys[i];
+        const int bk = bucket_of(key, lo, scale);
+        const uint32_t o = float_order_key(key);
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+          if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) && o == prefix[w])
+            atomicAdd(&ms->fine[w][i >> 7], 1);
+      }
+      __syncthreads();
+      for (int t = tid; t < CS * ntl * 2; t += kThreads) {
+        const int q = t / (ntl * 2), r = t - q * (ntl * 2);
+        const int w = r / ntl, lt = r - w * ntl;
+        st_cl_u32(mapa(tin_a + 4u * (uint32_t)(w * 512 + b + lt * CS), (uint32_t)q),
+                  (uint32_t)ms->fine[w][lt]);
+      }
+      cluster_sync();  // every tile's count of equal keys pushed
+#pragma unroll 1
+      for (int w = 0; w < 2; ++w) {
+        if (!(w == 0 ? slow0 : slow1)) continue;
+        const int v = tid < tiles ? tin[w * 512 + tid] : 0;
+        int tot;
+        const int excl = block_scan(v, ms->scan, &tot);
+        if (tid < tiles && excl < kp[w] && excl + v >= kp[w]) {
+          ms->owner[w] = tid;
+          ms->candp[w][0] = excl;  // equal keys in earlier tiles
+        }
+        __syncthreads();
+      }
+      if (tid < 2 && (tid == 0 ? slow0 : slow1)) {
+        const int w = tid, tile = ms->owner[w];
+        if (tile >= 0 && tile % CS == b) {
+          const int lt = (tile - b) / CS;
+          const int r = kp[w] - ms->candp[w][0];  // 1-based inside the tile
+          int seen = 0;
+          for (int i = lt * kTileC; i < min(nid, (lt + 1) * kTileC); ++i) {
+            const float key = keys[i];
+            if (bucket_of(key, lo, scale) == (w == 0 ? bk0 : bk1) &&
+                float_order_key(key) == prefix[w] && ++seen == r) {
+              ms->pub_tid[w] = tile * kTileC + (i & (kTileC - 1));
+              break;
+            }
+          }
+        }
+      }
+      cluster_sync();  // the boundary ids named
+      if (tid < 2 && (tid == 0 ? slow0 : slow1)) {
+        const int w = tid;
+        const int tile = ms->owner[w];
+        const int id = tile >= 0 ? (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tid[w]),
+                                                       (uint32_t)(tile % CS)))
+                                 : -1;
+        ms->thr[w] = ord64(prefix[w], id);
+        if (tile < 0 || id < 0) record_status(status, RI_ERR_INVALID_ARG);
+      }
+      __syncthreads();
+    }
+
 // ------------------------------------------------------------------ kernel
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -413,11 +533,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int C = p.C;
   const unsigned long long lim = p.wait_ns;
   const bool selecting = p.mode != kModeAttend && C > 0;
-  // this block's tiles [t0, t1) of the unit's ceil(C / 128) tiles
-  const int t0 = (int)((long long)p.tiles * b / CS), t1 = (int)((long long)p.tiles * (b + 1) / CS);
-  const int id0 = t0 * kTileC;
-  const int nid = selecting ? max(0, min(C, t1 * kTileC) - id0) : 0;
-  const int ntiles = (nid + kTileC - 1) / kTileC;
+  // this block's tiles: b, b + CS, b + 2 CS, ... of the unit's ceil(C / 128)
+  // tiles (interleaved, so that relevant clusters crowded into a few
+  // segments still spread over the blocks); local id i is cluster id_of(i)
+  const int ntiles = (selecting && b < p.tiles) ? (p.tiles - 1 - b) / CS + 1 : 0;
+  const bool has_last = ntiles > 0 && (p.tiles - 1 - b) % CS == 0;
+  const int nid = ntiles * kTileC - (has_last ? p.tiles * kTileC - C : 0);
+  auto id_of = [&](int i) { return (b + (i >> 7) * CS) * kTileC + (i & (kTileC - 1)); };
   const uint32_t sm_base = smem_u32(sm);
 
   if (tid == 0) {
@@ -483,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* stage = sm + st * kTileBytes;
         mbar_arrive_expect_tx(&ms->fullA[st], kTileBytes);
-        const int row = u * C + id0 + it * kTileC;
+        const int row = u * C + (b + it * CS) * kTileC;
         if (!(p.fault == RI_FAULT_SCORE_COPY && it == 0)) {
           tma_load_2d(stage, &tm_cent, 0, row, &ms->fullA[st]);
           tma_load_2d(stage + kTileC * 128, &tm_cent, 64, row, &ms->fullA[st]);
@@ -532,15 +654,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 8) {
       // sizes and first rows of the block's clusters, all loads in flight at
       // once while the tiles arrive
-      const int32_t* cg = p.counts + (size_t)u * C + id0;
-      const int32_t* og = p.offsets + (size_t)u * (C + 1) + id0;
+      const int32_t* cg = p.counts + (size_t)u * C;
+      const int32_t* og = p.offsets + (size_t)u * (C + 1);
       for (int i0 = tid - 256; i0 < nid; i0 += 4 * 256) {
         int cv[4], ov[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int i = i0 + r * 256;
-          cv[r] = i < nid ? __ldg(cg + i) : 0;
-          ov[r] = i < nid ? __ldg(og + i) : 0;
+          cv[r] = i < nid ? __ldg(cg + id_of(i)) : 0;
+          ov[r] = i < nid ? __ldg(og + id_of(i)) : 0;
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r)
@@ -558,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < ntiles; ++it) {
         const int cl = it * kTileC + rr;
         const bool valid = cl < nid;
-        const size_t gc = (size_t)u * C + id0 + cl;
+        const size_t gc = (size_t)u * C + id_of(cl);
         ok = ok && wait_bar(&ms->tdone[it], 0, lim);
         if (epilogue_any(!ok)) {  // the 128 threads leave together
           if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
@@ -626,7 +748,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kA = p.kr, kB = p.kr + p.ke;
   const bool onA = kA > 0, onB = p.ke > 0;
   if (selecting) {
-    const int DS = (256 + CS - 1) / CS;  // radix digits per block (crowded buckets)
     int* hist = reinterpret_cast<int*>(sm + kRHist);
     int* dig = reinterpret_cast<int*>(sm + kRDig);
     int* lgs = reinterpret_cast<int*>(sm + kRLgs);
@@ -754,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               prefetch_l2_bulk(p.Vr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
             }
           } else if (sureE) {
-            prefetch_l2_bulk(p.vsum + ((size_t)u * C + id0 + i) * kHeadDim, 512u);
+            prefetch_l2_bulk(p.vsum + ((size_t)u * C + id_of(i)) * kHeadDim, 512u);
           }
         }
       }
@@ -806,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((w == 0 ? fast0 : fast1) && bk == (w == 0 ? bk0 : bk1)) {
             const int slot = atomicAdd(&ms->own_ncand[w], 1);
             if (slot < kCand)
-              cin[(w * kMaxCS + b) * kCand + slot] = ord64(float_order_key(key), id0 + i);
+              cin[(w * kMaxCS + b) * kCand + slot] = ord64(float_order_key(key), id_of(i));
           }
         }
       }
@@ -870,119 +991,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- crowded bucket: radix walk over the order key, then the id count
-    if (slow0 || slow1) {
-      RI_STAMP(16, 0);
-      uint32_t prefix[2] = {0u, 0u}, mask[2] = {0u, 0u};
-      int kp[2] = {ms->kp[0], ms->kp[1]};
-      for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = tid; i < nid; i += kThreads) {
-          const float key = keys[i];
-          const int bk = bucket_of(key, lo, scale);
-          const uint32_t o = float_order_key(key);
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) &&
-                (o & mask[w]) == prefix[w]) {
-              const int d = (int)((o >> shift) & 255u);
-              red_cl_add(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
-                              (uint32_t)(d / DS)),
-                         1u);
-            }
-          }
-        }
-        cluster_sync();  // digit counts of this pass complete
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (!(w == 0 ? slow0 : slow1)) continue;
-          const int d = 255 - tid;  // thread order = digits from the top
-          int v = 0;
-          if (tid < 256)
-            v = (int)ld_cl_u32(mapa(dig_a + 4u * (uint32_t)((pass * 2 + w) * 256 + d % DS),
-                                    (uint32_t)(d / DS)));
-          int tot;
-          const int excl = block_scan(v, ms->scan, &tot);
-          if (tid < 256 && excl < kp[w] && excl + v >= kp[w]) {
-            ms->digit[w] = d;
-            ms->above[w] = excl;
-          }
-          __syncthreads();
-          prefix[w] |= (uint32_t)ms->digit[w] << shift;
-          mask[w] |= 255u << shift;
-          kp[w] -= ms->above[w];
-          __syncthreads();
-        }
-      }
-      // members equal to the found key, in id order: per-block counts, then
-      // the block holding the kp-th one names its id
-      const int kper = (max(nid, 1) + kThreads - 1) / kThreads;
-      const int i0 = tid * kper, i1 = min(i0 + kper, nid);
-      int eqc[2] = {0, 0};
-      for (int i = i0; i < i1; ++i) {
-        const float key = keys[i];
-        const int bk = bucket_of(key, lo, scale);
-        const uint32_t o = float_order_key(key);
-#pragma unroll
-        for (int w = 0; w < 2; ++w)
-          if ((w == 0 ? slow0 : slow1) && bk == (w == 0 ? bk0 : bk1) && o == prefix[w]) ++eqc[w];
-      }
-      int ex[2], tot[2];
-#pragma unroll
-      for (int w = 0; w < 2; ++w) ex[w] = block_scan(eqc[w], ms->scan, &tot[w]);
-      if (tid == 0) {
-        ms->pub_idcnt[0] = tot[0];
-        ms->pub_idcnt[1] = tot[1];
-      }
-      cluster_sync();  // per-block counts of equal keys published
-      if (warp < 2) {
-        const int w = warp;
-        int n = 0;
-        if (lane < CS) n = (int)ld_cl_u32(mapa(smem_u32(&ms->pub_idcnt[w]), lane));
-        int incl = n;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int t = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += t;
-        }
-        const unsigned hit =
-            __ballot_sync(0xffffffffu, lane < CS && incl - n < kp[w] && incl >= kp[w]);
-        if (lane == 0) ms->owner[w] = hit ? __ffs(hit) - 1 : -1;
-        if (hit && lane == __ffs(hit) - 1) ms->candp[w][0] = incl - n;  // equal keys before it
-      }
-      __syncthreads();
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        if (!(w == 0 ? slow0 : slow1) || ms->owner[w] != b) continue;
-        const int r = kp[w] - ms->candp[w][0];  // 1-based among this block's equal keys
-        if (eqc[w] > 0 && ex[w] < r && ex[w] + eqc[w] >= r) {
-          int seen = ex[w];
-          for (int i = i0; i < i1; ++i) {
-            const float key = keys[i];
-            if (bucket_of(key, lo, scale) == (w == 0 ? bk0 : bk1) &&
-                float_order_key(key) == prefix[w] && ++seen == r) {
-              ms->pub_tid[w] = id0 + i;
-              break;
-            }
-          }
-        }
-      }
-      cluster_sync();  // the boundary ids named
-      if (tid < 2 && (tid == 0 ? slow0 : slow1)) {
-        const int w = tid;
-        const int ob = ms->owner[w];
-        const int id =
-            ob >= 0 ? (int)ld_cl_u32(mapa(smem_u32(&ms->pub_tid[w]), (uint32_t)ob)) : -1;
-        ms->thr[w] = ord64(prefix[w], id);
-        if (ob < 0 || id < 0) record_status(p.status, RI_ERR_INVALID_ARG);
-      }
-      __syncthreads();
-    }
+    if (slow0 || slow1)
+      crowded_thresholds(keys, nid, lo, scale, bk0, bk1, slow0, slow1, ms, dig_a,
+                         reinterpret_cast<const int*>(sm + kRTin), sm_base + kRTin, CS, b,
+                         ntiles, p.tiles, p.status);
     const unsigned long long thrA = onA ? ms->thr[0] : ~0ull, thrB = onB ? ms->thr[1] : ~0ull;
     RI_STAMP(4, 0);
 
-    // ---- classification of the block's ids and the id-ordered lists
+    // ---- classification of the block's ids and the id-ordered lists:
+    // R entries (first row, token prefix in the block) then E entries (id,
+    // size); per own tile the counts (R, E, R tokens) for the outputs
+    const bool need_out = p.mode == kModeSelect || p.sel_user || p.rpre_user;
+    int* tcl = ms->gsum;  // [32 own tiles][3], free after the boundary search
+    for (int i = tid; i < 3 * kMaxTilesPerBlock; i += kThreads) tcl[i] = 0;
+    __syncthreads();
     {
-      const int kper = (max(nid, 1) + kThreads - 1) / kThreads;
+      // thread t takes kper consecutive local ids; kper is a power of two, so
+      // no thread's ids straddle a tile
+      int kper = 1;
+      while (kper * kThreads < nid) kper <<= 1;
       const int i0 = tid * kper, i1 = min(i0 + kper, nid);
       float kk[kKPT];
       int2 mm[kKPT];
@@ -1001,7 +1028,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < kKPT; ++j) {
         const int i = i0 + j;
         if (!(j < kper && i < i1)) continue;
-        const unsigned long long o = ord64(float_order_key(kk[j]), id0 + i);
+        const unsigned long long o = ord64(float_order_key(kk[j]), id_of(i));
         const bool inR = onA && o >= thrA;
         const bool inE = !inR && onB && o >= thrB;
         if (inR || inE) {
@@ -1018,6 +1045,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mE |= (uint32_t)inE << j;
       }
       if (bad) record_status(p.status, RI_ERR_INVALID_ARG);
+      if (need_out && i0 < i1 && (mR | mE)) {
+        const int lt = i0 >> 7;
+        atomicAdd(&tcl[3 * lt], __popc(mR));
+        atomicAdd(&tcl[3 * lt + 1], __popc(mE));
+        atomicAdd(&tcl[3 * lt + 2], tokr);
+      }
       int tot, ttot;
       const int excl = block_scan((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
       int texcl = block_scan(tokr, ms->scan, &ttot);
@@ -1033,7 +1066,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           texcl += mm[j].y;
           ++pr;
         } else if ((mE >> j) & 1u) {
-          lists[pe++] = make_int2(id0 + i0 + j, mm[j].y);
+          lists[pe++] = make_int2(id_of(i0 + j), mm[j].y);
         }
       }
       if (tid == 0) {
@@ -1041,80 +1074,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         ms->own_nE = nE;
         ms->own_tokR = ttot;
       }
-      if (tid < CS)
-        st_cl_v4(mapa(smem_u32(&ms->tot_in[b]), (uint32_t)tid),
-                 make_uint4((uint32_t)nR, (uint32_t)nE, (uint32_t)ttot, 0u));
     }
     RI_STAMP(17, 0);
-    cluster_sync();  // 4: every block's lists published and totals pushed
-    RI_STAMP(5, 0);
-    if (warp == 0) {
-      int a = 0, e = 0, t = 0;
-      if (lane < CS) {
-        const uint4 v = ms->tot_in[lane];
-        a = (int)v.x;
-        e = (int)v.y;
-        t = (int)v.z;
+    if (need_out) {
+      // every own tile's counts pushed to every block, then the prefixes
+      // over all tiles (in id order) place the block's ids
+      __syncthreads();
+      for (int t = tid; t < CS * ntiles; t += kThreads) {
+        const int q = t / ntiles, lt = t - q * ntiles;
+        st_cl_v4(mapa(sm_base + kRTcnt + 16u * (uint32_t)(b + lt * CS), (uint32_t)q),
+                 make_uint4((uint32_t)tcl[3 * lt], (uint32_t)tcl[3 * lt + 1],
+                            (uint32_t)tcl[3 * lt + 2], 0u));
       }
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, a, off);
-        const int y = __shfl_up_sync(0xffffffffu, e, off);
-        const int z = __shfl_up_sync(0xffffffffu, t, off);
-        if (lane >= off) {
-          a += x;
-          e += y;
-          t += z;
-        }
+      cluster_sync();  // 4: every tile's counts pushed
+      RI_STAMP(5, 0);
+      const uint4* tc = reinterpret_cast<const uint4*>(sm + kRTcnt);
+      const uint4 v = tid < p.tiles ? tc[tid] : make_uint4(0u, 0u, 0u, 0u);
+      int totRE, totT;
+      const int exRE = block_scan((int)((v.x << 16) | v.y), ms->scan, &totRE);
+      const int exT = block_scan((int)v.z, ms->scan, &totT);
+      // tile prefixes into the tile-count area (only the own tiles are used)
+      int4* tp = reinterpret_cast<int4*>(sm + kRTcnt);
+      if (tid < p.tiles) tp[tid] = make_int4(exRE >> 16, exRE & 0xFFFF, exT, 0);
+      if (tid == 0) {
+        ms->nRp[0] = totRE >> 16;  // cluster-wide totals
+        ms->nEp[0] = totRE & 0xFFFF;
+        ms->tokRp[0] = totT;
       }
-      if (lane < CS) {
-        ms->nRp[lane + 1] = a;
-        ms->nEp[lane + 1] = e;
-        ms->tokRp[lane + 1] = t;
-      }
-      if (lane == 0) ms->nRp[0] = ms->nEp[0] = ms->tokRp[0] = 0;
-    }
-    __syncthreads();
-    RI_STAMP(18, 0);
-    // selected ids (R then E, each in id order) and the R token prefix
-    {
+      __syncthreads();
       const bool to_ws = p.mode == kModeSelect;
       const int ksel = p.k_r + p.k_e;
       int32_t* selw = to_ws ? p.sel + (size_t)u * ksel : nullptr;
       int32_t* selu = p.sel_user ? p.sel_user + (size_t)u * ksel : nullptr;
       int32_t* rpw = to_ws ? p.rpre + (size_t)u * (p.k_r + 1) : nullptr;
       int32_t* rpu = p.rpre_user ? p.rpre_user + (size_t)u * (p.k_r + 1) : nullptr;
-      if (selw || selu || rpw || rpu) {
-        const uint16_t* rid = reinterpret_cast<const uint16_t*>(sm + kRRid);
-        const int nR = ms->own_nR, nE = ms->own_nE;
-        const int rb = ms->nRp[b], eb = ms->nEp[b], tb = ms->tokRp[b];
-        for (int i = tid; i < nR; i += kThreads) {
-          const int g = rb + i;
-          if (g >= p.k_r) break;
-          if (selw) selw[g] = id0 + rid[i];
-          if (selu) selu[g] = id0 + rid[i];
-          if (rpw) rpw[g] = tb + lists[i].y;
-          if (rpu) rpu[g] = tb + lists[i].y;
+      const uint16_t* rid = reinterpret_cast<const uint16_t*>(sm + kRRid);
+      const int nR = ms->own_nR, nE = ms->own_nE;
+      // local starts of each own tile's R / E entries and R tokens
+      // (tcl becomes the exclusive prefix over own tiles)
+      if (tid == 0) {
+        int a = 0, e = 0, t = 0;
+        for (int lt = 0; lt < ntiles; ++lt) {
+          const int ca = tcl[3 * lt], ce = tcl[3 * lt + 1], ct = tcl[3 * lt + 2];
+          tcl[3 * lt] = a;
+          tcl[3 * lt + 1] = e;
+          tcl[3 * lt + 2] = t;
+          a += ca;
+          e += ce;
+          t += ct;
         }
-        for (int i = tid; i < nE; i += kThreads) {
-          const int e = eb + i;
-          if (e >= p.k_e) break;
-          if (selw) selw[p.k_r + e] = lists[nR + i].x;
-          if (selu) selu[p.k_r + e] = lists[nR + i].x;
+      }
+      __syncthreads();
+      for (int i = tid; i < nR; i += kThreads) {
+        const int lt = rid[i] >> 7;
+        const int4 tpv = tp[b + lt * CS];
+        const int g = tpv.x + i - tcl[3 * lt];
+        if (g >= p.k_r) continue;
+        const int id = id_of(rid[i]);
+        const int rp = tpv.z + lists[i].y - tcl[3 * lt + 2];
+        if (selw) selw[g] = id;
+        if (selu) selu[g] = id;
+        if (rpw) rpw[g] = rp;
+        if (rpu) rpu[g] = rp;
+      }
+      for (int i = tid; i < nE; i += kThreads) {
+        const int id = lists[nR + i].x;
+        const int lt = ((id >> 7) - b) / CS;
+        const int e = tp[id >> 7].y + i - tcl[3 * lt + 1];
+        if (e >= p.k_e) continue;
+        if (selw) selw[p.k_r + e] = id;
+        if (selu) selu[p.k_r + e] = id;
+      }
+      if (b == CS - 1) {
+        const int KRt = ms->nRp[0], KEt = ms->nEp[0];
+        for (int g = KRt + tid; g < p.k_r; g += kThreads) {
+          if (selw) selw[g] = -1;
+          if (selu) selu[g] = -1;
         }
-        if (b == CS - 1) {
-          for (int g = ms->nRp[CS] + tid; g < p.k_r; g += kThreads) {
-            if (selw) selw[g] = -1;
-            if (selu) selu[g] = -1;
-          }
-          for (int e = ms->nEp[CS] + tid; e < p.k_e; e += kThreads) {
-            if (selw) selw[p.k_r + e] = -1;
-            if (selu) selu[p.k_r + e] = -1;
-          }
-          for (int g = min(ms->nRp[CS], p.k_r) + tid; g <= p.k_r; g += kThreads) {
-            if (rpw) rpw[g] = ms->tokRp[CS];
-            if (rpu) rpu[g] = ms->tokRp[CS];
-          }
+        for (int e = KEt + tid; e < p.k_e; e += kThreads) {
+          if (selw) selw[p.k_r + e] = -1;
+          if (selu) selu[p.k_r + e] = -1;
+        }
+        for (int g = min(KRt, p.k_r) + tid; g <= p.k_r; g += kThreads) {
+          if (rpw) rpw[g] = ms->tokRp[0];
+          if (rpu) rpu[g] = ms->tokRp[0];
         }
       }
     }
@@ -1135,93 +1178,111 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.mode == kModeSelect) return;
 
   // ============================================================ step C
-  // the unit's totals: R clusters, R tokens, E clusters
-  int KR, KE, T_R;
+  // The block attends over the clusters it scored (its own R and E lists,
+  // in shared memory) and over an even share of the steady tokens.  After a
+  // separate select, the attend call rebuilds the same lists from the
+  // workspace by the same tile ownership, so the one-call decode and the
+  // split calls fold the same items in the same order.
   const bool exec = p.exec_rows > 0;
-  const int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
-  const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
   const long long lim_rows = exec ? p.exec_rows : p.M;
-  if (selecting) {
-    KR = ms->nRp[CS];
-    KE = ms->nEp[CS];
-    T_R = ms->tokRp[CS];
-  } else if (C > 0) {  // attend: the selection left in the workspace
-    KR = p.kr;
-    KE = p.ke;
-    if (tid == 0) ms->T_R = __ldcg(rpg + KR);
-    __syncthreads();
-    T_R = ms->T_R;
-    if (T_R < 0 || T_R > lim_rows) {
-      if (tid == 0) record_status(p.status, RI_ERR_INVALID_ARG);
-      T_R = 0;
-      KR = 0;
-    }
-  } else {
-    KR = KE = T_R = 0;
-  }
   const int n_st = p.n_steady;
-  const long long T = (long long)n_st + T_R;
-  const long long ta = T * b / CS, tb = T * (b + 1) / CS;
-  const int ea = (int)((long long)KE * b / CS), eb = (int)((long long)KE * (b + 1) / CS);
-  const int ne = min(eb - ea, kMaxIdsPerBlock);
-  // the block's E entries (id, size) into shared memory (the sizes and first
-  // rows of step A are no longer needed there), all loads in flight together:
-  // from the owners' lists in the cluster, or from the workspace after a select
-  int2* eplan = meta;
-  if (selecting) {
-    const uint32_t lists_a = sm_base + kOffKeys;
-    for (int e = tid; e < ne; e += kThreads) {
-      const int ge = ea + e;
-      int ob = 0;
-      while (ob + 1 < CS && ms->nEp[ob + 1] <= ge) ++ob;
-      const int nR_ob = ms->nRp[ob + 1] - ms->nRp[ob];
-      eplan[e] = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(nR_ob + ge - ms->nEp[ob]), (uint32_t)ob));
+  const int st0 = (int)((long long)n_st * b / CS), st1 = (int)((long long)n_st * (b + 1) / CS);
+  if (!selecting && C > 0) {
+    const int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
+    const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
+    const int32_t* off_u = p.offsets + (size_t)u * (C + 1);
+    // R: the workspace's retrieval clusters (id order) of this block's tiles
+    {
+      const int kr = p.kr;
+      const int per = (kr + kThreads - 1) / kThreads;  // <= 8 (kr <= 4096)
+      const int g0 = min(kr, tid * per), g1 = min(kr, g0 + per);
+      int rowv[kKPT], cntv[kKPT];
+      uint32_t mk = 0;
+      int tok = 0;
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < kKPT; ++j) {
+        const int g = g0 + j;
+        rowv[j] = 0;
+        cntv[j] = 0;
+        if (g < g1) {
+          const int id = __ldcg(selg + g);
+          if (id >= 0 && id < C && (id >> 7) % CS == b) {
+            const int r0 = __ldcg(rpg + g), cnt = __ldcg(rpg + g + 1) - r0;
+            const int row = exec ? r0 : __ldg(off_u + id);
+            if (cnt >= 0 && row >= 0 && (long long)row + cnt <= lim_rows) {
+              rowv[j] = row;
+              cntv[j] = cnt;
+            } else {
+              bad = true;
+            }
+            mk |= 1u << j;
+            tok += cntv[j];
+          } else if (id < -1 || id >= C) {
+            bad = true;
+          }
+        }
+      }
+      if (bad) record_status(p.status, RI_ERR_INVALID_ARG);
+      int tot, ttot;
+      const int ex = block_scan(__popc(mk), ms->scan, &tot);
+      int tex = block_scan(tok, ms->scan, &ttot);
+      int pos = ex;
+#pragma unroll
+      for (int j = 0; j < kKPT; ++j)
+        if ((mk >> j) & 1u) {
+          if (pos < kMaxIdsPerBlock) lists[pos] = make_int2(rowv[j], tex);
+          tex += cntv[j];
+          ++pos;
+        }
+      if (tid == 0) {
+        ms->own_nR = min(tot, kMaxIdsPerBlock);
+        ms->own_tokR = ttot;
+      }
     }
-  } else {
-    for (int e = tid; e < ne; e += kThreads) {
-      const int id = __ldcg(selg + p.k_r + ea + e);
-      const int cnt = (id >= 0 && id < C) ? __ldg(p.counts + (size_t)u * C + id) : 0;
-      eplan[e] = make_int2(id, cnt);
+    __syncthreads();
+    // E: the workspace's estimation clusters of this block's tiles, two
+    // passes over each thread's contiguous run (count, then write)
+    {
+      const int nRo = ms->own_nR;
+      const int ke = p.ke;
+      const int per = (ke + kThreads - 1) / kThreads;
+      const int g0 = min(ke, tid * per), g1 = min(ke, g0 + per);
+      int n = 0;
+      for (int g = g0; g < g1; ++g) {
+        const int id = __ldcg(selg + p.k_r + g);
+        n += id >= 0 && id < C && (id >> 7) % CS == b;
+      }
+      int tot;
+      int pos = nRo + block_scan(n, ms->scan, &tot);
+      for (int g = g0; g < g1; ++g) {
+        const int id = __ldcg(selg + p.k_r + g);
+        if (id >= 0 && id < C && (id >> 7) % CS == b) {
+          if (pos < kMaxIdsPerBlock)
+            lists[pos] = make_int2(id, max(0, __ldg(p.counts + (size_t)u * C + id)));
+          ++pos;
+        }
+      }
+      if (tid == 0) ms->own_nE = min(tot, kMaxIdsPerBlock - nRo);
     }
   }
+  // the ring was last written by the TMA (async proxy) and by step B: order
+  // both before the copies of step C
+  fence_proxy_async_smem();
+  __syncthreads();
+  const int nR = ms->own_nR, nE = ms->own_nE, tokR = ms->own_tokR;
+  const int ns = st1 - st0;            // steady tokens of this block
+  const long long ntok = (long long)ns + tokR;
 
-  // R list access for the planner: entry g -> (first row, first token) in the
-  // unit's token order (owners' lists in a cluster, the workspace after a
-  // select); g = KR gives (0, T_R)
-  const uint32_t lists_a = sm_base + kOffKeys;
-  auto r_entry = [&](int g, int& row, int& gs) {
-    if (g >= KR) {
-      row = 0;
-      gs = T_R;
-      return;
-    }
-    if (selecting) {
-      int ob = 0;
-      while (ob + 1 < CS && ms->nRp[ob + 1] <= g) ++ob;
-      const int2 e = ld_cl_v2(mapa(lists_a + 8u * (uint32_t)(g - ms->nRp[ob]), (uint32_t)ob));
-      row = e.x;
-      gs = ms->tokRp[ob] + e.y;
-    } else {
-      gs = __ldcg(rpg + g);
-      const int id = __ldcg(selg + g);
-      row = (id >= 0 && id < C) ? __ldcg(p.offsets + (size_t)u * (C + 1) + id) : -1;
-    }
-  };
-
-  // ---- tensor-core helpers of the token tiles are below the kernel's
-  // selection code; the state of the two kinds of warps:
+  // ---- the state of the two kinds of warps:
   //  token warps (0..7): O^T fragments ot[j][i] (lane holds dims 16 j + gid
   //   (+8), heads 2 tig (+1)), the running maximum tm of head gid (log2
   //   units) and the lane's share tl of head gid's denominator;
-  //  estimation warps (8..15): per head the maximum em, denominator el and
-  //   numerators eo[g][4] of dims 4 lane .. 4 lane + 3.
+  //  estimation warps (8..15): lane (head g, dim group dg) holds its head's
+  //   maximum em, denominator el and numerators of its dims.
   // Each kind of warp writes its partial into wo [kWarps][G][128] (the ring,
   // once every warp is done with it) and wm / wl.
   float* wo = reinterpret_cast<float*>(sm);
-  // the E entries are staged; the ring was last written by the TMA (async
-  // proxy) and by step B: order both before the copies of step C
-  fence_proxy_async_smem();
-  __syncthreads();
   RI_STAMP(19, 0);
   if (warp < kTokenWarps) {
     const int gid = lane >> 2, tig = lane & 3;
@@ -1253,65 +1314,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* rowtab = reinterpret_cast<int*>(sm + kOffRuns);
     // 16-byte chunk c of token row t of a tile, XOR-swizzled for ldmatrix
     auto row_chunk = [](int t, int c) { return (uint32_t)(t * 256 + ((c ^ (t & 7)) << 4)); };
-    long long wt = ta;
-    while (true) {
-      // ---- planner (warp 0): the window's token rows (R rows >= 0, steady
-      // rows as -1 - row, INT_MIN for rows out of range)
-      if (warp == 0) {
-        const long long wend = min(tb, wt + kWindowTokens);
-        long long cur = wt;
-        if (cur < n_st && cur < wend) {
-          const int s1 = (int)min(wend, (long long)n_st);
-          for (int t = (int)cur + lane; t < s1; t += 32) rowtab[t - wt] = -1 - t;
-          cur = s1;
+    const int tt = tid;  // 0 .. 255 over the token warps
+    for (long long wt = 0; wt < ntok; wt += kWindowTokens) {
+      // ---- the window's token rows (R rows >= 0, steady rows as -1 - row),
+      // written by the 256 threads of the token warps from the local lists
+      const int nwt = (int)min((long long)kWindowTokens, ntok - wt);
+      for (int t = tt; t < nwt; t += kTokenWarps * 32) {
+        const long long bt = wt + t;
+        if (bt < ns) rowtab[t] = -1 - (st0 + (int)bt);
+      }
+      {
+        const long long j0 = max(0ll, wt - ns), j1 = wt + nwt - ns;  // R tokens of the window
+        for (int i = tt; i < nR && j0 < j1; i += kTokenWarps * 32) {
+          const int2 e = lists[i];
+          const int cnt = (i + 1 < nR ? lists[i + 1].y : tokR) - e.y;
+          const long long lo = max(j0, (long long)e.y), hi = min(j1, (long long)e.y + cnt);
+          for (long long j = lo; j < hi; ++j) rowtab[(int)(j + ns - wt)] = e.x + (int)(j - e.y);
         }
-        if (cur < wend && exec) {
-          for (long long t = cur + lane; t < wend; t += 32) {
-            const long long j = t - n_st;
-            rowtab[t - wt] = j < lim_rows ? (int)j : INT_MIN;
-          }
-          if (lane == 0 && (long long)(wend - n_st) > lim_rows)
-            record_status(p.status, RI_ERR_INVALID_ARG);
-          cur = wend;
-        } else if (cur < wend) {
-          // first R entry whose tokens reach R token j0 (32-ary search)
-          const int j0 = (int)(cur - n_st), j1 = (int)(wend - n_st);
-          int lo_g = 0, hi_g = KR;
-          while (hi_g - lo_g > 1) {
-            const int step = (hi_g - lo_g + 31) / 32;
-            const int gg = lo_g + lane * step;
-            int row, gs = INT_MAX;
-            if (gg < hi_g) r_entry(gg, row, gs);
-            const unsigned le = __ballot_sync(0xffffffffu, gg < hi_g && gs <= j0);
-            const int L = le ? 31 - __clz(le) : 0;
-            lo_g = lo_g + L * step;
-            hi_g = min(hi_g, lo_g + step);
-            if (step == 1) break;
-          }
-          // batches of 32 entries, one per lane: each lane writes its rows
-          for (int g = lo_g; g < KR; g += 32) {
-            int row, gs, nrow, ngs;
-            r_entry(g + lane, row, gs);
-            r_entry(g + 32, nrow, ngs);
-            const int next = __shfl_down_sync(0xffffffffu, gs, 1);
-            const int cnt = (lane == 31 ? ngs : next) - gs;
-            const int lo_t = max(j0, gs), hi_t = min(j1, gs + cnt);
-            if (g + lane < KR && lo_t < hi_t) {
-              const long long r0 = (long long)row + (lo_t - gs);
-              const bool ok = row >= 0 && r0 + (hi_t - lo_t) <= lim_rows;
-              if (!ok) record_status(p.status, RI_ERR_INVALID_ARG);
-              for (int t = lo_t; t < hi_t; ++t)
-                rowtab[t + n_st - wt] = ok ? (int)(r0 + (t - lo_t)) : INT_MIN;
-            }
-            const int bend = __shfl_sync(0xffffffffu, gs + cnt, 31);
-            if (bend >= j1) break;
-          }
-          cur = wend;
-        }
-        if (lane == 0) ms->wend_lo = (int)(cur - wt);
       }
       token_bar();
-      const int nwt = ms->wend_lo;
+      RI_STAMP(25, 0);
       const int ntile = (nwt + 15) >> 4;
       // ---- tiles warp, warp + kTokenWarps, ...: copies one tile ahead
       auto issue = [&](int tj, int slot) {
@@ -1418,10 +1440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cp_async_wait<0>();
       token_bar();  // the row table is rebuilt for the next window
-      const long long wend = wt + nwt;
-      if (wend >= tb) break;
-      wt = wend;
     }
+    RI_STAMP(23, 0);
     __syncthreads();  // every warp done with step C: the ring is free
     tl += __shfl_xor_sync(0xffffffffu, tl, 1);
     tl += __shfl_xor_sync(0xffffffffu, tl, 2);
@@ -1441,74 +1461,98 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
   } else {
-    float em[G], el[G], eo[G][4];
+    // ---- estimation clusters: the block's E list split over the E warps.
+    // Lane (head g, dim group dg): GP = G rounded up to a power of two, 32 /
+    // GP lanes per head, each with 4 GP consecutive dims, so a lane follows
+    // one head alone (no shuffles).  Each warp streams its clusters' value
+    // sums and scores through its own ring of slots in shared memory with
+    // 16-byte cp.async copies, kEAhead clusters ahead.
+    constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+    constexpr int kDims = 4 * GP;  // dims per lane
+    const int g = lane / (32 / GP), dg = lane % (32 / GP);
+    const bool live = g < G;
+    float em = -INFINITY, el = 0.f, eo[kDims];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      em[g] = -INFINITY;
-      el[g] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) eo[g][i] = 0.f;
-    }
-    // ---- estimation clusters [ea', eb') of this warp, in batches: value-sum
-    // rows (lane: dims 4 lane .. 4 lane + 3) and scores straight from L2
-    constexpr int kEB = G <= 4 ? 8 : 4;  // clusters per batch
+    for (int i = 0; i < kDims; ++i) eo[i] = 0.f;
     const int ew = warp - kTokenWarps;
-    const int e0 = ne * ew / kEWarps, e1 = ne * (ew + 1) / kEWarps;
-    for (int eb0 = e0; eb0 < e1; eb0 += kEB) {
-      float4 vv[kEB];
-      float sc[kEB][Gp];
-      float nf[kEB];
-#pragma unroll
-      for (int k = 0; k < kEB; ++k) {
-        const int e = eb0 + k;
-        const int2 ev = e < e1 ? eplan[e] : make_int2(-1, 0);
-        const bool ok = ev.x >= 0 && ev.x < C && ev.y > 0;
-        nf[k] = ok ? (float)ev.y : 0.f;
-        const size_t uc = (size_t)u * C + (ok ? ev.x : 0);
-        vv[k] = ok ? __ldg(reinterpret_cast<const float4*>(p.vsum + uc * kHeadDim) + lane)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int g4 = 0; g4 < Gp / 4; ++g4) {
-          const float4 s4 = ok ? __ldcg(reinterpret_cast<const float4*>(p.score + uc * Gp) + g4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          sc[k][4 * g4] = s4.x;
-          sc[k][4 * g4 + 1] = s4.y;
-          sc[k][4 * g4 + 2] = s4.z;
-          sc[k][4 * g4 + 3] = s4.w;
+    const int e0 = nE * ew / kEWarps, e1 = nE * (ew + 1) / kEWarps;
+    const int2* elist = lists + nR;
+    uint8_t* ering = sm + kOffMeta + ew * kEWarpBytes;
+    auto issue = [&](int e) {
+      if (e < e1) {
+        const int2 ev = elist[e];
+        if (ev.y > 0) {
+          uint8_t* slot = ering + (uint32_t)(e % kESlots) * kSlotE;
+          const size_t uc = (size_t)u * C + ev.x;
+          cp_async16(slot + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
+          if (lane < Gp / 4) cp_async16(slot + 512 + lane * 16, p.score + uc * Gp + lane * 4);
         }
       }
+      cp_async_commit();
+    };
+    for (int k = 0; k < kESlots - 1; ++k) issue(e0 + k);
+#ifdef RI_DEBUG_PHASES
+    long long cyc_w = 0, cyc_c = 0, cyc_t = clock64();
+#endif
+    for (int e = e0; e < e1; ++e) {
+      issue(e + kESlots - 1);
+      cp_async_wait<kESlots - 1>();
+      __syncwarp();
+#ifdef RI_DEBUG_PHASES
+      {
+        const long long n_ = clock64();
+        cyc_w += n_ - cyc_t;
+        cyc_t = n_;
+      }
+#endif
+      const int2 ev = elist[e];
+      if (ev.y > 0 && live) {
+        const uint8_t* slot = ering + (uint32_t)(e % kESlots) * kSlotE;
+        const float x = reinterpret_cast<const float*>(slot + 512)[g] * kLog2e;
+        if (x > em + kRescale2) {  // new reference (also the first cluster)
+          const float c = em == -INFINITY ? 0.f : ex2f(em - x);
+          el *= c;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float bm = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < kEB; ++k)
-          if (nf[k] > 0.f) bm = fmaxf(bm, sc[k][g] * kLog2e);
-        if (bm > em[g] + kRescale2) {  // new reference
-          const float c = em[g] == -INFINITY ? 0.f : ex2f(em[g] - bm);
-          el[g] *= c;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) eo[g][i] *= c;
-          em[g] = bm;
+          for (int i = 0; i < kDims; ++i) eo[i] *= c;
+          em = x;
         }
+        const float w = ex2f(x - em);
+        el = fmaf((float)ev.y, w, el);
+        const float4* vr = reinterpret_cast<const float4*>(slot) + dg * GP;
 #pragma unroll
-        for (int k = 0; k < kEB; ++k) {
-          const float w = nf[k] > 0.f ? ex2f(sc[k][g] * kLog2e - em[g]) : 0.f;
-          el[g] = fmaf(nf[k], w, el[g]);
-          eo[g][0] = fmaf(w, vv[k].x, eo[g][0]);
-          eo[g][1] = fmaf(w, vv[k].y, eo[g][1]);
-          eo[g][2] = fmaf(w, vv[k].z, eo[g][2]);
-          eo[g][3] = fmaf(w, vv[k].w, eo[g][3]);
+        for (int i = 0; i < GP; ++i) {
+          const float4 v = vr[i];
+          eo[4 * i] = fmaf(w, v.x, eo[4 * i]);
+          eo[4 * i + 1] = fmaf(w, v.y, eo[4 * i + 1]);
+          eo[4 * i + 2] = fmaf(w, v.z, eo[4 * i + 2]);
+          eo[4 * i + 3] = fmaf(w, v.w, eo[4 * i + 3]);
         }
       }
+      __syncwarp();
+#ifdef RI_DEBUG_PHASES
+      {
+        const long long n_ = clock64();
+        cyc_c += n_ - cyc_t;
+        cyc_t = n_;
+      }
+#endif
     }
+#ifdef RI_DEBUG_PHASES
+    RI_STAMP_VAL(40, kTokenWarps * 32, cyc_w);
+    RI_STAMP_VAL(41, kTokenWarps * 32, cyc_c);
+    RI_STAMP_VAL(42, kTokenWarps * 32, e1 - e0);
+#endif
+    cp_async_wait<0>();
+    RI_STAMP(24, kTokenWarps * 32);
     __syncthreads();  // every warp done with step C: the ring is free
+    if (live) {
+      float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + dg * kDims);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      *reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + lane * 4) =
-          make_float4(eo[g][0], eo[g][1], eo[g][2], eo[g][3]);
-      if (lane == 0) {
-        ms->wm[warp][g] = em[g];
-        ms->wl[warp][g] = el[g];
+      for (int i = 0; i < GP; ++i)
+        dst[i] = make_float4(eo[4 * i], eo[4 * i + 1], eo[4 * i + 2], eo[4 * i + 3]);
+      if (dg == 0) {
+        ms->wm[warp][g] = em;
+        ms->wl[warp][g] = el;
       }
     }
   }

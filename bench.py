@@ -6,7 +6,13 @@ geometry (batch 1, 32 query heads, 8 KV heads, head_dim 128, sixteen 8K
 segments of 512 clusters; retrieval 147 and estimation 1884 clusters per KV
 head), with HBM GB/s of the dominant kernel against the measured copy
 bandwidth, and the segmented k-means build (8 KV heads x 128K tokens, 10
-iterations) in key vectors clustered per second.
+iterations) in key vectors clustered per second.  At one GPU the line also
+carries the other workloads, each with its own clock record:
+  config1   one KV head, 8K context: single-step latency;
+  config4   Qwen2.5-7B geometry, batch 16 x 128K, 32 drifting steps;
+  config5   Llama3-8B-1048K geometry, 1M context, K/V in pinned host memory
+            behind a 5 % LRU block cache, 64 steps, synchronous and
+            asynchronous cache update.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -41,6 +47,7 @@ UNIT = "steps/s"
 B, H, G, N = 1, 8, 4, 131072
 LAYERS = 32
 WORKLOAD = "llama3.1-8b decode, 128K context, batch 1, 32 q / 8 kv heads, d 128"
+MIN_TIMED_MS = 200.0  # the K-step timed region is repeated until this much device time
 
 
 def _peaks():
@@ -110,17 +117,18 @@ def _dist():
     return ws, rank, local
 
 
-def _traffic_from_profiles(kernel_src: str):
-    """DRAM bytes per launch recorded by an ncu capture of the current kernel
-    source (null when the kernel changed since)."""
+def _traffic_from_profiles(kernel_src: str, kernel: str):
+    """DRAM bytes per launch recorded by an ncu capture of `kernel` from the
+    current kernel source (null when the source changed since)."""
     sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    pat = re.compile(r"traffic_bytes_per_launch:\s*(\d+)\s+source_sha256_16:\s*([0-9a-f]{16})")
     for fn in sorted(os.listdir(os.path.join(ROOT, "profiles"))):
-        if not fn.endswith(".md"):
+        if not (fn.startswith(kernel) and fn.endswith(".md")):
             continue
         text = open(os.path.join(ROOT, "profiles", fn), encoding="utf-8").read()
-        m = re.search(r"traffic_bytes_per_launch:\s*(\d+)\s+source_sha256_16:\s*([0-9a-f]{16})", text)
-        if m and m.group(2) == sha:
-            return int(m.group(1)), sha
+        for m in pat.finditer(text):
+            if m.group(2) == sha:
+                return int(m.group(1)), sha
     return None, sha
 
 
@@ -130,6 +138,60 @@ def _segment_sizes(geom, seg_len=8192, clusters=512):
     M = geom.middle
     return [(min(seg_len, M - s * seg_len), min(clusters, M - s * seg_len))
             for s in range(geom.num_segments)]
+
+
+def headline_config(ws_n, C, k_r, k_e):
+    """The headline workload's config keys, printed alike by both arms."""
+    return {"workload": WORKLOAD, "global_batch": B * ws_n, "seq_len": N, "kv_heads": H,
+            "q_heads": H * G, "head_dim": 128, "clusters_per_head": C, "k_retrieval": k_r,
+            "k_estimation": k_e, "parallelism": f"replicas x{ws_n}"}
+
+
+def step_bytes(counts, sel, rr, C, k_r, k_e, steady, G_):
+    """Algorithmic bytes of one decode step, from its realised selection:
+    what any implementation must move (centroids and sizes of every cluster,
+    steady and retrieval K/V rows, value sums of live estimation clusters,
+    offsets of R, the selected ids, q in, out and lse out), summed over the
+    (sequence, KV head) units.  counts int [U][C]; sel int [U][k_r + k_e];
+    rr int [U][k_r + 1] (retrieval-row prefix)."""
+    total = 0
+    for u in range(counts.shape[0]):
+        T_R = int(rr[u, -1])
+        E = sel[u, k_r:k_r + k_e]
+        E = E[E >= 0]
+        live_E = int((counts[u, E] > 0).sum())
+        total += C * 128 * 2 + C * 4 + (steady + T_R) * 128 * 2 * 2 + live_E * 128 * 4 + \
+            (k_r + k_e) * 4 + k_r * 4 + G_ * 128 * 2 * 2 + G_ * 4
+    return total
+
+
+def timed_region(fn, ws_n, stream, min_ms=MIN_TIMED_MS, max_reps=200):
+    """Device time of fn() (one K-step region), bracketed by a barrier and a
+    synchronize on both sides and timed with CUDA events on `stream`;
+    repeated until min_ms of device time (at most max_reps times).  Returns
+    (median ms, every sample)."""
+    samples = []
+    while True:
+        if ws_n > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if ws_n > 1:
+            torch.distributed.barrier()
+        samples.append(e0.elapsed_time(e1))
+        # every rank takes the same number of repetitions (decided on rank 0's clock)
+        stop = sum(samples) >= min_ms or len(samples) >= max_reps
+        if ws_n > 1:
+            t = torch.tensor([1 if stop else 0], device=torch.cuda.current_device())
+            torch.distributed.broadcast(t, 0)
+            stop = bool(t.item())
+        if stop:
+            return statistics.median(samples), samples
 
 
 # --------------------------------------------------------------------- ours
@@ -158,7 +220,7 @@ def run_ours(args, ws_n, rank, local):
     assert R.read_device_status(base._build_ws) == 0
     build_ws = base._build_ws
     kms = []
-    for _ in range(3):
+    for _ in range(5):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         R.build_index(Kd, Vd, cfg, init_pos=ipd, out=base, workspace=build_ws)
@@ -177,23 +239,20 @@ def run_ours(args, ws_n, rank, local):
     layers = [clone_index(base) for _ in range(LAYERS)]
     del Kd, Vd
     qs = [S.make_queries(kv, G, seed=1000 * rank + 10 + i).to(dev) for i in range(LAYERS)]
-    wsb = R.decode_workspace_bytes(cfg, dcfg)
-    wss = [R.alloc_workspace(wsb, dev) for _ in range(LAYERS)]
-    outs = [torch.empty((B, H * G, 128), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
-    lses = [torch.empty((B, H * G), dtype=torch.float32, device=dev) for _ in range(LAYERS)]
+    decs = [R.Decoder(layers[i], dcfg) for i in range(LAYERS)]
     sels = [torch.empty((B, H, dcfg.k_retrieval + dcfg.k_estimation), dtype=torch.int32,
                         device=dev) for _ in range(LAYERS)]
     rrows = [torch.empty((B, H, dcfg.k_retrieval + 1), dtype=torch.int32, device=dev)
              for _ in range(LAYERS)]
 
     def step(i):
-        R.decode(qs[i], layers[i], dcfg, workspace=wss[i], out=outs[i], lse=lses[i])
+        decs[i](qs[i])
 
     def sel_call(i):
-        R.select_clusters(qs[i], layers[i], dcfg, wss[i], sel=sels[i], retr_rows=rrows[i])
+        R.select_clusters(qs[i], layers[i], dcfg, decs[i].ws, sel=sels[i], retr_rows=rrows[i])
 
     def att_call(i):
-        R.attend_selected(qs[i], layers[i], dcfg, wss[i], out=outs[i], lse=lses[i])
+        R.attend_selected(qs[i], layers[i], dcfg, decs[i].ws, out=decs[i].out, lse=decs[i].lse)
 
     for i in range(max(args.warmup, 3)):
         step(i % LAYERS)
@@ -201,35 +260,26 @@ def run_ours(args, ws_n, rank, local):
         sel_call(i)
     torch.cuda.synchronize()
     for i in range(LAYERS):
-        assert R.read_device_status(wss[i]) == 0
+        assert R.read_device_status(decs[i].ws) == 0
 
     # ---- algorithmic bytes of each step, from the realised selections
-    counts = base.counts.cpu().numpy().astype(np.int64)
+    counts = base.counts.cpu().numpy().astype(np.int64).reshape(B * H, -1)
     C, k_r, k_e = geom.clusters, dcfg.k_retrieval, dcfg.k_estimation
-    # step: what any implementation must move (centroids, sizes, steady and
-    # retrieval K/V rows, value sums of live estimation clusters, offsets of
-    # R, selected ids, q in, out and lse out); per call: the call's own
-    # interface traffic, including the scores the select call hands over.
-    bytes_sel, bytes_att, step_bytes = [], [], []
+    step_b, bytes_sel, bytes_att = [], [], []
     for i in range(LAYERS):
-        sel = sels[i].cpu().numpy()
-        rr = rrows[i].cpu().numpy()
-        b_sel = b_att = b_step = 0
-        for h in range(H):
-            T_R = int(rr[0, h, -1])
-            E = sel[0, h, k_r:k_r + k_e]
-            E = E[E >= 0]
-            live_E = int((counts[0, h, E] > 0).sum())
-            kv_rows = (geom.steady + T_R) * 128 * 2 * 2
-            b_step += C * 128 * 2 + C * 4 + kv_rows + live_E * 128 * 4 + (k_r + k_e) * 4 + \
-                k_r * 4 + G * 128 * 2 * 2 + G * 4
-            b_sel += C * 128 * 2 + C * 4 + G * 128 * 2 + (G + 1) * C * 4 + \
-                (k_r + k_e) * 4 + (k_r + 1) * 4
-            b_att += kv_rows + live_E * 128 * 4 + (k_r + k_e) * 4 + (k_r + 1) * 4 + k_r * 4 + \
-                k_e * 4 + G * k_e * 4 + G * 128 * 2 * 2 + G * 4
-        bytes_sel.append(b_sel)
-        bytes_att.append(b_att)
-        step_bytes.append(b_step)
+        sel = sels[i].cpu().numpy().reshape(B * H, -1)
+        rr = rrows[i].cpu().numpy().reshape(B * H, -1)
+        step_b.append(step_bytes(counts, sel, rr, C, k_r, k_e, geom.steady, G))
+        # per split call: its own interface traffic, including the scores the
+        # select call hands over
+        kv_b = sum((geom.steady + int(rr[u, -1])) * 128 * 2 * 2 for u in range(B * H))
+        live = sum(int((counts[u, sel[u, k_r:][sel[u, k_r:] >= 0]] > 0).sum())
+                   for u in range(B * H))
+        bytes_sel.append(B * H * (C * 128 * 2 + C * 4 + G * 128 * 2 + (G + 1) * C * 4 +
+                                  (k_r + k_e) * 4 + (k_r + 1) * 4))
+        bytes_att.append(kv_b + live * 128 * 4 + B * H * ((k_r + k_e) * 4 + (k_r + 1) * 4 +
+                                                          k_r * 4 + k_e * 4 + G * k_e * 4 +
+                                                          G * 128 * 2 * 2 + G * 4))
 
     # ---- CUDA graphs: the timed loop replays captured decode calls
     stream = torch.cuda.Stream(dev)
@@ -251,20 +301,6 @@ def run_ours(args, ws_n, rank, local):
         g_full.replay()
     torch.cuda.synchronize()
 
-    def timed(fn):
-        if ws_n > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        if ws_n > 1:
-            torch.distributed.barrier()
-        return e0.elapsed_time(e1)
-
     def main_loop():
         for _ in range(K // LAYERS):
             g_full.replay()
@@ -273,12 +309,11 @@ def run_ours(args, ws_n, rank, local):
 
     clocks = ClockSampler(local)
     clocks.start()
-    ms = timed(main_loop)
+    ms, ms_samples = timed_region(main_loop, ws_n, stream)
     clk = clocks.stop()
-    # per-call timings for the roofline (same graphs, rotating layers)
-    reps = max(1, min(200, (K + LAYERS - 1) // LAYERS))
-    ms_sel = timed(lambda: [g_sel.replay() for _ in range(reps)]) / (reps * LAYERS)
-    ms_att = timed(lambda: [g_att.replay() for _ in range(reps)]) / (reps * LAYERS)
+    # per-call timings for the split calls (same graphs, rotating layers)
+    ms_sel = timed_region(lambda: g_sel.replay(), ws_n, stream, min_ms=50)[0] / LAYERS
+    ms_att = timed_region(lambda: g_att.replay(), ws_n, stream, min_ms=50)[0] / LAYERS
 
     ms, ms_sel, ms_att, build_ms = max_over_ranks([ms, ms_sel, ms_att, build_ms], dev)
 
@@ -286,54 +321,54 @@ def run_ours(args, ws_n, rank, local):
     q_host = [qs[i].cpu().pin_memory() for i in range(LAYERS)]
     o_host = torch.empty((B, H * G, 128), dtype=torch.bfloat16).pin_memory()
     q_dev = torch.empty_like(qs[0])
-    k_e2e = min(K, 2000)
+    k_e2e = min(max(K, 1000), 4000)
+    cur = torch.cuda.current_stream(dev)
 
     def e2e_loop():
         for i in range(k_e2e):
             j = i % LAYERS
             q_dev.copy_(q_host[j], non_blocking=True)
-            R.decode(q_dev, layers[j], dcfg, workspace=wss[j], out=outs[j], lse=lses[j])
-            o_host.copy_(outs[j], non_blocking=True)
-            torch.cuda.current_stream().synchronize()
+            out, _ = decs[j](q_dev, cur)
+            o_host.copy_(out, non_blocking=True)
+            cur.synchronize()
 
     for i in range(3):
         q_dev.copy_(q_host[i], non_blocking=True)
-        R.decode(q_dev, layers[i], dcfg, workspace=wss[i], out=outs[i], lse=lses[i])
-        o_host.copy_(outs[i], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-    ms_e2e = max_over_ranks([timed(e2e_loop)], dev)[0]
+        decs[i](q_dev, cur)
+        o_host.copy_(decs[i].out, non_blocking=True)
+        cur.synchronize()
+    ms_e2e = max_over_ranks([timed_region(e2e_loop, ws_n, cur, min_ms=0)[0]], dev)[0]
 
     ms_per_step = ms / K
     value = K * ws_n / (ms / 1e3)
-    mean_bytes = float(np.mean(step_bytes))
+    mean_bytes = float(np.mean(step_b))
     gbs_sel = float(np.mean(bytes_sel)) / (ms_sel * 1e-3) / 1e9
     gbs_att = float(np.mean(bytes_att)) / (ms_att * 1e-3) / 1e9
-    # one decode_kernel launch (cooperative, S1-S6) plus a small memset node
-    # (status word and counters) per decode step: the step time is an upper
-    # bound on the kernel's duration
-    dominant = ("decode_kernel (S1-S6, one cooperative launch per step)",
-                mean_bytes / (ms_per_step * 1e-3) / 1e9, ms_per_step, mean_bytes)
+    # one decode_kernel launch (S1-S6) per decode step and nothing else: the
+    # step time is the kernel's duration plus the gap between graph nodes
+    achieved = mean_bytes / (ms_per_step * 1e-3) / 1e9
     traffic, sha = _traffic_from_profiles(os.path.join(ROOT, "kv_cache_vector_segmented_b200",
-                                                       "csrc", "decode.cu"))
+                                                       "csrc", "decode.cu"), "decode_kernel")
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 data, fp32 math",
         "data": "synthetic (seeded mixture-of-Gaussians keys, Gaussian values; the pages' "
                 "RULER/LongBench/NIAH workloads are not in this container)",
-        "config": {"workload": WORKLOAD, "global_batch": B * ws_n, "seq_len": N,
-                   "kv_heads": H, "q_heads": H * G, "head_dim": 128, "clusters_per_head": C,
-                   "k_retrieval": k_r, "k_estimation": k_e, "parallelism": f"replicas x{ws_n}",
-                   "l2": f"rotating {LAYERS} layer instances, {LAYERS * mean_bytes / 1e6:.0f} MB "
+        "config": headline_config(ws_n, C, k_r, k_e),
+        "timing": {"l2": f"rotating {LAYERS} layer instances, {LAYERS * mean_bytes / 1e6:.0f} MB "
                          "touched per cycle (> 126 MB L2)",
-                   "timing": "CUDA graphs of decode calls, CUDA events on the launch stream"},
+                   "method": "CUDA graphs of decode calls, CUDA events on the launch stream; "
+                             f"the {K}-step region timed {len(ms_samples)} times, median",
+                   "region_ms_samples": [round(x, 4) for x in ms_samples[:50]]},
         "step_bytes": mean_bytes,
-        "step_gbs": mean_bytes / (ms_per_step * 1e-3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": dominant[0], "achieved": dominant[1],
-                     "peak": hbm_peak, "unit": "GB/s", "frac": dominant[1] / hbm_peak,
-                     "peak_kind": peak_kind, "bytes_per_launch": dominant[3],
-                     "us_per_launch": dominant[2] * 1e3, "traffic": traffic,
-                     "frac_of_8tbs": dominant[1] / 8000.0},
+        "step_gbs": achieved,
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel (S1-S6, one launch per step: "
+                                               "a thread-block cluster per (sequence, KV head))",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "bytes_per_launch": mean_bytes, "us_per_launch": ms_per_step * 1e3,
+                     "traffic": traffic, "frac_of_8tbs": achieved / 8000.0},
         "split_calls": {"select_us": ms_sel * 1e3, "select_gbs": gbs_sel,
                         "attend_us": ms_att * 1e3, "attend_gbs": gbs_att},
         "kmeans": {"tok_per_s": H * M / (build_ms * 1e-3), "ms_per_build": build_ms,
@@ -343,13 +378,279 @@ def run_ours(args, ws_n, rank, local):
         "clocks": clk,
         "e2e": {"value": k_e2e * ws_n / (ms_e2e / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": B * H * G * 128 * 2,
-                "d2h_bytes_per_step": B * H * G * 128 * 2, "steps": k_e2e},
+                "d2h_bytes_per_step": B * H * G * 128 * 2, "steps": k_e2e,
+                "call": "Decoder (ri_decode_attention with marshalled arguments), pinned q "
+                        "H2D, out D2H, stream sync per step"},
         "gpu_launches": K,
     }
+    del g_full, g_rem, g_sel, g_att, layers, decs
+    torch.cuda.empty_cache()
+    if rank == 0 and ws_n == 1 and not args.headline_only:
+        res["config1"] = run_config1(dev, hbm_peak, local)
+        torch.cuda.empty_cache()
+        res["config4"] = run_config4(dev, hbm_peak, local)
+        torch.cuda.empty_cache()
+        res["config5"] = run_config5(dev, local)
+        torch.cuda.empty_cache()
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(kv, budget_s=20.0)
-    del g_full, g_rem, g_sel, g_att
     return res
+
+
+# ------------------------------------------------------------ other workloads
+def _build_for(R, dev, Bc, Hc, Gc, Nc, seed, host_gen=False):
+    """A k-means index (10 iterations, seeded initial positions) of a seeded
+    workload; returns (index, kv) with kv drawn on the host (small cases) or
+    on the device."""
+    cfg = R.IndexConfig.make(Bc, Hc, Gc, Nc, iters=10)
+    geom = R.geometry(cfg)
+    segs = _segment_sizes(geom)
+    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], Bc, Hc, seed=seed + 3)
+    if host_gen:
+        kv = S.make_kv(Bc, Hc, Nc, seed=seed)
+        Kd, Vd = kv.K.to(dev), kv.V.to(dev)
+    else:
+        kv = S.make_kv_device(Bc, Hc, Nc, dev, seed=seed)
+        Kd, Vd = kv.K, kv.V
+    idx = R.build_index(Kd, Vd, cfg, init_pos=torch.from_numpy(ip).to(dev))
+    torch.cuda.synchronize()
+    assert R.read_device_status(idx._build_ws) == 0
+    idx._build_ws = None
+    if not host_gen:
+        kv.K = kv.V = None
+    return idx, kv
+
+
+def run_config1(dev, hbm_peak, local):
+    """One KV head (GQA 4), 8K context, one 8K segment of 512 clusters: the
+    latency of one decode step.  512 index instances rotate so the cycle
+    touches more than L2 holds."""
+    import kv_cache_vector_segmented_b200 as R
+    n_inst, G1 = 512, 4
+    idx, kv = _build_for(R, dev, 1, 1, G1, 8192, seed=0, host_gen=True)
+    geom = idx.geom
+    d = R.default_budgets(geom.clusters)
+    f = {k: getattr(idx, k) for k in ("Kp", "Vp", "perm", "centroid", "counts", "offsets",
+                                       "vsum", "Ks", "Vs")}
+    insts = [R.Index(cfg=idx.cfg, geom=geom, **{k: v.clone() for k, v in f.items()})
+             for _ in range(n_inst)]
+    q = S.make_queries(kv, G1, seed=1).to(dev)
+    decs = [R.Decoder(x, d) for x in insts]
+    sel, rr = R.select_clusters(q, insts[0], d, decs[0].ws)
+    counts = idx.counts.cpu().numpy().reshape(1, -1)
+    sb = step_bytes(counts, sel.cpu().numpy().reshape(1, -1), rr.cpu().numpy().reshape(1, -1),
+                    geom.clusters, d.k_retrieval, d.k_estimation, geom.steady, G1)
+    stream = torch.cuda.Stream(dev)
+    for x in decs[:3]:
+        x(q)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for x in decs:
+            x(q, stream)
+    g.replay()
+    torch.cuda.synchronize()
+    assert all(R.read_device_status(x.ws) == 0 for x in decs[:4])
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, samples = timed_region(lambda: g.replay(), 1, stream, min_ms=100)
+    clk = clocks.stop()
+    us = ms * 1e3 / n_inst
+    del g
+    return {"workload": "1 kv head (GQA 4), 8K context, one segment of 512 clusters, "
+                        f"k_r {d.k_retrieval}, k_e {d.k_estimation}",
+            "us_per_step": us, "steps_per_s": 1e6 / us, "bytes_per_step": sb,
+            "gbs": sb / (us * 1e-6) / 1e9, "frac_of_hbm": sb / (us * 1e-6) / 1e9 / hbm_peak,
+            "timing": f"CUDA graph of {n_inst} decode calls on {n_inst} index instances "
+                      f"({n_inst * sb / 1e6:.0f} MB per cycle), median of {len(samples)}",
+            "clocks": clk}
+
+
+def run_config4(dev, hbm_peak, local):
+    """Qwen2.5-7B geometry, batched decode: batch 16 x 4 KV heads x GQA 7,
+    128K context, 32 consecutive steps with queries drifting N(0, 0.05^2)."""
+    import kv_cache_vector_segmented_b200 as R
+    B4, H4, G4, N4, steps = 16, 4, 7, 131072, 32
+    idx, kv = _build_for(R, dev, B4, H4, G4, N4, seed=41)
+    geom = idx.geom
+    d = R.default_budgets(geom.clusters)
+    qs = S.drift_queries_device(S.make_queries_device(kv, G4, seed=42), steps, seed=43)
+    dec = R.Decoder(idx, d)
+    counts = idx.counts.cpu().numpy().reshape(B4 * H4, -1)
+    sb = []
+    for q in qs:
+        sel, rr = R.select_clusters(q, idx, d, dec.ws)
+        sb.append(step_bytes(counts, sel.cpu().numpy().reshape(B4 * H4, -1),
+                             rr.cpu().numpy().reshape(B4 * H4, -1), geom.clusters,
+                             d.k_retrieval, d.k_estimation, geom.steady, G4))
+    mean_b = float(np.mean(sb))
+    stream = torch.cuda.Stream(dev)
+    for q in qs[:3]:
+        dec(q)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for q in qs:
+            dec(q, stream)
+    g.replay()
+    torch.cuda.synchronize()
+    assert R.read_device_status(dec.ws) == 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, samples = timed_region(lambda: g.replay(), 1, stream, min_ms=200)
+    clk = clocks.stop()
+    us = ms * 1e3 / steps
+    del g
+    return {"workload": "qwen2.5-7b batched decode, batch 16 x 128K, 28 q / 4 kv heads, "
+                        f"{geom.clusters} clusters per head, k_r {d.k_retrieval}, "
+                        f"k_e {d.k_estimation}, 32 drifting steps",
+            "us_per_step": us, "steps_per_s": 1e6 / us, "tokens_per_s": B4 * 1e6 / us,
+            "bytes_per_step": mean_b, "gbs": mean_b / (us * 1e-6) / 1e9,
+            "frac_of_hbm": mean_b / (us * 1e-6) / 1e9 / hbm_peak,
+            "timing": f"CUDA graph of the 32 steps (one decode_kernel launch each; "
+                      f"{mean_b / 1e6:.0f} MB per step > L2), median of {len(samples)}",
+            "data": "synthetic, drawn on the device (same recipe as the host generator)",
+            "clocks": clk}
+
+
+def _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode):
+    """One pass of the 1M-token host-memory workload with a fresh cache:
+    `mode` "sync" (ri_cache_plan between select and gather) or "async" (cache
+    worker: lookup on the critical path, LRU update and admit copies on a
+    host thread and a side stream)."""
+    units, k_r, br = counts.shape[0], d.k_retrieval, 8
+    blocks = (counts.astype(np.int64) + br - 1) // br
+    cap = max(1, int(0.05 * blocks.sum(axis=1).max()))
+    cache = R.BlockCache(units, cap, br)
+    shp = (idx.cfg.batch, idx.cfg.num_kv_heads)
+    cK = torch.zeros((*shp, cache.pool_rows, 128), dtype=torch.bfloat16, device=dev)
+    cV = torch.zeros_like(cK)
+    exec_rows = int(R.max_retrieval_rows(counts, k_r).max())
+    eK = torch.empty((*shp, exec_rows, 128), dtype=torch.bfloat16, device=dev)
+    eV = torch.empty_like(eK)
+    ws = R.alloc_workspace(R.decode_workspace_bytes(idx.cfg, d), dev)
+    gws = R.alloc_workspace(256, dev)
+    out = torch.empty((idx.cfg.batch, idx.cfg.num_kv_heads * idx.cfg.group_size, 128),
+                      dtype=torch.bfloat16, device=dev)
+    sel_host = torch.empty((units, k_r), dtype=torch.int32).pin_memory()
+    sel_np = sel_host.numpy()
+    stream = torch.cuda.current_stream(dev)
+    worker = None
+    if mode == "async":
+        wgws = R.alloc_workspace(256, dev)
+        worker = R.CacheWorker(cache, host_K=hK, host_V=hV, cache_K=cK, cache_V=cV, exec_K=eK,
+                               exec_V=eV, gather_workspace=wgws)
+    else:  # pinned staging of the two copy lists, so their H2D copies do not block
+        cap_l = units * exec_rows
+        stage = torch.empty((2, cap_l, 6), dtype=torch.int32).pin_memory()
+        stage_d = torch.empty((2, cap_l, 6), dtype=torch.int32, device=dev)
+    t_cache, t_wait, t_upd, gather_ms = [], [], [], 0.0
+    hit_rows = miss_rows = 0
+    t0 = time.perf_counter()
+    for i, qd in enumerate(qs):
+        if i == warm:
+            torch.cuda.synchronize()
+            t_cache, t_wait, t_upd, gather_ms = [], [], [], 0.0
+            hit_rows = miss_rows = 0
+            t0 = time.perf_counter()
+        sel, _ = R.select_clusters(qd, idx, d, ws)
+        sel_host.copy_(sel.reshape(units, -1)[:, :k_r])  # waits for the selection
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if worker is None:
+            s0 = time.perf_counter()
+            fetch, admit, st = cache.plan(sel_np, k_r, counts, offsets)
+            t_cache.append(time.perf_counter() - s0)
+            nf, na = len(fetch), len(admit)
+            stage[0, :nf].numpy()[:] = fetch
+            stage[1, :na].numpy()[:] = admit
+            stage_d[0, :nf].copy_(stage[0, :nf], non_blocking=True)
+            stage_d[1, :na].copy_(stage[1, :na], non_blocking=True)
+            e0.record(stream)
+            R.gather_blocks(stage_d[0, :nf], hK, hV, eK, eV, gws, cK, cV)
+            e1.record(stream)
+            R.gather_blocks(stage_d[1, :na], hK, hV, eK, eV, gws, cK, cV)
+        else:
+            s0 = time.perf_counter()
+            worker.wait()            # the previous update, normally already applied
+            s1 = time.perf_counter()
+            fl, st = worker.lookup(sel_np, k_r, counts, offsets, stream)
+            s2 = time.perf_counter()
+            fd = worker.fetch_to_device(stream)
+            e0.record(stream)
+            R.gather_blocks(fd, hK, hV, eK, eV, gws, cK, cV)
+            e1.record(stream)
+            s3 = time.perf_counter()
+            worker.update_async(stream)
+            s4 = time.perf_counter()
+            t_wait.append(s1 - s0)
+            t_cache.append(s2 - s1)
+            t_upd.append(s4 - s3)
+        hit_rows += st["hit_rows"]
+        miss_rows += st["miss_rows"]
+        R.attend_selected(qd, idx, d, ws, exec_K=eK, exec_V=eV, out=out)
+        e1.synchronize()
+        gather_ms += e0.elapsed_time(e1)
+    torch.cuda.synchronize()
+    wall_s = time.perf_counter() - t0
+    steps = len(qs) - warm
+    status = max(R.read_device_status(ws), R.read_device_status(gws))
+    if worker is not None:
+        worker.close()
+        torch.cuda.synchronize()
+        status = max(status, R.read_device_status(wgws))
+    cache.validate()
+    cache.close()
+    host_bytes = miss_rows * 2 * 128 * 2  # K and V rows of the misses, bf16
+    res = {"steps_per_s": steps / wall_s, "ms_per_step": 1e3 * wall_s / steps,
+           "hit_rate_rows": hit_rows / max(1, hit_rows + miss_rows),
+           "host_bytes_per_step": host_bytes / steps,
+           "fetch_gather_ms_per_step": gather_ms / steps,
+           "host_link_gbs": host_bytes / max(1e-9, gather_ms * 1e-3) / 1e9,
+           "device_status": int(status)}
+    if worker is None:
+        res["plan_us_median"] = 1e6 * statistics.median(t_cache)
+    else:
+        res["lookup_us_median"] = 1e6 * statistics.median(t_cache)
+        res["wait_for_update_us_median"] = 1e6 * statistics.median(t_wait)
+        res["update_handoff_us_median"] = 1e6 * statistics.median(t_upd)
+        res["update_cost_on_critical_path_us"] = 1e6 * (statistics.median(t_wait) +
+                                                         statistics.median(t_upd))
+    return res, {"cache_blocks_per_head": cap, "exec_rows": exec_rows}
+
+
+def run_config5(dev, local):
+    """Llama3-8B-1048K geometry, batch 1, 1M-token context: K/V rows in pinned
+    host memory, a GPU block cache of 5 % of each head's 2 KB blocks (LRU),
+    64 decode steps with drifting queries, once with the synchronous cache
+    plan and once with the asynchronous update.  Wall clock per step (the
+    host's part of the step is on its critical path); the fetch gather is
+    also timed with CUDA events for the host-link rate."""
+    import kv_cache_vector_segmented_b200 as R
+    B5, H5, G5, N5, steps, warm = 1, 8, 4, 1 << 20, 64, 3
+    idx, kv = _build_for(R, dev, B5, H5, G5, N5, seed=51)
+    C = idx.geom.clusters
+    d = R.default_budgets(C)
+    hK = idx.Kp.cpu().pin_memory()
+    hV = idx.Vp.cpu().pin_memory()
+    counts = idx.counts.cpu().numpy().reshape(B5 * H5, C)
+    offsets = idx.offsets.cpu().numpy().reshape(B5 * H5, C + 1)
+    qs = S.drift_queries_device(S.make_queries_device(kv, G5, seed=52), warm + steps, seed=53)
+    out = {"workload": "llama3-8b-1048k decode, 1M context, batch 1, 32 q / 8 kv heads, "
+                       "K/V rows in pinned host memory, 5 % LRU block cache per head",
+           "clusters_per_head": C, "k_retrieval": d.k_retrieval, "k_estimation": d.k_estimation,
+           "steps": steps, "warmup": warm,
+           "timing": "wall clock per step (selection, its D2H, the cache step on the host, "
+                     "gathers, attention); fetch gather by CUDA events",
+           "data": "synthetic, drawn on the device; queries drift N(0, 0.05^2) per step"}
+    for mode in ("sync", "async"):
+        clocks = ClockSampler(local)
+        clocks.start()
+        r, geo = _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode)
+        r["clocks"] = clocks.stop()
+        out[mode] = r
+        out.update(geo)
+        torch.cuda.empty_cache()
+    return out
 
 
 # --------------------------------------------------------------------- oracle
@@ -372,24 +673,41 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(kv, budget_s=20.0):
-    """The oracle, as it stands, on the host cores: decode of sampled KV heads
-    (scaled to one 8-head step) and k-means of one segment."""
+def _oracle_decode_sample(idx, q, heads, budget_s, max_n=40):
+    """Per-head decode times of the oracle over `heads`, for about budget_s."""
     import oracle as O
-    t0 = time.time()
-    heads = [0, 1]
-    idx = _oracle_index(kv, heads)
-    q = S.make_queries(kv, G, seed=10).double().numpy()
     k_r, k_e = O.default_budgets(idx[0]["C"])
     per_head = []
-    while time.time() - t0 < budget_s * 0.5 or len(per_head) < 2:
+    t0 = time.time()
+    while time.time() - t0 < budget_s or len(per_head) < 2:
         for j, h in enumerate(heads):
             s = time.perf_counter()
             O.tripartite_attention(q[0, h * G:(h + 1) * G], idx[j], k_r, k_e)
             per_head.append(time.perf_counter() - s)
-        if len(per_head) >= 40:
+        if len(per_head) >= max_n:
             break
+    return per_head
+
+
+def cpu_baseline(kv, budget_s=20.0):
+    """The oracle, as it stands, on the host cores: decode of sampled KV heads
+    (scaled to one 8-head step) with numpy's BLAS on every core and on one
+    thread, and k-means of one segment (all cores)."""
+    import oracle as O
+    heads = [0, 1]
+    idx = _oracle_index(kv, heads)
+    q = S.make_queries(kv, G, seed=10).double().numpy()
+    per_head = _oracle_decode_sample(idx, q, heads, budget_s * 0.35)
     step_s = float(np.median(per_head)) * H
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            ph1 = _oracle_decode_sample(idx, q, heads, budget_s * 0.35)
+        single = {"value": 1.0 / (float(np.median(ph1)) * H), "unit": UNIT, "cores": 1,
+                  "sample": f"{len(ph1)} single-KV-head decodes, scaled x8"}
+    except Exception as e:  # threadpoolctl missing: say so
+        single = {"unavailable": f"threadpoolctl: {e}"}
     m0, M = O.middle_range(N)
     X = kv.K[0, 0, m0:m0 + 8192].double().numpy()
     init = np.random.default_rng(0).choice(8192, 512, replace=False)
@@ -400,6 +718,7 @@ def cpu_baseline(kv, budget_s=20.0):
             "sample": f"{len(per_head)} single-KV-head decodes (heads 0-1 of 8, 4 q heads each, "
                       f"147+1884 clusters) scaled x8 to one step; k-means: 1 segment of 8192 "
                       f"keys x 512 clusters x 10 iterations",
+            "single_thread": single,
             "kmeans_tok_per_s": 8192 / km_s, "host_cpu_count": os.cpu_count()}
 
 
@@ -429,124 +748,50 @@ def run_reference(args, ws_n, rank):
     step_s = float(np.mean(times))
     v = 1.0 / step_s
     sample = f"{n_heads} of {H} KV heads per step (4 q heads each), time scaled x{H / n_heads:g}"
+    C = idx0[0]["C"]
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": ws_n,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": N},
+            "data": "synthetic", "config": headline_config(ws_n, C, k_r, k_e),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "setup_s": time.perf_counter() - t0 - sum(times)}
 
 
-def run_profile_case():
-    """Small case for an ncu capture of the two kernels of the path: one
-    128K-token layer of the benchmark geometry (about 1.1 GB on the device),
-    one index build (10 k-means iterations) and 6 decode calls."""
+def run_profile_case(which):
+    """Small cases for ncu captures.  "decode": one 128K-token layer of the
+    headline geometry (about 1.1 GB on the device), one index build (10
+    k-means iterations) and 6 decode calls.  "gather": the 1M-token host
+    memory workload at 2 KV heads, 6 steps of select / plan / gather /
+    attend (the fetch and admit copies are gather_kernel launches)."""
     import kv_cache_vector_segmented_b200 as R
     dev = torch.device("cuda", 0)
-    cfg = R.IndexConfig.make(B, H, G, N, iters=10)
-    kv = S.make_kv(B, H, N, seed=0)
-    segs = _segment_sizes(R.geometry(cfg))
-    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B, H, seed=3)
-    idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
-    q = S.make_queries(kv, G, seed=10).to(dev)
-    dcfg = R.default_budgets(idx.geom.clusters)
-    ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, dcfg), dev)
-    for _ in range(6):
-        R.decode(q, idx, dcfg, workspace=ws)
-    torch.cuda.synchronize()
-    assert R.read_device_status(ws) == 0
-    print("profile case done", flush=True)
-
-
-def run_cfg5():
-    """Llama3-8B-1048K geometry, batch 1, 1M-token context: K/V rows in pinned
-    host memory, a GPU block cache of 5 % of each head's 2 KB blocks (LRU),
-    64 decode steps with drifting queries.  Each step: selection on the
-    device, the cache plan on the host, the gather of hits (cache) and misses
-    (host) into the execution buffer, admission of the misses, attention.
-    Wall-clock per step (the host plan and the step's sync are part of the
-    synchronous access path); the gather of the fetch list is also timed
-    with CUDA events for the host-link rate."""
-    import kv_cache_vector_segmented_b200 as R
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    B5, H5, G5, N5 = 1, 8, 4, 1 << 20
-    steps, warm = 64, 3
-    cfg = R.IndexConfig.make(B5, H5, G5, N5, iters=10)
-    geom = R.geometry(cfg)
-    kv = S.make_kv(B5, H5, N5, seed=0)
-    segs = _segment_sizes(geom)
-    ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B5, H5, seed=3)
-    idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg, init_pos=torch.from_numpy(ip).to(dev))
-    torch.cuda.synchronize()
-    del kv.K, kv.V  # the host copy that matters from here on is the permuted one
-    C = geom.clusters
-    d = R.default_budgets(C)
-    k_r = d.k_retrieval
-    hK = idx.Kp.cpu().pin_memory()
-    hV = idx.Vp.cpu().pin_memory()
-    counts = idx.counts.cpu().numpy().reshape(B5 * H5, C)
-    offsets = idx.offsets.cpu().numpy().reshape(B5 * H5, C + 1)
-    br = 8
-    blocks = (counts.astype(np.int64) + br - 1) // br
-    cache = R.BlockCache(B5 * H5, max(1, int(0.05 * blocks.sum(axis=1).max())), br)
-    cK = torch.zeros((B5, H5, cache.pool_rows, 128), dtype=torch.bfloat16, device=dev)
-    cV = torch.zeros_like(cK)
-    exec_rows = int(R.max_retrieval_rows(counts, k_r).max())
-    eK = torch.empty((B5, H5, exec_rows, 128), dtype=torch.bfloat16, device=dev)
-    eV = torch.empty_like(eK)
-    ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, d), dev)
-    gws = R.alloc_workspace(256, dev)
-    out = torch.empty((B5, H5 * G5, 128), dtype=torch.bfloat16, device=dev)
-    qs = [q.contiguous().to(dev) for q in
-          S.drift_queries(S.make_queries(kv, G5, seed=52), warm + steps, seed=53)]
-    hit_rows = miss_rows = 0
-    gather_ms = 0.0
-    t0 = time.perf_counter()
-    for i, qd in enumerate(qs):
-        if i == warm:
-            torch.cuda.synchronize()
-            hit_rows = miss_rows = 0
-            gather_ms = 0.0
-            t0 = time.perf_counter()
-        sel, _ = R.select_clusters(qd, idx, d, ws)
-        # only the retrieval ids (the first k_r of each unit) go back to the host
-        sel_r = sel.reshape(B5 * H5, -1)[:, :k_r].cpu().numpy()
-        fetch, admit, st = cache.plan(sel_r, k_r, counts, offsets)
-        hit_rows += st["hit_rows"]
-        miss_rows += st["miss_rows"]
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        fd = torch.from_numpy(fetch).to(dev)
-        e0.record()
-        R.gather_blocks(fd, hK, hV, eK, eV, gws, cK, cV)
-        e1.record()
-        R.gather_blocks(torch.from_numpy(admit).to(dev), hK, hV, eK, eV, gws, cK, cV)
-        R.attend_selected(qd, idx, d, ws, exec_K=eK, exec_V=eV, out=out)
-        e1.synchronize()
-        gather_ms += e0.elapsed_time(e1)
-    torch.cuda.synchronize()
-    wall_s = time.perf_counter() - t0
-    status = max(R.read_device_status(ws), R.read_device_status(gws))
-    cache.close()
-    host_bytes = miss_rows * 2 * 128 * 2  # K and V rows of the misses, bf16
-    return {
-        "leg": "config 5", "metric": "decode steps/s with K/V in host memory", "unit": "steps/s",
-        "value": steps / wall_s, "ms_per_step": 1e3 * wall_s / steps, "steps": steps,
-        "warmup": warm, "n_gpus": 1, "data": "synthetic",
-        "config": {"workload": "llama3-8b-1048k decode, 1M context, batch 1, 32 q / 8 kv heads, "
-                               "K/V rows in pinned host memory, 5 % LRU block cache per head",
-                   "clusters_per_head": C, "k_retrieval": k_r, "k_estimation": d.k_estimation,
-                   "cache_blocks_per_head": cache.cfg.blocks_per_unit, "exec_rows": exec_rows,
-                   "timing": "wall clock per step, host plan and the step's device sync "
-                             "included; fetch gather by CUDA events"},
-        "hit_rate_rows": hit_rows / max(1, hit_rows + miss_rows),
-        "host_bytes_per_step": host_bytes / steps,
-        "fetch_gather_ms_per_step": gather_ms / steps,
-        "host_link_gbs": host_bytes / max(1e-9, gather_ms * 1e-3) / 1e9,
-        "device_status": int(status),
-    }
+    if which == "decode":
+        cfg = R.IndexConfig.make(B, H, G, N, iters=10)
+        kv = S.make_kv(B, H, N, seed=0)
+        segs = _segment_sizes(R.geometry(cfg))
+        ip = S.init_positions([L for L, _ in segs], [k for _, k in segs], B, H, seed=3)
+        idx = R.build_index(kv.K.to(dev), kv.V.to(dev), cfg,
+                            init_pos=torch.from_numpy(ip).to(dev))
+        q = S.make_queries(kv, G, seed=10).to(dev)
+        dcfg = R.default_budgets(idx.geom.clusters)
+        ws = R.alloc_workspace(R.decode_workspace_bytes(cfg, dcfg), dev)
+        for _ in range(6):
+            R.decode(q, idx, dcfg, workspace=ws)
+        torch.cuda.synchronize()
+        assert R.read_device_status(ws) == 0
+    else:
+        idx, kv = _build_for(R, dev, 1, 2, 4, 1 << 20, seed=51)
+        C = idx.geom.clusters
+        d = R.default_budgets(C)
+        hK, hV = idx.Kp.cpu().pin_memory(), idx.Vp.cpu().pin_memory()
+        counts = idx.counts.cpu().numpy().reshape(2, C)
+        offsets = idx.offsets.cpu().numpy().reshape(2, C + 1)
+        qs = S.drift_queries_device(S.make_queries_device(kv, 4, seed=52), 6, seed=53)
+        r, _ = _cfg5_mode(R, dev, 0, idx, d, hK, hV, counts, offsets, qs, 1, "sync")
+        assert r["device_status"] == 0
+    print(f"profile case {which} done", flush=True)
 
 
 def main():
@@ -556,17 +801,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", action="store_true",
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the config1 / config4 / config5 legs")
+    ap.add_argument("--ncu-case", choices=["decode", "gather"], default=None,
                     help="run only the small case used for ncu captures")
-    ap.add_argument("--cfg5", action="store_true",
-                    help="run only the 1M-token host-memory leg (block cache, gather, "
-                         "attention) and print its own JSON line")
     args = ap.parse_args()
     if args.ncu_case:
-        run_profile_case()
-        return
-    if args.cfg5:
-        print(json.dumps(run_cfg5()), flush=True)
+        run_profile_case(args.ncu_case)
         return
     if args.warmup < 3:
         args.warmup = 3

@@ -273,13 +273,17 @@ typedef struct {
  * only (the device pool is caller-owned, see ri_gather_buffers). */
 typedef struct ri_cache ri_cache;
 
-/* Per-call counts from ri_cache_plan (summed over units). */
+/* Per-call counts from ri_cache_plan (summed over units).  Requested
+ * clusters of zero rows are counted in empty_clusters only. */
 typedef struct {
   int64_t hit_clusters, miss_clusters, uncached_clusters; /* uncached: served, not admitted */
   int64_t hit_rows, miss_rows;                            /* rows from the cache / the host */
+  int64_t empty_clusters;                                 /* requested clusters of 0 rows  */
 } ri_cache_stats;
 
 ri_status ri_cache_create(const ri_cache_config* cfg, ri_cache** out);
+/* Frees the host state.  A worker attached to the cache must be destroyed
+ * first. */
 void ri_cache_destroy(ri_cache* cache);
 
 /* One step of the synchronous access path, on the host.  For every unit u:
@@ -298,13 +302,26 @@ void ri_cache_destroy(ri_cache* cache);
  * most 16 rows (a cluster's blocks that are adjacent in the pool share one
  * copy); *n_fetch / *n_admit get their lengths.  Fails with
  * RI_ERR_CAPACITY (state unchanged) when a list would exceed its capacity,
- * RI_ERR_INVALID_ARG for bad pointers, ids or sizes.  Not thread-safe for one
- * cache. */
+ * RI_ERR_INVALID_ARG for bad pointers, ids or sizes, or when a worker is
+ * attached to the cache.  Not thread-safe for one cache. */
 ri_status ri_cache_plan(ri_cache* cache, const int32_t* sel_ids, int32_t sel_stride,
                         int32_t k_retrieval, const int32_t* counts, const int32_t* offsets,
                         int32_t clusters, ri_copy_desc* fetch, int32_t fetch_cap,
                         int32_t* n_fetch, ri_copy_desc* admit, int32_t admit_cap,
                         int32_t* n_admit, ri_cache_stats* stats);
+
+/* The blocks holding cluster `cluster` of unit `unit`, in row order, written
+ * to blocks[0 .. cap); *n_blocks = their number (0: not resident).  Host
+ * state only; RI_ERR_CAPACITY when cap is too small (*n_blocks still set).
+ * Not to be called while a worker's update may be running. */
+ri_status ri_cache_resident(const ri_cache* cache, int32_t unit, int32_t cluster,
+                            int32_t* blocks, int32_t cap, int32_t* n_blocks);
+
+/* Checks the invariants of the host state: per unit every block is free or
+ * held by exactly one resident cluster, block chains have their recorded
+ * lengths, and the LRU list holds exactly the resident clusters.  RI_OK or
+ * RI_ERR_INVALID_ARG with ri_last_error() naming the first violation. */
+ri_status ri_cache_validate(const ri_cache* cache);
 
 /* Rows of the execution buffer one step can need, per unit: the sum of the
  * k_retrieval largest cluster sizes (the retrieval zone is the k_retrieval
@@ -347,6 +364,93 @@ typedef struct {
  * the status word of `workspace` (>= 256 device bytes; cleared by the call). */
 ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
                            int32_t n_desc, void* workspace, ri_stream_t stream);
+
+/* ---- Asynchronous cache update [P2 §2.2 异步更新路径: a background thread
+ * runs the LRU replacement and updates the mapping table late, so the
+ * update's cost hides behind GPU work; P4 §2B; P1 三] ------------------------
+ * A worker attached to an ri_cache splits each ri_cache_plan step in two:
+ *  (1) ri_cache_lookup, on the caller's critical path: waits until the
+ *      previous step's update has been applied (host), makes `stream` wait
+ *      for that update's admit copies (device), then reads the mapping table
+ *      without changing it and writes the step's fetch list (cache->exec for
+ *      resident clusters, host->exec for the others: the same list
+ *      ri_cache_plan writes) and the step's lookup counts;
+ *  (2) ri_cache_update_async, after the caller has issued the fetch copies
+ *      on `stream`: records an event on `stream` and hands the update to the
+ *      worker thread, which applies ri_cache_plan's replacement rule to the
+ *      state, writes the admit list and, when admit_dev is given, copies the
+ *      list to the device and runs the admit copies (ri_gather_blocks'
+ *      kernel) on side_stream after the event.
+ * Every step therefore sees the state and gets the fetch list ri_cache_plan
+ * would have given it, so the execution buffer, and the attention over it,
+ * are identical to the synchronous path's.
+ * Failures of an update (injected, or a CUDA error issuing its copies) are
+ * reported once, by the next ri_cache_lookup (which then does nothing and
+ * may be called again) or ri_cache_worker_wait.  A failed update leaves a
+ * consistent state: the clusters it admitted before failing keep their admit
+ * copies; the step's other misses are not admitted and later units keep
+ * their previous state (a CUDA error takes the update's admissions back). */
+typedef struct ri_cache_worker ri_cache_worker;
+
+typedef struct {
+  ri_gather_buffers bufs;   /* as for ri_gather_blocks; units and pool_rows
+                               must match the cache; ignored without admit_dev */
+  ri_copy_desc* admit_dev;  /* device array of admit_cap descriptors, or NULL:
+                               host-only worker (no device work; the admit
+                               lists are left for the caller)              */
+  ri_copy_desc* admit_host; /* host array of admit_cap descriptors (pinned when
+                               admit_dev is given; NULL: worker-owned) */
+  int32_t admit_cap;        /* bounds one step's admit copies (RI_ERR_CAPACITY
+                               from the lookup when a step could exceed it) */
+  void* gather_workspace;   /* >= 256 device bytes: status word of the admit
+                               copies (sticky; read with ri_read_device_status) */
+  ri_stream_t side_stream;  /* stream of the admit copies (best: non-blocking) */
+  int32_t device;           /* CUDA device of the buffers and streams        */
+  uint64_t wait_limit_ns;   /* limit of every wait on the worker (0 = 10 s)  */
+  int32_t lookup_threads;   /* threads of the lookup, units split among them
+                               [P2 §2.2 同步访问路径: multi-threaded lookup of
+                               the mapping table]; 0 = min(8, cores / 2), never
+                               more than the units                          */
+} ri_cache_worker_config;
+
+/* Starts the worker thread of `cache` (one worker per cache; ri_cache_plan is
+ * refused while it is attached).  Creates two CUDA events on `device` when
+ * admit_dev is given. */
+ri_status ri_cache_worker_create(ri_cache* cache, const ri_cache_worker_config* cfg,
+                                 ri_cache_worker** out);
+/* Applies every handed-over update, waits (bounded) for their admit copies,
+ * stops the thread and frees the worker; returns a failure not yet
+ * reported. */
+ri_status ri_cache_worker_destroy(ri_cache_worker* worker);
+
+/* Step part (1); arguments as ri_cache_plan's, minus the admit list.  The
+ * stats carry the lookup counts (hits, misses, rows, empty clusters;
+ * uncached_clusters is 0: the update decides it).  RI_ERR_TIMEOUT when the
+ * previous update was not applied within the limit (nothing done);
+ * RI_ERR_CAPACITY when the fetch list, or the admit list of every miss,
+ * could exceed its capacity (state unchanged, nothing handed over). */
+ri_status ri_cache_lookup(ri_cache_worker* worker, const int32_t* sel_ids, int32_t sel_stride,
+                          int32_t k_retrieval, const int32_t* counts, const int32_t* offsets,
+                          int32_t clusters, ri_copy_desc* fetch, int32_t fetch_cap,
+                          int32_t* n_fetch, ri_cache_stats* stats, ri_stream_t stream);
+
+/* Step part (2): hands the last lookup's update to the worker.  Call after
+ * the fetch copies were issued on `stream`; RI_ERR_INVALID_ARG without a
+ * lookup to apply. */
+ri_status ri_cache_update_async(ri_cache_worker* worker, ri_stream_t stream);
+
+/* Waits (bounded) until every handed-over update has been applied; returns
+ * the update counts of the last one (uncached_clusters) and its number of
+ * admit copies, whose list is then in admit_host (or the worker's own list)
+ * until the next update starts.  Returns a failure not yet reported. */
+ri_status ri_cache_worker_wait(ri_cache_worker* worker, ri_cache_stats* stats, int32_t* n_admit);
+
+/* Test hooks of the update path: update number fail_update (0 = the first
+ * handed to this worker; -1 = none) stops after fail_after_admissions
+ * admissions with RI_ERR_HOST; every update first sleeps delay_us
+ * microseconds. */
+ri_status ri_cache_worker_test_hooks(ri_cache_worker* worker, int64_t fail_update,
+                                     int64_t fail_after_admissions, uint32_t delay_us);
 
 /* Synchronises `stream` and returns the status word previous calls wrote
  * into `workspace` (RI_OK if no device-side failure was recorded); a failure

@@ -17,7 +17,8 @@ _EXPORTS = (
     "lib", "read_device_status", "select_clusters", "selftest_wait_timeout", "decode_static",
     "STATIC_SCRATCH_BYTES", "BlockCache", "CopyDesc", "gather_blocks", "SRC_HOST", "SRC_CACHE",
     "SRC_EXEC", "DST_EXEC", "DST_CACHE", "max_retrieval_rows", "selftest_decode_timeout",
-    "FAULT_SCORE_COPY", "FAULT_SCORE_COMMIT", "FAULT_SCORE_SIZES")
+    "FAULT_SCORE_COPY", "FAULT_SCORE_COMMIT", "FAULT_SCORE_SIZES", "CacheWorker",
+    "Decoder")
 
 __all__ = list(_EXPORTS)
 

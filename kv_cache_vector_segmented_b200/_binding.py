@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 import os
+import re
 from typing import Optional
 
 import numpy as np
@@ -126,7 +127,7 @@ class CacheConfig(ctypes.Structure):
 class CacheStats(ctypes.Structure):
     _fields_ = [("hit_clusters", ctypes.c_int64), ("miss_clusters", ctypes.c_int64),
                 ("uncached_clusters", ctypes.c_int64), ("hit_rows", ctypes.c_int64),
-                ("miss_rows", ctypes.c_int64)]
+                ("miss_rows", ctypes.c_int64), ("empty_clusters", ctypes.c_int64)]
 
 
 class GatherBuffers(ctypes.Structure):
@@ -151,6 +152,34 @@ lib.ri_max_retrieval_rows.restype = ctypes.c_int
 lib.ri_max_retrieval_rows.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
 lib.ri_gather_blocks.restype = ctypes.c_int
 lib.ri_gather_blocks.argtypes = [_P(GatherBuffers), _vp, ctypes.c_int32, _vp, _vp]
+lib.ri_cache_resident.restype = ctypes.c_int
+lib.ri_cache_resident.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_int32,
+                                  _P(ctypes.c_int32)]
+lib.ri_cache_validate.restype = ctypes.c_int
+lib.ri_cache_validate.argtypes = [_vp]
+
+
+class CacheWorkerConfig(ctypes.Structure):
+    _fields_ = [("bufs", GatherBuffers), ("admit_dev", _vp), ("admit_host", _vp),
+                ("admit_cap", ctypes.c_int32), ("gather_workspace", _vp),
+                ("side_stream", _vp), ("device", ctypes.c_int32),
+                ("wait_limit_ns", ctypes.c_uint64), ("lookup_threads", ctypes.c_int32)]
+
+
+lib.ri_cache_worker_create.restype = ctypes.c_int
+lib.ri_cache_worker_create.argtypes = [_vp, _P(CacheWorkerConfig), _P(_vp)]
+lib.ri_cache_worker_destroy.restype = ctypes.c_int
+lib.ri_cache_worker_destroy.argtypes = [_vp]
+lib.ri_cache_lookup.restype = ctypes.c_int
+lib.ri_cache_lookup.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp,
+                                ctypes.c_int32, _vp, ctypes.c_int32, _P(ctypes.c_int32),
+                                _P(CacheStats), _vp]
+lib.ri_cache_update_async.restype = ctypes.c_int
+lib.ri_cache_update_async.argtypes = [_vp, _vp]
+lib.ri_cache_worker_wait.restype = ctypes.c_int
+lib.ri_cache_worker_wait.argtypes = [_vp, _P(CacheStats), _P(ctypes.c_int32)]
+lib.ri_cache_worker_test_hooks.restype = ctypes.c_int
+lib.ri_cache_worker_test_hooks.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_uint32]
 
 
 def check(status: int, where: str) -> None:
@@ -334,6 +363,46 @@ def decode(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = None,
     return out, lse, sel
 
 
+class Decoder:
+    """ri_decode_attention with the arguments marshalled once: a fixed index,
+    budgets, workspace and output tensors; each call passes only the query's
+    device pointer (same checks on the query's shape, dtype and device as
+    `decode`).  For callers that decode step after step on one layer."""
+
+    def __init__(self, index: Index, dcfg: Optional[DecodeConfig] = None,
+                 workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+        cfg = index.cfg
+        dev = index.device
+        B, H, G, d = cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.head_dim
+        self.dcfg = dcfg if dcfg is not None else default_budgets(index.geom.clusters)
+        nbytes = decode_workspace_bytes(cfg, self.dcfg)
+        self.ws = workspace if workspace is not None else alloc_workspace(nbytes, dev)
+        if self.ws.numel() < nbytes:
+            raise ValueError(f"workspace needs {nbytes} bytes")
+        self.out = out if out is not None else torch.empty((B, H * G, d), dtype=torch.bfloat16,
+                                                            device=dev)
+        _need(self.out, "out", torch.bfloat16, (B, H * G, d), dev)
+        if lse is None and want_lse:
+            lse = torch.empty((B, H * G), dtype=torch.float32, device=dev)
+        self.lse = lse
+        self.index, self.dev = index, dev
+        self._qshape = (B, H * G, d)
+        self._cfg, self._cidx = cfg, index.c_struct()
+        self._args = (ctypes.byref(cfg), ctypes.byref(self.dcfg))
+        self._tail = (ctypes.byref(self._cidx), self.out.data_ptr(), _ptr(self.lse), None,
+                      self.ws.data_ptr(), self.ws.numel())
+
+    def __call__(self, q: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+        if q.dtype != torch.bfloat16 or q.device != self.dev or \
+                tuple(q.shape) != self._qshape or not q.is_contiguous():
+            _need(q, "q", torch.bfloat16, self._qshape, self.dev)
+        s = (stream or torch.cuda.current_stream(self.dev)).cuda_stream
+        check(lib.ri_decode_attention(*self._args, q.data_ptr(), *self._tail, s),
+              "ri_decode_attention")
+        return self.out, self.lse
+
+
 STATIC_SCRATCH_BYTES = 4 << 20  # RI_STATIC_SCRATCH_BYTES
 
 
@@ -499,6 +568,23 @@ class BlockCache:
         stats = {f: getattr(st, f) for f, _ in CacheStats._fields_}
         return fetch[:nf.value].copy(), admit[:na.value].copy(), stats
 
+    def resident(self, unit: int, cluster: int) -> list:
+        """Blocks holding a cluster, in row order ([] when not resident)."""
+        buf = np.zeros(64, dtype=np.int32)
+        n = ctypes.c_int32(0)
+        rc = lib.ri_cache_resident(self._h, unit, cluster, buf.ctypes.data, buf.size,
+                                   ctypes.byref(n))
+        if rc == STATUS_CODES["RI_ERR_CAPACITY"]:
+            buf = np.zeros(n.value, dtype=np.int32)
+            rc = lib.ri_cache_resident(self._h, unit, cluster, buf.ctypes.data, buf.size,
+                                       ctypes.byref(n))
+        check(rc, "ri_cache_resident")
+        return [int(b) for b in buf[:n.value]]
+
+    def validate(self) -> None:
+        """ri_cache_validate: raises RIError naming the first broken invariant."""
+        check(lib.ri_cache_validate(self._h), "ri_cache_validate")
+
     def close(self) -> None:
         if getattr(self, "_h", None):
             self._destroy(self._h)
@@ -506,6 +592,166 @@ class BlockCache:
 
     def __del__(self):
         self.close()
+
+
+class CacheWorker:
+    """Asynchronous update path of a BlockCache (ri_cache_worker_*).
+
+    Each step: `lookup` (the critical path: waits for the previous update,
+    reads the mapping table, returns the fetch list), the caller's fetch
+    gather on `stream`, then `update_async` (the worker thread applies the
+    LRU replacement and, with device buffers, runs the admit copies on its
+    side stream).  Without exec_K / cache_K the worker is host-only: no device
+    work, the admit list of the last update is returned by `wait`."""
+
+    def __init__(self, cache: BlockCache, admit_cap: Optional[int] = None, *,
+                 host_K: Optional[torch.Tensor] = None, host_V: Optional[torch.Tensor] = None,
+                 cache_K: Optional[torch.Tensor] = None, cache_V: Optional[torch.Tensor] = None,
+                 exec_K: Optional[torch.Tensor] = None, exec_V: Optional[torch.Tensor] = None,
+                 gather_workspace: Optional[torch.Tensor] = None,
+                 side_stream: Optional[torch.cuda.Stream] = None, wait_limit_ns: int = 0,
+                 lookup_threads: int = 0):
+        self.cache = cache
+        units = cache.cfg.units
+        self.device_mode = exec_K is not None
+        cfg = CacheWorkerConfig()
+        cfg.wait_limit_ns = wait_limit_ns
+        cfg.lookup_threads = lookup_threads
+        if self.device_mode:
+            dev = exec_K.device
+            B, H, rows, d = exec_K.shape
+            if admit_cap is None:
+                admit_cap = max(1, units * rows)  # ceil(n / block_rows) <= n per cluster
+            if not (host_K.is_pinned() and host_V.is_pinned()):
+                raise ValueError("host_K and host_V must be pinned")
+            _need(exec_V, "exec_V", torch.bfloat16, tuple(exec_K.shape), dev)
+            _need(cache_K, "cache_K", torch.bfloat16, (B, H, cache.pool_rows, d), dev)
+            _need(cache_V, "cache_V", torch.bfloat16, (B, H, cache.pool_rows, d), dev)
+            self._admit_dev = torch.empty((admit_cap, 6), dtype=torch.int32, device=dev)
+            self._admit_host = torch.empty((admit_cap, 6), dtype=torch.int32).pin_memory()
+            self._side = side_stream or torch.cuda.Stream(dev)
+            self._gws = gather_workspace if gather_workspace is not None else \
+                alloc_workspace(256, dev)
+            self._keep = (host_K, host_V, cache_K, cache_V, exec_K, exec_V)
+            cfg.bufs = GatherBuffers(host_K.data_ptr(), host_V.data_ptr(), cache_K.data_ptr(),
+                                     cache_V.data_ptr(), exec_K.data_ptr(), exec_V.data_ptr(),
+                                     B * H, host_K.shape[2], cache.pool_rows, rows)
+            cfg.admit_dev = self._admit_dev.data_ptr()
+            cfg.admit_host = self._admit_host.data_ptr()
+            cfg.gather_workspace = self._gws.data_ptr()
+            cfg.side_stream = self._side.cuda_stream
+            cfg.device = dev.index if dev.index is not None else torch.cuda.current_device()
+            self.dev = dev
+            self._admit_np = self._admit_host.numpy()
+        else:
+            if admit_cap is None:
+                raise ValueError("a host-only worker needs admit_cap")
+            self._admit_np = np.empty((admit_cap, 6), dtype=np.int32)
+            cfg.admit_host = self._admit_np.ctypes.data
+            self.dev = None
+        cfg.admit_cap = admit_cap
+        self._cfg = cfg
+        self._fetch_cap = 0
+        self._fetch_copied = None  # event after the last H2D copy of the fetch list
+        h = _vp()
+        check(lib.ri_cache_worker_create(cache._h, ctypes.byref(cfg), ctypes.byref(h)),
+              "ri_cache_worker_create")
+        self._h = h
+        self._destroy = lib.ri_cache_worker_destroy
+
+    def _grow_fetch(self, cap: int) -> None:
+        if self._fetch_copied is not None:
+            self._fetch_copied.synchronize()
+        self._fetch_cap = cap
+        if self.device_mode:
+            self._fetch_host = torch.empty((cap, 6), dtype=torch.int32).pin_memory()
+            self._fetch_np = self._fetch_host.numpy()
+            self._fetch_dev = torch.empty((cap, 6), dtype=torch.int32, device=self.dev)
+        else:
+            self._fetch_np = np.empty((cap, 6), dtype=np.int32)
+
+    def _stream_ptr(self, stream) -> int:
+        if not self.device_mode:
+            return 0
+        return (stream or torch.cuda.current_stream(self.dev)).cuda_stream
+
+    def lookup(self, sel_ids: np.ndarray, k_retrieval: int, counts: np.ndarray,
+               offsets: np.ndarray, stream: Optional[torch.cuda.Stream] = None):
+        """ri_cache_lookup.  Returns (fetch int32 [n][6] numpy view, valid until the
+        next lookup, and the lookup stats)."""
+        units = self.cache.cfg.units
+        sel = np.ascontiguousarray(sel_ids, dtype=np.int32).reshape(units, -1)
+        cnt = np.ascontiguousarray(counts, dtype=np.int32).reshape(units, -1)
+        off = np.ascontiguousarray(offsets, dtype=np.int32).reshape(units, -1)
+        if self._fetch_cap < 1:
+            self._grow_fetch(max(1024, 4 * units * max(1, k_retrieval)))
+        elif self._fetch_copied is not None:
+            self._fetch_copied.synchronize()  # the pinned list is read by the last copy
+        nf = ctypes.c_int32(0)
+        st = CacheStats()
+        while True:
+            rc = lib.ri_cache_lookup(self._h, sel.ctypes.data, sel.shape[1], k_retrieval,
+                                     cnt.ctypes.data, off.ctypes.data, cnt.shape[1],
+                                     self._fetch_np.ctypes.data, self._fetch_cap,
+                                     ctypes.byref(nf), ctypes.byref(st),
+                                     self._stream_ptr(stream))
+            if rc != STATUS_CODES["RI_ERR_CAPACITY"]:
+                break
+            # a list that could overflow is refused with the state unchanged:
+            # grow the fetch list when it is the one, and look up again
+            m = re.match(r"cache lookup: (\d+) fetch / up to \d+ admit", lib_last_error())
+            if not m or int(m.group(1)) <= self._fetch_cap:
+                break
+            self._grow_fetch(int(m.group(1)))
+        check(rc, "ri_cache_lookup")
+        self._n_fetch = nf.value
+        return self._fetch_np[:nf.value], {f: getattr(st, f) for f, _ in CacheStats._fields_}
+
+    def fetch_to_device(self, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """The last lookup's fetch list copied (non-blocking, pinned) to the
+        device on `stream`: int32 [n][6]."""
+        s = stream or torch.cuda.current_stream(self.dev)
+        n = self._n_fetch
+        with torch.cuda.stream(s):
+            self._fetch_dev[:n].copy_(self._fetch_host[:n], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s)
+        self._fetch_copied = ev
+        return self._fetch_dev[:n]
+
+    def update_async(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        check(lib.ri_cache_update_async(self._h, self._stream_ptr(stream)),
+              "ri_cache_update_async")
+
+    def wait(self):
+        """ri_cache_worker_wait: (stats of the last update, its admit list)."""
+        st = CacheStats()
+        na = ctypes.c_int32(0)
+        check(lib.ri_cache_worker_wait(self._h, ctypes.byref(st), ctypes.byref(na)),
+              "ri_cache_worker_wait")
+        return {f: getattr(st, f) for f, _ in CacheStats._fields_}, \
+            self._admit_np[:na.value].copy()
+
+    def test_hooks(self, fail_update: int = -1, fail_after: int = 0, delay_us: int = 0) -> None:
+        check(lib.ri_cache_worker_test_hooks(self._h, fail_update, fail_after, delay_us),
+              "ri_cache_worker_test_hooks")
+
+    def close(self) -> None:
+        """Stops the worker (after every handed-over update); raises RIError
+        for a failure not yet reported."""
+        if getattr(self, "_h", None):
+            h, self._h = self._h, None
+            check(self._destroy(h), "ri_cache_worker_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lib_last_error() -> str:
+    return lib.ri_last_error().decode()
 
 
 def max_retrieval_rows(counts: np.ndarray, k_retrieval: int) -> np.ndarray:

@@ -214,6 +214,23 @@ static ri_status cuda_fail(cudaError_t e, const char* what) {
   return RI_ERR_CUDA;
 }
 
+namespace ri {
+ri_status check_gather_buffers(const ri_gather_buffers* bufs) {
+  RI_CHECK(bufs, RI_ERR_INVALID_ARG, "gather buffers are NULL");
+  RI_CHECK(bufs->units >= 1 && bufs->M >= 0 && bufs->pool_rows >= 0 && bufs->exec_rows >= 0,
+           RI_ERR_INVALID_ARG, "bad gather buffer sizes");
+  const void* ptrs[] = {bufs->host_K, bufs->host_V, bufs->cache_K, bufs->cache_V, bufs->exec_K,
+                        bufs->exec_V};
+  for (const void* q : ptrs)
+    RI_CHECK(!q || aligned16(q), RI_ERR_INVALID_ARG, "gather buffers must be 16-byte aligned");
+  RI_CHECK((bufs->host_K == nullptr) == (bufs->host_V == nullptr) &&
+               (bufs->cache_K == nullptr) == (bufs->cache_V == nullptr) &&
+               (bufs->exec_K == nullptr) == (bufs->exec_V == nullptr),
+           RI_ERR_INVALID_ARG, "K and V buffers must be given together");
+  return RI_OK;
+}
+}  // namespace ri
+
 extern "C" {
 
 const char* ri_status_string(ri_status s) {
@@ -492,21 +509,12 @@ ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config*
 
 ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
                            int32_t n_desc, void* workspace, ri_stream_t stream) {
-  RI_CHECK(bufs, RI_ERR_INVALID_ARG, "gather buffers are NULL");
   RI_CHECK(n_desc >= 0, RI_ERR_INVALID_ARG, "n_desc must be >= 0");
   RI_CHECK(n_desc == 0 || desc, RI_ERR_INVALID_ARG, "descriptors are NULL");
   RI_CHECK(workspace && aligned16(workspace), RI_ERR_INVALID_ARG,
            "workspace must be non-NULL and 16-byte aligned");
-  RI_CHECK(bufs->units >= 1 && bufs->M >= 0 && bufs->pool_rows >= 0 && bufs->exec_rows >= 0,
-           RI_ERR_INVALID_ARG, "bad gather buffer sizes");
-  const void* ptrs[] = {bufs->host_K, bufs->host_V, bufs->cache_K, bufs->cache_V, bufs->exec_K,
-                        bufs->exec_V};
-  for (const void* q : ptrs)
-    RI_CHECK(!q || aligned16(q), RI_ERR_INVALID_ARG, "gather buffers must be 16-byte aligned");
-  RI_CHECK((bufs->host_K == nullptr) == (bufs->host_V == nullptr) &&
-               (bufs->cache_K == nullptr) == (bufs->cache_V == nullptr) &&
-               (bufs->exec_K == nullptr) == (bufs->exec_V == nullptr),
-           RI_ERR_INVALID_ARG, "K and V buffers must be given together");
+  const ri_status bs = check_gather_buffers(bufs);
+  if (bs != RI_OK) return bs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytesHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");

@@ -113,6 +113,8 @@ struct GatherArgs {
 };
 cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_desc, int* status,
                           cudaStream_t s);
+// Argument checks of ri_gather_buffers (pointers, alignment, sizes).
+ri_status check_gather_buffers(const ri_gather_buffers* bufs);
 
 // --------------------------------------------------------------- build
 constexpr int kMaxSegLen = 16384;  // segment tokens (the sort stages labels in shared memory)

@@ -122,3 +122,64 @@ def init_positions(segment_lengths: list[int], clusters: list[int], batch: int,
             out[b, h, base:base + k] = rng.choice(L, size=k, replace=False)
             base += k
     return out
+
+
+@dataclasses.dataclass
+class DeviceKV:
+    """Keys/values drawn on a device (large benchmark workloads)."""
+
+    K: torch.Tensor          # bf16 [B][H_kv][N][d]
+    V: torch.Tensor          # bf16 [B][H_kv][N][d]
+    centres: torch.Tensor    # fp32 [B][H_kv][N_CENTRES][d]
+
+
+def make_kv_device(batch: int, num_kv_heads: int, seq_len: int, device, head_dim: int = 128,
+                   seed: int = 0, n_centres: int = N_CENTRES) -> DeviceKV:
+    """The recipe of `make_kv` drawn with torch's generator on `device`, one
+    generator per (sequence, KV head) seeded ``seed * 1_000_003 + unit``.  Same
+    distributions, different numbers than `make_kv` (which draws on the host
+    with numpy); used where only the shape and statistics of the workload
+    matter (throughput), so multi-GB inputs take milliseconds to draw."""
+    B, H, N, d = batch, num_kv_heads, seq_len, head_dim
+    K = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=device)
+    V = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=device)
+    centres = torch.empty((B, H, n_centres, d), dtype=torch.float32, device=device)
+    for u in range(B * H):
+        b, h = divmod(u, H)
+        g = torch.Generator(device=device)
+        g.manual_seed(seed * 1_000_003 + u)
+        c = torch.randn((n_centres, d), generator=g, device=device)
+        lab = torch.randint(0, n_centres, (N,), generator=g, device=device)
+        k = c[lab] + KEY_NOISE * torch.randn((N, d), generator=g, device=device)
+        n_out = min(N_OUTLIERS, N)
+        if n_out:
+            pos = torch.randperm(N, generator=g, device=device)[:n_out]
+            k[pos] *= OUTLIER_SCALE
+        K[b, h] = k.to(torch.bfloat16)
+        V[b, h] = torch.randn((N, d), generator=g, device=device).to(torch.bfloat16)
+        centres[b, h] = c
+    return DeviceKV(K=K, V=V, centres=centres)
+
+
+def make_queries_device(kv: DeviceKV, group_size: int, seed: int = 1) -> torch.Tensor:
+    """Queries of the `make_queries` recipe from a DeviceKV: bf16 [B][H_kv*G][d]."""
+    B, H, n_c, d = kv.centres.shape
+    g = torch.Generator(device=kv.centres.device)
+    g.manual_seed(seed)
+    j = torch.randint(0, n_c, (B, H, group_size), generator=g, device=kv.centres.device)
+    sel = torch.gather(kv.centres, 2, j[..., None].expand(B, H, group_size, d))
+    q = QUERY_CENTRE_WEIGHT * sel + QUERY_NOISE * torch.randn(
+        sel.shape, generator=g, device=kv.centres.device)
+    return q.reshape(B, H * group_size, d).to(torch.bfloat16)
+
+
+def drift_queries_device(q: torch.Tensor, steps: int, seed: int = 2) -> list[torch.Tensor]:
+    """`drift_queries` drawn on q's device."""
+    g = torch.Generator(device=q.device)
+    g.manual_seed(seed)
+    cur = q.float()
+    out = [q.clone()]
+    for _ in range(steps - 1):
+        cur = cur + QUERY_DRIFT * torch.randn(cur.shape, generator=g, device=q.device)
+        out.append(cur.to(torch.bfloat16))
+    return out

@@ -38,7 +38,8 @@ def _block_copies(unit, sk, dk, pieces):
 
 def expected_plan(models, sel, k_r, counts, offsets, br):
     fetch, admit = [], []
-    stats = dict(hit_clusters=0, miss_clusters=0, uncached_clusters=0, hit_rows=0, miss_rows=0)
+    stats = dict(hit_clusters=0, miss_clusters=0, uncached_clusters=0, hit_rows=0, miss_rows=0,
+                 empty_clusters=0)
     for u, model in enumerate(models):
         ids = [int(c) for c in sel[u, :k_r] if c >= 0]
         erow, run = {}, 0
@@ -50,7 +51,7 @@ def expected_plan(models, sel, k_r, counts, offsets, br):
         for c in ids:
             n = int(counts[u, c])
             if n == 0:
-                stats["hit_clusters"] += 1
+                stats["empty_clusters"] += 1
                 continue
             if c in before:
                 stats["hit_clusters"] += 1
@@ -153,6 +154,7 @@ def test_cluster_larger_than_the_cache_is_served_uncached():
     assert all(int(r[1]) == R.SRC_HOST for r in f)
     f, a, st = c.plan(steps[2], 3, counts, offsets)
     assert st["hit_clusters"] == 2 and st["uncached_clusters"] == 1
+    c.validate()
     c.close()
 
 
@@ -207,3 +209,204 @@ def test_max_retrieval_rows_rejects_bad_input():
     big = np.full((1, 3), 2 ** 30, dtype=np.int32)
     with pytest.raises(R.RIError):
         R.max_retrieval_rows(big, 3)   # 3 * 2^30 rows do not fit an int32
+
+
+# ---------------------------------------------------------------- cache worker
+# The asynchronous update path ("KV缓存技术与RetroInfer系统在长上下文推理中的优化实践"
+# (framerc.cn) §2.2 异步更新路径): lookup on the caller's thread, LRU update on
+# the worker's.  Host-only workers (no device buffers) run here without a GPU.
+
+def _random_steps(seed, units=3, C=64, k_r=12, n_steps=25):
+    rng = np.random.default_rng(seed)
+    sizes = rng.integers(0, 40, size=(units, C))
+    sizes[:, ::17] = 0
+    counts, offsets = _index_arrays(sizes)
+    cap = int(rng.integers(4, 30))
+    hot = [rng.choice(C, size=20, replace=False) for _ in range(units)]
+    steps = []
+    for _ in range(n_steps):
+        rows = []
+        for u in range(units):
+            pool = hot[u] if rng.random() < 0.7 else np.arange(C)
+            rows.append(rng.choice(pool, size=int(rng.integers(0, k_r + 1)), replace=False))
+        steps.append(_sel(rows, k_r))
+    return counts, offsets, cap, steps
+
+
+def _lookup_keys(st):
+    return {k: v for k, v in st.items() if k != "uncached_clusters"}
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+@pytest.mark.parametrize("delay_us", [0, 3000])
+def test_worker_steps_equal_the_synchronous_plan(seed, delay_us):
+    """Per step: the lookup's fetch list and counts, and the update's admit
+    list and uncached count, equal ri_cache_plan's on a second cache fed the
+    same steps.  With a delayed worker the lookup has to wait for the
+    previous update; the results must not change."""
+    units, k_r, br = 3, 12, 8
+    counts, offsets, cap, steps = _random_steps(seed, units=units, k_r=k_r)
+    sync = R.BlockCache(units, cap, br)
+    acache = R.BlockCache(units, cap, br)
+    w = R.CacheWorker(acache, admit_cap=units * 2000)
+    w.test_hooks(delay_us=delay_us)
+    for sel in steps:
+        f, a, st = sync.plan(sel, k_r, counts, offsets)
+        fl, lst = w.lookup(sel, k_r, counts, offsets)
+        assert _rows(fl) == _rows(f)
+        assert _lookup_keys(lst) == _lookup_keys(st) and lst["uncached_clusters"] == 0
+        w.update_async()
+        ust, al = w.wait()
+        assert _rows(al) == _rows(a)
+        assert ust["uncached_clusters"] == st["uncached_clusters"]
+    w.close()
+    acache.validate()
+    for u in range(units):
+        for c in range(counts.shape[1]):
+            assert acache.resident(u, c) == sync.resident(u, c)
+    sync.close()
+    acache.close()
+
+
+def test_worker_lookup_waits_for_the_previous_update():
+    """Back-to-back steps with no wait in between: each lookup must see the
+    previous step's admissions (a miss admitted at step t is a hit at t+1)."""
+    br = 8
+    counts, offsets = _index_arrays([[8, 16, 8, 8]])
+    c = R.BlockCache(1, 8, br)
+    w = R.CacheWorker(c, admit_cap=64)
+    w.test_hooks(delay_us=20000)  # 20 ms per update: the lookup must block
+    f0, s0 = w.lookup(_sel([[0, 1]], 3), 3, counts, offsets)
+    assert s0["miss_clusters"] == 2
+    w.update_async()
+    f1, s1 = w.lookup(_sel([[0, 1, 2]], 3), 3, counts, offsets)
+    assert s1["hit_clusters"] == 2 and s1["miss_clusters"] == 1
+    assert [int(r[1]) for r in f1] == [R.SRC_CACHE, R.SRC_CACHE, R.SRC_HOST]
+    w.update_async()
+    w.close()
+    c.validate()
+    assert len(c.resident(0, 2)) == 1
+    c.close()
+
+
+def test_worker_wait_limit_expires_and_recovers():
+    import time
+    counts, offsets = _index_arrays([[8, 16, 8, 8]])
+    c = R.BlockCache(1, 8, 8)
+    w = R.CacheWorker(c, admit_cap=64, wait_limit_ns=30_000_000)  # 30 ms
+    w.test_hooks(delay_us=300_000)                               # 300 ms update
+    w.lookup(_sel([[0, 1]], 3), 3, counts, offsets)
+    w.update_async()
+    with pytest.raises(R.RIError) as e:
+        w.lookup(_sel([[0, 2]], 3), 3, counts, offsets)
+    assert e.value.status == R.STATUS_CODES["RI_ERR_TIMEOUT"]
+    time.sleep(0.4)
+    f, st = w.lookup(_sel([[0, 2]], 3), 3, counts, offsets)  # the update has landed
+    assert st["hit_clusters"] == 1 and st["miss_clusters"] == 1
+    w.update_async()
+    w.close()
+    c.validate()
+    c.close()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_worker_injected_failure_leaves_a_consistent_cache(seed):
+    """Update number `t` fails before its first admission.  The failure is
+    reported once by the next lookup; the state is then exactly the oracle
+    model's after: units before the failing one updated, the failing unit's
+    requested residents made most recent (nothing admitted or evicted), later
+    units untouched.  From there on the worker again matches the model."""
+    units, k_r, br = 3, 12, 8
+    counts, offsets, cap, steps = _random_steps(seed + 10, units=units, k_r=k_r, n_steps=14)
+    t = 6
+    c = R.BlockCache(units, cap, br)
+    w = R.CacheWorker(c, admit_cap=units * 2000)
+    w.test_hooks(fail_update=t, fail_after=0)
+    models = [O.LRUClusterCache(cap, blocks=lambda cl, u=u: -(-int(counts[u, cl]) // br))
+              for u in range(units)]
+    failed_seen = False
+    for i, sel in enumerate(steps):
+        if i == t + 1:
+            with pytest.raises(R.RIError) as e:
+                w.lookup(sel, k_r, counts, offsets)
+            assert e.value.status == R.STATUS_CODES["RI_ERR_HOST"]
+            failed_seen = True
+        fl, _ = w.lookup(sel, k_r, counts, offsets)
+        if i == t:
+            # the failing update on the model: units in order until the first
+            # with a miss, which only refreshes its requested residents
+            for u in range(units):
+                ids = [int(x) for x in sel[u, :k_r] if x >= 0 and counts[u, x] > 0]
+                if any(x not in models[u].slot_of for x in ids):
+                    models[u].access([x for x in ids if x in models[u].slot_of])
+                    break
+                models[u].access(ids)
+            w.update_async()
+            continue
+        ef, ea, _ = expected_plan(models, sel, k_r, counts, offsets, br)
+        assert _rows(fl) == ef
+        w.update_async()
+        _, al = w.wait()
+        assert _rows(al) == ea
+    assert failed_seen
+    w.close()
+    c.validate()
+    c.close()
+
+
+def test_worker_failure_after_some_admissions_keeps_invariants():
+    units, k_r, br = 3, 12, 8
+    counts, offsets, cap, steps = _random_steps(7, units=units, k_r=k_r, n_steps=12)
+    c = R.BlockCache(units, cap, br)
+    w = R.CacheWorker(c, admit_cap=units * 2000)
+    w.test_hooks(fail_update=4, fail_after=2)
+    errors = 0
+    for sel in steps:
+        try:
+            fl, st = w.lookup(sel, k_r, counts, offsets)
+        except R.RIError as e:
+            assert e.status == R.STATUS_CODES["RI_ERR_HOST"]
+            errors += 1
+            fl, st = w.lookup(sel, k_r, counts, offsets)
+        # every cache-sourced copy reads blocks of a resident requested cluster
+        for r in fl:
+            if int(r[1]) == R.SRC_CACHE:
+                assert 0 <= int(r[2]) and int(r[2]) + int(r[5]) <= cap * br
+        w.update_async()
+        try:
+            w.wait()
+        except R.RIError as e:  # the failure is reported once, by the first to ask
+            assert e.status == R.STATUS_CODES["RI_ERR_HOST"]
+            errors += 1
+        c.validate()
+    assert errors == 1
+    w.close()
+    c.close()
+
+
+def test_worker_refusals():
+    counts, offsets = _index_arrays([[8, 16, 8, 8]])
+    c = R.BlockCache(1, 8, 8)
+    w = R.CacheWorker(c, admit_cap=1)
+    with pytest.raises(R.RIError):          # update without a lookup
+        w.update_async()
+    with pytest.raises(R.RIError):          # ri_cache_plan while a worker is attached
+        c.plan(_sel([[0]], 3), 3, counts, offsets)
+    with pytest.raises(R.RIError) as e:     # admit list could overflow: state unchanged
+        w.lookup(_sel([[0, 1]], 3), 3, counts, offsets)
+    assert e.value.status == R.STATUS_CODES["RI_ERR_CAPACITY"]
+    f, st = w.lookup(_sel([[0]], 3), 3, counts, offsets)
+    assert st["miss_clusters"] == 1
+    w.update_async()
+    w.close()
+    c.validate()
+    f, a, st = c.plan(_sel([[0]], 3), 3, counts, offsets)  # detached: plan works again
+    assert st["hit_clusters"] == 1
+    c.close()
+
+
+def test_validate_accepts_a_fresh_cache_and_rejects_null():
+    assert R.lib.ri_cache_validate(None) == R.STATUS_CODES["RI_ERR_INVALID_ARG"]
+    c = R.BlockCache(2, 5, 8)
+    c.validate()
+    c.close()

@@ -62,8 +62,9 @@ def test_gather_access_path(R, cache_frac):
         sel_h = sel.cpu().numpy().reshape(B * H, -1)
         fetch, admit, st = cache.plan(sel_h, k_r, counts, offsets)
         if step == 0:
-            assert st["hit_clusters"] == int((counts[np.arange(B * H)[:, None],
-                                                     np.maximum(sel_h[:, :k_r], 0)] == 0).sum())
+            assert st["hit_clusters"] == 0
+            assert st["empty_clusters"] == int((counts[np.arange(B * H)[:, None],
+                                                       np.maximum(sel_h[:, :k_r], 0)] == 0).sum())
         hits_seen += st["hit_rows"]
         for plan in (fetch, admit):  # fetch first, then admission into the pool
             R.gather_blocks(torch.from_numpy(plan).to(dev), hK, hV, eK, eV, gws, cK, cV)

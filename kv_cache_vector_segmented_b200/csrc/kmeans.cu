@@ -46,8 +46,8 @@ constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
 constexpr int kCand = 8;          // candidate slots per row
 constexpr int kUpdateWarps = 8;   // update / finalise: one warp per cluster
 constexpr int kSortThreads = 1024;
-constexpr int kGatherRows = 32;   // member rows per cp.async chunk of the update
-constexpr int kUpdateSmem = kUpdateWarps * kGatherRows * 128 * 2;  // 64 KB
+constexpr int kGatherRows = 16;   // member rows per cp.async chunk of the update
+constexpr int kUpdateSmem = kUpdateWarps * kGatherRows * 128 * 2;  // 32 KB
 constexpr int kFinRows = 16;      // member rows (K and V) per cp.async chunk of the finalise
 constexpr int kFinSmem = kUpdateWarps * kFinRows * 512;             // 64 KB
 constexpr uint16_t kCandNone = 0xFFFF;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     mbar_init(cent_empty, 1);
     for (int h = 0; h < 2; ++h) {
       mbar_init(&tfull[h], 1);
-      mbar_init(&tempty[h], 8 * 32);  // the 8 epilogue warps reading that half
+      mbar_init(&tempty[h], kEpiWarps * 32);  // every epilogue warp reads a slice of each half
     }
     mbar_init(drain, 1);
     for (int i = 0; i < 4; ++i) {
@@ -337,23 +337,26 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     mbar_wait_suspend(drain, 0);
   } else if (warp >= 2) {
     // ----------------------------------------------------------- epilogue
-    // Warp (lane quadrant q, column quarter Qc) reads columns
-    // [128 Qc, 128 Qc + 128) of the 32 TMEM lanes of quadrant q once per
-    // tile.  Per 32-column chunk: its maximum, and the mask of entries within
-    // the window of the running maximum R (w_j >= R - delta; a threshold at
-    // or below the row's final one keeps every candidate).  Masks of chunks
-    // whose maximum ends below R_quarter - delta are dropped: what remains
-    // holds every entry with w_j >= R_quarter - delta, and an entry outside
-    // that window only in a chunk whose own maximum is a second candidate.
-    // Quarters 0-2 hand (R, masks) to quarter 3, which decides the row: a
-    // quarter takes part iff its maximum is within delta of the row maximum
-    // W (then its entries are candidates, or the row has two or more
-    // candidates anyway).
+    // Warp (lane quadrant q, column slice Qc) reads columns [64 Qc, 64 Qc +
+    // 64) of each half (256 columns) of the 32 TMEM lanes of quadrant q once
+    // per tile: half 0 first, released to the MMA issuer as soon as all 16
+    // warps have read it, so the next tile's MMA into half 0 overlaps the
+    // epilogue of half 1.  Per 32-column chunk: its maximum, and the mask of
+    // entries within the window of the running maximum R (w_j >= R - delta;
+    // a threshold at or below the row's final one keeps every candidate).
+    // Masks of chunks whose maximum ends below R_slice - delta are dropped:
+    // what remains holds every entry with w_j >= R_slice - delta, and an
+    // entry outside that window only in a chunk whose own maximum is a second
+    // candidate.  Slices 0-2 hand (R, masks) to slice 3, which decides the
+    // row: a slice takes part iff its maximum is within delta of the row
+    // maximum W (then its entries are candidates, or the row has two or more
+    // candidates anyway).  Chunk c of slice Qc covers columns
+    // 256 (c >> 1) + 64 Qc + 32 (c & 1).
     const int ew = warp - 2;
-    const int Qc = ew >> 2;  // column quarter; half Qc / 2
+    const int Qc = ew >> 2;  // column slice
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(Qc * kQuarterN);
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(Qc * 64);
     float* xR = reinterpret_cast<float*>(sm + kSmXR);             // [3][128]
     uint32_t* xm = reinterpret_cast<uint32_t*>(sm + kSmXMask);    // [3][4][128]
     int prev_unit = -1;
@@ -370,23 +373,25 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       const bool valid = t < u.L;
       const float kn = valid ? knorm[(size_t)u.bh * d.M + u.seg_start + t] : 0.f;
       if (*abort_flag) break;
-      if (!mbar_wait_suspend(&tfull[Qc >> 1], (uint32_t)(it & 1))) {
-        record_status(status, RI_ERR_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
       // half the window a_j <= min a + 2 (||k|| E + C), in units of w = -a / 2
       const float delta = kn * uE + uC;
       float cm[4];
       uint32_t hit[4];
       float R = -FLT_MAX;
-      tc_fence_after();
+      bool timed_out = false;
 #pragma unroll
-      for (int cp = 0; cp < 2; ++cp) {
+      for (int cp = 0; cp < 2; ++cp) {  // cp = half of the accumulator
+        if (!mbar_wait_suspend(&tfull[cp], (uint32_t)(it & 1))) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
         uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(taddr + cp * 64, r0);
-        tmem_ld32_nowait(taddr + cp * 64 + 32, r1);
+        tmem_ld32_nowait(taddr + cp * kHalfN, r0);
+        tmem_ld32_nowait(taddr + cp * kHalfN + 32, r1);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[cp]);  // these columns are free for the next tile
         // both chunk maxima first (independent chains), one threshold
         float m4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
         float n4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
@@ -409,8 +414,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         hit[2 * cp] = (a4[0] | a4[1]) | (a4[2] | a4[3]);
         hit[2 * cp + 1] = (b4[0] | b4[1]) | (b4[2] | b4[3]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[Qc >> 1]);  // these columns are free for the next tile
+      if (timed_out) {
+        record_status(status, RI_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
       const float thr = R - delta;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -446,12 +454,19 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       for (int c = 0; c < 4; ++c) mq[12 + c] = hit[c];
       if (!valid) continue;
       const float W = fmaxf(fmaxf(Rq[0], Rq[1]), fmaxf(Rq[2], Rq[3]));
+      // chunks in column order: column chunk cc = 8 h + 2 Qc + j is chunk
+      // 2 h + j of slice Qc
+      uint32_t mc[16];
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const int k = (cc & 7) >> 1, c = ((cc >> 3) << 1) | (cc & 1);
+        mc[cc] = Rq[k] < W - delta ? 0u : mq[k * 4 + c];  // slice without candidates
+      }
       int ntot = 0, lab = -1;
 #pragma unroll
       for (int c = 15; c >= 0; --c) {
-        if (Rq[c >> 2] < W - delta) mq[c] = 0u;  // quarter without candidates
-        ntot += __popc(mq[c]);
-        if (mq[c]) lab = c * 32 + __ffs(mq[c]) - 1;
+        ntot += __popc(mc[c]);
+        if (mc[c]) lab = c * 32 + __ffs(mc[c]) - 1;
       }
       const int grow = u.bh * d.M + u.seg_start + t;
       labels[grow] = lab >= 0 ? lab : 0;
@@ -467,7 +482,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           int k = 0;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            uint32_t m = mq[c];
+            uint32_t m = mc[c];
             while (m) {
               const int b = __ffs(m) - 1;
               m &= m - 1u;
@@ -716,7 +731,7 @@ __global__ void __launch_bounds__(kSortThreads)
 // centroid and the cluster size.  Members are fetched 32 rows at a time with
 // 16-byte cp.async copies into the warp's 8 KB of shared memory (the
 // transfers need no registers, so a warp keeps a whole chunk in flight).
-__global__ void __launch_bounds__(kUpdateWarps * 32, 3)
+__global__ void __launch_bounds__(kUpdateWarps * 32, 6)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ members,
                   const int32_t* __restrict__ mstart, BuildDims d, float* __restrict__ mu,
                   __nv_bfloat16* __restrict__ mu_bf16, uint8_t* __restrict__ nsplit,
@@ -727,7 +742,7 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 3)
   const int bh = unit / d.S, s = unit % d.S;
   const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
   if (j >= Ks) return;
-  uint8_t* wb = smem_g + (size_t)warp * kGatherRows * kHeadDim * 2;  // [32 rows][256 B]
+  uint8_t* wb = smem_g + (size_t)warp * kGatherRows * kHeadDim * 2;  // [16 rows][256 B]
   const int seg_start = s * d.seg_len;
   const int32_t* ms = mstart + (size_t)unit * (kMaxClustersPerSeg + 1);
   const int b = ms[j], e = ms[j + 1];
@@ -736,7 +751,7 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 3)
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int i = b; i < e; i += kGatherRows) {
     const int nb = min(kGatherRows, e - i);
-    const int pos = lane < nb ? mem[i + lane] : 0;  // 32 member positions, one load
+    const int pos = lane < nb ? mem[i + lane] : 0;  // the chunk's member positions, one load
     // row r = 2 k + (lane >> 4), 16-byte chunk lane & 15
 #pragma unroll
     for (int k = 0; k < kGatherRows / 2; ++k) {

@@ -420,3 +420,167 @@ class LRUClusterCache:
                 self.order.remove(i)
                 self.order.append(i)
         return hits, misses
+
+
+# --------------------------------------------------------------------------
+# index maintenance during decode  [P2 §2.1 item 1 and pseudocode; reading]
+# --------------------------------------------------------------------------
+def open_slots(seg_len: int, k_last: int) -> int:
+    """Member slots of one open cluster when the last closed segment has
+    k_last clusters: ceil(2 * seg_len / k_last) (reading: twice the mean
+    occupancy, so the open segment always has room for seg_len tokens)."""
+    return -(-2 * seg_len // k_last)
+
+
+class GrowingIndex:
+    """The wave index of one (sequence, KV head) kept up to date while the
+    sequence grows by one token per decode step.
+
+    The pages fix the zones (the steady zone holds the first 4 and the most
+    recent 64 tokens, [P2 §2.1 item 1]) and that the index is k-means over
+    8K-token segments [P2 §2.1 pseudocode]; they are silent on what happens
+    to a token that leaves the recent window.  Reading (the plainest that
+    keeps every token in exactly one zone and the index segmented):
+
+    * appending token N moves token N - s1 out of the recent window into the
+      *open segment*;
+    * the open segment has K open clusters (K = min(clusters, seg_len)); the
+      moving token joins open cluster j, where j is its nearest centroid
+      (squared Euclidean distance to the stored bf16 centroids, lower id on
+      ties) among the K_last clusters of the last closed segment, counting
+      only clusters with a free slot (each open cluster has
+      ceil(2 seg_len / K_last) slots); n_j and Vsum_j grow by the token; open
+      cluster j is scored with
+      the centroid of cluster j of the last closed segment (the open clusters
+      beyond K_last stay empty);
+    * when the open segment holds seg_len tokens it is closed: k-means over
+      its tokens in position order (seeds floor(j L / K), the build's
+      iteration count) makes it a closed segment like the prefill's, and a
+      new empty open segment follows it.
+
+    Cluster ids: closed segments in order (the prefill's, then the closed
+    appended ones), then the K open clusters.  All of a token's arithmetic
+    is fp64 on the exact bf16 inputs.  Pinned by invariants (sizes sum to
+    the middle count, value sums equal member sums, every open member at a
+    nearest centroid with room, steady zone = first s0 and last s1 tokens),
+    by equality with a one-shot build of the longer sequence when the
+    segments line up, and by a hand-derived golden sequence."""
+
+    def __init__(self, K, V, base_len: int, init_pos=None, iters: int = DEFAULT_ITERS,
+                 seg_len: int = SEGMENT_TOKENS, clusters_per_seg: int = CLUSTERS_PER_SEGMENT,
+                 s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT):
+        # K, V: fp64 [N_max][d], every token the sequence will hold, by position
+        self.K = np.asarray(K, dtype=np.float64)
+        self.V = np.asarray(V, dtype=np.float64)
+        if base_len <= s0 + s1:
+            raise ValueError("the prefill must leave at least one middle token")
+        self.seg_len, self.iters, self.s0, self.s1 = seg_len, iters, s0, s1
+        self.Kc = min(clusters_per_seg, seg_len)
+        self.N = base_len
+        idx = build_index_head(self.K[:base_len], self.V[:base_len], init_pos, iters, seg_len,
+                               clusters_per_seg, s0, s1)
+        # closed clusters: members (positions, position order) and bf16 centroid
+        self.members: list[list[int]] = []
+        self.centroid: list[np.ndarray] = []
+        self.segments: list[tuple[int, int]] = []   # (first cluster id, clusters)
+        for c in range(idx["C"]):
+            a, n = idx["offsets"][c], idx["counts"][c]
+            self.members.append([int(p) for p in idx["perm"][a:a + n]])
+            self.centroid.append(idx["centroid"][c].copy())
+        base = 0
+        for _, _, Ks in segments(base_len - s0 - s1, seg_len, clusters_per_seg):
+            self.segments.append((base, Ks))
+            base += Ks
+        self._open_new()
+
+    def _open_new(self):
+        first, k_last = self.segments[-1]
+        self.targets = [self.centroid[first + j] for j in range(k_last)]
+        self.cap = open_slots(self.seg_len, k_last)
+        self.open: list[list[int]] = [[] for _ in range(self.Kc)]
+        self.open_start = self._middle_end()          # first position of the open segment
+
+    def _middle_end(self) -> int:
+        return self.N - self.s1
+
+    def open_distances(self, key: np.ndarray) -> np.ndarray:
+        """||key - c_j||^2 to the last closed segment's centroids."""
+        return np.array([float(((key - c) ** 2).sum()) for c in self.targets])
+
+    def choose(self, key: np.ndarray) -> int:
+        """Open cluster of a moving token: nearest target with a free slot,
+        lower id on ties."""
+        d = self.open_distances(key)
+        room = [j for j in range(len(self.targets)) if len(self.open[j]) < self.cap]
+        return min(room, key=lambda j: (d[j], j))
+
+    def append(self, chosen: int | None = None, close_labels=None) -> dict:
+        """Token N joins the sequence; token N - s1 moves into the open
+        segment (to `chosen` when given: another implementation's choice,
+        accepted when it has room and its distance is within 1e-5 relative of
+        the nearest with room).  Closes the open segment when it is full
+        (with `close_labels`, when given, as the clustering of its tokens:
+        another implementation's k-means result, used to mirror its state).
+        Returns {"moved": position, "cluster": open id, "closed": bool}."""
+        if self.N >= self.K.shape[0]:
+            raise ValueError("no more tokens to append")
+        p = self.N - self.s1
+        key = self.K[p]
+        j = self.choose(key)
+        if chosen is not None:
+            d = self.open_distances(key)
+            ok = (0 <= chosen < len(self.targets) and len(self.open[chosen]) < self.cap and
+                  d[chosen] <= d[j] + 1e-5 * (1.0 + d[j]))
+            if not ok:
+                raise AssertionError(f"open cluster {chosen} is not a nearest one with room "
+                                     f"(nearest {j}, distances {d[chosen]} vs {d[j]})")
+            j = chosen
+        self.open[j].append(p)
+        self.N += 1
+        closed = sum(len(m) for m in self.open) == self.seg_len
+        if closed:
+            self._close(close_labels)
+        return dict(moved=p, cluster=j, closed=closed)
+
+    def _close(self, labels=None):
+        pos = np.arange(self.open_start, self.open_start + self.seg_len)
+        X = self.K[pos]
+        L, Ks = self.seg_len, self.Kc
+        if labels is None:
+            res = kmeans(X, strided_init(L, Ks), self.iters)
+            labels, mu = res["labels"], res["mu"]
+        else:
+            labels = np.asarray(labels, dtype=np.int64)
+            mu, _ = update(X, labels, np.zeros((Ks, X.shape[1])))
+        first = len(self.members)
+        for c in range(Ks):
+            self.members.append([int(p) for p in pos[labels == c]])
+            self.centroid.append(bf16_round(mu[c]))
+        self.segments.append((first, Ks))
+        self.last_labels = labels
+        self._open_new()
+
+    # ---- views
+    def clusters(self) -> int:
+        """Live cluster ids: the closed ones and the K open ones."""
+        return len(self.members) + self.Kc
+
+    def steady(self) -> np.ndarray:
+        return steady_positions(self.N, self.s0, self.s1)
+
+    def to_index(self) -> dict:
+        """The state as an index dict for `tripartite_attention` (rows in id
+        order, members in position order; open clusters beyond K_last empty
+        with zero centroids)."""
+        d = self.K.shape[1]
+        mem = self.members + self.open
+        cent = self.centroid + [self.targets[j] if j < len(self.targets) else np.zeros(d)
+                                for j in range(self.Kc)]
+        counts = np.array([len(m) for m in mem], dtype=np.int64)
+        offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+        perm = np.array([p for m in mem for p in m], dtype=np.int64)
+        vsum = np.array([self.V[m].sum(axis=0) if m else np.zeros(d) for m in mem])
+        sp = self.steady()
+        return dict(N=self.N, C=len(mem), perm=perm, counts=counts, offsets=offsets,
+                    centroid=np.array(cent), vsum=vsum, Kp=self.K[perm], Vp=self.V[perm],
+                    Ks=self.K[sp], Vs=self.V[sp])

@@ -391,3 +391,137 @@ def test_lru_model_golden_sequence():
         assert sorted(cache.slot_of) == sorted(int(x) for x in resident)
         used = [b for bl in cache.slot_of.values() for b in bl]
         assert len(used) == len(set(used)) == len(cache.slot_of)
+
+
+# ---------------------------------------------------------------- index maintenance
+def _growing_golden():
+    rows = _golden_rows("growing_index.txt")
+    g = {"keys": {}, "append": [], "members": {}, "centroid": {}, "vsum": {}}
+    for r in rows:
+        t = r.split()
+        if t[0] == "params":
+            g["params"] = {k: int(v) for k, v in (x.split("=") for x in t[1:])}
+        elif t[0] == "key":
+            g["keys"][int(t[1])] = (float(t[2]), float(t[3]))
+        elif t[0] == "append":
+            g["append"].append((int(t[1]), int(t[2]), len(t) > 3 and t[3] == "close"))
+        elif t[0] in ("prefill_members", "closed_members"):
+            g["members"][int(t[1])] = [int(x) for x in t[3:]]
+        elif t[0] in ("prefill_centroid", "closed_centroid"):
+            g["centroid"][int(t[1])] = [float(x) for x in t[3:]]
+        elif t[0] == "close_labels":
+            g["close_labels"] = [int(x) for x in t[1:]]
+        elif t[0] == "final_steady":
+            g["steady"] = [int(x) for x in t[1:]]
+        elif t[0] == "final_counts":
+            g["counts"] = [int(x) for x in t[1:]]
+        elif t[0] == "final_vsum":
+            g["vsum"][int(t[1])] = [float(x) for x in t[3:]]
+    return g
+
+
+def test_growing_index_golden_sequence():
+    """Hand-derived prefill, four moves into the open segment, its close by
+    k-means and one move after the close."""
+    g = _growing_golden()
+    p = g["params"]
+    n = len(g["keys"])
+    K = np.array([g["keys"][i] for i in range(n)])
+    V = np.array([(i, 1.0) for i in range(n)])
+    gi = O.GrowingIndex(K, V, p["base_len"], iters=p["iters"], seg_len=p["seg_len"],
+                        clusters_per_seg=p["clusters"], s0=p["s0"], s1=p["s1"])
+    for c in (0, 1):
+        assert gi.members[c] == g["members"][c]
+        np.testing.assert_array_equal(gi.centroid[c], g["centroid"][c])
+    for moved, cl, closes in g["append"]:
+        r = gi.append()
+        assert (r["moved"], r["cluster"], r["closed"]) == (moved, cl, closes)
+        if closes:
+            assert list(gi.last_labels) == g["close_labels"]
+            for c in (2, 3):
+                assert gi.members[c] == g["members"][c]
+                np.testing.assert_array_equal(gi.centroid[c], g["centroid"][c])
+    idx = gi.to_index()
+    assert list(gi.steady()) == g["steady"]
+    assert list(idx["counts"]) == g["counts"]
+    for c, v in g["vsum"].items():
+        np.testing.assert_array_equal(idx["vsum"][c], v)
+
+
+def _growing_case(seed, N_max=700, base_len=68 + 150, seg_len=64, clusters=8, d=16):
+    rng = np.random.default_rng(seed)
+    centres = rng.standard_normal((12, d))
+    lab = rng.integers(0, 12, N_max)
+    K = O.bf16_round(centres[lab] + 0.3 * rng.standard_normal((N_max, d)))
+    V = O.bf16_round(rng.standard_normal((N_max, d)))
+    return K, V, O.GrowingIndex(K, V, base_len, iters=4, seg_len=seg_len,
+                                clusters_per_seg=clusters)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_growing_index_invariants(seed):
+    """After every append: sizes sum to the middle count, every middle
+    position is in exactly one cluster, value sums are member sums, the
+    steady zone is the first 4 and last 64 positions, and every open member
+    sits at a nearest target with room (brute force, direct differences)."""
+    K, V, gi = _growing_case(seed)
+    closes = 0
+    while gi.N < K.shape[0]:
+        before = [len(m) for m in gi.open]
+        targets = [t.copy() for t in gi.targets]
+        r = gi.append()
+        closes += r["closed"]
+        if not r["closed"]:
+            dist = [float(((K[r["moved"]] - t) ** 2).sum()) for t in targets]
+            room = [j for j in range(len(targets)) if before[j] < gi.cap]
+            best = min(room, key=lambda j: (dist[j], j))
+            assert r["cluster"] == best
+        idx = gi.to_index()
+        M = gi.N - 4 - 64
+        assert idx["counts"].sum() == M
+        assert sorted(idx["perm"].tolist()) == list(range(4, 4 + M))
+        assert list(gi.steady()) == list(range(4)) + list(range(gi.N - 64, gi.N))
+        for c in range(idx["C"]):
+            a, n = idx["offsets"][c], idx["counts"][c]
+            np.testing.assert_allclose(idx["vsum"][c], V[idx["perm"][a:a + n]].sum(axis=0),
+                                       atol=1e-12)
+    assert closes >= 7
+
+
+def test_growing_index_full_slots_send_tokens_to_the_next_nearest():
+    """Every key equal: all go to target 0 until its slots are full, then to
+    target 1, and so on (lower id on ties, only clusters with room)."""
+    d, seg_len, clusters = 4, 64, 8          # 16 slots per open cluster
+    N_max = 68 + seg_len + 40
+    rng = np.random.default_rng(3)
+    K = O.bf16_round(rng.standard_normal((N_max, d)))
+    K[68 + seg_len - 64:] = K[0]              # the moving tokens: one repeated key
+    V = np.ones((N_max, d))
+    gi = O.GrowingIndex(K, V, 68 + seg_len, iters=2, seg_len=seg_len, clusters_per_seg=clusters)
+    d2 = gi.open_distances(K[0])
+    order = sorted(range(len(gi.targets)), key=lambda j: (d2[j], j))
+    got = [gi.append()["cluster"] for _ in range(2 * gi.cap + 1)]
+    assert got == [order[0]] * gi.cap + [order[1]] * gi.cap + [order[2]]
+
+
+def test_growing_index_equals_one_shot_build_when_segments_line_up():
+    """A prefill of one full segment plus seg_len appends gives the same
+    closed clusters as building the longer sequence in one go (both seeded
+    by floor(j L / K)): the window, the move order and the close reproduce
+    the segmented build."""
+    d, seg_len, clusters, iters = 8, 128, 16, 5
+    base_len = 4 + seg_len + 64
+    N_end = base_len + seg_len
+    rng = np.random.default_rng(11)
+    centres = rng.standard_normal((20, d))
+    K = O.bf16_round(centres[rng.integers(0, 20, N_end)] + 0.3 * rng.standard_normal((N_end, d)))
+    V = O.bf16_round(rng.standard_normal((N_end, d)))
+    gi = O.GrowingIndex(K, V, base_len, iters=iters, seg_len=seg_len, clusters_per_seg=clusters)
+    for _ in range(seg_len):
+        gi.append()
+    one = O.build_index_head(K, V, None, iters, seg_len, clusters)
+    assert one["C"] == 2 * clusters == len(gi.members)
+    for c in range(one["C"]):
+        a, n = one["offsets"][c], one["counts"][c]
+        assert gi.members[c] == one["perm"][a:a + n].tolist()
+        np.testing.assert_array_equal(gi.centroid[c], one["centroid"][c])

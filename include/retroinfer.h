@@ -77,13 +77,22 @@ typedef struct {
   int32_t iters;            /* Lloyd iterations T (10)              */
   int32_t steady_initial;   /* 4                                    */
   int32_t steady_recent;    /* 64                                   */
+  /* Growing index (ri_index_open / ri_index_append; 0 = seq_len for both,
+   * a compact index):                                                    */
+  int32_t base_len;         /* tokens the prefill build indexed     */
+  int32_t capacity;         /* most tokens the layout has room for  */
 } ri_index_config;
 
 typedef struct {
   int32_t middle;       /* M                                         */
   int32_t num_segments; /* S = ceil(M / seg_len)                     */
-  int32_t clusters;     /* C = sum of K_s over segments              */
+  int32_t clusters;     /* C = sum of K_s over segments (growing: the
+                           live clusters, open segment included)     */
   int32_t steady;       /* min(N, steady_initial + steady_recent)    */
+  int32_t cluster_stride; /* clusters per unit in the index arrays (C
+                             when compact)                           */
+  int32_t row_stride;     /* Kp / Vp / perm rows per unit (M when
+                             compact)                                */
 } ri_geometry;
 
 /* Derived sizes of a configuration.  Host only; validates the config. */
@@ -140,6 +149,57 @@ size_t ri_build_index_workspace(const ri_index_config* cfg);
 ri_status ri_build_index(const ri_index_config* cfg, const void* K, const void* V,
                          const int32_t* init_pos, const ri_index* out, void* workspace,
                          size_t workspace_bytes, ri_stream_t stream);
+
+/* ---- Index maintenance during decode ---------------------------------
+ * [P2 §2.1 item 1: the steady zone holds the first 4 and the most recent 64
+ * tokens, so each decode step moves one token out of the recent window;
+ * P2 §2.1 pseudocode: k-means per 8K-token segment.  The pages give no
+ * mechanism; this is the reading the library implements.]
+ * A growing index is described by a config with base_len (tokens of the
+ * prefill build) < capacity; seq_len is the current length.  Every step
+ * appends token seq_len: the token at seq_len - steady_recent leaves the
+ * recent window and joins the *open segment* in the open cluster of its
+ * nearest centroid (squared Euclidean distance to the stored bf16
+ * centroids, ties to the lower id) among the K_last clusters of the last
+ * closed segment that still have a free slot (ceil(2 seg_len / K_last)
+ * slots per open cluster); that cluster's size and value sum grow by the
+ * token, and it is scored with the same centroid.  When the open segment
+ * holds seg_len tokens, k-means over them (position order, seeds
+ * floor(j L / K), `iters` iterations) makes it a closed segment and a new
+ * empty open segment of K = min(clusters_per_seg, seg_len) clusters follows.
+ * Layout per unit (ri_index_geometry gives the strides): clusters
+ * [cluster_stride], ids: the prefill's segments, the closed appended
+ * segments, then the K open clusters (live clusters C = those); rows
+ * [row_stride]: closed segments cluster-contiguous from row 0, the open
+ * clusters' slots after every closed row the capacity allows, members in
+ * arrival order; offsets[c] is cluster c's first row (counts[c] rows
+ * follow), offsets[cluster_stride] = row_stride.  Ks / Vs keep the first
+ * steady_initial tokens and the recent window as a ring (position p at
+ * slot steady_initial + ((p - base_len) mod steady_recent)).  The decode
+ * calls take the growing config with the current seq_len; labels and
+ * objective are not kept. */
+
+/* Copies a compact index built by ri_build_index (its config: cfg with
+ * base_len = capacity = 0 and seq_len = cfg->base_len) into the layout of
+ * the growing config cfg (seq_len == base_len < capacity) and sets up the
+ * first open segment.  `out` arrays sized by cfg's strides. */
+ri_status ri_index_open(const ri_index_config* cfg, const ri_index* compact, const ri_index* out,
+                        ri_stream_t stream);
+
+/* Bytes of workspace ri_index_append needs (0 unless cfg is growing). */
+size_t ri_index_append_workspace(const ri_index_config* cfg);
+
+/* One step of index maintenance for token cfg->seq_len of every (sequence,
+ * KV head): k_new, v_new bf16 [B][H_kv][d] (its key and value) enter the
+ * recent window, the leaving token joins the open segment, and the open
+ * segment is closed by k-means when it becomes full.  Call before the
+ * step's decode (whose config then has seq_len + 1).  assigned: optional
+ * int32 [B][H_kv], the open cluster (0..K_last-1) each leaving token joined.
+ * RI_ERR_CAPACITY when seq_len == capacity.  Device-side failures go to
+ * the workspace status word (sticky, like the decode calls'). */
+ri_status ri_index_append(const ri_index_config* cfg, const void* k_new, const void* v_new,
+                          const ri_index* idx, int32_t* assigned, void* workspace,
+                          size_t workspace_bytes, ri_stream_t stream);
 
 /* Zone budgets in clusters: k_retrieval = round(0.018 C), k_estimation =
  * round(0.23 C) by default [P2 §2.1 items 2-3].  The zones are clamped to

@@ -47,19 +47,25 @@ class IndexConfig(ctypes.Structure):
                 ("group_size", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("seq_len", ctypes.c_int32), ("seg_len", ctypes.c_int32),
                 ("clusters_per_seg", ctypes.c_int32), ("iters", ctypes.c_int32),
-                ("steady_initial", ctypes.c_int32), ("steady_recent", ctypes.c_int32)]
+                ("steady_initial", ctypes.c_int32), ("steady_recent", ctypes.c_int32),
+                ("base_len", ctypes.c_int32), ("capacity", ctypes.c_int32)]
 
     @classmethod
     def make(cls, batch: int, num_kv_heads: int, group_size: int, seq_len: int,
              seg_len: int = 8192, clusters_per_seg: int = 512, iters: int = 10,
-             steady_initial: int = 4, steady_recent: int = 64, head_dim: int = 128):
+             steady_initial: int = 4, steady_recent: int = 64, head_dim: int = 128,
+             base_len: int = 0, capacity: int = 0):
         return cls(batch, num_kv_heads, group_size, head_dim, seq_len, seg_len,
-                   clusters_per_seg, iters, steady_initial, steady_recent)
+                   clusters_per_seg, iters, steady_initial, steady_recent, base_len, capacity)
+
+    def copy(self) -> "IndexConfig":
+        return IndexConfig(*[getattr(self, f) for f, _ in self._fields_])
 
 
 class Geometry(ctypes.Structure):
     _fields_ = [("middle", ctypes.c_int32), ("num_segments", ctypes.c_int32),
-                ("clusters", ctypes.c_int32), ("steady", ctypes.c_int32)]
+                ("clusters", ctypes.c_int32), ("steady", ctypes.c_int32),
+                ("cluster_stride", ctypes.c_int32), ("row_stride", ctypes.c_int32)]
 
 
 class CIndex(ctypes.Structure):
@@ -109,6 +115,12 @@ lib.ri_read_device_status.argtypes = [_vp, _vp]
 lib.ri_selftest_wait_timeout.restype = ctypes.c_int
 lib.ri_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
 lib.ri_selftest_decode_timeout.restype = ctypes.c_int
+lib.ri_index_open.restype = ctypes.c_int
+lib.ri_index_open.argtypes = [_P(IndexConfig), _P(CIndex), _P(CIndex), _vp]
+lib.ri_index_append_workspace.restype = ctypes.c_size_t
+lib.ri_index_append_workspace.argtypes = [_P(IndexConfig)]
+lib.ri_index_append.restype = ctypes.c_int
+lib.ri_index_append.argtypes = [_P(IndexConfig), _vp, _vp, _P(CIndex), _vp, _vp, _sz, _vp]
 lib.ri_selftest_decode_timeout.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex),
                                            _vp, _vp, _sz, ctypes.c_int32, ctypes.c_uint64, _vp]
 
@@ -275,7 +287,7 @@ class Index:
     def empty(cls, cfg: IndexConfig, device, labels: bool = True, objective: bool = True):
         g = geometry(cfg)
         B, H, d = cfg.batch, cfg.num_kv_heads, cfg.head_dim
-        M, C, S, ns = g.middle, g.clusters, g.num_segments, g.steady
+        M, C, S, ns = g.row_stride, g.cluster_stride, g.num_segments, g.steady
         bf, i32, f32 = torch.bfloat16, torch.int32, torch.float32
         return cls(cfg=cfg, geom=g,
                    Kp=torch.empty((B, H, M, d), dtype=bf, device=device),
@@ -293,7 +305,7 @@ class Index:
     def check_shapes(self) -> None:
         cfg, g = self.cfg, self.geom
         B, H, d = cfg.batch, cfg.num_kv_heads, cfg.head_dim
-        M, C, ns = g.middle, g.clusters, g.steady
+        M, C, ns = g.row_stride, g.cluster_stride, g.steady
         dev = self.device
         _need(self.Kp, "Kp", torch.bfloat16, (B, H, M, d), dev)
         _need(self.Vp, "Vp", torch.bfloat16, (B, H, M, d), dev)
@@ -361,6 +373,48 @@ def decode(q: torch.Tensor, index: Index, dcfg: Optional[DecodeConfig] = None,
                                   ws.data_ptr(), ws.numel(), _stream(dev)),
           "ri_decode_attention")
     return out, lse, sel
+
+
+def index_open(compact: Index, capacity: int) -> Index:
+    """ri_index_open: a growing copy of a compact index (built over the
+    prefill), with room for `capacity` tokens per sequence."""
+    c = compact.cfg
+    cfg = IndexConfig.make(c.batch, c.num_kv_heads, c.group_size, c.seq_len, c.seg_len,
+                           c.clusters_per_seg, c.iters, c.steady_initial, c.steady_recent,
+                           c.head_dim, base_len=c.seq_len, capacity=capacity)
+    dev = compact.device
+    out = Index.empty(cfg, dev, labels=False, objective=False)
+    cc, co = compact.c_struct(), out.c_struct()
+    check(lib.ri_index_open(ctypes.byref(cfg), ctypes.byref(cc), ctypes.byref(co), _stream(dev)),
+          "ri_index_open")
+    return out
+
+
+def index_append_workspace_bytes(cfg: IndexConfig) -> int:
+    n = lib.ri_index_append_workspace(ctypes.byref(cfg))
+    if n == 0:
+        raise RIError(STATUS_CODES["RI_ERR_INVALID_ARG"], "ri_index_append_workspace")
+    return n
+
+
+def index_append(index: Index, k_new: torch.Tensor, v_new: torch.Tensor,
+                 workspace: torch.Tensor, assigned: Optional[torch.Tensor] = None) -> None:
+    """ri_index_append for token index.cfg.seq_len (k_new, v_new bf16
+    [B][H_kv][d]); advances index.cfg.seq_len and index.geom by one."""
+    cfg = index.cfg
+    dev = index.device
+    B, H, d = cfg.batch, cfg.num_kv_heads, cfg.head_dim
+    _need(k_new, "k_new", torch.bfloat16, (B, H, d), dev)
+    _need(v_new, "v_new", torch.bfloat16, (B, H, d), dev)
+    if assigned is not None:
+        _need(assigned, "assigned", torch.int32, (B, H), dev)
+    cidx = index.c_struct()
+    check(lib.ri_index_append(ctypes.byref(cfg), k_new.data_ptr(), v_new.data_ptr(),
+                              ctypes.byref(cidx), _ptr(assigned), workspace.data_ptr(),
+                              workspace.numel(), _stream(dev)),
+          "ri_index_append")
+    cfg.seq_len += 1
+    index.geom = geometry(cfg)
 
 
 class Decoder:

@@ -12,7 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libretroinfer.so")
-SOURCES = ["api.cpp", "cache.cpp", "decode.cu", "gather.cu", "kmeans.cu", "static_scratch.cu"]
+SOURCES = ["api.cpp", "cache.cpp", "decode.cu", "gather.cu", "grow.cu", "kmeans.cu",
+           "static_scratch.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

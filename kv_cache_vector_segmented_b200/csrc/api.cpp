@@ -125,6 +125,53 @@ bool make_geometry(const ri_index_config* cfg, Geometry* g) {
     g->L_last = g->K_last = g->C = 0;
     g->tiles_full = g->tiles_last = g->tiles_bh = 0;
   }
+  g->Cs = g->C;
+  g->Ms = g->M;
+  g->growing = false;
+  g->base_len = g->capacity = g->C0 = g->K_last0 = g->F = g->Fmax = g->L_open = 0;
+  g->open_id = g->tgt_id = g->K_tgt = g->cap = g->R0 = 0;
+  g->closed_rows = g->M;
+  const int base = c.base_len > 0 ? c.base_len : c.seq_len;
+  const int capa = c.capacity > 0 ? c.capacity : c.seq_len;
+  if (c.base_len < 0 || c.capacity < 0) {
+    set_error("base_len and capacity must be >= 0");
+    return false;
+  }
+  if (base == c.seq_len && capa == c.seq_len) return true;  // compact
+  // growing index: the prefill's segments, then whole appended segments,
+  // then one open segment of K_full clusters
+  if (!(base <= c.seq_len && c.seq_len <= capa) || base <= steady || c.steady_recent < 1) {
+    set_error("growing index needs steady_initial + steady_recent < base_len <= seq_len <= "
+              "capacity and steady_recent >= 1 (got %d, %d, %d)", base, c.seq_len, capa);
+    return false;
+  }
+  if ((long long)c.batch * c.num_kv_heads * capa > (1ll << 31) - 1) {
+    set_error("batch * num_kv_heads * capacity must be < 2^31");
+    return false;
+  }
+  g->growing = true;
+  g->base_len = base;
+  g->capacity = capa;
+  const int M0 = base - (int)steady;
+  const int S0 = (M0 + c.seg_len - 1) / c.seg_len;
+  const int L0 = M0 - (S0 - 1) * c.seg_len;
+  g->K_last0 = c.clusters_per_seg < L0 ? c.clusters_per_seg : L0;
+  g->C0 = (S0 - 1) * g->K_full + g->K_last0;
+  const int A = c.seq_len - base;
+  g->F = A / c.seg_len;
+  g->L_open = A % c.seg_len;
+  g->Fmax = (capa - base) / c.seg_len;
+  g->open_id = g->C0 + g->F * g->K_full;
+  g->C = g->open_id + g->K_full;
+  g->Cs = g->C0 + g->Fmax * g->K_full + g->K_full;
+  g->tgt_id = g->F == 0 ? g->C0 - g->K_last0 : g->C0 + (g->F - 1) * g->K_full;
+  g->K_tgt = g->F == 0 ? g->K_last0 : g->K_full;
+  g->cap = (2 * c.seg_len + g->K_tgt - 1) / g->K_tgt;
+  g->closed_rows = M0 + g->F * c.seg_len;
+  g->R0 = M0 + g->Fmax * c.seg_len;
+  g->Ms = g->R0 + 2 * c.seg_len + g->K_full;
+  g->S = S0 + g->F + 1;  // closed segments and the open one
+  // the k-means build geometry fields describe the prefill only
   return true;
 }
 
@@ -159,7 +206,7 @@ ri_status make_decode_layout(const Geometry& g, const ri_decode_config* dcfg, De
   const long long BH = g.BH();
   size_t off = kStatusBytesHost;
   L->off_score = off;
-  off = align_up(off + (size_t)BH * g.C * L->Gp * 4, 256);
+  off = align_up(off + (size_t)BH * g.Cs * L->Gp * 4, 256);  // room for every live C
   L->off_sel = off;
   off = align_up(off + (size_t)BH * (L->k_r + L->k_e) * 4, 256);
   L->off_rpre = off;
@@ -193,6 +240,37 @@ bool make_build_layout(const Geometry& g, BuildLayout* L) {
   off = align_up(off + BH * g.S * 513 * 4, 256);
   L->off_ecs = off;
   off = align_up(off + BH * g.S * 512 * 8, 256);
+  L->total = off;
+  return true;
+}
+
+bool make_append_layout(const Geometry& g, const ri_index_config* cfg, AppendLayout* L) {
+  ri_index_config c = *cfg;
+  c.seq_len = c.seg_len;  // one segment per unit, no steady zone
+  c.steady_initial = c.steady_recent = 0;
+  c.base_len = c.capacity = 0;
+  if (!make_geometry(&c, &L->gb)) return false;
+  make_build_layout(L->gb, &L->bl);
+  const size_t BH = (size_t)g.BH(), n = (size_t)g.seg_len, K = (size_t)g.K_full;
+  size_t off = align_up(L->bl.total, 1024);
+  L->off_sK = off;
+  off = align_up(off + BH * n * 256, 1024);
+  L->off_sV = off;
+  off = align_up(off + BH * n * 256, 1024);
+  L->off_Kp = off;
+  off = align_up(off + BH * n * 256, 1024);
+  L->off_Vp = off;
+  off = align_up(off + BH * n * 256, 1024);
+  L->off_perm = off;
+  off = align_up(off + BH * n * 4, 256);
+  L->off_cent = off;
+  off = align_up(off + BH * K * 256, 256);
+  L->off_counts = off;
+  off = align_up(off + BH * K * 4, 256);
+  L->off_offsets = off;
+  off = align_up(off + BH * (K + 1) * 4, 256);
+  L->off_vsum = off;
+  off = align_up(off + BH * K * 512, 256);
   L->total = off;
   return true;
 }
@@ -256,6 +334,8 @@ ri_status ri_index_geometry(const ri_index_config* cfg, ri_geometry* out) {
   out->middle = g.M;
   out->num_segments = g.S;
   out->clusters = g.C;
+  out->cluster_stride = g.Cs;
+  out->row_stride = g.Ms;
   out->steady = g.n_steady;
   return RI_OK;
 }
@@ -271,7 +351,7 @@ ri_status ri_default_budgets(int32_t clusters, ri_decode_config* out) {
 
 size_t ri_build_index_workspace(const ri_index_config* cfg) {
   Geometry g;
-  if (!make_geometry(cfg, &g)) return 0;
+  if (!make_geometry(cfg, &g) || g.growing) return 0;
   BuildLayout L;
   make_build_layout(g, &L);
   return L.total;
@@ -317,6 +397,9 @@ ri_status ri_build_index(const ri_index_config* cfg, const void* K, const void* 
                          size_t workspace_bytes, ri_stream_t stream) {
   Geometry g;
   if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(!g.growing, RI_ERR_UNSUPPORTED,
+           "the build makes a compact index (base_len and capacity 0 or seq_len); open it "
+           "with ri_index_open to let it grow");
   RI_CHECK(K && V, RI_ERR_INVALID_ARG, "K and V must be non-NULL");
   RI_CHECK(aligned16(K) && aligned16(V), RI_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
   RI_CHECK(!init_pos || aligned16(init_pos), RI_ERR_INVALID_ARG,
@@ -531,6 +614,114 @@ ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* de
   a.exec_rows = bufs->exec_rows;
   e = launch_gather(a, desc, n_desc, static_cast<int*>(workspace), s);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return RI_OK;
+}
+
+ri_status ri_index_open(const ri_index_config* cfg, const ri_index* compact, const ri_index* out,
+                        ri_stream_t stream) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(g.growing && cfg->seq_len == g.base_len, RI_ERR_INVALID_ARG,
+           "index open: cfg must describe a growing index at its prefill (seq_len == base_len "
+           "< capacity)");
+  ri_index_config cc = *cfg;
+  cc.base_len = cc.capacity = 0;
+  Geometry gc;
+  if (!make_geometry(&cc, &gc)) return RI_ERR_INVALID_ARG;
+  ri_status st = check_index_pointers(gc, compact, false);
+  if (st != RI_OK) return st;
+  if ((st = check_index_pointers(g, out, false)) != RI_OK) return st;
+  RI_CHECK(out->perm && compact->perm, RI_ERR_INVALID_ARG, "index open: perm is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t BH = (size_t)g.BH();
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t elem, dst_n, src_n;
+  } copies[] = {
+      {out->Kp, compact->Kp, 256, (size_t)g.Ms, (size_t)gc.M},
+      {out->Vp, compact->Vp, 256, (size_t)g.Ms, (size_t)gc.M},
+      {out->perm, compact->perm, 4, (size_t)g.Ms, (size_t)gc.M},
+      {out->centroid, compact->centroid, 256, (size_t)g.Cs, (size_t)gc.C},
+      {out->counts, compact->counts, 4, (size_t)g.Cs, (size_t)gc.C},
+      {out->offsets, compact->offsets, 4, (size_t)g.Cs + 1, (size_t)gc.C + 1},
+      {out->vsum, compact->vsum, 512, (size_t)g.Cs, (size_t)gc.C},
+  };
+  for (const Copy& c : copies) {
+    cudaError_t e = cudaMemcpy2DAsync(c.dst, c.dst_n * c.elem, c.src, c.src_n * c.elem,
+                                      c.src_n * c.elem, BH, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "index open: cudaMemcpy2DAsync");
+  }
+  const size_t steady_bytes = BH * (size_t)g.n_steady * 256;
+  cudaError_t e = cudaMemcpyAsync(out->Ks, compact->Ks, steady_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(out->Vs, compact->Vs, steady_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = launch_open_init(g, *out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "index open");
+  return RI_OK;
+}
+
+size_t ri_index_append_workspace(const ri_index_config* cfg) {
+  Geometry g;
+  if (!make_geometry(cfg, &g) || !g.growing) return 0;
+  AppendLayout L;
+  if (!make_append_layout(g, cfg, &L)) return 0;
+  return L.total;
+}
+
+ri_status ri_index_append(const ri_index_config* cfg, const void* k_new, const void* v_new,
+                          const ri_index* idx, int32_t* assigned, void* workspace,
+                          size_t workspace_bytes, ri_stream_t stream) {
+  Geometry g;
+  if (!make_geometry(cfg, &g)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(g.growing, RI_ERR_INVALID_ARG, "index append: cfg is not a growing index");
+  RI_CHECK(cfg->seq_len < g.capacity, RI_ERR_CAPACITY,
+           "index append: the layout is full (%d tokens)", g.capacity);
+  RI_CHECK(k_new && v_new && aligned16(k_new) && aligned16(v_new), RI_ERR_INVALID_ARG,
+           "k_new and v_new must be non-NULL and 16-byte aligned");
+  RI_CHECK(!assigned || aligned4(assigned), RI_ERR_INVALID_ARG, "assigned must be aligned");
+  ri_status st = check_index_pointers(g, idx, false);
+  if (st != RI_OK) return st;
+  RI_CHECK(idx->perm, RI_ERR_INVALID_ARG, "index append: perm is NULL");
+  AppendLayout L;
+  if (!make_append_layout(g, cfg, &L)) return RI_ERR_INVALID_ARG;
+  RI_CHECK(workspace && (reinterpret_cast<uintptr_t>(workspace) & 1023u) == 0,
+           RI_ERR_INVALID_ARG, "workspace must be non-NULL and 1024-byte aligned");
+  RI_CHECK(workspace_bytes >= L.total, RI_ERR_WORKSPACE,
+           "workspace has %zu bytes, append needs %zu", workspace_bytes, L.total);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  cudaError_t e = launch_append(g, *idx, k_new, v_new, assigned, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "index append");
+  if ((g.L_open + 1) % g.seg_len != 0) return RI_OK;
+  // the open segment is full: k-means turns it into a closed segment
+  e = launch_close_gather(g, *idx, ws + L.off_sK, ws + L.off_sV, status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "index append: close gather");
+  ri_index seg = {};
+  seg.Kp = ws + L.off_Kp;
+  seg.Vp = ws + L.off_Vp;
+  seg.perm = reinterpret_cast<int32_t*>(ws + L.off_perm);
+  seg.centroid = ws + L.off_cent;
+  seg.counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
+  seg.offsets = reinterpret_cast<int32_t*>(ws + L.off_offsets);
+  seg.vsum = reinterpret_cast<float*>(ws + L.off_vsum);
+  BuildArgs a;
+  a.K = ws + L.off_sK;
+  a.V = ws + L.off_sV;
+  a.init_pos = nullptr;
+  a.out = seg;
+  a.ws = ws;
+  st = launch_build(L.gb, L.bl, a, s);
+  if (st != RI_OK) return st;
+  e = launch_close_scatter(g, *idx, seg, s);
+  if (e != cudaSuccess) return cuda_fail(e, "index append: close scatter");
+  ri_index_config next = *cfg;
+  next.seq_len += 1;
+  Geometry gn;
+  if (!make_geometry(&next, &gn)) return RI_ERR_INVALID_ARG;
+  e = launch_open_init(gn, *idx, s);
+  if (e != cudaSuccess) return cuda_fail(e, "index append: open segment");
   return RI_OK;
 }
 

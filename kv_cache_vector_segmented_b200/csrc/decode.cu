@@ -167,13 +167,13 @@ struct Params {
   float* lse;
   int32_t* sel_user;
   int32_t* rpre_user;
-  float* score;   // ws [BH][C][Gp]
+  float* score;   // ws [BH][Cs][Gp]
   int32_t* sel;   // ws [BH][k_r + k_e]
   int32_t* rpre;  // ws [BH][k_r + 1]
   int* status;
   unsigned long long wait_ns;
   int fault;
-  int BH, C, M, n_steady, k_r, k_e, kr, ke, tiles, exec_rows, mode;
+  int BH, C, Cs, Ms, n_steady, k_r, k_e, kr, ke, tiles, exec_rows, mode;
 };
 
 struct Misc {
@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int CS = (int)cluster_nrank();
   const int b = (int)cluster_rank();
   const int u = (int)blockIdx.x / CS;
-  const int C = p.C;
+  const int C = p.C, Cs = p.Cs;  // live clusters, per-unit stride
   const unsigned long long lim = p.wait_ns;
   const bool selecting = p.mode != kModeAttend && C > 0;
   // this block's tiles: b, b + CS, b + 2 CS, ... of the unit's ceil(C / 128)
@@ -605,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* stage = sm + st * kTileBytes;
         mbar_arrive_expect_tx(&ms->fullA[st], kTileBytes);
-        const int row = u * C + (b + it * CS) * kTileC;
+        const int row = u * Cs + (b + it * CS) * kTileC;
         if (!(p.fault == RI_FAULT_SCORE_COPY && it == 0)) {
           tma_load_2d(stage, &tm_cent, 0, row, &ms->fullA[st]);
           tma_load_2d(stage + kTileC * 128, &tm_cent, 64, row, &ms->fullA[st]);
@@ -654,8 +654,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 8) {
       // sizes and first rows of the block's clusters, all loads in flight at
       // once while the tiles arrive
-      const int32_t* cg = p.counts + (size_t)u * C;
-      const int32_t* og = p.offsets + (size_t)u * (C + 1);
+      const int32_t* cg = p.counts + (size_t)u * Cs;
+      const int32_t* og = p.offsets + (size_t)u * (Cs + 1);
       for (int i0 = tid - 256; i0 < nid; i0 += 4 * 256) {
         int cv[4], ov[4];
 #pragma unroll
@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < ntiles; ++it) {
         const int cl = it * kTileC + rr;
         const bool valid = cl < nid;
-        const size_t gc = (size_t)u * C + id_of(cl);
+        const size_t gc = (size_t)u * Cs + id_of(cl);
         ok = ok && wait_bar(&ms->tdone[it], 0, lim);
         if (epilogue_any(!ok)) {  // the 128 threads leave together
           if (!ok) record_status(p.status, RI_ERR_TIMEOUT);
@@ -869,13 +869,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool sureE = !sureR && ((finB && g > gB) || infB) && (!onA || (finA && g < gA));
           if (sureR) {
             const int2 mt = meta[i];
-            if (mt.y > 0 && mt.x >= 0 && (long long)mt.x + mt.y <= p.M) {
-              const size_t r0 = (size_t)u * p.M + mt.x;
+            if (mt.y > 0 && mt.x >= 0 && (long long)mt.x + mt.y <= p.Ms) {
+              const size_t r0 = (size_t)u * p.Ms + mt.x;
               prefetch_l2_bulk(p.Kr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
               prefetch_l2_bulk(p.Vr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
             }
           } else if (sureE) {
-            prefetch_l2_bulk(p.vsum + ((size_t)u * C + id_of(i)) * kHeadDim, 512u);
+            prefetch_l2_bulk(p.vsum + ((size_t)u * Cs + id_of(i)) * kHeadDim, 512u);
           }
         }
       }
@@ -1033,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool inE = !inR && onB && o >= thrB;
         if (inR || inE) {
           const int off = mm[j].x, cnt = mm[j].y;
-          const bool ok = inR ? (cnt >= 0 && off >= 0 && (long long)off + cnt <= p.M)
+          const bool ok = inR ? (cnt >= 0 && off >= 0 && (long long)off + cnt <= p.Ms)
                               : cnt >= 0;
           if (!ok) {
             bad = true;
@@ -1184,13 +1184,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // workspace by the same tile ownership, so the one-call decode and the
   // split calls fold the same items in the same order.
   const bool exec = p.exec_rows > 0;
-  const long long lim_rows = exec ? p.exec_rows : p.M;
+  const long long lim_rows = exec ? p.exec_rows : p.Ms;
   const int n_st = p.n_steady;
   const int st0 = (int)((long long)n_st * b / CS), st1 = (int)((long long)n_st * (b + 1) / CS);
   if (!selecting && C > 0) {
     const int32_t* selg = p.sel + (size_t)u * (p.k_r + p.k_e);
     const int32_t* rpg = p.rpre + (size_t)u * (p.k_r + 1);
-    const int32_t* off_u = p.offsets + (size_t)u * (C + 1);
+    const int32_t* off_u = p.offsets + (size_t)u * (Cs + 1);
     // R: the workspace's retrieval clusters (id order) of this block's tiles
     {
       const int kr = p.kr;
@@ -1259,7 +1259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int id = __ldcg(selg + p.k_r + g);
         if (id >= 0 && id < C && (id >> 7) % CS == b) {
           if (pos < kMaxIdsPerBlock)
-            lists[pos] = make_int2(id, max(0, __ldg(p.counts + (size_t)u * C + id)));
+            lists[pos] = make_int2(id, max(0, __ldg(p.counts + (size_t)u * Cs + id)));
           ++pos;
         }
       }
@@ -1483,7 +1483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int2 ev = elist[e];
         if (ev.y > 0) {
           uint8_t* slot = ering + (uint32_t)(e % kESlots) * kSlotE;
-          const size_t uc = (size_t)u * C + ev.x;
+          const size_t uc = (size_t)u * Cs + ev.x;
           cp_async16(slot + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
           if (lane < Gp / 4) cp_async16(slot + 512 + lane * 16, p.score + uc * Gp + lane * 4);
         }
@@ -1778,7 +1778,8 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   p.fault = a.fault;
   p.BH = (int)g.BH();
   p.C = g.C;
-  p.M = g.M;
+  p.Cs = g.Cs;
+  p.Ms = g.Ms;
   p.n_steady = g.n_steady;
   p.k_r = L.k_r;
   p.k_e = L.k_e;
@@ -1792,7 +1793,7 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   memset(&map_c, 0, sizeof(map_c));
   memset(&map_q, 0, sizeof(map_q));
   if (g.C > 0 && mode != kModeAttend) {
-    cudaError_t e = encode_rows(&map_c, a.centroid, (unsigned long long)g.BH() * g.C, kTileC);
+    cudaError_t e = encode_rows(&map_c, a.centroid, (unsigned long long)g.BH() * g.Cs, kTileC);
     if (e == cudaSuccess) e = encode_rows(&map_q, a.q, (unsigned long long)g.BH() * G, kQRows);
     if (e != cudaSuccess) return e;
   }

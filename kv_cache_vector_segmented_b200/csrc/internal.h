@@ -30,6 +30,21 @@ struct Geometry {
   int K_full;              // clusters of a full segment = min(K, seg_len)
   int L_last, K_last;      // length / clusters of the last segment
   int tiles_full, tiles_last, tiles_bh;  // 128-row assignment tiles
+  // Layout strides per unit: Cs clusters, Ms rows (= C, M for a compact
+  // index; the capacity layout of a growing index otherwise).
+  int Cs, Ms;
+  // Growing index (index maintenance during decode; all 0 / false when
+  // compact): prefill of base_len tokens, room for `capacity` tokens.
+  bool growing;
+  int base_len, capacity;
+  int C0, K_last0;   // clusters of the prefill's segments, of its last segment
+  int F, Fmax;       // closed appended segments (now / at capacity)
+  int L_open;        // tokens in the open segment
+  int open_id;       // first open cluster id (K_full open clusters follow)
+  int tgt_id, K_tgt; // the last closed segment's clusters (assignment targets)
+  int cap;           // member slots of one open cluster
+  int R0;            // first row of the open region
+  int closed_rows;   // rows of the closed segments (cluster-contiguous from row 0)
   long long BH() const { return (long long)B * H; }
 };
 
@@ -147,6 +162,26 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
 
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
                                          cudaStream_t s);
+
+// --------------------------------------------------------------- growing index
+// Workspace of ri_index_append: the close's segment build from offset 0 (its
+// status word is the call's), then the open tokens in position order
+// (sK, sV [BH][seg_len][d]) and the built segment (a compact index of one
+// segment per unit).
+struct AppendLayout {
+  Geometry gb;     // geometry of the close's build (seq_len = seg_len, no steady zone)
+  BuildLayout bl;
+  size_t off_sK, off_sV, off_Kp, off_Vp, off_perm, off_cent, off_counts, off_offsets, off_vsum;
+  size_t total;
+};
+bool make_append_layout(const Geometry& g, const ri_index_config* cfg, AppendLayout* L);
+cudaError_t launch_open_init(const Geometry& g, const ri_index& idx, cudaStream_t s);
+cudaError_t launch_append(const Geometry& g, const ri_index& idx, const void* k_new,
+                          const void* v_new, int32_t* assigned, int* status, cudaStream_t s);
+cudaError_t launch_close_gather(const Geometry& g, const ri_index& idx, void* sK, void* sV,
+                                int* status, cudaStream_t s);
+cudaError_t launch_close_scatter(const Geometry& g, const ri_index& idx, const ri_index& seg,
+                                 cudaStream_t s);
 
 // Thread-local last error.
 void set_error(const char* fmt, ...);

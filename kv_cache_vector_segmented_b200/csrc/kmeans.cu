@@ -39,7 +39,6 @@ namespace {
 
 constexpr int kRows = 128;        // keys per tile = MMA M
 constexpr int kHalfN = 256;       // centroids per MMA = MMA N
-constexpr int kQuarterN = 128;    // centroid columns per epilogue warp
 constexpr int kStages = 2;        // key tile ring
 constexpr int kEpiWarps = 16;       // assignment epilogue: 4 lane quadrants x 4 column quarters
 constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
@@ -65,9 +64,9 @@ constexpr uint32_t kSmBar = kSmOnes + kRows * 32;
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1 + 8;
 constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
 // hand-over from column quarters 0-2 to quarter 3 of a TMEM lane quadrant
-constexpr uint32_t kSmXR = (kSmMisc + 64 + 15) / 16 * 16;            // [3][128] f32
-constexpr uint32_t kSmXMask = kSmXR + 3 * kRows * 4;                  // [3][4 chunks][128] u32
-constexpr uint32_t kAssignSmem = kSmXMask + 3 * 4 * kRows * 4 + 1024;  // + alignment
+constexpr uint32_t kSmXR = (kSmMisc + 64 + 15) / 16 * 16;            // [4][128] f32
+constexpr uint32_t kSmXMask = kSmXR + 4 * kRows * 4;                  // [4][4 chunks][128] u32
+constexpr uint32_t kAssignSmem = kSmXMask + 4 * 4 * kRows * 4 + 1024;  // + alignment
 static_assert(kAssignSmem <= 227 * 1024, "assignment kernel shared memory");
 
 // Queue of rows whose label needs an exact decision.
@@ -347,8 +346,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     // Masks of chunks whose maximum ends below R_slice - delta are dropped:
     // what remains holds every entry with w_j >= R_slice - delta, and an
     // entry outside that window only in a chunk whose own maximum is a second
-    // candidate.  Slices 0-2 hand (R, masks) to slice 3, which decides the
-    // row: a slice takes part iff its maximum is within delta of the row
+    // candidate.  Three slices hand (R, masks) to the fourth (slice
+    // tile mod 4), which decides the row: a slice takes part iff its
+    // maximum is within delta of the row
     // maximum W (then its entries are candidates, or the row has two or more
     // candidates anyway).  Chunk c of slice Qc covers columns
     // 256 (c >> 1) + 64 Qc + 32 (c & 1).
@@ -423,7 +423,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         if (cm[c] < thr) hit[c] = 0u;
-      if (Qc < 3) {
+      // the slice that decides the rows of this quadrant rotates with the
+      // tile, so the decision work is shared by the four slices' warps
+      const int dq = it & 3;
+      if (Qc != dq) {
         if (it >= 1 && !mbar_wait_suspend(&xempty[q], (uint32_t)((it - 1) & 1))) {
           record_status(status, RI_ERR_TIMEOUT);
           *abort_flag = 1;
@@ -443,15 +446,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       float Rq[4];
       uint32_t mq[16];
 #pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        Rq[k] = xR[k * kRows + row];
+      for (int k = 0; k < 4; ++k) {
+        if (k == Qc) {
+          Rq[k] = R;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) mq[k * 4 + c] = xm[(k * 4 + c) * kRows + row];
+          for (int c = 0; c < 4; ++c) mq[k * 4 + c] = hit[c];
+        } else {
+          Rq[k] = xR[k * kRows + row];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) mq[k * 4 + c] = xm[(k * 4 + c) * kRows + row];
+        }
       }
       mbar_arrive(&xempty[q]);
-      Rq[3] = R;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) mq[12 + c] = hit[c];
       if (!valid) continue;
       const float W = fmaxf(fmaxf(Rq[0], Rq[1]), fmaxf(Rq[2], Rq[3]));
       // chunks in column order: column chunk cc = 8 h + 2 Qc + j is chunk

@@ -468,7 +468,7 @@ class GrowingIndex:
 
     def __init__(self, K, V, base_len: int, init_pos=None, iters: int = DEFAULT_ITERS,
                  seg_len: int = SEGMENT_TOKENS, clusters_per_seg: int = CLUSTERS_PER_SEGMENT,
-                 s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT):
+                 s0: int = STEADY_INITIAL, s1: int = STEADY_RECENT, prefill: dict | None = None):
         # K, V: fp64 [N_max][d], every token the sequence will hold, by position
         self.K = np.asarray(K, dtype=np.float64)
         self.V = np.asarray(V, dtype=np.float64)
@@ -477,13 +477,17 @@ class GrowingIndex:
         self.seg_len, self.iters, self.s0, self.s1 = seg_len, iters, s0, s1
         self.Kc = min(clusters_per_seg, seg_len)
         self.N = base_len
-        idx = build_index_head(self.K[:base_len], self.V[:base_len], init_pos, iters, seg_len,
-                               clusters_per_seg, s0, s1)
+        # the prefill's clustering: built here, or given (perm, counts,
+        # offsets, centroid of another implementation's prefill index, to
+        # follow its state)
+        idx = prefill if prefill is not None else build_index_head(
+            self.K[:base_len], self.V[:base_len], init_pos, iters, seg_len, clusters_per_seg,
+            s0, s1)
         # closed clusters: members (positions, position order) and bf16 centroid
         self.members: list[list[int]] = []
         self.centroid: list[np.ndarray] = []
         self.segments: list[tuple[int, int]] = []   # (first cluster id, clusters)
-        for c in range(idx["C"]):
+        for c in range(len(idx["counts"])):
             a, n = idx["offsets"][c], idx["counts"][c]
             self.members.append([int(p) for p in idx["perm"][a:a + n]])
             self.centroid.append(idx["centroid"][c].copy())

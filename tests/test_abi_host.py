@@ -152,3 +152,51 @@ def test_build_workspace_holds_every_array(R, B, H, N):
             + BH * C * 4 + BH * M * 4 + BH * M * 4 + BH * M * 20 + BH * M * 4
             + BH * S * 513 * 4 + BH * S * 512 * 8)
     assert R.build_workspace_bytes(R.IndexConfig.make(B, H, 4, N)) >= need
+
+
+# ---------------------------------------------------------------- growing index
+@pytest.mark.parametrize("base_len,appended,seg_len,clusters", [
+    (68 + 300, 0, 128, 16), (68 + 300, 127, 128, 16), (68 + 300, 128, 128, 16),
+    (68 + 300, 300, 128, 16), (68 + 2 * 8192 + 700, 150, 8192, 512), (69, 5, 8192, 512)])
+def test_growing_geometry_matches_oracle(R, base_len, appended, seg_len, clusters):
+    """Live clusters of a growing index = the oracle's: the prefill's
+    segments, one closed segment per seg_len appended tokens, K open ones."""
+    cap = base_len + 400
+    cfg = R.IndexConfig.make(1, 2, 4, base_len + appended, seg_len=seg_len,
+                             clusters_per_seg=clusters, base_len=base_len, capacity=cap)
+    g = R.geometry(cfg)
+    pre = O.segments(base_len - 68, seg_len, clusters)
+    K = min(clusters, seg_len)
+    C = sum(k for _, _, k in pre) + (appended // seg_len) * K + K
+    assert g.clusters == C
+    assert g.middle == base_len + appended - 68
+    Fmax = (cap - base_len) // seg_len
+    assert g.cluster_stride == sum(k for _, _, k in pre) + Fmax * K + K
+    assert g.row_stride == base_len - 68 + Fmax * seg_len + 2 * seg_len + K
+
+
+def test_growing_calls_reject_bad_arguments(R):
+    import torch
+    cfg = R.IndexConfig.make(1, 2, 4, 368, seg_len=128, clusters_per_seg=16, base_len=368,
+                             capacity=400)
+    # the build makes compact indexes only
+    assert R.lib.ri_build_index_workspace(ctypes.byref(cfg)) == 0
+    bad = R.IndexConfig.make(1, 2, 4, 368, base_len=400, capacity=500)  # seq_len < base_len
+    assert R.lib.ri_index_append_workspace(ctypes.byref(bad)) == 0
+    compact = R.IndexConfig.make(1, 2, 4, 368, seg_len=128, clusters_per_seg=16)
+    assert R.lib.ri_index_append_workspace(ctypes.byref(compact)) == 0
+    full = R.IndexConfig.make(1, 2, 4, 400, seg_len=128, clusters_per_seg=16, base_len=368,
+                              capacity=400)
+    idx = R.CIndex()
+    st = R.lib.ri_index_append(ctypes.byref(full), None, None, ctypes.byref(idx), None, None, 0,
+                               None)
+    assert st == R.STATUS_CODES["RI_ERR_CAPACITY"]
+    st = R.lib.ri_index_append(ctypes.byref(cfg), None, None, ctypes.byref(idx), None, None, 0,
+                               None)
+    assert st == R.STATUS_CODES["RI_ERR_INVALID_ARG"]
+    # open needs the config at its prefill (seq_len == base_len)
+    later = R.IndexConfig.make(1, 2, 4, 370, seg_len=128, clusters_per_seg=16, base_len=368,
+                               capacity=400)
+    st = R.lib.ri_index_open(ctypes.byref(later), ctypes.byref(idx), ctypes.byref(idx), None)
+    assert st == R.STATUS_CODES["RI_ERR_INVALID_ARG"]
+    assert torch  # noqa

@@ -229,6 +229,8 @@ def run_ours(args, ws_n, rank, local):
         kms.append(e0.elapsed_time(e1))
     build_ms = statistics.median(kms)
     assign_flop = 2.0 * H * M * 512 * 128 * 10
+    prefill = (build_beside_prefill(R, Kd, Vd, cfg, ipd, base, build_ws, dev)
+               if ws_n == 1 and not args.headline_only else None)
 
     # ---- 32 layer instances (distinct memory, so L2 cannot hold a cycle)
     def clone_index(ix):
@@ -374,7 +376,8 @@ def run_ours(args, ws_n, rank, local):
         "kmeans": {"tok_per_s": H * M / (build_ms * 1e-3), "ms_per_build": build_ms,
                    "iters": 10, "segments_per_head": len(segs), "clusters_per_segment": 512,
                    "assign_tflops_lower_bound": assign_flop / (build_ms * 1e-3) / 1e12,
-                   "assign_frac_of_sustained_bf16": assign_flop / (build_ms * 1e-3) / 1e12 / tf_sus},
+                   "assign_frac_of_sustained_bf16": assign_flop / (build_ms * 1e-3) / 1e12 / tf_sus,
+                   "beside_prefill": prefill},
         "clocks": clk,
         "e2e": {"value": k_e2e * ws_n / (ms_e2e / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": B * H * G * 128 * 2,
@@ -395,6 +398,72 @@ def run_ours(args, ws_n, rank, local):
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(kv, budget_s=20.0)
     return res
+
+
+# ------------------------------------------------------------ build and prefill
+def build_beside_prefill(R, Kd, Vd, cfg, ipd, base, build_ws, dev):
+    """The index build next to the prefill it belongs to: causal attention of
+    the same layer (32 query heads on 8 KV heads, 128K tokens, torch's SDPA
+    flash kernel, a library call used only as the yardstick) timed alone,
+    the build alone, and both at once on two streams; and the build with 16K
+    segments (512 clusters each).  CUDA events; medians of 3."""
+    Bq, Hq, Nq = cfg.batch, cfg.num_kv_heads * cfg.group_size, cfg.seq_len
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    q = torch.randn((Bq, Hq, Nq, 128), generator=g, device=dev).to(torch.bfloat16)
+    k = Kd.repeat_interleave(cfg.group_size, dim=1)
+    v = Vd.repeat_interleave(cfg.group_size, dim=1)
+    s_pre, s_bld = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def prefill():
+        torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+
+    def build():
+        R.build_index(Kd, Vd, cfg, init_pos=ipd, out=base, workspace=build_ws)
+
+    def timed(fns):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ends = []
+        for st, fn in fns:
+            st.wait_event(e0)
+            with torch.cuda.stream(st):
+                fn()
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(st)
+                ends.append(e)
+        torch.cuda.synchronize()
+        return max(e0.elapsed_time(e) for e in ends)
+
+    timed([(s_pre, prefill)])  # warm-up (SDPA's first call)
+    t_pre = statistics.median(timed([(s_pre, prefill)]) for _ in range(3))
+    t_bld = statistics.median(timed([(s_bld, build)]) for _ in range(3))
+    t_both = statistics.median(timed([(s_pre, prefill), (s_bld, build)]) for _ in range(3))
+    assert R.read_device_status(build_ws) == 0
+    del q, k, v
+    cfg16 = R.IndexConfig.make(cfg.batch, cfg.num_kv_heads, cfg.group_size, cfg.seq_len,
+                               seg_len=16384, clusters_per_seg=512, iters=cfg.iters)
+    segs16 = _segment_sizes(R.geometry(cfg16), seg_len=16384)
+    ip16 = S.init_positions([L for L, _ in segs16], [kk for _, kk in segs16], cfg.batch,
+                            cfg.num_kv_heads, seed=7)
+    ip16 = torch.from_numpy(ip16).to(dev)
+    idx16 = R.build_index(Kd, Vd, cfg16, init_pos=ip16)
+    t16 = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        R.build_index(Kd, Vd, cfg16, init_pos=ip16, out=idx16, workspace=idx16._build_ws)
+        e1.record()
+        torch.cuda.synchronize()
+        t16.append(e0.elapsed_time(e1))
+    assert R.read_device_status(idx16._build_ws) == 0
+    del idx16
+    return {"prefill_attention_ms": t_pre, "build_ms": t_bld, "both_on_two_streams_ms": t_both,
+            "build_share_of_prefill_attention": t_bld / t_pre,
+            "added_by_build_when_overlapped_ms": t_both - t_pre,
+            "build_seg16k_ms": statistics.median(t16), "seg16k_clusters_per_segment": 512,
+            "prefill": "causal SDPA (flash), 32 q heads x 128K tokens x d 128, bf16, one layer"}
 
 
 # ------------------------------------------------------------ other workloads
@@ -545,16 +614,19 @@ def _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode):
         stage = torch.empty((2, cap_l, 6), dtype=torch.int32).pin_memory()
         stage_d = torch.empty((2, cap_l, 6), dtype=torch.int32, device=dev)
     t_cache, t_wait, t_upd, gather_ms = [], [], [], 0.0
-    hit_rows = miss_rows = 0
+    hit_rows = miss_rows = rows_req = blocks_req = 0
     t0 = time.perf_counter()
     for i, qd in enumerate(qs):
         if i == warm:
             torch.cuda.synchronize()
             t_cache, t_wait, t_upd, gather_ms = [], [], [], 0.0
-            hit_rows = miss_rows = 0
+            hit_rows = miss_rows = rows_req = blocks_req = 0
             t0 = time.perf_counter()
         sel, _ = R.select_clusters(qd, idx, d, ws)
         sel_host.copy_(sel.reshape(units, -1)[:, :k_r])  # waits for the selection
+        nreq = counts[np.arange(units)[:, None], np.maximum(sel_np, 0)] * (sel_np >= 0)
+        rows_req += int(nreq.sum())
+        blocks_req += int(((nreq + br - 1) // br).sum())
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if worker is None:
             s0 = time.perf_counter()
@@ -606,6 +678,7 @@ def _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode):
            "host_bytes_per_step": host_bytes / steps,
            "fetch_gather_ms_per_step": gather_ms / steps,
            "host_link_gbs": host_bytes / max(1e-9, gather_ms * 1e-3) / 1e9,
+           "fragment_rows_skipped_frac": 1.0 - rows_req / max(1, br * blocks_req),
            "device_status": int(status)}
     if worker is None:
         res["plan_us_median"] = 1e6 * statistics.median(t_cache)

@@ -10,13 +10,14 @@
 //   S5 estimation term    each c in E adds n_c e^{s} / e^{s} Vsum_c
 //   S6 merge              log-sum-exp over the split partials
 //
-// The CS blocks of a cluster share one unit.  Block b owns a contiguous,
-// balanced range of the unit's 128-centroid tiles; the blocks exchange data
-// only through distributed shared memory and the cluster barrier, never
-// through global counters, so no block waits on another cluster.  Data a
-// block needs from the others is pushed into its shared memory before the
-// barrier that publishes it wherever possible (a remote load costs a round
-// trip after the barrier; a remote store does not).
+// The CS blocks of a cluster share one unit.  Block b owns the unit's
+// 128-centroid tiles b, b + CS, b + 2 CS, ... (dealt round-robin, so the
+// blocks' shares differ by at most one tile); the blocks exchange data only
+// through distributed shared memory and the cluster barrier, never through
+// global counters, so no block waits on another cluster.  Data a block
+// needs from the others is pushed into its shared memory before the barrier
+// that publishes it wherever possible (a remote load costs a round trip
+// after the barrier; a remote store does not).
 //   A) Scoring: TMA brings the block's centroid tiles (128-byte swizzle, a
 //      ring of 4 stages) and the unit's query rows once; one thread issues
 //      tcgen05.mma (M = 128 centroids, N = 16 query rows, K = 128), each tile
@@ -37,20 +38,25 @@
 //      row, token prefix) and E clusters (id, size) in id order and pushes
 //      its totals (barrier 4).  Rows of clusters certain to be selected are
 //      prefetched into L2 as soon as the boundary groups are known.
-//   C) Attention: the unit's items (steady tokens, R tokens, E clusters) are
-//      split evenly over the blocks and, inside a block, over its sixteen
-//      warps.  A planner warp turns the block's token range into row runs
-//      (from the owners' lists); every warp then streams its items through
-//      its own ring of shared-memory slots with 16-byte cp.async copies, six
-//      steps ahead, and folds them into an online-softmax state on CUDA
-//      cores, half a warp per item (16 lanes x 8 dims, warp-shuffle
-//      reductions for q.k).  A token adds e^{x} v after its logit x; an E
-//      cluster adds n_c e^{s} to the denominator and e^{s} Vsum_c to the
-//      numerator.
+//   C) Attention: each block attends over the clusters it scored (its own
+//      R and E lists) and an even share of the steady tokens.  Warps 0-7
+//      take the token rows in windows: 16-row K and V tiles copied with
+//      16-byte cp.async into an XOR-swizzled layout, S = Q K^T and
+//      O^T += V^T P^T on mma.sync.m16n8k16 bf16 tiles (ldmatrix /
+//      ldmatrix.trans, the query rows padded to 16).  Warps 8-15 fold the E
+//      clusters on CUDA cores in fp32 (lane = head x dim group), each warp
+//      streaming value sums and scores through its own ring of slots.  Both
+//      keep an online softmax in log2 units, rescaled only when the maximum
+//      grows by more than e^8.  After a separate select call, the attend
+//      call rebuilds the same lists by the same tile ownership, so both
+//      paths fold the same items in the same order.
 //   D) Merge: the block's warps are combined in shared memory, every block
 //      writes its partial (max, denominator, numerator) into block 0's
 //      shared memory (barriers 5 and 6) and block 0 merges them by
 //      log-sum-exp into out and lse.
+// A growing index (index maintenance during decode) is read through
+// separate per-unit strides: Cs clusters and Ms rows, of which the first C
+// clusters are live.
 // Every wait on an mbarrier is bounded; on expiry the block records
 // RI_ERR_TIMEOUT in the status word, stops issuing work, lets the copies it
 // issued land and still takes part in every cluster barrier.
@@ -1319,17 +1325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- the window's token rows (R rows >= 0, steady rows as -1 - row),
       // written by the 256 threads of the token warps from the local lists
       const int nwt = (int)min((long long)kWindowTokens, ntok - wt);
+      // one token per thread: a steady token, or R token j found in its
+      // cluster by a binary search over the R list's token prefix
       for (int t = tt; t < nwt; t += kTokenWarps * 32) {
         const long long bt = wt + t;
-        if (bt < ns) rowtab[t] = -1 - (st0 + (int)bt);
-      }
-      {
-        const long long j0 = max(0ll, wt - ns), j1 = wt + nwt - ns;  // R tokens of the window
-        for (int i = tt; i < nR && j0 < j1; i += kTokenWarps * 32) {
-          const int2 e = lists[i];
-          const int cnt = (i + 1 < nR ? lists[i + 1].y : tokR) - e.y;
-          const long long lo = max(j0, (long long)e.y), hi = min(j1, (long long)e.y + cnt);
-          for (long long j = lo; j < hi; ++j) rowtab[(int)(j + ns - wt)] = e.x + (int)(j - e.y);
+        if (bt < ns) {
+          rowtab[t] = -1 - (st0 + (int)bt);
+        } else {
+          const int j = (int)(bt - ns);
+          int lo = 0, hi = nR - 1;  // last entry with prefix <= j
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (lists[mid].y <= j) lo = mid; else hi = mid - 1;
+          }
+          const int2 e = lists[lo];
+          rowtab[t] = e.x + (j - e.y);
         }
       }
       token_bar();
@@ -1478,25 +1488,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e0 = nE * ew / kEWarps, e1 = nE * (ew + 1) / kEWarps;
     const int2* elist = lists + nR;
     uint8_t* ering = sm + kOffMeta + ew * kEWarpBytes;
-    auto issue = [&](int e) {
-      if (e < e1) {
-        const int2 ev = elist[e];
-        if (ev.y > 0) {
-          uint8_t* slot = ering + (uint32_t)(e % kESlots) * kSlotE;
-          const size_t uc = (size_t)u * Cs + ev.x;
-          cp_async16(slot + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
-          if (lane < Gp / 4) cp_async16(slot + 512 + lane * 16, p.score + uc * Gp + lane * 4);
+    // items in pairs (two independent chains per step); kPairs pairs of
+    // slots in flight
+    constexpr int kPairs = kESlots / 2;
+    auto issue = [&](int e, int pair) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (e + k < e1) {
+          const int2 ev = elist[e + k];
+          if (ev.y > 0) {
+            uint8_t* slot = ering + (uint32_t)(2 * pair + k) * kSlotE;
+            const size_t uc = (size_t)u * Cs + ev.x;
+            cp_async16(slot + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
+            if (lane < Gp / 4) cp_async16(slot + 512 + lane * 16, p.score + uc * Gp + lane * 4);
+          }
         }
       }
       cp_async_commit();
     };
-    for (int k = 0; k < kESlots - 1; ++k) issue(e0 + k);
+    for (int k = 0; k < kPairs - 1; ++k) issue(e0 + 2 * k, k);
 #ifdef RI_DEBUG_PHASES
     long long cyc_w = 0, cyc_c = 0, cyc_t = clock64();
 #endif
-    for (int e = e0; e < e1; ++e) {
-      issue(e + kESlots - 1);
-      cp_async_wait<kESlots - 1>();
+    int pr = 0;  // ring pair of item e
+    for (int e = e0; e < e1; e += 2) {
+      issue(e + 2 * (kPairs - 1), pr == 0 ? kPairs - 1 : pr - 1);
+      cp_async_wait<kPairs - 1>();
       __syncwarp();
 #ifdef RI_DEBUG_PHASES
       {
@@ -1505,29 +1522,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         cyc_t = n_;
       }
 #endif
-      const int2 ev = elist[e];
-      if (ev.y > 0 && live) {
-        const uint8_t* slot = ering + (uint32_t)(e % kESlots) * kSlotE;
-        const float x = reinterpret_cast<const float*>(slot + 512)[g] * kLog2e;
-        if (x > em + kRescale2) {  // new reference (also the first cluster)
-          const float c = em == -INFINITY ? 0.f : ex2f(em - x);
-          el *= c;
+      const int2 ea = elist[e];
+      const int2 eb = e + 1 < e1 ? elist[e + 1] : make_int2(0, 0);
+      const bool va = ea.y > 0 && live, vb = eb.y > 0 && live;
+      const uint8_t* sa = ering + (uint32_t)(2 * pr) * kSlotE;
+      const uint8_t* sb = sa + kSlotE;
+      const float xa = va ? reinterpret_cast<const float*>(sa + 512)[g] * kLog2e : -INFINITY;
+      const float xb = vb ? reinterpret_cast<const float*>(sb + 512)[g] * kLog2e : -INFINITY;
+      const float xm = fmaxf(xa, xb);
+      if (xm > em + kRescale2) {  // new reference (also the first cluster)
+        const float c = em == -INFINITY ? 0.f : ex2f(em - xm);
+        el *= c;
 #pragma unroll
-          for (int i = 0; i < kDims; ++i) eo[i] *= c;
-          em = x;
-        }
-        const float w = ex2f(x - em);
-        el = fmaf((float)ev.y, w, el);
-        const float4* vr = reinterpret_cast<const float4*>(slot) + dg * GP;
-#pragma unroll
-        for (int i = 0; i < GP; ++i) {
-          const float4 v = vr[i];
-          eo[4 * i] = fmaf(w, v.x, eo[4 * i]);
-          eo[4 * i + 1] = fmaf(w, v.y, eo[4 * i + 1]);
-          eo[4 * i + 2] = fmaf(w, v.z, eo[4 * i + 2]);
-          eo[4 * i + 3] = fmaf(w, v.w, eo[4 * i + 3]);
-        }
+        for (int i = 0; i < kDims; ++i) eo[i] *= c;
+        em = xm;
       }
+      const float wa = va ? ex2f(xa - em) : 0.f, wb = vb ? ex2f(xb - em) : 0.f;
+      el = fmaf((float)eb.y, wb, fmaf((float)ea.y, wa, el));
+      const float4* ra = reinterpret_cast<const float4*>(sa) + dg * GP;
+      const float4* rb = reinterpret_cast<const float4*>(sb) + dg * GP;
+#pragma unroll
+      for (int i = 0; i < GP; ++i) {
+        const float4 a4 = va ? ra[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b4 = vb ? rb[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        eo[4 * i] = fmaf(wb, b4.x, fmaf(wa, a4.x, eo[4 * i]));
+        eo[4 * i + 1] = fmaf(wb, b4.y, fmaf(wa, a4.y, eo[4 * i + 1]));
+        eo[4 * i + 2] = fmaf(wb, b4.z, fmaf(wa, a4.z, eo[4 * i + 2]));
+        eo[4 * i + 3] = fmaf(wb, b4.w, fmaf(wa, a4.w, eo[4 * i + 3]));
+      }
+      pr = pr + 1 == kPairs ? 0 : pr + 1;
       __syncwarp();
 #ifdef RI_DEBUG_PHASES
       {

@@ -638,9 +638,11 @@ def _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode):
             stage_d[0, :nf].copy_(stage[0, :nf], non_blocking=True)
             stage_d[1, :na].copy_(stage[1, :na], non_blocking=True)
             e0.record(stream)
-            R.gather_blocks(stage_d[0, :nf], hK, hV, eK, eV, gws, cK, cV)
+            R.gather_blocks(stage_d[0, :nf], hK, hV, eK, eV, gws, cK, cV,
+                            shape=R.gather_shape(int((fetch[:, 1] == R.SRC_HOST).sum()), nf))
             e1.record(stream)
-            R.gather_blocks(stage_d[1, :na], hK, hV, eK, eV, gws, cK, cV)
+            R.gather_blocks(stage_d[1, :na], hK, hV, eK, eV, gws, cK, cV,
+                            shape=R.gather_shape(0, na))
         else:
             s0 = time.perf_counter()
             worker.wait()            # the previous update, normally already applied
@@ -649,7 +651,8 @@ def _cfg5_mode(R, dev, local, idx, d, hK, hV, counts, offsets, qs, warm, mode):
             s2 = time.perf_counter()
             fd = worker.fetch_to_device(stream)
             e0.record(stream)
-            R.gather_blocks(fd, hK, hV, eK, eV, gws, cK, cV)
+            R.gather_blocks(fd, hK, hV, eK, eV, gws, cK, cV,
+                            shape=R.gather_shape(int((fl[:, 1] == R.SRC_HOST).sum()), len(fl)))
             e1.record(stream)
             s3 = time.perf_counter()
             worker.update_async(stream)
@@ -867,6 +870,69 @@ def run_profile_case(which):
     print(f"profile case {which} done", flush=True)
 
 
+def run_gather_shapes():
+    """Launch-shape sweep of the gather kernel (threads per block x blocks per
+    SM) for four copy lists on the 1M-context geometry (8 units): 16-row
+    copies from pinned host memory (cache misses), 16-row copies of which 2 %
+    are misses (the host-memory workload's usual mix), and 8-row and 16-row
+    copies from the device block pool (cache hits).  CUDA events, median of
+    5."""
+    import kv_cache_vector_segmented_b200 as R
+    dev = torch.device("cuda", 0)
+    U, M, POOL, EXE = 8, 131072, 65536, 65536
+    g = torch.Generator()
+    g.manual_seed(9)
+    hK = torch.randn((1, U, M, 128), generator=g).to(torch.bfloat16).pin_memory()
+    hV = torch.randn((1, U, M, 128), generator=g).to(torch.bfloat16).pin_memory()
+    cK = torch.randn((1, U, POOL, 128), device=dev).to(torch.bfloat16)
+    cV = torch.randn_like(cK)
+    eK = torch.empty((1, U, EXE, 128), dtype=torch.bfloat16, device=dev)
+    eV = torch.empty_like(eK)
+    ws = R.alloc_workspace(256, dev)
+    rng = np.random.default_rng(0)
+
+    def copy_list(host_frac, n_per_unit, rows):
+        out = []
+        for u in range(U):
+            dst = rng.permutation(EXE // rows)[:n_per_unit] * rows
+            hsrc = rng.integers(0, M - rows, n_per_unit)
+            csrc = rng.permutation(POOL // rows)[:n_per_unit] * rows
+            host = rng.random(n_per_unit) < host_frac
+            out += [(u, R.SRC_HOST if h else R.SRC_CACHE, int(a if h else c), R.DST_EXEC, int(b),
+                     rows) for h, a, c, b in zip(host, hsrc, csrc, dst)]
+        return torch.tensor(out, dtype=torch.int32, device=dev)
+
+    lists = {"host_16rows": copy_list(1.0, 400, 16),
+             "mixed_16rows_2pct_host": copy_list(0.02, 2000, 16),
+             "device_8rows": copy_list(0.0, 4000, 8),
+             "device_16rows": copy_list(0.0, 2000, 16)}
+    res = {}
+    for name, d in lists.items():
+        row = {}
+        for threads in (64, 128, 256, 512):
+            for bps in (1, 2, 4, 8, 16, 32):
+                if threads * bps > 2048:
+                    continue
+                for _ in range(2):
+                    R.gather_blocks(d, hK, hV, eK, eV, ws, cK, cV, shape=(threads, bps))
+                ts = []
+                for _ in range(5):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    R.gather_blocks(d, hK, hV, eK, eV, ws, cK, cV, shape=(threads, bps))
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1) * 1e3)
+                row[f"{threads}x{bps}"] = round(float(np.median(ts)), 1)
+        host = int(d[:, 1].eq(R.SRC_HOST).sum().item())
+        chosen = R.gather_shape(host, d.shape[0])
+        res[name] = {"copies": int(d.shape[0]), "us_by_threads_x_blocks_per_sm": row,
+                     "best": min(row, key=row.get), "chosen": f"{chosen[0]}x{chosen[1]}"}
+    assert R.read_device_status(ws) == 0
+    return {"leg": "gather launch shapes", "unit": "us per launch", "lists": res}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -878,9 +944,14 @@ def main():
                     help="skip the config1 / config4 / config5 legs")
     ap.add_argument("--ncu-case", choices=["decode", "gather"], default=None,
                     help="run only the small case used for ncu captures")
+    ap.add_argument("--gather-shapes", action="store_true",
+                    help="run only the launch-shape sweep of the gather kernel")
     args = ap.parse_args()
     if args.ncu_case:
         run_profile_case(args.ncu_case)
+        return
+    if args.gather_shapes:
+        print(json.dumps(run_gather_shapes()), flush=True)
         return
     if args.warmup < 3:
         args.warmup = 3

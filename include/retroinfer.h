@@ -512,6 +512,21 @@ ri_status ri_cache_worker_wait(ri_cache_worker* worker, ri_cache_stats* stats, i
 ri_status ri_cache_worker_test_hooks(ri_cache_worker* worker, int64_t fail_update,
                                      int64_t fail_after_admissions, uint32_t delay_us);
 
+/* ri_gather_blocks with the launch shape given: threads per block (0, or a
+ * multiple of 32 in [32, 512]; one warp per copy) and the most blocks per SM
+ * the grid may hold (0..64; 0 = default).  [P2 §3.2: the copy kernel adapts
+ * its thread-block size to the cache-hit pattern.] */
+ri_status ri_gather_blocks_shaped(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
+                                  int32_t n_desc, int32_t threads, int32_t blocks_per_sm,
+                                  void* workspace, ri_stream_t stream);
+
+/* The launch shape for a copy list of total_copies copies of which
+ * host_copies read pinned host memory (cache misses): lists with host
+ * copies get the most warps in flight, device-only lists fewer, larger
+ * blocks (the shapes measured best for each on B200).  Host only. */
+ri_status ri_gather_shape(int64_t host_copies, int64_t total_copies, int32_t* threads,
+                          int32_t* blocks_per_sm);
+
 /* Synchronises `stream` and returns the status word previous calls wrote
  * into `workspace` (RI_OK if no device-side failure was recorded); a failure
  * read is cleared, so the next read reports only later failures. */

@@ -18,7 +18,8 @@ _EXPORTS = (
     "STATIC_SCRATCH_BYTES", "BlockCache", "CopyDesc", "gather_blocks", "SRC_HOST", "SRC_CACHE",
     "SRC_EXEC", "DST_EXEC", "DST_CACHE", "max_retrieval_rows", "selftest_decode_timeout",
     "FAULT_SCORE_COPY", "FAULT_SCORE_COMMIT", "FAULT_SCORE_SIZES", "CacheWorker",
-    "Decoder", "index_open", "index_append", "index_append_workspace_bytes")
+    "Decoder", "index_open", "index_append", "index_append_workspace_bytes",
+    "gather_shape")
 
 __all__ = list(_EXPORTS)
 

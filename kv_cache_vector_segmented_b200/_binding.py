@@ -164,6 +164,12 @@ lib.ri_max_retrieval_rows.restype = ctypes.c_int
 lib.ri_max_retrieval_rows.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
 lib.ri_gather_blocks.restype = ctypes.c_int
 lib.ri_gather_blocks.argtypes = [_P(GatherBuffers), _vp, ctypes.c_int32, _vp, _vp]
+lib.ri_gather_blocks_shaped.restype = ctypes.c_int
+lib.ri_gather_blocks_shaped.argtypes = [_P(GatherBuffers), _vp, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, _vp, _vp]
+lib.ri_gather_shape.restype = ctypes.c_int
+lib.ri_gather_shape.argtypes = [ctypes.c_int64, ctypes.c_int64, _P(ctypes.c_int32),
+                                _P(ctypes.c_int32)]
 lib.ri_cache_resident.restype = ctypes.c_int
 lib.ri_cache_resident.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, ctypes.c_int32,
                                   _P(ctypes.c_int32)]
@@ -820,10 +826,18 @@ def max_retrieval_rows(counts: np.ndarray, k_retrieval: int) -> np.ndarray:
     return out
 
 
+def gather_shape(host_copies: int, total_copies: int) -> tuple:
+    """ri_gather_shape: (threads per block, blocks per SM) for a copy list."""
+    t, b = ctypes.c_int32(0), ctypes.c_int32(0)
+    check(lib.ri_gather_shape(host_copies, total_copies, ctypes.byref(t), ctypes.byref(b)),
+          "ri_gather_shape")
+    return t.value, b.value
+
+
 def gather_blocks(desc: torch.Tensor, host_K: torch.Tensor, host_V: torch.Tensor,
                   exec_K: torch.Tensor, exec_V: torch.Tensor, workspace: torch.Tensor,
                   cache_K: Optional[torch.Tensor] = None,
-                  cache_V: Optional[torch.Tensor] = None) -> None:
+                  cache_V: Optional[torch.Tensor] = None, shape: Optional[tuple] = None) -> None:
     """ri_gather_blocks: desc int32 [n][6] on the device; host_K/V pinned CPU
     bf16 [B][H][M][d]; exec_K/V device bf16 [B][H][rows][d]; cache_K/V device
     bf16 [B][H][pool_rows][d] or None."""
@@ -841,6 +855,7 @@ def gather_blocks(desc: torch.Tensor, host_K: torch.Tensor, host_V: torch.Tensor
         _need(cache_V, "cache_V", torch.bfloat16, (B, H, pool, d), dev)
     bufs = GatherBuffers(host_K.data_ptr(), host_V.data_ptr(), _ptr(cache_K), _ptr(cache_V),
                          exec_K.data_ptr(), exec_V.data_ptr(), B * H, M, pool, rows)
-    check(lib.ri_gather_blocks(ctypes.byref(bufs), desc.data_ptr(), desc.shape[0],
-                               workspace.data_ptr(), _stream(dev)),
-          "ri_gather_blocks")
+    threads, bps = shape if shape is not None else (0, 0)
+    check(lib.ri_gather_blocks_shaped(ctypes.byref(bufs), desc.data_ptr(), desc.shape[0],
+                                      threads, bps, workspace.data_ptr(), _stream(dev)),
+          "ri_gather_blocks_shaped")

@@ -592,6 +592,36 @@ ri_status ri_attend_selected(const ri_index_config* cfg, const ri_decode_config*
 
 ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
                            int32_t n_desc, void* workspace, ri_stream_t stream) {
+  return ri_gather_blocks_shaped(bufs, desc, n_desc, 0, 0, workspace, stream);
+}
+
+ri_status ri_gather_shape(int64_t host_copies, int64_t total_copies, int32_t* threads,
+                          int32_t* blocks_per_sm) {
+  RI_CHECK(threads && blocks_per_sm, RI_ERR_INVALID_ARG, "gather shape: NULL output");
+  RI_CHECK(host_copies >= 0 && total_copies >= host_copies, RI_ERR_INVALID_ARG,
+           "gather shape: bad copy counts (%lld host of %lld)", (long long)host_copies,
+           (long long)total_copies);
+  // a list with any copy from host memory waits on the host link: the most
+  // warps in flight (2048 threads per SM) keep the device copies from
+  // queueing behind the slow ones; lists served from the device's own
+  // memory stream at fewer, larger blocks
+  if (host_copies > 0) {
+    *threads = kGatherHostThreads;
+    *blocks_per_sm = kGatherHostBlocksPerSM;
+  } else {
+    *threads = kGatherDeviceThreads;
+    *blocks_per_sm = kGatherDeviceBlocksPerSM;
+  }
+  return RI_OK;
+}
+
+ri_status ri_gather_blocks_shaped(const ri_gather_buffers* bufs, const ri_copy_desc* desc,
+                                  int32_t n_desc, int32_t threads, int32_t blocks_per_sm,
+                                  void* workspace, ri_stream_t stream) {
+  RI_CHECK(threads == 0 || (threads >= 32 && threads <= 512 && threads % 32 == 0),
+           RI_ERR_INVALID_ARG, "threads per block must be 0 or a multiple of 32 in [32, 512]");
+  RI_CHECK(blocks_per_sm >= 0 && blocks_per_sm <= 64, RI_ERR_INVALID_ARG,
+           "blocks per SM must be in [0, 64]");
   RI_CHECK(n_desc >= 0, RI_ERR_INVALID_ARG, "n_desc must be >= 0");
   RI_CHECK(n_desc == 0 || desc, RI_ERR_INVALID_ARG, "descriptors are NULL");
   RI_CHECK(workspace && aligned16(workspace), RI_ERR_INVALID_ARG,
@@ -612,7 +642,7 @@ ri_status ri_gather_blocks(const ri_gather_buffers* bufs, const ri_copy_desc* de
   a.M = bufs->M;
   a.pool_rows = bufs->pool_rows;
   a.exec_rows = bufs->exec_rows;
-  e = launch_gather(a, desc, n_desc, static_cast<int*>(workspace), s);
+  e = launch_gather(a, desc, n_desc, static_cast<int*>(workspace), s, threads, blocks_per_sm);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   return RI_OK;
 }

@@ -847,7 +847,7 @@ void run_update(ri_cache_worker* w, long long seq) {
       a.pool_rows = b.pool_rows;
       a.exec_rows = b.exec_rows;
       e = ri::launch_gather(a, w->cfg.admit_dev, nao, static_cast<int*>(w->cfg.gather_workspace),
-                            side);
+                            side, ri::kGatherDeviceThreads, ri::kGatherDeviceBlocksPerSM);
     }
     if (e == cudaSuccess) e = cudaEventRecord(w->ev_admit, side);
     if (e == cudaSuccess) {

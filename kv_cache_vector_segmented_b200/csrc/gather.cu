@@ -13,14 +13,15 @@ namespace ri {
 
 namespace {
 
-constexpr int kGatherThreads = 256;
+constexpr int kMaxGatherThreads = 512;
 constexpr int kMaxRows = 16;  // rows per descriptor (the plan's chunk size)
 
-__global__ void __launch_bounds__(kGatherThreads)
+__global__ void __launch_bounds__(kMaxGatherThreads)
     gather_kernel(GatherArgs a, const ri_copy_desc* __restrict__ desc, int n_desc, int* status) {
   const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (kGatherThreads / 32);
-  for (int w = blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); w < n_desc; w += warps) {
+  const int wpb = blockDim.x >> 5;  // warps per block (the launch shape)
+  const int warps = gridDim.x * wpb;
+  for (int w = blockIdx.x * wpb + (threadIdx.x >> 5); w < n_desc; w += warps) {
     const ri_copy_desc d = desc[w];
     const bool v_half = lane >= 16;
     const int chunk = lane & 15;
@@ -76,13 +77,15 @@ __global__ void __launch_bounds__(kGatherThreads)
 }  // namespace
 
 cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_desc, int* status,
-                          cudaStream_t s) {
+                          cudaStream_t s, int threads, int blocks_per_sm) {
   if (n_desc <= 0) return cudaSuccess;
-  const int per_block = kGatherThreads / 32;
+  if (threads <= 0) threads = kGatherDefaultThreads;
+  if (blocks_per_sm <= 0) blocks_per_sm = kGatherDefaultBlocksPerSM;
+  const int per_block = threads / 32;
   int blocks = (n_desc + per_block - 1) / per_block;
-  const int cap = 8 * num_sms();
+  const int cap = blocks_per_sm * num_sms();
   if (blocks > cap) blocks = cap;
-  gather_kernel<<<blocks, kGatherThreads, 0, s>>>(a, desc, n_desc, status);
+  gather_kernel<<<blocks, threads, 0, s>>>(a, desc, n_desc, status);
   return cudaGetLastError();
 }
 

@@ -126,8 +126,17 @@ struct GatherArgs {
   void* exec_V;
   int units, M, pool_rows, exec_rows;
 };
+// Launch shape of the gather: threads per block (a multiple of 32, at most
+// 512) and the most blocks per SM the grid may hold; 0 picks the defaults.
+constexpr int kGatherDefaultThreads = 256;
+constexpr int kGatherDefaultBlocksPerSM = 8;
+// shapes ri_gather_shape picks per hit pattern (from a sweep on B200: lists
+// with host copies want the most warps in flight, device-only lists need
+// about 1024 threads per SM and are flat beyond)
+constexpr int kGatherHostThreads = 256, kGatherHostBlocksPerSM = 8;
+constexpr int kGatherDeviceThreads = 512, kGatherDeviceBlocksPerSM = 1;
 cudaError_t launch_gather(const GatherArgs& a, const ri_copy_desc* desc, int n_desc, int* status,
-                          cudaStream_t s);
+                          cudaStream_t s, int threads = 0, int blocks_per_sm = 0);
 // Argument checks of ri_gather_buffers (pointers, alignment, sizes).
 ri_status check_gather_buffers(const ri_gather_buffers* bufs);
 

@@ -200,3 +200,23 @@ def test_growing_calls_reject_bad_arguments(R):
     st = R.lib.ri_index_open(ctypes.byref(later), ctypes.byref(idx), ctypes.byref(idx), None)
     assert st == R.STATUS_CODES["RI_ERR_INVALID_ARG"]
     assert torch  # noqa
+
+
+def test_gather_shape_per_hit_pattern(R):
+    """Host-link bound lists and device-memory bound lists get their own
+    launch shapes; bad counts are refused on the host."""
+    host = R.gather_shape(20, 1000)      # any copy from host memory
+    dev = R.gather_shape(0, 1000)        # device-only list
+    assert host != dev and R.gather_shape(1000, 1000) == host
+    for t, b in (host, dev):
+        assert t % 32 == 0 and 32 <= t <= 512 and 1 <= b <= 64
+    assert R.gather_shape(0, 0) == dev
+    with pytest.raises(R.RIError):
+        R.gather_shape(5, 4)
+    with pytest.raises(R.RIError):
+        R.gather_shape(-1, 4)
+    bufs = R._binding.GatherBuffers()
+    assert R.lib.ri_gather_blocks_shaped(ctypes.byref(bufs), None, 0, 48, 4, None, None) == \
+        R.STATUS_CODES["RI_ERR_INVALID_ARG"]           # not a multiple of 32
+    assert R.lib.ri_gather_blocks_shaped(ctypes.byref(bufs), None, 0, 1024, 4, None, None) == \
+        R.STATUS_CODES["RI_ERR_INVALID_ARG"]           # above 512

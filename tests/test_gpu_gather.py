@@ -66,8 +66,14 @@ def test_gather_access_path(R, cache_frac):
             assert st["empty_clusters"] == int((counts[np.arange(B * H)[:, None],
                                                        np.maximum(sel_h[:, :k_r], 0)] == 0).sum())
         hits_seen += st["hit_rows"]
+        # every launch shape copies the same bytes: rotate through a few, and
+        # the one the chooser picks for the list's hit pattern
+        shapes = [None, (32, 1), (64, 16), (512, 1), (128, 8), None]
         for plan in (fetch, admit):  # fetch first, then admission into the pool
-            R.gather_blocks(torch.from_numpy(plan).to(dev), hK, hV, eK, eV, gws, cK, cV)
+            shape = shapes[step % len(shapes)] or R.gather_shape(
+                int((plan[:, 1] == R.SRC_HOST).sum()), len(plan))
+            R.gather_blocks(torch.from_numpy(plan).to(dev), hK, hV, eK, eV, gws, cK, cV,
+                            shape=shape)
         torch.cuda.synchronize()
         assert R.read_device_status(gws) == 0
         rr_h = rr.cpu().numpy().reshape(B * H, -1)

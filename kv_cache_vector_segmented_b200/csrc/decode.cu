@@ -1472,9 +1472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
   } else {
     // ---- estimation clusters: the block's E list split over the E warps.
-    // Lane (head g, dim group dg): GP = G rounded up to a power of two, 32 /
-    // GP lanes per head, each with 4 GP consecutive dims, so a lane follows
-    // one head alone (no shuffles).  Each warp streams its clusters' value
+    // Lane (head g, dim group dg): GP = G rounded up to a power of two,
+    // LPH = 32 / GP lanes per head; the lane holds the GP float4 groups of
+    // dims with group index i LPH + dg (i < GP), so the lanes of a head read
+    // consecutive 16-byte groups (no bank conflicts) and a lane follows one
+    // head alone (no shuffles).  Each warp streams its clusters' value
     // sums and scores through its own ring of slots in shared memory with
     // 16-byte cp.async copies, kEAhead clusters ahead.
     constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
@@ -1489,18 +1491,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int2* elist = lists + nR;
     uint8_t* ering = sm + kOffMeta + ew * kEWarpBytes;
     // items in pairs (two independent chains per step); kPairs pairs of
-    // slots in flight
+    // slots in flight.  The unit's value-sum and score rows and this lane's
+    // part of them are fixed for the loop: taken once, as plain pointers.
     constexpr int kPairs = kESlots / 2;
+    const float* vs_lane = p.vsum + (size_t)u * Cs * kHeadDim + lane * 4;
+    const float* sc_lane = p.score + (size_t)u * Cs * Gp + lane * 4;
+    const uint32_t ering_lane = smem_u32(ering) + lane * 16;
+    const bool sc_lane_on = lane < Gp / 4;
     auto issue = [&](int e, int pair) {
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         if (e + k < e1) {
           const int2 ev = elist[e + k];
           if (ev.y > 0) {
-            uint8_t* slot = ering + (uint32_t)(2 * pair + k) * kSlotE;
-            const size_t uc = (size_t)u * Cs + ev.x;
-            cp_async16(slot + lane * 16, p.vsum + uc * kHeadDim + lane * 4);
-            if (lane < Gp / 4) cp_async16(slot + 512 + lane * 16, p.score + uc * Gp + lane * 4);
+            const uint32_t slot = ering_lane + (uint32_t)(2 * pair + k) * kSlotE;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(slot),
+                         "l"(vs_lane + (size_t)ev.x * kHeadDim)
+                         : "memory");
+            if (sc_lane_on)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(slot + 512u),
+                           "l"(sc_lane + (size_t)ev.x * Gp)
+                           : "memory");
           }
         }
       }
@@ -1511,6 +1522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long cyc_w = 0, cyc_c = 0, cyc_t = clock64();
 #endif
     int pr = 0;  // ring pair of item e
+#pragma unroll 1
     for (int e = e0; e < e1; e += 2) {
       issue(e + 2 * (kPairs - 1), pr == 0 ? kPairs - 1 : pr - 1);
       cp_async_wait<kPairs - 1>();
@@ -1539,12 +1551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float wa = va ? ex2f(xa - em) : 0.f, wb = vb ? ex2f(xb - em) : 0.f;
       el = fmaf((float)eb.y, wb, fmaf((float)ea.y, wa, el));
-      const float4* ra = reinterpret_cast<const float4*>(sa) + dg * GP;
-      const float4* rb = reinterpret_cast<const float4*>(sb) + dg * GP;
+      const float4* ra = reinterpret_cast<const float4*>(sa) + dg;
+      const float4* rb = reinterpret_cast<const float4*>(sb) + dg;
 #pragma unroll
       for (int i = 0; i < GP; ++i) {
-        const float4 a4 = va ? ra[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 b4 = vb ? rb[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 a4 = va ? ra[i * (32 / GP)] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b4 = vb ? rb[i * (32 / GP)] : make_float4(0.f, 0.f, 0.f, 0.f);
         eo[4 * i] = fmaf(wb, b4.x, fmaf(wa, a4.x, eo[4 * i]));
         eo[4 * i + 1] = fmaf(wb, b4.y, fmaf(wa, a4.y, eo[4 * i + 1]));
         eo[4 * i + 2] = fmaf(wb, b4.z, fmaf(wa, a4.z, eo[4 * i + 2]));
@@ -1569,10 +1581,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     RI_STAMP(24, kTokenWarps * 32);
     __syncthreads();  // every warp done with step C: the ring is free
     if (live) {
-      float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim + dg * kDims);
+      float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim) + dg;
 #pragma unroll
       for (int i = 0; i < GP; ++i)
-        dst[i] = make_float4(eo[4 * i], eo[4 * i + 1], eo[4 * i + 2], eo[4 * i + 3]);
+        dst[i * (32 / GP)] = make_float4(eo[4 * i], eo[4 * i + 1], eo[4 * i + 2], eo[4 * i + 3]);
       if (dg == 0) {
         ms->wm[warp][g] = em;
         ms->wl[warp][g] = el;

@@ -35,9 +35,9 @@
 //      every block when there are few of them (barrier 3), else found by a
 //      radix walk over the 32-bit order key and a final id count (crowded
 //      buckets, heavy ties).  Each block lists its own R clusters (first
-//      row, token prefix) and E clusters (id, size) in id order and pushes
-//      its totals (barrier 4).  Rows of clusters certain to be selected are
-//      prefetched into L2 as soon as the boundary groups are known.
+//      row, token prefix) and E clusters (id, size) in id order; when the
+//      selection is written out, every block pushes its per-tile counts
+//      (barrier 4) and places its ids by the prefixes over all tiles.
 //   C) Attention: each block attends over the clusters it scored (its own
 //      R and E lists) and an even share of the steady tokens.  Warps 0-7
 //      take the token rows in windows: 16-row K and V tiles copied with
@@ -858,31 +858,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (v.y) atomicAdd(&ms->fine[w][4 * j + 1], v.y);
           if (v.z) atomicAdd(&ms->fine[w][4 * j + 2], v.z);
           if (v.w) atomicAdd(&ms->fine[w][4 * j + 3], v.w);
-        }
-      }
-      if (p.mode == kModeFull) {
-        // clusters certain to be selected whatever the exact order inside the
-        // boundary groups: their rows (R) and value sums (E) start moving
-        // into L2 while the selection finishes
-        const int gA = ms->digit[0], gB = ms->digit[1];
-        const bool finA = onA && kA <= nfin, infA = onA && kA > nfin;
-        const bool finB = onB && kB <= nfin, infB = onB && kB > nfin;
-        for (int i = tid; i < nid; i += kThreads) {
-          const float key = keys[i];
-          if (key == -INFINITY) continue;
-          const int g = bucket_of(key, lo, scale) >> 5;
-          const bool sureR = infA || (finA && g > gA);
-          const bool sureE = !sureR && ((finB && g > gB) || infB) && (!onA || (finA && g < gA));
-          if (sureR) {
-            const int2 mt = meta[i];
-            if (mt.y > 0 && mt.x >= 0 && (long long)mt.x + mt.y <= p.Ms) {
-              const size_t r0 = (size_t)u * p.Ms + mt.x;
-              prefetch_l2_bulk(p.Kr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
-              prefetch_l2_bulk(p.Vr + r0 * kHeadDim, (uint32_t)mt.y * 256u);
-            }
-          } else if (sureE) {
-            prefetch_l2_bulk(p.vsum + ((size_t)u * Cs + id_of(i)) * kHeadDim, 512u);
-          }
         }
       }
       __syncthreads();

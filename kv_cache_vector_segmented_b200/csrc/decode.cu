@@ -102,11 +102,11 @@ constexpr int kKPT = kMaxIdsPerBlock / kThreads;  // own ids per thread (contigu
 constexpr int kTokenWarps = 8;
 constexpr int kEWarps = kWarps - kTokenWarps;
 constexpr uint32_t kTokenWarpBytes = 16384;
-constexpr int kWindowTokens = 4096;
+constexpr int kWindowTokens = 1024;
 // estimation warps: rings of kESlots slots (value sum 512 B + scores 32 B)
-// in the size-and-row area of step A, free by then
+// in the size-and-row area of step A, free by then, and the area after it
 constexpr uint32_t kSlotE = 544;
-constexpr uint32_t kEWarpBytes = 4096;
+constexpr uint32_t kEWarpBytes = 6912;
 constexpr int kESlots = (int)(kEWarpBytes / kSlotE);
 
 // Shared memory map (byte offsets from a 1024-byte aligned base).
@@ -115,7 +115,9 @@ static_assert(kStagesA * kTileBytes == kRingBytes, "ring");
 constexpr uint32_t kOffQ = kRingBytes;                          // q tile (4 KB)
 constexpr uint32_t kOffKeys = kOffQ + kQBytes;                  // float keys[P], then lists
 constexpr uint32_t kOffMeta = kOffKeys + kMaxIdsPerBlock * 8;   // int2 (first row, size)[P]
-constexpr uint32_t kOffRuns = kOffMeta + kMaxIdsPerBlock * 8;   // int token rows[kWindowTokens]
+constexpr uint32_t kERingBytes = kEWarps * kEWarpBytes;  // from kOffMeta, step C
+static_assert(kERingBytes >= kMaxIdsPerBlock * 8, "estimation rings cover the meta area");
+constexpr uint32_t kOffRuns = kOffMeta + kERingBytes;          // int token rows[kWindowTokens]
 constexpr uint32_t kOffMisc = kOffRuns + kWindowTokens * 4;
 constexpr uint32_t kMiscBytes = 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + base alignment slack
@@ -205,7 +207,7 @@ struct Misc {
   unsigned long long thr[2];
   int gsum[kGroups];  // cluster-wide group counts
   int fine[2][32];    // cluster-wide bucket counts of the two boundary groups
-  int scan[kWarps + 4];
+  alignas(16) int scan[2 * kWarps];
   int T_R, nruns, wend_lo, wend_hi;
   float wm[kWarps][8], wl[kWarps][8];
 };
@@ -311,9 +313,12 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// Block-wide exclusive prefix of one int per thread (thread order); the
-// block total goes to *total.  One warp scans the per-warp totals.
-__device__ __noinline__ int block_scan(int v, int* scratch /* [kWarps + 1] */, int* total) {
+// Exclusive prefix sum over the block's threads (thread order) and the
+// total, with one barrier: each warp scans its lanes and publishes its total
+// in scratch[warp]; after the barrier every thread adds up the totals of the
+// warps before it.  The scratch array is read after the barrier, so the
+// caller separates two uses of one array by a barrier of its own.
+__device__ __forceinline__ int block_scan(int v, int* scratch /* [kWarps] */, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -323,22 +328,50 @@ __device__ __noinline__ int block_scan(int v, int* scratch /* [kWarps + 1] */, i
   }
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const int wt = lane < kWarps ? scratch[lane] : 0;
-    int wi = wt;
+  int before = 0, all = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += t;
-    }
-    if (lane < kWarps) scratch[lane] = wi - wt;
-    if (lane == 31) scratch[kWarps] = wi;
+  for (int w4 = 0; w4 < kWarps / 4; ++w4) {
+    const int4 t = reinterpret_cast<const int4*>(scratch)[w4];
+    before += (4 * w4 < warp ? t.x : 0) + (4 * w4 + 1 < warp ? t.y : 0) +
+              (4 * w4 + 2 < warp ? t.z : 0) + (4 * w4 + 3 < warp ? t.w : 0);
+    all += t.x + t.y + t.z + t.w;
   }
+  *total = all;
+  return before + incl - v;
+}
+
+// Two prefix sums at once (scratch [2 * kWarps]), one barrier.
+__device__ __forceinline__ int2 block_scan2(int a, int b, int* scratch, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int ta = __shfl_up_sync(0xffffffffu, ia, off);
+    const int tb = __shfl_up_sync(0xffffffffu, ib, off);
+    if (lane >= off) {
+      ia += ta;
+      ib += tb;
+    }
+  }
+  if (lane == 31) reinterpret_cast<int2*>(scratch)[warp] = make_int2(ia, ib);
   __syncthreads();
-  const int excl = scratch[warp] + incl - v;
-  *total = scratch[kWarps];
-  __syncthreads();  // scratch is reused by the next scan
-  return excl;
+  int2 before = make_int2(0, 0), all = make_int2(0, 0);
+#pragma unroll
+  for (int w2 = 0; w2 < kWarps / 2; ++w2) {
+    const int4 t = reinterpret_cast<const int4*>(scratch)[w2];  // warps 2 w2, 2 w2 + 1
+    if (2 * w2 < warp) {
+      before.x += t.x;
+      before.y += t.y;
+    }
+    if (2 * w2 + 1 < warp) {
+      before.x += t.z;
+      before.y += t.w;
+    }
+    all.x += t.x + t.z;
+    all.y += t.y + t.w;
+  }
+  *total = all;
+  return make_int2(before.x + ia - a, before.y + ib - b);
 }
 
 // OR of a predicate over the 128 threads of warps 4-7 (named barrier 1).
@@ -802,11 +835,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bk >= 0) atomicAdd(&hist[bk], 1);
     }
     __syncthreads();
+    RI_STAMP(26, 0);
     for (int g = warp; g < kGroups; g += kWarps) {
       const int v = __reduce_add_sync(0xffffffffu, hist[g * 32 + lane]);
       if (lane == 0) lgs[g] = v;
     }
     __syncthreads();
+    RI_STAMP(27, 0);
     if (tid < 32 * CS) {
       const int q = tid >> 5, j = tid & 31;  // target block, 16-byte piece
       const int4 v = reinterpret_cast<const int4*>(lgs)[j];
@@ -847,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
+      RI_STAMP(28, 0);
       // the two boundary groups' bucket counts, summed over the blocks
       if (tid < 2 * 8 * CS) {
         const int w = tid / (8 * CS), r = tid - w * 8 * CS;
@@ -861,6 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
+      RI_STAMP(29, 0);
       if (warp < 2 && ms->digit[warp] >= 0) {
         const int w = warp, g = ms->digit[w];
         const int k = w == 0 ? kA : kB;
@@ -986,6 +1023,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* tcl = ms->gsum;  // [32 own tiles][3], free after the boundary search
     for (int i = tid; i < 3 * kMaxTilesPerBlock; i += kThreads) tcl[i] = 0;
     __syncthreads();
+    RI_STAMP(30, 0);
     {
       // thread t takes kper consecutive local ids; kper is a power of two, so
       // no thread's ids straddle a tile
@@ -1032,9 +1070,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicAdd(&tcl[3 * lt + 1], __popc(mE));
         atomicAdd(&tcl[3 * lt + 2], tokr);
       }
-      int tot, ttot;
-      const int excl = block_scan((__popc(mR) << 16) | __popc(mE), ms->scan, &tot);
-      int texcl = block_scan(tokr, ms->scan, &ttot);
+      RI_STAMP(31, 0);
+      int2 tots;
+      const int2 exs = block_scan2((__popc(mR) << 16) | __popc(mE), tokr, ms->scan, &tots);
+      RI_STAMP(32, 0);
+      const int excl = exs.x, tot = tots.x, ttot = tots.y;
+      int texcl = exs.y;
       const int nR = tot >> 16, nE = tot & 0xFFFF;
       // keys are all in registers now: the lists take their place
       uint16_t* rid = reinterpret_cast<uint16_t*>(sm + kRRid);
@@ -1071,9 +1112,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       RI_STAMP(5, 0);
       const uint4* tc = reinterpret_cast<const uint4*>(sm + kRTcnt);
       const uint4 v = tid < p.tiles ? tc[tid] : make_uint4(0u, 0u, 0u, 0u);
-      int totRE, totT;
-      const int exRE = block_scan((int)((v.x << 16) | v.y), ms->scan, &totRE);
-      const int exT = block_scan((int)v.z, ms->scan, &totT);
+      int2 tots;
+      const int2 exs = block_scan2((int)((v.x << 16) | v.y), (int)v.z, ms->scan, &tots);
+      const int exRE = exs.x, exT = exs.y, totRE = tots.x, totT = tots.y;
       // tile prefixes into the tile-count area (only the own tiles are used)
       int4* tp = reinterpret_cast<int4*>(sm + kRTcnt);
       if (tid < p.tiles) tp[tid] = make_int4(exRE >> 16, exRE & 0xFFFF, exT, 0);
@@ -1205,9 +1246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (bad) record_status(p.status, RI_ERR_INVALID_ARG);
-      int tot, ttot;
-      const int ex = block_scan(__popc(mk), ms->scan, &tot);
-      int tex = block_scan(tok, ms->scan, &ttot);
+      int2 tots;
+      const int2 exs = block_scan2(__popc(mk), tok, ms->scan, &tots);
+      const int ex = exs.x, tot = tots.x, ttot = tots.y;
+      int tex = exs.y;
       int pos = ex;
 #pragma unroll
       for (int j = 0; j < kKPT; ++j)
@@ -1286,6 +1328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         qa[kk][0] = qa[kk][1] = 0u;
       }
     }
+    RI_STAMP(33, 0);
     const __nv_bfloat16* Kr = p.Kr + (size_t)u * lim_rows * kHeadDim;
     const __nv_bfloat16* Vr = p.Vr + (size_t)u * lim_rows * kHeadDim;
     const __nv_bfloat16* Ksu = p.Ks + (size_t)u * n_st * kHeadDim;
@@ -1453,7 +1496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // consecutive 16-byte groups (no bank conflicts) and a lane follows one
     // head alone (no shuffles).  Each warp streams its clusters' value
     // sums and scores through its own ring of slots in shared memory with
-    // 16-byte cp.async copies, kEAhead clusters ahead.
+    // 16-byte cp.async copies, up to five pairs of clusters ahead.
     constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
     constexpr int kDims = 4 * GP;  // dims per lane
     const int g = lane / (32 / GP), dg = lane % (32 / GP);

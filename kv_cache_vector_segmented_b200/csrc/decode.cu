@@ -143,15 +143,21 @@ enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
 #ifdef RI_DEBUG_PHASES
 constexpr int kStampBlocks = 4096, kStamps = 64;
 __device__ unsigned long long g_phase_ns[kStampBlocks][kStamps];
+// stamps are kept in shared memory (Misc::stamps) and written out at the
+// block's exit, so no global store sits between two phases
 #define RI_STAMP(i, t)                                          \
   do {                                                          \
-    if (threadIdx.x == (t) && blockIdx.x < kStampBlocks)        \
-      g_phase_ns[blockIdx.x][(i)] = globaltimer_ns();           \
+    if (threadIdx.x == (t)) ms->stamps[(i)] = globaltimer_ns(); \
   } while (0)
-#define RI_STAMP_VAL(i, t, v)                                   \
-  do {                                                          \
-    if (threadIdx.x == (t) && blockIdx.x < kStampBlocks)        \
-      g_phase_ns[blockIdx.x][(i)] = (unsigned long long)(v);    \
+#define RI_STAMP_VAL(i, t, v)                                          \
+  do {                                                                 \
+    if (threadIdx.x == (t)) ms->stamps[(i)] = (unsigned long long)(v); \
+  } while (0)
+#define RI_STAMP_DUMP()                                                        \
+  do {                                                                         \
+    __syncthreads();                                                           \
+    if (threadIdx.x < kStamps && blockIdx.x < kStampBlocks)                    \
+      g_phase_ns[blockIdx.x][threadIdx.x] = ms->stamps[threadIdx.x];           \
   } while (0)
 #else
 #define RI_STAMP(i, t) \
@@ -159,6 +165,9 @@ __device__ unsigned long long g_phase_ns[kStampBlocks][kStamps];
   } while (0)
 #define RI_STAMP_VAL(i, t, v) \
   do {                        \
+  } while (0)
+#define RI_STAMP_DUMP() \
+  do {                  \
   } while (0)
 #endif
 
@@ -208,7 +217,10 @@ struct Misc {
   int gsum[kGroups];  // cluster-wide group counts
   int fine[2][32];    // cluster-wide bucket counts of the two boundary groups
   alignas(16) int scan[2 * kWarps];
-  int T_R, nruns, wend_lo, wend_hi;
+  int max_own;  // largest own list (R + E entries) over the cluster's blocks
+#ifdef RI_DEBUG_PHASES
+  unsigned long long stamps[kStamps];
+#endif
   float wm[kWarps][8], wl[kWarps][8];
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area");
@@ -581,6 +593,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto id_of = [&](int i) { return (b + (i >> 7) * CS) * kTileC + (i & (kTileC - 1)); };
   const uint32_t sm_base = smem_u32(sm);
 
+#ifdef RI_DEBUG_PHASES
+  if (tid < kStamps) ms->stamps[tid] = 0ull;
+#endif
   if (tid == 0) {
     ms->abort_flag = 0;
     ms->own_kmax = ms->own_kmin = 0u;
@@ -1197,7 +1212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   // after barrier 4 nothing reads another block's shared memory in a select
-  if (p.mode == kModeSelect) return;
+  if (p.mode == kModeSelect) {
+    RI_STAMP_DUMP();
+    return;
+  }
 
   // ============================================================ step C
   // The block attends over the clusters it scored (its own R and E lists,
@@ -1293,9 +1311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // both before the copies of step C
   fence_proxy_async_smem();
   __syncthreads();
-  const int nR = ms->own_nR, nE = ms->own_nE, tokR = ms->own_tokR;
-  const int ns = st1 - st0;            // steady tokens of this block
-  const long long ntok = (long long)ns + tokR;
+
+  const int2* rlist = lists;
+  const int2* elist_all = lists + ms->own_nR;
+  const int nR = ms->own_nR, nE = ms->own_nE;
+  const int ns_loc = st1 - st0, st_start = st0;  // steady tokens of this block
+  const long long kofs = 0, ntok = (long long)ns_loc + ms->own_tokR;
+  const long long rend = ms->own_tokR;  // search key past the last R entry's tokens
 
   // ---- the state of the two kinds of warps:
   //  token warps (0..7): O^T fragments ot[j][i] (lane holds dims 16 j + gid
@@ -1347,40 +1369,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       // cluster by a binary search over the R list's token prefix
       for (int t = tt; t < nwt; t += kTokenWarps * 32) {
         const long long bt = wt + t;
-        if (bt < ns) {
-          rowtab[t] = -1 - (st0 + (int)bt);
+        if (bt < ns_loc) {
+          rowtab[t] = -1 - (st_start + (int)bt);
         } else {
-          const int j = (int)(bt - ns);
+          const int j = (int)(bt - ns_loc + kofs);
           int lo = 0, hi = nR - 1;  // last entry with prefix <= j
           while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (lists[mid].y <= j) lo = mid; else hi = mid - 1;
+            if (rlist[mid].y <= j) lo = mid; else hi = mid - 1;
           }
-          const int2 e = lists[lo];
-          rowtab[t] = e.x + (j - e.y);
+          const int2 e = rlist[lo];
+          const long long end = lo + 1 < nR ? (long long)rlist[lo + 1].y : rend;
+          // an entry without a row (failed checks) or a key outside it: masked
+          rowtab[t] = (nR > 0 && e.x >= 0 && j >= e.y && j < end) ? e.x + (j - e.y) : INT_MIN;
         }
       }
       token_bar();
       RI_STAMP(25, 0);
       const int ntile = (nwt + 15) >> 4;
       // ---- tiles warp, warp + kTokenWarps, ...: copies one tile ahead
+      // copies of a tile: each instruction moves two whole rows (lanes 0-15
+      // row 2 k, lanes 16-31 row 2 k + 1, 16 bytes each), so every 32-byte
+      // sector is requested once
       auto issue = [&](int tj, int slot) {
         if (tj < ntile) {
           uint8_t* kb = wbuf + slot * 8192;
-          const int t = lane >> 1, c0 = (lane & 1) * 8;
-          const int tok = tj * 16 + t;
-          const int code = tok < nwt ? rowtab[tok] : INT_MIN;
-          const __nv_bfloat16 *ks = safe, *vs = safe;
-          bool fill = code != INT_MIN;
-          if (code >= 0) {
-            ks = Kr + (size_t)code * kHeadDim;
-            vs = Vr + (size_t)code * kHeadDim;
-          } else if (fill) {
-            ks = Ksu + (size_t)(-1 - code) * kHeadDim;
-            vs = Vsu + (size_t)(-1 - code) * kHeadDim;
-          }
+          const int tok = tj * 16 + (lane & 15);
+          const int code_l = tok < nwt ? rowtab[tok] : INT_MIN;  // lane r < 16: row r
+          const int c = lane & 15, h = lane >> 4;
 #pragma unroll
-          for (int c = c0; c < c0 + 8; ++c) {
+          for (int k = 0; k < 8; ++k) {
+            const int t = 2 * k + h;
+            const int code = __shfl_sync(0xffffffffu, code_l, t);
+            const __nv_bfloat16 *ks = safe, *vs = safe;
+            const bool fill = code != INT_MIN;
+            if (code >= 0) {
+              ks = Kr + (size_t)code * kHeadDim;
+              vs = Vr + (size_t)code * kHeadDim;
+            } else if (fill) {
+              ks = Ksu + (size_t)(-1 - code) * kHeadDim;
+              vs = Vsu + (size_t)(-1 - code) * kHeadDim;
+            }
             cp_async16_zfill(kb + row_chunk(t, c), fill ? ks + c * 8 : safe, fill);
             cp_async16_zfill(kb + 4096 + row_chunk(t, c), fill ? vs + c * 8 : safe, fill);
           }
@@ -1506,7 +1535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kDims; ++i) eo[i] = 0.f;
     const int ew = warp - kTokenWarps;
     const int e0 = nE * ew / kEWarps, e1 = nE * (ew + 1) / kEWarps;
-    const int2* elist = lists + nR;
+    const int2* elist = elist_all;
     uint8_t* ering = sm + kOffMeta + ew * kEWarpBytes;
     // items in pairs (two independent chains per step); kPairs pairs of
     // slots in flight.  The unit's value-sum and score rows and this lane's
@@ -1658,7 +1687,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   cluster_arrive();  // 6: partials stored (release)
-  if (b != 0) return;
+  if (b != 0) {
+    RI_STAMP_DUMP();
+    return;
+  }
   cluster_wait();
   const float* pa = reinterpret_cast<const float*>(sm);
   for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
@@ -1682,6 +1714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 #endif
   RI_STAMP(8, 0);
+  RI_STAMP_DUMP();
 }
 
 // ------------------------------------------------------------------ host

@@ -195,6 +195,8 @@ struct Params {
 
 struct Misc {
   uint64_t fullA[kStagesA], emptyA[kStagesA], tdone[kMaxTilesPerBlock], qbar, drain, metabar;
+  uint64_t go;   // step D: completed by block 0 once its ring takes partials
+  uint64_t mrg;  // step D, block 0: completed by the bytes of the other partials
   uint32_t tmem;
   int abort_flag;
   uint32_t own_kmax, own_kmin;  // this block's key range (order keys) and empty clusters
@@ -250,6 +252,11 @@ __device__ __forceinline__ void cluster_sync() {
   cluster_arrive();
   cluster_wait();
 }
+// Arrival that orders none of the thread's memory accesses.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 // Address of the same shared-memory location in block `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   uint32_t r;
@@ -282,6 +289,46 @@ __device__ __forceinline__ void st_cl_v4(uint32_t addr, uint4 v) {
 }
 __device__ __forceinline__ void st_cl_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// Store into another block's shared memory whose bytes complete on an
+// mbarrier of that block (both addresses from mapa).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::
+                   "r"(addr),
+               "f"(a), "f"(b), "r"(bar)
+               : "memory");
+}
+// Arrive (release, cluster scope) on an mbarrier of another block.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Bounded wait with acquire at cluster scope (data or arrivals from other
+// blocks of the cluster).
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity,
+                                             unsigned long long limit_ns) {
+  auto probe = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (probe()) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (probe()) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
 }
 __device__ __forceinline__ void red_cl_add(uint32_t addr, uint32_t v) {
   asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -568,6 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_cent,
                   const __grid_constant__ CUtensorMap tm_q, const Params p) {
   constexpr int Gp = G <= 4 ? 4 : 8;        // scores stored per cluster
+  constexpr uint32_t kPartStride = (kHeadDim + 4) * 4;  // step D: a head's partial in block 0
+  constexpr uint32_t kPartBytes = G * (kHeadDim + 2) * 4;  // bytes of a block partial sent
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -613,7 +662,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ms->qbar, 1);
     mbar_init(&ms->drain, 1);
     mbar_init(&ms->metabar, 8);
+    mbar_init(&ms->go, 1);
+    mbar_init(&ms->mrg, 1);
     fence_barrier_init();
+    // block 0 takes the other blocks' partials in step D
+    if (b == 0) mbar_arrive_expect_tx(&ms->mrg, (uint32_t)(CS - 1) * kPartBytes);
   }
   __syncthreads();
   // 0: the block has started (waited on before the first remote access)
@@ -1642,67 +1695,80 @@ __global__ void __launch_bounds__(kThreads, 1)
   RI_STAMP(6, 0);
 
   // ============================================================ step D
-  // warps -> block partial (max in log2 units, denominator, numerator)
-  constexpr int kOutPer = (G * kHeadDim + kThreads - 1) / kThreads;
-  float bo[kOutPer], bmv[kOutPer], blv[kOutPer];
+  // warps -> block partial (max in log2 units, denominator, numerator):
+  // thread t < 32 G takes head t / 32 and dims 4 (t % 32) .. + 3
+  const bool pt = tid < G * 32;
+  const int pg = pt ? tid >> 5 : 0, pd = (tid & 31) * 4;
+  float4 bo4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  float bm = -INFINITY, bl = 0.f;
+  if (pt) {
 #pragma unroll
-  for (int r = 0; r < kOutPer; ++r) {
-    const int idx = tid + r * kThreads;
-    bo[r] = 0.f;
-    bmv[r] = -INFINITY;
-    blv[r] = 0.f;
-    if (idx < G * kHeadDim) {
-      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-      float mx = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) bm = fmaxf(bm, ms->wm[w][pg]);
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, ms->wm[w][g]);
-      float L = 0.f, O = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = ms->wm[w][g];
-        const float f = mw == -INFINITY ? 0.f : ex2f(mw - mx);
-        L = fmaf(f, ms->wl[w][g], L);
-        O = fmaf(f, wo[((size_t)w * G + g) * kHeadDim + d], O);
-      }
-      bo[r] = O;
-      bmv[r] = mx;
-      blv[r] = L;
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = ms->wm[w][pg];
+      const float f = mw == -INFINITY ? 0.f : ex2f(mw - bm);
+      bl = fmaf(f, ms->wl[w][pg], bl);
+      const float4 o = *reinterpret_cast<const float4*>(wo + ((size_t)w * G + pg) * kHeadDim + pd);
+      bo4.x = fmaf(f, o.x, bo4.x);
+      bo4.y = fmaf(f, o.y, bo4.y);
+      bo4.z = fmaf(f, o.z, bo4.z);
+      bo4.w = fmaf(f, o.w, bo4.w);
     }
   }
-  cluster_sync();  // 5: every block done with step C (block 0's ring is free)
+  // every block's partial into block 0: per block and head 132 floats
+  // (numerator[128], max, denominator, 2 unused) at the start of its ring.
+  // Block 0 releases the ring with a remote arrive on every other block's
+  // `go` (after its own warps' partials are read); the others store theirs
+  // with st.async, whose bytes complete block 0's `mrg` (armed at the start
+  // for CS - 1 partials).  A block waits only for block 0 and block 0 only
+  // for the partials; one last cluster barrier, whose arrivals come early,
+  // keeps every block alive until block 0's remote arrive has landed.
   RI_STAMP(7, 0);
-  // every block's partial into block 0: [CS][G][2 + 128] floats
   const uint32_t area = sm_base;
-#pragma unroll
-  for (int r = 0; r < kOutPer; ++r) {
-    const int idx = tid + r * kThreads;
-    if (idx < G * kHeadDim) {
-      const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-      const uint32_t base = area + 4u * (uint32_t)((b * G + g) * (kHeadDim + 2));
-      st_cl_f32(mapa(base + 4u * (2 + d), 0), bo[r]);
-      if (d == 0) {
-        st_cl_f32(mapa(base, 0), bmv[r]);
-        st_cl_f32(mapa(base + 4u, 0), blv[r]);
-      }
-    }
-  }
-  cluster_arrive();  // 6: partials stored (release)
   if (b != 0) {
+    const bool go = mbar_wait_cl(&ms->go, 0, lim);
+    if (!go) {
+      record_status(p.status, RI_ERR_TIMEOUT);
+    } else if (pt) {
+      const uint32_t mrg = mapa(smem_u32(&ms->mrg), 0);
+      const uint32_t base = area + (uint32_t)((b * G + pg) * kPartStride);
+      st_async_v4(mapa(base + 4u * (uint32_t)pd, 0), bo4, mrg);
+      if (pd == 0) st_async_v2(mapa(base + 4u * kHeadDim, 0), bm, bl, mrg);
+    }
+    cluster_arrive_relaxed();  // 5
+    cluster_wait();
     RI_STAMP_DUMP();
     return;
   }
-  cluster_wait();
+  __syncthreads();  // every warp's partial read: the ring takes the block partials
+  if (tid > 0 && tid < CS) mbar_arrive_remote(mapa(smem_u32(&ms->go), (uint32_t)tid));
+  if (warp == 0)
+    cluster_arrive();  // 5 (release: the remote arrives land before any block exits)
+  else
+    cluster_arrive_relaxed();
+  if (pt) {
+    float* base = reinterpret_cast<float*>(sm + pg * kPartStride);
+    *reinterpret_cast<float4*>(base + pd) = bo4;
+    if (pd == 0) {
+      base[kHeadDim] = bm;
+      base[kHeadDim + 1] = bl;
+    }
+  }
+  if (!mbar_wait_cl(&ms->mrg, 0, lim)) record_status(p.status, RI_ERR_TIMEOUT);
+  __syncthreads();  // block 0's own partial written
   const float* pa = reinterpret_cast<const float*>(sm);
+  constexpr int kPS = (int)(kPartStride / 4);
   for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
     const int g = idx / kHeadDim, d = idx - g * kHeadDim;
     float mx = -INFINITY;
-    for (int q = 0; q < CS; ++q) mx = fmaxf(mx, pa[(q * G + g) * (kHeadDim + 2)]);
+    for (int q = 0; q < CS; ++q) mx = fmaxf(mx, pa[(q * G + g) * kPS + kHeadDim]);
     float L = 0.f, O = 0.f;
     for (int q = 0; q < CS; ++q) {
-      const float* pq = pa + (q * G + g) * (kHeadDim + 2);
-      const float f = pq[0] == -INFINITY ? 0.f : ex2f(pq[0] - mx);
-      L = fmaf(f, pq[1], L);
-      O = fmaf(f, pq[2 + d], O);
+      const float* pq = pa + (q * G + g) * kPS;
+      const float f = pq[kHeadDim] == -INFINITY ? 0.f : ex2f(pq[kHeadDim] - mx);
+      L = fmaf(f, pq[kHeadDim + 1], L);
+      O = fmaf(f, pq[d], O);
     }
     // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
     const bool any = L > 0.f;
@@ -1715,6 +1781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #endif
   RI_STAMP(8, 0);
   RI_STAMP_DUMP();
+  cluster_wait();  // 5
 }
 
 // ------------------------------------------------------------------ host

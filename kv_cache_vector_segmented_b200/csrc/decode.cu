@@ -134,7 +134,6 @@ constexpr uint32_t kRLgs = kRRid + kMaxIdsPerBlock * 2;  // int [kGroups] own gr
 constexpr uint32_t kRTin = kRLgs + kGroups * 4;  // int [2][512] pushed per-tile equal-key counts
 constexpr uint32_t kRTcnt = kRTin + 2 * 512 * 4;  // int4 [512] pushed per-tile list counts
 static_assert(kRTcnt + 512 * 16 <= kRingBytes, "selection scratch");
-static_assert(kCand == 256 && kThreads == 2 * kCand, "ranking maps two boundaries to 2 x 256 threads");
 
 enum Mode { kModeFull = 0, kModeSelect = 1, kModeAttend = 2 };
 
@@ -286,9 +285,6 @@ __device__ __forceinline__ void st_cl_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
-}
-__device__ __forceinline__ void st_cl_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 // Store into another block's shared memory whose bytes complete on an
 // mbarrier of that block (both addresses from mapa).
@@ -1035,37 +1031,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       RI_STAMP(13, 0);
       cluster_sync();  // 3: every block's boundary members pushed
       RI_STAMP(14, 0);
-      if (warp < 2) {
+      // warp w ranks the members of boundary w: lane q copies block q's
+      // members (pushed to cin[w][q][0 .. n_q)) to their place in all[w]
+      // (a warp scan over the n_q), then lane i ranks member i by counting
+      // the larger ones
+      if (warp < 2 && (warp == 0 ? fast0 : fast1)) {
         const int w = warp;
-        const int n = lane < CS ? min(kCand, ms->candn_in[w][lane]) : 0;
-        int incl = n;
+        unsigned long long* aw = all + w * kCand;
+        const int cq = lane < CS ? min(kCand, ms->candn_in[w][lane]) : 0;
+        int incl = cq;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const int t = __shfl_up_sync(0xffffffffu, incl, off);
           if (lane >= off) incl += t;
         }
-        if (lane < CS) ms->candp[w][lane + 1] = incl;
-        if (lane == 0) ms->candp[w][0] = 0;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        if (!(w == 0 ? fast0 : fast1)) continue;
-        const int n = min(kCand, ms->candp[w][CS]);
-        for (int j = tid; j < n; j += kThreads) {
-          int ob = 0;
-          while (ob + 1 < CS && ms->candp[w][ob + 1] <= j) ++ob;
-          all[w * kCand + j] = cin[(w * kMaxCS + ob) * kCand + j - ms->candp[w][ob]];
+        const int n = min(kCand, __shfl_sync(0xffffffffu, incl, 31));
+        const unsigned long long* src = cin + (w * kMaxCS + lane) * kCand;
+        for (int k = 0; k < cq; ++k) {
+          const int pos = incl - cq + k;
+          if (pos < kCand) aw[pos] = src[k];
         }
-      }
-      __syncthreads();
-      {
-        // threads [256 w, 256 w + n) rank boundary w's members (kCand = 256)
-        const int w = tid >> 8, j = tid & 255;
-        const int n = min(kCand, ms->candp[w][CS]);
-        if ((w == 0 ? fast0 : fast1) && j < n) {
-          const unsigned long long* aw = all + w * kCand;
-          const unsigned long long me = aw[j];
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+          const unsigned long long me = aw[i];
           int greater = 0;
 #pragma unroll 8
           for (int t = 0; t < n; ++t) greater += aw[t] > me;
@@ -1102,8 +1090,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int2 mm[kKPT];
 #pragma unroll
       for (int j = 0; j < kKPT; ++j) {
+        if (j >= kper) break;  // kper is the same in every thread
         const int i = i0 + j;
-        if (j < kper && i < i1) {
+        if (i < i1) {
           kk[j] = keys[i];
           mm[j] = meta[i];
         }
@@ -1113,8 +1102,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool bad = false;
 #pragma unroll
       for (int j = 0; j < kKPT; ++j) {
+        if (j >= kper) break;
         const int i = i0 + j;
-        if (!(j < kper && i < i1)) continue;
+        if (i >= i1) continue;
         const unsigned long long o = ord64(float_order_key(kk[j]), id_of(i));
         const bool inR = onA && o >= thrA;
         const bool inE = !inR && onB && o >= thrB;
@@ -1150,6 +1140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pr = excl >> 16, pe = nR + (excl & 0xFFFF);
 #pragma unroll
       for (int j = 0; j < kKPT; ++j) {
+        if (j >= kper) break;
         if ((mR >> j) & 1u) {
           lists[pr] = make_int2(mm[j].x, texcl);
           rid[pr] = (uint16_t)(i0 + j);

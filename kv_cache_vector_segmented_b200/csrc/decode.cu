@@ -865,10 +865,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < kNB; i += kThreads) hist[i] = 0;
     for (int i = tid; i < 4 * 2 * 256; i += kThreads) dig[i] = 0;
     if (tid < 64) ms->fine[tid >> 5][tid & 31] = 0;
+    for (int i = tid; i < kGroups; i += kThreads) lgs[i] = 0;
     cluster_sync();  // 1: key ranges pushed
     RI_STAMP(2, 0);
 
-    if (warp == 0) {
+    // every warp takes the cluster's key range and empty count itself
+    float lo, scale;
+    int nfin, ninf;
+    {
       uint32_t kx = 0, kn = 0;
       int ni = 0;
       if (lane < CS) {
@@ -880,32 +884,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       kx = __reduce_max_sync(0xffffffffu, kx);
       kn = __reduce_max_sync(0xffffffffu, kn);
       ni = __reduce_add_sync(0xffffffffu, ni);
-      if (lane == 0) {
-        const int nfin = C - ni;
-        const float lo = nfin > 0 ? float_from_order_key(~kn) : 0.f;
-        const float hi = nfin > 0 ? float_from_order_key(kx) : 0.f;
-        ms->lo = lo;
-        ms->scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
-        ms->nfin = nfin;
-        ms->ninf = ni;
+      nfin = C - ni;
+      ninf = ni;
+      lo = nfin > 0 ? float_from_order_key(~kn) : 0.f;
+      const float hi = nfin > 0 ? float_from_order_key(kx) : 0.f;
+      scale = (nfin > 0 && hi > lo) ? (float)kNB / (hi - lo) : 0.f;
+    }
+    // the block's histogram of its own keys and its sums over groups of 32
+    // buckets; the group sums are pushed
+    for (int i = tid; i < nid; i += kThreads) {
+      const int bk = bucket_of(keys[i], lo, scale);
+      if (bk >= 0) {
+        atomicAdd(&hist[bk], 1);
+        atomicAdd(&lgs[bk >> 5], 1);
       }
     }
     __syncthreads();
-    const float lo = ms->lo, scale = ms->scale;
-    const int nfin = ms->nfin, ninf = ms->ninf;
-    // the block's own histogram and group sums; the group sums are pushed
-    for (int i = tid; i < nid; i += kThreads) {
-      const int bk = bucket_of(keys[i], lo, scale);
-      if (bk >= 0) atomicAdd(&hist[bk], 1);
-    }
-    __syncthreads();
     RI_STAMP(26, 0);
-    for (int g = warp; g < kGroups; g += kWarps) {
-      const int v = __reduce_add_sync(0xffffffffu, hist[g * 32 + lane]);
-      if (lane == 0) lgs[g] = v;
-    }
-    __syncthreads();
-    RI_STAMP(27, 0);
     if (tid < 32 * CS) {
       const int q = tid >> 5, j = tid & 31;  // target block, 16-byte piece
       const int4 v = reinterpret_cast<const int4*>(lgs)[j];

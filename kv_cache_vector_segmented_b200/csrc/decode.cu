@@ -667,6 +667,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   // 0: the block has started (waited on before the first remote access)
   cluster_arrive();
+  // a launch that follows this one may start its own set-up now; this one
+  // touches no global memory before the launch it follows has completed
+  // (both are no-ops without a programmatic dependency)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   RI_STAMP(0, 0);
   if (p.mode != kModeSelect && tid == 32 * 3 && p.n_steady > 0) {
     // this block's share of the steady rows into L2 (read in step C)
@@ -1941,13 +1946,17 @@ cudaError_t launch_g(const Geometry& g, const DecodeLayout& L, const DecodeArgs&
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)L.CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the set-up of this launch (barriers,
+  // tensor memory) may overlap the end of the kernel before it on the stream
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<G>, map_c, map_q, p);
 }
 

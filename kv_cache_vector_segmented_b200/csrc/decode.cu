@@ -470,6 +470,21 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// D += A B on the tensor cores, m16n8k4, TF32 inputs, fp32 accumulation:
+// A rows gid, gid + 8 at column tig (a0, a1), B row tig at column gid (b0).
+__device__ __forceinline__ void mma_tf32_1684(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k4.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+__device__ __forceinline__ uint32_t tf32_rn(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -1562,40 +1577,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
   } else {
-    // ---- estimation clusters: the block's E list split over the E warps.
-    // Lane (head g, dim group dg): GP = G rounded up to a power of two,
-    // LPH = 32 / GP lanes per head; the lane holds the GP float4 groups of
-    // dims with group index i LPH + dg (i < GP), so the lanes of a head read
-    // consecutive 16-byte groups (no bank conflicts) and a lane follows one
-    // head alone (no shuffles).  Each warp streams its clusters' value
-    // sums and scores through its own ring of slots in shared memory with
-    // 16-byte cp.async copies, up to five pairs of clusters ahead.
-    constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
-    constexpr int kDims = 4 * GP;  // dims per lane
-    const int g = lane / (32 / GP), dg = lane % (32 / GP);
-    const bool live = g < G;
-    float em = -INFINITY, el = 0.f, eo[kDims];
+    // ---- estimation clusters: the block's E list split over the E warps,
+    // folded on the tensor cores in groups of 4 clusters:
+    //   O^T[d][g] += sum_k Vsum_k[d] w_k[g],  w_k[g] = 2^(x_k[g] - m_g),
+    // one mma.m16n8k4 (TF32 inputs, fp32 sums) per 16 dims.  Lane (gid,
+    // tig) supplies cluster tig of the group: the value sums of dims
+    // 16 t + 2 gid and + 1 as rows gid and gid + 8 of A (the dims of a
+    // 16-dim tile are permuted so both come from one 8-byte load) and the
+    // weight of head gid as B[tig][gid]; it accumulates dims 16 t + 2 gid
+    // (+1) of heads 2 tig and 2 tig + 1.  The running maximum is per head
+    // (the 4 lanes of head gid agree), the denominator summed per lane.
+    // Each warp streams its clusters' value sums and scores through its
+    // own ring of slots with 16-byte cp.async copies, two groups ahead.
+    const int gid = lane >> 2, tig = lane & 3;
+    float dacc[8][4];
 #pragma unroll
-    for (int i = 0; i < kDims; ++i) eo[i] = 0.f;
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dacc[mt][i] = 0.f;
+    float em = -INFINITY, el = 0.f;  // head gid: maximum (log2 units), lane's denominator
     const int ew = warp - kTokenWarps;
     const int e0 = nE * ew / kEWarps, e1 = nE * (ew + 1) / kEWarps;
     const int2* elist = elist_all;
     uint8_t* ering = sm + kOffMeta + ew * kEWarpBytes;
-    // items in pairs (two independent chains per step); kPairs pairs of
-    // slots in flight.  The unit's value-sum and score rows and this lane's
-    // part of them are fixed for the loop: taken once, as plain pointers.
-    constexpr int kPairs = kESlots / 2;
+    constexpr int kQuads = kESlots / 4;
     const float* vs_lane = p.vsum + (size_t)u * Cs * kHeadDim + lane * 4;
     const float* sc_lane = p.score + (size_t)u * Cs * Gp + lane * 4;
     const uint32_t ering_lane = smem_u32(ering) + lane * 16;
     const bool sc_lane_on = lane < Gp / 4;
-    auto issue = [&](int e, int pair) {
+    auto issue = [&](int e, int quad) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < 4; ++k) {
         if (e + k < e1) {
           const int2 ev = elist[e + k];
           if (ev.y > 0) {
-            const uint32_t slot = ering_lane + (uint32_t)(2 * pair + k) * kSlotE;
+            const uint32_t slot = ering_lane + (uint32_t)(4 * quad + k) * kSlotE;
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(slot),
                          "l"(vs_lane + (size_t)ev.x * kHeadDim)
                          : "memory");
@@ -1608,15 +1624,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cp_async_commit();
     };
-    for (int k = 0; k < kPairs - 1; ++k) issue(e0 + 2 * k, k);
+    for (int k = 0; k < kQuads - 1; ++k) issue(e0 + 4 * k, k);
 #ifdef RI_DEBUG_PHASES
     long long cyc_w = 0, cyc_c = 0, cyc_t = clock64();
 #endif
-    int pr = 0;  // ring pair of item e
+    int qr = 0;  // ring group of item e
 #pragma unroll 1
-    for (int e = e0; e < e1; e += 2) {
-      issue(e + 2 * (kPairs - 1), pr == 0 ? kPairs - 1 : pr - 1);
-      cp_async_wait<kPairs - 1>();
+    for (int e = e0; e < e1; e += 4) {
+      issue(e + 4 * (kQuads - 1), qr == 0 ? kQuads - 1 : qr - 1);
+      cp_async_wait<kQuads - 1>();
       __syncwarp();
 #ifdef RI_DEBUG_PHASES
       {
@@ -1625,35 +1641,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         cyc_t = n_;
       }
 #endif
-      const int2 ea = elist[e];
-      const int2 eb = e + 1 < e1 ? elist[e + 1] : make_int2(0, 0);
-      const bool va = ea.y > 0 && live, vb = eb.y > 0 && live;
-      const uint8_t* sa = ering + (uint32_t)(2 * pr) * kSlotE;
-      const uint8_t* sb = sa + kSlotE;
-      const float xa = va ? reinterpret_cast<const float*>(sa + 512)[g] * kLog2e : -INFINITY;
-      const float xb = vb ? reinterpret_cast<const float*>(sb + 512)[g] * kLog2e : -INFINITY;
-      const float xm = fmaxf(xa, xb);
+      const uint8_t* st = ering + (uint32_t)(4 * qr + tig) * kSlotE;  // cluster tig's slot
+      const int2 ev = e + tig < e1 ? elist[e + tig] : make_int2(0, 0);
+      const bool v = ev.y > 0;  // the slot holds this cluster's sums
+      const bool vh = v && gid < G;
+      const float x = vh ? reinterpret_cast<const float*>(st + 512)[gid] * kLog2e : -INFINITY;
+      float xm = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+      xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 2));
+      float corr = 1.f;
       if (xm > em + kRescale2) {  // new reference (also the first cluster)
-        const float c = em == -INFINITY ? 0.f : ex2f(em - xm);
-        el *= c;
-#pragma unroll
-        for (int i = 0; i < kDims; ++i) eo[i] *= c;
+        corr = em == -INFINITY ? 0.f : ex2f(em - xm);
         em = xm;
+        el *= corr;
       }
-      const float wa = va ? ex2f(xa - em) : 0.f, wb = vb ? ex2f(xb - em) : 0.f;
-      el = fmaf((float)eb.y, wb, fmaf((float)ea.y, wa, el));
-      const float4* ra = reinterpret_cast<const float4*>(sa) + dg;
-      const float4* rb = reinterpret_cast<const float4*>(sb) + dg;
+      if (__any_sync(0xffffffffu, corr != 1.f)) {
+        // columns 2 tig, 2 tig + 1 rescale by those heads' factors
+        const float c0 = __shfl_sync(0xffffffffu, corr, (tig * 2) * 4);
+        const float c1 = __shfl_sync(0xffffffffu, corr, (tig * 2 + 1) * 4);
 #pragma unroll
-      for (int i = 0; i < GP; ++i) {
-        const float4 a4 = va ? ra[i * (32 / GP)] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 b4 = vb ? rb[i * (32 / GP)] : make_float4(0.f, 0.f, 0.f, 0.f);
-        eo[4 * i] = fmaf(wb, b4.x, fmaf(wa, a4.x, eo[4 * i]));
-        eo[4 * i + 1] = fmaf(wb, b4.y, fmaf(wa, a4.y, eo[4 * i + 1]));
-        eo[4 * i + 2] = fmaf(wb, b4.z, fmaf(wa, a4.z, eo[4 * i + 2]));
-        eo[4 * i + 3] = fmaf(wb, b4.w, fmaf(wa, a4.w, eo[4 * i + 3]));
+        for (int mt = 0; mt < 8; ++mt) {
+          dacc[mt][0] *= c0;
+          dacc[mt][1] *= c1;
+          dacc[mt][2] *= c0;
+          dacc[mt][3] *= c1;
+        }
       }
-      pr = pr + 1 == kPairs ? 0 : pr + 1;
+      const float w = vh ? ex2f(x - em) : 0.f;
+      el = fmaf((float)ev.y, w, el);
+      const uint32_t b0 = tf32_rn(w);
+      const float* arow = reinterpret_cast<const float*>(st) + 2 * gid;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const float2 a = v ? *reinterpret_cast<const float2*>(arow + 16 * mt) : make_float2(0.f, 0.f);
+        mma_tf32_1684(dacc[mt], tf32_rn(a.x), tf32_rn(a.y), b0);
+      }
+      qr = qr + 1 == kQuads ? 0 : qr + 1;
       __syncwarp();
 #ifdef RI_DEBUG_PHASES
       {
@@ -1668,19 +1690,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     RI_STAMP_VAL(41, kTokenWarps * 32, cyc_c);
     RI_STAMP_VAL(42, kTokenWarps * 32, e1 - e0);
 #endif
+    el += __shfl_xor_sync(0xffffffffu, el, 1);
+    el += __shfl_xor_sync(0xffffffffu, el, 2);
     cp_async_wait<0>();
     RI_STAMP(24, kTokenWarps * 32);
     __syncthreads();  // every warp done with step C: the ring is free
-    if (live) {
-      float4* dst = reinterpret_cast<float4*>(wo + ((size_t)warp * G + g) * kHeadDim) + dg;
-#pragma unroll
-      for (int i = 0; i < GP; ++i)
-        dst[i * (32 / GP)] = make_float4(eo[4 * i], eo[4 * i + 1], eo[4 * i + 2], eo[4 * i + 3]);
-      if (dg == 0) {
-        ms->wm[warp][g] = em;
-        ms->wl[warp][g] = el;
-      }
+    if (tig == 0 && gid < G) {
+      ms->wm[warp][gid] = em;
+      ms->wl[warp][gid] = el;
     }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int h = tig * 2 + k;
+        if (h < G) {
+          float* rg = wo + ((size_t)warp * G + h) * kHeadDim + 16 * mt + 2 * gid;
+          rg[0] = dacc[mt][k];
+          rg[1] = dacc[mt][2 + k];
+        }
+      }
   }
   __syncthreads();
   RI_STAMP(6, 0);

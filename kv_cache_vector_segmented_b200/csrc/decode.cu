@@ -679,7 +679,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block 0 takes the other blocks' partials in step D
     if (b == 0) mbar_arrive_expect_tx(&ms->mrg, (uint32_t)(CS - 1) * kPartBytes);
   }
+  // tensor memory for step A's accumulators (a column group per tile),
+  // before the wait on the launch this one follows
+  uint32_t ncols = 32;
+  while (ncols < (uint32_t)ntiles * kQRows) ncols <<= 1;
+  if (ntiles > 0 && warp == 1) {
+    tmem_alloc(&ms->tmem, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   // 0: the block has started (waited on before the first remote access)
   cluster_arrive();
   // a launch that follows this one may start its own set-up now; this one
@@ -700,15 +710,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ============================================================ step A
   if (ntiles > 0) {
-    uint32_t ncols = 32;
-    while (ncols < (uint32_t)ntiles * kQRows) ncols <<= 1;
-    if (warp == 1) {
-      tmem_alloc(&ms->tmem, ncols);
-      tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     const uint32_t tmem = ms->tmem;
     if (warp == 0 && lane == 0) {
       // TMA producer: the unit's query rows once, then the block's tiles
@@ -1781,14 +1782,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kPS = (int)(kPartStride / 4);
   for (int idx = tid; idx < G * kHeadDim; idx += kThreads) {
     const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+    // (loops unrolled over the largest cluster, so the loads are issued together)
+    float pm[kMaxCS];
     float mx = -INFINITY;
-    for (int q = 0; q < CS; ++q) mx = fmaxf(mx, pa[(q * G + g) * kPS + kHeadDim]);
+#pragma unroll
+    for (int q = 0; q < kMaxCS; ++q) {
+      pm[q] = q < CS ? pa[(q * G + g) * kPS + kHeadDim] : -INFINITY;
+      mx = fmaxf(mx, pm[q]);
+    }
     float L = 0.f, O = 0.f;
-    for (int q = 0; q < CS; ++q) {
-      const float* pq = pa + (q * G + g) * kPS;
-      const float f = pq[kHeadDim] == -INFINITY ? 0.f : ex2f(pq[kHeadDim] - mx);
-      L = fmaf(f, pq[kHeadDim + 1], L);
-      O = fmaf(f, pq[d], O);
+#pragma unroll
+    for (int q = 0; q < kMaxCS; ++q) {
+      if (q < CS) {
+        const float* pq = pa + (q * G + g) * kPS;
+        const float f = pm[q] == -INFINITY ? 0.f : ex2f(pm[q] - mx);
+        L = fmaf(f, pq[kHeadDim + 1], L);
+        O = fmaf(f, pq[d], O);
+      }
     }
     // no token and no cluster contributed (empty steady zone and budgets): 0, lse -inf
     const bool any = L > 0.f;

@@ -117,11 +117,32 @@ def _dist():
     return ws, rank, local
 
 
+def _code_sha16(path: str) -> str:
+    """First 16 hex digits of the sha256 of a source file's code: text after
+    // (outside string literals) and blank lines dropped, so an edit of the
+    comments alone keeps the value."""
+    out = []
+    for line in open(path, encoding="utf-8"):
+        code, quoted, i = [], False, 0
+        while i < len(line):
+            c = line[i]
+            if c == '"' and (i == 0 or line[i - 1] != "\\"):
+                quoted = not quoted
+            if not quoted and line.startswith("//", i):
+                break
+            code.append(c)
+            i += 1
+        t = "".join(code).strip()
+        if t:
+            out.append(t)
+    return hashlib.sha256("\n".join(out).encode()).hexdigest()[:16]
+
+
 def _traffic_from_profiles(kernel_src: str, kernel: str):
     """DRAM bytes per launch recorded by an ncu capture of `kernel` from the
-    current kernel source (null when the source changed since)."""
-    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
-    pat = re.compile(r"traffic_bytes_per_launch:\s*(\d+)\s+source_sha256_16:\s*([0-9a-f]{16})")
+    current kernel code (null when the code changed since)."""
+    sha = _code_sha16(kernel_src)
+    pat = re.compile(r"traffic_bytes_per_launch:\s*(\d+)\s+code_sha256_16:\s*([0-9a-f]{16})")
     for fn in sorted(os.listdir(os.path.join(ROOT, "profiles"))):
         if not (fn.startswith(kernel) and fn.endswith(".md")):
             continue

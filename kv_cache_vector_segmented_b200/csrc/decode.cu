@@ -26,34 +26,43 @@
 //      to the workspace (the estimation term reads them back).  Eight other
 //      warps load the clusters' sizes and first rows meanwhile.
 //   B) Selection, exact, cluster-wide: the key range (barrier 1), each
-//      block's histogram of its own keys over 4096 value buckets and its
-//      sums over groups of 32 buckets, the group sums pushed to every block
-//      (barrier 2); every block finds the two boundary groups (ranks k_r and
-//      k_r + k_e from the top), reads those groups' 32 bucket counts from
-//      every block and finds the boundary buckets.  The members of a
-//      boundary bucket are ranked exactly by (key desc, id asc): pushed to
-//      every block when there are few of them (barrier 3), else found by a
-//      radix walk over the 32-bit order key and a final id count (crowded
-//      buckets, heavy ties).  Each block lists its own R clusters (first
-//      row, token prefix) and E clusters (id, size) in id order; when the
-//      selection is written out, every block pushes its per-tile counts
-//      (barrier 4) and places its ids by the prefixes over all tiles.
+//      block's histogram of its own keys over 4096 value buckets with its
+//      sums over groups of 32 buckets counted alongside, the group sums
+//      pushed to every block (barrier 2); every block finds the two boundary
+//      groups (ranks k_r and k_r + k_e from the top), reads those groups' 32
+//      bucket counts from every block and finds the boundary buckets.  The
+//      members of a boundary bucket are ranked exactly by (key desc, id
+//      asc): pushed to every block when there are few of them (barrier 3)
+//      and ranked by one warp per boundary, else found by a radix walk over
+//      the 32-bit order key and a final id count (crowded buckets, heavy
+//      ties).  Each block lists its own R clusters (first row, token prefix)
+//      and E clusters (id, size) in id order; when the selection is written
+//      out, every block pushes its per-tile counts (barrier 4) and places its
+//      ids by the prefixes over all tiles.
 //   C) Attention: each block attends over the clusters it scored (its own
 //      R and E lists) and an even share of the steady tokens.  Warps 0-7
 //      take the token rows in windows: 16-row K and V tiles copied with
-//      16-byte cp.async into an XOR-swizzled layout, S = Q K^T and
-//      O^T += V^T P^T on mma.sync.m16n8k16 bf16 tiles (ldmatrix /
-//      ldmatrix.trans, the query rows padded to 16).  Warps 8-15 fold the E
-//      clusters on CUDA cores in fp32 (lane = head x dim group), each warp
+//      16-byte cp.async (two whole rows per instruction) into an
+//      XOR-swizzled layout, S = Q K^T and O^T += V^T P^T on
+//      mma.sync.m16n8k16 bf16 tiles (ldmatrix / ldmatrix.trans, the query
+//      rows padded to 16).  Warps 8-15 fold the E clusters four at a time
+//      on the tensor cores (mma.sync.m16n8k4, TF32 value sums and weights,
+//      fp32 sums; the denominator n_c e^s in fp32 on CUDA cores), each warp
 //      streaming value sums and scores through its own ring of slots.  Both
 //      keep an online softmax in log2 units, rescaled only when the maximum
 //      grows by more than e^8.  After a separate select call, the attend
 //      call rebuilds the same lists by the same tile ownership, so both
 //      paths fold the same items in the same order.
-//   D) Merge: the block's warps are combined in shared memory, every block
-//      writes its partial (max, denominator, numerator) into block 0's
-//      shared memory (barriers 5 and 6) and block 0 merges them by
-//      log-sum-exp into out and lse.
+//   D) Merge: the block's warps are combined in shared memory; block 0
+//      releases its ring with a remote mbarrier arrive and the other blocks
+//      store their partials (max, denominator, numerator) into it with
+//      st.async, whose bytes complete an mbarrier of block 0; block 0 merges
+//      them by log-sum-exp into out and lse.  A last cluster barrier, whose
+//      arrivals come early, keeps every block alive until the remote arrives
+//      have landed.
+// Launches go out with programmatic dependent launch: a launch sets up its
+// barriers and tensor memory while the launch before it finishes and waits
+// for it (griddepcontrol.wait) before its first global access.
 // A growing index (index maintenance during decode) is read through
 // separate per-unit strides: Cs clusters and Ms rows, of which the first C
 // clusters are live.

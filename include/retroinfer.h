@@ -242,6 +242,22 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
                               int32_t* sel_ids, void* workspace, size_t workspace_bytes,
                               ri_stream_t stream);
 
+/* One decode step with the query and the output in host memory: copies
+ * q_host (bf16 [B][H_kv*G][d]) to q_dev, runs ri_decode_attention on `stream`
+ * (out_dev, lse, workspace as there; no selection output), copies out_dev to
+ * out_host and waits for the stream, so out_host holds the step's output on
+ * return.  q_dev and out_dev are device buffers of the same shape owned by
+ * the caller (16-byte aligned); page-locked host buffers make the two copies
+ * asynchronous with respect to other host work.  Errors: as
+ * ri_decode_attention, plus RI_ERR_INVALID_ARG for a NULL host pointer and
+ * RI_ERR_CUDA when a copy or the synchronisation fails (then out_host is not
+ * valid).  The pages describe the decode step, not this convenience; it is
+ * the call an application without device tensors of its own makes. */
+ri_status ri_decode_attention_host(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                   const void* q_host, void* q_dev, const ri_index* idx,
+                                   void* out_dev, void* out_host, float* lse, void* workspace,
+                                   size_t workspace_bytes, ri_stream_t stream);
+
 /* ri_decode_attention without a caller workspace.  The pages describe no
  * such call; it exists for callers that must not allocate (or own) scratch:
  * the scratch is a fixed device array of RI_STATIC_SCRATCH_BYTES inside this

@@ -101,6 +101,9 @@ lib.ri_decode_workspace.argtypes = [_P(IndexConfig), _P(DecodeConfig)]
 lib.ri_decode_attention.restype = ctypes.c_int
 lib.ri_decode_attention.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex), _vp,
                                     _vp, _vp, _vp, _sz, _vp]
+lib.ri_decode_attention_host.restype = ctypes.c_int
+lib.ri_decode_attention_host.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _vp, _P(CIndex),
+                                         _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.ri_decode_attention_static.restype = ctypes.c_int
 lib.ri_decode_attention_static.argtypes = [_P(IndexConfig), _P(DecodeConfig), _vp, _P(CIndex),
                                            _vp, _vp, _vp, _vp, _vp]
@@ -461,6 +464,27 @@ class Decoder:
         check(lib.ri_decode_attention(*self._args, q.data_ptr(), *self._tail, s),
               "ri_decode_attention")
         return self.out, self.lse
+
+    def step_host(self, q_host: torch.Tensor, out_host: torch.Tensor,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """One step with host buffers (ri_decode_attention_host): q_host is
+        copied to the device, the step runs, the output comes back into
+        out_host (both CPU bf16 tensors of the query's shape, page-locked for
+        asynchronous copies); returns out_host once it holds the output."""
+        for t, name in ((q_host, "q_host"), (out_host, "out_host")):
+            if t.device.type != "cpu" or t.dtype != torch.bfloat16 or \
+                    tuple(t.shape) != self._qshape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CPU bfloat16 tensor of shape "
+                                 f"{self._qshape}")
+        if not hasattr(self, "_qdev"):
+            self._qdev = torch.empty(self._qshape, dtype=torch.bfloat16, device=self.dev)
+        s = (stream or torch.cuda.current_stream(self.dev)).cuda_stream
+        check(lib.ri_decode_attention_host(*self._args, q_host.data_ptr(), self._qdev.data_ptr(),
+                                           ctypes.byref(self._cidx), self.out.data_ptr(),
+                                           out_host.data_ptr(), _ptr(self.lse),
+                                           self.ws.data_ptr(), self.ws.numel(), s),
+              "ri_decode_attention_host")
+        return out_host
 
 
 STATIC_SCRATCH_BYTES = 4 << 20  # RI_STATIC_SCRATCH_BYTES

@@ -487,6 +487,32 @@ ri_status ri_decode_attention(const ri_index_config* cfg, const ri_decode_config
   return RI_OK;
 }
 
+ri_status ri_decode_attention_host(const ri_index_config* cfg, const ri_decode_config* dcfg,
+                                   const void* q_host, void* q_dev, const ri_index* idx,
+                                   void* out_dev, void* out_host, float* lse, void* workspace,
+                                   size_t workspace_bytes, ri_stream_t stream) {
+  Geometry g;
+  DecodeLayout L;
+  ri_status st = prepare_decode(cfg, dcfg, q_dev, idx, workspace, workspace_bytes, &g, &L);
+  if (st != RI_OK) return st;
+  RI_CHECK(q_host && out_host, RI_ERR_INVALID_ARG, "q_host and out_host must be non-NULL");
+  RI_CHECK(out_dev && aligned16(out_dev), RI_ERR_INVALID_ARG,
+           "out_dev must be non-NULL and 16-byte aligned");
+  if (!decode_plan(g, &L)) return RI_ERR_UNSUPPORTED;
+  const size_t bytes = (size_t)g.BH() * g.G * g.d * 2;  // q and out: bf16 [B][H G][d]
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "query copy to the device");
+  DecodeArgs a = decode_args(q_dev, idx, out_dev, lse, nullptr, nullptr, workspace);
+  e = launch_decode(g, L, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  e = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "output copy to the host");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
+  return RI_OK;
+}
+
 ri_status ri_selftest_decode_timeout(const ri_index_config* cfg, const ri_decode_config* dcfg,
                                      const void* q, const ri_index* idx, void* out,
                                      void* workspace, size_t workspace_bytes, int32_t hand_off,

@@ -120,6 +120,18 @@ def test_decode_rejects_bad_arguments_before_launch(R):
     assert lib.ri_attend_selected(ctypes.byref(cfg), ctypes.byref(d), 4096, ctypes.byref(idx),
                                   4096, None, 10, 4096, None, 4096, need, None) == bad["RI_ERR_INVALID_ARG"]
     assert lib.ri_selftest_wait_timeout(None, 1000, None) == bad["RI_ERR_INVALID_ARG"]
+    # the host-buffer step: host pointers, device output and workspace checked first
+    hq = ctypes.create_string_buffer(64)
+    assert lib.ri_decode_attention_host(ctypes.byref(cfg), ctypes.byref(d), None, 4096,
+                                        ctypes.byref(idx), 4096, hq, None, 4096, need,
+                                        None) == bad["RI_ERR_INVALID_ARG"]
+    assert "q_host" in lib.ri_last_error().decode()
+    assert lib.ri_decode_attention_host(ctypes.byref(cfg), ctypes.byref(d), hq, 4096,
+                                        ctypes.byref(idx), None, hq, None, 4096, need,
+                                        None) == bad["RI_ERR_INVALID_ARG"]
+    assert lib.ri_decode_attention_host(ctypes.byref(cfg), ctypes.byref(d), hq, 4096,
+                                        ctypes.byref(idx), 4096, hq, None, 4096, need - 4,
+                                        None) == bad["RI_ERR_WORKSPACE"]
 
 
 def test_status_strings(R):

@@ -172,6 +172,26 @@ def test_select_then_attend_equals_decode(R):
     assert torch.equal(out2, ref_out)
 
 
+def test_decoder_host_buffers_equal_device_call(R):
+    """Decoder.step_host (ri_decode_attention_host: query and output in
+    page-locked host memory, copies and the wait inside the call) returns
+    the device call's output bit for bit, step after step."""
+    dev = torch.device("cuda:0")
+    kv = S.make_kv(1, 2, 30000, seed=18)
+    heads = U.oracle_index_heads(kv, use_labels=True)
+    cfg = R.IndexConfig.make(1, 2, 4, 30000)
+    idx = U.to_device_index(R, cfg, heads, dev)
+    dec = R.Decoder(idx)
+    o_host = torch.empty((1, 8, 128), dtype=torch.bfloat16).pin_memory()
+    for seed in (19, 20, 21):
+        q = S.make_queries(kv, 4, seed=seed)
+        ref, _ = dec(q.to(dev))
+        ref = ref.cpu()
+        got = dec.step_host(q.pin_memory(), o_host)
+        assert got is o_host and torch.equal(o_host, ref)
+    assert R.read_device_status(dec.ws) == 0
+
+
 def test_wait_timeout_selftest_reports_status(R):
     dev = torch.device("cuda:0")
     ws = R.alloc_workspace(1024, dev)

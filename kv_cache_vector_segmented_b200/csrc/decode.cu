@@ -211,12 +211,10 @@ struct Misc {
   int own_ninf;
   int own_ncand[2];
   int own_nR, own_nE, own_tokR;
-  int pub_idcnt[2];  // crowded path: read by the other blocks
   int pub_tid[2];
   // pushed by every block of the cluster (slot = the sender's rank)
   uint4 rng_in[kMaxCS];   // (max key, max complemented key, empty clusters, 0)
   int candn_in[2][kMaxCS];
-  uint4 tot_in[kMaxCS];   // (R clusters, E clusters, R tokens, 0)
   // cluster-wide values
   int nRp[kMaxCS + 1], nEp[kMaxCS + 1], tokRp[kMaxCS + 1];
   int candp[2][kMaxCS + 1];
@@ -227,7 +225,6 @@ struct Misc {
   int gsum[kGroups];  // cluster-wide group counts
   int fine[2][32];    // cluster-wide bucket counts of the two boundary groups
   alignas(16) int scan[2 * kWarps];
-  int max_own;  // largest own list (R + E entries) over the cluster's blocks
 #ifdef RI_DEBUG_PHASES
   unsigned long long stamps[kStamps];
 #endif
@@ -670,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ms->own_kmax = ms->own_kmin = 0u;
     ms->own_ninf = 0;
     ms->own_ncand[0] = ms->own_ncand[1] = 0;
-    ms->pub_idcnt[0] = ms->pub_idcnt[1] = 0;
     ms->pub_tid[0] = ms->pub_tid[1] = -1;
     ms->own_nR = ms->own_nE = ms->own_tokR = 0;
     ms->thr[0] = ms->thr[1] = 0ull;

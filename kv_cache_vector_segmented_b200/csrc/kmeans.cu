@@ -404,15 +404,22 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         cm[2 * cp] = fmax3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         cm[2 * cp + 1] = fmax3f(n4[0], n4[1], fmaxf(n4[2], n4[3]));
         R = fmax3f(R, cm[2 * cp], cm[2 * cp + 1]);
+        // w_i >= tr iff the sign bit of the rounded difference w_i - tr is
+        // clear (rounding keeps the sign; w_i == tr gives +0).  A funnel shift
+        // moves each sign bit into an accumulator: one integer instruction per
+        // entry, the subtraction on the FP32 pipe.  Two chains per chunk
+        // (entries 15..0 and 31..16, the last one shifted in lands in bit 0).
         const float tr = R - delta;
-        uint32_t a4[4] = {0u, 0u, 0u, 0u}, b4[4] = {0u, 0u, 0u, 0u};
+        uint32_t alo = 0u, ahi = 0u, blo = 0u, bhi = 0u;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          a4[i & 3] |= (__uint_as_float(r0[i]) >= tr ? 1u : 0u) << i;
-          b4[i & 3] |= (__uint_as_float(r1[i]) >= tr ? 1u : 0u) << i;
+        for (int i = 15; i >= 0; --i) {
+          alo = __funnelshift_l(__float_as_uint(__fsub_rn(__uint_as_float(r0[i]), tr)), alo, 1);
+          ahi = __funnelshift_l(__float_as_uint(__fsub_rn(__uint_as_float(r0[i + 16]), tr)), ahi, 1);
+          blo = __funnelshift_l(__float_as_uint(__fsub_rn(__uint_as_float(r1[i]), tr)), blo, 1);
+          bhi = __funnelshift_l(__float_as_uint(__fsub_rn(__uint_as_float(r1[i + 16]), tr)), bhi, 1);
         }
-        hit[2 * cp] = (a4[0] | a4[1]) | (a4[2] | a4[3]);
-        hit[2 * cp + 1] = (b4[0] | b4[1]) | (b4[2] | b4[3]);
+        hit[2 * cp] = ~(alo | (ahi << 16));
+        hit[2 * cp + 1] = ~(blo | (bhi << 16));
       }
       if (timed_out) {
         record_status(status, RI_ERR_TIMEOUT);

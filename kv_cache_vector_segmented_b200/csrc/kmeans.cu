@@ -66,7 +66,8 @@ constexpr uint32_t kSmMisc = kSmBar + kNumBars * 8;
 // hand-over from column quarters 0-2 to quarter 3 of a TMEM lane quadrant
 constexpr uint32_t kSmXR = (kSmMisc + 64 + 15) / 16 * 16;            // [4][128] f32
 constexpr uint32_t kSmXMask = kSmXR + 4 * kRows * 4;                  // [4][4 chunks][128] u32
-constexpr uint32_t kAssignSmem = kSmXMask + 4 * 4 * kRows * 4 + 1024;  // + alignment
+constexpr uint32_t kSmXSum = kSmXMask + 4 * 4 * kRows * 4;             // [4][128] u32
+constexpr uint32_t kAssignSmem = kSmXSum + 4 * kRows * 4 + 1024;       // + alignment
 static_assert(kAssignSmem <= 227 * 1024, "assignment kernel shared memory");
 
 // Queue of rows whose label needs an exact decision.
@@ -359,6 +360,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(Qc * 64);
     float* xR = reinterpret_cast<float*>(sm + kSmXR);             // [3][128]
     uint32_t* xm = reinterpret_cast<uint32_t*>(sm + kSmXMask);    // [3][4][128]
+    uint32_t* xs = reinterpret_cast<uint32_t*>(sm + kSmXSum);     // [3][128]
     int prev_unit = -1;
     float uE = 0.f, uC = 0.f;
     int it = 0;
@@ -427,9 +429,16 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         break;
       }
       const float thr = R - delta;
+      // the slice's candidates: how many, and the first in column order
+      // (chunk c = 2 h + j of this slice is column chunk 8 h + 2 Qc + j)
+      int ncand = 0, first = 512;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 3; c >= 0; --c) {
         if (cm[c] < thr) hit[c] = 0u;
+        ncand += __popc(hit[c]);
+        if (hit[c]) first = (8 * (c >> 1) + 2 * Qc + (c & 1)) * 32 + __ffs(hit[c]) - 1;
+      }
+      const uint32_t summ = (uint32_t)first | ((uint32_t)ncand << 16);
       // the slice that decides the rows of this quadrant rotates with the
       // tile, so the decision work is shared by the four slices' warps
       const int dq = it & 3;
@@ -440,6 +449,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           break;
         }
         xR[Qc * kRows + row] = R;
+        xs[Qc * kRows + row] = summ;
 #pragma unroll
         for (int c = 0; c < 4; ++c) xm[(Qc * 4 + c) * kRows + row] = hit[c];
         mbar_arrive(&xfull[q]);
@@ -451,15 +461,17 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         break;
       }
       float Rq[4];
-      uint32_t mq[16];
+      uint32_t sq[4], mq[16];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (k == Qc) {
           Rq[k] = R;
+          sq[k] = summ;
 #pragma unroll
           for (int c = 0; c < 4; ++c) mq[k * 4 + c] = hit[c];
         } else {
           Rq[k] = xR[k * kRows + row];
+          sq[k] = xs[k * kRows + row];
 #pragma unroll
           for (int c = 0; c < 4; ++c) mq[k * 4 + c] = xm[(k * 4 + c) * kRows + row];
         }
@@ -467,23 +479,28 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       mbar_arrive(&xempty[q]);
       if (!valid) continue;
       const float W = fmaxf(fmaxf(Rq[0], Rq[1]), fmaxf(Rq[2], Rq[3]));
-      // chunks in column order: column chunk cc = 8 h + 2 Qc + j is chunk
-      // 2 h + j of slice Qc
-      uint32_t mc[16];
+      const float wt = W - delta;
+      // a slice whose maximum is below W - delta holds no candidate; the
+      // others' counts add up and the first candidate is the least first one
+      int ntot = 0, lab = 512;
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const int k = (cc & 7) >> 1, c = ((cc >> 3) << 1) | (cc & 1);
-        mc[cc] = Rq[k] < W - delta ? 0u : mq[k * 4 + c];  // slice without candidates
-      }
-      int ntot = 0, lab = -1;
-#pragma unroll
-      for (int c = 15; c >= 0; --c) {
-        ntot += __popc(mc[c]);
-        if (mc[c]) lab = c * 32 + __ffs(mc[c]) - 1;
+      for (int k = 0; k < 4; ++k) {
+        if (!(Rq[k] < wt)) {
+          ntot += (int)(sq[k] >> 16);
+          lab = min(lab, (int)(sq[k] & 0xFFFFu));
+        }
       }
       const int grow = u.bh * d.M + u.seg_start + t;
-      labels[grow] = lab >= 0 ? lab : 0;
+      labels[grow] = lab < 512 ? lab : 0;
       if (ntot != 1) {
+        // chunks in column order: column chunk cc = 8 h + 2 Qc + j is chunk
+        // 2 h + j of slice Qc
+        uint32_t mc[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int k = (cc & 7) >> 1, c = ((cc >> 3) << 1) | (cc & 1);
+          mc[cc] = Rq[k] < wt ? 0u : mq[k * 4 + c];  // slice without candidates
+        }
         // two or more candidates (ids in increasing order): exact fix-up
         FixEntry e;
         e.row = grow;

@@ -43,12 +43,13 @@ constexpr int kStages = 2;        // key tile ring
 constexpr int kEpiWarps = 16;       // assignment epilogue: 4 lane quadrants x 4 column quarters
 constexpr int kAssignThreads = 64 + 32 * kEpiWarps;
 constexpr int kCand = 8;          // candidate slots per row
-constexpr int kUpdateWarps = 8;   // update / finalise: one warp per cluster
+constexpr int kUpdateWarps = 2;   // update: one warp per cluster, warps per block (48 per SM)
+constexpr int kFinWarps = 2;      // finalise: one warp per cluster, warps per block (24 per SM)
 constexpr int kSortThreads = 1024;
 constexpr int kGatherRows = 16;   // member rows per cp.async chunk of the update
-constexpr int kUpdateSmem = kUpdateWarps * kGatherRows * 128 * 2;  // 32 KB
+constexpr int kUpdateSmem = kUpdateWarps * kGatherRows * 128 * 2;  // 8 KB
 constexpr int kFinRows = 16;      // member rows (K and V) per cp.async chunk of the finalise
-constexpr int kFinSmem = kUpdateWarps * kFinRows * 512;             // 64 KB
+constexpr int kFinSmem = kFinWarps * kFinRows * 512;                // 16 KB
 constexpr uint16_t kCandNone = 0xFFFF;
 constexpr uint16_t kCandFullScan = 0xFFFE;
 
@@ -683,10 +684,12 @@ __global__ void unit_max_kernel(const float2* __restrict__ ecs, BuildDims d,
 // positions [w P, w P + P): per-warp histograms, a column scan over warps,
 // then each warp places its positions in order (ranks among equal labels of
 // one 32-position step by match_any).
+// Block 0 also zeroes the fix-up queue count of the next assignment pass
+// (the fix-up that read it ran before this kernel).
 // Shared memory: lab[L] u16, cnt[32][512] i32, tot scan scratch.
 __global__ void __launch_bounds__(kSortThreads)
     sort_kernel(const int32_t* __restrict__ labels, BuildDims d, int32_t* __restrict__ members,
-                int32_t* __restrict__ mstart) {
+                int32_t* __restrict__ mstart, int* __restrict__ queue_count) {
   extern __shared__ __align__(16) uint8_t smem_s[];
   constexpr int NW = kSortThreads / 32;
   int* cnt = reinterpret_cast<int*>(smem_s);                                  // [NW][512]
@@ -700,6 +703,7 @@ __global__ void __launch_bounds__(kSortThreads)
   const int seg_start = s * d.seg_len;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* src = labels + (size_t)bh * d.M + seg_start;
+  if (unit == 0 && threadIdx.x == 0) *queue_count = 0;  // for the next assignment pass
   for (int i = threadIdx.x; i < NW * kMaxClustersPerSeg; i += kSortThreads) cnt[i] = 0;
   for (int i = threadIdx.x; i < L; i += kSortThreads) lab[i] = (uint16_t)src[i];
   __syncthreads();
@@ -758,10 +762,12 @@ __global__ void __launch_bounds__(kSortThreads)
 
 // One warp per cluster: mu_j = mean of the members (fp32, summed in position
 // order; an empty cluster keeps mu_j), the column constants of the new
-// centroid and the cluster size.  Members are fetched 32 rows at a time with
-// 16-byte cp.async copies into the warp's 8 KB of shared memory (the
+// centroid and the cluster size.  Members are fetched 16 rows at a time with
+// 16-byte cp.async copies into the warp's 4 KB of shared memory (the
 // transfers need no registers, so a warp keeps a whole chunk in flight).
-__global__ void __launch_bounds__(kUpdateWarps * 32, 6)
+// Blocks of two warps: a block holds its shared memory until its slower
+// warp is done, so small blocks keep a large cluster from idling many warps.
+__global__ void __launch_bounds__(kUpdateWarps * 32, 48 / kUpdateWarps)
     update_kernel(const __nv_bfloat16* __restrict__ K, const int32_t* __restrict__ members,
                   const int32_t* __restrict__ mstart, BuildDims d, float* __restrict__ mu,
                   __nv_bfloat16* __restrict__ mu_bf16, uint8_t* __restrict__ nsplit,
@@ -828,7 +834,7 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 6)
 // last sort): one warp per cluster copies its members' K and V rows in
 // (cluster, position) order, with the permutation, offsets, sizes, value
 // sums, the bf16 centroid and the members' squared distances.
-__global__ void __launch_bounds__(kUpdateWarps * 32, 3)
+__global__ void __launch_bounds__(kFinWarps * 32, 24 / kFinWarps)
     finalise_kernel(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                     const int32_t* __restrict__ labels, const int32_t* __restrict__ members,
                     const int32_t* __restrict__ mstart, BuildDims d,
@@ -836,12 +842,12 @@ __global__ void __launch_bounds__(kUpdateWarps * 32, 3)
   extern __shared__ __align__(16) uint8_t smem_f[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   {
-    const int unit = blockIdx.x, j = blockIdx.y * kUpdateWarps + warp;
+    const int unit = blockIdx.x, j = blockIdx.y * kFinWarps + warp;
     const int bh = unit / d.S, s = unit % d.S;
     const int Ks = s == d.S - 1 ? d.K_last : d.K_full;
     const int L = s == d.S - 1 ? d.L_last : d.seg_len;
-    if (out.labels && blockIdx.y == 0)
-      for (int t = threadIdx.x; t < L; t += blockDim.x)
+    if (out.labels)  // the unit's blocks share the copy of its labels
+      for (int t = blockIdx.y * blockDim.x + threadIdx.x; t < L; t += gridDim.y * blockDim.x)
         out.labels[(size_t)bh * d.M + s * d.seg_len + t] =
             labels[(size_t)bh * d.M + s * d.seg_len + t];
     if (blockIdx.y == 0 && s == d.S - 1 && threadIdx.x == 0)
@@ -1055,16 +1061,17 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   const int sms = num_sms();
   const unsigned grid_assign = (unsigned)(d.total_tiles < sms ? d.total_tiles : sms);
   const dim3 grid_upd((unsigned)units, (unsigned)(kMaxClustersPerSeg / kUpdateWarps));
+  const dim3 grid_fin((unsigned)units, (unsigned)(kMaxClustersPerSeg / kFinWarps));
   const int rounds = g.iters > 0 ? g.iters : 1;
+  RI_CUDA_TRY(cudaMemsetAsync(queue_count, 0, sizeof(int), st));  // later passes: the sort
   for (int t = 0; t < rounds; ++t) {
-    RI_CUDA_TRY(cudaMemsetAsync(queue_count, 0, sizeof(int), st));
     assign_kernel<<<grid_assign, kAssignThreads, kAssignSmem, st>>>(
         tm_keys, tm_cent, d, knorm, nsplit, ust, labels, queue, queue_count, status);
     RI_CUDA_TRY(cudaGetLastError());
     fixup_kernel<<<(unsigned)(4 * sms), 256, 0, st>>>(K, mu, d, queue, queue_count, labels);
     RI_CUDA_TRY(cudaGetLastError());
-    sort_kernel<<<(unsigned)units, kSortThreads, sort_smem(g.seg_len), st>>>(labels, d, members,
-                                                                             mstart);
+    sort_kernel<<<(unsigned)units, kSortThreads, sort_smem(g.seg_len), st>>>(
+        labels, d, members, mstart, queue_count);
     RI_CUDA_TRY(cudaGetLastError());
     update_kernel<<<grid_upd, kUpdateWarps * 32, kUpdateSmem, st>>>(
         K, members, mstart, d, mu, mu_bf16, nsplit, ecs, counts, g.iters > 0 ? 1 : 0);
@@ -1074,7 +1081,7 @@ ri_status launch_build(const Geometry& g, const BuildLayout& L, const BuildArgs&
   }
   if (a.out.objective)
     RI_CUDA_TRY(cudaMemsetAsync(a.out.objective, 0, units * sizeof(float), st));
-  finalise_kernel<<<grid_upd, kUpdateWarps * 32, kFinSmem, st>>>(K, V, labels, members, mstart,
+  finalise_kernel<<<grid_fin, kFinWarps * 32, kFinSmem, st>>>(K, V, labels, members, mstart,
                                                                  d, mu, a.out);
   RI_CUDA_TRY(cudaGetLastError());
   return RI_OK;

@@ -408,11 +408,14 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         cm[2 * cp + 1] = fmax3f(n4[0], n4[1], fmaxf(n4[2], n4[3]));
         R = fmax3f(R, cm[2 * cp], cm[2 * cp + 1]);
         // w_i >= tr iff the sign bit of the rounded difference w_i - tr is
-        // clear (rounding keeps the sign; w_i == tr gives +0).  A funnel shift
-        // moves each sign bit into an accumulator: one integer instruction per
-        // entry, the subtraction on the FP32 pipe.  Two chains per chunk
-        // (entries 15..0 and 31..16, the last one shifted in lands in bit 0).
-        const float tr = R - delta;
+        // clear (rounding keeps the sign; w_i == tr gives +0).  The one
+        // exception, -0 - (+0) = -0, is avoided by taking a zero threshold
+        // as -0.  A funnel shift moves each sign bit into an accumulator: one
+        // integer instruction per entry, the subtraction on the FP32 pipe.
+        // Two chains per chunk (entries 15..0 and 31..16, the last one
+        // shifted in lands in bit 0).
+        const float tr0 = R - delta;
+        const float tr = tr0 == 0.f ? -0.f : tr0;
         uint32_t alo = 0u, ahi = 0u, blo = 0u, bhi = 0u;
 #pragma unroll
         for (int i = 15; i >= 0; --i) {
